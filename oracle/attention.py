@@ -1,0 +1,99 @@
+"""fp64 GQA decode attention over the effective view (oracle; test infrastructure only).
+
+Source: "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
+Serving", Abstract -- fused attention over the quantized paged cache; the
+query gets the same block-diagonal Hadamard rotation as the keys, so the
+scores of the rotated problem equal those of the original one.
+
+Readings of this library:
+
+* q_rot = bf16_round(fwht_fp32(q)): queries are bf16 and stay bf16 after the
+  rotation (the kernel can then use 16-bit tensor-core inputs without extra
+  error).
+* scores s_p = sigma * <q_rot, k^_p> with sigma = 1/sqrt(D) unless the caller
+  passes another scale (textbook scaled dot-product attention).
+* a = softmax(s) over every cached position 0..L-1 (including the token the
+  same decode step appended); o_rot = sum_p a_p v^_p; o = H_blk o_rot (H is
+  symmetric and orthonormal, so it is its own inverse); out = bf16(o).
+* GQA grouping is contiguous: query head j uses KV head j // (Hq / Hkv).
+* The bf16 output is rounded fp64 -> fp32 -> bf16 (two round-to-nearest-even
+  steps); the tests allow one bf16 ulp between two bf16 outputs for this
+  reason.
+"""
+
+import numpy as np
+
+from .hadamard import fwht_fp32, block_diag_hadamard
+from .quant import bf16_round
+
+
+def attention_fp64(q, k, v, scale):
+    """Textbook GQA attention for one query token.
+
+    q: [Hq, D]; k, v: [L, Hkv, D]; returns o [Hq, D] in fp64:
+    o[j] = sum_p softmax_p(scale * <q[j], k[p, j // G]>) v[p, j // G].
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    Hq, D = q.shape
+    L, Hkv, _ = k.shape
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    o = np.zeros((Hq, D), np.float64)
+    for j in range(Hq):
+        h = j // G
+        s = scale * (k[:, h, :] @ q[j])
+        a = np.exp(s - s.max())
+        a /= a.sum()
+        o[j] = a @ v[:, h, :]
+    return o
+
+
+def _bf16_of_f64(x):
+    return bf16_round(np.asarray(x, np.float64).astype(np.float32))
+
+
+def rotate_query(q, Bh):
+    """q_rot = bf16_round(fwht_fp32(q)) for bf16 queries q [..., D]."""
+    return bf16_round(fwht_fp32(q, Bh))
+
+
+def decode_attention(cache, layer, seq_ids, q, scale=None, protected=True):
+    """Decode attention of one query token per sequence over an OracleKV4Cache.
+
+    q: [n, Hq, D] bf16 values.  Returns dict with
+      out_f64  [n, Hq, D]  fp64 output in the original (unrotated) basis,
+      out_bf16 [n, Hq, D]  the same rounded to bf16 (held in fp32),
+      q_rot    [n, Hq, D]  the rotated bf16 queries.
+    """
+    q = np.asarray(q, np.float32)
+    D = cache.D
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(D)
+    H = block_diag_hadamard(D, cache.Bh)
+    n = len(seq_ids)
+    out = np.zeros((n,) + q.shape[1:], np.float64)
+    q_rot = rotate_query(q, cache.Bh)
+    for i, seq in enumerate(seq_ids):
+        kh, vh = cache.view(layer, int(seq), protected=protected)
+        if kh.shape[0] == 0:
+            raise ValueError("attention over an empty sequence")
+        o_rot = attention_fp64(q_rot[i], kh, vh, scale)
+        out[i] = o_rot @ H.T
+    return {"out_f64": out, "out_bf16": _bf16_of_f64(out), "q_rot": q_rot}
+
+
+def decode_attention_bf16(cache, layer, seq_ids, q, scale=None):
+    """Plain decode attention over an OracleBF16Cache (no rotation, no quantization)."""
+    q = np.asarray(q, np.float32)
+    D = cache.D
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(D)
+    n = len(seq_ids)
+    out = np.zeros((n,) + q.shape[1:], np.float64)
+    for i, seq in enumerate(seq_ids):
+        k, v = cache.view(layer, int(seq))
+        out[i] = attention_fp64(q[i], k, v, scale)
+    return {"out_f64": out, "out_bf16": _bf16_of_f64(out)}

@@ -1,0 +1,179 @@
+"""Byte placement of codes and scales inside a 16-token tile (oracle; test infrastructure only).
+
+The pages ask for a quantized cache that keeps "paged memory layouts, regular
+memory access, and fused attention execution" ("SAW-INT4: System-Aware 4-Bit
+KV-Cache Quantization for Real-World LLM Serving", Abstract) but print no
+layout.  This module DEFINES the one this library uses; the CUDA path must
+place every byte where these functions say.
+
+Unit of storage: a tile of 16 consecutive token slots of one KV head.
+
+INT4 tile (16*D + 128 bytes):   [K codes 8*D][V codes 8*D][scales 128]
+INT8 tile (32*D + 128 bytes):   [K codes 16*D][V codes 16*D][scales 128]
+BF16 tile (64*D bytes):         [K 16*D bf16][V 16*D bf16]      (baseline cache)
+
+Inside the code blocks the order of nibbles/bytes follows the operand order
+of the 16x8x16 tensor-core multiply the decode kernel feeds from them; the
+functions below state each placement in closed form.  Properties that the
+tests check: every (token, dim) owns exactly one nibble (or byte, or bf16
+element), and every byte of a code block belongs to exactly one token (so a
+token can be written without reading its neighbours).
+
+Scales: a 128-byte block of 32 half2 (s, z) entries.  Entry for token r of
+tensor T (K = 0, V = 1) sits at byte 16*(r % 8) + 4*(2*T + r // 8); the half
+at +0 is the scale s, the half at +2 the zero point z.
+"""
+
+import numpy as np
+
+TILE = 16
+
+
+def int4_tile_bytes(D):
+    return 16 * D + 128
+
+
+def int8_tile_bytes(D):
+    return 32 * D + 128
+
+
+def bf16_tile_bytes(D):
+    return 64 * D
+
+
+def int4_k_nibble(D, r, d):
+    """(byte offset inside the K code block, nibble: 0 = low, 1 = high) of token r, dim d.
+
+    Token r owns the D/2 bytes [r*D/2, (r+1)*D/2).  With d = 32*kk + 8*j + 2*t + e
+    (kk < D/32, j < 4, t < 4, e < 2) and i = j + 4*e, the nibble is number i of
+    the 32-bit word at byte r*D/2 + t*D/8 + 4*kk.
+    """
+    kk, rem = divmod(d, 32)
+    j, rem = divmod(rem, 8)
+    t, e = divmod(rem, 2)
+    i = j + 4 * e
+    return r * (D // 2) + t * (D // 8) + 4 * kk + i // 2, i % 2
+
+
+def int4_v_nibble(D, r, d):
+    """(byte offset inside the V code block, nibble) of token r, dim d.
+
+    With d = 16*m + 8*dh + g (g < 8, dh < 2) and r = 8*th + 2*t + e
+    (t < 4, e < 2, th < 2), the nibble is number i = dh + 2*th + 4*e of the
+    32-bit word at byte 512*(m // 4) + 16*(4*g + t) + 4*(m % 4).
+    """
+    m, rr = divmod(d, 16)
+    dh, g = divmod(rr, 8)
+    th, tt = divmod(r, 8)
+    t, e = divmod(tt, 2)
+    i = dh + 2 * th + 4 * e
+    return 512 * (m // 4) + 16 * (4 * g + t) + 4 * (m % 4) + i // 2, i % 2
+
+
+def int8_k_byte(D, r, d):
+    """Byte offset inside the INT8 K code block of token r, dim d.
+
+    With r = 8*rowhi + g, d = 16*k + 8*h8 + 2*t + e: byte h8 + 2*e of the word
+    at 16*(32*(rowhi*D/64 + k//4) + 4*g + t) + 4*(k % 4).
+    """
+    rowhi, g = divmod(r, 8)
+    k, c = divmod(d, 16)
+    h8, c2 = divmod(c, 8)
+    t, e = divmod(c2, 2)
+    return 16 * (32 * (rowhi * (D // 64) + k // 4) + 4 * g + t) + 4 * (k % 4) + h8 + 2 * e
+
+
+def int8_v_byte(D, r, d):
+    """Byte offset inside the INT8 V code block of token r, dim d.
+
+    With d = 16*m + 8*dh + g and r = 8*th + 2*t + e: word w = 2*m + th, byte
+    dh + 2*e of the word at 16*(32*(w//4) + 4*g + t) + 4*(w % 4).
+    """
+    m, rr = divmod(d, 16)
+    dh, g = divmod(rr, 8)
+    th, tt = divmod(r, 8)
+    t, e = divmod(tt, 2)
+    w = 2 * m + th
+    return 16 * (32 * (w // 4) + 4 * g + t) + 4 * (w % 4) + dh + 2 * e
+
+
+def bf16_k_elem(D, r, d):
+    """Element index (bf16 units) inside the BF16 K block of token r, dim d."""
+    rowhi, g = divmod(r, 8)
+    k, c = divmod(d, 16)
+    h8, c2 = divmod(c, 8)
+    t, e = divmod(c2, 2)
+    reg = rowhi + 2 * h8
+    return 8 * (32 * k + 4 * g + t) + 2 * reg + e
+
+
+def bf16_v_elem(D, r, d):
+    """Element index (bf16 units) inside the BF16 V block of token r, dim d."""
+    m, rr = divmod(d, 16)
+    dh, g = divmod(rr, 8)
+    th, tt = divmod(r, 8)
+    t, e = divmod(tt, 2)
+    reg = dh + 2 * th
+    return 8 * (32 * m + 4 * g + t) + 2 * reg + e
+
+
+def scale_offset(r, tensor):
+    """Byte offset of the half2 (s, z) of token r inside the 128-byte scale block; tensor 0 = K, 1 = V."""
+    return 16 * (r % 8) + 4 * (2 * tensor + r // 8)
+
+
+# ---------------------------------------------------------------------------
+# Tables used by the oracle cache.  For a token slot r they list, per byte of
+# the code block that the token owns, which dims go into the byte.
+
+class Int4Tables:
+    """For token slot r: byte offsets (D/2,) and the dims in the low / high nibble."""
+
+    def __init__(self, D):
+        self.D = D
+        self.k_byte = np.zeros((TILE, D // 2), np.int64)
+        self.k_lo = np.zeros((TILE, D // 2), np.int64)
+        self.k_hi = np.zeros((TILE, D // 2), np.int64)
+        self.v_byte = np.zeros((TILE, D // 2), np.int64)
+        self.v_lo = np.zeros((TILE, D // 2), np.int64)
+        self.v_hi = np.zeros((TILE, D // 2), np.int64)
+        for which, fn, tb, tlo, thi in (("k", int4_k_nibble, self.k_byte, self.k_lo, self.k_hi),
+                                        ("v", int4_v_nibble, self.v_byte, self.v_lo, self.v_hi)):
+            for r in range(TILE):
+                owned = {}
+                for d in range(D):
+                    byte, half = fn(D, r, d)
+                    owned.setdefault(byte, [None, None])[half] = d
+                if len(owned) != D // 2 or any(None in v for v in owned.values()):
+                    raise AssertionError("INT4 %s layout: token %d does not own whole bytes" % (which, r))
+                for n, byte in enumerate(sorted(owned)):
+                    tb[r, n] = byte
+                    tlo[r, n], thi[r, n] = owned[byte]
+
+
+class Int8Tables:
+    """For token slot r: byte offset of each dim (D,) in the K and V code blocks."""
+
+    def __init__(self, D):
+        self.D = D
+        self.k_byte = np.array([[int8_k_byte(D, r, d) for d in range(D)] for r in range(TILE)], np.int64)
+        self.v_byte = np.array([[int8_v_byte(D, r, d) for d in range(D)] for r in range(TILE)], np.int64)
+
+
+class BF16Tables:
+    """For token slot r: bf16 element index of each dim (D,) in the K and V blocks."""
+
+    def __init__(self, D):
+        self.D = D
+        self.k_elem = np.array([[bf16_k_elem(D, r, d) for d in range(D)] for r in range(TILE)], np.int64)
+        self.v_elem = np.array([[bf16_v_elem(D, r, d) for d in range(D)] for r in range(TILE)], np.int64)
+
+
+_cache = {}
+
+
+def tables(kind, D):
+    key = (kind, D)
+    if key not in _cache:
+        _cache[key] = {"int4": Int4Tables, "int8": Int8Tables, "bf16": BF16Tables}[kind](D)
+    return _cache[key]

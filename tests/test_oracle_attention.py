@@ -1,0 +1,155 @@
+"""Pins of the oracle's attention: library SDPA, rotation invariance, special cases, brute force."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import (attention_fp64, decode_attention, decode_attention_bf16, OracleKV4Cache, OracleBF16Cache,
+                    block_diag_hadamard, bf16_round)
+
+
+def _sdpa(q, k, v, scale):
+    Hq, D = q.shape
+    L, Hkv, _ = k.shape
+    G = Hq // Hkv
+    qt = torch.from_numpy(np.asarray(q, np.float64))[:, None, :]                 # [Hq, 1, D]
+    kt = torch.from_numpy(np.asarray(k, np.float64)).permute(1, 0, 2).repeat_interleave(G, 0)
+    vt = torch.from_numpy(np.asarray(v, np.float64)).permute(1, 0, 2).repeat_interleave(G, 0)
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)[:, 0, :].numpy()
+
+
+@pytest.mark.parametrize("Hq,Hkv,L", [(4, 1, 37), (32, 8, 300), (8, 8, 5), (16, 2, 1)])
+def test_matches_torch_sdpa(Hq, Hkv, L):
+    rng = np.random.default_rng(0)
+    q = rng.standard_normal((Hq, 64))
+    k = rng.standard_normal((L, Hkv, 64)) * 2
+    v = rng.standard_normal((L, Hkv, 64))
+    np.testing.assert_allclose(attention_fp64(q, k, v, 0.125), _sdpa(q, k, v, 0.125), rtol=1e-12, atol=1e-13)
+
+
+def test_brute_force_loops():
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal((4, 8))
+    k = rng.standard_normal((6, 2, 8))
+    v = rng.standard_normal((6, 2, 8))
+    out = attention_fp64(q, k, v, 0.3)
+    for j in range(4):
+        h = j // 2
+        s = [0.3 * sum(q[j, d] * k[p, h, d] for d in range(8)) for p in range(6)]
+        m = max(s)
+        e = [np.exp(x - m) for x in s]
+        o = [sum(e[p] * v[p, h, d] for p in range(6)) / sum(e) for d in range(8)]
+        np.testing.assert_allclose(out[j], o, rtol=1e-13)
+
+
+def test_rotation_invariance():
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal((8, 128))
+    k = rng.standard_normal((50, 2, 128))
+    v = rng.standard_normal((50, 2, 128))
+    for Bh in (128, 64, 16):
+        H = block_diag_hadamard(128, Bh)
+        rot = attention_fp64(q @ H.T, k @ H.T, v @ H.T, 0.1) @ H    # H^{-1} = H^T
+        np.testing.assert_allclose(rot, attention_fp64(q, k, v, 0.1), atol=1e-12)
+
+
+def test_gqa_grouping_is_contiguous():
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((8, 16))
+    k = rng.standard_normal((9, 2, 16))
+    v = rng.standard_normal((9, 2, 16))
+    a = attention_fp64(q, k, v, 0.25)
+    v2 = v.copy()
+    v2[:, 0] += 1.0
+    b = attention_fp64(q, k, v2, 0.25)
+    assert np.all(np.abs(a[:4] - b[:4]) > 0.5) and np.array_equal(a[4:], b[4:])
+
+
+def _cfg(D=64, Bh=64, S=4, W=32, Hkv=1, Hq=4):
+    return dict(num_layers=1, max_seqs=2, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D, page_size=16,
+                num_pages=40, max_pages_per_seq=20, hadamard_block=Bh, sink_tokens=S, recent_window=W)
+
+
+def _table():
+    t = np.arange(40, dtype=np.int32).reshape(2, 20)[:, ::-1].copy()
+    return t
+
+
+def test_quantization_free_reduction_to_textbook():
+    # Bh = 1 and values z + c4*17*2^-k with codes c4 = 0..15 present: the INT4
+    # scale is 17*2^-k and the INT8 scale 2^-k (codes 17*c4), so both encodings
+    # are exact and decode attention is textbook attention on the inputs.
+    cfg = _cfg(Bh=1)
+    rng = np.random.default_rng(4)
+    L = 70
+    codes = rng.integers(0, 16, (L, 1, 64))
+    codes[:, :, 0], codes[:, :, 1] = 0, 15
+    k = (codes * (17 / 64) - 2.0).astype(np.float32)
+    v = (np.roll(codes, 3, axis=2) * (17 / 128) + 1.0).astype(np.float32)
+    q = bf16_round(rng.standard_normal((1, 4, 64)).astype(np.float32))
+    cache = OracleKV4Cache(cfg, _table())
+    cache.append(0, [1], [0, L], k, v)
+    res = decode_attention(cache, 0, [1], q)
+    np.testing.assert_allclose(res["out_f64"][0], _sdpa(q[0], k, v, 0.125), atol=1e-12)
+    np.testing.assert_allclose(decode_attention(cache, 0, [1], q, protected=False)["out_f64"][0],
+                               _sdpa(q[0], k, v, 0.125), atol=1e-12)
+
+
+def test_single_token_context_returns_its_value():
+    cfg = _cfg()
+    rng = np.random.default_rng(5)
+    k = bf16_round(rng.standard_normal((1, 1, 64)).astype(np.float32))
+    v = bf16_round(rng.standard_normal((1, 1, 64)).astype(np.float32))
+    cache = OracleKV4Cache(cfg, _table())
+    cache.append(0, [0], [0, 1], k, v)
+    q = bf16_round(rng.standard_normal((1, 4, 64)).astype(np.float32))
+    out = decode_attention(cache, 0, [0], q)["out_f64"][0]
+    vh = cache.view(0, 0)[1][0, 0].astype(np.float64) @ block_diag_hadamard(64, 64).T
+    for j in range(4):
+        np.testing.assert_allclose(out[j], vh, atol=1e-12)
+    # the INT8 sink is within its s/2 of the input
+    assert np.max(np.abs(vh - v[0, 0])) < 0.02
+
+
+def test_uniform_keys_give_the_mean_value():
+    # identical keys stay identical only inside one encoding: check the INT4-only
+    # view, and a window covering the whole context (every position INT8)
+    rng = np.random.default_rng(6)
+    L = 48
+    k = np.repeat(bf16_round(rng.standard_normal((1, 1, 64)).astype(np.float32)), L, axis=0)
+    v = bf16_round(rng.standard_normal((L, 1, 64)).astype(np.float32))
+    q = bf16_round(rng.standard_normal((1, 4, 64)).astype(np.float32))
+    for W, protected in ((16, False), (64, True)):
+        cache = OracleKV4Cache(_cfg(S=0, W=W), _table())
+        cache.append(0, [0], [0, L], k, v)
+        out = decode_attention(cache, 0, [0], q, protected=protected)["out_f64"][0]
+        vh = cache.view(0, 0, protected=protected)[1][:, 0].astype(np.float64) @ block_diag_hadamard(64, 64).T
+        for j in range(4):
+            np.testing.assert_allclose(out[j], vh.mean(0), atol=1e-12)
+
+
+def test_quantized_attention_close_to_exact():
+    # INT4 with rotation stays near the unquantized answer (sanity of the whole chain).
+    cfg = _cfg(D=128, Bh=128, W=32)
+    rng = np.random.default_rng(7)
+    L = 300
+    k = bf16_round(rng.standard_normal((L, 1, 128)).astype(np.float32))
+    v = bf16_round(rng.standard_normal((L, 1, 128)).astype(np.float32))
+    cache = OracleKV4Cache(cfg, _table())
+    cache.append(0, [0], [0, L], k, v)
+    q = bf16_round(rng.standard_normal((1, 4, 128)).astype(np.float32))
+    out = decode_attention(cache, 0, [0], q)["out_f64"][0]
+    exact = attention_fp64(q[0], k, v, 1 / np.sqrt(128))
+    assert np.linalg.norm(out - exact) / np.linalg.norm(exact) < 0.2
+
+
+def test_bf16_baseline_oracle():
+    cfg = _cfg(D=128, Bh=128)
+    rng = np.random.default_rng(8)
+    k = bf16_round(rng.standard_normal((77, 1, 128)).astype(np.float32))
+    v = bf16_round(rng.standard_normal((77, 1, 128)).astype(np.float32))
+    cache = OracleBF16Cache(cfg, _table())
+    cache.append(0, [1], [0, 77], k, v)
+    q = bf16_round(rng.standard_normal((1, 4, 128)).astype(np.float32))
+    out = decode_attention_bf16(cache, 0, [1], q)["out_f64"][0]
+    np.testing.assert_allclose(out, _sdpa(q[0], k, v, 1 / np.sqrt(128)), atol=1e-12)

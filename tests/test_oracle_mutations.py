@@ -1,0 +1,106 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that a pin catches each one.
+
+Each case swaps one oracle function for a mutated copy inside the test only
+(monkeypatch) and re-runs the property that pins that function.
+"""
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+import oracle
+from oracle import hadamard, quant, cache as cache_mod, attention as attn_mod
+from oracle.hadamard import rotation_constant_fp32
+
+
+def _fwht_swapped_signs(x, Bh):
+    x = np.asarray(x, np.float32)
+    lead, D = x.shape[:-1], x.shape[-1]
+    y = x.reshape(lead + (D // Bh, Bh)).copy()
+    h = 1
+    while h < Bh:
+        y = y.reshape(lead + (D // Bh, Bh // (2 * h), 2, h))
+        a, b = y[..., 0, :], y[..., 1, :]
+        y = np.stack([a - b, a + b], axis=-2)      # mistake: outputs swapped
+        h *= 2
+    return (y.reshape(lead + (D,)) * rotation_constant_fp32(Bh)).astype(np.float32)
+
+
+def _fwht_unscaled(x, Bh):
+    return (hadamard.fwht_fp32(x, Bh) / rotation_constant_fp32(Bh)).astype(np.float32)  # mistake: no 1/sqrt(Bh)
+
+
+@pytest.mark.parametrize("bad", [_fwht_swapped_signs, _fwht_unscaled])
+def test_fwht_mistakes_fail_the_column_pin(bad):
+    Bh = 64
+    out = bad(np.eye(Bh, dtype=np.float32), Bh)
+    expect = (scipy.linalg.hadamard(Bh) / np.sqrt(Bh)).T.astype(np.float32)
+    assert not np.array_equal(out, expect)
+
+
+def _quantize_rne_zero(x, bits):
+    Q = np.float32(2 ** bits - 1)
+    x = quant.clamp_fp16_range(x)
+    mn, mx = x.min(-1), x.max(-1)
+    z16 = mn.astype(np.float16)                      # mistake: nearest instead of downward
+    z = z16.astype(np.float32)
+    r = (mx - z).astype(np.float32)
+    s16 = quant.fp16_round_up((r / Q).astype(np.float32))
+    s16 = np.where(r == 0, np.float16(1), s16).astype(np.float16)
+    s = s16.astype(np.float32)
+    c = np.clip(np.rint(((x - z[..., None]) / s[..., None]).astype(np.float32)), 0, Q).astype(np.uint8)
+    return c, s16, z16
+
+
+def test_zero_point_rounding_mistake_fails_the_definition_pin():
+    rng = np.random.default_rng(0)
+    x = (rng.standard_normal((300, 64)) * 3 + 40).astype(np.float32)
+    c, s, z = _quantize_rne_zero(x, 4)
+    assert np.any(z.astype(np.float64) > x.min(1))    # the pin requires z <= min
+
+
+def test_dropped_zero_point_fails_the_round_trip_pin():
+    x = (np.arange(16, dtype=np.float32) * 0.5 - 3.0)[None]
+    c, s, z = quant.quantize_groups(x, 4)
+    wrong = (c.astype(np.float64) * s.astype(np.float64)[..., None]).astype(np.float32)   # mistake: no + z
+    assert not np.array_equal(wrong, x)
+    np.testing.assert_array_equal(quant.dequantize_groups(c, s, z), x)
+
+
+def test_wrong_gqa_mapping_fails_the_sdpa_pin(monkeypatch):
+    def bad_attention(q, k, v, scale):
+        q, k, v = (np.asarray(a, np.float64) for a in (q, k, v))
+        Hq, D = q.shape
+        Hkv = k.shape[1]
+        o = np.zeros((Hq, D))
+        for j in range(Hq):
+            h = j % Hkv                                  # mistake: interleaved grouping
+            s = scale * (k[:, h] @ q[j])
+            a = np.exp(s - s.max())
+            o[j] = (a / a.sum()) @ v[:, h]
+        return o
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal((8, 16))
+    k = rng.standard_normal((9, 2, 16))
+    v = rng.standard_normal((9, 2, 16))
+    good = attn_mod.attention_fp64(q, k, v, 0.25)
+    assert not np.allclose(bad_attention(q, k, v, 0.25), good)
+
+
+def test_wrong_ring_slot_fails_the_direct_construction_pin(monkeypatch):
+    cfg = dict(num_layers=1, max_seqs=1, num_q_heads=4, num_kv_heads=1, head_dim=64, page_size=16,
+               num_pages=16, max_pages_per_seq=16, hadamard_block=64, sink_tokens=4, recent_window=32)
+    table = np.arange(16, dtype=np.int32)[None]
+    rng = np.random.default_rng(2)
+    k = oracle.bf16_round(rng.standard_normal((80, 1, 64)).astype(np.float32))
+    v = k.copy()
+    good = cache_mod.OracleKV4Cache(cfg, table)
+    for i in range(80):
+        good.append(0, [0], [0, 1], k[i:i + 1], v[i:i + 1])
+    monkeypatch.setattr(cache_mod, "prot_slot", lambda p, S, W: p if p < S else S + (p - S + 1) % W)
+    bad = cache_mod.OracleKV4Cache(cfg, table)
+    for i in range(80):
+        bad.append(0, [0], [0, 1], k[i:i + 1], v[i:i + 1])
+    monkeypatch.undo()
+    # reading the mutated store through the correct slot rule gives wrong values
+    assert not np.array_equal(bad.view(0, 0)[0], good.view(0, 0)[0])
