@@ -1,0 +1,490 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the paged INT4/INT8-protected KV cache on B200.
+
+One step = the whole hot path for one batch: fused rotate+quantize+append of one
+new token per sequence, then decode attention (query rotation and work plan,
+split-K attention over the INT4 pages and the INT8 sink/recent store, merge and
+inverse rotation).  The metric is the algorithmic KV bytes the attention reads
+per step divided by the step time (GB/s), with decode tokens/s and the fraction
+of the measured HBM bandwidth beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl kv4|reference]
+
+Under torchrun each rank runs its own replica of the workload (independent
+sequences, weak scaling, no collective on the data path); the step time is the
+device time (CUDA events) summed over the K steps, maximum over ranks.
+`--impl reference` times the CPU oracle (tests-only restatement of the method)
+on a bounded sample of the same workload.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "decode-attention KV GB/s and tokens/s (INT4+INT8-protect), % of B200 HBM peak"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=32)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="qwen3_8b_layer")
+    ap.add_argument("--impl", default="kv4", choices=["kv4", "reference"])
+    ap.add_argument("--no-compare", action="store_true", help="skip the BF16-KV and INT4-only legs")
+    ap.add_argument("--cpu-seqs", type=int, default=4, help="sequences in the CPU oracle sample")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- helpers
+
+def kv_bytes(lengths, Hkv, D, S, W, int4_only=False):
+    """Algorithmic KV bytes one attention call reads: INT4 136 B and INT8 264 B per token and KV head at D=128."""
+    L = np.asarray(lengths, np.int64)
+    prot = np.zeros_like(L) if int4_only else np.minimum(L, S + W)
+    return int(np.sum(Hkv * ((L - prot) * 2 * (D // 2 + 4) + prot * 2 * (D + 4))))
+
+
+def bf16_bytes(lengths, Hkv, D):
+    return int(np.sum(np.asarray(lengths, np.int64) * Hkv * 2 * D * 2))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha1()
+    for name in ("kv4_attention.cu", "kv4_common.cuh"):
+        with open(os.path.join(ROOT, "int4_kv_cache_paged_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per split-K launch from the committed ncu summary, if it matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "split_k_attention_%s.md" % workload)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "source_sha1")):
+            k, v = line.split(":", 1)
+            vals[k.strip().lstrip("- ")] = v.strip().strip("`")
+    if vals.get("source_sha1") != kernel_source_hash():
+        return None
+    try:
+        return int(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- GPU workload
+
+class Workload:
+    """One replica: INT4 cache populated to L_b - 1 tokens, per-step new tokens and queries on the device."""
+
+    def __init__(self, w, device, extra_tokens, torch):
+        import int4_kv_cache_paged_b200 as kv4
+        self.w = w
+        self.device = device
+        self.L = workloads.context_lengths(w)
+        self.B = len(self.L)
+        table, num_pages, mpps = workloads.block_table(w, self.L, extra_tokens=extra_tokens)
+        self.table = table
+        self.cfg = workloads.cache_config(w, num_pages, mpps)
+        self.cache = kv4.KV4Cache(self.cfg, torch.from_numpy(table), device)
+        self.seq_ids = torch.arange(self.B, dtype=torch.int32, device=device)
+        self.cu_one = torch.arange(self.B + 1, dtype=torch.int32, device=device)
+        self.steps_k = []  # per step: k [B, Hkv, D] bf16
+        self.steps_v = []
+        self.populate(torch, self.cache.append, extra_tokens)
+
+    def populate(self, torch, append_fn, extra_tokens, layer=0, keep_steps=True):
+        w, dev = self.w, self.device
+        batch_k, batch_v, counts, ids = [], [], [], []
+        step_k = [[None] * self.B for _ in range(extra_tokens)]
+        step_v = [[None] * self.B for _ in range(extra_tokens)]
+        budget = 0
+        for s in range(self.B):
+            L = int(self.L[s])
+            k, v = workloads.kv_sequence(w, layer, s, L - 1 + extra_tokens, device=dev)
+            batch_k.append(k[:L - 1])
+            batch_v.append(v[:L - 1])
+            counts.append(L - 1)
+            ids.append(s)
+            for j in range(extra_tokens):
+                step_k[j][s] = k[L - 1 + j]
+                step_v[j][s] = v[L - 1 + j]
+            budget += L
+            if budget > 2_000_000 or s == self.B - 1:
+                cu = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int32, device=dev)
+                append_fn(layer, torch.tensor(ids, dtype=torch.int32, device=dev), cu,
+                          torch.cat(batch_k).contiguous(), torch.cat(batch_v).contiguous(), total_new=int(sum(counts)))
+                batch_k, batch_v, counts, ids, budget = [], [], [], [], 0
+        if keep_steps:
+            self.steps_k = [torch.stack(x).contiguous() for x in step_k]
+            self.steps_v = [torch.stack(x).contiguous() for x in step_v]
+        torch.cuda.synchronize()
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import int4_kv_cache_paged_b200 as kv4
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=device)
+
+    W_, K = args.warmup, args.steps
+    w = workloads.workload(args.workload)
+    if rank > 0:
+        w = workloads.workload(args.workload, seed=w["seed"] + 7919 * rank)   # independent sequences per rank
+    if w["layers"] > 1:
+        raise SystemExit("the benchmark times single-layer workloads; use the stack test for %s" % args.workload)
+    extra = W_ + 2 * K + 1
+    t0 = time.time()
+    wl = Workload(w, device, extra, torch)
+    setup_s = time.time() - t0
+    B, Hkv, D, S, Wn = wl.B, w["Hkv"], w["D"], w["S"], w["W"]
+    ws = wl.cache.workspace(B)
+    out = torch.empty((B, w["Hq"], D), dtype=torch.bfloat16, device=device)
+    qs = [workloads.queries(w, 0, i, device=device) for i in range(W_ + K)]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    n = W_ + K
+    e_step = [(ev(), ev()) for _ in range(n)]
+    e_attn = [(ev(), ev()) for _ in range(n)]
+    e_kern = [(ev(), ev()) for _ in range(n)]
+    step_bytes = []
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    barrier()
+    with ClockSampler(local) as clocks:
+        for i in range(n):
+            if i == W_:
+                barrier()
+            flush.fill_(i & 0xFF)                  # evict the KV of the previous step from L2 (not timed)
+            kv4.kv4_set_attention_events(wl.cache.handle, *e_kern[i])
+            e_step[i][0].record(stream)
+            wl.cache.append(0, wl.seq_ids, wl.cu_one, wl.steps_k[i], wl.steps_v[i], total_new=B)
+            e_attn[i][0].record(stream)
+            wl.cache.attention(0, wl.seq_ids, qs[i], out=out, workspace=ws)
+            e_attn[i][1].record(stream)
+            e_step[i][1].record(stream)
+            step_bytes.append(kv_bytes(wl.L + i, Hkv, D, S, Wn))
+        barrier()
+    kv4.kv4_set_attention_events(wl.cache.handle, None, None)
+    status = wl.cache.status()
+
+    timed = range(W_, n)
+    t_step = sum(e_step[i][0].elapsed_time(e_step[i][1]) for i in timed) / 1e3
+    t_attn = sum(e_attn[i][0].elapsed_time(e_attn[i][1]) for i in timed) / 1e3
+    t_kern = sum(e_kern[i][0].elapsed_time(e_kern[i][1]) for i in timed) / 1e3
+    bytes_timed = sum(step_bytes[i] for i in timed)
+    lens_after = wl.L + n - 1                       # length at the last timed attention call
+
+    # ---- e2e through the public API with host buffers (pinned), copies inside the timed region
+    hk = [wl.steps_k[n + j].cpu().pin_memory() for j in range(K)]
+    hv = [wl.steps_v[n + j].cpu().pin_memory() for j in range(K)]
+    hq = [workloads.queries(w, 0, n + j, device="cpu").pin_memory() for j in range(K)]
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dk, dv, dq = torch.empty_like(wl.steps_k[0]), torch.empty_like(wl.steps_v[0]), torch.empty_like(qs[0])
+    e_e2e = [(ev(), ev()) for _ in range(K)]
+    e2e_bytes = 0
+    barrier()
+    for j in range(K):
+        flush.fill_(j & 0xFF)
+        e_e2e[j][0].record(stream)
+        dk.copy_(hk[j], non_blocking=True)
+        dv.copy_(hv[j], non_blocking=True)
+        dq.copy_(hq[j], non_blocking=True)
+        wl.cache.append(0, wl.seq_ids, wl.cu_one, dk, dv, total_new=B)
+        wl.cache.attention(0, wl.seq_ids, dq, out=out, workspace=ws)
+        hout.copy_(out, non_blocking=True)
+        e_e2e[j][1].record(stream)
+        e2e_bytes += kv_bytes(wl.L + n + j, Hkv, D, S, Wn)
+    barrier()
+    t_e2e = sum(a.elapsed_time(b) for a, b in e_e2e) / 1e3
+    h2d = dk.numel() * 2 + dv.numel() * 2 + dq.numel() * 2
+    d2h = hout.numel() * 2
+
+    # ---- comparison legs on identical inputs (rank-local, untimed by the contract)
+    compare = None
+    if not args.no_compare and world == 1:
+        compare = compare_legs(torch, kv4, w, wl, K, device, flush)
+
+    totals = torch.tensor([t_step, t_e2e, float(bytes_timed), float(e2e_bytes)], dtype=torch.float64, device=device)
+    if world > 1:
+        tmax = totals[:2].clone()
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+        bsum = totals[2:].clone()
+        dist.all_reduce(bsum, op=dist.ReduceOp.SUM)
+        t_step_all, t_e2e_all = tmax.tolist()
+        bytes_all, e2e_bytes_all = bsum.tolist()
+    else:
+        t_step_all, t_e2e_all, bytes_all, e2e_bytes_all = t_step, t_e2e, float(bytes_timed), float(e2e_bytes)
+
+    result = None
+    if rank == 0:
+        peaks, peak_kind = measured_peaks()
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+        achieved = bytes_timed / t_kern / 1e9
+        value = bytes_all / t_step_all / 1e9
+        traffic = profiled_traffic(args.workload)
+        clk = clocks.summary()
+        result = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": W_,
+            "ms_per_step": round(t_step_all / K * 1e3, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "int4/int8 codes, fp16 scales, bf16 q/out, fp16 tensor-core operands, fp32 accumulate",
+            "data": "synthetic (seeded N(0,1) K/V with outlier K channels and a large-norm sink, bf16)",
+            "config": {"workload": args.workload, "batch": B, "q_heads": w["Hq"], "kv_heads": Hkv, "head_dim": D,
+                       "page": w["P"], "hadamard_block": w["Bh"], "sinks": S, "recent_window": Wn,
+                       "context": "%s, mean %.0f at the first timed step" % (w["ctx"][0], float(np.mean(wl.L + W_))),
+                       "kv_bytes_per_step_mb": round(bytes_timed / K / 1e6, 1),
+                       "l2": "flushed before every step by a 256 MB write outside the timed events; "
+                             "per-step KV also exceeds the 126 MB L2",
+                       "parallelism": "replica per GPU" if world > 1 else "single GPU"},
+            "tokens_per_s": round(B * world * K / t_step_all, 1),
+            "hbm_frac_of_%s" % peak_kind: round(value / hbm, 4),
+            "attention_kv_gbs": round(bytes_timed / t_attn / 1e9, 2),
+            "append_us_per_step": round((t_step - t_attn) / K * 1e6, 2),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
+                         "frac": round(achieved / hbm, 4), "traffic": traffic,
+                         "kernel": "attn_kernel (split-K over INT4 pages + INT8 store)",
+                         "peak_source": peak_kind, "bytes_per_launch": int(bytes_timed / K)},
+            "e2e": {"value": round(e2e_bytes_all / t_e2e_all / 1e9, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                    "tokens_per_s": round(B * world * K / t_e2e_all, 1)},
+            "gpu_launches": 4 * K,
+            "clocks": clk,
+            "device_status": status,
+            "setup_s": round(setup_s, 1),
+        }
+        if compare:
+            result["compare"] = compare
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def compare_legs(torch, kv4, w, wl, K, device, flush):
+    """Attention-only time of the INT4 path, the INT4-only mode and the BF16-KV kernel on identical inputs."""
+    B, Hkv, D, S, Wn = wl.B, w["Hkv"], w["D"], w["S"], w["W"]
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    qs = [workloads.queries(w, 0, 1000 + i, device=device) for i in range(K)]
+    out = torch.empty((B, w["Hq"], D), dtype=torch.bfloat16, device=device)
+    L_now = wl.L + int(wl.cache.seq_lens()[0, 0].item()) - int(wl.L[0])
+
+    def time_attn(fn):
+        es = [(ev(), ev()) for _ in range(K)]
+        for i in range(3):
+            fn(qs[i])
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            es[i][0].record()
+            fn(qs[i])
+            es[i][1].record()
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in es) / 1e3 / K
+
+    ws = wl.cache.workspace(B)
+    t_int4 = time_attn(lambda q: wl.cache.attention(0, wl.seq_ids, q, out=out, workspace=ws))
+    t_only = time_attn(lambda q: wl.cache.attention(0, wl.seq_ids, q, out=out, workspace=ws,
+                                                    mode=kv4.KV4_MODE_INT4_ONLY))
+    res = {"int4_protected": {"attention_ms": round(t_int4 * 1e3, 4),
+                              "kv_gbs": round(kv_bytes(L_now, Hkv, D, S, Wn) / t_int4 / 1e9, 1)},
+           "int4_only": {"attention_ms": round(t_only * 1e3, 4),
+                         "kv_gbs": round(kv_bytes(L_now, Hkv, D, S, Wn, int4_only=True) / t_only / 1e9, 1)}}
+    need = bf16_bytes(L_now, Hkv, D)
+    free = torch.cuda.mem_get_info()[0]
+    if need * 1.3 < free:
+        cache16 = kv4.BF16Cache(wl.cfg, torch.from_numpy(wl.table), device)
+        lens = L_now
+        extra_w = dict(w)
+        # identical K/V values: regenerate the same per-sequence tokens up to the current length
+        tmp = Workload.__new__(Workload)
+        tmp.w, tmp.device, tmp.B = w, device, B
+        tmp.L = lens + 1
+        tmp.populate(torch, cache16.append, 0, keep_steps=False)
+        ws16 = cache16.workspace(B)
+        t_bf16 = time_attn(lambda q: cache16.attention(0, wl.seq_ids, q, out=out, workspace=ws16))
+        res["bf16_kv"] = {"attention_ms": round(t_bf16 * 1e3, 4), "kv_gbs": round(need / t_bf16 / 1e9, 1),
+                          "speedup_int4_protected_vs_bf16": round(t_bf16 / t_int4, 3)}
+        del cache16, extra_w
+    else:
+        res["bf16_kv"] = {"skipped": "BF16 cache of %.1f GB does not fit" % (need / 1e9)}
+    return res
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def run_oracle_sample(w, n_seqs, steps, warm=1):
+    """The oracle on `n_seqs` sequences of the workload: populate (untimed), then `steps` decode steps."""
+    import torch
+    from threadpoolctl import threadpool_limits
+    from oracle import OracleKV4Cache, decode_attention
+
+    L = workloads.context_lengths(w)[:n_seqs]
+    table, num_pages, mpps = workloads.block_table(dict(w, batch=n_seqs), L, extra_tokens=steps + warm + 1)
+    cfg = workloads.cache_config(w, num_pages, mpps, max_seqs=n_seqs)
+    orc = OracleKV4Cache(cfg, table)
+    toks = []
+    with threadpool_limits(1):
+        for s in range(n_seqs):
+            k, v = workloads.kv_sequence(w, 0, s, int(L[s]) + steps + warm, device="cpu")
+            k, v = k.float().numpy(), v.float().numpy()
+            orc.append(0, [s], [0, int(L[s]) - 1], k[:L[s] - 1], v[:L[s] - 1])
+            toks.append((k, v))
+        times, nbytes = [], []
+        for i in range(steps + warm):
+            kn = np.stack([toks[s][0][L[s] - 1 + i] for s in range(n_seqs)])
+            vn = np.stack([toks[s][1][L[s] - 1 + i] for s in range(n_seqs)])
+            q = workloads.queries(w, 0, i, n=n_seqs, device="cpu").float().numpy()
+            t0 = time.perf_counter()
+            orc.append(0, list(range(n_seqs)), np.arange(n_seqs + 1), kn, vn)
+            decode_attention(orc, 0, list(range(n_seqs)), q)
+            dt = time.perf_counter() - t0
+            if i >= warm:
+                times.append(dt)
+                nbytes.append(kv_bytes(L + i, w["Hkv"], w["D"], w["S"], w["W"]))
+    return sum(nbytes) / sum(times) / 1e9, times, int(np.mean(L))
+
+
+def cpu_baseline(w, n_seqs):
+    gbs, times, mean_l = run_oracle_sample(w, n_seqs, steps=2)
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "%d of %d sequences (mean context %d), 2 decode steps (append + attention), numpy, "
+                      "BLAS limited to 1 thread; %.1f s per step" % (n_seqs, w["batch"], mean_l, np.mean(times))}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    w = workloads.workload(args.workload)
+    n_seqs = max(1, min(args.cpu_seqs, 2))
+    gbs, times, mean_l = run_oracle_sample(w, n_seqs, steps=args.steps, warm=args.warmup)
+    t = sum(times)
+    base = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "%d of %d sequences (mean context %d) per step, numpy, BLAS limited to 1 thread"
+                      % (n_seqs, w["batch"], mean_l)}
+    return {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 attention, f32 codes",
+            "data": "synthetic", "config": {"workload": args.workload, "batch_sample": n_seqs},
+            "cpu_baseline": base, "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                                          "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        res = run_reference(args)
+        if res is not None:
+            print(json.dumps(res))
+        return
+    res = run_gpu(args)
+    if res is not None:
+        if res["n_gpus"] == 1:
+            res["cpu_baseline"] = cpu_baseline(workloads.workload(args.workload), args.cpu_seqs)
+        print(json.dumps(res))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,233 @@
+/*
+ * kv4.h -- C ABI of a paged INT4 KV cache with INT8-protected positions and
+ * its decode attention, for NVIDIA B200 (sm_100a).
+ *
+ * What it computes
+ * ----------------
+ * New keys/values of each token are rotated by a block-diagonal Hadamard
+ * transform and quantized token-wise (one group per token, KV head and K/V)
+ * to asymmetric INT4 with an fp16 scale and zero point, then written into the
+ * page of a paged cache that the block table names ("SAW-INT4: System-Aware
+ * 4-Bit KV-Cache Quantization for Real-World LLM Serving", Abstract).  A
+ * bounded set of positions -- the first S tokens (attention sinks) and the
+ * W most recent tokens -- is also kept in INT8 and read from there ("KV4-RL:
+ * Unlocking Faster Asynchronous Rollouts for RLVR with INT4 KV Cache
+ * Quantization", Abstract).  Decode attention rotates the bf16 queries by the
+ * same Hadamard transform, attends over the mixed INT4/INT8 cache and rotates
+ * the output back.
+ *
+ * Conventions
+ * -----------
+ * - Every function returns KV4_OK (0) or a negative KV4_ERR_* code; nothing
+ *   aborts the process.  Kernels run asynchronously on the given stream; a
+ *   fault found on the device (bad block-table entry, capacity overflow,
+ *   out-of-range input, a wait that gave up) sets a bit in a device status
+ *   word and skips the affected write, it never traps.  Read the word with
+ *   kv4_get_status().
+ * - All device pointers are caller-owned, 16-byte aligned (the cache buffer
+ *   and the workspace 256-byte aligned), and must stay valid until the work
+ *   queued on the stream has finished.  The library never allocates device
+ *   memory.  A cache lives on the device that holds its buffer; every call on
+ *   it runs there, whatever device the calling thread has selected, and the
+ *   stream must belong to that device.
+ * - Calls on one cache handle must be ordered on one stream; a handle is not
+ *   thread-safe.  Caches on different handles are independent.
+ * - Keys are passed after RoPE; RoPE is not part of this library.
+ * - GQA grouping is contiguous: query head j reads KV head j / (Hq / Hkv).
+ * - bf16 arrays are IEEE bfloat16 bit patterns (uint16); the layout of the
+ *   cache buffer is defined by this library (16-token tiles whose byte order
+ *   follows the tensor-core operand order of the attention kernel).
+ */
+#ifndef KV4_H
+#define KV4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t); NULL means the legacy default stream. */
+typedef struct CUstream_st* kv4_stream_t;
+
+/* Return codes. */
+enum {
+  KV4_OK = 0,
+  KV4_ERR_INVALID_ARG = -1,   /* a null pointer, a negative count, a misaligned pointer   */
+  KV4_ERR_UNSUPPORTED = -2,   /* a shape this build does not support (see kv4_config)     */
+  KV4_ERR_CAPACITY = -3,      /* a buffer smaller than kv4_cache_required_bytes()          */
+  KV4_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed                      */
+  KV4_ERR_DEVICE_FAULT = -5,  /* kv4_get_status() found device status bits set             */
+  KV4_ERR_WORKSPACE = -6      /* workspace smaller than kv4_attention_workspace_bytes()    */
+};
+
+/* Bits of the device status word. */
+enum {
+  KV4_DEV_BAD_PAGE = 1,       /* block-table entry < 0 or >= num_pages: token not written  */
+  KV4_DEV_OVERFLOW = 2,       /* append past max_pages_per_seq * page_size: seq skipped    */
+  KV4_DEV_RANGE = 4,          /* a rotated value was non-finite or beyond +-65504: clamped  */
+  KV4_DEV_TIMEOUT = 8,        /* a bounded wait inside a kernel gave up (~1 s)              */
+  KV4_DEV_BAD_SEQ = 16,       /* a sequence id outside [0, max_seqs): entry skipped        */
+  KV4_DEV_WORKSPACE = 32      /* the attention plan did not fit the workspace              */
+};
+
+/* kv4_decode_attention mode bits. */
+enum {
+  KV4_MODE_PROTECTED = 0,     /* INT8 for protected positions, INT4 elsewhere (the method) */
+  KV4_MODE_INT4_ONLY = 1,     /* read the INT4 pages for every position (ablation)         */
+  KV4_MODE_OUT_F32 = 2        /* write fp32 output instead of bf16 (checking mode)          */
+};
+
+/* kv4_dequantize_debug views. */
+enum {
+  KV4_VIEW_EFFECTIVE = 0,     /* what attention reads in KV4_MODE_PROTECTED                 */
+  KV4_VIEW_INT4 = 1           /* the INT4 page copy of every position                       */
+};
+
+/*
+ * Cache configuration.
+ *   num_layers          >= 1   independent per-layer caches sharing one block table
+ *   max_seqs            >= 1   sequence ids are 0 .. max_seqs-1
+ *   num_q_heads         Hq, a multiple of num_kv_heads with Hq/Hkv <= 8
+ *   num_kv_heads        Hkv >= 1
+ *   head_dim            D, 64 or 128
+ *   page_size           P, a multiple of 16, at most 1024
+ *   num_pages           pages in each layer's pool
+ *   max_pages_per_seq   columns of the block table
+ *   hadamard_block      Bh, a power of two dividing D (1 = no rotation)
+ *   sink_tokens         S >= 0
+ *   recent_window       W >= 1, S + W <= 4096
+ */
+typedef struct {
+  int32_t num_layers, max_seqs, num_q_heads, num_kv_heads, head_dim;
+  int32_t page_size, num_pages, max_pages_per_seq;
+  int32_t hadamard_block;
+  int32_t sink_tokens, recent_window;
+} kv4_config;
+
+typedef struct kv4_cache kv4_cache;   /* opaque host handle owned by the library */
+
+/* Bytes of device memory a cache with this configuration needs (INT4 pools,
+ * INT8 sink/ring stores, sequence lengths and a small state block). */
+int kv4_cache_required_bytes(const kv4_config* cfg, size_t* bytes);
+
+/* Create a cache inside the caller's device buffer `dev_buf` (>= required
+ * bytes, 256-byte aligned).  `dev_block_table` is caller-owned device memory,
+ * int32 [max_seqs][max_pages_per_seq]: entry [s][i] is the page (in every
+ * layer's pool) holding positions [i*P, (i+1)*P) of sequence s, -1 when
+ * unmapped; the caller may update it between calls.  Sequence lengths and the
+ * state block are zeroed on `stream`; pool contents stay undefined. */
+int kv4_cache_create(const kv4_config* cfg, void* dev_buf, size_t bytes, int32_t* dev_block_table,
+                     kv4_stream_t stream, kv4_cache** out);
+
+/* Free the host handle (the device buffer stays the caller's). */
+int kv4_cache_destroy(kv4_cache* cache);
+
+/* Device addresses inside the cache buffer for layer `layer` (any pointer may
+ * be NULL): the INT4 page pool, uint8 [num_pages][Hkv][P/16][16*D+128]; the
+ * INT8 store, uint8 [max_seqs][Hkv][ceil((S+W)/16)][32*D+128]; and the
+ * sequence lengths int32 [num_layers][max_seqs] (all layers). */
+int kv4_cache_layout(const kv4_cache* cache, int32_t layer, void** dev_pages, void** dev_protected,
+                     int32_t** dev_seq_lens);
+
+/* Set the length of sequence `seq_id` to 0 in every layer (its pages can then
+ * be reused or remapped). */
+int kv4_seq_reset(kv4_cache* cache, int32_t seq_id, kv4_stream_t stream);
+
+/*
+ * Fused rotate + quantize + pack + append ("SAW-INT4 ...", Abstract: the
+ * fused rotation-quantization kernel writing into the paged layout).
+ *   dev_seq_ids  int32 [n_seqs], distinct sequence ids
+ *   dev_cu_new   int32 [n_seqs+1], cu_new[0] = 0, non-decreasing; sequence
+ *                seq_ids[i] receives rows cu_new[i] .. cu_new[i+1]-1
+ *   total_new    = cu_new[n_seqs] (host copy, sizes the launch)
+ *   k_new, v_new bf16 [total_new][Hkv][D], post-RoPE keys and values
+ * Every new position p is INT4-encoded into page block_table[s][p / P], slot
+ * p % P; positions p < S and p >= L_new - W are also INT8-encoded into the
+ * sequence's protected store (sink slot p, or ring slot S + (p - S) mod W).
+ * The sequence length of this layer advances by the number of new rows.
+ */
+int kv4_rotate_quantize_append(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids,
+                               const int32_t* dev_cu_new, int32_t n_seqs, int32_t total_new,
+                               const void* k_new, const void* v_new, kv4_stream_t stream);
+
+/* Workspace bytes for kv4_decode_attention over up to `n_seqs` sequences of at
+ * most `max_ctx` tokens each (max_ctx <= 0: the cache capacity
+ * max_pages_per_seq * page_size). */
+int kv4_attention_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_t max_ctx, size_t* bytes);
+
+/*
+ * Decode attention of one query token per sequence over every cached position
+ * 0 .. L-1 of that sequence ("SAW-INT4 ...", Abstract: fused attention over
+ * the paged quantized cache; "KV4-RL ...", Abstract: INT8 sinks and recent
+ * context).
+ *   dev_seq_ids    int32 [n_seqs]
+ *   q              bf16 [n_seqs][Hq][D] (not yet rotated)
+ *   out            bf16 [n_seqs][Hq][D] (fp32 with KV4_MODE_OUT_F32), in the
+ *                  unrotated basis: softmax(scale * q_rot . K^) V^ rotated back
+ *   softmax_scale  <= 0 means 1/sqrt(D)
+ *   mode           KV4_MODE_* bits
+ *   dev_workspace  >= kv4_attention_workspace_bytes(cache, n_seqs, max L, ...)
+ * A sequence of length 0 gives an all-zero output row.
+ * Steps: a planning kernel (query rotation, chunking of every sequence into
+ * work items), a persistent split-K kernel (pages staged by bulk copies,
+ * INT4/INT8 codes turned into tensor-core operands in registers, online
+ * softmax), and a merge kernel (log-sum-exp merge, inverse rotation, store).
+ */
+int kv4_decode_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs,
+                         const void* q, void* out, float softmax_scale, int32_t mode,
+                         void* dev_workspace, size_t ws_bytes, kv4_stream_t stream);
+
+/* Dequantized keys/values of positions [start, start+count) of one sequence,
+ * fp32 [count][Hkv][D], in the rotated basis: x^ = fma(code, s, z) from the
+ * INT4 page or the INT8 store as `view` selects.  For inspection and tests. */
+int kv4_dequantize_debug(kv4_cache* cache, int32_t layer, int32_t seq_id, int32_t start, int32_t count,
+                         int32_t view, float* dev_k_out, float* dev_v_out, kv4_stream_t stream);
+
+/* Synchronize `stream`, return the device status word in *device_status and
+ * clear it.  Returns KV4_ERR_DEVICE_FAULT when any bit was set. */
+int kv4_get_status(kv4_cache* cache, kv4_stream_t stream, int32_t* device_status);
+
+/* Timing hook: record the CUDA events `ev_before` and `ev_after` (cudaEvent_t,
+ * created by the caller on the cache's device) on the call's stream right
+ * before and right after the split-K attention kernel of every later
+ * kv4_decode_attention call on this cache.  NULL, NULL turns it off.  The
+ * events stay owned by the caller. */
+int kv4_set_attention_events(kv4_cache* cache, void* ev_before, void* ev_after);
+
+/* Static text for a return code. */
+const char* kv4_status_string(int status);
+
+/* Build identification: "kv4 <version> sm_100a". */
+const char* kv4_version(void);
+
+/*
+ * BF16 baseline cache: the same paging, block table, split-K attention and
+ * merge, with bf16 keys/values stored as they arrive (no rotation, no
+ * quantization, no protected store).  It exists to measure what the INT4
+ * format saves; hadamard_block, sink_tokens and recent_window are ignored.
+ * Page pool: bf16 [num_pages][Hkv][P/16][16-token tile of 32*D elements].
+ */
+typedef struct kv4bf16_cache kv4bf16_cache;
+
+int kv4bf16_cache_required_bytes(const kv4_config* cfg, size_t* bytes);
+int kv4bf16_cache_create(const kv4_config* cfg, void* dev_buf, size_t bytes, int32_t* dev_block_table,
+                         kv4_stream_t stream, kv4bf16_cache** out);
+int kv4bf16_cache_destroy(kv4bf16_cache* cache);
+int kv4bf16_cache_layout(const kv4bf16_cache* cache, int32_t layer, void** dev_pages, int32_t** dev_seq_lens);
+int kv4bf16_append(kv4bf16_cache* cache, int32_t layer, const int32_t* dev_seq_ids, const int32_t* dev_cu_new,
+                   int32_t n_seqs, int32_t total_new, const void* k_new, const void* v_new, kv4_stream_t stream);
+int kv4bf16_attention_workspace_bytes(const kv4bf16_cache* cache, int32_t n_seqs, int32_t max_ctx, size_t* bytes);
+/* mode: only KV4_MODE_OUT_F32 is meaningful. */
+int kv4bf16_decode_attention(kv4bf16_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs,
+                             const void* q, void* out, float softmax_scale, int32_t mode,
+                             void* dev_workspace, size_t ws_bytes, kv4_stream_t stream);
+int kv4bf16_get_status(kv4bf16_cache* cache, kv4_stream_t stream, int32_t* device_status);
+int kv4bf16_set_attention_events(kv4bf16_cache* cache, void* ev_before, void* ev_after);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KV4_H */

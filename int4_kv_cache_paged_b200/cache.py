@@ -1,0 +1,157 @@
+"""Owning wrappers: device buffers allocated by torch, all work done by libkv4.so."""
+
+import torch
+
+from . import (make_config, kv4_cache_required_bytes, kv4_cache_create, kv4_cache_destroy, kv4_cache_layout,
+               kv4_seq_reset, kv4_rotate_quantize_append, kv4_attention_workspace_bytes, kv4_decode_attention,
+               kv4_dequantize_debug, kv4_get_status, kv4bf16_cache_required_bytes, kv4bf16_cache_create,
+               kv4bf16_cache_destroy, kv4bf16_cache_layout, kv4bf16_append, kv4bf16_attention_workspace_bytes,
+               kv4bf16_decode_attention, kv4bf16_get_status, KV4_VIEW_EFFECTIVE, KV4_MODE_OUT_F32)
+
+TILE = 16
+
+
+def _tile4(D):
+    return 16 * D + 128
+
+
+def _tile8(D):
+    return 32 * D + 128
+
+
+def _tile16(D):
+    return 64 * D
+
+
+class _Base:
+    def _view(self, ptr, nbytes, shape):
+        off = ptr - self.buf.data_ptr()
+        return self.buf[off:off + nbytes].view(*shape)
+
+    def seq_lens(self):
+        c = self.cfg
+        return self._view(self._lens_ptr, 4 * c["num_layers"] * c["max_seqs"], (-1,)).view(torch.int32).view(
+            c["num_layers"], c["max_seqs"])
+
+    def workspace(self, n_seqs, max_ctx=0):
+        nbytes = self._ws_bytes(self.handle, n_seqs, max_ctx)
+        if self._ws is None or self._ws.numel() < nbytes:
+            self._ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def __del__(self):
+        self.close()
+
+
+class KV4Cache(_Base):
+    """A kv4 cache in one torch-allocated device buffer.
+
+    cfg: dict with the kv4_config fields; block_table: int32 [max_seqs, max_pages_per_seq] (any device, copied).
+    """
+
+    def __init__(self, cfg, block_table, device="cuda", stream=None):
+        self.cfg = dict(cfg)
+        self.device = torch.device(device)
+        self.c = make_config(**self.cfg)
+        nbytes = kv4_cache_required_bytes(self.c)
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.block_table = torch.as_tensor(block_table, dtype=torch.int32).to(self.device).contiguous()
+        self._ws = None
+        self._ws_bytes = kv4_attention_workspace_bytes
+        self.handle = kv4_cache_create(self.c, self.buf, self.block_table, stream)
+        _, _, self._lens_ptr = kv4_cache_layout(self.handle, 0)
+
+    def close(self):
+        if getattr(self, "handle", None) is not None:
+            kv4_cache_destroy(self.handle)
+            self.handle = None
+
+    def pages(self, layer):
+        c = self.cfg
+        ptr, _, _ = kv4_cache_layout(self.handle, layer)
+        shape = (c["num_pages"], c["num_kv_heads"], c["page_size"] // TILE, _tile4(c["head_dim"]))
+        n = shape[0] * shape[1] * shape[2] * shape[3]
+        return self._view(ptr, n, shape)
+
+    def protected(self, layer):
+        c = self.cfg
+        _, ptr, _ = kv4_cache_layout(self.handle, layer)
+        npt = -(-(c["sink_tokens"] + c["recent_window"]) // TILE)
+        shape = (c["max_seqs"], c["num_kv_heads"], npt, _tile8(c["head_dim"]))
+        n = shape[0] * shape[1] * shape[2] * shape[3]
+        return self._view(ptr, n, shape)
+
+    def append(self, layer, seq_ids, cu_new, k_new, v_new, total_new=None, stream=None):
+        if total_new is None:
+            total_new = int(k_new.shape[0])
+        kv4_rotate_quantize_append(self.handle, layer, seq_ids, cu_new, int(seq_ids.numel()), total_new,
+                                   k_new, v_new, stream)
+
+    def attention(self, layer, seq_ids, q, out=None, scale=0.0, mode=0, workspace=None, stream=None):
+        n = int(seq_ids.numel())
+        if out is None:
+            dt = torch.float32 if (mode & KV4_MODE_OUT_F32) else torch.bfloat16
+            out = torch.empty(q.shape, dtype=dt, device=self.device)
+        if workspace is None:
+            workspace = self.workspace(n)
+        kv4_decode_attention(self.handle, layer, seq_ids, n, q, out, scale, mode, workspace, stream)
+        return out
+
+    def dequantize(self, layer, seq, start, count, view=KV4_VIEW_EFFECTIVE, stream=None):
+        c = self.cfg
+        k = torch.empty((count, c["num_kv_heads"], c["head_dim"]), dtype=torch.float32, device=self.device)
+        v = torch.empty_like(k)
+        kv4_dequantize_debug(self.handle, layer, seq, start, count, view, k, v, stream)
+        return k, v
+
+    def reset(self, seq, stream=None):
+        kv4_seq_reset(self.handle, seq, stream)
+
+    def status(self, stream=None):
+        return kv4_get_status(self.handle, stream)
+
+
+class BF16Cache(_Base):
+    """The BF16 baseline cache (same paging and attention structure, no quantization)."""
+
+    def __init__(self, cfg, block_table, device="cuda", stream=None):
+        self.cfg = dict(cfg)
+        self.device = torch.device(device)
+        self.c = make_config(**self.cfg)
+        nbytes = kv4bf16_cache_required_bytes(self.c)
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.block_table = torch.as_tensor(block_table, dtype=torch.int32).to(self.device).contiguous()
+        self._ws = None
+        self._ws_bytes = kv4bf16_attention_workspace_bytes
+        self.handle = kv4bf16_cache_create(self.c, self.buf, self.block_table, stream)
+        _, self._lens_ptr = kv4bf16_cache_layout(self.handle, 0)
+
+    def close(self):
+        if getattr(self, "handle", None) is not None:
+            kv4bf16_cache_destroy(self.handle)
+            self.handle = None
+
+    def pages(self, layer):
+        c = self.cfg
+        ptr, _ = kv4bf16_cache_layout(self.handle, layer)
+        shape = (c["num_pages"], c["num_kv_heads"], c["page_size"] // TILE, _tile16(c["head_dim"]))
+        n = shape[0] * shape[1] * shape[2] * shape[3]
+        return self._view(ptr, n, shape)
+
+    def append(self, layer, seq_ids, cu_new, k_new, v_new, total_new=None, stream=None):
+        if total_new is None:
+            total_new = int(k_new.shape[0])
+        kv4bf16_append(self.handle, layer, seq_ids, cu_new, int(seq_ids.numel()), total_new, k_new, v_new, stream)
+
+    def attention(self, layer, seq_ids, q, out=None, scale=0.0, mode=0, workspace=None, stream=None):
+        n = int(seq_ids.numel())
+        if out is None:
+            dt = torch.float32 if (mode & KV4_MODE_OUT_F32) else torch.bfloat16
+            out = torch.empty(q.shape, dtype=dt, device=self.device)
+        if workspace is None:
+            workspace = self.workspace(n)
+        kv4bf16_decode_attention(self.handle, layer, seq_ids, n, q, out, scale, mode, workspace, stream)
+        return out
+
+    def status(self, stream=None):
+        return kv4bf16_get_status(self.handle, stream)

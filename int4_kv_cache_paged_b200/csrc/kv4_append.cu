@@ -1,0 +1,455 @@
+// Fused rotate + quantize + pack + append, the BF16 append, debug dequantization
+// and sequence reset.
+//
+// Method: "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
+// Serving", Abstract -- a fused kernel rotates new K/V with a block-diagonal
+// Hadamard transform, quantizes them token-wise to INT4 and writes them straight
+// into the paged layout; "KV4-RL: Unlocking Faster Asynchronous Rollouts for
+// RLVR with INT4 KV Cache Quantization", Abstract -- sinks and recent tokens are
+// also kept in INT8.
+//
+// One warp handles one (token, KV head, K-or-V) group of D values, D/32 values
+// per lane at dims VPL*lane .. VPL*lane+VPL-1.  The fp32 arithmetic follows a
+// fixed order so the codes are reproducible bit for bit:
+//   rotation: butterfly stages h = 1, 2, ..., Bh/2 (x_i, x_{i+h}) ->
+//             (x_i + x_{i+h}, x_i - x_{i+h}), then one multiply by fp32(1/sqrt(Bh));
+//   quantizer: clamp to +-65504; z = fp16 round-down(min); r = max - z;
+//             s = fp16 round-up(r / Q) (1 when r == 0); code = rint((x - z) / s)
+//             clamped to [0, Q]; every operation round-to-nearest-even fp32.
+#include "kv4_common.cuh"
+
+namespace kv4 {
+
+namespace {
+
+constexpr int APPEND_WARPS = 8;
+
+struct AppendParams {
+  uint8_t* pool;             // INT4 or BF16 pool of the layer
+  uint8_t* prot;             // INT8 store of the layer (INT4 cache only)
+  const int32_t* block_table;
+  int32_t* seq_lens;         // this layer's row
+  const int32_t* seq_ids;
+  const int32_t* cu_new;
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  State* state;
+  int n_seqs, total_new, Hkv, D, P, S, W, Bh;
+  int max_seqs, num_pages, max_pages_per_seq;
+  float rot_c;               // fp32(1/sqrt(Bh))
+};
+
+template <int VPL>
+__device__ __forceinline__ void fwht_warp(float (&x)[VPL], int Bh, float c, int lane) {
+  for (int h = 1; h < Bh; h <<= 1) {
+    if (h < VPL) {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        if ((i & h) == 0) {
+          const float a = x[i], b = x[i + h];
+          x[i] = __fadd_rn(a, b);
+          x[i + h] = __fsub_rn(a, b);
+        }
+      }
+    } else {
+      const int lm = h / VPL;
+      const bool upper = (lane & lm) != 0;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const float other = __shfl_xor_sync(0xffffffffu, x[i], lm);
+        // lower element: x_i + x_{i+h}; upper element: x_i - x_{i+h} (x_i is the partner)
+        x[i] = upper ? __fsub_rn(other, x[i]) : __fadd_rn(x[i], other);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) x[i] = __fmul_rn(x[i], c);
+}
+
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Quantize the warp's group with Q = 2^bits - 1; codes go to smem, (s, z) are returned packed as half2 bits.
+template <int VPL>
+__device__ __forceinline__ uint32_t quantize_group(const float (&x)[VPL], float mn, float mx, float Q,
+                                                   uint8_t* codes, int lane) {
+  const __half z16 = __float2half_rd(mn);
+  const float z = __half2float(z16);
+  const float r = __fsub_rn(mx, z);
+  const __half s16 = (r == 0.f) ? __float2half(1.f) : __float2half_ru(__fdiv_rn(r, Q));
+  const float s = __half2float(s16);
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    float c = rintf(__fdiv_rn(__fsub_rn(x[i], z), s));
+    c = fminf(fmaxf(c, 0.f), Q);
+    codes[VPL * lane + i] = static_cast<uint8_t>(c);
+  }
+  return static_cast<uint32_t>(__half_as_ushort(s16)) | (static_cast<uint32_t>(__half_as_ushort(z16)) << 16);
+}
+
+// Write one token's INT4 codes (K: tensor 0, V: tensor 1) and scales into its tile.
+__device__ __forceinline__ void store_int4(uint8_t* tile, int r, int tensor, const uint8_t* codes, uint32_t sz,
+                                           int D, int lane) {
+  if (tensor == 0) {
+    const int nkk = D / 32;
+    if (lane < D / 8) {
+      const int t = lane / nkk, kk = lane % nkk;
+      uint32_t w = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int d = 32 * kk + 8 * (i & 3) + 2 * t + (i >> 2);
+        w |= static_cast<uint32_t>(codes[d]) << (4 * i);
+      }
+      *reinterpret_cast<uint32_t*>(tile + r * (D / 2) + t * (D / 8) + 4 * kk) = w;
+    }
+  } else {
+    const int t = (r & 7) >> 1, e = r & 1, th = r >> 3;
+    for (int q = lane; q < D / 2; q += 32) {
+      const int m = q >> 3, g = q & 7;
+      const uint8_t b = static_cast<uint8_t>(codes[16 * m + g] | (codes[16 * m + g + 8] << 4));
+      tile[8 * D + 512 * (m >> 2) + 16 * (4 * g + t) + 4 * (m & 3) + th + 2 * e] = b;
+    }
+  }
+  if (lane == 0) *reinterpret_cast<uint32_t*>(tile + 16 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3))) = sz;
+}
+
+// Write one token's INT8 codes and scales into its protected tile.
+__device__ __forceinline__ void store_int8(uint8_t* tile, int r, int tensor, const uint8_t* codes, uint32_t sz,
+                                           int D, int lane) {
+  const int rowhi = r >> 3, g = r & 7;
+  if (tensor == 0) {
+    if (lane < D / 4) {
+      const int k = lane >> 2, t = lane & 3;
+      const uint32_t w = static_cast<uint32_t>(codes[16 * k + 2 * t]) |
+                         (static_cast<uint32_t>(codes[16 * k + 8 + 2 * t]) << 8) |
+                         (static_cast<uint32_t>(codes[16 * k + 2 * t + 1]) << 16) |
+                         (static_cast<uint32_t>(codes[16 * k + 8 + 2 * t + 1]) << 24);
+      *reinterpret_cast<uint32_t*>(tile + 16 * (32 * (rowhi * (D / 64) + (k >> 2)) + 4 * g + t) + 4 * (k & 3)) = w;
+    }
+  } else {
+    const int t = (r & 7) >> 1, e = r & 1, th = r >> 3;
+    for (int q = lane; q < D / 2; q += 32) {
+      const int m = q >> 3, gg = q & 7;
+      const int w = 2 * m + th;
+      const uint16_t v = static_cast<uint16_t>(codes[16 * m + gg] | (codes[16 * m + gg + 8] << 8));
+      *reinterpret_cast<uint16_t*>(tile + 16 * D + 16 * (32 * (w >> 2) + 4 * gg + t) + 4 * (w & 3) + 2 * e) = v;
+    }
+  }
+  if (lane == 0) *reinterpret_cast<uint32_t*>(tile + 32 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3))) = sz;
+}
+
+__device__ __forceinline__ int find_seq(const int* cu, int n_seqs, int n) {
+  int lo = 0, hi = n_seqs;  // largest i with cu[i] <= n
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (cu[mid] <= n) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// Last block of an append launch: advance the sequence lengths and re-arm the counter.
+__device__ void finish_append(const AppendParams& p) {
+  __shared__ int s_last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = (atomicAdd(&p.state->append_done, 1) == static_cast<int>(gridDim.x) - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int cap = p.max_pages_per_seq * p.P;
+  for (int i = threadIdx.x; i < p.n_seqs; i += blockDim.x) {
+    const int seq = p.seq_ids[i];
+    if (seq < 0 || seq >= p.max_seqs) continue;
+    const int n = p.cu_new[i + 1] - p.cu_new[i];
+    const int L = p.seq_lens[seq];
+    if (n > 0 && L + n <= cap) p.seq_lens[seq] = L + n;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) p.state->append_done = 0;
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams p) {
+  constexpr int VPL = D / 32;
+  extern __shared__ int s_cu[];
+  __shared__ uint8_t s_codes[APPEND_WARPS][2][D];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i <= p.n_seqs; i += blockDim.x) s_cu[i] = p.cu_new[i];
+  __syncthreads();
+
+  const long long job = static_cast<long long>(blockIdx.x) * APPEND_WARPS + warp;
+  const long long n_jobs = static_cast<long long>(p.total_new) * p.Hkv * 2;
+  if (job < n_jobs) {
+    const int tensor = static_cast<int>(job & 1);
+    const int h = static_cast<int>((job >> 1) % p.Hkv);
+    const int n = static_cast<int>((job >> 1) / p.Hkv);
+    const int i = find_seq(s_cu, p.n_seqs, n);
+    const int seq = p.seq_ids[i];
+    const int cap = p.max_pages_per_seq * p.P;
+    bool ok = true;
+    if (seq < 0 || seq >= p.max_seqs) {
+      if (lane == 0) atomicOr(&p.state->status, KV4_DEV_BAD_SEQ);
+      ok = false;
+    }
+    int pos = 0, L_new = 0;
+    if (ok) {
+      const int L_old = p.seq_lens[seq];
+      L_new = L_old + (s_cu[i + 1] - s_cu[i]);
+      pos = L_old + (n - s_cu[i]);
+      if (L_new > cap) {
+        if (lane == 0) atomicOr(&p.state->status, KV4_DEV_OVERFLOW);
+        ok = false;
+      }
+    }
+    int page = -1;
+    if (ok) {
+      page = p.block_table[static_cast<long long>(seq) * p.max_pages_per_seq + pos / p.P];
+      if (page < 0 || page >= p.num_pages) {
+        if (lane == 0) atomicOr(&p.state->status, KV4_DEV_BAD_PAGE);
+        ok = false;
+      }
+    }
+    if (ok) {
+      const uint16_t* src = (tensor ? p.v_new : p.k_new) + (static_cast<long long>(n) * p.Hkv + h) * D;
+      uint16_t raw[VPL];
+      if constexpr (VPL == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(src + 4 * lane);
+        raw[0] = u.x & 0xFFFF; raw[1] = u.x >> 16; raw[2] = u.y & 0xFFFF; raw[3] = u.y >> 16;
+      } else {
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(src + 2 * lane);
+        raw[0] = u & 0xFFFF; raw[1] = u >> 16;
+      }
+      const int r = pos & (TILE - 1);
+      const long long tile_idx = (static_cast<long long>(page) * p.Hkv + h) * (p.P / TILE) + (pos % p.P) / TILE;
+      if constexpr (BF16) {
+        uint16_t* tile = reinterpret_cast<uint16_t*>(p.pool + tile_idx * tile16_bytes(D));
+        // share the row through smem so each lane can store element pairs
+        uint16_t* row = reinterpret_cast<uint16_t*>(s_codes[warp][0]);
+#pragma unroll
+        for (int k = 0; k < VPL; ++k) row[VPL * lane + k] = raw[k];
+        __syncwarp();
+        const int rowhi = r >> 3, g = r & 7;
+        if (tensor == 0) {
+          for (int q = lane; q < D / 2; q += 32) {   // q = (k, h8, t): dims 16k + 8h8 + 2t + {0,1}
+            const int k = q >> 3, h8 = (q >> 2) & 1, t = q & 3;
+            const int d = 16 * k + 8 * h8 + 2 * t;
+            const uint32_t v = static_cast<uint32_t>(row[d]) | (static_cast<uint32_t>(row[d + 1]) << 16);
+            *reinterpret_cast<uint32_t*>(tile + 8 * (32 * k + 4 * g + t) + 2 * (rowhi + 2 * h8)) = v;
+          }
+        } else {
+          const int t = (r & 7) >> 1, e = r & 1, th = r >> 3;
+          for (int d = lane; d < D; d += 32) {
+            const int m = d >> 4, dh = (d >> 3) & 1, gg = d & 7;
+            tile[16 * D + 8 * (32 * m + 4 * gg + t) + 2 * (dh + 2 * th) + e] = row[d];
+          }
+        }
+      } else {
+        float x[VPL];
+        bool bad = false;
+#pragma unroll
+        for (int k = 0; k < VPL; ++k) {
+          const float v = __bfloat162float(__ushort_as_bfloat16(raw[k]));
+          bad |= !(fabsf(v) <= 3.0e38f);
+          x[k] = v;
+        }
+        fwht_warp<VPL>(x, p.Bh, p.rot_c, lane);
+#pragma unroll
+        for (int k = 0; k < VPL; ++k) {
+          const float c = fminf(fmaxf(x[k], -65504.f), 65504.f);
+          bad |= (c != x[k]);
+          x[k] = c;
+        }
+        if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&p.state->status, KV4_DEV_RANGE);
+        float mn = x[0], mx = x[0];
+#pragma unroll
+        for (int k = 1; k < VPL; ++k) { mn = fminf(mn, x[k]); mx = fmaxf(mx, x[k]); }
+        mn = warp_min(mn);
+        mx = warp_max(mx);
+        uint8_t* c4 = s_codes[warp][0];
+        uint8_t* c8 = s_codes[warp][1];
+        const uint32_t sz4 = quantize_group<VPL>(x, mn, mx, 15.f, c4, lane);
+        const bool protect = pos < p.S || pos >= L_new - p.W;
+        uint32_t sz8 = 0;
+        if (protect) sz8 = quantize_group<VPL>(x, mn, mx, 255.f, c8, lane);
+        __syncwarp();
+        store_int4(p.pool + tile_idx * tile4_bytes(D), r, tensor, c4, sz4, D, lane);
+        if (protect) {
+          const int slot = pos < p.S ? pos : p.S + (pos - p.S) % p.W;
+          const int npt = n_prot_tiles(p.S, p.W);
+          uint8_t* t8 = p.prot + ((static_cast<long long>(seq) * p.Hkv + h) * npt + slot / TILE) * tile8_bytes(D);
+          store_int8(t8, slot & (TILE - 1), tensor, c8, sz8, D, lane);
+        }
+      }
+    }
+  }
+  finish_append(p);
+}
+
+// ---------------------------------------------------------------------------
+
+struct DequantParams {
+  const uint8_t* pool;
+  const uint8_t* prot;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  State* state;
+  float* k_out;
+  float* v_out;
+  int seq, start, count, view;
+  int Hkv, D, P, S, W, max_pages_per_seq, num_pages;
+};
+
+__global__ void dequant_kernel(DequantParams p) {
+  const int lane = threadIdx.x & 31;
+  const long long job = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (job >= static_cast<long long>(p.count) * p.Hkv * 2) return;
+  const int tensor = static_cast<int>(job & 1);
+  const int h = static_cast<int>((job >> 1) % p.Hkv);
+  const int j = static_cast<int>((job >> 1) / p.Hkv);
+  const int pos = p.start + j;
+  const int L = p.seq_lens[p.seq];
+  const int D = p.D;
+  float* out = (tensor ? p.v_out : p.k_out) + (static_cast<long long>(j) * p.Hkv + h) * D;
+  const bool protect = p.view == KV4_VIEW_EFFECTIVE && (pos < p.S || pos >= L - p.W);
+  if (protect) {
+    const int slot = pos < p.S ? pos : p.S + (pos - p.S) % p.W;
+    const int r = slot & 15, rowhi = r >> 3, g = r & 7;
+    const uint8_t* tile = p.prot + ((static_cast<long long>(p.seq) * p.Hkv + h) * n_prot_tiles(p.S, p.W) + slot / 16) *
+                                       tile8_bytes(D);
+    const uint32_t sz = *reinterpret_cast<const uint32_t*>(tile + 32 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3)));
+    const float s = half_lo(sz), z = half_hi(sz);
+    for (int d = lane; d < D; d += 32) {
+      int off;
+      if (tensor == 0) {
+        const int k = d >> 4, c = d & 15, h8 = c >> 3, t = (c & 7) >> 1, e = c & 1;
+        off = 16 * (32 * (rowhi * (D / 64) + (k >> 2)) + 4 * g + t) + 4 * (k & 3) + h8 + 2 * e;
+      } else {
+        const int m = d >> 4, dh = (d >> 3) & 1, gg = d & 7, th = r >> 3, t = (r & 7) >> 1, e = r & 1;
+        const int w = 2 * m + th;
+        off = 16 * D + 16 * (32 * (w >> 2) + 4 * gg + t) + 4 * (w & 3) + dh + 2 * e;
+      }
+      out[d] = __fmaf_rn(static_cast<float>(tile[off]), s, z);
+    }
+  } else {
+    const int page = p.block_table[static_cast<long long>(p.seq) * p.max_pages_per_seq + pos / p.P];
+    if (page < 0 || page >= p.num_pages) {
+      if (lane == 0) atomicOr(&p.state->status, KV4_DEV_BAD_PAGE);
+      return;
+    }
+    const int r = pos & 15;
+    const uint8_t* tile = p.pool + ((static_cast<long long>(page) * p.Hkv + h) * (p.P / 16) + (pos % p.P) / 16) *
+                                       tile4_bytes(D);
+    const uint32_t sz = *reinterpret_cast<const uint32_t*>(tile + 16 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3)));
+    const float s = half_lo(sz), z = half_hi(sz);
+    for (int d = lane; d < D; d += 32) {
+      int byte, half;
+      if (tensor == 0) {
+        const int kk = d >> 5, jj = (d >> 3) & 3, t = (d >> 1) & 3, e = d & 1, i = jj + 4 * e;
+        byte = r * (D / 2) + t * (D / 8) + 4 * kk + (i >> 1);
+        half = i & 1;
+      } else {
+        const int m = d >> 4, dh = (d >> 3) & 1, g = d & 7, th = r >> 3, t = (r & 7) >> 1, e = r & 1;
+        byte = 8 * D + 512 * (m >> 2) + 16 * (4 * g + t) + 4 * (m & 3) + th + 2 * e;
+        half = dh;
+      }
+      const int code = (tile[byte] >> (4 * half)) & 15;
+      out[d] = __fmaf_rn(static_cast<float>(code), s, z);
+    }
+  }
+}
+
+__global__ void seq_reset_kernel(int32_t* seq_lens, int num_layers, int max_seqs, int seq) {
+  const int l = blockIdx.x * blockDim.x + threadIdx.x;
+  if (l < num_layers) seq_lens[static_cast<long long>(l) * max_seqs + seq] = 0;
+}
+
+}  // namespace
+
+int launch_append(kv4_cache* c, int layer, const int32_t* seq_ids, const int32_t* cu_new, int n_seqs, int total_new,
+                  const void* k_new, const void* v_new, cudaStream_t stream) {
+  const kv4_config& cfg = c->cfg;
+  AppendParams p{};
+  uint8_t* lbase = c->base + c->pool_offset + static_cast<size_t>(layer) * c->layer_stride;
+  p.pool = lbase;
+  p.prot = c->bf16 ? nullptr : lbase + c->pool_bytes;
+  p.block_table = c->block_table;
+  p.seq_lens = c->seq_lens + static_cast<size_t>(layer) * cfg.max_seqs;
+  p.seq_ids = seq_ids;
+  p.cu_new = cu_new;
+  p.k_new = static_cast<const uint16_t*>(k_new);
+  p.v_new = static_cast<const uint16_t*>(v_new);
+  p.state = c->state;
+  p.n_seqs = n_seqs;
+  p.total_new = total_new;
+  p.Hkv = cfg.num_kv_heads;
+  p.D = cfg.head_dim;
+  p.P = cfg.page_size;
+  p.S = cfg.sink_tokens;
+  p.W = cfg.recent_window;
+  p.Bh = c->bf16 ? 1 : cfg.hadamard_block;
+  p.max_seqs = cfg.max_seqs;
+  p.num_pages = cfg.num_pages;
+  p.max_pages_per_seq = cfg.max_pages_per_seq;
+  p.rot_c = static_cast<float>(1.0 / sqrt(static_cast<double>(p.Bh)));
+  const long long jobs = static_cast<long long>(total_new) * p.Hkv * 2;
+  const long long blocks = (jobs + APPEND_WARPS - 1) / APPEND_WARPS;
+  if (blocks > 0x7fffffffLL) return KV4_ERR_UNSUPPORTED;
+  const size_t smem = sizeof(int) * (n_seqs + 1);
+  if (smem > 48 * 1024) return KV4_ERR_UNSUPPORTED;
+  dim3 grid(static_cast<unsigned>(blocks)), block(32 * APPEND_WARPS);
+  if (p.D == 128) {
+    if (c->bf16) append_kernel<128, true><<<grid, block, smem, stream>>>(p);
+    else append_kernel<128, false><<<grid, block, smem, stream>>>(p);
+  } else {
+    if (c->bf16) append_kernel<64, true><<<grid, block, smem, stream>>>(p);
+    else append_kernel<64, false><<<grid, block, smem, stream>>>(p);
+  }
+  return cudaGetLastError() == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+}
+
+int launch_dequantize_debug(kv4_cache* c, int layer, int seq_id, int start, int count, int view, float* k_out,
+                            float* v_out, cudaStream_t stream) {
+  const kv4_config& cfg = c->cfg;
+  DequantParams p{};
+  const uint8_t* lbase = c->base + c->pool_offset + static_cast<size_t>(layer) * c->layer_stride;
+  p.pool = lbase;
+  p.prot = lbase + c->pool_bytes;
+  p.block_table = c->block_table;
+  p.seq_lens = c->seq_lens + static_cast<size_t>(layer) * cfg.max_seqs;
+  p.state = c->state;
+  p.k_out = k_out;
+  p.v_out = v_out;
+  p.seq = seq_id;
+  p.start = start;
+  p.count = count;
+  p.view = view;
+  p.Hkv = cfg.num_kv_heads;
+  p.D = cfg.head_dim;
+  p.P = cfg.page_size;
+  p.S = cfg.sink_tokens;
+  p.W = cfg.recent_window;
+  p.max_pages_per_seq = cfg.max_pages_per_seq;
+  p.num_pages = cfg.num_pages;
+  const long long threads = static_cast<long long>(count) * p.Hkv * 2 * 32;
+  const long long blocks = (threads + 255) / 256;
+  dequant_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+}
+
+int launch_seq_reset(kv4_cache* c, int seq_id, cudaStream_t stream) {
+  const int L = c->cfg.num_layers;
+  seq_reset_kernel<<<(L + 127) / 128, 128, 0, stream>>>(c->seq_lens, L, c->cfg.max_seqs, seq_id);
+  return cudaGetLastError() == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+}
+
+}  // namespace kv4

@@ -1,0 +1,877 @@
+// Split-K decode attention over the paged INT4/INT8 cache (and the BF16 baseline).
+//
+// Method: "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
+// Serving", Abstract -- fused attention over a paged, token-wise INT4 cache whose
+// keys were rotated by a block-diagonal Hadamard transform (the query receives the
+// same rotation); "KV4-RL: Unlocking Faster Asynchronous Rollouts for RLVR with
+// INT4 KV Cache Quantization", Abstract -- sinks and recent positions are read
+// from INT8.  Scale and zero point are folded out of the inner products, in the
+// spirit of the folded-scale kernels of "KV Cache Quantization" (topic page),
+// item 2:
+//     q . k^  = s_k * (q . c_k) + z_k * sum(q)
+//     sum_p a_p v^_p = sum_p (a_p s_p) c_p + sum_p a_p z_p
+// so the tensor cores multiply raw integer codes (exact in fp16) by fp16 q
+// (scaled by a power of two) and by fp16 a_p * s_p.
+//
+// Three kernels per call:
+//   prep    one warp per (sequence, KV head): rotates the G queries (fp32 FWHT,
+//           bf16 rounding), lays them out as B operands, and cuts the sequence
+//           into work items (chunks of 16-token tiles plus one item for the INT8
+//           store), appended to three lists by atomics: full chunks, tail chunks,
+//           protected items -- largest first for the dynamic scheduler.
+//   attn    persistent, 2 CTAs per SM, 7 consumer warps + 1 producer warp.  The
+//           producer claims items with an atomic counter and streams their tiles
+//           into a shared-memory ring with 1-D bulk copies (mbarrier completion);
+//           consumer warp w takes tiles w, w+7, ... of the item, turns codes into
+//           16x8x16 tensor-core operands in registers, keeps an online softmax per
+//           query head, and the 7 warps merge into one partial (m, l, o) per item.
+//   merge   one warp per (sequence, query head): log-sum-exp merge of the item
+//           partials, inverse Hadamard rotation, store.
+#include "kv4_common.cuh"
+
+#include <math.h>
+
+namespace kv4 {
+
+namespace {
+
+constexpr int NW = 7;                  // consumer warps (+1 producer: 16 warps per SM at 2 CTAs)
+constexpr int THREADS = 32 * (NW + 1); // + producer warp
+constexpr int QD = 2;                  // item queue depth
+constexpr int PREP_WARPS = 4;
+constexpr float NEG_INF = -INFINITY;
+
+template <int D, bool BF16>
+struct KCfg {
+  static constexpr int STAGE = BF16 ? tile16_bytes(D) : tile8_bytes(D);
+  static constexpr int NS = BF16 ? 10 : 16;
+  static constexpr int QBLOB = qblob_bytes(D);
+};
+
+// Partial of one item: per query head, o[D] (unnormalised, rotated basis), m, l,
+// padded to D + 4 floats so every head row starts on a 16-byte boundary.
+__host__ __device__ constexpr int head_stride(int D) { return D + 4; }
+__host__ __device__ inline int partial_stride(int G, int D) { return G * head_stride(D); }
+
+template <int D, bool BF16>
+__host__ __device__ inline size_t attn_smem_bytes(int G) {
+  using C = KCfg<D, BF16>;
+  return static_cast<size_t>(C::NS) * C::STAGE + static_cast<size_t>(QD) * C::QBLOB +
+         static_cast<size_t>(NW) * G * head_stride(D) * sizeof(float) + QD * sizeof(Item) +
+         (2 * C::NS + 2 * QD) * sizeof(uint64_t) + 16;
+}
+
+// ---------------------------------------------------------------------------
+// prep: query rotation + work items
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(32 * PREP_WARPS) prep_kernel(AttnParams p) {
+  constexpr int VPL = D / 32;
+  extern __shared__ float s_q[];  // [PREP_WARPS][G][D]
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int gw = blockIdx.x * PREP_WARPS + wib;
+  if (gw >= p.n_seqs * p.Hkv) return;
+  const int b = gw / p.Hkv, h = gw % p.Hkv;
+  const int G = p.G;
+  const int seq = p.seq_ids[b];
+  int L = 0;
+  if (seq >= 0 && seq < p.max_seqs) {
+    L = p.seq_lens[seq];
+  } else if (lane == 0) {
+    atomicOr(&p.state->status, KV4_DEV_BAD_SEQ);
+  }
+
+  // ---- work items
+  int lo4, hi4, nprot;
+  if (BF16 || (p.mode & KV4_MODE_INT4_ONLY)) {
+    lo4 = 0; hi4 = L; nprot = 0;
+  } else {
+    nprot = min(L, p.S + p.W);
+    lo4 = p.S; hi4 = L - p.W;
+  }
+  int t0 = 0, t1 = 0;
+  if (hi4 > lo4) { t0 = lo4 / TILE; t1 = (hi4 + TILE - 1) / TILE; }
+  const int C = p.chunk_tiles;
+  const int tiles = t1 - t0;
+  const int nfull = tiles / C, rem = (tiles % C) ? 1 : 0, prot = nprot > 0 ? 1 : 0;
+  const int nparts = nfull + rem + prot;
+  int base0 = 0, base1 = 0, base2 = 0, pbase = 0;
+  if (lane == 0) {
+    if (nfull) base0 = atomicAdd(&p.state->n_items[0], nfull);
+    if (rem) base1 = atomicAdd(&p.state->n_items[1], 1);
+    if (prot) base2 = atomicAdd(&p.state->n_items[2], 1);
+    if (nparts) pbase = atomicAdd(&p.state->n_parts, nparts);
+    if (base0 + nfull > p.cap[0] || base1 + rem > p.cap[1] || base2 + prot > p.cap[2] ||
+        pbase + nparts > p.cap_parts)
+      atomicOr(&p.state->status, KV4_DEV_WORKSPACE);
+  }
+  base0 = __shfl_sync(0xffffffffu, base0, 0);
+  base1 = __shfl_sync(0xffffffffu, base1, 0);
+  base2 = __shfl_sync(0xffffffffu, base2, 0);
+  pbase = __shfl_sync(0xffffffffu, pbase, 0);
+  const int kind4 = BF16 ? 2 : 0;
+  for (int j = lane; j < nfull; j += 32) {
+    if (base0 + j >= p.cap[0]) break;
+    Item it{};
+    it.b = b; it.seq = seq; it.h = h; it.kind = kind4;
+    it.t_begin = t0 + j * C; it.t_end = t0 + (j + 1) * C;
+    it.lo = lo4; it.hi = hi4; it.part = pbase + j;
+    p.items[0][base0 + j] = it;
+  }
+  if (lane == 0) {
+    if (rem && base1 < p.cap[1]) {
+      Item it{};
+      it.b = b; it.seq = seq; it.h = h; it.kind = kind4;
+      it.t_begin = t0 + nfull * C; it.t_end = t1;
+      it.lo = lo4; it.hi = hi4; it.part = pbase + nfull;
+      p.items[1][base1] = it;
+    }
+    if (prot && base2 < p.cap[2]) {
+      Item it{};
+      it.b = b; it.seq = seq; it.h = h; it.kind = 1;
+      it.t_begin = 0; it.t_end = (nprot + TILE - 1) / TILE;
+      it.lo = 0; it.hi = nprot; it.part = pbase + nfull + rem;
+      p.items[2][base2] = it;
+    }
+    SeqHead sh;
+    sh.part_base = pbase; sh.n_parts = nparts; sh.len = L; sh.pad = 0;
+    p.seqhead[gw] = sh;
+  }
+
+  // ---- queries: rotate (INT4 cache), round to bf16, lay out as B operands
+  float* sq = s_q + wib * G * D;
+  float qsum[MAX_G];
+  float amax = 0.f;
+  const float rot_c = p.rot_c;
+  for (int g = 0; g < G; ++g) {
+    const uint16_t* src = p.q + (static_cast<long long>(b) * p.Hq + h * G + g) * D;
+    float x[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) x[i] = __bfloat162float(__ushort_as_bfloat16(src[VPL * lane + i]));
+    if constexpr (!BF16) {
+      for (int hh = 1; hh < p.Bh; hh <<= 1) {
+        if (hh < VPL) {
+#pragma unroll
+          for (int i = 0; i < VPL; ++i)
+            if ((i & hh) == 0) {
+              const float a = x[i], c = x[i + hh];
+              x[i] = __fadd_rn(a, c);
+              x[i + hh] = __fsub_rn(a, c);
+            }
+        } else {
+          const int lm = hh / VPL;
+          const bool upper = (lane & lm) != 0;
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) {
+            const float o = __shfl_xor_sync(0xffffffffu, x[i], lm);
+            x[i] = upper ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) x[i] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(x[i], rot_c)));
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      sq[g * D + VPL * lane + i] = x[i];
+      s += x[i];
+      amax = fmaxf(amax, fabsf(x[i]));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    qsum[g] = s;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  __syncwarp();
+  // fp16 operands: q * 2^e with max|q| * 2^e in [2^14, 2^15) (exact for normal values)
+  int e = 0;
+  if (!BF16 && amax > 0.f && amax <= 3.0e38f) {
+    int ex;
+    frexpf(amax, &ex);
+    e = 15 - ex;
+  }
+  uint32_t* blob = reinterpret_cast<uint32_t*>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D));
+  const int g = lane >> 2, t = lane & 3;
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t r[4];
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      const int k = 2 * c + kk;
+#pragma unroll
+      for (int reg = 0; reg < 2; ++reg) {
+        const int d = 16 * k + 2 * t + 8 * reg;
+        float a = 0.f, bb = 0.f;
+        if (g < G) { a = sq[g * D + d]; bb = sq[g * D + d + 1]; }
+        if constexpr (BF16) {
+          r[2 * kk + reg] = pack_bf162(a, bb);
+        } else {
+          r[2 * kk + reg] = pack_half2(ldexpf(a, e), ldexpf(bb, e));
+        }
+      }
+    }
+    reinterpret_cast<uint4*>(blob)[c * 32 + lane] = make_uint4(r[0], r[1], r[2], r[3]);
+  }
+  float* tail = reinterpret_cast<float*>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D) + 16 * D);
+  if (lane < MAX_G) {
+    float v = 0.f;
+#pragma unroll
+    for (int gg = 0; gg < MAX_G; ++gg)
+      if (gg == lane && gg < G) v = qsum[gg];
+    tail[lane] = BF16 ? 0.f : v * p.scale_log2;
+  }
+  if (lane == MAX_G) tail[MAX_G] = ldexpf(p.scale_log2, -e);
+}
+
+// ---------------------------------------------------------------------------
+// attention: per-warp online-softmax state
+
+template <int D>
+struct WarpState {
+  float o[D / 16][4];  // o^T fragments: (dim 16m+g, head 2t), (16m+g, 2t+1), (16m+g+8, 2t), (16m+g+8, 2t+1)
+  float m0, m1, l0, l1, z0, z1;
+};
+
+template <int D>
+struct QFrag {
+  uint32_t b[D / 16][2];
+  float qs0, qs1, kscale;
+};
+
+template <int D>
+__device__ __forceinline__ void online_softmax_pv(WarpState<D>& ws, float x0, float x1, float x2, float x3,
+                                                  float& p0, float& p1, float& p2, float& p3) {
+  float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+  }
+  const float n0 = fmaxf(ws.m0, mx0), n1 = fmaxf(ws.m1, mx1);
+  if (__any_sync(0xffffffffu, n0 > ws.m0 || n1 > ws.m1)) {
+    const float a0 = ex2(ws.m0 - n0), a1 = ex2(ws.m1 - n1);
+    ws.l0 *= a0; ws.l1 *= a1; ws.z0 *= a0; ws.z1 *= a1;
+#pragma unroll
+    for (int m = 0; m < D / 16; ++m) {
+      ws.o[m][0] *= a0; ws.o[m][1] *= a1; ws.o[m][2] *= a0; ws.o[m][3] *= a1;
+    }
+    ws.m0 = n0; ws.m1 = n1;
+  }
+  p0 = ex2(x0 - ws.m0); p1 = ex2(x1 - ws.m1); p2 = ex2(x2 - ws.m0); p3 = ex2(x3 - ws.m1);
+}
+
+// One INT4 tile at shared address st.
+template <int D, bool MASKED>
+__device__ __forceinline__ void tile_int4(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, bool vg,
+                                          bool vg8, uint32_t empty_bar) {
+  constexpr int NKK = D / 32;
+  uint32_t kw0[NKK], kw1[NKK], vw[D / 16];
+  if constexpr (D == 128) {
+    const uint4 a = lds128(st + lane * 16), bq = lds128(st + 512 + lane * 16);
+    kw0[0] = a.x; kw0[1] = a.y; kw0[2] = a.z; kw0[3] = a.w;
+    kw1[0] = bq.x; kw1[1] = bq.y; kw1[2] = bq.z; kw1[3] = bq.w;
+    const uint4 v0 = lds128(st + 8 * D + lane * 16), v1 = lds128(st + 8 * D + 512 + lane * 16);
+    vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+    vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
+  } else {
+    const uint2 a = lds64(st + lane * 8), bq = lds64(st + 256 + lane * 8);
+    kw0[0] = a.x; kw0[1] = a.y; kw1[0] = bq.x; kw1[1] = bq.y;
+    const uint4 v0 = lds128(st + 8 * D + lane * 16);
+    vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+  }
+  const uint4 sz = lds128(st + 16 * D + (lane >> 2) * 16);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty_bar);  // the tile is in registers: hand the stage back
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int kk = 0; kk < NKK; ++kk) {
+    const uint32_t w0 = kw0[kk], w1 = kw1[kk];
+    mma_f16(acc, nib_lo(w0), nib_lo(w1), nib_hi(w0), nib_hi(w1), qf.b[2 * kk][0], qf.b[2 * kk][1]);
+    const uint32_t u0 = w0 >> 8, u1 = w1 >> 8;
+    mma_f16(acc, nib_lo(u0), nib_lo(u1), nib_hi(u0), nib_hi(u1), qf.b[2 * kk + 1][0], qf.b[2 * kk + 1][1]);
+  }
+  const float sKg = half_lo(sz.x) * qf.kscale, zKg = half_hi(sz.x);
+  const float sKg8 = half_lo(sz.y) * qf.kscale, zKg8 = half_hi(sz.y);
+  float x0 = fmaf(acc[0], sKg, zKg * qf.qs0);
+  float x1 = fmaf(acc[1], sKg, zKg * qf.qs1);
+  float x2 = fmaf(acc[2], sKg8, zKg8 * qf.qs0);
+  float x3 = fmaf(acc[3], sKg8, zKg8 * qf.qs1);
+  if constexpr (MASKED) {
+    if (!vg) { x0 = NEG_INF; x1 = NEG_INF; }
+    if (!vg8) { x2 = NEG_INF; x3 = NEG_INF; }
+  }
+  float p0, p1, p2, p3;
+  online_softmax_pv<D>(ws, x0, x1, x2, x3, p0, p1, p2, p3);
+  const float sVg = half_lo(sz.z), zVg = half_hi(sz.z), sVg8 = half_lo(sz.w), zVg8 = half_hi(sz.w);
+  float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
+  float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
+  if constexpr (MASKED) {
+    if (!vg) { P0 = 0.f; P1 = 0.f; zg0 = 0.f; zg1 = 0.f; }
+    if (!vg8) { P2 = 0.f; P3 = 0.f; zg80 = 0.f; zg81 = 0.f; }
+  }
+  ws.l0 += p0 + p2; ws.l1 += p1 + p3;
+  ws.z0 += zg0 + zg80; ws.z1 += zg1 + zg81;
+  const uint32_t B0 = movmatrix_trans(pack_half2(P0, P1));
+  const uint32_t B1 = movmatrix_trans(pack_half2(P2, P3));
+#pragma unroll
+  for (int m = 0; m < D / 16; ++m) {
+    const uint32_t w = vw[m], u = w >> 8;
+    mma_f16(ws.o[m], nib_lo(w), nib_hi(w), nib_lo(u), nib_hi(u), B0, B1);
+  }
+}
+
+// One INT8 tile (protected store).
+template <int D, bool MASKED>
+__device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, bool vg,
+                                          bool vg8, uint32_t empty_bar) {
+  constexpr int NK = D / 16;
+  uint32_t kw[2][NK], vw[2 * NK];
+#pragma unroll
+  for (int rowhi = 0; rowhi < 2; ++rowhi)
+#pragma unroll
+    for (int kq = 0; kq < D / 64; ++kq) {
+      const uint4 a = lds128(st + 16 * (32 * (rowhi * (D / 64) + kq) + lane));
+      kw[rowhi][4 * kq] = a.x; kw[rowhi][4 * kq + 1] = a.y; kw[rowhi][4 * kq + 2] = a.z; kw[rowhi][4 * kq + 3] = a.w;
+    }
+#pragma unroll
+  for (int q4 = 0; q4 < NK / 2; ++q4) {
+    const uint4 a = lds128(st + 16 * D + 16 * (32 * q4 + lane));
+    vw[4 * q4] = a.x; vw[4 * q4 + 1] = a.y; vw[4 * q4 + 2] = a.z; vw[4 * q4 + 3] = a.w;
+  }
+  const uint4 sz = lds128(st + 32 * D + (lane >> 2) * 16);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty_bar);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int k = 0; k < NK; ++k) {
+    const uint32_t w0 = kw[0][k], w1 = kw[1][k];
+    mma_f16(acc, byte_lo(w0), byte_lo(w1), byte_lo(w0 >> 8), byte_lo(w1 >> 8), qf.b[k][0], qf.b[k][1]);
+  }
+  const float sKg = half_lo(sz.x) * qf.kscale, zKg = half_hi(sz.x);
+  const float sKg8 = half_lo(sz.y) * qf.kscale, zKg8 = half_hi(sz.y);
+  float x0 = fmaf(acc[0], sKg, zKg * qf.qs0);
+  float x1 = fmaf(acc[1], sKg, zKg * qf.qs1);
+  float x2 = fmaf(acc[2], sKg8, zKg8 * qf.qs0);
+  float x3 = fmaf(acc[3], sKg8, zKg8 * qf.qs1);
+  if constexpr (MASKED) {
+    if (!vg) { x0 = NEG_INF; x1 = NEG_INF; }
+    if (!vg8) { x2 = NEG_INF; x3 = NEG_INF; }
+  }
+  float p0, p1, p2, p3;
+  online_softmax_pv<D>(ws, x0, x1, x2, x3, p0, p1, p2, p3);
+  const float sVg = half_lo(sz.z), zVg = half_hi(sz.z), sVg8 = half_lo(sz.w), zVg8 = half_hi(sz.w);
+  float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
+  float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
+  if constexpr (MASKED) {
+    if (!vg) { P0 = 0.f; P1 = 0.f; zg0 = 0.f; zg1 = 0.f; }
+    if (!vg8) { P2 = 0.f; P3 = 0.f; zg80 = 0.f; zg81 = 0.f; }
+  }
+  ws.l0 += p0 + p2; ws.l1 += p1 + p3;
+  ws.z0 += zg0 + zg80; ws.z1 += zg1 + zg81;
+  const uint32_t B0 = movmatrix_trans(pack_half2(P0, P1));
+  const uint32_t B1 = movmatrix_trans(pack_half2(P2, P3));
+#pragma unroll
+  for (int m = 0; m < NK; ++m) {
+    const uint32_t w0 = vw[2 * m], w1 = vw[2 * m + 1];
+    mma_f16(ws.o[m], byte_lo(w0), byte_lo(w0 >> 8), byte_lo(w1), byte_lo(w1 >> 8), B0, B1);
+  }
+}
+
+// One BF16 tile (baseline cache).  Holds the stage until the V loads are done.
+template <int D, bool MASKED>
+__device__ __forceinline__ void tile_bf16(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, bool vg,
+                                          bool vg8, uint32_t empty_bar) {
+  constexpr int NK = D / 16;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int k = 0; k < NK; ++k) {
+    const uint4 a = lds128(st + 16 * (32 * k + lane));
+    mma_bf16(acc, a.x, a.y, a.z, a.w, qf.b[k][0], qf.b[k][1]);
+  }
+  uint4 v[NK];
+#pragma unroll
+  for (int m = 0; m < NK; ++m) v[m] = lds128(st + 32 * D + 16 * (32 * m + lane));
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty_bar);
+  float x0 = acc[0] * qf.kscale, x1 = acc[1] * qf.kscale, x2 = acc[2] * qf.kscale, x3 = acc[3] * qf.kscale;
+  if constexpr (MASKED) {
+    if (!vg) { x0 = NEG_INF; x1 = NEG_INF; }
+    if (!vg8) { x2 = NEG_INF; x3 = NEG_INF; }
+  }
+  float p0, p1, p2, p3;
+  online_softmax_pv<D>(ws, x0, x1, x2, x3, p0, p1, p2, p3);
+  ws.l0 += p0 + p2; ws.l1 += p1 + p3;
+  const uint32_t B0 = movmatrix_trans(pack_bf162(p0, p1));
+  const uint32_t B1 = movmatrix_trans(pack_bf162(p2, p3));
+#pragma unroll
+  for (int m = 0; m < NK; ++m) mma_bf16(ws.o[m], v[m].x, v[m].y, v[m].z, v[m].w, B0, B1);
+}
+
+template <int D, bool BF16>
+__device__ __forceinline__ const uint8_t* tile_source(const AttnParams& p, const Item& it, int tile) {
+  if (it.kind == 1)
+    return p.prot + ((static_cast<long long>(it.seq) * p.Hkv + it.h) * n_prot_tiles(p.S, p.W) + tile) *
+                        tile8_bytes(D);
+  const int pos = tile * TILE;
+  int page = p.block_table[static_cast<long long>(it.seq) * p.max_pages_per_seq + pos / p.P];
+  if (page < 0 || page >= p.num_pages) {
+    atomicOr(&p.state->status, KV4_DEV_BAD_PAGE);
+    page = 0;
+  }
+  constexpr int TB = BF16 ? tile16_bytes(D) : tile4_bytes(D);
+  return p.pool + ((static_cast<long long>(page) * p.Hkv + it.h) * (p.P / TILE) + (pos % p.P) / TILE) * TB;
+}
+
+__device__ __forceinline__ void named_barrier_consumers() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * NW) : "memory");
+}
+
+
+// Bounded wait used only to drain this CTA's own bulk copies before exit.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > 1000000000ull) return;
+  }
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(THREADS, 2) attn_kernel(AttnParams p) {
+  using C = KCfg<D, BF16>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* ring = smem;
+  uint8_t* qbuf = ring + C::NS * C::STAGE;
+  float* merge = reinterpret_cast<float*>(qbuf + QD * C::QBLOB);
+  Item* itemq = reinterpret_cast<Item*>(merge + NW * p.G * head_stride(D));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(itemq + QD);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * C::NS + 2 * QD);
+  volatile int* go_flag = abort_flag + 1;
+  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * C::NS;
+  const uint32_t iqf0 = full0 + 16 * C::NS, iqe0 = iqf0 + 8 * QD;
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
+    for (int s = 0; s < QD; ++s) { mbar_init(iqf0 + 8 * s, 1); mbar_init(iqe0 + 8 * s, NW); }
+    *abort_flag = 0;
+    *go_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int n0 = min(p.state->n_items[0], p.cap[0]);
+  const int n1 = min(p.state->n_items[1], p.cap[1]);
+  const int n2 = min(p.state->n_items[2], p.cap[2]);
+  const int total = n0 + n1 + n2;
+  int* status = &p.state->status;
+
+  if (warp == NW) {
+    // ------------------------------------------------------------ producer
+    // Claims run one item ahead: while the tiles of `cur` stream, the item
+    // after it is loaded and the one after that is claimed.
+    auto load_item = [&](int k) -> Item {
+      if (k < n0) return p.items[0][k];
+      if (k < n0 + n1) return p.items[1][k - n0];
+      return p.items[2][k - n0 - n1];
+    };
+    int k_cur = 0, k_nxt = 0;
+    if (lane == 0) { k_cur = atomicAdd(&p.state->work, 1); k_nxt = atomicAdd(&p.state->work, 1); }
+    k_cur = __shfl_sync(0xffffffffu, k_cur, 0);
+    k_nxt = __shfl_sync(0xffffffffu, k_nxt, 0);
+    Item cur{};
+    if (k_cur < total) cur = load_item(k_cur);
+    uint32_t it = 0;
+    int q = 0;
+    bool ok = true;
+    for (;; ++q) {
+      const int slot = q % QD;
+      if (lane == 0) ok = mbar_wait(iqe0 + 8 * slot, ((q / QD) & 1) ^ 1, abort_flag, status);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      if (k_cur >= total) {
+        if (lane == 0) { itemq[slot].kind = -1; mbar_arrive(iqf0 + 8 * slot); }
+        break;
+      }
+      Item nxt{};
+      if (k_nxt < total) nxt = load_item(k_nxt);
+      int k_new = total;
+      if (lane == 0 && k_nxt < total) k_new = atomicAdd(&p.state->work, 1);
+      if (lane == 0) {
+        itemq[slot] = cur;
+        mbar_arrive_expect_tx(iqf0 + 8 * slot, C::QBLOB);
+        bulk_g2s(smem_u32(qbuf + slot * C::QBLOB),
+                 p.qblob + static_cast<size_t>(cur.b * p.Hkv + cur.h) * C::QBLOB, C::QBLOB, iqf0 + 8 * slot);
+      }
+      const int ntiles = cur.t_end - cur.t_begin;
+      const uint32_t tbytes = cur.kind == 1 ? tile8_bytes(D) : (BF16 ? tile16_bytes(D) : tile4_bytes(D));
+      for (int base = 0; base < ntiles && ok; base += 32) {
+        const uint8_t* src = nullptr;
+        if (base + lane < ntiles) src = tile_source<D, BF16>(p, cur, cur.t_begin + base + lane);
+        const int n = min(32, ntiles - base);
+        for (int j = 0; j < n; ++j) {
+          const unsigned long long a = __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(src), j);
+          if (lane == 0) {
+            const int s = it % C::NS;
+            ok = mbar_wait(empty0 + 8 * s, ((it / C::NS) & 1) ^ 1, abort_flag, status);
+            if (ok) {
+              mbar_arrive_expect_tx(full0 + 8 * s, tbytes);
+              bulk_g2s(smem_u32(ring + s * C::STAGE), reinterpret_cast<const void*>(a), tbytes, full0 + 8 * s);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          ++it;
+        }
+      }
+      if (!ok) break;
+      cur = nxt;
+      k_cur = k_nxt;
+      k_nxt = __shfl_sync(0xffffffffu, k_new, 0);
+    }
+    if (!ok && lane == 0) {
+      // aborted: let this CTA's copies land before the shared memory is released
+      const uint32_t first = it > static_cast<uint32_t>(C::NS) ? it - C::NS : 0u;
+      for (uint32_t j = first; j < it; ++j) mbar_drain(full0 + 8 * (j % C::NS), (j / C::NS) & 1);
+      for (int j = q > QD ? q - QD : 0; j < q; ++j) mbar_drain(iqf0 + 8 * (j % QD), (j / QD) & 1);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int g = lane >> 2, t = lane & 3;
+  const int G = p.G;
+  const int pstride = partial_stride(G, D);
+  uint32_t it = 0;
+  for (int q = 0;; ++q) {
+    const int slot = q % QD;
+    const uint32_t iq_parity = (q / QD) & 1;
+    if (warp == 0 && lane == 0) {
+      const bool ok = mbar_wait(iqf0 + 8 * slot, iq_parity, abort_flag, status);
+      *go_flag = ok && itemq[slot].kind >= 0;
+    }
+    named_barrier_consumers();  // uniform exit decision; also orders the previous combine before new merge writes
+    if (!*go_flag) break;
+    mbar_wait(iqf0 + 8 * slot, iq_parity, abort_flag, status);  // completed: acquire for this thread
+    const Item cur = itemq[slot];
+    QFrag<D> qf;
+    {
+      const uint32_t qb = smem_u32(qbuf + slot * C::QBLOB);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        const uint4 v = lds128(qb + 16 * (32 * c + lane));
+        qf.b[2 * c][0] = v.x; qf.b[2 * c][1] = v.y; qf.b[2 * c + 1][0] = v.z; qf.b[2 * c + 1][1] = v.w;
+      }
+      const float* tail = reinterpret_cast<const float*>(qbuf + slot * C::QBLOB + 16 * D);
+      qf.qs0 = tail[(2 * t) & 7];
+      qf.qs1 = tail[(2 * t + 1) & 7];
+      qf.kscale = tail[MAX_G];
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(iqe0 + 8 * slot);
+
+    WarpState<D> ws;
+#pragma unroll
+    for (int m = 0; m < D / 16; ++m) ws.o[m][0] = ws.o[m][1] = ws.o[m][2] = ws.o[m][3] = 0.f;
+    ws.m0 = ws.m1 = NEG_INF;
+    ws.l0 = ws.l1 = ws.z0 = ws.z1 = 0.f;
+
+    const int ntiles = cur.t_end - cur.t_begin;
+    for (int i = warp; i < ntiles; i += NW) {
+      const uint32_t j = it + i;
+      const int s = j % C::NS;
+      if (!mbar_wait(full0 + 8 * s, (j / C::NS) & 1, abort_flag, status)) break;
+      const uint32_t st = smem_u32(ring + s * C::STAGE);
+      const int pos0 = (cur.t_begin + i) * TILE;
+      const bool inside = pos0 >= cur.lo && pos0 + TILE <= cur.hi;
+      const bool vg = pos0 + g >= cur.lo && pos0 + g < cur.hi;
+      const bool vg8 = pos0 + g + 8 >= cur.lo && pos0 + g + 8 < cur.hi;
+      const uint32_t eb = empty0 + 8 * s;
+      if constexpr (BF16) {
+        if (inside) tile_bf16<D, false>(st, qf, ws, lane, vg, vg8, eb);
+        else tile_bf16<D, true>(st, qf, ws, lane, vg, vg8, eb);
+      } else if (cur.kind == 1) {
+        if (inside) tile_int8<D, false>(st, qf, ws, lane, vg, vg8, eb);
+        else tile_int8<D, true>(st, qf, ws, lane, vg, vg8, eb);
+      } else {
+        if (inside) tile_int4<D, false>(st, qf, ws, lane, vg, vg8, eb);
+        else tile_int4<D, true>(st, qf, ws, lane, vg, vg8, eb);
+      }
+    }
+    it += ntiles;
+
+    // ---- merge the NW warps into one partial
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      ws.l0 += __shfl_xor_sync(0xffffffffu, ws.l0, o);
+      ws.l1 += __shfl_xor_sync(0xffffffffu, ws.l1, o);
+      ws.z0 += __shfl_xor_sync(0xffffffffu, ws.z0, o);
+      ws.z1 += __shfl_xor_sync(0xffffffffu, ws.z1, o);
+    }
+    constexpr int HS = head_stride(D);
+    float* mw = merge + warp * G * HS;
+    const int h0 = 2 * t, h1 = 2 * t + 1;
+    if (h0 < G) {
+      float* r = mw + h0 * HS;
+#pragma unroll
+      for (int m = 0; m < D / 16; ++m) { r[16 * m + g] = ws.o[m][0] + ws.z0; r[16 * m + g + 8] = ws.o[m][2] + ws.z0; }
+      if (g == 0) { r[D] = ws.m0; r[D + 1] = ws.l0; }
+    }
+    if (h1 < G) {
+      float* r = mw + h1 * HS;
+#pragma unroll
+      for (int m = 0; m < D / 16; ++m) { r[16 * m + g] = ws.o[m][1] + ws.z1; r[16 * m + g + 8] = ws.o[m][3] + ws.z1; }
+      if (g == 0) { r[D] = ws.m1; r[D + 1] = ws.l1; }
+    }
+    named_barrier_consumers();
+    if (cur.part >= 0 && cur.part < p.cap_parts) {
+      float* part = p.partials + static_cast<size_t>(cur.part) * pstride;
+      for (int idx = warp * 32 + lane; idx < G * D; idx += NW * 32) {
+        const int hq = idx / D, d = idx % D;
+        float M = NEG_INF;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, merge[(w * G + hq) * HS + D]);
+        float acc = 0.f, lsum = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          const float* r = merge + (w * G + hq) * HS;
+          const float mwv = r[D];
+          if (mwv > NEG_INF) {
+            const float f = ex2(mwv - M);
+            acc = fmaf(f, r[d], acc);
+            lsum = fmaf(f, r[D + 1], lsum);
+          }
+        }
+        part[hq * HS + d] = acc;
+        if (d == 0) { part[hq * HS + D] = M; part[hq * HS + D + 1] = lsum; }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// merge: log-sum-exp over the item partials, inverse rotation, store
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) merge_kernel(AttnParams p) {
+  constexpr int VPL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    // the attention kernel has finished: re-arm the per-call counters
+    p.state->n_items[0] = 0; p.state->n_items[1] = 0; p.state->n_items[2] = 0;
+    p.state->n_parts = 0; p.state->work = 0;
+  }
+  if (gw >= p.n_seqs * p.Hq) return;
+  const int b = gw / p.Hq, hq = gw % p.Hq, h = hq / p.G, gq = hq % p.G;
+  const SeqHead sh = p.seqhead[b * p.Hkv + h];
+  const int pstride = partial_stride(p.G, D);
+  float o[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) o[i] = 0.f;
+  if (sh.n_parts > 0 && sh.part_base >= 0 && sh.part_base + sh.n_parts <= p.cap_parts) {
+    const float* base = p.partials + static_cast<size_t>(sh.part_base) * pstride + gq * head_stride(D);
+    float M = NEG_INF;
+    for (int j = 0; j < sh.n_parts; ++j) M = fmaxf(M, base[static_cast<size_t>(j) * pstride + D]);
+    float lsum = 0.f;
+    for (int j = 0; j < sh.n_parts; ++j) {
+      const float* r = base + static_cast<size_t>(j) * pstride;
+      const float f = ex2(r[D] - M);
+      lsum = fmaf(f, r[D + 1], lsum);
+      if constexpr (VPL == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(r + 4 * lane);
+        o[0] = fmaf(f, v.x, o[0]); o[1] = fmaf(f, v.y, o[1]); o[2] = fmaf(f, v.z, o[2]); o[3] = fmaf(f, v.w, o[3]);
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(r + 2 * lane);
+        o[0] = fmaf(f, v.x, o[0]); o[1] = fmaf(f, v.y, o[1]);
+      }
+    }
+    const float inv = 1.f / lsum;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) o[i] *= inv;
+    if constexpr (!BF16) {
+      // o = H_blk o_rot (the normalised Hadamard matrix is its own inverse)
+      for (int hh = 1; hh < p.Bh; hh <<= 1) {
+        if (hh < VPL) {
+#pragma unroll
+          for (int i = 0; i < VPL; ++i)
+            if ((i & hh) == 0) {
+              const float a = o[i], c = o[i + hh];
+              o[i] = a + c;
+              o[i + hh] = a - c;
+            }
+        } else {
+          const int lm = hh / VPL;
+          const bool upper = (lane & lm) != 0;
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) {
+            const float other = __shfl_xor_sync(0xffffffffu, o[i], lm);
+            o[i] = upper ? other - o[i] : o[i] + other;
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) o[i] *= p.rot_c;
+    }
+  }
+  const size_t off = (static_cast<size_t>(b) * p.Hq + hq) * D + VPL * lane;
+  if (p.mode & KV4_MODE_OUT_F32) {
+    float* out = static_cast<float*>(p.out) + off;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) out[i] = o[i];
+  } else {
+    uint16_t* out = static_cast<uint16_t*>(p.out) + off;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(o[i]));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+
+struct WsLayout {
+  size_t seqhead, qblob, items0, items1, items2, partials, total;
+  int cap0, cap_side, cap_parts;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+inline int chunk_tiles_for(const kv4_cache* c, int n_seqs) {
+  const kv4_config& cfg = c->cfg;
+  const long long cap_tiles = static_cast<long long>(cfg.max_pages_per_seq) * cfg.page_size / TILE + 1;
+  const long long work = static_cast<long long>(n_seqs) * cfg.num_kv_heads * cap_tiles;
+  const long long target = 4LL * c->num_sms * (c->attn_blocks_per_sm > 0 ? c->attn_blocks_per_sm : 2);
+  long long ct = (work + target - 1) / target;
+  if (ct < 8) ct = 8;
+  if (ct > 64) ct = 64;
+  return static_cast<int>(ct);
+}
+
+inline WsLayout ws_layout(const kv4_cache* c, int n_seqs, int cap0) {
+  const kv4_config& cfg = c->cfg;
+  const int G = cfg.num_q_heads / cfg.num_kv_heads, D = cfg.head_dim;
+  const size_t nsh = static_cast<size_t>(n_seqs) * cfg.num_kv_heads;
+  WsLayout w{};
+  w.cap0 = cap0;
+  w.cap_side = static_cast<int>(nsh);
+  w.cap_parts = cap0 + 2 * static_cast<int>(nsh);
+  size_t off = 0;
+  w.seqhead = off; off = align256(off + nsh * sizeof(SeqHead));
+  w.qblob = off; off = align256(off + nsh * qblob_bytes(D));
+  w.items0 = off; off = align256(off + static_cast<size_t>(cap0) * sizeof(Item));
+  w.items1 = off; off = align256(off + nsh * sizeof(Item));
+  w.items2 = off; off = align256(off + nsh * sizeof(Item));
+  w.partials = off; off = align256(off + static_cast<size_t>(w.cap_parts) * partial_stride(G, D) * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+template <int D, bool BF16>
+int occupancy(int G) {
+  // the attribute is per kernel and process-wide: allow the largest group size once
+  const size_t smem = attn_smem_bytes<D, BF16>(G);
+  if (cudaFuncSetAttribute(attn_kernel<D, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(attn_smem_bytes<D, BF16>(MAX_G))) != cudaSuccess)
+    return -1;
+  int blocks = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, attn_kernel<D, BF16>, THREADS, smem) != cudaSuccess)
+    return -1;
+  return blocks;
+}
+
+template <int D, bool BF16>
+int launch_attention_t(kv4_cache* c, AttnParams& p, cudaStream_t stream) {
+  const int blocks_per_sm = c->attn_blocks_per_sm;
+  if (blocks_per_sm <= 0) return KV4_ERR_UNSUPPORTED;
+  const int nsh = p.n_seqs * p.Hkv;
+  const size_t prep_smem = static_cast<size_t>(PREP_WARPS) * p.G * D * sizeof(float);
+  prep_kernel<D, BF16><<<(nsh + PREP_WARPS - 1) / PREP_WARPS, 32 * PREP_WARPS, prep_smem, stream>>>(p);
+  // no more CTAs than items can exist
+  long long max_items = static_cast<long long>(p.cap[0]) + p.cap[1] + p.cap[2];
+  long long grid = static_cast<long long>(c->num_sms) * blocks_per_sm;
+  if (grid > max_items) grid = max_items;
+  if (grid < 1) grid = 1;
+  if (c->ev_before) cudaEventRecord(c->ev_before, stream);
+  attn_kernel<D, BF16><<<static_cast<unsigned>(grid), THREADS, attn_smem_bytes<D, BF16>(p.G), stream>>>(p);
+  if (c->ev_after) cudaEventRecord(c->ev_after, stream);
+  const int merge_warps = p.n_seqs * p.Hq;
+  merge_kernel<D, BF16><<<(merge_warps + 7) / 8, 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+}
+
+}  // namespace
+
+int attention_blocks_per_sm(kv4_cache* c) {
+  const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
+  if (c->cfg.head_dim == 128) return c->bf16 ? occupancy<128, true>(G) : occupancy<128, false>(G);
+  return c->bf16 ? occupancy<64, true>(G) : occupancy<64, false>(G);
+}
+
+size_t attention_workspace_bytes(const kv4_cache* c, int n_seqs, int max_ctx) {
+  const kv4_config& cfg = c->cfg;
+  const long long cap_ctx = static_cast<long long>(cfg.max_pages_per_seq) * cfg.page_size;
+  const long long ctx = (max_ctx <= 0 || max_ctx > cap_ctx) ? cap_ctx : max_ctx;
+  const long long tiles = (ctx + TILE - 1) / TILE + 1;
+  const int ct = chunk_tiles_for(c, n_seqs);
+  const long long cap0 = static_cast<long long>(n_seqs) * cfg.num_kv_heads * ((tiles + ct - 1) / ct);
+  return ws_layout(c, n_seqs, static_cast<int>(cap0)).total;
+}
+
+int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, const void* q, void* out,
+                     float softmax_scale, int mode, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const kv4_config& cfg = c->cfg;
+  const int D = cfg.head_dim;
+  const int G = cfg.num_q_heads / cfg.num_kv_heads;
+  // largest first-list capacity that fits the caller's workspace
+  const WsLayout w0 = ws_layout(c, n_seqs, 0);
+  const size_t per_item = sizeof(Item) + static_cast<size_t>(partial_stride(G, D)) * sizeof(float);
+  if (ws_bytes < w0.total) return KV4_ERR_WORKSPACE;
+  long long cap0 = static_cast<long long>((ws_bytes - w0.total) / per_item);
+  if (cap0 > (1LL << 30)) cap0 = 1LL << 30;
+  WsLayout w = ws_layout(c, n_seqs, static_cast<int>(cap0));
+  while (w.total > ws_bytes && cap0 > 0) { --cap0; w = ws_layout(c, n_seqs, static_cast<int>(cap0)); }
+  if (w.total > ws_bytes) return KV4_ERR_WORKSPACE;
+
+  AttnParams p{};
+  const uint8_t* lbase = c->base + c->pool_offset + static_cast<size_t>(layer) * c->layer_stride;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  p.pool = lbase;
+  p.prot = c->bf16 ? nullptr : lbase + c->pool_bytes;
+  p.block_table = c->block_table;
+  p.seq_lens = c->seq_lens + static_cast<size_t>(layer) * cfg.max_seqs;
+  p.seq_ids = seq_ids;
+  p.q = static_cast<const uint16_t*>(q);
+  p.out = out;
+  p.state = c->state;
+  p.items[0] = reinterpret_cast<Item*>(wsb + w.items0);
+  p.items[1] = reinterpret_cast<Item*>(wsb + w.items1);
+  p.items[2] = reinterpret_cast<Item*>(wsb + w.items2);
+  p.cap[0] = w.cap0;
+  p.cap[1] = w.cap_side;
+  p.cap[2] = w.cap_side;
+  p.seqhead = reinterpret_cast<SeqHead*>(wsb + w.seqhead);
+  p.qblob = wsb + w.qblob;
+  p.partials = reinterpret_cast<float*>(wsb + w.partials);
+  p.cap_parts = w.cap_parts;
+  p.n_seqs = n_seqs;
+  p.Hq = cfg.num_q_heads;
+  p.Hkv = cfg.num_kv_heads;
+  p.G = G;
+  p.D = D;
+  p.P = cfg.page_size;
+  p.S = cfg.sink_tokens;
+  p.W = cfg.recent_window;
+  p.Bh = c->bf16 ? 1 : cfg.hadamard_block;
+  p.rot_c = static_cast<float>(1.0 / sqrt(static_cast<double>(p.Bh)));
+  p.max_seqs = cfg.max_seqs;
+  p.num_pages = cfg.num_pages;
+  p.max_pages_per_seq = cfg.max_pages_per_seq;
+  p.chunk_tiles = chunk_tiles_for(c, n_seqs);
+  p.mode = mode;
+  const double scale = softmax_scale > 0.f ? static_cast<double>(softmax_scale) : 1.0 / sqrt(static_cast<double>(D));
+  p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+  if (D == 128) return c->bf16 ? launch_attention_t<128, true>(c, p, stream) : launch_attention_t<128, false>(c, p, stream);
+  return c->bf16 ? launch_attention_t<64, true>(c, p, stream) : launch_attention_t<64, false>(c, p, stream);
+}
+
+}  // namespace kv4

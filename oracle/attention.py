@@ -16,6 +16,8 @@ Readings of this library:
   same decode step appended); o_rot = sum_p a_p v^_p; o = H_blk o_rot (H is
   symmetric and orthonormal, so it is its own inverse); out = bf16(o).
 * GQA grouping is contiguous: query head j uses KV head j // (Hq / Hkv).
+* A sequence with no cached position gives an all-zero output row (the
+  library's convention; softmax over an empty set is undefined).
 * The bf16 output is rounded fp64 -> fp32 -> bf16 (two round-to-nearest-even
   steps); the tests allow one bf16 ulp between two bf16 outputs for this
   reason.
@@ -79,7 +81,7 @@ def decode_attention(cache, layer, seq_ids, q, scale=None, protected=True):
     for i, seq in enumerate(seq_ids):
         kh, vh = cache.view(layer, int(seq), protected=protected)
         if kh.shape[0] == 0:
-            raise ValueError("attention over an empty sequence")
+            continue                      # an empty sequence has an all-zero output row
         o_rot = attention_fp64(q_rot[i], kh, vh, scale)
         out[i] = o_rot @ H.T
     return {"out_f64": out, "out_bf16": _bf16_of_f64(out), "q_rot": q_rot}
@@ -95,5 +97,6 @@ def decode_attention_bf16(cache, layer, seq_ids, q, scale=None):
     out = np.zeros((n,) + q.shape[1:], np.float64)
     for i, seq in enumerate(seq_ids):
         k, v = cache.view(layer, int(seq))
-        out[i] = attention_fp64(q[i], k, v, scale)
+        if k.shape[0]:
+            out[i] = attention_fp64(q[i], k, v, scale)
     return {"out_f64": out, "out_bf16": _bf16_of_f64(out)}

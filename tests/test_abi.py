@@ -1,0 +1,66 @@
+"""CPU checks of the C ABI: the library loads, exports every function include/kv4.h declares,
+and rejects bad arguments before touching a device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kv4.h")
+LIB = os.path.join(ROOT, "int4_kv_cache_paged_b200", "libkv4.so")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|const char\*)\s+(kv4\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        pytest.fail("libkv4.so is missing; __graft_entry__.build() must run first")
+    return ctypes.CDLL(LIB)
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("kv4_cache_create", "kv4_rotate_quantize_append", "kv4_decode_attention", "kv4_dequantize_debug"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert missing == []
+
+
+def test_binding_names_match_header():
+    import int4_kv_cache_paged_b200 as kv4
+    for n in _declared():
+        assert n in kv4.EXPORTS and callable(getattr(kv4, n, None) or getattr(kv4._lib, n)), n
+
+
+def test_host_side_validation_without_a_device():
+    import int4_kv_cache_paged_b200 as kv4
+    good = dict(num_layers=1, max_seqs=2, num_q_heads=8, num_kv_heads=2, head_dim=128, page_size=16, num_pages=10,
+                max_pages_per_seq=5, hadamard_block=128, sink_tokens=4, recent_window=16)
+    n = kv4.kv4_cache_required_bytes(kv4.make_config(**good))
+    # state 256 + seq_lens (256) + pool 10*2*1*2176 + INT8 store 2*2*2*4224, each rounded to 256
+    pool = ((10 * 2 * 2176 + 255) // 256) * 256
+    prot = ((2 * 2 * 2 * 4224 + 255) // 256) * 256
+    assert n == 256 + 256 + pool + prot
+    for bad, code in ((dict(head_dim=96), kv4.KV4_ERR_UNSUPPORTED), (dict(num_q_heads=7), kv4.KV4_ERR_INVALID_ARG),
+                      (dict(num_q_heads=32, num_kv_heads=2), kv4.KV4_ERR_UNSUPPORTED),
+                      (dict(page_size=24), kv4.KV4_ERR_UNSUPPORTED), (dict(hadamard_block=3), kv4.KV4_ERR_INVALID_ARG),
+                      (dict(hadamard_block=256), kv4.KV4_ERR_INVALID_ARG), (dict(recent_window=0), kv4.KV4_ERR_INVALID_ARG),
+                      (dict(sink_tokens=-1), kv4.KV4_ERR_INVALID_ARG), (dict(num_pages=0), kv4.KV4_ERR_INVALID_ARG)):
+        with pytest.raises(kv4.KV4Error) as e:
+            kv4.kv4_cache_required_bytes(kv4.make_config(**dict(good, **bad)))
+        assert e.value.code == code, bad
+    # BF16 cache ignores the quantization fields
+    kv4.kv4bf16_cache_required_bytes(kv4.make_config(**dict(good, hadamard_block=3, recent_window=0)))
+    assert kv4._lib.kv4_cache_destroy(None) == kv4.KV4_ERR_INVALID_ARG
+    assert kv4._lib.kv4_status_string(kv4.KV4_ERR_WORKSPACE) == b"workspace too small"
+    assert kv4.version().endswith("sm_100a")

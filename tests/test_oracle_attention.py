@@ -153,3 +153,13 @@ def test_bf16_baseline_oracle():
     q = bf16_round(rng.standard_normal((1, 4, 128)).astype(np.float32))
     out = decode_attention_bf16(cache, 0, [1], q)["out_f64"][0]
     np.testing.assert_allclose(out, _sdpa(q[0], k, v, 1 / np.sqrt(128)), atol=1e-12)
+
+
+def test_empty_sequence_gives_zero_row():
+    cache = OracleKV4Cache(_cfg(), _table())
+    rng = np.random.default_rng(9)
+    k = bf16_round(rng.standard_normal((5, 1, 64)).astype(np.float32))
+    cache.append(0, [1], [0, 5], k, k)
+    q = bf16_round(rng.standard_normal((2, 4, 64)).astype(np.float32))
+    out = decode_attention(cache, 0, [0, 1], q)["out_f64"]
+    assert np.all(out[0] == 0) and np.all(np.abs(out[1]) > 0)
