@@ -25,6 +25,8 @@ def flags(verbose_ptxas=False):
          "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"), "-I", os.path.join(HERE, "csrc")]
     if verbose_ptxas:
         f += ["-Xptxas", "-v"]
+    if os.environ.get("KV4_DEBUG_CHECKS") == "1":
+        f += ["-DKV4_DEBUG_CHECKS"]   # self-checking kernels: bad accesses are recorded and skipped
     return f
 
 
@@ -38,7 +40,7 @@ def build(verbose_ptxas=False, force=False):
         path = os.path.join(HERE, "csrc", src)
         obj = os.path.join(OBJDIR, src.replace(".cu", ".o"))
         objs.append(obj)
-        if (not force and os.path.exists(obj) and os.path.getmtime(obj) >= os.path.getmtime(path)
+        if (not force and os.environ.get("KV4_DEBUG_CHECKS") != "1" and os.path.exists(obj) and os.path.getmtime(obj) >= os.path.getmtime(path)
                 and os.path.getmtime(obj) >= newest_header and not verbose_ptxas):
             continue
         cmd = [nvcc()] + flags(verbose_ptxas) + ["-c", path, "-o", obj]

@@ -40,7 +40,10 @@ class _Base:
         return self._ws
 
     def __del__(self):
-        self.close()
+        try:
+            self.close()
+        except Exception:  # interpreter shutdown: the library may already be unloaded
+            pass
 
 
 class KV4Cache(_Base):

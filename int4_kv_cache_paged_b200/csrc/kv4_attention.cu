@@ -22,7 +22,8 @@
 //   attn    persistent, 2 CTAs per SM, 7 consumer warps + 1 producer warp.  The
 //           producer claims items with an atomic counter and streams their tiles
 //           into a shared-memory ring with 1-D bulk copies (mbarrier completion);
-//           consumer warp w takes tiles w, w+7, ... of the item, turns codes into
+//           consumer warp w takes the tiles j with j % 7 == w (j counts tiles over
+//           the CTA's whole item stream), turns codes into
 //           16x8x16 tensor-core operands in registers, keeps an online softmax per
 //           query head, and the 7 warps merge into one partial (m, l, o) per item.
 //   merge   one warp per (sequence, query head): log-sum-exp merge of the item
@@ -33,6 +34,7 @@
 
 namespace kv4 {
 
+
 namespace {
 
 constexpr int NW = 7;                  // consumer warps (+1 producer: 16 warps per SM at 2 CTAs)
@@ -41,12 +43,21 @@ constexpr int QD = 2;                  // item queue depth
 constexpr int PREP_WARPS = 4;
 constexpr float NEG_INF = -INFINITY;
 
+// Ring of shared-memory stages filled by the producer.  Stage s is always
+// consumed by warp s % NW: global tile j goes to stage j % ns and warp j % NW,
+// and ns is a multiple of NW.  A warp therefore waits on the phases of each of
+// its stages strictly in order, which the mbarrier parity test needs (bulk
+// copies may land out of order, so a stage must never be queried two phases
+// ahead of the last fill its consumer has seen).
+// A stage holds one unit: two INT4 tiles (32 tokens), one INT8 tile, or one BF16 tile.
 template <int D, bool BF16>
 struct KCfg {
-  static constexpr int STAGE = BF16 ? tile16_bytes(D) : tile8_bytes(D);
-  static constexpr int NS = BF16 ? 10 : 16;
+  static constexpr int UNIT4 = 2;   // INT4 tiles per unit
+  static constexpr int STAGE = BF16 ? tile16_bytes(D)
+                                    : (UNIT4 * tile4_bytes(D) > tile8_bytes(D) ? UNIT4 * tile4_bytes(D) : tile8_bytes(D));
   static constexpr int QBLOB = qblob_bytes(D);
 };
+constexpr int NS_CHOICES[4] = {4 * NW, 3 * NW, 2 * NW, NW};
 
 // Partial of one item: per query head, o[D] (unnormalised, rotated basis), m, l,
 // padded to D + 4 floats so every head row starts on a 16-byte boundary.
@@ -54,11 +65,11 @@ __host__ __device__ constexpr int head_stride(int D) { return D + 4; }
 __host__ __device__ inline int partial_stride(int G, int D) { return G * head_stride(D); }
 
 template <int D, bool BF16>
-__host__ __device__ inline size_t attn_smem_bytes(int G) {
+__host__ __device__ inline size_t attn_smem_bytes(int G, int ns) {
   using C = KCfg<D, BF16>;
-  return static_cast<size_t>(C::NS) * C::STAGE + static_cast<size_t>(QD) * C::QBLOB +
+  return static_cast<size_t>(ns) * C::STAGE + static_cast<size_t>(QD) * C::QBLOB +
          static_cast<size_t>(NW) * G * head_stride(D) * sizeof(float) + QD * sizeof(Item) +
-         (2 * C::NS + 2 * QD) * sizeof(uint64_t) + 16;
+         (2 * ns + 2 * QD) * sizeof(uint64_t) + 16 + ns * sizeof(int);
 }
 
 // ---------------------------------------------------------------------------
@@ -194,6 +205,11 @@ __global__ void __launch_bounds__(32 * PREP_WARPS) prep_kernel(AttnParams p) {
   }
   uint32_t* blob = reinterpret_cast<uint32_t*>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D));
   const int g = lane >> 2, t = lane & 3;
+  // B-operand column n holds query head n % G when the column split applies
+  // (G = 1, 2, 4: the spare columns carry the low part of the P.V weights),
+  // otherwise head n for n < G and zeros.
+  const bool colsplit = (G == 1 || G == 2 || G == 4);
+  const int gsrc = colsplit ? g % G : g;
   for (int c = 0; c < D / 32; ++c) {
     uint32_t r[4];
 #pragma unroll
@@ -203,7 +219,7 @@ __global__ void __launch_bounds__(32 * PREP_WARPS) prep_kernel(AttnParams p) {
       for (int reg = 0; reg < 2; ++reg) {
         const int d = 16 * k + 2 * t + 8 * reg;
         float a = 0.f, bb = 0.f;
-        if (g < G) { a = sq[g * D + d]; bb = sq[g * D + d + 1]; }
+        if (gsrc < G) { a = sq[gsrc * D + d]; bb = sq[gsrc * D + d + 1]; }
         if constexpr (BF16) {
           r[2 * kk + reg] = pack_bf162(a, bb);
         } else {
@@ -215,10 +231,11 @@ __global__ void __launch_bounds__(32 * PREP_WARPS) prep_kernel(AttnParams p) {
   }
   float* tail = reinterpret_cast<float*>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D) + 16 * D);
   if (lane < MAX_G) {
+    const int src = colsplit ? lane % G : lane;
     float v = 0.f;
 #pragma unroll
     for (int gg = 0; gg < MAX_G; ++gg)
-      if (gg == lane && gg < G) v = qsum[gg];
+      if (gg == src && gg < G) v = qsum[gg];
     tail[lane] = BF16 ? 0.f : v * p.scale_log2;
   }
   if (lane == MAX_G) tail[MAX_G] = ldexpf(p.scale_log2, -e);
@@ -231,6 +248,12 @@ template <int D>
 struct WarpState {
   float o[D / 16][4];  // o^T fragments: (dim 16m+g, head 2t), (16m+g, 2t+1), (16m+g+8, 2t), (16m+g+8, 2t+1)
   float m0, m1, l0, l1, z0, z1;
+};
+
+// Column split of the P.V weights (see pv_operands): part of each of the thread's two columns.
+struct ColSplit {
+  bool colsplit;
+  int part0, part1;
 };
 
 template <int D>
@@ -261,29 +284,45 @@ __device__ __forceinline__ void online_softmax_pv(WarpState<D>& ws, float x0, fl
   p0 = ex2(x0 - ws.m0); p1 = ex2(x1 - ws.m1); p2 = ex2(x2 - ws.m0); p3 = ex2(x3 - ws.m1);
 }
 
-// One INT4 tile at shared address st.
-template <int D, bool MASKED>
-__device__ __forceinline__ void tile_int4(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, bool vg,
-                                          bool vg8, uint32_t empty_bar) {
+
+// P.V weights of this thread's two columns (c0 = 2t, c1 = 2t+1) for tokens g and
+// g+8.  With the column split (G = 1, 2, 4), column c carries part c / G of the
+// weight of head c % G: part 0 = hi = fp16(P), part 1 = lo = fp16(P - hi),
+// parts >= 2 are zero; one 16x8x16 multiply then accumulates both parts.
+// Without it (other G) the hi parts go to (B0, B1) and the lo parts to (C0, C1).
+__device__ __forceinline__ void pv_operands(float P0, float P1, float P2, float P3, int part0, int part1,
+                                            bool colsplit, uint32_t& B0, uint32_t& B1, uint32_t& C0, uint32_t& C1) {
+  const uint32_t h01 = pack_half2(P0, P1), h23 = pack_half2(P2, P3);
+  const uint32_t l01 = pack_half2(P0 - half_lo(h01), P1 - half_hi(h01));
+  const uint32_t l23 = pack_half2(P2 - half_lo(h23), P3 - half_hi(h23));
+  if (colsplit) {
+    const uint32_t m0 = part0 == 0 ? 0x0000FFFFu : 0u, m1 = part1 == 0 ? 0xFFFF0000u : 0u;
+    const uint32_t n0 = part0 == 1 ? 0x0000FFFFu : 0u, n1 = part1 == 1 ? 0xFFFF0000u : 0u;
+    B0 = movmatrix_trans((h01 & (m0 | m1)) | (l01 & (n0 | n1)));
+    B1 = movmatrix_trans((h23 & (m0 | m1)) | (l23 & (n0 | n1)));
+    C0 = C1 = 0u;
+  } else {
+    B0 = movmatrix_trans(h01);
+    B1 = movmatrix_trans(h23);
+    C0 = movmatrix_trans(l01);
+    C1 = movmatrix_trans(l23);
+  }
+}
+
+// QK^T of one INT4 tile: acc = (q * 2^e) . codes for tokens g, g+8 and heads 2t, 2t+1.
+template <int D>
+__device__ __forceinline__ void qk_int4(uint32_t st, const QFrag<D>& qf, int lane, float (&acc)[4]) {
   constexpr int NKK = D / 32;
-  uint32_t kw0[NKK], kw1[NKK], vw[D / 16];
+  uint32_t kw0[NKK], kw1[NKK];
   if constexpr (D == 128) {
     const uint4 a = lds128(st + lane * 16), bq = lds128(st + 512 + lane * 16);
     kw0[0] = a.x; kw0[1] = a.y; kw0[2] = a.z; kw0[3] = a.w;
     kw1[0] = bq.x; kw1[1] = bq.y; kw1[2] = bq.z; kw1[3] = bq.w;
-    const uint4 v0 = lds128(st + 8 * D + lane * 16), v1 = lds128(st + 8 * D + 512 + lane * 16);
-    vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
-    vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
   } else {
     const uint2 a = lds64(st + lane * 8), bq = lds64(st + 256 + lane * 8);
     kw0[0] = a.x; kw0[1] = a.y; kw1[0] = bq.x; kw1[1] = bq.y;
-    const uint4 v0 = lds128(st + 8 * D + lane * 16);
-    vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
   }
-  const uint4 sz = lds128(st + 16 * D + (lane >> 2) * 16);
-  __syncwarp();
-  if (lane == 0) mbar_arrive(empty_bar);  // the tile is in registers: hand the stage back
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
 #pragma unroll
   for (int kk = 0; kk < NKK; ++kk) {
     const uint32_t w0 = kw0[kk], w1 = kw1[kk];
@@ -291,40 +330,124 @@ __device__ __forceinline__ void tile_int4(uint32_t st, const QFrag<D>& qf, WarpS
     const uint32_t u0 = w0 >> 8, u1 = w1 >> 8;
     mma_f16(acc, nib_lo(u0), nib_lo(u1), nib_hi(u0), nib_hi(u1), qf.b[2 * kk + 1][0], qf.b[2 * kk + 1][1]);
   }
-  const float sKg = half_lo(sz.x) * qf.kscale, zKg = half_hi(sz.x);
-  const float sKg8 = half_lo(sz.y) * qf.kscale, zKg8 = half_hi(sz.y);
-  float x0 = fmaf(acc[0], sKg, zKg * qf.qs0);
-  float x1 = fmaf(acc[1], sKg, zKg * qf.qs1);
-  float x2 = fmaf(acc[2], sKg8, zKg8 * qf.qs0);
-  float x3 = fmaf(acc[3], sKg8, zKg8 * qf.qs1);
-  if constexpr (MASKED) {
-    if (!vg) { x0 = NEG_INF; x1 = NEG_INF; }
-    if (!vg8) { x2 = NEG_INF; x3 = NEG_INF; }
+}
+
+// P.V of one INT4 tile: o^T[m] += V^T codes * (hi + lo) weights.
+template <int D>
+__device__ __forceinline__ void pv_int4(uint32_t st, WarpState<D>& ws, int lane, uint32_t B0, uint32_t B1,
+                                        uint32_t C0, uint32_t C1, bool colsplit) {
+  uint32_t vw[D / 16];
+  if constexpr (D == 128) {
+    const uint4 v0 = lds128(st + 8 * D + lane * 16), v1 = lds128(st + 8 * D + 512 + lane * 16);
+    vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+    vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
+  } else {
+    const uint4 v0 = lds128(st + 8 * D + lane * 16);
+    vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
   }
-  float p0, p1, p2, p3;
-  online_softmax_pv<D>(ws, x0, x1, x2, x3, p0, p1, p2, p3);
-  const float sVg = half_lo(sz.z), zVg = half_hi(sz.z), sVg8 = half_lo(sz.w), zVg8 = half_hi(sz.w);
-  float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
-  float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
-  if constexpr (MASKED) {
-    if (!vg) { P0 = 0.f; P1 = 0.f; zg0 = 0.f; zg1 = 0.f; }
-    if (!vg8) { P2 = 0.f; P3 = 0.f; zg80 = 0.f; zg81 = 0.f; }
-  }
-  ws.l0 += p0 + p2; ws.l1 += p1 + p3;
-  ws.z0 += zg0 + zg80; ws.z1 += zg1 + zg81;
-  const uint32_t B0 = movmatrix_trans(pack_half2(P0, P1));
-  const uint32_t B1 = movmatrix_trans(pack_half2(P2, P3));
 #pragma unroll
   for (int m = 0; m < D / 16; ++m) {
     const uint32_t w = vw[m], u = w >> 8;
-    mma_f16(ws.o[m], nib_lo(w), nib_hi(w), nib_lo(u), nib_hi(u), B0, B1);
+    const uint32_t a0 = nib_lo(w), a1 = nib_hi(w), a2 = nib_lo(u), a3 = nib_hi(u);
+    mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
+    if (!colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
+  }
+}
+
+// One unit of NT (1 or 2) INT4 tiles at st, st + tile4_bytes(D): scores, one
+// online-softmax update for the NT*16 tokens, P.V.  valid[u] bit 0 / bit 1:
+// token g / g+8 of tile u is inside the item's range (used when MASKED).  The
+// stage is handed back after its last shared-memory load.
+template <int D, int NT, bool MASKED>
+__device__ __forceinline__ void unit_int4(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane,
+                                          const int (&valid)[2], uint32_t empty_bar, const ColSplit& cs) {
+  constexpr int TB = tile4_bytes(D);
+  float x[NT][4];
+  uint4 sz[NT];
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    float acc[4];
+    qk_int4<D>(st + u * TB, qf, lane, acc);
+    sz[u] = lds128(st + u * TB + 16 * D + (lane >> 2) * 16);
+    const float sKg = half_lo(sz[u].x) * qf.kscale, zKg = half_hi(sz[u].x);
+    const float sKg8 = half_lo(sz[u].y) * qf.kscale, zKg8 = half_hi(sz[u].y);
+    x[u][0] = fmaf(acc[0], sKg, zKg * qf.qs0);
+    x[u][1] = fmaf(acc[1], sKg, zKg * qf.qs1);
+    x[u][2] = fmaf(acc[2], sKg8, zKg8 * qf.qs0);
+    x[u][3] = fmaf(acc[3], sKg8, zKg8 * qf.qs1);
+    if constexpr (MASKED) {
+      if (!(valid[u] & 1)) { x[u][0] = NEG_INF; x[u][1] = NEG_INF; }
+      if (!(valid[u] & 2)) { x[u][2] = NEG_INF; x[u][3] = NEG_INF; }
+    }
+  }
+  // online softmax over the unit: max over tokens g, g+8 of every tile, then over the 8 row groups
+  float mx0 = fmaxf(x[0][0], x[0][2]), mx1 = fmaxf(x[0][1], x[0][3]);
+#pragma unroll
+  for (int u = 1; u < NT; ++u) {
+    mx0 = fmaxf(mx0, fmaxf(x[u][0], x[u][2]));
+    mx1 = fmaxf(mx1, fmaxf(x[u][1], x[u][3]));
+  }
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+  }
+  const float n0 = fmaxf(ws.m0, mx0), n1 = fmaxf(ws.m1, mx1);
+  if (__any_sync(0xffffffffu, n0 > ws.m0 || n1 > ws.m1)) {
+    const float a0 = ex2(ws.m0 - n0), a1 = ex2(ws.m1 - n1);
+    ws.l0 *= a0; ws.l1 *= a1; ws.z0 *= a0; ws.z1 *= a1;
+#pragma unroll
+    for (int m = 0; m < D / 16; ++m) {
+      ws.o[m][0] *= a0; ws.o[m][1] *= a1; ws.o[m][2] *= a0; ws.o[m][3] *= a1;
+    }
+    ws.m0 = n0; ws.m1 = n1;
+  }
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    const float p0 = ex2(x[u][0] - ws.m0), p1 = ex2(x[u][1] - ws.m1);
+    const float p2 = ex2(x[u][2] - ws.m0), p3 = ex2(x[u][3] - ws.m1);
+    const float sVg = half_lo(sz[u].z), zVg = half_hi(sz[u].z), sVg8 = half_lo(sz[u].w), zVg8 = half_hi(sz[u].w);
+    float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
+    float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
+    if constexpr (MASKED) {   // unwritten slots may hold non-finite scales
+      if (!(valid[u] & 1)) { P0 = 0.f; P1 = 0.f; zg0 = 0.f; zg1 = 0.f; }
+      if (!(valid[u] & 2)) { P2 = 0.f; P3 = 0.f; zg80 = 0.f; zg81 = 0.f; }
+    }
+    ws.l0 += p0 + p2; ws.l1 += p1 + p3;
+    ws.z0 += zg0 + zg80; ws.z1 += zg1 + zg81;
+    uint32_t B0, B1, C0, C1;
+    pv_operands(P0, P1, P2, P3, cs.part0, cs.part1, cs.colsplit, B0, B1, C0, C1);
+    if (u == NT - 1) {
+      // last tile: load its V codes, then hand the stage back before the math
+      const uint32_t t = st + u * TB;
+      uint32_t vw[D / 16];
+      if constexpr (D == 128) {
+        const uint4 v0 = lds128(t + 8 * D + lane * 16), v1 = lds128(t + 8 * D + 512 + lane * 16);
+        vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+        vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
+      } else {
+        const uint4 v0 = lds128(t + 8 * D + lane * 16);
+        vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar);
+#pragma unroll
+      for (int m = 0; m < D / 16; ++m) {
+        const uint32_t w = vw[m], uu = w >> 8;
+        const uint32_t a0 = nib_lo(w), a1 = nib_hi(w), a2 = nib_lo(uu), a3 = nib_hi(uu);
+        mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
+        if (!cs.colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
+      }
+    } else {
+      pv_int4<D>(st + u * TB, ws, lane, B0, B1, C0, C1, cs.colsplit);
+    }
   }
 }
 
 // One INT8 tile (protected store).
 template <int D, bool MASKED>
 __device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, bool vg,
-                                          bool vg8, uint32_t empty_bar) {
+                                          bool vg8, uint32_t empty_bar, const ColSplit& cs) {
   constexpr int NK = D / 16;
   uint32_t kw[2][NK], vw[2 * NK];
 #pragma unroll
@@ -369,19 +492,24 @@ __device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpS
   }
   ws.l0 += p0 + p2; ws.l1 += p1 + p3;
   ws.z0 += zg0 + zg80; ws.z1 += zg1 + zg81;
-  const uint32_t B0 = movmatrix_trans(pack_half2(P0, P1));
-  const uint32_t B1 = movmatrix_trans(pack_half2(P2, P3));
+  uint32_t B0, B1, C0, C1;
+  pv_operands(P0, P1, P2, P3, cs.part0, cs.part1, cs.colsplit, B0, B1, C0, C1);
 #pragma unroll
   for (int m = 0; m < NK; ++m) {
     const uint32_t w0 = vw[2 * m], w1 = vw[2 * m + 1];
-    mma_f16(ws.o[m], byte_lo(w0), byte_lo(w0 >> 8), byte_lo(w1), byte_lo(w1 >> 8), B0, B1);
+    const uint32_t a0 = byte_lo(w0), a1 = byte_lo(w0 >> 8), a2 = byte_lo(w1), a3 = byte_lo(w1 >> 8);
+    mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
+    if (!cs.colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
   }
 }
 
 // One BF16 tile (baseline cache).  Holds the stage until the V loads are done.
+// vmask01 / vmask89: per-thread masks of the V operand halves of tokens 2t, 2t+1
+// and 2t+8, 2t+9 (unwritten slots of a page may hold NaN bit patterns, and
+// 0 * NaN would poison the accumulator).
 template <int D, bool MASKED>
 __device__ __forceinline__ void tile_bf16(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, bool vg,
-                                          bool vg8, uint32_t empty_bar) {
+                                          bool vg8, uint32_t empty_bar, uint32_t vmask01, uint32_t vmask89) {
   constexpr int NK = D / 16;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -391,7 +519,12 @@ __device__ __forceinline__ void tile_bf16(uint32_t st, const QFrag<D>& qf, WarpS
   }
   uint4 v[NK];
 #pragma unroll
-  for (int m = 0; m < NK; ++m) v[m] = lds128(st + 32 * D + 16 * (32 * m + lane));
+  for (int m = 0; m < NK; ++m) {
+    v[m] = lds128(st + 32 * D + 16 * (32 * m + lane));
+    if constexpr (MASKED) {
+      v[m].x &= vmask01; v[m].y &= vmask01; v[m].z &= vmask89; v[m].w &= vmask89;
+    }
+  }
   __syncwarp();
   if (lane == 0) mbar_arrive(empty_bar);
   float x0 = acc[0] * qf.kscale, x1 = acc[1] * qf.kscale, x2 = acc[2] * qf.kscale, x3 = acc[3] * qf.kscale;
@@ -441,21 +574,24 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(AttnParams p) {
   using C = KCfg<D, BF16>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
-  uint8_t* qbuf = ring + C::NS * C::STAGE;
+  const int NS = p.ns;
+  uint8_t* qbuf = ring + NS * C::STAGE;
   float* merge = reinterpret_cast<float*>(qbuf + QD * C::QBLOB);
   Item* itemq = reinterpret_cast<Item*>(merge + NW * p.G * head_stride(D));
   uint64_t* bars = reinterpret_cast<uint64_t*>(itemq + QD);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * C::NS + 2 * QD);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * NS + 2 * QD);
   volatile int* go_flag = abort_flag + 1;
-  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * C::NS;
-  const uint32_t iqf0 = full0 + 16 * C::NS, iqe0 = iqf0 + 8 * QD;
+  int* last_fill = const_cast<int*>(abort_flag) + 4;   // [NS]: global index of the last tile copied into each stage
+  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * NS;
+  const uint32_t iqf0 = full0 + 16 * NS, iqe0 = iqf0 + 8 * QD;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NS; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
+    for (int s = 0; s < NS; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
     for (int s = 0; s < QD; ++s) { mbar_init(iqf0 + 8 * s, 1); mbar_init(iqe0 + 8 * s, NW); }
     *abort_flag = 0;
     *go_flag = 0;
+    for (int st = 0; st < NS; ++st) last_fill[st] = -1;
     fence_barrier_init();
   }
   __syncthreads();
@@ -481,6 +617,30 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(AttnParams p) {
     k_nxt = __shfl_sync(0xffffffffu, k_nxt, 0);
     Item cur{};
     if (k_cur < total) cur = load_item(k_cur);
+    const int nbatch = NS < 32 ? NS : 32;
+    auto units_of = [&](const Item& itm) {
+      const int UT = (BF16 || itm.kind == 1) ? 1 : C::UNIT4;
+      return (itm.t_end - itm.t_begin + UT - 1) / UT;
+    };
+    auto source = [&](const Item& itm, int u, int k) -> const uint8_t* {   // tile k of unit u
+      const int UT = (BF16 || itm.kind == 1) ? 1 : C::UNIT4;
+      const int i = u * UT + k;
+      const uint8_t* a = nullptr;
+      if (lane < nbatch && k < UT && i < itm.t_end - itm.t_begin) {
+        a = tile_source<D, BF16>(p, itm, itm.t_begin + i);
+#ifdef KV4_DEBUG_CHECKS
+        const uint8_t* lo = itm.kind == 1 ? p.prot : p.pool;
+        const size_t ext = itm.kind == 1 ? p.prot_bytes : p.pool_bytes;
+        const uint32_t tb = itm.kind == 1 ? tile8_bytes(D) : (BF16 ? tile16_bytes(D) : tile4_bytes(D));
+        if (a < lo || a + tb > lo + ext) { dbg_fail(10, a - lo, ext); a = nullptr; }
+#endif
+      }
+      return a;
+    };
+    const uint8_t* pre0 = nullptr;
+    const uint8_t* pre1 = nullptr;
+    bool have_pre = false;
+    Item nxt{};
     uint32_t it = 0;
     int q = 0;
     bool ok = true;
@@ -493,37 +653,60 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(AttnParams p) {
         if (lane == 0) { itemq[slot].kind = -1; mbar_arrive(iqf0 + 8 * slot); }
         break;
       }
-      Item nxt{};
+      nxt = Item{};
       if (k_nxt < total) nxt = load_item(k_nxt);
       int k_new = total;
       if (lane == 0 && k_nxt < total) k_new = atomicAdd(&p.state->work, 1);
+#ifdef KV4_DEBUG_CHECKS
+      if (static_cast<size_t>(cur.b * p.Hkv + cur.h + 1) * C::QBLOB > p.qblob_total) dbg_fail(11, cur.b, cur.h);
+      if (!KV4_SMEM_OK(smem_u32(itemq + slot), sizeof(Item), 4, 12)) { ok = false; }
+#endif
       if (lane == 0) {
         itemq[slot] = cur;
         mbar_arrive_expect_tx(iqf0 + 8 * slot, C::QBLOB);
         bulk_g2s(smem_u32(qbuf + slot * C::QBLOB),
                  p.qblob + static_cast<size_t>(cur.b * p.Hkv + cur.h) * C::QBLOB, C::QBLOB, iqf0 + 8 * slot);
       }
-      const int ntiles = cur.t_end - cur.t_begin;
+      // a unit is UT tiles (2 for INT4 pages, 1 for INT8 and BF16 tiles) copied into one stage
+      const int nunits = units_of(cur);
       const uint32_t tbytes = cur.kind == 1 ? tile8_bytes(D) : (BF16 ? tile16_bytes(D) : tile4_bytes(D));
-      for (int base = 0; base < ntiles && ok; base += 32) {
-        const uint8_t* src = nullptr;
-        if (base + lane < ntiles) src = tile_source<D, BF16>(p, cur, cur.t_begin + base + lane);
-        const int n = min(32, ntiles - base);
-        for (int j = 0; j < n; ++j) {
-          const unsigned long long a = __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(src), j);
-          if (lane == 0) {
-            const int s = it % C::NS;
-            ok = mbar_wait(empty0 + 8 * s, ((it / C::NS) & 1) ^ 1, abort_flag, status);
-            if (ok) {
-              mbar_arrive_expect_tx(full0 + 8 * s, tbytes);
-              bulk_g2s(smem_u32(ring + s * C::STAGE), reinterpret_cast<const void*>(a), tbytes, full0 + 8 * s);
-            }
+      // Lanes issue in parallel, one unit each; a batch of at most NS units never
+      // uses a stage twice, so every lane waits only for its own stage.  Source
+      // addresses (block-table lookups) are loaded one batch ahead, and those of
+      // the next item's first batch while this item streams.
+      const uint8_t* nxt0 = have_pre ? pre0 : source(cur, lane, 0);
+      const uint8_t* nxt1 = have_pre ? pre1 : source(cur, lane, 1);
+      have_pre = false;
+      for (int base = 0; base < nunits; base += nbatch) {
+        const uint8_t* src0 = nxt0;
+        const uint8_t* src1 = nxt1;
+        nxt0 = source(cur, base + nbatch + lane, 0);
+        nxt1 = source(cur, base + nbatch + lane, 1);
+        bool lane_ok = true;
+        if (lane < nbatch && base + lane < nunits) {
+          const uint32_t j = it + base + lane;
+          const int s = j % NS;
+          lane_ok = src0 != nullptr && mbar_wait(empty0 + 8 * s, ((j / NS) & 1) ^ 1, abort_flag, status);
+          if (lane_ok) {
+            const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * C::STAGE);
+            mbar_arrive_expect_tx(full0 + 8 * s, src1 ? 2 * tbytes : tbytes);
+            bulk_g2s(dst, src0, tbytes, full0 + 8 * s);
+            if (src1) bulk_g2s(dst + tbytes, src1, tbytes, full0 + 8 * s);
+            last_fill[s] = static_cast<int>(j);
+          } else {
+            *abort_flag = 1;
           }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) break;
-          ++it;
+        }
+        ok = __all_sync(0xffffffffu, lane_ok);
+        if (!ok) break;
+        if (base == 0 && k_nxt < total) {
+          // the next item's descriptor has arrived by now: start its first block-table loads
+          pre0 = source(nxt, lane, 0);
+          pre1 = source(nxt, lane, 1);
+          have_pre = true;
         }
       }
+      it += nunits;
       if (!ok) break;
       cur = nxt;
       k_cur = k_nxt;
@@ -531,8 +714,8 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(AttnParams p) {
     }
     if (!ok && lane == 0) {
       // aborted: let this CTA's copies land before the shared memory is released
-      const uint32_t first = it > static_cast<uint32_t>(C::NS) ? it - C::NS : 0u;
-      for (uint32_t j = first; j < it; ++j) mbar_drain(full0 + 8 * (j % C::NS), (j / C::NS) & 1);
+      for (int st = 0; st < NS; ++st)
+        if (last_fill[st] >= 0) mbar_drain(full0 + 8 * st, (last_fill[st] / NS) & 1);
       for (int j = q > QD ? q - QD : 0; j < q; ++j) mbar_drain(iqf0 + 8 * (j % QD), (j / QD) & 1);
     }
     return;
@@ -542,6 +725,10 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(AttnParams p) {
   const int g = lane >> 2, t = lane & 3;
   const int G = p.G;
   const int pstride = partial_stride(G, D);
+  ColSplit cs;
+  cs.colsplit = !BF16 && (G == 1 || G == 2 || G == 4);
+  cs.part0 = cs.colsplit ? (2 * t) / G : 0;
+  cs.part1 = cs.colsplit ? (2 * t + 1) / G : 0;
   uint32_t it = 0;
   for (int q = 0;; ++q) {
     const int slot = q % QD;
@@ -577,30 +764,65 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(AttnParams p) {
     ws.l0 = ws.l1 = ws.z0 = ws.z1 = 0.f;
 
     const int ntiles = cur.t_end - cur.t_begin;
-    for (int i = warp; i < ntiles; i += NW) {
-      const uint32_t j = it + i;
-      const int s = j % C::NS;
-      if (!mbar_wait(full0 + 8 * s, (j / C::NS) & 1, abort_flag, status)) break;
-      const uint32_t st = smem_u32(ring + s * C::STAGE);
-      const int pos0 = (cur.t_begin + i) * TILE;
-      const bool inside = pos0 >= cur.lo && pos0 + TILE <= cur.hi;
-      const bool vg = pos0 + g >= cur.lo && pos0 + g < cur.hi;
-      const bool vg8 = pos0 + g + 8 >= cur.lo && pos0 + g + 8 < cur.hi;
+    const int UT = (BF16 || cur.kind == 1) ? 1 : C::UNIT4;
+    const int nunits = (ntiles + UT - 1) / UT;
+    // this warp's units: global unit index j = it + u with j % NW == warp (it owns stage j % NS)
+    const int u0 = (warp - static_cast<int>(it % NW) + NW) % NW;
+    for (int u = u0; u < nunits; u += NW) {
+      const uint32_t j = it + u;
+      const int s = j % NS;
+      if (!mbar_wait(full0 + 8 * s, (j / NS) & 1, abort_flag, status)) break;
+      const uint32_t st = smem_u32(ring + static_cast<size_t>(s) * C::STAGE);
+      const int tile0 = cur.t_begin + u * UT;
+      const int nt = min(UT, cur.t_end - tile0);
+      const int pos0 = tile0 * TILE;
+      const bool inside = pos0 >= cur.lo && pos0 + nt * TILE <= cur.hi;
+      auto valid_bits = [&](int k) {
+        const int pg = pos0 + k * TILE + g;
+        return (pg >= cur.lo && pg < cur.hi ? 1 : 0) | (pg + 8 >= cur.lo && pg + 8 < cur.hi ? 2 : 0);
+      };
       const uint32_t eb = empty0 + 8 * s;
       if constexpr (BF16) {
-        if (inside) tile_bf16<D, false>(st, qf, ws, lane, vg, vg8, eb);
-        else tile_bf16<D, true>(st, qf, ws, lane, vg, vg8, eb);
+        const int vb = valid_bits(0);
+        if (inside) {
+          tile_bf16<D, false>(st, qf, ws, lane, true, true, eb, 0u, 0u);
+        } else {
+          auto ok_pos = [&](int r) { return pos0 + r >= cur.lo && pos0 + r < cur.hi; };
+          const uint32_t m01 = (ok_pos(2 * t) ? 0x0000FFFFu : 0u) | (ok_pos(2 * t + 1) ? 0xFFFF0000u : 0u);
+          const uint32_t m89 = (ok_pos(2 * t + 8) ? 0x0000FFFFu : 0u) | (ok_pos(2 * t + 9) ? 0xFFFF0000u : 0u);
+          tile_bf16<D, true>(st, qf, ws, lane, vb & 1, vb & 2, eb, m01, m89);
+        }
       } else if (cur.kind == 1) {
-        if (inside) tile_int8<D, false>(st, qf, ws, lane, vg, vg8, eb);
-        else tile_int8<D, true>(st, qf, ws, lane, vg, vg8, eb);
+        const int vb = valid_bits(0);
+        if (inside) tile_int8<D, false>(st, qf, ws, lane, true, true, eb, cs);
+        else tile_int8<D, true>(st, qf, ws, lane, vb & 1, vb & 2, eb, cs);
       } else {
-        if (inside) tile_int4<D, false>(st, qf, ws, lane, vg, vg8, eb);
-        else tile_int4<D, true>(st, qf, ws, lane, vg, vg8, eb);
+        const int valid[2] = {valid_bits(0), valid_bits(1)};
+        if (nt == 2) {
+          if (inside) unit_int4<D, 2, false>(st, qf, ws, lane, valid, eb, cs);
+          else unit_int4<D, 2, true>(st, qf, ws, lane, valid, eb, cs);
+        } else {
+          if (inside) unit_int4<D, 1, false>(st, qf, ws, lane, valid, eb, cs);
+          else unit_int4<D, 1, true>(st, qf, ws, lane, valid, eb, cs);
+        }
       }
     }
-    it += ntiles;
+    it += nunits;
 
     // ---- merge the NW warps into one partial
+    if (cs.colsplit) {
+      // fold the low-part columns into the high-part ones (column c + G into column c)
+      if (G == 1) {
+#pragma unroll
+        for (int m = 0; m < D / 16; ++m) { ws.o[m][0] += ws.o[m][1]; ws.o[m][2] += ws.o[m][3]; }
+      } else {
+        const int x = G == 4 ? 2 : 1;
+#pragma unroll
+        for (int m = 0; m < D / 16; ++m)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) ws.o[m][i] += __shfl_xor_sync(0xffffffffu, ws.o[m][i], x);
+      }
+    }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       ws.l0 += __shfl_xor_sync(0xffffffffu, ws.l0, o);
@@ -610,6 +832,9 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(AttnParams p) {
     }
     constexpr int HS = head_stride(D);
     float* mw = merge + warp * G * HS;
+#ifdef KV4_DEBUG_CHECKS
+    if (!KV4_SMEM_OK(smem_u32(mw), G * HS * 4, 4, 13)) continue;
+#endif
     const int h0 = 2 * t, h1 = 2 * t + 1;
     if (h0 < G) {
       float* r = mw + h0 * HS;
@@ -766,17 +991,28 @@ inline WsLayout ws_layout(const kv4_cache* c, int n_seqs, int cap0) {
   return w;
 }
 
+// Deepest ring (a multiple of NW) that keeps 2 CTAs per SM, else 1 CTA per SM.
 template <int D, bool BF16>
-int occupancy(int G) {
-  // the attribute is per kernel and process-wide: allow the largest group size once
-  const size_t smem = attn_smem_bytes<D, BF16>(G);
-  if (cudaFuncSetAttribute(attn_kernel<D, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(attn_smem_bytes<D, BF16>(MAX_G))) != cudaSuccess)
+int choose_ring(int device, int G, int* blocks_per_sm) {
+  int optin = 0;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess) return -1;
+  // the attribute is per kernel and process-wide: allow the device maximum once
+  if (cudaFuncSetAttribute(attn_kernel<D, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess)
     return -1;
-  int blocks = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, attn_kernel<D, BF16>, THREADS, smem) != cudaSuccess)
-    return -1;
-  return blocks;
+  for (int want = 2; want >= 1; --want) {
+    for (int ns : NS_CHOICES) {
+      const size_t smem = attn_smem_bytes<D, BF16>(G, ns);
+      if (smem > static_cast<size_t>(optin)) continue;
+      int blocks = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, attn_kernel<D, BF16>, THREADS, smem) != cudaSuccess)
+        return -1;
+      if (blocks >= want) {
+        *blocks_per_sm = blocks > 2 ? 2 : blocks;
+        return ns;
+      }
+    }
+  }
+  return -1;
 }
 
 template <int D, bool BF16>
@@ -792,7 +1028,7 @@ int launch_attention_t(kv4_cache* c, AttnParams& p, cudaStream_t stream) {
   if (grid > max_items) grid = max_items;
   if (grid < 1) grid = 1;
   if (c->ev_before) cudaEventRecord(c->ev_before, stream);
-  attn_kernel<D, BF16><<<static_cast<unsigned>(grid), THREADS, attn_smem_bytes<D, BF16>(p.G), stream>>>(p);
+  attn_kernel<D, BF16><<<static_cast<unsigned>(grid), THREADS, attn_smem_bytes<D, BF16>(p.G, p.ns), stream>>>(p);
   if (c->ev_after) cudaEventRecord(c->ev_after, stream);
   const int merge_warps = p.n_seqs * p.Hq;
   merge_kernel<D, BF16><<<(merge_warps + 7) / 8, 256, 0, stream>>>(p);
@@ -801,10 +1037,24 @@ int launch_attention_t(kv4_cache* c, AttnParams& p, cudaStream_t stream) {
 
 }  // namespace
 
+#ifdef KV4_DEBUG_CHECKS
+extern "C" int kv4_debug_read(unsigned long long* out4) {
+  if (cudaMemcpyFromSymbol(out4, kv4_debug_slot, 4 * sizeof(unsigned long long)) != cudaSuccess) return KV4_ERR_CUDA;
+  const unsigned long long zero[4] = {0, 0, 0, 0};
+  return cudaMemcpyToSymbol(kv4_debug_slot, zero, sizeof(zero)) == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+}
+#endif
+
 int attention_blocks_per_sm(kv4_cache* c) {
   const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
-  if (c->cfg.head_dim == 128) return c->bf16 ? occupancy<128, true>(G) : occupancy<128, false>(G);
-  return c->bf16 ? occupancy<64, true>(G) : occupancy<64, false>(G);
+  int blocks = 0, ns;
+  if (c->cfg.head_dim == 128)
+    ns = c->bf16 ? choose_ring<128, true>(c->device, G, &blocks) : choose_ring<128, false>(c->device, G, &blocks);
+  else
+    ns = c->bf16 ? choose_ring<64, true>(c->device, G, &blocks) : choose_ring<64, false>(c->device, G, &blocks);
+  if (ns <= 0) return -1;
+  c->attn_ring = ns;
+  return blocks;
 }
 
 size_t attention_workspace_bytes(const kv4_cache* c, int n_seqs, int max_ctx) {
@@ -852,6 +1102,9 @@ int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs
   p.seqhead = reinterpret_cast<SeqHead*>(wsb + w.seqhead);
   p.qblob = wsb + w.qblob;
   p.partials = reinterpret_cast<float*>(wsb + w.partials);
+  p.pool_bytes = c->pool_bytes;
+  p.prot_bytes = c->prot_bytes;
+  p.qblob_total = static_cast<size_t>(n_seqs) * cfg.num_kv_heads * qblob_bytes(D);
   p.cap_parts = w.cap_parts;
   p.n_seqs = n_seqs;
   p.Hq = cfg.num_q_heads;
@@ -867,6 +1120,7 @@ int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs
   p.num_pages = cfg.num_pages;
   p.max_pages_per_seq = cfg.max_pages_per_seq;
   p.chunk_tiles = chunk_tiles_for(c, n_seqs);
+  p.ns = c->attn_ring;
   p.mode = mode;
   const double scale = softmax_scale > 0.f ? static_cast<double>(softmax_scale) : 1.0 / sqrt(static_cast<double>(D));
   p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);

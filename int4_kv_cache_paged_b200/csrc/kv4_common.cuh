@@ -94,7 +94,44 @@ struct AttnParams {
   int mode;
   float scale_log2;           // softmax_scale * log2(e)
   float rot_c;                // fp32(1/sqrt(Bh))
+  size_t pool_bytes, prot_bytes, qblob_total;   // extents, for the self-checks of debug builds
+  int ns;                     // shared-memory ring depth of the attention kernel
 };
+
+// ---------------------------------------------------------------------------
+// Self-checks (debug builds, -DKV4_DEBUG_CHECKS): every shared-memory access,
+// bulk copy and mbarrier address is checked against its buffer; a bad access is
+// recorded in kv4_debug_slot (first failure wins) and skipped.
+
+#ifdef KV4_DEBUG_CHECKS
+static __device__ unsigned long long kv4_debug_slot[4];   // code, value a, value b, count (per translation unit)
+extern __shared__ __align__(128) uint8_t kv4_dyn_smem[];
+__device__ __forceinline__ uint32_t dyn_smem_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ bool dbg_fail(int code, unsigned long long a, unsigned long long b) {
+  if (atomicCAS(&kv4_debug_slot[0], 0ull, static_cast<unsigned long long>(code)) == 0ull) {
+    kv4_debug_slot[1] = a;
+    kv4_debug_slot[2] = b;
+  }
+  atomicAdd(&kv4_debug_slot[3], 1ull);
+  return true;
+}
+// true when [addr, addr+bytes) is inside the dynamic shared window and aligned
+__device__ __forceinline__ bool smem_ok(uint32_t addr, uint32_t bytes, uint32_t align, int code) {
+  const uint32_t lo = static_cast<uint32_t>(__cvta_generic_to_shared(kv4_dyn_smem));
+  if (addr < lo || addr + bytes > lo + dyn_smem_size() || (addr & (align - 1))) {
+    dbg_fail(code, addr - lo, bytes);
+    return false;
+  }
+  return true;
+}
+#define KV4_SMEM_OK(addr, bytes, align, code) ::kv4::smem_ok((addr), (bytes), (align), (code))
+#else
+#define KV4_SMEM_OK(addr, bytes, align, code) true
+#endif
 
 // ---------------------------------------------------------------------------
 // PTX helpers
@@ -104,20 +141,24 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  if (!KV4_SMEM_OK(bar, 8, 8, 1)) return;
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  if (!KV4_SMEM_OK(bar, 8, 8, 2)) return;
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  if (!KV4_SMEM_OK(bar, 8, 8, 3)) return;
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
                "r"(bytes)
                : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  if (!KV4_SMEM_OK(bar, 8, 8, 4)) return true;
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
@@ -153,6 +194,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 
 // 1-D bulk copy global -> shared (no multicast), completion on an mbarrier.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  if (!KV4_SMEM_OK(dst, bytes, 16, 5) || !KV4_SMEM_OK(bar, 8, 8, 6)) return;
+#ifdef KV4_DEBUG_CHECKS
+  if ((reinterpret_cast<uintptr_t>(src) & 15) || (bytes & 15)) {
+    dbg_fail(7, reinterpret_cast<uintptr_t>(src), bytes);
+    return;
+  }
+#endif
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar)
@@ -169,12 +217,14 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
+  if (!KV4_SMEM_OK(addr, 16, 16, 8)) return make_uint4(0, 0, 0, 0);
   asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
 }
 
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
+  if (!KV4_SMEM_OK(addr, 8, 8, 9)) return make_uint2(0, 0);
   asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
@@ -276,6 +326,7 @@ struct kv4_cache {
   size_t pool_bytes;         // per layer
   size_t prot_bytes;         // per layer (INT4 cache only)
   int attn_blocks_per_sm;
+  int attn_ring;             // ring depth chosen for the attention kernel
   cudaEvent_t ev_before;     // optional timing events around the split-K kernel
   cudaEvent_t ev_after;
 };

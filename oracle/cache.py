@@ -51,17 +51,6 @@ def is_protected(p, L, S, W):
     return p < S or p >= L - W
 
 
-def _write_half2(buf, off, s16, z16):
-    buf[off:off + 2] = np.frombuffer(np.float16(s16).tobytes(), np.uint8)
-    buf[off + 2:off + 4] = np.frombuffer(np.float16(z16).tobytes(), np.uint8)
-
-
-def _read_half2(buf, off):
-    s = np.frombuffer(buf[off:off + 2].tobytes(), np.float16)[0]
-    z = np.frombuffer(buf[off + 2:off + 4].tobytes(), np.float16)[0]
-    return s, z
-
-
 class OracleKV4Cache:
     """The cache state: per-layer INT4 pages, per-(layer, seq) INT8 store, sequence lengths.
 
@@ -92,70 +81,118 @@ class OracleKV4Cache:
         self.t8 = tables("int8", self.D)
 
     # -- storage helpers -------------------------------------------------
-    def _page_tile(self, layer, seq, p):
-        page = int(self.block_table[seq, p // self.P])
-        if page < 0 or page >= self.cfg["num_pages"]:
-            raise ValueError("block table entry %d for seq %d page %d is unmapped" % (page, seq, p // self.P))
+    def _page_tiles(self, layer, page):
         key = (layer, page)
         if key not in self.pages:
             self.pages[key] = np.zeros((self.Hkv, self.P // TILE, int4_tile_bytes(self.D)), np.uint8)
-        return self.pages[key][:, (p % self.P) // TILE, :], p % TILE
+        return self.pages[key]
 
-    def _prot_tile(self, layer, seq, slot):
+    def _prot_tiles(self, layer, seq):
         key = (layer, seq)
         if key not in self.prot:
             self.prot[key] = np.zeros((self.Hkv, n_prot_tiles(self.S, self.W), int8_tile_bytes(self.D)), np.uint8)
-        return self.prot[key][:, slot // TILE, :], slot % TILE
+        return self.prot[key]
 
-    def _put_int4(self, tiles_h, r, codes, s16, z16, tensor):
-        """tiles_h: [Hkv, tile bytes] view; codes [Hkv, D]; s16/z16 [Hkv]."""
-        D = self.D
-        base = 0 if tensor == 0 else 8 * D
-        if tensor == 0:
-            byte, lo, hi = self.t4.k_byte[r], self.t4.k_lo[r], self.t4.k_hi[r]
-        else:
-            byte, lo, hi = self.t4.v_byte[r], self.t4.v_lo[r], self.t4.v_hi[r]
-        tiles_h[:, base + byte] = codes[:, lo] | (codes[:, hi] << 4)
-        off = 16 * D + scale_offset(r, tensor)
+    def _pages_of(self, seq, pos):
+        """Physical page of every position (raises on an unmapped entry)."""
+        page = self.block_table[seq, pos // self.P]
+        if np.any((page < 0) | (page >= self.cfg["num_pages"])):
+            raise ValueError("block table entry of sequence %d is unmapped" % seq)
+        return page
+
+    @staticmethod
+    def _sz_bytes(s16, z16):
+        """[m, Hkv] fp16 scale / zero -> [m, Hkv, 4] bytes (s low, s high, z low, z high)."""
+        sb = np.ascontiguousarray(s16, np.float16).view(np.uint8).reshape(s16.shape + (2,))
+        zb = np.ascontiguousarray(z16, np.float16).view(np.uint8).reshape(z16.shape + (2,))
+        return np.concatenate([sb, zb], axis=-1)
+
+    @staticmethod
+    def _sz_values(b):
+        """[..., 4] bytes -> (s16, z16)."""
+        b = np.ascontiguousarray(b)
+        s16 = b[..., 0:2].copy().view(np.float16)[..., 0]
+        z16 = b[..., 2:4].copy().view(np.float16)[..., 0]
+        return s16, z16
+
+    def _scatter(self, tiles, ti, byte_idx, vals):
+        """tiles [Hkv, T, bytes]; ti [m]; byte_idx [m, k]; vals [m, Hkv, k] -> tiles[h, ti_j, byte_idx_j] = vals[j, h]."""
         for h in range(self.Hkv):
-            _write_half2(tiles_h[h], off, s16[h], z16[h])
+            tiles[h][ti[:, None], byte_idx] = vals[:, h, :]
 
-    def _put_int8(self, tiles_h, r, codes, s16, z16, tensor):
-        D = self.D
-        base = 0 if tensor == 0 else 16 * D
-        byte = self.t8.k_byte[r] if tensor == 0 else self.t8.v_byte[r]
-        tiles_h[:, base + byte] = codes
-        off = 32 * D + scale_offset(r, tensor)
-        for h in range(self.Hkv):
-            _write_half2(tiles_h[h], off, s16[h], z16[h])
+    def _gather(self, tiles, ti, byte_idx):
+        """Inverse of _scatter: returns [m, Hkv, k]."""
+        return np.stack([tiles[h][ti[:, None], byte_idx] for h in range(self.Hkv)], axis=1)
 
-    def _get_int4(self, tiles_h, r, tensor):
-        D = self.D
-        base = 0 if tensor == 0 else 8 * D
-        if tensor == 0:
-            byte, lo, hi = self.t4.k_byte[r], self.t4.k_lo[r], self.t4.k_hi[r]
-        else:
-            byte, lo, hi = self.t4.v_byte[r], self.t4.v_lo[r], self.t4.v_hi[r]
-        b = tiles_h[:, base + byte]
-        codes = np.zeros((self.Hkv, D), np.uint8)
-        codes[:, lo] = b & 15
-        codes[:, hi] = b >> 4
-        off = 16 * D + scale_offset(r, tensor)
-        sz = [_read_half2(tiles_h[h], off) for h in range(self.Hkv)]
-        s16 = np.array([a for a, _ in sz], np.float16)
-        z16 = np.array([b_ for _, b_ in sz], np.float16)
-        return codes, s16, z16
+    def _write_int4(self, layer, seq, pos, enc_k, enc_v):
+        """INT4 codes and scales of positions `pos` (enc_*: codes [m, Hkv, D], s16, z16 [m, Hkv])."""
+        D, t4 = self.D, self.t4
+        page = self._pages_of(seq, pos)
+        r = pos % TILE
+        ti = (pos % self.P) // TILE
+        for pg in np.unique(page):
+            sel = page == pg
+            tiles = self._page_tiles(layer, int(pg))
+            rs, ts = r[sel], ti[sel]
+            for tensor, (codes, s16, z16) in enumerate((enc_k, enc_v)):
+                if tensor == 0:
+                    byte, lo, hi, base = t4.k_byte[rs], t4.k_lo[rs], t4.k_hi[rs], 0
+                else:
+                    byte, lo, hi, base = t4.v_byte[rs], t4.v_lo[rs], t4.v_hi[rs], 8 * D
+                c = codes[sel]                                            # [m, Hkv, D]
+                lo_c = np.take_along_axis(c, lo[:, None, :], axis=2)      # low-nibble dims of each byte
+                hi_c = np.take_along_axis(c, hi[:, None, :], axis=2)
+                self._scatter(tiles, ts, base + byte, lo_c | (hi_c << 4))
+                off = 16 * D + np.array([scale_offset(int(x), tensor) for x in rs])
+                self._scatter(tiles, ts, off[:, None] + np.arange(4), self._sz_bytes(s16[sel], z16[sel]))
 
-    def _get_int8(self, tiles_h, r, tensor):
-        D = self.D
-        base = 0 if tensor == 0 else 16 * D
-        byte = self.t8.k_byte[r] if tensor == 0 else self.t8.v_byte[r]
-        codes = tiles_h[:, base + byte].astype(np.uint8)
-        off = 32 * D + scale_offset(r, tensor)
-        sz = [_read_half2(tiles_h[h], off) for h in range(self.Hkv)]
-        s16 = np.array([a for a, _ in sz], np.float16)
-        z16 = np.array([b_ for _, b_ in sz], np.float16)
-        return codes, s16, z16
+    def _write_int8(self, layer, seq, slots, enc_k, enc_v):
+        D, t8 = self.D, self.t8
+        tiles = self._prot_tiles(layer, seq)
+        r, ti = slots % TILE, slots // TILE
+        for tensor, (codes, s16, z16) in enumerate((enc_k, enc_v)):
+            byte = (t8.k_byte if tensor == 0 else 16 * D + t8.v_byte)[r]     # [m, D]: byte of each dim
+            self._scatter(tiles, ti, byte, codes)
+            off = 32 * D + np.array([scale_offset(int(x), tensor) for x in r])
+            self._scatter(tiles, ti, off[:, None] + np.arange(4), self._sz_bytes(s16, z16))
+
+    def _read_int4(self, layer, seq, pos):
+        """Dequantized K^, V^ [m, Hkv, D] of positions `pos` from the pages."""
+        D, t4 = self.D, self.t4
+        page = self._pages_of(seq, pos)
+        r = pos % TILE
+        ti = (pos % self.P) // TILE
+        out = [np.zeros((len(pos), self.Hkv, D), np.float32) for _ in range(2)]
+        for pg in np.unique(page):
+            sel = np.nonzero(page == pg)[0]
+            tiles = self._page_tiles(layer, int(pg))
+            rs, ts = r[sel], ti[sel]
+            for tensor in (0, 1):
+                if tensor == 0:
+                    byte, lo, hi, base = t4.k_byte[rs], t4.k_lo[rs], t4.k_hi[rs], 0
+                else:
+                    byte, lo, hi, base = t4.v_byte[rs], t4.v_lo[rs], t4.v_hi[rs], 8 * D
+                b = self._gather(tiles, ts, base + byte)                      # [m, Hkv, D/2]
+                codes = np.zeros((len(sel), self.Hkv, D), np.uint8)
+                np.put_along_axis(codes, lo[:, None, :], b & 15, axis=2)
+                np.put_along_axis(codes, hi[:, None, :], b >> 4, axis=2)
+                off = 16 * D + np.array([scale_offset(int(x), tensor) for x in rs])
+                s16, z16 = self._sz_values(self._gather(tiles, ts, off[:, None] + np.arange(4)))
+                out[tensor][sel] = dequantize_groups(codes, s16, z16)
+        return out
+
+    def _read_int8(self, layer, seq, slots):
+        D, t8 = self.D, self.t8
+        tiles = self._prot_tiles(layer, seq)
+        r, ti = slots % TILE, slots // TILE
+        out = []
+        for tensor in (0, 1):
+            byte = (t8.k_byte if tensor == 0 else 16 * D + t8.v_byte)[r]
+            codes = self._gather(tiles, ti, byte)
+            off = 32 * D + np.array([scale_offset(int(x), tensor) for x in r])
+            s16, z16 = self._sz_values(self._gather(tiles, ti, off[:, None] + np.arange(4)))
+            out.append(dequantize_groups(codes, s16, z16))
+        return out
 
     # -- the method --------------------------------------------------------
     def rotate_quantize(self, x):
@@ -180,18 +217,15 @@ class OracleKV4Cache:
             L_new = L_old + n
             if L_new > cap:
                 raise ValueError("sequence %d would exceed its capacity of %d tokens" % (seq, cap))
-            enc = [self.rotate_quantize(k_new[a:b]), self.rotate_quantize(v_new[a:b])]
-            for j in range(n):
-                p = L_old + j
-                tiles_h, r = self._page_tile(layer, seq, p)
-                for tensor in (0, 1):
-                    _, (c4, s4, z4), _ = enc[tensor]
-                    self._put_int4(tiles_h, r, c4[j], s4[j], z4[j], tensor)
-                if p < self.S or p >= L_new - self.W:
-                    ptiles, r8 = self._prot_tile(layer, seq, prot_slot(p, self.S, self.W))
-                    for tensor in (0, 1):
-                        _, _, (c8, s8, z8) = enc[tensor]
-                        self._put_int8(ptiles, r8, c8[j], s8[j], z8[j], tensor)
+            _, k4, k8 = self.rotate_quantize(k_new[a:b])
+            _, v4, v8 = self.rotate_quantize(v_new[a:b])
+            pos = L_old + np.arange(n)
+            self._write_int4(layer, seq, pos, k4, v4)           # every position: INT4 page copy
+            prot = (pos < self.S) | (pos >= L_new - self.W)      # sinks, and the last W of this append
+            if np.any(prot):
+                j = np.nonzero(prot)[0]
+                slots = np.array([prot_slot(int(p), self.S, self.W) for p in pos[j]])
+                self._write_int8(layer, seq, slots, tuple(x[j] for x in k8), tuple(x[j] for x in v8))
             self.seq_lens[layer, seq] = L_new
 
     def view(self, layer, seq, protected=True, start=0, count=None):
@@ -206,18 +240,19 @@ class OracleKV4Cache:
         if start < 0 or start + count > L:
             raise ValueError("range outside the sequence")
         out = [np.zeros((count, self.Hkv, self.D), np.float32) for _ in range(2)]
-        for j in range(count):
-            p = start + j
-            if protected and is_protected(p, L, self.S, self.W):
-                tiles_h, r = self._prot_tile(layer, seq, prot_slot(p, self.S, self.W))
-                for tensor in (0, 1):
-                    c, s, z = self._get_int8(tiles_h, r, tensor)
-                    out[tensor][j] = dequantize_groups(c, s, z)
+        if count == 0:
+            return out[0], out[1]
+        pos = start + np.arange(count)
+        from_int8 = np.array([protected and is_protected(int(p), L, self.S, self.W) for p in pos])
+        for src, sel in ((False, ~from_int8), (True, from_int8)):
+            if not np.any(sel):
+                continue
+            if src:
+                slots = np.array([prot_slot(int(p), self.S, self.W) for p in pos[sel]])
+                kv = self._read_int8(layer, seq, slots)
             else:
-                tiles_h, r = self._page_tile(layer, seq, p)
-                for tensor in (0, 1):
-                    c, s, z = self._get_int4(tiles_h, r, tensor)
-                    out[tensor][j] = dequantize_groups(c, s, z)
+                kv = self._read_int4(layer, seq, pos[sel])
+            out[0][sel], out[1][sel] = kv
         return out[0], out[1]
 
 
