@@ -125,9 +125,11 @@ int kv4_cache_create(const kv4_config* cfg, void* dev_buf, size_t bytes, int32_t
 int kv4_cache_destroy(kv4_cache* cache);
 
 /* Device addresses inside the cache buffer for layer `layer` (any pointer may
- * be NULL): the INT4 page pool, uint8 [num_pages][Hkv][P/16][16*D+128]; the
- * INT8 store, uint8 [max_seqs][Hkv][ceil((S+W)/16)][32*D+128]; and the
- * sequence lengths int32 [num_layers][max_seqs] (all layers). */
+ * be NULL): the INT4 page pool, uint8 [num_pages][P/16][Hkv][16*D+128]; the
+ * INT8 store, uint8 [max_seqs][ceil((S+W)/16)][Hkv][32*D+128]; and the
+ * sequence lengths int32 [num_layers][max_seqs] (all layers).  KV heads are
+ * innermost, so the 16-token tiles of all heads at one page position are
+ * contiguous (one bulk copy feeds eight heads). */
 int kv4_cache_layout(const kv4_cache* cache, int32_t layer, void** dev_pages, void** dev_protected,
                      int32_t** dev_seq_lens);
 
@@ -207,7 +209,7 @@ const char* kv4_version(void);
  * merge, with bf16 keys/values stored as they arrive (no rotation, no
  * quantization, no protected store).  It exists to measure what the INT4
  * format saves; hadamard_block, sink_tokens and recent_window are ignored.
- * Page pool: bf16 [num_pages][Hkv][P/16][16-token tile of 32*D elements].
+ * Page pool: bf16 [num_pages][P/16][Hkv][16-token tile of 32*D elements].
  */
 typedef struct kv4bf16_cache kv4bf16_cache;
 

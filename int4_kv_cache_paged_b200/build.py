@@ -10,7 +10,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = ["kv4_api.cu", "kv4_append.cu", "kv4_attention.cu"]
+SOURCES = ["kv4_api.cu", "kv4_append.cu", "kv4_attention.cu", "kv4_attention_grouped.cu"]
 LIB = os.path.join(HERE, "libkv4.so")
 OBJDIR = os.path.join(ROOT, "_build")
 
@@ -34,7 +34,8 @@ def build(verbose_ptxas=False, force=False):
     """Compile every source to an object in _build/ and link libkv4.so next to this file."""
     os.makedirs(OBJDIR, exist_ok=True)
     objs = []
-    headers = [os.path.join(HERE, "csrc", "kv4_common.cuh"), os.path.join(ROOT, "include", "kv4.h")]
+    headers = [os.path.join(HERE, "csrc", h) for h in ("kv4_common.cuh", "kv4_attn_tiles.cuh")] + \
+        [os.path.join(ROOT, "include", "kv4.h")]
     newest_header = max(os.path.getmtime(h) for h in headers)
     for src in SOURCES:
         path = os.path.join(HERE, "csrc", src)

@@ -72,7 +72,7 @@ class KV4Cache(_Base):
     def pages(self, layer):
         c = self.cfg
         ptr, _, _ = kv4_cache_layout(self.handle, layer)
-        shape = (c["num_pages"], c["num_kv_heads"], c["page_size"] // TILE, _tile4(c["head_dim"]))
+        shape = (c["num_pages"], c["page_size"] // TILE, c["num_kv_heads"], _tile4(c["head_dim"]))
         n = shape[0] * shape[1] * shape[2] * shape[3]
         return self._view(ptr, n, shape)
 
@@ -80,7 +80,7 @@ class KV4Cache(_Base):
         c = self.cfg
         _, ptr, _ = kv4_cache_layout(self.handle, layer)
         npt = -(-(c["sink_tokens"] + c["recent_window"]) // TILE)
-        shape = (c["max_seqs"], c["num_kv_heads"], npt, _tile8(c["head_dim"]))
+        shape = (c["max_seqs"], npt, c["num_kv_heads"], _tile8(c["head_dim"]))
         n = shape[0] * shape[1] * shape[2] * shape[3]
         return self._view(ptr, n, shape)
 
@@ -137,7 +137,7 @@ class BF16Cache(_Base):
     def pages(self, layer):
         c = self.cfg
         ptr, _ = kv4bf16_cache_layout(self.handle, layer)
-        shape = (c["num_pages"], c["num_kv_heads"], c["page_size"] // TILE, _tile16(c["head_dim"]))
+        shape = (c["num_pages"], c["page_size"] // TILE, c["num_kv_heads"], _tile16(c["head_dim"]))
         n = shape[0] * shape[1] * shape[2] * shape[3]
         return self._view(ptr, n, shape)
 

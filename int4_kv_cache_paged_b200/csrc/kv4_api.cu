@@ -95,6 +95,14 @@ int create(const kv4_config* cfg, bool bf16, void* dev_buf, size_t bytes, int32_
     delete c;
     return KV4_ERR_CUDA;
   }
+  c->gattn_ring = 0;
+  if (kv4::grouped_path(c)) {
+    c->gattn_ring = kv4::grouped_ring(c);
+    if (c->gattn_ring <= 0) {
+      delete c;
+      return KV4_ERR_CUDA;
+    }
+  }
   if (cudaMemsetAsync(c->base, 0, kv4::STATE_BYTES + s.seq_lens, stream) != cudaSuccess) {
     delete c;
     return KV4_ERR_CUDA;

@@ -230,7 +230,8 @@ __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams 
         raw[0] = u & 0xFFFF; raw[1] = u >> 16;
       }
       const int r = pos & (TILE - 1);
-      const long long tile_idx = (static_cast<long long>(page) * p.Hkv + h) * (p.P / TILE) + (pos % p.P) / TILE;
+      // head-innermost pool: [page][P/16][Hkv][tile]
+      const long long tile_idx = (static_cast<long long>(page) * (p.P / TILE) + (pos % p.P) / TILE) * p.Hkv + h;
       if constexpr (BF16) {
         uint16_t* tile = reinterpret_cast<uint16_t*>(p.pool + tile_idx * tile16_bytes(D));
         // share the row through smem so each lane can store element pairs
@@ -286,7 +287,7 @@ __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams 
         if (protect) {
           const int slot = pos < p.S ? pos : p.S + (pos - p.S) % p.W;
           const int npt = n_prot_tiles(p.S, p.W);
-          uint8_t* t8 = p.prot + ((static_cast<long long>(seq) * p.Hkv + h) * npt + slot / TILE) * tile8_bytes(D);
+          uint8_t* t8 = p.prot + ((static_cast<long long>(seq) * npt + slot / TILE) * p.Hkv + h) * tile8_bytes(D);
           store_int8(t8, slot & (TILE - 1), tensor, c8, sz8, D, lane);
         }
       }
@@ -324,7 +325,7 @@ __global__ void dequant_kernel(DequantParams p) {
   if (protect) {
     const int slot = pos < p.S ? pos : p.S + (pos - p.S) % p.W;
     const int r = slot & 15, rowhi = r >> 3, g = r & 7;
-    const uint8_t* tile = p.prot + ((static_cast<long long>(p.seq) * p.Hkv + h) * n_prot_tiles(p.S, p.W) + slot / 16) *
+    const uint8_t* tile = p.prot + ((static_cast<long long>(p.seq) * n_prot_tiles(p.S, p.W) + slot / 16) * p.Hkv + h) *
                                        tile8_bytes(D);
     const uint32_t sz = *reinterpret_cast<const uint32_t*>(tile + 32 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3)));
     const float s = half_lo(sz), z = half_hi(sz);
@@ -347,7 +348,7 @@ __global__ void dequant_kernel(DequantParams p) {
       return;
     }
     const int r = pos & 15;
-    const uint8_t* tile = p.pool + ((static_cast<long long>(page) * p.Hkv + h) * (p.P / 16) + (pos % p.P) / 16) *
+    const uint8_t* tile = p.pool + ((static_cast<long long>(page) * (p.P / 16) + (pos % p.P) / 16) * p.Hkv + h) *
                                        tile4_bytes(D);
     const uint32_t sz = *reinterpret_cast<const uint32_t*>(tile + 16 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3)));
     const float s = half_lo(sz), z = half_hi(sz);

@@ -28,7 +28,7 @@
 //           query head, and the 7 warps merge into one partial (m, l, o) per item.
 //   merge   one warp per (sequence, query head): log-sum-exp merge of the item
 //           partials, inverse Hadamard rotation, store.
-#include "kv4_common.cuh"
+#include "kv4_attn_tiles.cuh"
 
 #include <math.h>
 
@@ -37,11 +37,12 @@ namespace kv4 {
 
 namespace {
 
+using namespace tiles;
+
 constexpr int NW = 7;                  // consumer warps (+1 producer: 16 warps per SM at 2 CTAs)
 constexpr int THREADS = 32 * (NW + 1); // + producer warp
 constexpr int QD = 2;                  // item queue depth
 constexpr int PREP_WARPS = 4;
-constexpr float NEG_INF = -INFINITY;
 
 // Ring of shared-memory stages filled by the producer.  Stage s is always
 // consumed by warp s % NW: global tile j goes to stage j % ns and warp j % NW,
@@ -59,10 +60,6 @@ struct KCfg {
 };
 constexpr int NS_CHOICES[4] = {4 * NW, 3 * NW, 2 * NW, NW};
 
-// Partial of one item: per query head, o[D] (unnormalised, rotated basis), m, l,
-// padded to D + 4 floats so every head row starts on a 16-byte boundary.
-__host__ __device__ constexpr int head_stride(int D) { return D + 4; }
-__host__ __device__ inline int partial_stride(int G, int D) { return G * head_stride(D); }
 
 template <int D, bool BF16>
 __host__ __device__ inline size_t attn_smem_bytes(int G, int ns) {
@@ -77,7 +74,6 @@ __host__ __device__ inline size_t attn_smem_bytes(int G, int ns) {
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(32 * PREP_WARPS) prep_kernel(AttnParams p) {
-  constexpr int VPL = D / 32;
   extern __shared__ float s_q[];  // [PREP_WARPS][G][D]
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int gw = blockIdx.x * PREP_WARPS + wib;
@@ -145,406 +141,18 @@ __global__ void __launch_bounds__(32 * PREP_WARPS) prep_kernel(AttnParams p) {
       p.items[2][base2] = it;
     }
     SeqHead sh;
-    sh.part_base = pbase; sh.n_parts = nparts; sh.len = L; sh.pad = 0;
+    sh.part_base = pbase; sh.n_parts = nparts; sh.len = L; sh.pad = 1;
     p.seqhead[gw] = sh;
   }
 
   // ---- queries: rotate (INT4 cache), round to bf16, lay out as B operands
-  float* sq = s_q + wib * G * D;
-  float qsum[MAX_G];
-  float amax = 0.f;
-  const float rot_c = p.rot_c;
-  for (int g = 0; g < G; ++g) {
-    const uint16_t* src = p.q + (static_cast<long long>(b) * p.Hq + h * G + g) * D;
-    float x[VPL];
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) x[i] = __bfloat162float(__ushort_as_bfloat16(src[VPL * lane + i]));
-    if constexpr (!BF16) {
-      for (int hh = 1; hh < p.Bh; hh <<= 1) {
-        if (hh < VPL) {
-#pragma unroll
-          for (int i = 0; i < VPL; ++i)
-            if ((i & hh) == 0) {
-              const float a = x[i], c = x[i + hh];
-              x[i] = __fadd_rn(a, c);
-              x[i + hh] = __fsub_rn(a, c);
-            }
-        } else {
-          const int lm = hh / VPL;
-          const bool upper = (lane & lm) != 0;
-#pragma unroll
-          for (int i = 0; i < VPL; ++i) {
-            const float o = __shfl_xor_sync(0xffffffffu, x[i], lm);
-            x[i] = upper ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
-          }
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) x[i] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(x[i], rot_c)));
-    }
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      sq[g * D + VPL * lane + i] = x[i];
-      s += x[i];
-      amax = fmaxf(amax, fabsf(x[i]));
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    qsum[g] = s;
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  __syncwarp();
-  // fp16 operands: q * 2^e with max|q| * 2^e in [2^14, 2^15) (exact for normal values)
-  int e = 0;
-  if (!BF16 && amax > 0.f && amax <= 3.0e38f) {
-    int ex;
-    frexpf(amax, &ex);
-    e = 15 - ex;
-  }
-  uint32_t* blob = reinterpret_cast<uint32_t*>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D));
-  const int g = lane >> 2, t = lane & 3;
-  // B-operand column n holds query head n % G when the column split applies
-  // (G = 1, 2, 4: the spare columns carry the low part of the P.V weights),
-  // otherwise head n for n < G and zeros.
-  const bool colsplit = (G == 1 || G == 2 || G == 4);
-  const int gsrc = colsplit ? g % G : g;
-  for (int c = 0; c < D / 32; ++c) {
-    uint32_t r[4];
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-      const int k = 2 * c + kk;
-#pragma unroll
-      for (int reg = 0; reg < 2; ++reg) {
-        const int d = 16 * k + 2 * t + 8 * reg;
-        float a = 0.f, bb = 0.f;
-        if (gsrc < G) { a = sq[gsrc * D + d]; bb = sq[gsrc * D + d + 1]; }
-        if constexpr (BF16) {
-          r[2 * kk + reg] = pack_bf162(a, bb);
-        } else {
-          r[2 * kk + reg] = pack_half2(ldexpf(a, e), ldexpf(bb, e));
-        }
-      }
-    }
-    reinterpret_cast<uint4*>(blob)[c * 32 + lane] = make_uint4(r[0], r[1], r[2], r[3]);
-  }
-  float* tail = reinterpret_cast<float*>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D) + 16 * D);
-  if (lane < MAX_G) {
-    const int src = colsplit ? lane % G : lane;
-    float v = 0.f;
-#pragma unroll
-    for (int gg = 0; gg < MAX_G; ++gg)
-      if (gg == src && gg < G) v = qsum[gg];
-    tail[lane] = BF16 ? 0.f : v * p.scale_log2;
-  }
-  if (lane == MAX_G) tail[MAX_G] = ldexpf(p.scale_log2, -e);
-}
-
-// ---------------------------------------------------------------------------
-// attention: per-warp online-softmax state
-
-template <int D>
-struct WarpState {
-  float o[D / 16][4];  // o^T fragments: (dim 16m+g, head 2t), (16m+g, 2t+1), (16m+g+8, 2t), (16m+g+8, 2t+1)
-  float m0, m1, l0, l1, z0, z1;
-};
-
-// Column split of the P.V weights (see pv_operands): part of each of the thread's two columns.
-struct ColSplit {
-  bool colsplit;
-  int part0, part1;
-};
-
-template <int D>
-struct QFrag {
-  uint32_t b[D / 16][2];
-  float qs0, qs1, kscale;
-};
-
-template <int D>
-__device__ __forceinline__ void online_softmax_pv(WarpState<D>& ws, float x0, float x1, float x2, float x3,
-                                                  float& p0, float& p1, float& p2, float& p3) {
-  float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-  }
-  const float n0 = fmaxf(ws.m0, mx0), n1 = fmaxf(ws.m1, mx1);
-  if (__any_sync(0xffffffffu, n0 > ws.m0 || n1 > ws.m1)) {
-    const float a0 = ex2(ws.m0 - n0), a1 = ex2(ws.m1 - n1);
-    ws.l0 *= a0; ws.l1 *= a1; ws.z0 *= a0; ws.z1 *= a1;
-#pragma unroll
-    for (int m = 0; m < D / 16; ++m) {
-      ws.o[m][0] *= a0; ws.o[m][1] *= a1; ws.o[m][2] *= a0; ws.o[m][3] *= a1;
-    }
-    ws.m0 = n0; ws.m1 = n1;
-  }
-  p0 = ex2(x0 - ws.m0); p1 = ex2(x1 - ws.m1); p2 = ex2(x2 - ws.m0); p3 = ex2(x3 - ws.m1);
-}
-
-
-// P.V weights of this thread's two columns (c0 = 2t, c1 = 2t+1) for tokens g and
-// g+8.  With the column split (G = 1, 2, 4), column c carries part c / G of the
-// weight of head c % G: part 0 = hi = fp16(P), part 1 = lo = fp16(P - hi),
-// parts >= 2 are zero; one 16x8x16 multiply then accumulates both parts.
-// Without it (other G) the hi parts go to (B0, B1) and the lo parts to (C0, C1).
-__device__ __forceinline__ void pv_operands(float P0, float P1, float P2, float P3, int part0, int part1,
-                                            bool colsplit, uint32_t& B0, uint32_t& B1, uint32_t& C0, uint32_t& C1) {
-  const uint32_t h01 = pack_half2(P0, P1), h23 = pack_half2(P2, P3);
-  const uint32_t l01 = pack_half2(P0 - half_lo(h01), P1 - half_hi(h01));
-  const uint32_t l23 = pack_half2(P2 - half_lo(h23), P3 - half_hi(h23));
-  if (colsplit) {
-    const uint32_t m0 = part0 == 0 ? 0x0000FFFFu : 0u, m1 = part1 == 0 ? 0xFFFF0000u : 0u;
-    const uint32_t n0 = part0 == 1 ? 0x0000FFFFu : 0u, n1 = part1 == 1 ? 0xFFFF0000u : 0u;
-    B0 = movmatrix_trans((h01 & (m0 | m1)) | (l01 & (n0 | n1)));
-    B1 = movmatrix_trans((h23 & (m0 | m1)) | (l23 & (n0 | n1)));
-    C0 = C1 = 0u;
-  } else {
-    B0 = movmatrix_trans(h01);
-    B1 = movmatrix_trans(h23);
-    C0 = movmatrix_trans(l01);
-    C1 = movmatrix_trans(l23);
-  }
-}
-
-// QK^T of one INT4 tile: acc = (q * 2^e) . codes for tokens g, g+8 and heads 2t, 2t+1.
-template <int D>
-__device__ __forceinline__ void qk_int4(uint32_t st, const QFrag<D>& qf, int lane, float (&acc)[4]) {
-  constexpr int NKK = D / 32;
-  uint32_t kw0[NKK], kw1[NKK];
-  if constexpr (D == 128) {
-    const uint4 a = lds128(st + lane * 16), bq = lds128(st + 512 + lane * 16);
-    kw0[0] = a.x; kw0[1] = a.y; kw0[2] = a.z; kw0[3] = a.w;
-    kw1[0] = bq.x; kw1[1] = bq.y; kw1[2] = bq.z; kw1[3] = bq.w;
-  } else {
-    const uint2 a = lds64(st + lane * 8), bq = lds64(st + 256 + lane * 8);
-    kw0[0] = a.x; kw0[1] = a.y; kw1[0] = bq.x; kw1[1] = bq.y;
-  }
-  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < NKK; ++kk) {
-    const uint32_t w0 = kw0[kk], w1 = kw1[kk];
-    mma_f16(acc, nib_lo(w0), nib_lo(w1), nib_hi(w0), nib_hi(w1), qf.b[2 * kk][0], qf.b[2 * kk][1]);
-    const uint32_t u0 = w0 >> 8, u1 = w1 >> 8;
-    mma_f16(acc, nib_lo(u0), nib_lo(u1), nib_hi(u0), nib_hi(u1), qf.b[2 * kk + 1][0], qf.b[2 * kk + 1][1]);
-  }
-}
-
-// P.V of one INT4 tile: o^T[m] += V^T codes * (hi + lo) weights.
-template <int D>
-__device__ __forceinline__ void pv_int4(uint32_t st, WarpState<D>& ws, int lane, uint32_t B0, uint32_t B1,
-                                        uint32_t C0, uint32_t C1, bool colsplit) {
-  uint32_t vw[D / 16];
-  if constexpr (D == 128) {
-    const uint4 v0 = lds128(st + 8 * D + lane * 16), v1 = lds128(st + 8 * D + 512 + lane * 16);
-    vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
-    vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
-  } else {
-    const uint4 v0 = lds128(st + 8 * D + lane * 16);
-    vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
-  }
-#pragma unroll
-  for (int m = 0; m < D / 16; ++m) {
-    const uint32_t w = vw[m], u = w >> 8;
-    const uint32_t a0 = nib_lo(w), a1 = nib_hi(w), a2 = nib_lo(u), a3 = nib_hi(u);
-    mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
-    if (!colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
-  }
-}
-
-// One unit of NT (1 or 2) INT4 tiles at st, st + tile4_bytes(D): scores, one
-// online-softmax update for the NT*16 tokens, P.V.  valid[u] bit 0 / bit 1:
-// token g / g+8 of tile u is inside the item's range (used when MASKED).  The
-// stage is handed back after its last shared-memory load.
-template <int D, int NT, bool MASKED>
-__device__ __forceinline__ void unit_int4(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane,
-                                          const int (&valid)[2], uint32_t empty_bar, const ColSplit& cs) {
-  constexpr int TB = tile4_bytes(D);
-  float x[NT][4];
-  uint4 sz[NT];
-#pragma unroll
-  for (int u = 0; u < NT; ++u) {
-    float acc[4];
-    qk_int4<D>(st + u * TB, qf, lane, acc);
-    sz[u] = lds128(st + u * TB + 16 * D + (lane >> 2) * 16);
-    const float sKg = half_lo(sz[u].x) * qf.kscale, zKg = half_hi(sz[u].x);
-    const float sKg8 = half_lo(sz[u].y) * qf.kscale, zKg8 = half_hi(sz[u].y);
-    x[u][0] = fmaf(acc[0], sKg, zKg * qf.qs0);
-    x[u][1] = fmaf(acc[1], sKg, zKg * qf.qs1);
-    x[u][2] = fmaf(acc[2], sKg8, zKg8 * qf.qs0);
-    x[u][3] = fmaf(acc[3], sKg8, zKg8 * qf.qs1);
-    if constexpr (MASKED) {
-      if (!(valid[u] & 1)) { x[u][0] = NEG_INF; x[u][1] = NEG_INF; }
-      if (!(valid[u] & 2)) { x[u][2] = NEG_INF; x[u][3] = NEG_INF; }
-    }
-  }
-  // online softmax over the unit: max over tokens g, g+8 of every tile, then over the 8 row groups
-  float mx0 = fmaxf(x[0][0], x[0][2]), mx1 = fmaxf(x[0][1], x[0][3]);
-#pragma unroll
-  for (int u = 1; u < NT; ++u) {
-    mx0 = fmaxf(mx0, fmaxf(x[u][0], x[u][2]));
-    mx1 = fmaxf(mx1, fmaxf(x[u][1], x[u][3]));
-  }
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-  }
-  const float n0 = fmaxf(ws.m0, mx0), n1 = fmaxf(ws.m1, mx1);
-  if (__any_sync(0xffffffffu, n0 > ws.m0 || n1 > ws.m1)) {
-    const float a0 = ex2(ws.m0 - n0), a1 = ex2(ws.m1 - n1);
-    ws.l0 *= a0; ws.l1 *= a1; ws.z0 *= a0; ws.z1 *= a1;
-#pragma unroll
-    for (int m = 0; m < D / 16; ++m) {
-      ws.o[m][0] *= a0; ws.o[m][1] *= a1; ws.o[m][2] *= a0; ws.o[m][3] *= a1;
-    }
-    ws.m0 = n0; ws.m1 = n1;
-  }
-#pragma unroll
-  for (int u = 0; u < NT; ++u) {
-    const float p0 = ex2(x[u][0] - ws.m0), p1 = ex2(x[u][1] - ws.m1);
-    const float p2 = ex2(x[u][2] - ws.m0), p3 = ex2(x[u][3] - ws.m1);
-    const float sVg = half_lo(sz[u].z), zVg = half_hi(sz[u].z), sVg8 = half_lo(sz[u].w), zVg8 = half_hi(sz[u].w);
-    float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
-    float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
-    if constexpr (MASKED) {   // unwritten slots may hold non-finite scales
-      if (!(valid[u] & 1)) { P0 = 0.f; P1 = 0.f; zg0 = 0.f; zg1 = 0.f; }
-      if (!(valid[u] & 2)) { P2 = 0.f; P3 = 0.f; zg80 = 0.f; zg81 = 0.f; }
-    }
-    ws.l0 += p0 + p2; ws.l1 += p1 + p3;
-    ws.z0 += zg0 + zg80; ws.z1 += zg1 + zg81;
-    uint32_t B0, B1, C0, C1;
-    pv_operands(P0, P1, P2, P3, cs.part0, cs.part1, cs.colsplit, B0, B1, C0, C1);
-    if (u == NT - 1) {
-      // last tile: load its V codes, then hand the stage back before the math
-      const uint32_t t = st + u * TB;
-      uint32_t vw[D / 16];
-      if constexpr (D == 128) {
-        const uint4 v0 = lds128(t + 8 * D + lane * 16), v1 = lds128(t + 8 * D + 512 + lane * 16);
-        vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
-        vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
-      } else {
-        const uint4 v0 = lds128(t + 8 * D + lane * 16);
-        vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty_bar);
-#pragma unroll
-      for (int m = 0; m < D / 16; ++m) {
-        const uint32_t w = vw[m], uu = w >> 8;
-        const uint32_t a0 = nib_lo(w), a1 = nib_hi(w), a2 = nib_lo(uu), a3 = nib_hi(uu);
-        mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
-        if (!cs.colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
-      }
-    } else {
-      pv_int4<D>(st + u * TB, ws, lane, B0, B1, C0, C1, cs.colsplit);
-    }
-  }
-}
-
-// One INT8 tile (protected store).
-template <int D, bool MASKED>
-__device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, bool vg,
-                                          bool vg8, uint32_t empty_bar, const ColSplit& cs) {
-  constexpr int NK = D / 16;
-  uint32_t kw[2][NK], vw[2 * NK];
-#pragma unroll
-  for (int rowhi = 0; rowhi < 2; ++rowhi)
-#pragma unroll
-    for (int kq = 0; kq < D / 64; ++kq) {
-      const uint4 a = lds128(st + 16 * (32 * (rowhi * (D / 64) + kq) + lane));
-      kw[rowhi][4 * kq] = a.x; kw[rowhi][4 * kq + 1] = a.y; kw[rowhi][4 * kq + 2] = a.z; kw[rowhi][4 * kq + 3] = a.w;
-    }
-#pragma unroll
-  for (int q4 = 0; q4 < NK / 2; ++q4) {
-    const uint4 a = lds128(st + 16 * D + 16 * (32 * q4 + lane));
-    vw[4 * q4] = a.x; vw[4 * q4 + 1] = a.y; vw[4 * q4 + 2] = a.z; vw[4 * q4 + 3] = a.w;
-  }
-  const uint4 sz = lds128(st + 32 * D + (lane >> 2) * 16);
-  __syncwarp();
-  if (lane == 0) mbar_arrive(empty_bar);
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int k = 0; k < NK; ++k) {
-    const uint32_t w0 = kw[0][k], w1 = kw[1][k];
-    mma_f16(acc, byte_lo(w0), byte_lo(w1), byte_lo(w0 >> 8), byte_lo(w1 >> 8), qf.b[k][0], qf.b[k][1]);
-  }
-  const float sKg = half_lo(sz.x) * qf.kscale, zKg = half_hi(sz.x);
-  const float sKg8 = half_lo(sz.y) * qf.kscale, zKg8 = half_hi(sz.y);
-  float x0 = fmaf(acc[0], sKg, zKg * qf.qs0);
-  float x1 = fmaf(acc[1], sKg, zKg * qf.qs1);
-  float x2 = fmaf(acc[2], sKg8, zKg8 * qf.qs0);
-  float x3 = fmaf(acc[3], sKg8, zKg8 * qf.qs1);
-  if constexpr (MASKED) {
-    if (!vg) { x0 = NEG_INF; x1 = NEG_INF; }
-    if (!vg8) { x2 = NEG_INF; x3 = NEG_INF; }
-  }
-  float p0, p1, p2, p3;
-  online_softmax_pv<D>(ws, x0, x1, x2, x3, p0, p1, p2, p3);
-  const float sVg = half_lo(sz.z), zVg = half_hi(sz.z), sVg8 = half_lo(sz.w), zVg8 = half_hi(sz.w);
-  float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
-  float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
-  if constexpr (MASKED) {
-    if (!vg) { P0 = 0.f; P1 = 0.f; zg0 = 0.f; zg1 = 0.f; }
-    if (!vg8) { P2 = 0.f; P3 = 0.f; zg80 = 0.f; zg81 = 0.f; }
-  }
-  ws.l0 += p0 + p2; ws.l1 += p1 + p3;
-  ws.z0 += zg0 + zg80; ws.z1 += zg1 + zg81;
-  uint32_t B0, B1, C0, C1;
-  pv_operands(P0, P1, P2, P3, cs.part0, cs.part1, cs.colsplit, B0, B1, C0, C1);
-#pragma unroll
-  for (int m = 0; m < NK; ++m) {
-    const uint32_t w0 = vw[2 * m], w1 = vw[2 * m + 1];
-    const uint32_t a0 = byte_lo(w0), a1 = byte_lo(w0 >> 8), a2 = byte_lo(w1), a3 = byte_lo(w1 >> 8);
-    mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
-    if (!cs.colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
-  }
-}
-
-// One BF16 tile (baseline cache).  Holds the stage until the V loads are done.
-// vmask01 / vmask89: per-thread masks of the V operand halves of tokens 2t, 2t+1
-// and 2t+8, 2t+9 (unwritten slots of a page may hold NaN bit patterns, and
-// 0 * NaN would poison the accumulator).
-template <int D, bool MASKED>
-__device__ __forceinline__ void tile_bf16(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, bool vg,
-                                          bool vg8, uint32_t empty_bar, uint32_t vmask01, uint32_t vmask89) {
-  constexpr int NK = D / 16;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int k = 0; k < NK; ++k) {
-    const uint4 a = lds128(st + 16 * (32 * k + lane));
-    mma_bf16(acc, a.x, a.y, a.z, a.w, qf.b[k][0], qf.b[k][1]);
-  }
-  uint4 v[NK];
-#pragma unroll
-  for (int m = 0; m < NK; ++m) {
-    v[m] = lds128(st + 32 * D + 16 * (32 * m + lane));
-    if constexpr (MASKED) {
-      v[m].x &= vmask01; v[m].y &= vmask01; v[m].z &= vmask89; v[m].w &= vmask89;
-    }
-  }
-  __syncwarp();
-  if (lane == 0) mbar_arrive(empty_bar);
-  float x0 = acc[0] * qf.kscale, x1 = acc[1] * qf.kscale, x2 = acc[2] * qf.kscale, x3 = acc[3] * qf.kscale;
-  if constexpr (MASKED) {
-    if (!vg) { x0 = NEG_INF; x1 = NEG_INF; }
-    if (!vg8) { x2 = NEG_INF; x3 = NEG_INF; }
-  }
-  float p0, p1, p2, p3;
-  online_softmax_pv<D>(ws, x0, x1, x2, x3, p0, p1, p2, p3);
-  ws.l0 += p0 + p2; ws.l1 += p1 + p3;
-  const uint32_t B0 = movmatrix_trans(pack_bf162(p0, p1));
-  const uint32_t B1 = movmatrix_trans(pack_bf162(p2, p3));
-#pragma unroll
-  for (int m = 0; m < NK; ++m) mma_bf16(ws.o[m], v[m].x, v[m].y, v[m].z, v[m].w, B0, B1);
+  build_qblob<D, BF16>(p, b, h, lane, s_q + wib * G * D);
 }
 
 template <int D, bool BF16>
 __device__ __forceinline__ const uint8_t* tile_source(const AttnParams& p, const Item& it, int tile) {
   if (it.kind == 1)
-    return p.prot + ((static_cast<long long>(it.seq) * p.Hkv + it.h) * n_prot_tiles(p.S, p.W) + tile) *
+    return p.prot + ((static_cast<long long>(it.seq) * n_prot_tiles(p.S, p.W) + tile) * p.Hkv + it.h) *
                         tile8_bytes(D);
   const int pos = tile * TILE;
   int page = p.block_table[static_cast<long long>(it.seq) * p.max_pages_per_seq + pos / p.P];
@@ -553,7 +161,7 @@ __device__ __forceinline__ const uint8_t* tile_source(const AttnParams& p, const
     page = 0;
   }
   constexpr int TB = BF16 ? tile16_bytes(D) : tile4_bytes(D);
-  return p.pool + ((static_cast<long long>(page) * p.Hkv + it.h) * (p.P / TILE) + (pos % p.P) / TILE) * TB;
+  return p.pool + ((static_cast<long long>(page) * (p.P / TILE) + (pos % p.P) / TILE) * p.Hkv + it.h) * TB;
 }
 
 __device__ __forceinline__ void named_barrier_consumers() {
@@ -798,12 +406,13 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(AttnParams p) {
         else tile_int8<D, true>(st, qf, ws, lane, vb & 1, vb & 2, eb, cs);
       } else {
         const int valid[2] = {valid_bits(0), valid_bits(1)};
+        const uint32_t tl[2] = {st, st + static_cast<uint32_t>(tile4_bytes(D))};
         if (nt == 2) {
-          if (inside) unit_int4<D, 2, false>(st, qf, ws, lane, valid, eb, cs);
-          else unit_int4<D, 2, true>(st, qf, ws, lane, valid, eb, cs);
+          if (inside) unit_int4<D, 2, false>(tl, qf, ws, lane, valid, eb, eb, cs);
+          else unit_int4<D, 2, true>(tl, qf, ws, lane, valid, eb, eb, cs);
         } else {
-          if (inside) unit_int4<D, 1, false>(st, qf, ws, lane, valid, eb, cs);
-          else unit_int4<D, 1, true>(st, qf, ws, lane, valid, eb, cs);
+          if (inside) unit_int4<D, 1, false>(tl, qf, ws, lane, valid, eb, eb, cs);
+          else unit_int4<D, 1, true>(tl, qf, ws, lane, valid, eb, eb, cs);
         }
       }
     }
@@ -894,13 +503,15 @@ __global__ void __launch_bounds__(256) merge_kernel(AttnParams p) {
   float o[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) o[i] = 0.f;
-  if (sh.n_parts > 0 && sh.part_base >= 0 && sh.part_base + sh.n_parts <= p.cap_parts) {
+  const int stride = sh.pad;
+  if (sh.n_parts > 0 && sh.part_base >= 0 && stride >= 1 && sh.part_base + (sh.n_parts - 1) * stride < p.cap_parts) {
     const float* base = p.partials + static_cast<size_t>(sh.part_base) * pstride + gq * head_stride(D);
+    const size_t step = static_cast<size_t>(stride) * pstride;
     float M = NEG_INF;
-    for (int j = 0; j < sh.n_parts; ++j) M = fmaxf(M, base[static_cast<size_t>(j) * pstride + D]);
+    for (int j = 0; j < sh.n_parts; ++j) M = fmaxf(M, base[j * step + D]);
     float lsum = 0.f;
     for (int j = 0; j < sh.n_parts; ++j) {
-      const float* r = base + static_cast<size_t>(j) * pstride;
+      const float* r = base + j * step;
       const float f = ex2(r[D] - M);
       lsum = fmaf(f, r[D + 1], lsum);
       if constexpr (VPL == 4) {
@@ -1016,6 +627,12 @@ int choose_ring(int device, int G, int* blocks_per_sm) {
 }
 
 template <int D, bool BF16>
+void launch_merge(const AttnParams& p, cudaStream_t stream) {
+  const int merge_warps = p.n_seqs * p.Hq;
+  merge_kernel<D, BF16><<<(merge_warps + 7) / 8, 256, 0, stream>>>(p);
+}
+
+template <int D, bool BF16>
 int launch_attention_t(kv4_cache* c, AttnParams& p, cudaStream_t stream) {
   const int blocks_per_sm = c->attn_blocks_per_sm;
   if (blocks_per_sm <= 0) return KV4_ERR_UNSUPPORTED;
@@ -1057,7 +674,42 @@ int attention_blocks_per_sm(kv4_cache* c) {
   return blocks;
 }
 
+// Fields of AttnParams shared by both attention paths.
+void fill_common(const kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, const void* q, void* out,
+                 float softmax_scale, int mode, AttnParams& p) {
+  const kv4_config& cfg = c->cfg;
+  const uint8_t* lbase = c->base + c->pool_offset + static_cast<size_t>(layer) * c->layer_stride;
+  p.pool = lbase;
+  p.prot = c->bf16 ? nullptr : lbase + c->pool_bytes;
+  p.block_table = c->block_table;
+  p.seq_lens = c->seq_lens + static_cast<size_t>(layer) * cfg.max_seqs;
+  p.seq_ids = seq_ids;
+  p.q = static_cast<const uint16_t*>(q);
+  p.out = out;
+  p.state = c->state;
+  p.n_seqs = n_seqs;
+  p.Hq = cfg.num_q_heads;
+  p.Hkv = cfg.num_kv_heads;
+  p.G = cfg.num_q_heads / cfg.num_kv_heads;
+  p.D = cfg.head_dim;
+  p.P = cfg.page_size;
+  p.S = cfg.sink_tokens;
+  p.W = cfg.recent_window;
+  p.Bh = c->bf16 ? 1 : cfg.hadamard_block;
+  p.rot_c = static_cast<float>(1.0 / sqrt(static_cast<double>(p.Bh)));
+  p.max_seqs = cfg.max_seqs;
+  p.num_pages = cfg.num_pages;
+  p.max_pages_per_seq = cfg.max_pages_per_seq;
+  p.mode = mode;
+  const double scale = softmax_scale > 0.f ? static_cast<double>(softmax_scale) : 1.0 / sqrt(static_cast<double>(p.D));
+  p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+  p.pool_bytes = c->pool_bytes;
+  p.prot_bytes = c->prot_bytes;
+  p.qblob_total = static_cast<size_t>(n_seqs) * cfg.num_kv_heads * qblob_bytes(p.D);
+}
+
 size_t attention_workspace_bytes(const kv4_cache* c, int n_seqs, int max_ctx) {
+  if (grouped_path(c)) return grouped_workspace_bytes(c, n_seqs);
   const kv4_config& cfg = c->cfg;
   const long long cap_ctx = static_cast<long long>(cfg.max_pages_per_seq) * cfg.page_size;
   const long long ctx = (max_ctx <= 0 || max_ctx > cap_ctx) ? cap_ctx : max_ctx;
@@ -1072,6 +724,11 @@ int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs
   const kv4_config& cfg = c->cfg;
   const int D = cfg.head_dim;
   const int G = cfg.num_q_heads / cfg.num_kv_heads;
+  if (grouped_path(c)) {
+    AttnParams p{};
+    fill_common(c, layer, seq_ids, n_seqs, q, out, softmax_scale, mode, p);
+    return launch_grouped(c, p, ws, ws_bytes, stream, D == 128 ? launch_merge<128, false> : launch_merge<64, false>);
+  }
   // largest first-list capacity that fits the caller's workspace
   const WsLayout w0 = ws_layout(c, n_seqs, 0);
   const size_t per_item = sizeof(Item) + static_cast<size_t>(partial_stride(G, D)) * sizeof(float);

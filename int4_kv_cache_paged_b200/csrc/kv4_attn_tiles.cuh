@@ -1,0 +1,466 @@
+// Tile routines of the split-K decode attention kernels: turn the codes of one
+// 16-token tile in shared memory into 16x8x16 tensor-core operands, run the
+// scores, the online softmax and P.V.  Shared by the per-head and the
+// page-major kernels.
+//
+// Method: "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
+// Serving", Abstract (fused attention over the rotated token-wise INT4 cache);
+// scale and zero point are folded out of the inner products as in the
+// folded-scale kernels of "KV Cache Quantization" (topic page), item 2:
+//     q . k^  = s_k * (q . c_k) + z_k * sum(q)
+//     sum_p a_p v^_p = sum_p (a_p s_p) c_p + sum_p a_p z_p
+#pragma once
+
+#include "kv4_common.cuh"
+
+#include <math.h>
+
+namespace kv4 {
+namespace tiles {
+
+constexpr float NEG_INF = -INFINITY;
+
+// Partial of one item: per query head, o[D] (unnormalised, rotated basis), m, l,
+// padded to D + 4 floats so every head row starts on a 16-byte boundary.
+__host__ __device__ constexpr int head_stride(int D) { return D + 4; }
+__host__ __device__ inline int partial_stride(int G, int D) { return G * head_stride(D); }
+
+// ---------------------------------------------------------------------------
+// per-warp online-softmax state
+
+template <int D>
+struct WarpState {
+  float o[D / 16][4];  // o^T fragments: (dim 16m+g, head 2t), (16m+g, 2t+1), (16m+g+8, 2t), (16m+g+8, 2t+1)
+  float m0, m1, l0, l1, z0, z1;
+};
+
+// Column split of the P.V weights (see pv_operands): part of each of the thread's two columns.
+struct ColSplit {
+  bool colsplit;
+  int part0, part1;
+};
+
+template <int D>
+struct QFrag {
+  uint32_t b[D / 16][2];
+  float qs0, qs1, kscale;
+};
+
+template <int D>
+__device__ __forceinline__ void online_softmax_pv(WarpState<D>& ws, float x0, float x1, float x2, float x3,
+                                                  float& p0, float& p1, float& p2, float& p3) {
+  float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+  }
+  const float n0 = fmaxf(ws.m0, mx0), n1 = fmaxf(ws.m1, mx1);
+  if (__any_sync(0xffffffffu, n0 > ws.m0 || n1 > ws.m1)) {
+    const float a0 = ex2(ws.m0 - n0), a1 = ex2(ws.m1 - n1);
+    ws.l0 *= a0; ws.l1 *= a1; ws.z0 *= a0; ws.z1 *= a1;
+#pragma unroll
+    for (int m = 0; m < D / 16; ++m) {
+      ws.o[m][0] *= a0; ws.o[m][1] *= a1; ws.o[m][2] *= a0; ws.o[m][3] *= a1;
+    }
+    ws.m0 = n0; ws.m1 = n1;
+  }
+  p0 = ex2(x0 - ws.m0); p1 = ex2(x1 - ws.m1); p2 = ex2(x2 - ws.m0); p3 = ex2(x3 - ws.m1);
+}
+
+
+// P.V weights of this thread's two columns (c0 = 2t, c1 = 2t+1) for tokens g and
+// g+8.  With the column split (G = 1, 2, 4), column c carries part c / G of the
+// weight of head c % G: part 0 = hi = fp16(P), part 1 = lo = fp16(P - hi),
+// parts >= 2 are zero; one 16x8x16 multiply then accumulates both parts.
+// Without it (other G) the hi parts go to (B0, B1) and the lo parts to (C0, C1).
+__device__ __forceinline__ void pv_operands(float P0, float P1, float P2, float P3, int part0, int part1,
+                                            bool colsplit, uint32_t& B0, uint32_t& B1, uint32_t& C0, uint32_t& C1) {
+  const uint32_t h01 = pack_half2(P0, P1), h23 = pack_half2(P2, P3);
+  const uint32_t l01 = pack_half2(P0 - half_lo(h01), P1 - half_hi(h01));
+  const uint32_t l23 = pack_half2(P2 - half_lo(h23), P3 - half_hi(h23));
+  if (colsplit) {
+    const uint32_t m0 = part0 == 0 ? 0x0000FFFFu : 0u, m1 = part1 == 0 ? 0xFFFF0000u : 0u;
+    const uint32_t n0 = part0 == 1 ? 0x0000FFFFu : 0u, n1 = part1 == 1 ? 0xFFFF0000u : 0u;
+    B0 = movmatrix_trans((h01 & (m0 | m1)) | (l01 & (n0 | n1)));
+    B1 = movmatrix_trans((h23 & (m0 | m1)) | (l23 & (n0 | n1)));
+    C0 = C1 = 0u;
+  } else {
+    B0 = movmatrix_trans(h01);
+    B1 = movmatrix_trans(h23);
+    C0 = movmatrix_trans(l01);
+    C1 = movmatrix_trans(l23);
+  }
+}
+
+// QK^T of one INT4 tile: acc = (q * 2^e) . codes for tokens g, g+8 and heads 2t, 2t+1.
+template <int D>
+__device__ __forceinline__ void qk_int4(uint32_t st, const QFrag<D>& qf, int lane, float (&acc)[4]) {
+  constexpr int NKK = D / 32;
+  uint32_t kw0[NKK], kw1[NKK];
+  if constexpr (D == 128) {
+    const uint4 a = lds128(st + lane * 16), bq = lds128(st + 512 + lane * 16);
+    kw0[0] = a.x; kw0[1] = a.y; kw0[2] = a.z; kw0[3] = a.w;
+    kw1[0] = bq.x; kw1[1] = bq.y; kw1[2] = bq.z; kw1[3] = bq.w;
+  } else {
+    const uint2 a = lds64(st + lane * 8), bq = lds64(st + 256 + lane * 8);
+    kw0[0] = a.x; kw0[1] = a.y; kw1[0] = bq.x; kw1[1] = bq.y;
+  }
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < NKK; ++kk) {
+    const uint32_t w0 = kw0[kk], w1 = kw1[kk];
+    mma_f16(acc, nib_lo(w0), nib_lo(w1), nib_hi(w0), nib_hi(w1), qf.b[2 * kk][0], qf.b[2 * kk][1]);
+    const uint32_t u0 = w0 >> 8, u1 = w1 >> 8;
+    mma_f16(acc, nib_lo(u0), nib_lo(u1), nib_hi(u0), nib_hi(u1), qf.b[2 * kk + 1][0], qf.b[2 * kk + 1][1]);
+  }
+}
+
+// P.V of one INT4 tile: o^T[m] += V^T codes * (hi + lo) weights.
+template <int D>
+__device__ __forceinline__ void pv_int4(uint32_t st, WarpState<D>& ws, int lane, uint32_t B0, uint32_t B1,
+                                        uint32_t C0, uint32_t C1, bool colsplit) {
+  uint32_t vw[D / 16];
+  if constexpr (D == 128) {
+    const uint4 v0 = lds128(st + 8 * D + lane * 16), v1 = lds128(st + 8 * D + 512 + lane * 16);
+    vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+    vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
+  } else {
+    const uint4 v0 = lds128(st + 8 * D + lane * 16);
+    vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+  }
+#pragma unroll
+  for (int m = 0; m < D / 16; ++m) {
+    const uint32_t w = vw[m], u = w >> 8;
+    const uint32_t a0 = nib_lo(w), a1 = nib_hi(w), a2 = nib_lo(u), a3 = nib_hi(u);
+    mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
+    if (!colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
+  }
+}
+
+// One unit of NT (1 or 2) INT4 tiles at shared addresses tile[0], tile[1]:
+// scores, one online-softmax update for the NT*16 tokens, P.V.  valid[u] bit 0 /
+// bit 1: token g / g+8 of tile u is inside the item's range (used when MASKED).
+// The stage(s) are handed back (empty barriers eb0, and eb1 when it differs)
+// after the last shared-memory load.
+template <int D, int NT, bool MASKED>
+__device__ __forceinline__ void unit_int4(const uint32_t (&tile)[2], const QFrag<D>& qf, WarpState<D>& ws, int lane,
+                                          const int (&valid)[2], uint32_t eb0, uint32_t eb1, const ColSplit& cs) {
+  float x[NT][4];
+  uint4 sz[NT];
+  // Q.K^T of the NT tiles, interleaved, each with two accumulators (even / odd
+  // k-steps): 2*NT independent chains of D/32 multiplies instead of NT chains of D/16.
+  constexpr int NKK = D / 32;
+  uint32_t kw[NT][2][NKK];
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    if constexpr (D == 128) {
+      const uint4 a = lds128(tile[u] + lane * 16), bq = lds128(tile[u] + 512 + lane * 16);
+      kw[u][0][0] = a.x; kw[u][0][1] = a.y; kw[u][0][2] = a.z; kw[u][0][3] = a.w;
+      kw[u][1][0] = bq.x; kw[u][1][1] = bq.y; kw[u][1][2] = bq.z; kw[u][1][3] = bq.w;
+    } else {
+      const uint2 a = lds64(tile[u] + lane * 8), bq = lds64(tile[u] + 256 + lane * 8);
+      kw[u][0][0] = a.x; kw[u][0][1] = a.y; kw[u][1][0] = bq.x; kw[u][1][1] = bq.y;
+    }
+    sz[u] = lds128(tile[u] + 16 * D + (lane >> 2) * 16);
+  }
+  float acc[NT][2][4];
+#pragma unroll
+  for (int u = 0; u < NT; ++u)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) acc[u][e][0] = acc[u][e][1] = acc[u][e][2] = acc[u][e][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < NKK; ++kk) {
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      const uint32_t w0 = kw[u][0][kk], w1 = kw[u][1][kk];
+      mma_f16(acc[u][0], nib_lo(w0), nib_lo(w1), nib_hi(w0), nib_hi(w1), qf.b[2 * kk][0], qf.b[2 * kk][1]);
+      const uint32_t u0 = w0 >> 8, u1 = w1 >> 8;
+      mma_f16(acc[u][1], nib_lo(u0), nib_lo(u1), nib_hi(u0), nib_hi(u1), qf.b[2 * kk + 1][0], qf.b[2 * kk + 1][1]);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    float acc_u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc_u[i] = acc[u][0][i] + acc[u][1][i];
+    float (&acc2)[4] = acc_u;
+    const float sKg = half_lo(sz[u].x) * qf.kscale, zKg = half_hi(sz[u].x);
+    const float sKg8 = half_lo(sz[u].y) * qf.kscale, zKg8 = half_hi(sz[u].y);
+    x[u][0] = fmaf(acc2[0], sKg, zKg * qf.qs0);
+    x[u][1] = fmaf(acc2[1], sKg, zKg * qf.qs1);
+    x[u][2] = fmaf(acc2[2], sKg8, zKg8 * qf.qs0);
+    x[u][3] = fmaf(acc2[3], sKg8, zKg8 * qf.qs1);
+    if constexpr (MASKED) {
+      if (!(valid[u] & 1)) { x[u][0] = NEG_INF; x[u][1] = NEG_INF; }
+      if (!(valid[u] & 2)) { x[u][2] = NEG_INF; x[u][3] = NEG_INF; }
+    }
+  }
+  // online softmax over the unit.  The running max only moves when some score
+  // exceeds it: vote first, and reduce over the 8 row groups and rescale only then.
+  float mx0 = fmaxf(x[0][0], x[0][2]), mx1 = fmaxf(x[0][1], x[0][3]);
+#pragma unroll
+  for (int u = 1; u < NT; ++u) {
+    mx0 = fmaxf(mx0, fmaxf(x[u][0], x[u][2]));
+    mx1 = fmaxf(mx1, fmaxf(x[u][1], x[u][3]));
+  }
+  if (__any_sync(0xffffffffu, mx0 > ws.m0 || mx1 > ws.m1)) {
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float n0 = fmaxf(ws.m0, mx0), n1 = fmaxf(ws.m1, mx1);
+    const float a0 = ex2(ws.m0 - n0), a1 = ex2(ws.m1 - n1);
+    ws.l0 *= a0; ws.l1 *= a1; ws.z0 *= a0; ws.z1 *= a1;
+#pragma unroll
+    for (int m = 0; m < D / 16; ++m) {
+      ws.o[m][0] *= a0; ws.o[m][1] *= a1; ws.o[m][2] *= a0; ws.o[m][3] *= a1;
+    }
+    ws.m0 = n0; ws.m1 = n1;
+  }
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    const float p0 = ex2(x[u][0] - ws.m0), p1 = ex2(x[u][1] - ws.m1);
+    const float p2 = ex2(x[u][2] - ws.m0), p3 = ex2(x[u][3] - ws.m1);
+    const float sVg = half_lo(sz[u].z), zVg = half_hi(sz[u].z), sVg8 = half_lo(sz[u].w), zVg8 = half_hi(sz[u].w);
+    float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
+    float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
+    if constexpr (MASKED) {   // unwritten slots may hold non-finite scales
+      if (!(valid[u] & 1)) { P0 = 0.f; P1 = 0.f; zg0 = 0.f; zg1 = 0.f; }
+      if (!(valid[u] & 2)) { P2 = 0.f; P3 = 0.f; zg80 = 0.f; zg81 = 0.f; }
+    }
+    ws.l0 += p0 + p2; ws.l1 += p1 + p3;
+    ws.z0 += zg0 + zg80; ws.z1 += zg1 + zg81;
+    uint32_t B0, B1, C0, C1;
+    pv_operands(P0, P1, P2, P3, cs.part0, cs.part1, cs.colsplit, B0, B1, C0, C1);
+    if (u == NT - 1) {
+      // last tile: load its V codes, then hand the stage(s) back before the math
+      const uint32_t t = tile[u];
+      uint32_t vw[D / 16];
+      if constexpr (D == 128) {
+        const uint4 v0 = lds128(t + 8 * D + lane * 16), v1 = lds128(t + 8 * D + 512 + lane * 16);
+        vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+        vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
+      } else {
+        const uint4 v0 = lds128(t + 8 * D + lane * 16);
+        vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(eb0);
+        if (eb1 != eb0) mbar_arrive(eb1);
+      }
+#pragma unroll
+      for (int m = 0; m < D / 16; ++m) {
+        const uint32_t w = vw[m], uu = w >> 8;
+        const uint32_t a0 = nib_lo(w), a1 = nib_hi(w), a2 = nib_lo(uu), a3 = nib_hi(uu);
+        mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
+        if (!cs.colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
+      }
+    } else {
+      pv_int4<D>(tile[u], ws, lane, B0, B1, C0, C1, cs.colsplit);
+    }
+  }
+}
+
+// One INT8 tile (protected store).
+template <int D, bool MASKED>
+__device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, bool vg,
+                                          bool vg8, uint32_t empty_bar, const ColSplit& cs) {
+  constexpr int NK = D / 16;
+  uint32_t kw[2][NK], vw[2 * NK];
+#pragma unroll
+  for (int rowhi = 0; rowhi < 2; ++rowhi)
+#pragma unroll
+    for (int kq = 0; kq < D / 64; ++kq) {
+      const uint4 a = lds128(st + 16 * (32 * (rowhi * (D / 64) + kq) + lane));
+      kw[rowhi][4 * kq] = a.x; kw[rowhi][4 * kq + 1] = a.y; kw[rowhi][4 * kq + 2] = a.z; kw[rowhi][4 * kq + 3] = a.w;
+    }
+#pragma unroll
+  for (int q4 = 0; q4 < NK / 2; ++q4) {
+    const uint4 a = lds128(st + 16 * D + 16 * (32 * q4 + lane));
+    vw[4 * q4] = a.x; vw[4 * q4 + 1] = a.y; vw[4 * q4 + 2] = a.z; vw[4 * q4 + 3] = a.w;
+  }
+  const uint4 sz = lds128(st + 32 * D + (lane >> 2) * 16);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty_bar);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int k = 0; k < NK; ++k) {
+    const uint32_t w0 = kw[0][k], w1 = kw[1][k];
+    mma_f16(acc, byte_lo(w0), byte_lo(w1), byte_lo(w0 >> 8), byte_lo(w1 >> 8), qf.b[k][0], qf.b[k][1]);
+  }
+  const float sKg = half_lo(sz.x) * qf.kscale, zKg = half_hi(sz.x);
+  const float sKg8 = half_lo(sz.y) * qf.kscale, zKg8 = half_hi(sz.y);
+  float x0 = fmaf(acc[0], sKg, zKg * qf.qs0);
+  float x1 = fmaf(acc[1], sKg, zKg * qf.qs1);
+  float x2 = fmaf(acc[2], sKg8, zKg8 * qf.qs0);
+  float x3 = fmaf(acc[3], sKg8, zKg8 * qf.qs1);
+  if constexpr (MASKED) {
+    if (!vg) { x0 = NEG_INF; x1 = NEG_INF; }
+    if (!vg8) { x2 = NEG_INF; x3 = NEG_INF; }
+  }
+  float p0, p1, p2, p3;
+  online_softmax_pv<D>(ws, x0, x1, x2, x3, p0, p1, p2, p3);
+  const float sVg = half_lo(sz.z), zVg = half_hi(sz.z), sVg8 = half_lo(sz.w), zVg8 = half_hi(sz.w);
+  float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
+  float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
+  if constexpr (MASKED) {
+    if (!vg) { P0 = 0.f; P1 = 0.f; zg0 = 0.f; zg1 = 0.f; }
+    if (!vg8) { P2 = 0.f; P3 = 0.f; zg80 = 0.f; zg81 = 0.f; }
+  }
+  ws.l0 += p0 + p2; ws.l1 += p1 + p3;
+  ws.z0 += zg0 + zg80; ws.z1 += zg1 + zg81;
+  uint32_t B0, B1, C0, C1;
+  pv_operands(P0, P1, P2, P3, cs.part0, cs.part1, cs.colsplit, B0, B1, C0, C1);
+#pragma unroll
+  for (int m = 0; m < NK; ++m) {
+    const uint32_t w0 = vw[2 * m], w1 = vw[2 * m + 1];
+    const uint32_t a0 = byte_lo(w0), a1 = byte_lo(w0 >> 8), a2 = byte_lo(w1), a3 = byte_lo(w1 >> 8);
+    mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
+    if (!cs.colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
+  }
+}
+
+// One BF16 tile (baseline cache).  Holds the stage until the V loads are done.
+// vmask01 / vmask89: per-thread masks of the V operand halves of tokens 2t, 2t+1
+// and 2t+8, 2t+9 (unwritten slots of a page may hold NaN bit patterns, and
+// 0 * NaN would poison the accumulator).
+template <int D, bool MASKED>
+__device__ __forceinline__ void tile_bf16(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, bool vg,
+                                          bool vg8, uint32_t empty_bar, uint32_t vmask01, uint32_t vmask89) {
+  constexpr int NK = D / 16;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int k = 0; k < NK; ++k) {
+    const uint4 a = lds128(st + 16 * (32 * k + lane));
+    mma_bf16(acc, a.x, a.y, a.z, a.w, qf.b[k][0], qf.b[k][1]);
+  }
+  uint4 v[NK];
+#pragma unroll
+  for (int m = 0; m < NK; ++m) {
+    v[m] = lds128(st + 32 * D + 16 * (32 * m + lane));
+    if constexpr (MASKED) {
+      v[m].x &= vmask01; v[m].y &= vmask01; v[m].z &= vmask89; v[m].w &= vmask89;
+    }
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty_bar);
+  float x0 = acc[0] * qf.kscale, x1 = acc[1] * qf.kscale, x2 = acc[2] * qf.kscale, x3 = acc[3] * qf.kscale;
+  if constexpr (MASKED) {
+    if (!vg) { x0 = NEG_INF; x1 = NEG_INF; }
+    if (!vg8) { x2 = NEG_INF; x3 = NEG_INF; }
+  }
+  float p0, p1, p2, p3;
+  online_softmax_pv<D>(ws, x0, x1, x2, x3, p0, p1, p2, p3);
+  ws.l0 += p0 + p2; ws.l1 += p1 + p3;
+  const uint32_t B0 = movmatrix_trans(pack_bf162(p0, p1));
+  const uint32_t B1 = movmatrix_trans(pack_bf162(p2, p3));
+#pragma unroll
+  for (int m = 0; m < NK; ++m) mma_bf16(ws.o[m], v[m].x, v[m].y, v[m].z, v[m].w, B0, B1);
+}
+
+
+// Rotated queries of one (sequence, KV head) as 16x8x16 B operands, written to
+// qblob[b * Hkv + h]: fp32 FWHT (same order as the append), bf16 rounding, then
+// fp16 with a power-of-two scale (INT4 cache) or plain bf16 (BF16 cache); the
+// tail holds sigma*log2(e)*sum(q) per column and the key scale factor.
+// sq: shared scratch of G*D floats for this warp.
+template <int D, bool BF16>
+__device__ __forceinline__ void build_qblob(const AttnParams& p, int b, int h, int lane, float* sq) {
+  constexpr int VPL = D / 32;
+  const int G = p.G;
+  const int gw = b * p.Hkv + h;
+  float qsum[MAX_G];
+  float amax = 0.f;
+  const float rot_c = p.rot_c;
+  for (int g = 0; g < G; ++g) {
+    const uint16_t* src = p.q + (static_cast<long long>(b) * p.Hq + h * G + g) * D;
+    float x[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) x[i] = __bfloat162float(__ushort_as_bfloat16(src[VPL * lane + i]));
+    if constexpr (!BF16) {
+      for (int hh = 1; hh < p.Bh; hh <<= 1) {
+        if (hh < VPL) {
+#pragma unroll
+          for (int i = 0; i < VPL; ++i)
+            if ((i & hh) == 0) {
+              const float a = x[i], c = x[i + hh];
+              x[i] = __fadd_rn(a, c);
+              x[i + hh] = __fsub_rn(a, c);
+            }
+        } else {
+          const int lm = hh / VPL;
+          const bool upper = (lane & lm) != 0;
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) {
+            const float o = __shfl_xor_sync(0xffffffffu, x[i], lm);
+            x[i] = upper ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) x[i] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(x[i], rot_c)));
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      sq[g * D + VPL * lane + i] = x[i];
+      s += x[i];
+      amax = fmaxf(amax, fabsf(x[i]));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    qsum[g] = s;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  __syncwarp();
+  // fp16 operands: q * 2^e with max|q| * 2^e in [2^14, 2^15) (exact for normal values)
+  int e = 0;
+  if (!BF16 && amax > 0.f && amax <= 3.0e38f) {
+    int ex;
+    frexpf(amax, &ex);
+    e = 15 - ex;
+  }
+  uint32_t* blob = reinterpret_cast<uint32_t*>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D));
+  const int g = lane >> 2, t = lane & 3;
+  // B-operand column n holds query head n % G when the column split applies
+  // (G = 1, 2, 4: the spare columns carry the low part of the P.V weights),
+  // otherwise head n for n < G and zeros.
+  const bool colsplit = (G == 1 || G == 2 || G == 4);
+  const int gsrc = colsplit ? g % G : g;
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t r[4];
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      const int k = 2 * c + kk;
+#pragma unroll
+      for (int reg = 0; reg < 2; ++reg) {
+        const int d = 16 * k + 2 * t + 8 * reg;
+        float a = 0.f, bb = 0.f;
+        if (gsrc < G) { a = sq[gsrc * D + d]; bb = sq[gsrc * D + d + 1]; }
+        if constexpr (BF16) {
+          r[2 * kk + reg] = pack_bf162(a, bb);
+        } else {
+          r[2 * kk + reg] = pack_half2(ldexpf(a, e), ldexpf(bb, e));
+        }
+      }
+    }
+    reinterpret_cast<uint4*>(blob)[c * 32 + lane] = make_uint4(r[0], r[1], r[2], r[3]);
+  }
+  float* tail = reinterpret_cast<float*>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D) + 16 * D);
+  if (lane < MAX_G) {
+    const int src = colsplit ? lane % G : lane;
+    float v = 0.f;
+#pragma unroll
+    for (int gg = 0; gg < MAX_G; ++gg)
+      if (gg == src && gg < G) v = qsum[gg];
+    tail[lane] = BF16 ? 0.f : v * p.scale_log2;
+  }
+  if (lane == MAX_G) tail[MAX_G] = ldexpf(p.scale_log2, -e);
+}
+
+}  // namespace tiles
+}  // namespace kv4

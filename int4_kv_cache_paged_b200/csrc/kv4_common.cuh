@@ -18,6 +18,9 @@
 //   BF16 K: element 8*(32*k + 4*g + t) + 2*(rowhi + 2*h8) + e
 //   BF16 V: element 8*(32*m + 4*g + t) + 2*(dh + 2*th) + e
 //   scales: half2 (s, z) of token r, tensor T (K=0, V=1) at byte 16*(r%8) + 4*(2*T + r/8)
+// Pools are head-innermost: INT4/BF16 pool [page][P/16][Hkv][tile], INT8 store
+// [seq][ceil((S+W)/16)][Hkv][tile8], so one page position of all KV heads is
+// one contiguous run.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -64,12 +67,13 @@ struct Item {
 };
 static_assert(sizeof(Item) == 48, "item size");
 
-// Per (sequence, KV head) record written by the planning kernel.
+// Per (sequence, KV head) record written by the planning kernel: the partials
+// of this head are part_base + j * stride, j < n_parts.
 struct SeqHead {
   int part_base;
   int n_parts;
   int len;
-  int pad;
+  int pad;    // stride between consecutive partials of the head
 };
 
 // Parameters shared by the attention kernels.
@@ -96,6 +100,7 @@ struct AttnParams {
   float rot_c;                // fp32(1/sqrt(Bh))
   size_t pool_bytes, prot_bytes, qblob_total;   // extents, for the self-checks of debug builds
   int ns;                     // shared-memory ring depth of the attention kernel
+  int grid;                   // CTAs of the page-major attention kernel
 };
 
 // ---------------------------------------------------------------------------
@@ -326,7 +331,9 @@ struct kv4_cache {
   size_t pool_bytes;         // per layer
   size_t prot_bytes;         // per layer (INT4 cache only)
   int attn_blocks_per_sm;
-  int attn_ring;             // ring depth chosen for the attention kernel
+  int attn_ring;             // ring depth chosen for the per-head attention kernel
+  int gattn_ring;            // ring depth of the page-major kernel (0: not used by this cache)
+  int gattn_pair;            // INT4 tiles per consumer iteration of the page-major kernel (1 or 2)
   cudaEvent_t ev_before;     // optional timing events around the split-K kernel
   cudaEvent_t ev_after;
 };
@@ -343,5 +350,11 @@ int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs
                      float softmax_scale, int mode, void* ws, size_t ws_bytes, cudaStream_t stream);
 size_t attention_workspace_bytes(const kv4_cache* c, int n_seqs, int max_ctx);
 int attention_blocks_per_sm(kv4_cache* c);
+// page-major path (INT4 cache, KV heads a multiple of 8)
+bool grouped_path(const kv4_cache* c);
+int grouped_ring(kv4_cache* c);
+size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs);
+int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes, cudaStream_t stream,
+                   void (*merge)(const AttnParams&, cudaStream_t));
 
 }  // namespace kv4

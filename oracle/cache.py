@@ -24,6 +24,12 @@ Readings of this library (the pages give none of these details):
 * K and V are quantized separately, each with its own (s, z), each after the
   same block-diagonal Hadamard rotation.
 * Keys arrive post-RoPE; RoPE is not part of this cache.
+* Device byte order (head-innermost, so that the tiles of all KV heads at one
+  page position are contiguous):
+    INT4 pool of a layer   uint8 [num_pages][P/16][Hkv][16*D + 128]
+    INT8 store of a layer  uint8 [max_seqs][ceil((S+W)/16)][Hkv][32*D + 128]
+    BF16 pool of a layer   bf16  [num_pages][P/16][Hkv][32*D]
+  The arrays below use the same order per page / per sequence.
 """
 
 import numpy as np
@@ -54,8 +60,8 @@ def is_protected(p, L, S, W):
 class OracleKV4Cache:
     """The cache state: per-layer INT4 pages, per-(layer, seq) INT8 store, sequence lengths.
 
-    Pages are held sparsely: pages[(layer, page)] is uint8 [Hkv, P/16, int4 tile];
-    prot[(layer, seq)] is uint8 [Hkv, n_prot_tiles, int8 tile].  Bytes never
+    Pages are held sparsely: pages[(layer, page)] is uint8 [P/16, Hkv, int4 tile];
+    prot[(layer, seq)] is uint8 [n_prot_tiles, Hkv, int8 tile].  Bytes never
     written are zero here and undefined on the device.
     """
 
@@ -84,13 +90,13 @@ class OracleKV4Cache:
     def _page_tiles(self, layer, page):
         key = (layer, page)
         if key not in self.pages:
-            self.pages[key] = np.zeros((self.Hkv, self.P // TILE, int4_tile_bytes(self.D)), np.uint8)
+            self.pages[key] = np.zeros((self.P // TILE, self.Hkv, int4_tile_bytes(self.D)), np.uint8)
         return self.pages[key]
 
     def _prot_tiles(self, layer, seq):
         key = (layer, seq)
         if key not in self.prot:
-            self.prot[key] = np.zeros((self.Hkv, n_prot_tiles(self.S, self.W), int8_tile_bytes(self.D)), np.uint8)
+            self.prot[key] = np.zeros((n_prot_tiles(self.S, self.W), self.Hkv, int8_tile_bytes(self.D)), np.uint8)
         return self.prot[key]
 
     def _pages_of(self, seq, pos):
@@ -116,13 +122,13 @@ class OracleKV4Cache:
         return s16, z16
 
     def _scatter(self, tiles, ti, byte_idx, vals):
-        """tiles [Hkv, T, bytes]; ti [m]; byte_idx [m, k]; vals [m, Hkv, k] -> tiles[h, ti_j, byte_idx_j] = vals[j, h]."""
+        """tiles [T, Hkv, bytes]; ti [m]; byte_idx [m, k]; vals [m, Hkv, k] -> tiles[ti_j, h, byte_idx_j] = vals[j, h]."""
         for h in range(self.Hkv):
-            tiles[h][ti[:, None], byte_idx] = vals[:, h, :]
+            tiles[ti[:, None], h, byte_idx] = vals[:, h, :]
 
     def _gather(self, tiles, ti, byte_idx):
         """Inverse of _scatter: returns [m, Hkv, k]."""
-        return np.stack([tiles[h][ti[:, None], byte_idx] for h in range(self.Hkv)], axis=1)
+        return np.stack([tiles[ti[:, None], h, byte_idx] for h in range(self.Hkv)], axis=1)
 
     def _write_int4(self, layer, seq, pos, enc_k, enc_v):
         """INT4 codes and scales of positions `pos` (enc_*: codes [m, Hkv, D], s16, z16 [m, Hkv])."""
@@ -275,8 +281,8 @@ class OracleBF16Cache:
             raise ValueError("unmapped page")
         key = (layer, page)
         if key not in self.pages:
-            self.pages[key] = np.zeros((self.Hkv, self.P // TILE, bf16_tile_bytes(self.D) // 2), np.uint16)
-        return self.pages[key][:, (p % self.P) // TILE, :], p % TILE
+            self.pages[key] = np.zeros((self.P // TILE, self.Hkv, bf16_tile_bytes(self.D) // 2), np.uint16)
+        return self.pages[key][(p % self.P) // TILE], p % TILE
 
     def append(self, layer, seq_ids, cu_new, k_new, v_new):
         k_bits = _bf16_bits(k_new)

@@ -95,8 +95,8 @@ def compare_int4_pages(pair, layer, seqs):
             ti, r = (p % P) // TILE, p % TILE
             idx = np.concatenate([t4.k_byte[r], 8 * D + t4.v_byte[r], 16 * D + scale_offset(r, 0) + ar4,
                                   16 * D + scale_offset(r, 1) + ar4])
-            g = pages[page, :, ti][:, idx]
-            o = pair.orc.pages[(layer, page)][:, ti][:, idx]
+            g = pages[page, ti][:, idx]
+            o = pair.orc.pages[(layer, page)][ti][:, idx]
             if not np.array_equal(g, o):
                 bad.append((seq, p, int(np.sum(g != o))))
     return bad
@@ -116,8 +116,8 @@ def compare_int8_store(pair, layer, seqs):
             ti, r = slot // TILE, slot % TILE
             idx = np.concatenate([t8.k_byte[r], 16 * D + t8.v_byte[r], 32 * D + scale_offset(r, 0) + ar4,
                                   32 * D + scale_offset(r, 1) + ar4])
-            g = prot[seq, :, ti][:, idx]
-            o = pair.orc.prot[(layer, seq)][:, ti][:, idx]
+            g = prot[seq, ti][:, idx]
+            o = pair.orc.prot[(layer, seq)][ti][:, idx]
             if not np.array_equal(g, o):
                 bad.append((seq, slot, int(np.sum(g != o))))
     return bad
@@ -135,7 +135,7 @@ def compare_bf16_pages(pair, layer, seqs):
             page = int(pair.table[seq, p // P])
             ti, r = (p % P) // TILE, p % TILE
             idx = np.concatenate([tb.k_elem[r], 16 * D + tb.v_elem[r]])
-            if not np.array_equal(pages[page, :, ti][:, idx], pair.orc.pages[(layer, page)][:, ti][:, idx]):
+            if not np.array_equal(pages[page, ti][:, idx], pair.orc.pages[(layer, page)][ti][:, idx]):
                 bad.append((seq, p))
     return bad
 

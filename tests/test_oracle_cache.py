@@ -87,7 +87,7 @@ def test_bulk_and_incremental_appends_store_identical_bytes():
     for p in range(150):
         if is_protected(p, 150, 4, 32):
             s = prot_slot(p, 4, 32)
-            np.testing.assert_array_equal(a.prot[(0, 0)][:, s // 16], b.prot[(0, 0)][:, s // 16])
+            np.testing.assert_array_equal(a.prot[(0, 0)][s // 16], b.prot[(0, 0)][s // 16])
     np.testing.assert_array_equal(a.view(0, 0)[0], b.view(0, 0)[0])
 
 
