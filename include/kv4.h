@@ -171,11 +171,17 @@ int kv4_attention_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_
  *   softmax_scale  <= 0 means 1/sqrt(D)
  *   mode           KV4_MODE_* bits
  *   dev_workspace  >= kv4_attention_workspace_bytes(cache, n_seqs, max L, ...)
- * A sequence of length 0 gives an all-zero output row.
- * Steps: a planning kernel (query rotation, chunking of every sequence into
- * work items), a persistent split-K kernel (pages staged by bulk copies,
- * INT4/INT8 codes turned into tensor-core operands in registers, online
- * softmax), and a merge kernel (log-sum-exp merge, inverse rotation, store).
+ * A sequence of length 0 gives an all-zero output row.  n_seqs <= max_seqs
+ * (KV4_ERR_INVALID_ARG otherwise).  Calls on one cache must be ordered on one
+ * stream: they share the cache's merge counters.
+ * Steps, with num_kv_heads a multiple of 8: one persistent kernel.  Every CTA
+ * derives the same stream-K split of all (sequence, 8-KV-head group) page
+ * stages from the sequence lengths, rotates its query heads into tensor-core
+ * operands, streams its stages through shared memory by bulk copies, turns
+ * INT4/INT8 codes into operands in registers (online softmax), and stores
+ * the rotated-back output; a group split over several CTAs is merged by the
+ * last of them (log-sum-exp merge over the workspace partials).  With other
+ * head counts: a planning kernel, a per-head split-K kernel and a merge kernel.
  */
 int kv4_decode_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs,
                          const void* q, void* out, float softmax_scale, int32_t mode,

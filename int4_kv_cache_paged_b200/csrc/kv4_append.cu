@@ -41,27 +41,7 @@ struct AppendParams {
 
 template <int VPL>
 __device__ __forceinline__ void fwht_warp(float (&x)[VPL], int Bh, float c, int lane) {
-  for (int h = 1; h < Bh; h <<= 1) {
-    if (h < VPL) {
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        if ((i & h) == 0) {
-          const float a = x[i], b = x[i + h];
-          x[i] = __fadd_rn(a, b);
-          x[i + h] = __fsub_rn(a, b);
-        }
-      }
-    } else {
-      const int lm = h / VPL;
-      const bool upper = (lane & lm) != 0;
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        const float other = __shfl_xor_sync(0xffffffffu, x[i], lm);
-        // lower element: x_i + x_{i+h}; upper element: x_i - x_{i+h} (x_i is the partner)
-        x[i] = upper ? __fsub_rn(other, x[i]) : __fadd_rn(x[i], other);
-      }
-    }
-  }
+  fwht_row<VPL>(x, Bh, lane);
 #pragma unroll
   for (int i = 0; i < VPL; ++i) x[i] = __fmul_rn(x[i], c);
 }

@@ -526,26 +526,7 @@ __global__ void __launch_bounds__(256) merge_kernel(AttnParams p) {
 #pragma unroll
     for (int i = 0; i < VPL; ++i) o[i] *= inv;
     if constexpr (!BF16) {
-      // o = H_blk o_rot (the normalised Hadamard matrix is its own inverse)
-      for (int hh = 1; hh < p.Bh; hh <<= 1) {
-        if (hh < VPL) {
-#pragma unroll
-          for (int i = 0; i < VPL; ++i)
-            if ((i & hh) == 0) {
-              const float a = o[i], c = o[i + hh];
-              o[i] = a + c;
-              o[i + hh] = a - c;
-            }
-        } else {
-          const int lm = hh / VPL;
-          const bool upper = (lane & lm) != 0;
-#pragma unroll
-          for (int i = 0; i < VPL; ++i) {
-            const float other = __shfl_xor_sync(0xffffffffu, o[i], lm);
-            o[i] = upper ? other - o[i] : o[i] + other;
-          }
-        }
-      }
+      fwht_row<VPL>(o, p.Bh, lane);   // o = H_blk o_rot (the normalised Hadamard matrix is its own inverse)
 #pragma unroll
       for (int i = 0; i < VPL; ++i) o[i] *= p.rot_c;
     }
@@ -624,12 +605,6 @@ int choose_ring(int device, int G, int* blocks_per_sm) {
     }
   }
   return -1;
-}
-
-template <int D, bool BF16>
-void launch_merge(const AttnParams& p, cudaStream_t stream) {
-  const int merge_warps = p.n_seqs * p.Hq;
-  merge_kernel<D, BF16><<<(merge_warps + 7) / 8, 256, 0, stream>>>(p);
 }
 
 template <int D, bool BF16>
@@ -727,7 +702,7 @@ int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs
   if (grouped_path(c)) {
     AttnParams p{};
     fill_common(c, layer, seq_ids, n_seqs, q, out, softmax_scale, mode, p);
-    return launch_grouped(c, p, ws, ws_bytes, stream, D == 128 ? launch_merge<128, false> : launch_merge<64, false>);
+    return launch_grouped(c, p, ws, ws_bytes, stream);
   }
   // largest first-list capacity that fits the caller's workspace
   const WsLayout w0 = ws_layout(c, n_seqs, 0);

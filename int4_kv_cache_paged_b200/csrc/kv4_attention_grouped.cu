@@ -6,21 +6,30 @@
 // cache) and "KV4-RL: Unlocking Faster Asynchronous Rollouts for RLVR with INT4
 // KV Cache Quantization", Abstract (sinks and recent positions read from INT8).
 //
+// One launch does the attention proper (a small query kernel runs alongside).
+//
 // Work decomposition.  A head group is 8 consecutive KV heads of one sequence.
 // Its work is a list of stages: one stage per 16-token INT4 tile position (the
 // tiles of the 8 heads are contiguous in the head-innermost pool, one 17 KB
 // bulk copy), then two stages per INT8 protected tile (heads 0-3, heads 4-7).
-// The planner concatenates the stage lists of all head groups (T stages) and
-// CTA c of the persistent grid (one per SM) takes stages [c*T/N, (c+1)*T/N):
-// every CTA streams the same number of bytes (stream-K), no scheduling atomics.
-// Where a CTA's range crosses head groups it works on segments; each segment
-// ends in one partial (m, l, o) per KV head and query head, merged later.
+// The stage lists of all head groups are concatenated (T stages) and CTA c of
+// the persistent grid takes stages [c*T/N, (c+1)*T/N): every CTA streams the
+// same number of bytes (stream-K).  Every CTA derives this plan itself from the
+// sequence lengths (a block scan over the head groups), so no planning kernel
+// runs first.  Where a CTA's range crosses head groups it works on segments.
 //
 // Inside a CTA: a producer warp issues the bulk copies into a ring of
 // shared-memory stages (each lane one stage of a batch, mbarrier completion);
 // consumer warp w handles KV head w of every stage, so every warp consumes
 // every stage in order (which keeps the mbarrier parity waits exact) and no
-// warp waits for another: each writes its own partial.
+// warp waits for another.  The rotated query operands come from a small
+// kernel launched just before (this kernel is its programmatic dependent and
+// waits for it only before its first operand read).  A group that one CTA
+// covers whole is normalised, rotated back and stored straight from registers;
+// a group split over several CTAs leaves one partial (m, l, o) per segment in
+// the workspace, and the warp whose partial arrives last (a counter per batch
+// entry and KV head, set back to zero by that warp) merges them and stores the
+// output.  A launch in which a wait gave up zeroes all counters at its end.
 #include "kv4_attn_tiles.cuh"
 
 namespace kv4 {
@@ -38,34 +47,43 @@ struct GCfg {
   static constexpr int STAGE4 = GW * tile4_bytes(D);        // one tile position, 8 heads
   static constexpr int STAGE8 = (GW / 2) * tile8_bytes(D);  // one protected tile, 4 heads
   static constexpr int STAGE = STAGE4 > STAGE8 ? STAGE4 : STAGE8;
-  static constexpr int QBLOBS = GW * qblob_bytes(D);         // the group's 8 query blobs
 };
 
-// Per head group, written by the planner.
+// One head group of the call: batch entry b, KV heads 8*hg .. 8*hg+7.
 struct Group {
-  int b, seq, hg;   // index into seq_ids, sequence id, head group (KV heads 8*hg .. 8*hg+7)
-  int n4;           // INT4 stages (tiles t0 .. t0+n4-1)
-  int t0, lo4, hi4; // first INT4 tile, valid INT4 positions [lo4, hi4)
-  int n8;           // INT8 tiles (2 stages each), valid slots [0, nprot)
+  int b, seq, hg, L;  // index into seq_ids, sequence id, head group, sequence length
+  int n4;             // INT4 stages (tiles t0 .. t0+n4-1)
+  int t0, lo4, hi4;   // first INT4 tile, valid INT4 positions [lo4, hi4)
+  int n8;             // INT8 tiles (2 stages each), valid slots [0, nprot)
   int nprot;
-  int start;        // first global stage index
-  int segbase;      // first segment (partial slot / 8) of this group
-  int c_first;      // first CTA whose range touches this group
+  int start;          // first global stage index
+  int pad;
 };
 static_assert(sizeof(Group) == 48, "group size");
 
-struct SegQ {       // one queued segment
+struct SegQ {         // one queued segment
   Group g;
-  int u0, n, k;     // local stages [u0, u0+n), segment index within the group
-  int pad;
+  int u0, n;          // local stages [u0, u0+n)
+  int k, nseg;        // segment index within the group, segments of the group
 };
 
-struct GHeader {
-  int T;            // total stages
-  int N;            // CTAs of the attention grid
-  int n_groups;
-  int pad[61];
+// Per-CTA bookkeeping in shared memory.
+struct GMisc {
+  int abort;          // a wait gave up
+  int exited;         // warps of this CTA that are done
+  int pad0;
+  Group first;        // the group holding the CTA's first stage (start filled in)
+  int n_empty;        // empty groups this CTA writes zeros for
+  int pad[3];
+  int red[32];        // block-scan scratch
+  int empty[32];
+  int last_fill[16];  // last ring fill per stage (drained before an aborting producer exits)
 };
+
+constexpr int MAX_NS = 16;
+// A CTA takes at least this many stages: a short batch is spread over fewer
+// CTAs, so that merging the partials costs less than the streaming it saves.
+constexpr int MIN_STAGES = 16;
 
 __host__ __device__ inline int group_stages(const Group& g) { return g.n4 + 2 * g.n8; }
 
@@ -77,8 +95,8 @@ __device__ __forceinline__ int cta_of(long long j, long long T, long long N) {
 template <int D>
 __host__ __device__ inline size_t gattn_smem_bytes(int ns) {
   using C = GCfg<D>;
-  return static_cast<size_t>(ns) * C::STAGE + static_cast<size_t>(GQD) * C::QBLOBS + GQD * sizeof(SegQ) +
-         (2 * ns + 2 * GQD) * sizeof(uint64_t) + 16 + ns * sizeof(int);
+  return static_cast<size_t>(ns) * C::STAGE + GQD * sizeof(SegQ) + (2 * ns + 2 * GQD) * sizeof(uint64_t) +
+         sizeof(GMisc);
 }
 
 // Block-wide exclusive scan of one value per thread; returns the thread's prefix, *total the sum.
@@ -108,100 +126,311 @@ __device__ int block_exclusive_scan(int v, int* s_tmp, int* total) {
   return before;
 }
 
-// ---------------------------------------------------------------------------
-// planner: blocks 0..nq-1 build the query blobs (one warp per (sequence, KV
-// head)); the last block describes the head groups and the stream-K partition.
+// Head group i of the call: which positions are read from INT4 pages and which
+// from the INT8 store.
+__device__ Group describe(const AttnParams& p, int i, int HGN, bool flag_bad) {
+  Group g;
+  g.b = i / HGN;
+  g.hg = i - g.b * HGN;
+  g.seq = p.seq_ids[g.b];
+  int L = 0;
+  if (g.seq >= 0 && g.seq < p.max_seqs) L = p.seq_lens[g.seq];
+  else if (flag_bad && g.hg == 0) atomicOr(&p.state->status, KV4_DEV_BAD_SEQ);
+  g.L = L;
+  int lo4, hi4, nprot;
+  if (p.mode & KV4_MODE_INT4_ONLY) { lo4 = 0; hi4 = L; nprot = 0; }
+  else { nprot = min(L, p.S + p.W); lo4 = p.S; hi4 = L - p.W; }
+  g.lo4 = lo4; g.hi4 = hi4; g.nprot = nprot;
+  g.t0 = 0; g.n4 = 0;
+  if (hi4 > lo4) { g.t0 = lo4 / TILE; g.n4 = (hi4 + TILE - 1) / TILE - g.t0; }
+  g.n8 = (nprot + TILE - 1) / TILE;
+  g.start = 0;
+  g.pad = 0;
+  return g;
+}
 
-template <int D>
-__global__ void __launch_bounds__(1024) gprep_kernel(AttnParams p, Group* groups, int* cta_first, GHeader* hdr,
-                                                     int n_qblocks) {
-  extern __shared__ float s_q[];   // [32][G][D] for the query blocks, scan scratch for the planner
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  if (static_cast<int>(blockIdx.x) < n_qblocks) {
-    const int gw = blockIdx.x * (blockDim.x >> 5) + wib;
-    if (gw >= p.n_seqs * p.Hkv) return;
-    build_qblob<D, false>(p, gw / p.Hkv, gw % p.Hkv, lane, s_q + wib * p.G * D);
-    return;
-  }
-  // ---- the planner block
-  int* s_tmp = reinterpret_cast<int*>(s_q);
+// Zeros for the output rows of head group i (a sequence of length 0), elements e0, e0+step, ...
+__device__ void zero_group(const AttnParams& p, int i, int e0, int step) {
   const int HGN = p.Hkv / GW;
-  const int n_groups = p.n_seqs * HGN;
-  const int per = (n_groups + blockDim.x - 1) / blockDim.x;
-  const int i0 = threadIdx.x * per, i1 = min(i0 + per, n_groups);
-  auto describe = [&](int i) -> Group {
-    Group g{};
-    g.b = i / HGN;
-    g.hg = i % HGN;
-    g.seq = p.seq_ids[g.b];
-    int L = 0;
-    if (g.seq >= 0 && g.seq < p.max_seqs) L = p.seq_lens[g.seq];
-    else if (g.hg == 0) atomicOr(&p.state->status, KV4_DEV_BAD_SEQ);
-    int lo4, hi4, nprot;
-    if (p.mode & KV4_MODE_INT4_ONLY) { lo4 = 0; hi4 = L; nprot = 0; }
-    else { nprot = min(L, p.S + p.W); lo4 = p.S; hi4 = L - p.W; }
-    g.lo4 = lo4; g.hi4 = hi4; g.nprot = nprot;
-    g.t0 = 0; g.n4 = 0;
-    if (hi4 > lo4) { g.t0 = lo4 / TILE; g.n4 = (hi4 + TILE - 1) / TILE - g.t0; }
-    g.n8 = (nprot + TILE - 1) / TILE;
-    return g;
-  };
-  // pass 1: stage counts -> starts, total T
-  int local = 0;
-  for (int i = i0; i < i1; ++i) local += group_stages(describe(i));
-  int T = 0;
-  int start = block_exclusive_scan(local, s_tmp, &T);
-  // partition over min(grid, T) CTAs: every active CTA owns at least one stage, so
-  // the CTAs touching a group are exactly its consecutive segments
-  const long long N = T < p.grid ? T : p.grid;
-  // pass 2: segments per group -> segment bases
-  int segs = 0;
-  {
-    int st = start;
-    for (int i = i0; i < i1; ++i) {
-      const int n = group_stages(describe(i));
-      if (n > 0) segs += cta_of(st + n - 1, T, N) - cta_of(st, T, N) + 1;
-      st += n;
+  const int b = i / HGN, hg = i - b * HGN;
+  const long long base = (static_cast<long long>(b) * p.Hq + hg * GW * p.G) * p.D;
+  const int n = GW * p.G * p.D;
+  if (p.mode & KV4_MODE_OUT_F32) {
+    float* out = static_cast<float*>(p.out) + base;
+    for (int e = e0; e < n; e += step) out[e] = 0.f;
+  } else {
+    uint16_t* out = static_cast<uint16_t*>(p.out) + base;
+    for (int e = e0; e < n; e += step) out[e] = 0;
+  }
+}
+
+// Normalise, rotate back and store the output of one KV head: lane (g8, t)
+// holds o for heads 2t, 2t+1 (valid when < G) at dimensions 16m+g8 (o[m][0],
+// o[m][1]) and 16m+g8+8 (o[m][2], o[m][3]).  out = c_B * H_blk (o / l): the
+// normalised block Hadamard is its own inverse.
+template <int D>
+__device__ __forceinline__ void store_head(const AttnParams& p, int b, int hkv, int lane, float (&o)[D / 16][4],
+                                           float l0, float l1) {
+  constexpr int NM = D / 16;
+  const int g8 = lane >> 2, t = lane & 3;
+  const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+#pragma unroll
+  for (int m = 0; m < NM; ++m) { o[m][0] *= inv0; o[m][2] *= inv0; o[m][1] *= inv1; o[m][3] *= inv1; }
+  const int Bh = p.Bh;
+  // stages 1, 2, 4: dimension bits 0-2 are the lane bits 2-4
+#pragma unroll
+  for (int hh = 1; hh <= 4; hh <<= 1) {
+    if (hh < Bh) {
+      const bool upper = (g8 & hh) != 0;
+#pragma unroll
+      for (int m = 0; m < NM; ++m)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float other = __shfl_xor_sync(0xffffffffu, o[m][i], 4 * hh);
+          o[m][i] = upper ? other - o[m][i] : o[m][i] + other;
+        }
     }
   }
-  int n_segs = 0;
-  int segbase = block_exclusive_scan(segs, s_tmp, &n_segs);
-  // pass 3: write groups, the first group of every CTA, the per-(sequence, head) merge records
-  {
-    int st = start, sb = segbase;
-    for (int i = i0; i < i1; ++i) {
-      Group g = describe(i);
-      const int n = group_stages(g);
-      g.start = st;
-      g.segbase = sb;
-      g.c_first = n > 0 ? cta_of(st, T, N) : 0;
-      const int nseg = n > 0 ? cta_of(st + n - 1, T, N) - g.c_first + 1 : 0;
-      groups[i] = g;
-      if (n > 0) {
-        for (int c = g.c_first; c < g.c_first + nseg; ++c) {
-          const long long b0 = static_cast<long long>(c) * T / N;   // first stage of CTA c
-          if (b0 >= st && b0 < st + n) cta_first[c] = i;
+  // stage 8: dimension bit 3 (o[m][0..1] vs o[m][2..3])
+  if (8 < Bh) {
+#pragma unroll
+    for (int m = 0; m < NM; ++m)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float a = o[m][i], c = o[m][i + 2];
+        o[m][i] = a + c;
+        o[m][i + 2] = a - c;
+      }
+  }
+  // stages 16, 32, ...: dimension bits 4.. (m)
+#pragma unroll
+  for (int mb = 1; mb < NM; mb <<= 1) {
+    if (16 * mb < Bh) {
+#pragma unroll
+      for (int m = 0; m < NM; ++m)
+        if ((m & mb) == 0)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float a = o[m][i], c = o[m + mb][i];
+            o[m][i] = a + c;
+            o[m + mb][i] = a - c;
+          }
+    }
+  }
+  const float rc = p.rot_c;
+  const int G = p.G;
+#pragma unroll
+  for (int hp = 0; hp < 2; ++hp) {
+    const int head = 2 * t + hp;
+    if (head >= G) continue;
+    const long long row = (static_cast<long long>(b) * p.Hq + hkv * G + head) * D;
+    if (p.mode & KV4_MODE_OUT_F32) {
+      float* out = static_cast<float*>(p.out) + row;
+#pragma unroll
+      for (int m = 0; m < NM; ++m) {
+        out[16 * m + g8] = o[m][hp] * rc;
+        out[16 * m + g8 + 8] = o[m][hp + 2] * rc;
+      }
+    } else {
+      uint16_t* out = static_cast<uint16_t*>(p.out) + row;
+#pragma unroll
+      for (int m = 0; m < NM; ++m) {
+        out[16 * m + g8] = __bfloat16_as_ushort(__float2bfloat16_rn(o[m][hp] * rc));
+        out[16 * m + g8 + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(o[m][hp + 2] * rc));
+      }
+    }
+  }
+}
+
+// The partials of one KV head of a split group: segment k lives on CTA cf + k,
+// in that CTA's slot 0 (its first segment) or slot 1 (its last segment).
+struct PartRef {
+  const float* base;
+  int cf, first_is_last, w, pstride;
+  __device__ __forceinline__ const float* operator()(int k) const {
+    const int sl = (k == 0 && first_is_last) ? 1 : 0;
+    return base + static_cast<size_t>(((cf + k) * 2 + sl) * GW + w) * pstride;
+  }
+};
+
+// Merge of the nseg partials of one KV head (G query heads) and store, lane
+// major: lane l holds dimensions VPL*l .. VPL*l+VPL-1 of every head.  The
+// maxima and the denominators take one pass with a segment per lane; the
+// numerators then stream the partials with U segments' loads in flight, the
+// weight of each segment broadcast from the lane that computed it.
+template <int D, int GG>
+__device__ __noinline__ void merge_store(const AttnParams& p, const PartRef& parts, int nseg, int b, int hkv,
+                                         int lane, bool dry) {
+  constexpr int VPL = D / 32;
+  constexpr int HS = head_stride(D);
+  constexpr int U = GG >= 16 ? 1 : 16 / GG;
+  float M[GG], Lh[GG], acc[GG][VPL];
+#pragma unroll
+  for (int h = 0; h < GG; ++h) {
+    M[h] = NEG_INF;
+    Lh[h] = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc[h][i] = 0.f;
+  }
+  auto load_o = [&](const float* r, int h, float (&v)[VPL]) {
+    if constexpr (VPL == 4) {
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(r + h * HS) + lane);
+      v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    } else {
+      const float2 x = __ldcg(reinterpret_cast<const float2*>(r + h * HS) + lane);
+      v[0] = x.x; v[1] = x.y;
+    }
+  };
+  if (nseg <= U) {
+    // one batch of loads: every partial at once
+    float mv[U][GG], lv[U][GG], v[U][GG][VPL];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float* r = parts(min(u, nseg - 1));
+#pragma unroll
+      for (int h = 0; h < GG; ++h) {
+        mv[u][h] = __ldcg(r + h * HS + D);
+        lv[u][h] = __ldcg(r + h * HS + D + 1);
+        load_o(r, h, v[u][h]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int h = 0; h < GG; ++h) M[h] = fmaxf(M[h], mv[u][h]);
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int h = 0; h < GG; ++h) {
+        const float f = u < nseg ? ex2(mv[u][h] - M[h]) : 0.f;
+        Lh[h] = fmaf(f, lv[u][h], Lh[h]);
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) acc[h][i] = fmaf(f, v[u][h][i], acc[h][i]);
+      }
+  } else {
+    // maxima with one segment per lane (the first 32 segments' m, l stay in registers)
+    float m0[GG], l0[GG];
+#pragma unroll
+    for (int h = 0; h < GG; ++h) { m0[h] = NEG_INF; l0[h] = 0.f; }
+    if (lane < nseg) {
+      const float* r = parts(lane);
+#pragma unroll
+      for (int h = 0; h < GG; ++h) { m0[h] = __ldcg(r + h * HS + D); l0[h] = __ldcg(r + h * HS + D + 1); M[h] = m0[h]; }
+    }
+    for (int k = lane + 32; k < nseg; k += 32) {
+      const float* r = parts(k);
+#pragma unroll
+      for (int h = 0; h < GG; ++h) M[h] = fmaxf(M[h], __ldcg(r + h * HS + D));
+    }
+#pragma unroll
+    for (int h = 0; h < GG; ++h)
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) M[h] = fmaxf(M[h], __shfl_xor_sync(0xffffffffu, M[h], o));
+    for (int k0 = 0; k0 < nseg; k0 += 32) {
+      float fr[GG];
+      const int k = k0 + lane;
+      if (k0 > 0 && k < nseg) {
+        const float* r = parts(k);
+#pragma unroll
+        for (int h = 0; h < GG; ++h) { m0[h] = __ldcg(r + h * HS + D); l0[h] = __ldcg(r + h * HS + D + 1); }
+      }
+#pragma unroll
+      for (int h = 0; h < GG; ++h) {
+        fr[h] = k < nseg ? ex2(m0[h] - M[h]) : 0.f;
+        Lh[h] = fmaf(fr[h], k < nseg ? l0[h] : 0.f, Lh[h]);
+      }
+      const int cnt = min(32, nseg - k0);
+      for (int kk = 0; kk < cnt; kk += U) {
+        float v[U][GG][VPL];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const float* r = parts(k0 + min(kk + u, cnt - 1));
+#pragma unroll
+          for (int h = 0; h < GG; ++h) load_o(r, h, v[u][h]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+#pragma unroll
+          for (int h = 0; h < GG; ++h) {
+            float f = __shfl_sync(0xffffffffu, fr[h], (kk + u) & 31);
+            if (kk + u >= cnt) f = 0.f;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) acc[h][i] = fmaf(f, v[u][h][i], acc[h][i]);
+          }
         }
       }
-      const int L = g.seq >= 0 && g.seq < p.max_seqs ? p.seq_lens[g.seq] : 0;
-      for (int w = 0; w < GW; ++w) {
-        SeqHead sh;
-        sh.part_base = (sb * GW + w);
-        sh.n_parts = nseg;
-        sh.len = L;
-        sh.pad = GW;   // stride between the segments' partials of one head
-        p.seqhead[g.b * p.Hkv + g.hg * GW + w] = sh;
-      }
-      if ((sb + nseg) * GW > p.cap_parts) atomicOr(&p.state->status, KV4_DEV_WORKSPACE);
-      st += n;
-      sb += nseg;
+    }
+#pragma unroll
+    for (int h = 0; h < GG; ++h)
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) Lh[h] += __shfl_xor_sync(0xffffffffu, Lh[h], o);
+  }
+  const float rc = p.rot_c;
+  const int Bh = p.Bh;
+#pragma unroll
+  for (int h = 0; h < GG; ++h) {
+    float o[VPL];
+    const float inv = Lh[h] > 0.f ? 1.f / Lh[h] : 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) o[i] = acc[h][i] * inv;
+    fwht_row<VPL>(o, Bh, lane);   // o = H_blk o_rot (the normalised block Hadamard is its own inverse)
+    const long long off = (static_cast<long long>(b) * p.Hq + hkv * GG + h) * D + VPL * lane;
+    if (dry) continue;
+    if (p.mode & KV4_MODE_OUT_F32) {
+      float* out = static_cast<float*>(p.out) + off;
+      if constexpr (VPL == 4) *reinterpret_cast<float4*>(out) = make_float4(o[0] * rc, o[1] * rc, o[2] * rc, o[3] * rc);
+      else *reinterpret_cast<float2*>(out) = make_float2(o[0] * rc, o[1] * rc);
+    } else {
+      uint16_t* out = static_cast<uint16_t*>(p.out) + off;
+      if constexpr (VPL == 4)
+        *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf162(o[0] * rc, o[1] * rc), pack_bf162(o[2] * rc, o[3] * rc));
+      else
+        *reinterpret_cast<uint32_t*>(out) = pack_bf162(o[0] * rc, o[1] * rc);
     }
   }
-  if (threadIdx.x == 0) {
-    hdr->T = T;
-    hdr->N = static_cast<int>(N);
-    hdr->n_groups = n_groups;
+}
+
+template <int D>
+__device__ __forceinline__ void merge_store_g(const AttnParams& p, const PartRef& parts, int nseg, int b, int hkv,
+                                              int lane, bool dry = false) {
+  switch (p.G) {
+    case 1: merge_store<D, 1>(p, parts, nseg, b, hkv, lane, dry); break;
+    case 2: merge_store<D, 2>(p, parts, nseg, b, hkv, lane, dry); break;
+    case 3: merge_store<D, 3>(p, parts, nseg, b, hkv, lane, dry); break;
+    case 4: merge_store<D, 4>(p, parts, nseg, b, hkv, lane, dry); break;
+    case 5: merge_store<D, 5>(p, parts, nseg, b, hkv, lane, dry); break;
+    case 6: merge_store<D, 6>(p, parts, nseg, b, hkv, lane, dry); break;
+    case 7: merge_store<D, 7>(p, parts, nseg, b, hkv, lane, dry); break;
+    default: merge_store<D, 8>(p, parts, nseg, b, hkv, lane, dry); break;
   }
+}
+
+
+// ---------------------------------------------------------------------------
+// query operands: one warp per (batch entry, KV head) rotates its G query
+// heads and stores the tensor-core B fragments (16 B per lane and 16-dim pair),
+// sum(q) per fragment column and the exponent scale.  The attention kernel is
+// launched as its programmatic dependent, so it plans and starts streaming
+// pages while this runs, and waits for it only before the first operand read.
+
+constexpr int QWARPS = 4;
+
+template <int D>
+__global__ void __launch_bounds__(32 * QWARPS) gq_kernel(AttnParams p) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * QWARPS + (threadIdx.x >> 5);
+  if (gw >= p.n_seqs * p.Hkv) return;
+  QFrag<D> qf;
+  load_qfrag<D>(p, gw / p.Hkv, gw % p.Hkv, lane, qf);
+  uint8_t* blob = p.qblob + static_cast<size_t>(gw) * qblob_bytes(D);
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc)
+    reinterpret_cast<uint4*>(blob)[cc * 32 + lane] =
+        make_uint4(qf.b[2 * cc][0], qf.b[2 * cc][1], qf.b[2 * cc + 1][0], qf.b[2 * cc + 1][1]);
+  float* tail = reinterpret_cast<float*>(blob + 16 * D);
+  if (lane < 4) { tail[2 * lane] = qf.qs0; tail[2 * lane + 1] = qf.qs1; }   // lanes 0-3: columns 2t, 2t+1
+  if (lane == 0) tail[MAX_G] = qf.kscale;
 }
 
 // ---------------------------------------------------------------------------
@@ -228,68 +457,151 @@ __device__ __forceinline__ const uint8_t* stage_source(const AttnParams& p, cons
                       tile8_bytes(D);
 }
 
+// Every warp of the CTA calls this once on its way out.  The last warp of the
+// CTA counts the CTA done; the last CTA of the launch re-arms the launch
+// counter and, if any CTA gave up a wait (its merges may be incomplete),
+// zeroes every merge counter.
+__device__ __forceinline__ void warp_exit(const AttnParams& p, unsigned long long* merge_ctr, GMisc* misc,
+                                          int lane) {
+  __syncwarp();
+  int last = 0;
+  if (lane == 0 && atomicAdd(&misc->exited, 1) == GW) {
+    if (misc->abort) atomicExch(&p.state->ctr_dirty, 1);
+    __threadfence();
+    last = atomicAdd(&p.state->cta_done, 1) == static_cast<int>(gridDim.x) - 1;
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __threadfence();
+  if (*reinterpret_cast<volatile int*>(&p.state->ctr_dirty)) {
+    const int n = p.max_seqs * p.Hkv;
+    for (int i = lane; i < n; i += 32) merge_ctr[i] = 0ull;
+    __syncwarp();
+    if (lane == 0) p.state->ctr_dirty = 0;
+  }
+  if (lane == 0) p.state->cta_done = 0;
+}
+
 // PAIR = INT4 tiles per iteration of a consumer warp: 2 (more independent work
 // per warp, 1 CTA per SM) or 1 (fewer registers, 2 CTAs per SM).
 template <int D, int PAIR>
-__global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p, const Group* groups,
-                                                                   const int* cta_first, const GHeader* hdr) {
+__global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p, unsigned long long* merge_ctr) {
   using C = GCfg<D>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int NS = p.ns;
   uint8_t* ring = smem;
-  uint8_t* qbuf = ring + static_cast<size_t>(NS) * C::STAGE;
-  SegQ* segq = reinterpret_cast<SegQ*>(qbuf + GQD * C::QBLOBS);
+  SegQ* segq = reinterpret_cast<SegQ*>(ring + static_cast<size_t>(NS) * C::STAGE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(segq + GQD);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * NS + 2 * GQD);
-  int* last_fill = const_cast<int*>(abort_flag) + 4;
+  GMisc* misc = reinterpret_cast<GMisc*>(bars + 2 * NS + 2 * GQD);
+  volatile int* abort_flag = &misc->abort;
   const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * NS;
   const uint32_t iqf0 = full0 + 16 * NS, iqe0 = iqf0 + 8 * GQD;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int* status = &p.state->status;
+  const int c = blockIdx.x;
+  const int HGN = p.Hkv / GW, n_groups = p.n_seqs * HGN;
 
-  const long long T = hdr->T, N = hdr->N;   // N = min(grid, T) active CTAs
-  const long long c = blockIdx.x;
-  if (c >= N) return;   // uniform over the CTA
-  const int j0 = static_cast<int>(c * T / N), j1 = static_cast<int>((c + 1) * T / N);
-  if (j0 >= j1) return;
-
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     for (int s = 0; s < NS; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, GW); }
     for (int s = 0; s < GQD; ++s) { mbar_init(iqf0 + 8 * s, 1); mbar_init(iqe0 + 8 * s, GW); }
-    *abort_flag = 0;
-    for (int s = 0; s < NS; ++s) last_fill[s] = -1;
+    misc->abort = 0;
+    misc->exited = 0;
+    misc->n_empty = 0;
+    for (int s = 0; s < MAX_NS; ++s) misc->last_fill[s] = -1;
     fence_barrier_init();
   }
+
+  // ---- plan (every CTA the same): stage counts of all head groups -> T, then
+  // the stream-K range [j0, j1) of this CTA and the group holding j0
+  Group my_g{};
+  int my_start = 0, T = 0;
+  for (int c0 = 0; c0 < n_groups; c0 += GTHREADS) {
+    const int i = c0 + tid;
+    Group gd{};
+    if (i < n_groups) gd = describe(p, i, HGN, c == 0);
+    int tot;
+    const int ex = block_exclusive_scan(group_stages(gd), misc->red, &tot);
+    if (c0 == 0) { my_g = gd; my_start = ex; }
+    T += tot;
+  }
+  long long N = (T + MIN_STAGES - 1) / MIN_STAGES;   // active CTAs: each owns at least one stage
+  if (N > p.grid) N = p.grid;
+  const bool zero_all = T == 0;
+  const int j0 = zero_all ? 0 : static_cast<int>(c * static_cast<long long>(T) / N);
+  const int j1 = zero_all ? 0 : static_cast<int>((c + 1) * static_cast<long long>(T) / N);
+  auto visit = [&](int i, const Group& gd, int st) {
+    if (i >= n_groups) return;
+    const int n = group_stages(gd);
+    if (n > 0) {
+      if (st <= j0 && j0 < st + n) {
+        misc->first = gd;
+        misc->first.start = st;
+      }
+    } else {
+      const int owner = zero_all ? 0 : cta_of(min(st, T - 1), T, N);
+      if (owner == c) {
+        const int k = atomicAdd(&misc->n_empty, 1);
+        if (k < 32) misc->empty[k] = i;
+        else zero_group(p, i, 0, 1);
+      }
+    }
+  };
+  if (n_groups <= GTHREADS) {
+    visit(tid, my_g, my_start);
+  } else {
+    int base = 0;
+    for (int c0 = 0; c0 < n_groups; c0 += GTHREADS) {
+      const int i = c0 + tid;
+      Group gd{};
+      if (i < n_groups) gd = describe(p, i, HGN, false);
+      int tot;
+      const int ex = block_exclusive_scan(group_stages(gd), misc->red, &tot);
+      visit(i, gd, base + ex);
+      base += tot;
+    }
+  }
   __syncthreads();
+  {
+    const int ne = min(misc->n_empty, 32);
+    for (int e = 0; e < ne; ++e) zero_group(p, misc->empty[e], tid, GTHREADS);
+  }
+  if (zero_all || c >= N || j0 >= j1) {
+    warp_exit(p, merge_ctr, misc, lane);
+    return;
+  }
 
   if (warp == GW) {
     // ------------------------------------------------------------ producer
     const int nbatch = NS < 32 ? NS : 32;
-    int gi = cta_first[c];
-    Group g = groups[gi];
+    Group g = misc->first;
+    int gi = g.b * HGN + g.hg;
     int u = j0 - g.start;
     int j = j0;
     uint32_t jj = 0;   // CTA-local stage counter
     int q = 0;
     bool ok = true;
     while (j < j1 && ok) {
-      const int n = min(g.start + group_stages(g) - j, j1 - j);
+      const int gst = group_stages(g);
+      const int n = min(g.start + gst - j, j1 - j);
       const int slot = q % GQD;
       if (lane == 0) ok = mbar_wait(iqe0 + 8 * slot, ((q / GQD) & 1) ^ 1, abort_flag, status);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       if (lane == 0) {
         SegQ sq;
-        sq.g = g; sq.u0 = u; sq.n = n; sq.k = static_cast<int>(c) - g.c_first; sq.pad = 0;
+        sq.g = g;
+        sq.u0 = u;
+        sq.n = n;
+        const int cf = cta_of(g.start, T, N);
+        sq.k = c - cf;
+        sq.nseg = cta_of(g.start + gst - 1, T, N) - cf + 1;
         segq[slot] = sq;
-        mbar_arrive_expect_tx(iqf0 + 8 * slot, C::QBLOBS);
-        bulk_g2s(smem_u32(qbuf + slot * C::QBLOBS),
-                 p.qblob + static_cast<size_t>(g.b * p.Hkv + g.hg * GW) * qblob_bytes(D), C::QBLOBS, iqf0 + 8 * slot);
+        mbar_arrive(iqf0 + 8 * slot);
       }
-      // the next group with stages (its descriptor load overlaps the copies below)
+      // the next group's descriptor (its loads overlap the copies below)
       int gn = gi + 1;
       Group nxt{};
-      if (j + n < j1) nxt = groups[gn];
+      if (j + n < j1) nxt = describe(p, gn, HGN, false);
       // stages u .. u+n-1: one lane per stage, batches of at most NS stages
       for (int base = 0; base < n; base += nbatch) {
         bool lane_ok = true;
@@ -302,7 +614,7 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
           if (lane_ok) {
             mbar_arrive_expect_tx(full0 + 8 * s, bytes);
             bulk_g2s(smem_u32(ring + static_cast<size_t>(s) * C::STAGE), src, bytes, full0 + 8 * s);
-            last_fill[s] = static_cast<int>(jl);
+            misc->last_fill[s] = static_cast<int>(jl);
           } else {
             *abort_flag = 1;
           }
@@ -313,8 +625,10 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
       jj += n;
       j += n;
       ++q;
-      if (j < j1) {
-        while (group_stages(nxt) == 0) nxt = groups[++gn];   // skip empty sequences
+      if (j < j1 && ok) {
+        const int next_start = g.start + gst;
+        while (group_stages(nxt) == 0) nxt = describe(p, ++gn, HGN, false);   // empty sequences own no stage
+        nxt.start = next_start;
         gi = gn;
         g = nxt;
         u = 0;
@@ -324,14 +638,18 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
       const int slot = q % GQD;
       if (lane == 0) ok = mbar_wait(iqe0 + 8 * slot, ((q / GQD) & 1) ^ 1, abort_flag, status);
       if (lane == 0 && ok) { segq[slot].n = -1; mbar_arrive(iqf0 + 8 * slot); }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
     }
     if (!ok && lane == 0) {
+      // let the copies in flight land before the CTA's shared memory goes away
       for (int st = 0; st < NS; ++st)
-        if (last_fill[st] >= 0) {
+        if (misc->last_fill[st] >= 0) {
           const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(full0 + 8 * st, (last_fill[st] / NS) & 1) && globaltimer_ns() - t0 < 1000000000ull) {}
+          while (!mbar_try_wait(full0 + 8 * st, (misc->last_fill[st] / NS) & 1) &&
+                 globaltimer_ns() - t0 < 1000000000ull) {}
         }
     }
+    warp_exit(p, merge_ctr, misc, lane);
     return;
   }
 
@@ -340,10 +658,12 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
   const int g8 = lane >> 2, t = lane & 3;
   const int G = p.G;
   constexpr int HS = head_stride(D);
+  const int pstride = partial_stride(G, D);
   ColSplit cs;
   cs.colsplit = (G == 1 || G == 2 || G == 4);
   cs.part0 = cs.colsplit ? (2 * t) / G : 0;
   cs.part1 = cs.colsplit ? (2 * t + 1) / G : 0;
+  const int h0 = 2 * t, h1 = 2 * t + 1;
   int s = 0;          // stage of the next CTA-local stage index
   uint32_t par = 0;   // its fill parity
   auto advance = [&]() {
@@ -353,22 +673,24 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
     const int slot = q % GQD;
     if (!mbar_wait(iqf0 + 8 * slot, (q / GQD) & 1, abort_flag, status)) break;
     const SegQ sq = segq[slot];
-    if (sq.n < 0) break;
-    QFrag<D> qf;
-    {
-      const uint32_t qb = smem_u32(qbuf + slot * C::QBLOBS + w * qblob_bytes(D));
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        const uint4 v = lds128(qb + 16 * (32 * cc + lane));
-        qf.b[2 * cc][0] = v.x; qf.b[2 * cc][1] = v.y; qf.b[2 * cc + 1][0] = v.z; qf.b[2 * cc + 1][1] = v.w;
-      }
-      const float* tail = reinterpret_cast<const float*>(qbuf + slot * C::QBLOBS + w * qblob_bytes(D) + 16 * D);
-      qf.qs0 = tail[(2 * t) & 7];
-      qf.qs1 = tail[(2 * t + 1) & 7];
-      qf.kscale = tail[MAX_G];
-    }
     __syncwarp();
     if (lane == 0) mbar_arrive(iqe0 + 8 * slot);
+    if (sq.n < 0) break;
+    const Group& g = sq.g;
+    if (q == 0) asm volatile("griddepcontrol.wait;" ::: "memory");   // the query operands are written
+    QFrag<D> qf;
+    {
+      const uint8_t* blob = p.qblob + static_cast<size_t>(g.b * p.Hkv + g.hg * GW + w) * qblob_bytes(D);
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(blob) + 32 * cc + lane);
+        qf.b[2 * cc][0] = v.x; qf.b[2 * cc][1] = v.y; qf.b[2 * cc + 1][0] = v.z; qf.b[2 * cc + 1][1] = v.w;
+      }
+      const float* tail = reinterpret_cast<const float*>(blob + 16 * D);
+      qf.qs0 = __ldcg(tail + 2 * t);
+      qf.qs1 = __ldcg(tail + 2 * t + 1);
+      qf.kscale = __ldcg(tail + MAX_G);
+    }
 
     WarpState<D> ws;
 #pragma unroll
@@ -376,7 +698,6 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
     ws.m0 = ws.m1 = NEG_INF;
     ws.l0 = ws.l1 = ws.z0 = ws.z1 = 0.f;
 
-    const Group& g = sq.g;
     const int u_end = sq.u0 + sq.n;
     bool ok = true;
     for (int u = sq.u0; u < u_end && ok;) {
@@ -436,7 +757,7 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
     }
     if (!ok) break;
 
-    // ---- this warp's partial for the segment
+    // ---- the segment's result for this warp's head
     if (cs.colsplit) {
       if (G == 1) {
 #pragma unroll
@@ -456,52 +777,74 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
       ws.z0 += __shfl_xor_sync(0xffffffffu, ws.z0, o);
       ws.z1 += __shfl_xor_sync(0xffffffffu, ws.z1, o);
     }
-    const int slotp = (g.segbase + sq.k) * GW + w;
-    if (slotp < p.cap_parts) {
-      float* part = p.partials + static_cast<size_t>(slotp) * partial_stride(G, D);
-      const int h0 = 2 * t, h1 = 2 * t + 1;
+#pragma unroll
+    for (int m = 0; m < D / 16; ++m) { ws.o[m][0] += ws.z0; ws.o[m][2] += ws.z0; ws.o[m][1] += ws.z1; ws.o[m][3] += ws.z1; }
+    const int hkv = g.hg * GW + w;
+    if (sq.nseg == 1) {
+      store_head<D>(p, g.b, hkv, lane, ws.o, ws.l0, ws.l1);
+      continue;
+    }
+    // several CTAs share the group: partial to the workspace (slot 0 = this
+    // CTA's first segment, slot 1 = its last), the last to arrive merges
+    {
+      const int slotp = (c * 2 + (q == 0 ? 0 : 1)) * GW + w;
+      float* part = p.partials + static_cast<size_t>(slotp) * pstride;
       if (h0 < G) {
         float* r = part + h0 * HS;
 #pragma unroll
-        for (int m = 0; m < D / 16; ++m) { r[16 * m + g8] = ws.o[m][0] + ws.z0; r[16 * m + g8 + 8] = ws.o[m][2] + ws.z0; }
+        for (int m = 0; m < D / 16; ++m) { r[16 * m + g8] = ws.o[m][0]; r[16 * m + g8 + 8] = ws.o[m][2]; }
         if (g8 == 0) { r[D] = ws.m0; r[D + 1] = ws.l0; }
       }
       if (h1 < G) {
         float* r = part + h1 * HS;
 #pragma unroll
-        for (int m = 0; m < D / 16; ++m) { r[16 * m + g8] = ws.o[m][1] + ws.z1; r[16 * m + g8 + 8] = ws.o[m][3] + ws.z1; }
+        for (int m = 0; m < D / 16; ++m) { r[16 * m + g8] = ws.o[m][1]; r[16 * m + g8 + 8] = ws.o[m][3]; }
         if (g8 == 0) { r[D] = ws.m1; r[D + 1] = ws.l1; }
       }
     }
+    __threadfence();
+    __syncwarp();
+    unsigned long long* ctr = merge_ctr + static_cast<size_t>(g.b) * p.Hkv + hkv;
+    int arrived = 0;
+    if (lane == 0) arrived = static_cast<int>(atomicAdd(ctr, 1ull)) + 1;
+    arrived = __shfl_sync(0xffffffffu, arrived, 0);
+    if (arrived != sq.nseg) continue;
+    if (lane == 0) *ctr = 0ull;   // every other segment has arrived: re-arm for the next call
+    __threadfence();
+    const int cf = c - sq.k;
+    PartRef pr;
+    pr.base = p.partials;
+    pr.cf = cf;
+    pr.first_is_last = g.start != static_cast<int>(cf * static_cast<long long>(T) / N);
+    pr.w = w;
+    pr.pstride = pstride;
+    merge_store_g<D>(p, pr, sq.nseg, g.b, hkv, lane);
   }
+  warp_exit(p, merge_ctr, misc, lane);
 }
 
 // ---------------------------------------------------------------------------
 // host side
 
-struct GLayout {
-  size_t seqhead, qblob, hdr, groups, cta_first, partials, total;
-  int cap_parts;
-};
-
 inline size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Grid of the kernel variant in use (CTAs per SM x SMs).
+inline int g_grid(const kv4_cache* c) { return c->num_sms * (c->gattn_pair == 1 ? 2 : 1); }
+
+// Workspace: the query operands of every (batch entry, KV head), then two
+// partial slots per CTA and KV head of a group (the CTA's first and last
+// segment; segments in between cover whole groups and need none).
+struct GLayout {
+  size_t qblob, partials, total;
+};
 
 GLayout g_layout(const kv4_cache* c, int n_seqs) {
   const kv4_config& cfg = c->cfg;
-  const int G = cfg.num_q_heads / cfg.num_kv_heads, D = cfg.head_dim;
-  const size_t nsh = static_cast<size_t>(n_seqs) * cfg.num_kv_heads;
-  const size_t ngroups = static_cast<size_t>(n_seqs) * (cfg.num_kv_heads / GW);
-  const size_t N = static_cast<size_t>(c->num_sms) * 2;   // upper bound of the grid over both variants
+  const int G = cfg.num_q_heads / cfg.num_kv_heads;
   GLayout l{};
-  l.cap_parts = static_cast<int>((N + ngroups) * GW);
-  size_t off = 0;
-  l.seqhead = off; off = al256(off + nsh * sizeof(SeqHead));
-  l.qblob = off; off = al256(off + nsh * qblob_bytes(D));
-  l.hdr = off; off = al256(off + sizeof(GHeader));
-  l.groups = off; off = al256(off + ngroups * sizeof(Group));
-  l.cta_first = off; off = al256(off + N * sizeof(int));
-  l.partials = off; off = al256(off + static_cast<size_t>(l.cap_parts) * partial_stride(G, D) * sizeof(float));
-  l.total = off;
+  l.qblob = 0;
+  l.partials = al256(static_cast<size_t>(n_seqs) * cfg.num_kv_heads * qblob_bytes(cfg.head_dim));
+  l.total = l.partials + al256(static_cast<size_t>(g_grid(c)) * 2 * GW * partial_stride(G, cfg.head_dim) * sizeof(float));
   return l;
 }
 
@@ -513,7 +856,7 @@ int g_choose_ring(int device) {
   if (cudaFuncSetAttribute(gattn_kernel<D, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess)
     return -1;
   const int want = PAIR == 1 ? 2 : 1;
-  for (int ns = 16; ns >= 2; --ns) {
+  for (int ns = MAX_NS; ns >= 2; --ns) {
     const size_t smem = gattn_smem_bytes<D>(ns);
     if (smem > static_cast<size_t>(optin)) continue;
     int blocks = 0;
@@ -525,35 +868,32 @@ int g_choose_ring(int device) {
 }
 
 template <int D>
-int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, void (*merge)(const AttnParams&, cudaStream_t)) {
+int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream) {
   const GLayout l = g_layout(c, p.n_seqs);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  p.seqhead = reinterpret_cast<SeqHead*>(wsb + l.seqhead);
   p.qblob = wsb + l.qblob;
   p.partials = reinterpret_cast<float*>(wsb + l.partials);
-  p.cap_parts = l.cap_parts;
-  const int per_sm = c->gattn_pair == 1 ? 2 : 1;
-  p.grid = c->num_sms * per_sm;
+  p.grid = g_grid(c);
+  p.cap_parts = p.grid * 2 * GW;
   p.ns = c->gattn_ring;
-  Group* groups = reinterpret_cast<Group*>(wsb + l.groups);
-  int* cta_first = reinterpret_cast<int*>(wsb + l.cta_first);
-  GHeader* hdr = reinterpret_cast<GHeader*>(wsb + l.hdr);
-  const int nsh = p.n_seqs * p.Hkv;
-  const int n_qblocks = (nsh + 31) / 32;
-  const size_t prep_smem = static_cast<size_t>(32) * p.G * D * sizeof(float);
-  if (prep_smem > 48 * 1024 &&
-      cudaFuncSetAttribute(gprep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(prep_smem)) !=
-          cudaSuccess)
-    return KV4_ERR_CUDA;
-  gprep_kernel<D><<<n_qblocks + 1, 1024, prep_smem, stream>>>(p, groups, cta_first, hdr, n_qblocks);
   if (c->ev_before) cudaEventRecord(c->ev_before, stream);
-  if (c->gattn_pair == 1)
-    gattn_kernel<D, 1><<<p.grid, GTHREADS, gattn_smem_bytes<D>(p.ns), stream>>>(p, groups, cta_first, hdr);
-  else
-    gattn_kernel<D, 2><<<p.grid, GTHREADS, gattn_smem_bytes<D>(p.ns), stream>>>(p, groups, cta_first, hdr);
+  const int pairs = p.n_seqs * p.Hkv;
+  gq_kernel<D><<<(pairs + QWARPS - 1) / QWARPS, 32 * QWARPS, 0, stream>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.grid);
+  cfg.blockDim = dim3(GTHREADS);
+  cfg.dynamicSmemBytes = gattn_smem_bytes<D>(p.ns);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  if (c->gattn_pair == 1) e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, 1>, p, c->merge_ctr);
+  else e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, 2>, p, c->merge_ctr);
   if (c->ev_after) cudaEventRecord(c->ev_after, stream);
-  merge(p, stream);
-  return cudaGetLastError() == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
 
 }  // namespace
@@ -573,11 +913,11 @@ int grouped_ring(kv4_cache* c) {
 
 size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs) { return g_layout(c, n_seqs).total; }
 
-int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes, cudaStream_t stream,
-                   void (*merge)(const AttnParams&, cudaStream_t)) {
+int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (ws_bytes < g_layout(c, p.n_seqs).total) return KV4_ERR_WORKSPACE;
-  if (c->gattn_ring <= 0) return KV4_ERR_UNSUPPORTED;
-  return p.D == 128 ? g_launch<128>(c, p, ws, stream, merge) : g_launch<64>(c, p, ws, stream, merge);
+  if (c->gattn_ring <= 0 || c->gattn_ring > MAX_NS || !c->merge_ctr) return KV4_ERR_UNSUPPORTED;
+  if (p.n_seqs > c->cfg.max_seqs) return KV4_ERR_INVALID_ARG;
+  return p.D == 128 ? g_launch<128>(c, p, ws, stream) : g_launch<64>(c, p, ws, stream);
 }
 
 }  // namespace kv4

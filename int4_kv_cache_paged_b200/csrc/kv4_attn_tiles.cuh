@@ -381,25 +381,7 @@ __device__ __forceinline__ void build_qblob(const AttnParams& p, int b, int h, i
 #pragma unroll
     for (int i = 0; i < VPL; ++i) x[i] = __bfloat162float(__ushort_as_bfloat16(src[VPL * lane + i]));
     if constexpr (!BF16) {
-      for (int hh = 1; hh < p.Bh; hh <<= 1) {
-        if (hh < VPL) {
-#pragma unroll
-          for (int i = 0; i < VPL; ++i)
-            if ((i & hh) == 0) {
-              const float a = x[i], c = x[i + hh];
-              x[i] = __fadd_rn(a, c);
-              x[i + hh] = __fsub_rn(a, c);
-            }
-        } else {
-          const int lm = hh / VPL;
-          const bool upper = (lane & lm) != 0;
-#pragma unroll
-          for (int i = 0; i < VPL; ++i) {
-            const float o = __shfl_xor_sync(0xffffffffu, x[i], lm);
-            x[i] = upper ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
-          }
-        }
-      }
+      fwht_row<VPL>(x, p.Bh, lane);
 #pragma unroll
       for (int i = 0; i < VPL; ++i) x[i] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(x[i], rot_c)));
     }
@@ -460,6 +442,122 @@ __device__ __forceinline__ void build_qblob(const AttnParams& p, int b, int h, i
     tail[lane] = BF16 ? 0.f : v * p.scale_log2;
   }
   if (lane == MAX_G) tail[MAX_G] = ldexpf(p.scale_log2, -e);
+}
+
+
+// The query operand of KV head h of batch entry b, built straight into the
+// registers of the 16x8x16 B fragments (no staging through memory).  Lane
+// (g8 = lane/4, t = lane%4) holds column g8 (query head g8 % G with the column
+// split, else g8, zero when that head does not exist) at dimensions
+// d = 16k + 8r + 2t + e, e in {0, 1}: dimension bits 0, 3 and 4.. are in-lane,
+// bits 1 and 2 are the lane bits 0 and 1.  The block-diagonal Hadamard runs in
+// ascending butterfly stages with the same fp32 operations as the rotation of
+// the keys, so q_rot is the same bf16 vector whichever lane holds it.
+template <int D>
+__device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, int lane, QFrag<D>& qf) {
+  constexpr int NK = D / 16;
+  const int G = p.G, g8 = lane >> 2, t = lane & 3;
+  const bool colsplit = (G == 1 || G == 2 || G == 4);
+  const int gsrc = colsplit ? g8 % G : g8;
+  const bool active = gsrc < G;
+  const uint16_t* src = p.q + (static_cast<long long>(b) * p.Hq + h * G + (active ? gsrc : 0)) * D + 2 * t;
+  float x[NK][2][2];
+#pragma unroll
+  for (int k = 0; k < NK; ++k)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const uint32_t w = active ? __ldg(reinterpret_cast<const unsigned int*>(src + 16 * k + 8 * r)) : 0u;
+      x[k][r][0] = __uint_as_float(w << 16);
+      x[k][r][1] = __uint_as_float(w & 0xFFFF0000u);
+    }
+  const int Bh = p.Bh;
+  // stage 1: dimension bit 0 (the two halves of one 32-bit word)
+  if (1 < Bh) {
+#pragma unroll
+    for (int k = 0; k < NK; ++k)
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const float a = x[k][r][0], c = x[k][r][1];
+        x[k][r][0] = __fadd_rn(a, c);
+        x[k][r][1] = __fsub_rn(a, c);
+      }
+  }
+  // stages 2 and 4: dimension bits 1 and 2 live in lane bits 0 and 1
+#pragma unroll
+  for (int lm = 1; lm <= 2; lm <<= 1) {
+    if (2 * lm < Bh) {
+      const bool upper = (t & lm) != 0;
+#pragma unroll
+      for (int k = 0; k < NK; ++k)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float o = __shfl_xor_sync(0xffffffffu, x[k][r][e], lm);
+            x[k][r][e] = upper ? __fsub_rn(o, x[k][r][e]) : __fadd_rn(x[k][r][e], o);
+          }
+    }
+  }
+  // stage 8: dimension bit 3 (r)
+  if (8 < Bh) {
+#pragma unroll
+    for (int k = 0; k < NK; ++k)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float a = x[k][0][e], c = x[k][1][e];
+        x[k][0][e] = __fadd_rn(a, c);
+        x[k][1][e] = __fsub_rn(a, c);
+      }
+  }
+  // stages 16, 32, ...: dimension bits 4.. (k)
+#pragma unroll
+  for (int kb = 1; kb < NK; kb <<= 1) {
+    if (16 * kb < Bh) {
+#pragma unroll
+      for (int k = 0; k < NK; ++k)
+        if ((k & kb) == 0)
+#pragma unroll
+          for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float a = x[k][r][e], c = x[k + kb][r][e];
+              x[k][r][e] = __fadd_rn(a, c);
+              x[k + kb][r][e] = __fsub_rn(a, c);
+            }
+    }
+  }
+  const float rot_c = p.rot_c;
+  float amax = 0.f, qs = 0.f;
+#pragma unroll
+  for (int k = 0; k < NK; ++k)
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float v = __bfloat162float(__float2bfloat16_rn(__fmul_rn(x[k][r][e], rot_c)));
+        x[k][r][e] = v;
+        qs += v;
+        amax = fmaxf(amax, fabsf(v));
+      }
+  qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+  qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  // fp16 operands: q * 2^e with max|q| * 2^e in [2^14, 2^15) (exact for normal values)
+  int ex2e = 0;
+  if (amax > 0.f && amax <= 3.0e38f) {
+    int ex;
+    frexpf(amax, &ex);
+    ex2e = 15 - ex;
+  }
+#pragma unroll
+  for (int k = 0; k < NK; ++k)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) qf.b[k][r] = pack_half2(ldexpf(x[k][r][0], ex2e), ldexpf(x[k][r][1], ex2e));
+  // sum(q) of the heads of this lane's columns 2t and 2t+1 (held by lanes 8t and 8t+4)
+  qf.qs0 = __shfl_sync(0xffffffffu, qs, 8 * t) * p.scale_log2;
+  qf.qs1 = __shfl_sync(0xffffffffu, qs, 8 * t + 4) * p.scale_log2;
+  qf.kscale = ldexpf(p.scale_log2, -ex2e);
 }
 
 }  // namespace tiles

@@ -49,7 +49,9 @@ struct State {
   int n_items[3];      // work items of the current attention call: full chunks, tails, protected
   int n_parts;         // partial slots allocated by the current attention call
   int work;            // next work item to claim (persistent attention kernel)
-  int pad[57];
+  int ctr_dirty;       // a page-major launch gave up: its merge counters need zeroing
+  int cta_done;        // CTAs of the current page-major launch that finished
+  int pad[55];
 };
 static_assert(sizeof(State) == STATE_BYTES, "state block size");
 
@@ -312,6 +314,37 @@ __device__ __forceinline__ float half_hi(uint32_t x) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(x >> 16)));
 }
 
+// Butterfly stages hh = 1, 2, 4, ... (ascending, those with hh < Bh) of the
+// block-diagonal Hadamard over a row of 32*VPL values held VPL per lane
+// (element d = VPL*lane + i): the lower element of each pair becomes a + b,
+// the upper a - b.  The stages are unrolled at compile time (static register
+// indices) and skipped at run time.
+template <int VPL>
+__device__ __forceinline__ void fwht_row(float (&x)[VPL], int Bh, int lane) {
+#pragma unroll
+  for (int hh = 1; hh < 32 * VPL; hh <<= 1) {
+    if (hh < Bh) {
+      if (hh < VPL) {
+#pragma unroll
+        for (int i = 0; i < VPL; ++i)
+          if ((i & hh) == 0) {
+            const float a = x[i], c = x[i + hh];
+            x[i] = __fadd_rn(a, c);
+            x[i + hh] = __fsub_rn(a, c);
+          }
+      } else {
+        const int lm = hh / VPL;
+        const bool upper = (lane & lm) != 0;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+          const float o = __shfl_xor_sync(0xffffffffu, x[i], lm);
+          x[i] = upper ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
+        }
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Host-side handle (one struct for both cache kinds).
 
@@ -334,6 +367,7 @@ struct kv4_cache {
   int attn_ring;             // ring depth chosen for the per-head attention kernel
   int gattn_ring;            // ring depth of the page-major kernel (0: not used by this cache)
   int gattn_pair;            // INT4 tiles per consumer iteration of the page-major kernel (1 or 2)
+  unsigned long long* merge_ctr;   // [max_seqs][Hkv] arrival counters of the page-major kernel
   cudaEvent_t ev_before;     // optional timing events around the split-K kernel
   cudaEvent_t ev_after;
 };
@@ -354,7 +388,6 @@ int attention_blocks_per_sm(kv4_cache* c);
 bool grouped_path(const kv4_cache* c);
 int grouped_ring(kv4_cache* c);
 size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs);
-int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes, cudaStream_t stream,
-                   void (*merge)(const AttnParams&, cudaStream_t));
+int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 }  // namespace kv4
