@@ -2,9 +2,9 @@
 """Decode-step benchmark of the paged INT4/INT8-protected KV cache on B200.
 
 One step = the whole hot path for one batch: fused rotate+quantize+append of one
-new token per sequence, then decode attention (query rotation and work plan,
-split-K attention over the INT4 pages and the INT8 sink/recent store, merge and
-inverse rotation).  The metric is the algorithmic KV bytes the attention reads
+new token per sequence, then decode attention (query rotation; one persistent
+stream-K kernel over the INT4 pages and the INT8 sink/recent store that plans
+its own split, merges split groups and rotates the output back).  The metric is the algorithmic KV bytes the attention reads
 per step divided by the step time (GB/s), with decode tokens/s and the fraction
 of the measured HBM bandwidth beside it.
 
@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--impl", default="kv4", choices=["kv4", "reference"])
     ap.add_argument("--no-compare", action="store_true", help="skip the BF16-KV and INT4-only legs")
     ap.add_argument("--cpu-seqs", type=int, default=4, help="sequences in the CPU oracle sample")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="time the device steps only (no e2e leg, comparison legs or CPU baseline): for profilers")
     return ap.parse_args()
 
 
@@ -72,26 +74,31 @@ def measured_peaks():
         return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
 
 
+KERNEL_SOURCES = ("kv4_attention_grouped.cu", "kv4_attn_tiles.cuh", "kv4_common.cuh")
+
+
 def kernel_source_hash():
+    """Digest of the sources of the timed attention kernel (a profile summary is valid for this digest only)."""
     h = hashlib.sha1()
-    for name in ("kv4_attention.cu", "kv4_common.cuh"):
+    for name in KERNEL_SOURCES:
         with open(os.path.join(ROOT, "int4_kv_cache_paged_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:12]
 
 
 def profiled_traffic(workload):
-    """DRAM bytes per split-K launch from the committed ncu summary, if it matches the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "split_k_attention_%s.md" % workload)
+    """DRAM bytes per attention launch from the committed ncu summary, if it matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "gattn_kernel_%s.md" % workload)
     try:
         text = open(path).read()
     except OSError:
         return None
     vals = {}
     for line in text.splitlines():
-        if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "source_sha1")):
-            k, v = line.split(":", 1)
-            vals[k.strip().lstrip("- ")] = v.strip().strip("`")
+        item = line.strip().lstrip("-* ").strip()
+        if ":" in item and item.startswith(("traffic_bytes_per_launch", "source_sha1")):
+            k, v = item.split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
     if vals.get("source_sha1") != kernel_source_hash():
         return None
     try:
@@ -101,55 +108,79 @@ def profiled_traffic(workload):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 100 ms during the timed region."""
+    """SM clock and clock-event reasons read through NVML every 2 ms by a background thread.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    `window()` brackets a timed region (host time after a device synchronize on
+    both sides); `summary()` reports the samples that fall inside the windows.
+    Only reads the GPU's state.
+    """
 
-    def __init__(self, gpu_index):
-        self.gpu_index = gpu_index
-        self.proc = None
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, torch_device):
+        self.dev = torch_device
+        self.samples = []
+        self.windows = []
+        self.error = None
+
+    def _handle(self, pynvml):
+        """NVML handle of the torch device, matched by its PCI address (torch reports the parts as integers)."""
+        import torch
+        props = torch.cuda.get_device_properties(self.dev)
+        dom = getattr(props, "pci_domain_id", None)
+        bus = getattr(props, "pci_bus_id", None)
+        dev = getattr(props, "pci_device_id", None)
+        if all(isinstance(x, int) for x in (dom, bus, dev)):
+            addr = "%08x:%02x:%02x.0" % (dom, bus, dev)
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                info = pynvml.nvmlDeviceGetPciInfo(h)
+                got = info.busId.decode() if isinstance(info.busId, bytes) else str(info.busId)
+                if got.lower().endswith(addr[-12:]):
+                    return h
+        return pynvml.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
+
+    def _run(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = self._handle(pynvml)
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            while not self.stop.is_set():
+                t = time.perf_counter()
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                self.samples.append((t, sm, smax, int(get_reasons(h))))
+                time.sleep(0.002)
+            pynvml.nvmlShutdown()
+        except Exception as e:   # no NVML: reported as unavailable
+            self.error = "%s: %s" % (type(e).__name__, e)
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+        import threading
+        self.stop = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+        time.sleep(0.05)
         return self
 
     def __exit__(self, *a):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        self.stop.set()
+        self.thread.join(timeout=5)
+
+    def window(self, t0, t1):
+        self.windows.append((t0, t1))
 
     def summary(self):
-        sm, smax, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in getattr(self, "lines", []):
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for name, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        inside = [x for x in self.samples if any(t0 <= x[0] <= t1 for t0, t1 in self.windows)]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0,
+                    "note": self.error or "no sample inside the timed region"}
+        reasons = sorted({name for x in inside for name, bit in self.REASONS if x[3] & bit})
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": max(x[2] for x in inside),
+                "reasons": reasons, "samples": len(inside), "source": "NVML, 2 ms period"}
 
 
 # --------------------------------------------------------------------------- GPU workload
@@ -245,10 +276,11 @@ def run_gpu(args):
         torch.cuda.synchronize()
 
     barrier()
-    with ClockSampler(local) as clocks:
+    with ClockSampler(device) as clocks:
         for i in range(n):
             if i == W_:
                 barrier()
+                t_window = time.perf_counter()
             flush.fill_(i & 0xFF)                  # evict the KV of the previous step from L2 (not timed)
             kv4.kv4_set_attention_events(wl.cache.handle, *e_kern[i])
             e_step[i][0].record(stream)
@@ -259,6 +291,7 @@ def run_gpu(args):
             e_step[i][1].record(stream)
             step_bytes.append(kv_bytes(wl.L + i, Hkv, D, S, Wn))
         barrier()
+        clocks.window(t_window, time.perf_counter())
     kv4.kv4_set_attention_events(wl.cache.handle, None, None)
     status = wl.cache.status()
 
@@ -270,15 +303,19 @@ def run_gpu(args):
     lens_after = wl.L + n - 1                       # length at the last timed attention call
 
     # ---- e2e through the public API with host buffers (pinned), copies inside the timed region
-    hk = [wl.steps_k[n + j].cpu().pin_memory() for j in range(K)]
-    hv = [wl.steps_v[n + j].cpu().pin_memory() for j in range(K)]
-    hq = [workloads.queries(w, 0, n + j, device="cpu").pin_memory() for j in range(K)]
+    if args.kernel_only:
+        K_e2e = 0
+    else:
+        K_e2e = K
+    hk = [wl.steps_k[n + j].cpu().pin_memory() for j in range(K_e2e)]
+    hv = [wl.steps_v[n + j].cpu().pin_memory() for j in range(K_e2e)]
+    hq = [workloads.queries(w, 0, n + j, device="cpu").pin_memory() for j in range(K_e2e)]
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     dk, dv, dq = torch.empty_like(wl.steps_k[0]), torch.empty_like(wl.steps_v[0]), torch.empty_like(qs[0])
-    e_e2e = [(ev(), ev()) for _ in range(K)]
+    e_e2e = [(ev(), ev()) for _ in range(K_e2e)]
     e2e_bytes = 0
     barrier()
-    for j in range(K):
+    for j in range(K_e2e):
         flush.fill_(j & 0xFF)
         e_e2e[j][0].record(stream)
         dk.copy_(hk[j], non_blocking=True)
@@ -290,13 +327,13 @@ def run_gpu(args):
         e_e2e[j][1].record(stream)
         e2e_bytes += kv_bytes(wl.L + n + j, Hkv, D, S, Wn)
     barrier()
-    t_e2e = sum(a.elapsed_time(b) for a, b in e_e2e) / 1e3
+    t_e2e = sum(a.elapsed_time(b) for a, b in e_e2e) / 1e3 if K_e2e else float("nan")
     h2d = dk.numel() * 2 + dv.numel() * 2 + dq.numel() * 2
     d2h = hout.numel() * 2
 
     # ---- comparison legs on identical inputs (rank-local, untimed by the contract)
     compare = None
-    if not args.no_compare and world == 1:
+    if not args.no_compare and not args.kernel_only and world == 1:
         compare = compare_legs(torch, kv4, w, wl, K, device, flush)
 
     totals = torch.tensor([t_step, t_e2e, float(bytes_timed), float(e2e_bytes)], dtype=torch.float64, device=device)
@@ -344,12 +381,14 @@ def run_gpu(args):
             "append_us_per_step": round((t_step - t_attn) / K * 1e6, 2),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(achieved / hbm, 4), "traffic": traffic,
-                         "kernel": "attn_kernel (split-K over INT4 pages + INT8 store)",
+                         "kernel": "gattn_kernel: persistent stream-K attention over the INT4 pages and the "
+                                   "INT8 store with the merge of split groups (the events also cover the "
+                                   "query-operand kernel it overlaps)",
                          "peak_source": peak_kind, "bytes_per_launch": int(bytes_timed / K)},
-            "e2e": {"value": round(e2e_bytes_all / t_e2e_all / 1e9, 2), "unit": "GB/s",
-                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                    "tokens_per_s": round(B * world * K / t_e2e_all, 1)},
-            "gpu_launches": 4 * K,
+            "e2e": ({"value": round(e2e_bytes_all / t_e2e_all / 1e9, 2), "unit": "GB/s",
+                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                     "tokens_per_s": round(B * world * K / t_e2e_all, 1)} if K_e2e else None),
+            "gpu_launches": 3 * K,   # per step: append_kernel, gq_kernel, gattn_kernel
             "clocks": clk,
             "device_status": status,
             "setup_s": round(setup_s, 1),
@@ -481,7 +520,7 @@ def main():
         return
     res = run_gpu(args)
     if res is not None:
-        if res["n_gpus"] == 1:
+        if res["n_gpus"] == 1 and not args.kernel_only:
             res["cpu_baseline"] = cpu_baseline(workloads.workload(args.workload), args.cpu_seqs)
         print(json.dumps(res))
 
