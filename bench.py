@@ -232,6 +232,23 @@ class Workload:
         torch.cuda.synchronize()
 
 
+def reduce_over_ranks(times, counts, device, world):
+    """Whole-job figures: the maximum of each timing and the sum of each count over all ranks.
+
+    Every rank calls this once with the same list lengths (one all-reduce each for
+    the max and the sum, in the same order on every rank); with one process it
+    returns the inputs."""
+    if world <= 1:
+        return list(times), list(counts)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(times, dtype=torch.float64, device=device)
+    c = torch.tensor(counts, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(c, op=dist.ReduceOp.SUM)
+    return t.tolist(), c.tolist()
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -336,16 +353,8 @@ def run_gpu(args):
     if not args.no_compare and not args.kernel_only and world == 1:
         compare = compare_legs(torch, kv4, w, wl, K, device, flush)
 
-    totals = torch.tensor([t_step, t_e2e, float(bytes_timed), float(e2e_bytes)], dtype=torch.float64, device=device)
-    if world > 1:
-        tmax = totals[:2].clone()
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-        bsum = totals[2:].clone()
-        dist.all_reduce(bsum, op=dist.ReduceOp.SUM)
-        t_step_all, t_e2e_all = tmax.tolist()
-        bytes_all, e2e_bytes_all = bsum.tolist()
-    else:
-        t_step_all, t_e2e_all, bytes_all, e2e_bytes_all = t_step, t_e2e, float(bytes_timed), float(e2e_bytes)
+    (t_step_all, t_e2e_all), (bytes_all, e2e_bytes_all) = reduce_over_ranks(
+        [t_step, t_e2e], [float(bytes_timed), float(e2e_bytes)], device, world)
 
     result = None
     if rank == 0:
