@@ -59,7 +59,9 @@ enum {
   KV4_ERR_CAPACITY = -3,      /* a buffer smaller than kv4_cache_required_bytes()          */
   KV4_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed                      */
   KV4_ERR_DEVICE_FAULT = -5,  /* kv4_get_status() found device status bits set             */
-  KV4_ERR_WORKSPACE = -6      /* workspace smaller than kv4_attention_workspace_bytes()    */
+  KV4_ERR_WORKSPACE = -6,     /* workspace smaller than kv4_attention_workspace_bytes()    */
+  KV4_ERR_SCRATCH = -7        /* kv4_decode_attention_noalloc: the call needs more scratch
+                                 than KV4_NOALLOC_SCRATCH_BYTES                             */
 };
 
 /* Bits of the device status word. */
@@ -186,6 +188,37 @@ int kv4_attention_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_
 int kv4_decode_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs,
                          const void* q, void* out, float softmax_scale, int32_t mode,
                          void* dev_workspace, size_t ws_bytes, kv4_stream_t stream);
+
+/*
+ * kv4_decode_attention_noalloc: kv4_decode_attention without a workspace
+ * argument.  Its scratch (query operands and split-K partials) lives in a
+ * static device array of this library, KV4_NOALLOC_SCRATCH_BYTES (16 MiB) per
+ * device, so the call itself allocates nothing and needs no buffer from the
+ * caller.  The method's pages have no counterpart of this call.
+ *
+ * For callers that cannot allocate device memory when they issue attention:
+ * an inference loop that must not call an allocator between steps (a caching
+ * allocator may synchronize the device or grow its pool at an arbitrary
+ * step), or a caller that holds no device memory of its own for scratch.
+ *
+ * Arguments, results and errors are those of kv4_decode_attention, plus:
+ *   KV4_ERR_SCRATCH when kv4_attention_workspace_bytes(cache, n_seqs, 0) is
+ *   above KV4_NOALLOC_SCRATCH_BYTES (with 8 or more KV heads that is
+ *   n_seqs * Hkv * (16*D + 64) bytes of query operands plus
+ *   2 * SMs * 8 * G * (D + 4) * 4 bytes of partials, e.g. about 6.1 MB for 64
+ *   sequences, 32/8 heads, D = 128, and 13.7 MB for 512 sequences);
+ *   nothing is launched then.
+ * The scratch is one per device and shared by every cache and stream of the
+ * process on that device: calls that can run at the same time (two streams,
+ * two host threads) race on it and give wrong results, so order them (one
+ * stream, or events).  Nothing in it has to start at zero.  The first call
+ * on a device looks the array up (cudaGetSymbolAddress, with the cache's
+ * device current) and should come before any stream capture.
+ */
+#define KV4_NOALLOC_SCRATCH_BYTES (16u << 20)
+int kv4_decode_attention_noalloc(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs,
+                                 const void* q, void* out, float softmax_scale, int32_t mode,
+                                 kv4_stream_t stream);
 
 /* Dequantized keys/values of positions [start, start+count) of one sequence,
  * fp32 [count][Hkv][D], in the rotated basis: x^ = fma(code, s, z) from the

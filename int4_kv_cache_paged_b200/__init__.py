@@ -34,6 +34,8 @@ KV4_ERR_CAPACITY = -3
 KV4_ERR_CUDA = -4
 KV4_ERR_DEVICE_FAULT = -5
 KV4_ERR_WORKSPACE = -6
+KV4_ERR_SCRATCH = -7
+KV4_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 KV4_DEV_BAD_PAGE = 1
 KV4_DEV_OVERFLOW = 2
@@ -52,6 +54,7 @@ KV4_VIEW_INT4 = 1
 EXPORTS = [
     "kv4_cache_required_bytes", "kv4_cache_create", "kv4_cache_destroy", "kv4_cache_layout", "kv4_seq_reset",
     "kv4_rotate_quantize_append", "kv4_attention_workspace_bytes", "kv4_decode_attention",
+    "kv4_decode_attention_noalloc",
     "kv4_dequantize_debug", "kv4_get_status", "kv4_set_attention_events", "kv4_status_string", "kv4_version",
     "kv4bf16_cache_required_bytes", "kv4bf16_cache_create", "kv4bf16_cache_destroy", "kv4bf16_cache_layout",
     "kv4bf16_append", "kv4bf16_attention_workspace_bytes", "kv4bf16_decode_attention", "kv4bf16_get_status",
@@ -79,6 +82,7 @@ _sigs = {
     "kv4_rotate_quantize_append": (_I, [_P, _I, _P, _P, _I, _I, _P, _P, _P]),
     "kv4_attention_workspace_bytes": (_I, [_P, _I, _I, ctypes.POINTER(_SZ)]),
     "kv4_decode_attention": (_I, [_P, _I, _P, _I, _P, _P, ctypes.c_float, _I, _P, _SZ, _P]),
+    "kv4_decode_attention_noalloc": (_I, [_P, _I, _P, _I, _P, _P, ctypes.c_float, _I, _P]),
     "kv4_dequantize_debug": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "kv4_get_status": (_I, [_P, _P, ctypes.POINTER(_I)]),
     "kv4_set_attention_events": (_I, [_P, _P, _P]),
@@ -176,6 +180,12 @@ def kv4_decode_attention(handle, layer, seq_ids, n_seqs, q, out, softmax_scale, 
                                      float(softmax_scale), mode, _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream)),
            "kv4_decode_attention")
+
+
+def kv4_decode_attention_noalloc(handle, layer, seq_ids, n_seqs, q, out, softmax_scale, mode, stream=None):
+    _check(_lib.kv4_decode_attention_noalloc(handle, layer, _ptr(seq_ids), n_seqs, _ptr(q), _ptr(out),
+                                             float(softmax_scale), mode, _stream(stream)),
+           "kv4_decode_attention_noalloc")
 
 
 def kv4_dequantize_debug(handle, layer, seq_id, start, count, view, k_out, v_out, stream=None):

@@ -10,7 +10,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = ["kv4_api.cu", "kv4_append.cu", "kv4_attention.cu", "kv4_attention_grouped.cu"]
+SOURCES = ["kv4_api.cu", "kv4_append.cu", "kv4_attention.cu", "kv4_attention_grouped.cu", "kv4_noalloc.cu"]
 LIB = os.path.join(HERE, "libkv4.so")
 OBJDIR = os.path.join(ROOT, "_build")
 

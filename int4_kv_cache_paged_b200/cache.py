@@ -4,6 +4,7 @@ import torch
 
 from . import (make_config, kv4_cache_required_bytes, kv4_cache_create, kv4_cache_destroy, kv4_cache_layout,
                kv4_seq_reset, kv4_rotate_quantize_append, kv4_attention_workspace_bytes, kv4_decode_attention,
+               kv4_decode_attention_noalloc,
                kv4_dequantize_debug, kv4_get_status, kv4bf16_cache_required_bytes, kv4bf16_cache_create,
                kv4bf16_cache_destroy, kv4bf16_cache_layout, kv4bf16_append, kv4bf16_attention_workspace_bytes,
                kv4bf16_decode_attention, kv4bf16_get_status, KV4_VIEW_EFFECTIVE, KV4_MODE_OUT_F32)
@@ -98,6 +99,11 @@ class KV4Cache(_Base):
         if workspace is None:
             workspace = self.workspace(n)
         kv4_decode_attention(self.handle, layer, seq_ids, n, q, out, scale, mode, workspace, stream)
+        return out
+
+    def attention_noalloc(self, layer, seq_ids, q, out, scale=0.0, mode=0, stream=None):
+        """Attention with the library's static scratch (no workspace); `out` must be given."""
+        kv4_decode_attention_noalloc(self.handle, layer, seq_ids, int(seq_ids.numel()), q, out, scale, mode, stream)
         return out
 
     def dequantize(self, layer, seq, start, count, view=KV4_VIEW_EFFECTIVE, stream=None):

@@ -256,6 +256,7 @@ const char* kv4_status_string(int status) {
     case KV4_ERR_CUDA: return "CUDA runtime error";
     case KV4_ERR_DEVICE_FAULT: return "device status bits set";
     case KV4_ERR_WORKSPACE: return "workspace too small";
+    case KV4_ERR_SCRATCH: return "needs more scratch than the static no-alloc array holds";
     default: return "unknown status";
   }
 }
