@@ -8,7 +8,7 @@
 // scale and zero point are folded out of the inner products as in the
 // folded-scale kernels of "KV Cache Quantization" (topic page), item 2:
 //     q . k^  = s_k * (q . c_k) + z_k * sum(q)
-//     sum_p a_p v^_p = sum_p (a_p s_p) c_p + sum_p a_p z_p
+//     sum_p a_p v^_p = sum_p (a_p s_p) (c_p - 8) + sum_p a_p (z_p + 8 s_p)     (INT4; 128 for INT8)
 #pragma once
 
 #include "kv4_common.cuh"
@@ -132,7 +132,7 @@ __device__ __forceinline__ void pv_int4(uint32_t st, WarpState<D>& ws, int lane,
 #pragma unroll
   for (int m = 0; m < D / 16; ++m) {
     const uint32_t w = vw[m], u = w >> 8;
-    const uint32_t a0 = nib_lo(w), a1 = nib_hi(w), a2 = nib_lo(u), a3 = nib_hi(u);
+    const uint32_t a0 = nib_lo_c(w), a1 = nib_hi_c(w), a2 = nib_lo_c(u), a3 = nib_hi_c(u);
     mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
     if (!colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
   }
@@ -223,7 +223,8 @@ __device__ __forceinline__ void unit_int4(const uint32_t (&tile)[2], const QFrag
   for (int u = 0; u < NT; ++u) {
     const float p0 = ex2(x[u][0] - ws.m0), p1 = ex2(x[u][1] - ws.m1);
     const float p2 = ex2(x[u][2] - ws.m0), p3 = ex2(x[u][3] - ws.m1);
-    const float sVg = half_lo(sz[u].z), zVg = half_hi(sz[u].z), sVg8 = half_lo(sz[u].w), zVg8 = half_hi(sz[u].w);
+    const float sVg = half_lo(sz[u].z), sVg8 = half_lo(sz[u].w);
+    const float zVg = fmaf(8.f, sVg, half_hi(sz[u].z)), zVg8 = fmaf(8.f, sVg8, half_hi(sz[u].w));   // centred codes
     float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
     float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
     if constexpr (MASKED) {   // unwritten slots may hold non-finite scales
@@ -254,7 +255,7 @@ __device__ __forceinline__ void unit_int4(const uint32_t (&tile)[2], const QFrag
 #pragma unroll
       for (int m = 0; m < D / 16; ++m) {
         const uint32_t w = vw[m], uu = w >> 8;
-        const uint32_t a0 = nib_lo(w), a1 = nib_hi(w), a2 = nib_lo(uu), a3 = nib_hi(uu);
+        const uint32_t a0 = nib_lo_c(w), a1 = nib_hi_c(w), a2 = nib_lo_c(uu), a3 = nib_hi_c(uu);
         mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
         if (!cs.colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
       }
@@ -303,7 +304,8 @@ __device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpS
   }
   float p0, p1, p2, p3;
   online_softmax_pv<D>(ws, x0, x1, x2, x3, p0, p1, p2, p3);
-  const float sVg = half_lo(sz.z), zVg = half_hi(sz.z), sVg8 = half_lo(sz.w), zVg8 = half_hi(sz.w);
+  const float sVg = half_lo(sz.z), sVg8 = half_lo(sz.w);
+  const float zVg = fmaf(128.f, sVg, half_hi(sz.z)), zVg8 = fmaf(128.f, sVg8, half_hi(sz.w));   // centred codes
   float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
   float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
   if constexpr (MASKED) {
@@ -317,7 +319,7 @@ __device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpS
 #pragma unroll
   for (int m = 0; m < NK; ++m) {
     const uint32_t w0 = vw[2 * m], w1 = vw[2 * m + 1];
-    const uint32_t a0 = byte_lo(w0), a1 = byte_lo(w0 >> 8), a2 = byte_lo(w1), a3 = byte_lo(w1 >> 8);
+    const uint32_t a0 = byte_lo_c(w0), a1 = byte_lo_c(w0 >> 8), a2 = byte_lo_c(w1), a3 = byte_lo_c(w1 >> 8);
     mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
     if (!cs.colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
   }

@@ -307,6 +307,29 @@ __device__ __forceinline__ uint32_t byte_lo(uint32_t w) {  // bytes 0 and 2
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Centred operands for P.V: a code c becomes c - 8 (INT4) or c - 128 (INT8),
+// still exact in fp16, and the zero point z becomes z + 8 s (or z + 128 s).
+// The code term then has both signs and no longer nearly cancels a large
+// zero-point sum after thousands of tensor-core accumulations.
+__device__ __forceinline__ uint32_t nib_lo_c(uint32_t w) {  // nibbles at bits 0-3 and 16-19, minus 8
+  uint32_t x = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
+  __half2 h = __hsub2(*reinterpret_cast<__half2*>(&x), __half2(__half(1032.f), __half(1032.f)));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t nib_hi_c(uint32_t w) {  // nibbles at bits 4-7 and 20-23, minus 8
+  uint32_t x = lop3_and_or(w, 0x00F000F0u, 0x64006400u);
+  __half2 h = __hfma2(*reinterpret_cast<__half2*>(&x), __half2(__half(0.0625f), __half(0.0625f)),
+                      __half2(__half(-72.f), __half(-72.f)));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t byte_lo_c(uint32_t w) {  // bytes 0 and 2, minus 128
+  uint32_t x = lop3_and_or(w, 0x00FF00FFu, 0x64006400u);
+  __half2 h = __hsub2(*reinterpret_cast<__half2*>(&x), __half2(__half(1152.f), __half(1152.f)));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 __device__ __forceinline__ float half_lo(uint32_t x) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(x & 0xFFFFu)));
 }
