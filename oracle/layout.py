@@ -13,8 +13,9 @@ INT8 tile (32*D + 128 bytes):   [K codes 16*D][V codes 16*D][scales 128]
 BF16 tile (64*D bytes):         [K 16*D bf16][V 16*D bf16]      (baseline cache)
 
 Inside the code blocks the order of nibbles/bytes follows the operand order
-of the 16x8x16 tensor-core multiply the decode kernel feeds from them; the
-functions below state each placement in closed form.  Properties that the
+of the tensor-core multiplies the decode kernel feeds from them (K: the
+16x8x32 integer multiply, V: the 16x8x16 fp16 multiply); the functions below
+state each placement in closed form.  Properties that the
 tests check: every (token, dim) owns exactly one nibble (or byte, or bf16
 element), and every byte of a code block belongs to exactly one token (so a
 token can be written without reading its neighbours).
@@ -44,15 +45,16 @@ def bf16_tile_bytes(D):
 def int4_k_nibble(D, r, d):
     """(byte offset inside the K code block, nibble: 0 = low, 1 = high) of token r, dim d.
 
-    Token r owns the D/2 bytes [r*D/2, (r+1)*D/2).  With d = 32*kk + 8*j + 2*t + e
-    (kk < D/32, j < 4, t < 4, e < 2) and i = j + 4*e, the nibble is number i of
-    the 32-bit word at byte r*D/2 + t*D/8 + 4*kk.
+    Token r owns the D/2 bytes [r*D/2, (r+1)*D/2).  With d = 32*kk + 16*hf + 4*t + j
+    (kk < D/32, hf < 2, t < 4, j < 4), the code is nibble hf of byte j of the
+    32-bit word at byte r*D/2 + t*D/8 + 4*kk: masking the word with 0x0F0F0F0F
+    gives the four dims 4t..4t+3 of the 32-dim block as bytes, shifting it right
+    by 4 first gives dims 16+4t..16+4t+3.
     """
-    kk, rem = divmod(d, 32)
-    j, rem = divmod(rem, 8)
-    t, e = divmod(rem, 2)
-    i = j + 4 * e
-    return r * (D // 2) + t * (D // 8) + 4 * kk + i // 2, i % 2
+    kk, dd = divmod(d, 32)
+    hf, rem = divmod(dd, 16)
+    t, j = divmod(rem, 4)
+    return r * (D // 2) + t * (D // 8) + 4 * kk + j, hf
 
 
 def int4_v_nibble(D, r, d):
@@ -73,14 +75,14 @@ def int4_v_nibble(D, r, d):
 def int8_k_byte(D, r, d):
     """Byte offset inside the INT8 K code block of token r, dim d.
 
-    With r = 8*rowhi + g, d = 16*k + 8*h8 + 2*t + e: byte h8 + 2*e of the word
-    at 16*(32*(rowhi*D/64 + k//4) + 4*g + t) + 4*(k % 4).
+    Token r owns the D bytes [r*D, (r+1)*D).  With d = 32*kk + 16*hf + 4*t + j,
+    the code is byte j of the word at r*D + (D/4)*t + 4*(2*kk + hf): one word
+    holds the dims 4t..4t+3 (hf = 0) or 16+4t..16+4t+3 (hf = 1) of a 32-dim block.
     """
-    rowhi, g = divmod(r, 8)
-    k, c = divmod(d, 16)
-    h8, c2 = divmod(c, 8)
-    t, e = divmod(c2, 2)
-    return 16 * (32 * (rowhi * (D // 64) + k // 4) + 4 * g + t) + 4 * (k % 4) + h8 + 2 * e
+    kk, dd = divmod(d, 32)
+    hf, rem = divmod(dd, 16)
+    t, j = divmod(rem, 4)
+    return r * D + (D // 4) * t + 4 * (2 * kk + hf) + j
 
 
 def int8_v_byte(D, r, d):

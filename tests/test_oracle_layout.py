@@ -1,9 +1,11 @@
 """Pins of the tile layout: bijections, byte ownership, and the tensor-core operand order it serves.
 
-The operand order of the 16x8x16 multiply (row-major A, 16 x 16): lane = 4*g + t
-holds A[g][2t, 2t+1] (a0a1), A[g+8][2t, 2t+1] (a2a3), A[g][2t+8, 2t+9] (a4a5),
-A[g+8][2t+8, 2t+9] (a6a7).  For Q.K^T the A matrix of k-step k is K[token][16k + col];
-for P.V it is V^T[16m + row][token].
+Scores use the 16x8x32 integer multiply (row-major A, 16 x 32 bytes): lane = 4*g + t
+holds A[g][4t..4t+3] (register 0), A[g+8][4t..4t+3] (1), A[g][16+4t..16+4t+3] (2),
+A[g+8][16+4t..16+4t+3] (3); the A matrix of k-block kk is K[token][32kk + col].
+P.V uses the 16x8x16 fp16 multiply (row-major A, 16 x 16): lane holds
+A[g][2t, 2t+1] (a0a1), A[g+8][2t, 2t+1] (a2a3), A[g][2t+8, 2t+9] (a4a5),
+A[g+8][2t+8, 2t+9] (a6a7), with A = V^T[16m + row][token].
 """
 
 import numpy as np
@@ -69,6 +71,11 @@ def _byte_pairs(w):
     return [(w & 255, (w >> 16) & 255), ((w >> 8) & 255, (w >> 24) & 255)]
 
 
+def _nib_bytes(w, hf):
+    """The four byte-wide codes the kernel extracts from one word: (w >> 4*hf) & 0x0F0F0F0F."""
+    return [(w >> (8 * j + 4 * hf)) & 15 for j in range(4)]
+
+
 @pytest.mark.parametrize("D", [64, 128])
 def test_int4_k_words_are_qk_a_operands(D):
     rng = np.random.default_rng(0)
@@ -77,13 +84,12 @@ def test_int4_k_words_are_qk_a_operands(D):
     for lane in range(32):
         g, t = divmod(lane, 4)
         for rowhi in (0, 1):
+            row = g + 8 * rowhi
             for kk in range(D // 32):
-                u = _nib_pairs(_word(blk, rowhi * 4 * D + lane * (D // 8) + 4 * kk))
-                row = g + 8 * rowhi
-                for half, k in ((0, 2 * kk), (1, 2 * kk + 1)):
-                    A = K[:, 16 * k:16 * k + 16]
-                    assert u[2 * half] == (A[row, 2 * t], A[row, 2 * t + 1])          # a0a1 / a2a3
-                    assert u[2 * half + 1] == (A[row, 2 * t + 8], A[row, 2 * t + 9])  # a4a5 / a6a7
+                w = _word(blk, rowhi * 4 * D + lane * (D // 8) + 4 * kk)
+                A = K[:, 32 * kk:32 * kk + 32]
+                assert _nib_bytes(w, 0) == list(A[row, 4 * t:4 * t + 4])           # register 0 / 1
+                assert _nib_bytes(w, 1) == list(A[row, 16 + 4 * t:16 + 4 * t + 4])  # register 2 / 3
 
 
 @pytest.mark.parametrize("D", [64, 128])
@@ -116,12 +122,12 @@ def test_int8_words_are_a_operands(D):
     for lane in range(32):
         g, t = divmod(lane, 4)
         for rowhi in (0, 1):
-            for k in range(D // 16):
-                u = _byte_pairs(_word(kb, 16 * (32 * (rowhi * (D // 64) + k // 4) + lane) + 4 * (k % 4)))
-                A = K[:, 16 * k:16 * k + 16]
-                row = g + 8 * rowhi
-                assert u[0] == (A[row, 2 * t], A[row, 2 * t + 1])
-                assert u[1] == (A[row, 2 * t + 8], A[row, 2 * t + 9])
+            row = g + 8 * rowhi
+            for kk in range(D // 32):
+                A = K[:, 32 * kk:32 * kk + 32]
+                for hf in (0, 1):
+                    w = _word(kb, rowhi * 8 * D + (D // 4) * lane + 4 * (2 * kk + hf))
+                    assert [(w >> (8 * j)) & 255 for j in range(4)] == list(A[row, 16 * hf + 4 * t:16 * hf + 4 * t + 4])
         for m in range(D // 16):
             AT = V[:, 16 * m:16 * m + 16].T
             for th in (0, 1):
