@@ -79,14 +79,15 @@ __device__ __forceinline__ uint32_t quantize_group(const float (&x)[VPL], float 
 __device__ __forceinline__ void store_int4(uint8_t* tile, int r, int tensor, const uint8_t* codes, uint32_t sz,
                                            int D, int lane) {
   if (tensor == 0) {
+    // word (t, kk): byte j holds dim 32kk + 4t + j (low nibble) and 32kk + 16 + 4t + j (high nibble)
     const int nkk = D / 32;
     if (lane < D / 8) {
       const int t = lane / nkk, kk = lane % nkk;
       uint32_t w = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int d = 32 * kk + 8 * (i & 3) + 2 * t + (i >> 2);
-        w |= static_cast<uint32_t>(codes[d]) << (4 * i);
+      for (int j = 0; j < 4; ++j) {
+        w |= static_cast<uint32_t>(codes[32 * kk + 4 * t + j]) << (8 * j);
+        w |= static_cast<uint32_t>(codes[32 * kk + 16 + 4 * t + j]) << (8 * j + 4);
       }
       *reinterpret_cast<uint32_t*>(tile + r * (D / 2) + t * (D / 8) + 4 * kk) = w;
     }
@@ -104,15 +105,14 @@ __device__ __forceinline__ void store_int4(uint8_t* tile, int r, int tensor, con
 // Write one token's INT8 codes and scales into its protected tile.
 __device__ __forceinline__ void store_int8(uint8_t* tile, int r, int tensor, const uint8_t* codes, uint32_t sz,
                                            int D, int lane) {
-  const int rowhi = r >> 3, g = r & 7;
   if (tensor == 0) {
+    // word L = (D/16) t + 2 kk + hf of the token: dims 32kk + 16hf + 4t + 0..3, one per byte
     if (lane < D / 4) {
-      const int k = lane >> 2, t = lane & 3;
-      const uint32_t w = static_cast<uint32_t>(codes[16 * k + 2 * t]) |
-                         (static_cast<uint32_t>(codes[16 * k + 8 + 2 * t]) << 8) |
-                         (static_cast<uint32_t>(codes[16 * k + 2 * t + 1]) << 16) |
-                         (static_cast<uint32_t>(codes[16 * k + 8 + 2 * t + 1]) << 24);
-      *reinterpret_cast<uint32_t*>(tile + 16 * (32 * (rowhi * (D / 64) + (k >> 2)) + 4 * g + t) + 4 * (k & 3)) = w;
+      const int t = lane / (D / 16), wi = lane % (D / 16), kk = wi >> 1, hf = wi & 1;
+      const int d = 32 * kk + 16 * hf + 4 * t;
+      const uint32_t w = static_cast<uint32_t>(codes[d]) | (static_cast<uint32_t>(codes[d + 1]) << 8) |
+                         (static_cast<uint32_t>(codes[d + 2]) << 16) | (static_cast<uint32_t>(codes[d + 3]) << 24);
+      *reinterpret_cast<uint32_t*>(tile + r * D + 4 * lane) = w;
     }
   } else {
     const int t = (r & 7) >> 1, e = r & 1, th = r >> 3;
@@ -162,7 +162,7 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams p) {
   constexpr int VPL = D / 32;
   extern __shared__ int s_cu[];
-  __shared__ uint8_t s_codes[APPEND_WARPS][2][D];
+  __shared__ __align__(16) uint8_t s_codes[APPEND_WARPS][2][D];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i <= p.n_seqs; i += blockDim.x) s_cu[i] = p.cu_new[i];
   __syncthreads();
@@ -173,6 +173,18 @@ __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams 
     const int tensor = static_cast<int>(job & 1);
     const int h = static_cast<int>((job >> 1) % p.Hkv);
     const int n = static_cast<int>((job >> 1) / p.Hkv);
+    // the row's values first: their load overlaps the dependent metadata loads below
+    uint16_t raw[VPL];
+    {
+      const uint16_t* src = (tensor ? p.v_new : p.k_new) + (static_cast<long long>(n) * p.Hkv + h) * D;
+      if constexpr (VPL == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(src + 4 * lane);
+        raw[0] = u.x & 0xFFFF; raw[1] = u.x >> 16; raw[2] = u.y & 0xFFFF; raw[3] = u.y >> 16;
+      } else {
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(src + 2 * lane);
+        raw[0] = u & 0xFFFF; raw[1] = u >> 16;
+      }
+    }
     const int i = find_seq(s_cu, p.n_seqs, n);
     const int seq = p.seq_ids[i];
     const int cap = p.max_pages_per_seq * p.P;
@@ -200,15 +212,6 @@ __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams 
       }
     }
     if (ok) {
-      const uint16_t* src = (tensor ? p.v_new : p.k_new) + (static_cast<long long>(n) * p.Hkv + h) * D;
-      uint16_t raw[VPL];
-      if constexpr (VPL == 4) {
-        const uint2 u = *reinterpret_cast<const uint2*>(src + 4 * lane);
-        raw[0] = u.x & 0xFFFF; raw[1] = u.x >> 16; raw[2] = u.y & 0xFFFF; raw[3] = u.y >> 16;
-      } else {
-        const uint32_t u = *reinterpret_cast<const uint32_t*>(src + 2 * lane);
-        raw[0] = u & 0xFFFF; raw[1] = u >> 16;
-      }
       const int r = pos & (TILE - 1);
       // head-innermost pool: [page][P/16][Hkv][tile]
       const long long tile_idx = (static_cast<long long>(page) * (p.P / TILE) + (pos % p.P) / TILE) * p.Hkv + h;
@@ -304,7 +307,7 @@ __global__ void dequant_kernel(DequantParams p) {
   const bool protect = p.view == KV4_VIEW_EFFECTIVE && (pos < p.S || pos >= L - p.W);
   if (protect) {
     const int slot = pos < p.S ? pos : p.S + (pos - p.S) % p.W;
-    const int r = slot & 15, rowhi = r >> 3, g = r & 7;
+    const int r = slot & 15;
     const uint8_t* tile = p.prot + ((static_cast<long long>(p.seq) * n_prot_tiles(p.S, p.W) + slot / 16) * p.Hkv + h) *
                                        tile8_bytes(D);
     const uint32_t sz = *reinterpret_cast<const uint32_t*>(tile + 32 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3)));
@@ -312,8 +315,8 @@ __global__ void dequant_kernel(DequantParams p) {
     for (int d = lane; d < D; d += 32) {
       int off;
       if (tensor == 0) {
-        const int k = d >> 4, c = d & 15, h8 = c >> 3, t = (c & 7) >> 1, e = c & 1;
-        off = 16 * (32 * (rowhi * (D / 64) + (k >> 2)) + 4 * g + t) + 4 * (k & 3) + h8 + 2 * e;
+        const int kk = d >> 5, hf = (d >> 4) & 1, t = (d >> 2) & 3, j = d & 3;
+        off = r * D + (D / 4) * t + 4 * (2 * kk + hf) + j;
       } else {
         const int m = d >> 4, dh = (d >> 3) & 1, gg = d & 7, th = r >> 3, t = (r & 7) >> 1, e = r & 1;
         const int w = 2 * m + th;
@@ -335,9 +338,9 @@ __global__ void dequant_kernel(DequantParams p) {
     for (int d = lane; d < D; d += 32) {
       int byte, half;
       if (tensor == 0) {
-        const int kk = d >> 5, jj = (d >> 3) & 3, t = (d >> 1) & 3, e = d & 1, i = jj + 4 * e;
-        byte = r * (D / 2) + t * (D / 8) + 4 * kk + (i >> 1);
-        half = i & 1;
+        const int kk = d >> 5, hf = (d >> 4) & 1, t = (d >> 2) & 3, j = d & 3;
+        byte = r * (D / 2) + t * (D / 8) + 4 * kk + j;
+        half = hf;
       } else {
         const int m = d >> 4, dh = (d >> 3) & 1, g = d & 7, th = r >> 3, t = (r & 7) >> 1, e = r & 1;
         byte = 8 * D + 512 * (m >> 2) + 16 * (4 * g + t) + 4 * (m & 3) + th + 2 * e;

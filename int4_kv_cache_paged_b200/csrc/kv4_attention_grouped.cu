@@ -12,11 +12,13 @@
 // Its work is a list of stages: one stage per 16-token INT4 tile position (the
 // tiles of the 8 heads are contiguous in the head-innermost pool, one 17 KB
 // bulk copy), then two stages per INT8 protected tile (heads 0-3, heads 4-7).
-// The stage lists of all head groups are concatenated (T stages) and CTA c of
-// the persistent grid takes stages [c*T/N, (c+1)*T/N): every CTA streams the
-// same number of bytes (stream-K).  Every CTA derives this plan itself from the
-// sequence lengths (a block scan over the head groups), so no planning kernel
-// runs first.  Where a CTA's range crosses head groups it works on segments.
+// The stage lists of all head groups are concatenated, each group charged a
+// few extra units for the cost of starting it (T units in all), and CTA c of
+// the persistent grid takes units [c*T/N, (c+1)*T/N): every CTA gets the same
+// share of bytes plus group starts (stream-K).  Every CTA derives this plan
+// itself from the sequence lengths (a block scan over the head groups), so no
+// planning kernel runs first.  Where a CTA's range crosses head groups it
+// works on segments.
 //
 // Inside a CTA: a producer warp issues the bulk copies into a ring of
 // shared-memory stages (each lane one stage of a batch, mbarrier completion);
@@ -27,9 +29,10 @@
 // waits for it only before its first operand read).  A group that one CTA
 // covers whole is normalised, rotated back and stored straight from registers;
 // a group split over several CTAs leaves one partial (m, l, o) per segment in
-// the workspace, and the warp whose partial arrives last (a counter per batch
-// entry and KV head, set back to zero by that warp) merges them and stores the
-// output.  A launch in which a wait gave up zeroes all counters at its end.
+// the workspace.  After its last segment each warp announces its partials (a
+// counter per batch entry and KV head); the warp that completes a count merges
+// them, stores the output and sets the counter back to zero.  A launch in
+// which a wait gave up zeroes all counters at its end.
 #include "kv4_attn_tiles.cuh"
 
 namespace kv4 {
@@ -84,8 +87,18 @@ constexpr int MAX_NS = 16;
 // A CTA takes at least this many stages: a short batch is spread over fewer
 // CTAs, so that merging the partials costs less than the streaming it saves.
 constexpr int MIN_STAGES = 16;
+// Extra stages charged to every head group in the split: starting a group
+// costs a CTA about as much as streaming this many stages (query operands,
+// the segment's result, its partial), so a CTA that starts more groups gets
+// fewer stages.
+constexpr int GROUP_COST = 4;
 
 __host__ __device__ inline int group_stages(const Group& g) { return g.n4 + 2 * g.n8; }
+// Length of a group in the units of the split: its stages plus the start cost (0 when empty).
+__host__ __device__ inline int group_cost(const Group& g) {
+  const int n = group_stages(g);
+  return n > 0 ? n + GROUP_COST : 0;
+}
 
 // CTA owning global stage j: the largest c with floor(c*T/N) <= j.
 __device__ __forceinline__ int cta_of(long long j, long long T, long long N) {
@@ -408,7 +421,7 @@ __device__ __forceinline__ void merge_store_g(const AttnParams& p, const PartRef
 
 // ---------------------------------------------------------------------------
 // query operands: one warp per (batch entry, KV head) rotates its G query
-// heads and stores the tensor-core B fragments (16 B per lane and 16-dim pair),
+// heads and stores the integer tensor-core B fragments of both query planes,
 // sum(q) per fragment column and the exponent scale.  The attention kernel is
 // launched as its programmatic dependent, so it plans and starts streaming
 // pages while this runs, and waits for it only before the first operand read.
@@ -423,14 +436,7 @@ __global__ void __launch_bounds__(32 * QWARPS) gq_kernel(AttnParams p) {
   if (gw >= p.n_seqs * p.Hkv) return;
   QFrag<D> qf;
   load_qfrag<D>(p, gw / p.Hkv, gw % p.Hkv, lane, qf);
-  uint8_t* blob = p.qblob + static_cast<size_t>(gw) * qblob_bytes(D);
-#pragma unroll
-  for (int cc = 0; cc < D / 32; ++cc)
-    reinterpret_cast<uint4*>(blob)[cc * 32 + lane] =
-        make_uint4(qf.b[2 * cc][0], qf.b[2 * cc][1], qf.b[2 * cc + 1][0], qf.b[2 * cc + 1][1]);
-  float* tail = reinterpret_cast<float*>(blob + 16 * D);
-  if (lane < 4) { tail[2 * lane] = qf.qs0; tail[2 * lane + 1] = qf.qs1; }   // lanes 0-3: columns 2t, 2t+1
-  if (lane == 0) tail[MAX_G] = qf.kscale;
+  store_qblob<D>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D), qf, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -511,8 +517,10 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
     fence_barrier_init();
   }
 
-  // ---- plan (every CTA the same): stage counts of all head groups -> T, then
-  // the stream-K range [j0, j1) of this CTA and the group holding j0
+  // ---- plan (every CTA the same): costs of all head groups -> T, then the
+  // stream-K range [j0, j1) of this CTA and the group holding j0.  Group i
+  // spans [S_i, S_i + GROUP_COST + n_i) in cost units; its stage u sits at
+  // S_i + GROUP_COST + u.
   Group my_g{};
   int my_start = 0, T = 0;
   for (int c0 = 0; c0 < n_groups; c0 += GTHREADS) {
@@ -520,7 +528,7 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
     Group gd{};
     if (i < n_groups) gd = describe(p, i, HGN, c == 0);
     int tot;
-    const int ex = block_exclusive_scan(group_stages(gd), misc->red, &tot);
+    const int ex = block_exclusive_scan(group_cost(gd), misc->red, &tot);
     if (c0 == 0) { my_g = gd; my_start = ex; }
     T += tot;
   }
@@ -531,7 +539,7 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
   const int j1 = zero_all ? 0 : static_cast<int>((c + 1) * static_cast<long long>(T) / N);
   auto visit = [&](int i, const Group& gd, int st) {
     if (i >= n_groups) return;
-    const int n = group_stages(gd);
+    const int n = group_cost(gd);
     if (n > 0) {
       if (st <= j0 && j0 < st + n) {
         misc->first = gd;
@@ -555,7 +563,7 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
       Group gd{};
       if (i < n_groups) gd = describe(p, i, HGN, false);
       int tot;
-      const int ex = block_exclusive_scan(group_stages(gd), misc->red, &tot);
+      const int ex = block_exclusive_scan(group_cost(gd), misc->red, &tot);
       visit(i, gd, base + ex);
       base += tot;
     }
@@ -575,14 +583,16 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
     const int nbatch = NS < 32 ? NS : 32;
     Group g = misc->first;
     int gi = g.b * HGN + g.hg;
-    int u = j0 - g.start;
-    int j = j0;
+    int j = j0;        // position in cost units
     uint32_t jj = 0;   // CTA-local stage counter
     int q = 0;
     bool ok = true;
     while (j < j1 && ok) {
       const int gst = group_stages(g);
-      const int n = min(g.start + gst - j, j1 - j);
+      const int a = g.start + GROUP_COST, e = a + gst;   // the group's stages in cost units
+      if (a >= j1) break;                                // only its start cost falls in this range
+      const int u = max(j, a) - a;
+      const int n = min(e, j1) - max(j, a);
       const int slot = q % GQD;
       if (lane == 0) ok = mbar_wait(iqe0 + 8 * slot, ((q / GQD) & 1) ^ 1, abort_flag, status);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -592,16 +602,16 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
         sq.g = g;
         sq.u0 = u;
         sq.n = n;
-        const int cf = cta_of(g.start, T, N);
+        const int cf = cta_of(a, T, N);
         sq.k = c - cf;
-        sq.nseg = cta_of(g.start + gst - 1, T, N) - cf + 1;
+        sq.nseg = cta_of(e - 1, T, N) - cf + 1;
         segq[slot] = sq;
         mbar_arrive(iqf0 + 8 * slot);
       }
       // the next group's descriptor (its loads overlap the copies below)
       int gn = gi + 1;
       Group nxt{};
-      if (j + n < j1) nxt = describe(p, gn, HGN, false);
+      if (e < j1) nxt = describe(p, gn, HGN, false);
       // stages u .. u+n-1: one lane per stage, batches of at most NS stages
       for (int base = 0; base < n; base += nbatch) {
         bool lane_ok = true;
@@ -623,15 +633,13 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
         if (!ok) break;
       }
       jj += n;
-      j += n;
+      j = e;
       ++q;
       if (j < j1 && ok) {
-        const int next_start = g.start + gst;
         while (group_stages(nxt) == 0) nxt = describe(p, ++gn, HGN, false);   // empty sequences own no stage
-        nxt.start = next_start;
+        nxt.start = e;
         gi = gn;
         g = nxt;
-        u = 0;
       }
     }
     if (ok) {
@@ -666,12 +674,18 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
   const int h0 = 2 * t, h1 = 2 * t + 1;
   int s = 0;          // stage of the next CTA-local stage index
   uint32_t par = 0;   // its fill parity
+  // partials whose arrival is deferred to the end: the CTA's first segment and its last
+  struct Deferred {
+    int b, hkv, nseg, k, gstart;
+  };
+  Deferred dfr0{0, 0, 0, 0, 0}, dfr1{0, 0, 0, 0, 0};
+  bool all_ok = true;
   auto advance = [&]() {
     if (++s == NS) { s = 0; par ^= 1u; }
   };
   for (int q = 0;; ++q) {
     const int slot = q % GQD;
-    if (!mbar_wait(iqf0 + 8 * slot, (q / GQD) & 1, abort_flag, status)) break;
+    if (!mbar_wait(iqf0 + 8 * slot, (q / GQD) & 1, abort_flag, status)) { all_ok = false; break; }
     const SegQ sq = segq[slot];
     __syncwarp();
     if (lane == 0) mbar_arrive(iqe0 + 8 * slot);
@@ -755,7 +769,7 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
         u += 1;
       }
     }
-    if (!ok) break;
+    if (!ok) { all_ok = false; break; }
 
     // ---- the segment's result for this warp's head
     if (cs.colsplit) {
@@ -785,7 +799,7 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
       continue;
     }
     // several CTAs share the group: partial to the workspace (slot 0 = this
-    // CTA's first segment, slot 1 = its last), the last to arrive merges
+    // CTA's first segment, slot 1 = its last); the last of them to arrive merges
     {
       const int slotp = (c * 2 + (q == 0 ? 0 : 1)) * GW + w;
       float* part = p.partials + static_cast<size_t>(slotp) * pstride;
@@ -802,23 +816,34 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
         if (g8 == 0) { r[D] = ws.m1; r[D + 1] = ws.l1; }
       }
     }
+    // arrive later: the fence and the counter round trips would stall the next segment
+    Deferred& dr = q == 0 ? dfr0 : dfr1;
+    dr.b = g.b; dr.hkv = hkv; dr.nseg = sq.nseg; dr.k = sq.k; dr.gstart = g.start;
+  }
+  if (all_ok && (dfr0.nseg > 0 || dfr1.nseg > 0)) {
     __threadfence();
     __syncwarp();
-    unsigned long long* ctr = merge_ctr + static_cast<size_t>(g.b) * p.Hkv + hkv;
-    int arrived = 0;
-    if (lane == 0) arrived = static_cast<int>(atomicAdd(ctr, 1ull)) + 1;
-    arrived = __shfl_sync(0xffffffffu, arrived, 0);
-    if (arrived != sq.nseg) continue;
-    if (lane == 0) *ctr = 0ull;   // every other segment has arrived: re-arm for the next call
-    __threadfence();
-    const int cf = c - sq.k;
-    PartRef pr;
-    pr.base = p.partials;
-    pr.cf = cf;
-    pr.first_is_last = g.start != static_cast<int>(cf * static_cast<long long>(T) / N);
-    pr.w = w;
-    pr.pstride = pstride;
-    merge_store_g<D>(p, pr, sq.nseg, g.b, hkv, lane);
+#pragma unroll
+    for (int d = 0; d < 2; ++d) {
+      const Deferred& dr = d == 0 ? dfr0 : dfr1;
+      if (dr.nseg == 0) continue;
+      unsigned long long* ctr = merge_ctr + static_cast<size_t>(dr.b) * p.Hkv + dr.hkv;
+      int arrived = 0;
+      if (lane == 0) arrived = static_cast<int>(atomicAdd(ctr, 1ull)) + 1;
+      arrived = __shfl_sync(0xffffffffu, arrived, 0);
+      if (arrived != dr.nseg) continue;
+      if (lane == 0) *ctr = 0ull;   // every other segment has arrived: re-arm for the next call
+      __threadfence();
+      const int cf = c - dr.k;
+      PartRef pr;
+      pr.base = p.partials;
+      pr.cf = cf;
+      // the group's segment on CTA cf is that CTA's last one when the CTA starts inside an earlier group
+      pr.first_is_last = static_cast<int>(cf * static_cast<long long>(T) / N) < dr.gstart;
+      pr.w = w;
+      pr.pstride = pstride;
+      merge_store_g<D>(p, pr, dr.nseg, dr.b, dr.hkv, lane);
+    }
   }
   warp_exit(p, merge_ctr, misc, lane);
 }

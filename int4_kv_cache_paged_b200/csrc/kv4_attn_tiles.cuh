@@ -40,11 +40,26 @@ struct ColSplit {
   int part0, part1;
 };
 
+// Query operand of the scores: q_rot * 2^e rounded to a 16-bit integer and split
+// into a signed high byte and an unsigned low byte (q = 256 hi + lo).  b[kk] is
+// the high-byte B fragment of 32-dim block kk, b[D/32 + kk] the low-byte one
+// (16x8x32 layout: register 0 holds dims 4t..4t+3 of column g, register 1
+// dims 16+4t..16+4t+3).  qs0/qs1: sum(q_rot) * scale_log2 of the thread's two
+// columns; kscale = scale_log2 * 2^-e.
 template <int D>
 struct QFrag {
   uint32_t b[D / 16][2];
   float qs0, qs1, kscale;
 };
+
+// Integer scores of one 32-dim block: A = the K codes as bytes (rows g and g+8,
+// dims 4t..4t+3 and 16+4t..16+4t+3), times both query planes.
+template <int D>
+__device__ __forceinline__ void qk_block(int (&hi)[4], int (&lo)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, const QFrag<D>& qf, int kk) {
+  imma_u8s8(hi, a0, a1, a2, a3, qf.b[kk][0], qf.b[kk][1]);
+  imma_u8u8(lo, a0, a1, a2, a3, qf.b[D / 32 + kk][0], qf.b[D / 32 + kk][1]);
+}
 
 template <int D>
 __device__ __forceinline__ void online_softmax_pv(WarpState<D>& ws, float x0, float x1, float x2, float x3,
@@ -93,29 +108,6 @@ __device__ __forceinline__ void pv_operands(float P0, float P1, float P2, float 
   }
 }
 
-// QK^T of one INT4 tile: acc = (q * 2^e) . codes for tokens g, g+8 and heads 2t, 2t+1.
-template <int D>
-__device__ __forceinline__ void qk_int4(uint32_t st, const QFrag<D>& qf, int lane, float (&acc)[4]) {
-  constexpr int NKK = D / 32;
-  uint32_t kw0[NKK], kw1[NKK];
-  if constexpr (D == 128) {
-    const uint4 a = lds128(st + lane * 16), bq = lds128(st + 512 + lane * 16);
-    kw0[0] = a.x; kw0[1] = a.y; kw0[2] = a.z; kw0[3] = a.w;
-    kw1[0] = bq.x; kw1[1] = bq.y; kw1[2] = bq.z; kw1[3] = bq.w;
-  } else {
-    const uint2 a = lds64(st + lane * 8), bq = lds64(st + 256 + lane * 8);
-    kw0[0] = a.x; kw0[1] = a.y; kw1[0] = bq.x; kw1[1] = bq.y;
-  }
-  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < NKK; ++kk) {
-    const uint32_t w0 = kw0[kk], w1 = kw1[kk];
-    mma_f16(acc, nib_lo(w0), nib_lo(w1), nib_hi(w0), nib_hi(w1), qf.b[2 * kk][0], qf.b[2 * kk][1]);
-    const uint32_t u0 = w0 >> 8, u1 = w1 >> 8;
-    mma_f16(acc, nib_lo(u0), nib_lo(u1), nib_hi(u0), nib_hi(u1), qf.b[2 * kk + 1][0], qf.b[2 * kk + 1][1]);
-  }
-}
-
 // P.V of one INT4 tile: o^T[m] += V^T codes * (hi + lo) weights.
 template <int D>
 __device__ __forceinline__ void pv_int4(uint32_t st, WarpState<D>& ws, int lane, uint32_t B0, uint32_t B1,
@@ -148,8 +140,9 @@ __device__ __forceinline__ void unit_int4(const uint32_t (&tile)[2], const QFrag
                                           const int (&valid)[2], uint32_t eb0, uint32_t eb1, const ColSplit& cs) {
   float x[NT][4];
   uint4 sz[NT];
-  // Q.K^T of the NT tiles, interleaved, each with two accumulators (even / odd
-  // k-steps): 2*NT independent chains of D/32 multiplies instead of NT chains of D/16.
+  // Q.K^T of the NT tiles on the integer tensor cores: each tile's K codes are
+  // unpacked to bytes with one mask per plane and multiplied by both query
+  // planes (2*NT independent accumulator chains of D/32 multiplies).
   constexpr int NKK = D / 32;
   uint32_t kw[NT][2][NKK];
 #pragma unroll
@@ -164,27 +157,25 @@ __device__ __forceinline__ void unit_int4(const uint32_t (&tile)[2], const QFrag
     }
     sz[u] = lds128(tile[u] + 16 * D + (lane >> 2) * 16);
   }
-  float acc[NT][2][4];
+  int ahi[NT][4], alo[NT][4];
 #pragma unroll
   for (int u = 0; u < NT; ++u)
 #pragma unroll
-    for (int e = 0; e < 2; ++e) acc[u][e][0] = acc[u][e][1] = acc[u][e][2] = acc[u][e][3] = 0.f;
+    for (int i = 0; i < 4; ++i) ahi[u][i] = alo[u][i] = 0;
 #pragma unroll
   for (int kk = 0; kk < NKK; ++kk) {
 #pragma unroll
     for (int u = 0; u < NT; ++u) {
       const uint32_t w0 = kw[u][0][kk], w1 = kw[u][1][kk];
-      mma_f16(acc[u][0], nib_lo(w0), nib_lo(w1), nib_hi(w0), nib_hi(w1), qf.b[2 * kk][0], qf.b[2 * kk][1]);
-      const uint32_t u0 = w0 >> 8, u1 = w1 >> 8;
-      mma_f16(acc[u][1], nib_lo(u0), nib_lo(u1), nib_hi(u0), nib_hi(u1), qf.b[2 * kk + 1][0], qf.b[2 * kk + 1][1]);
+      qk_block<D>(ahi[u], alo[u], w0 & 0x0F0F0F0Fu, w1 & 0x0F0F0F0Fu, (w0 >> 4) & 0x0F0F0F0Fu,
+                  (w1 >> 4) & 0x0F0F0F0Fu, qf, kk);
     }
   }
 #pragma unroll
   for (int u = 0; u < NT; ++u) {
-    float acc_u[4];
+    float acc2[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc_u[i] = acc[u][0][i] + acc[u][1][i];
-    float (&acc2)[4] = acc_u;
+    for (int i = 0; i < 4; ++i) acc2[i] = static_cast<float>(ahi[u][i] * 256 + alo[u][i]);
     const float sKg = half_lo(sz[u].x) * qf.kscale, zKg = half_hi(sz[u].x);
     const float sKg8 = half_lo(sz[u].y) * qf.kscale, zKg8 = half_hi(sz[u].y);
     x[u][0] = fmaf(acc2[0], sKg, zKg * qf.qs0);
@@ -271,11 +262,12 @@ __device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpS
                                           bool vg8, uint32_t empty_bar, const ColSplit& cs) {
   constexpr int NK = D / 16;
   uint32_t kw[2][NK], vw[2 * NK];
+  // K: per row (g, g+8) D/4 bytes at (D/4)*lane; word 2kk + hf holds dims 32kk + 16hf + 4t .. +3
 #pragma unroll
   for (int rowhi = 0; rowhi < 2; ++rowhi)
 #pragma unroll
     for (int kq = 0; kq < D / 64; ++kq) {
-      const uint4 a = lds128(st + 16 * (32 * (rowhi * (D / 64) + kq) + lane));
+      const uint4 a = lds128(st + rowhi * 8 * D + (D / 4) * lane + 16 * kq);
       kw[rowhi][4 * kq] = a.x; kw[rowhi][4 * kq + 1] = a.y; kw[rowhi][4 * kq + 2] = a.z; kw[rowhi][4 * kq + 3] = a.w;
     }
 #pragma unroll
@@ -286,12 +278,13 @@ __device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpS
   const uint4 sz = lds128(st + 32 * D + (lane >> 2) * 16);
   __syncwarp();
   if (lane == 0) mbar_arrive(empty_bar);
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int ahi[4] = {0, 0, 0, 0}, alo[4] = {0, 0, 0, 0};
 #pragma unroll
-  for (int k = 0; k < NK; ++k) {
-    const uint32_t w0 = kw[0][k], w1 = kw[1][k];
-    mma_f16(acc, byte_lo(w0), byte_lo(w1), byte_lo(w0 >> 8), byte_lo(w1 >> 8), qf.b[k][0], qf.b[k][1]);
-  }
+  for (int kk = 0; kk < D / 32; ++kk)
+    qk_block<D>(ahi, alo, kw[0][2 * kk], kw[1][2 * kk], kw[0][2 * kk + 1], kw[1][2 * kk + 1], qf, kk);
+  float acc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] = static_cast<float>(ahi[i] * 256 + alo[i]);
   const float sKg = half_lo(sz.x) * qf.kscale, zKg = half_hi(sz.x);
   const float sKg8 = half_lo(sz.y) * qf.kscale, zKg8 = half_hi(sz.y);
   float x0 = fmaf(acc[0], sKg, zKg * qf.qs0);
@@ -369,11 +362,22 @@ __device__ __forceinline__ void tile_bf16(uint32_t st, const QFrag<D>& qf, WarpS
 // fp16 with a power-of-two scale (INT4 cache) or plain bf16 (BF16 cache); the
 // tail holds sigma*log2(e)*sum(q) per column and the key scale factor.
 // sq: shared scratch of G*D floats for this warp.
+template <int D>
+__device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, int lane, QFrag<D>& qf);
+template <int D>
+__device__ __forceinline__ void store_qblob(uint8_t* blob, const QFrag<D>& qf, int lane);
+
 template <int D, bool BF16>
 __device__ __forceinline__ void build_qblob(const AttnParams& p, int b, int h, int lane, float* sq) {
   constexpr int VPL = D / 32;
   const int G = p.G;
   const int gw = b * p.Hkv + h;
+  if constexpr (!BF16) {   // INT4/INT8 caches: the integer query planes
+    QFrag<D> qf;
+    load_qfrag<D>(p, b, h, lane, qf);
+    store_qblob<D>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D), qf, lane);
+    return;
+  }
   float qsum[MAX_G];
   float amax = 0.f;
   const float rot_c = p.rot_c;
@@ -448,96 +452,107 @@ __device__ __forceinline__ void build_qblob(const AttnParams& p, int b, int h, i
 
 
 // The query operand of KV head h of batch entry b, built straight into the
-// registers of the 16x8x16 B fragments (no staging through memory).  Lane
-// (g8 = lane/4, t = lane%4) holds column g8 (query head g8 % G with the column
-// split, else g8, zero when that head does not exist) at dimensions
-// d = 16k + 8r + 2t + e, e in {0, 1}: dimension bits 0, 3 and 4.. are in-lane,
-// bits 1 and 2 are the lane bits 0 and 1.  The block-diagonal Hadamard runs in
-// ascending butterfly stages with the same fp32 operations as the rotation of
-// the keys, so q_rot is the same bf16 vector whichever lane holds it.
+// registers of the 16x8x32 B fragments.  Lane (g8 = lane/4, t = lane%4) holds
+// column g8 (query head g8 % G with the column split, else g8, zero when that
+// head does not exist) at dimensions d = 32kk + 16hf + 4t + j, j < 4: dimension
+// bits 0-1 (j), 4 (hf) and 5.. (kk) are in-lane, bits 2-3 are the lane bits 0-1.
+// The block-diagonal Hadamard runs in ascending butterfly stages with the same
+// fp32 operations as the rotation of the keys, so q_rot is the same bf16
+// vector whichever lane holds it.  Then q_rot * 2^e (max |q_rot| * 2^e in
+// [2^14, 2^15)) is rounded to a 16-bit integer and split into the planes
+// hi = floor(q / 256) (signed byte) and lo = q mod 256 (unsigned byte).
 template <int D>
 __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, int lane, QFrag<D>& qf) {
-  constexpr int NK = D / 16;
+  constexpr int NKK = D / 32;
   const int G = p.G, g8 = lane >> 2, t = lane & 3;
   const bool colsplit = (G == 1 || G == 2 || G == 4);
   const int gsrc = colsplit ? g8 % G : g8;
   const bool active = gsrc < G;
-  const uint16_t* src = p.q + (static_cast<long long>(b) * p.Hq + h * G + (active ? gsrc : 0)) * D + 2 * t;
-  float x[NK][2][2];
+  const uint16_t* src = p.q + (static_cast<long long>(b) * p.Hq + h * G + (active ? gsrc : 0)) * D + 4 * t;
+  float x[NKK][2][4];
 #pragma unroll
-  for (int k = 0; k < NK; ++k)
+  for (int kk = 0; kk < NKK; ++kk)
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const uint32_t w = active ? __ldg(reinterpret_cast<const unsigned int*>(src + 16 * k + 8 * r)) : 0u;
-      x[k][r][0] = __uint_as_float(w << 16);
-      x[k][r][1] = __uint_as_float(w & 0xFFFF0000u);
+    for (int hf = 0; hf < 2; ++hf) {
+      uint2 w = make_uint2(0u, 0u);
+      if (active) w = __ldg(reinterpret_cast<const uint2*>(src + 32 * kk + 16 * hf));
+      x[kk][hf][0] = __uint_as_float(w.x << 16);
+      x[kk][hf][1] = __uint_as_float(w.x & 0xFFFF0000u);
+      x[kk][hf][2] = __uint_as_float(w.y << 16);
+      x[kk][hf][3] = __uint_as_float(w.y & 0xFFFF0000u);
     }
   const int Bh = p.Bh;
-  // stage 1: dimension bit 0 (the two halves of one 32-bit word)
-  if (1 < Bh) {
+  // stages 1 and 2: dimension bits 0-1 (j)
 #pragma unroll
-    for (int k = 0; k < NK; ++k)
+  for (int jb = 1; jb <= 2; jb <<= 1) {
+    if (jb < Bh) {
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const float a = x[k][r][0], c = x[k][r][1];
-        x[k][r][0] = __fadd_rn(a, c);
-        x[k][r][1] = __fsub_rn(a, c);
-      }
+      for (int kk = 0; kk < NKK; ++kk)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if ((j & jb) == 0) {
+              const float a = x[kk][hf][j], c = x[kk][hf][j + jb];
+              x[kk][hf][j] = __fadd_rn(a, c);
+              x[kk][hf][j + jb] = __fsub_rn(a, c);
+            }
+    }
   }
-  // stages 2 and 4: dimension bits 1 and 2 live in lane bits 0 and 1
+  // stages 4 and 8: dimension bits 2-3 are the lane bits 0-1
 #pragma unroll
   for (int lm = 1; lm <= 2; lm <<= 1) {
-    if (2 * lm < Bh) {
+    if (4 * lm < Bh) {
       const bool upper = (t & lm) != 0;
 #pragma unroll
-      for (int k = 0; k < NK; ++k)
+      for (int kk = 0; kk < NKK; ++kk)
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
+        for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float o = __shfl_xor_sync(0xffffffffu, x[k][r][e], lm);
-            x[k][r][e] = upper ? __fsub_rn(o, x[k][r][e]) : __fadd_rn(x[k][r][e], o);
+          for (int j = 0; j < 4; ++j) {
+            const float o = __shfl_xor_sync(0xffffffffu, x[kk][hf][j], lm);
+            x[kk][hf][j] = upper ? __fsub_rn(o, x[kk][hf][j]) : __fadd_rn(x[kk][hf][j], o);
           }
     }
   }
-  // stage 8: dimension bit 3 (r)
-  if (8 < Bh) {
+  // stage 16: dimension bit 4 (hf)
+  if (16 < Bh) {
 #pragma unroll
-    for (int k = 0; k < NK; ++k)
+    for (int kk = 0; kk < NKK; ++kk)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float a = x[k][0][e], c = x[k][1][e];
-        x[k][0][e] = __fadd_rn(a, c);
-        x[k][1][e] = __fsub_rn(a, c);
+      for (int j = 0; j < 4; ++j) {
+        const float a = x[kk][0][j], c = x[kk][1][j];
+        x[kk][0][j] = __fadd_rn(a, c);
+        x[kk][1][j] = __fsub_rn(a, c);
       }
   }
-  // stages 16, 32, ...: dimension bits 4.. (k)
+  // stages 32, 64, ...: dimension bits 5.. (kk)
 #pragma unroll
-  for (int kb = 1; kb < NK; kb <<= 1) {
-    if (16 * kb < Bh) {
+  for (int kb = 1; kb < NKK; kb <<= 1) {
+    if (32 * kb < Bh) {
 #pragma unroll
-      for (int k = 0; k < NK; ++k)
-        if ((k & kb) == 0)
+      for (int kk = 0; kk < NKK; ++kk)
+        if ((kk & kb) == 0)
 #pragma unroll
-          for (int r = 0; r < 2; ++r)
+          for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const float a = x[k][r][e], c = x[k + kb][r][e];
-              x[k][r][e] = __fadd_rn(a, c);
-              x[k + kb][r][e] = __fsub_rn(a, c);
+            for (int j = 0; j < 4; ++j) {
+              const float a = x[kk][hf][j], c = x[kk + kb][hf][j];
+              x[kk][hf][j] = __fadd_rn(a, c);
+              x[kk + kb][hf][j] = __fsub_rn(a, c);
             }
     }
   }
   const float rot_c = p.rot_c;
   float amax = 0.f, qs = 0.f;
 #pragma unroll
-  for (int k = 0; k < NK; ++k)
+  for (int kk = 0; kk < NKK; ++kk)
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
+    for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float v = __bfloat162float(__float2bfloat16_rn(__fmul_rn(x[k][r][e], rot_c)));
-        x[k][r][e] = v;
+      for (int j = 0; j < 4; ++j) {
+        const float v = __bfloat162float(__float2bfloat16_rn(__fmul_rn(x[kk][hf][j], rot_c)));
+        x[kk][hf][j] = v;
         qs += v;
         amax = fmaxf(amax, fabsf(v));
       }
@@ -545,21 +560,44 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
   qs += __shfl_xor_sync(0xffffffffu, qs, 2);
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  // fp16 operands: q * 2^e with max|q| * 2^e in [2^14, 2^15) (exact for normal values)
-  int ex2e = 0;
+  int e = 0;
   if (amax > 0.f && amax <= 3.0e38f) {
     int ex;
     frexpf(amax, &ex);
-    ex2e = 15 - ex;
+    e = 15 - ex;
   }
 #pragma unroll
-  for (int k = 0; k < NK; ++k)
+  for (int kk = 0; kk < NKK; ++kk)
 #pragma unroll
-    for (int r = 0; r < 2; ++r) qf.b[k][r] = pack_half2(ldexpf(x[k][r][0], ex2e), ldexpf(x[k][r][1], ex2e));
+    for (int hf = 0; hf < 2; ++hf) {
+      uint32_t whi = 0u, wlo = 0u;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int qi = __float2int_rn(ldexpf(x[kk][hf][j], e));   // |qi| < 2^15
+        whi |= (static_cast<uint32_t>(qi >> 8) & 0xFFu) << (8 * j);
+        wlo |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * j);
+      }
+      qf.b[kk][hf] = whi;
+      qf.b[NKK + kk][hf] = wlo;
+    }
   // sum(q) of the heads of this lane's columns 2t and 2t+1 (held by lanes 8t and 8t+4)
   qf.qs0 = __shfl_sync(0xffffffffu, qs, 8 * t) * p.scale_log2;
   qf.qs1 = __shfl_sync(0xffffffffu, qs, 8 * t + 4) * p.scale_log2;
-  qf.kscale = ldexpf(p.scale_log2, -ex2e);
+  qf.kscale = ldexpf(p.scale_log2, -e);
+}
+
+// Store a query operand as the 16*D + 64 byte blob the attention kernels read:
+// the 16-byte B-fragment words of every lane, then the sums of the 8 columns
+// and kscale.
+template <int D>
+__device__ __forceinline__ void store_qblob(uint8_t* blob, const QFrag<D>& qf, int lane) {
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc)
+    reinterpret_cast<uint4*>(blob)[cc * 32 + lane] =
+        make_uint4(qf.b[2 * cc][0], qf.b[2 * cc][1], qf.b[2 * cc + 1][0], qf.b[2 * cc + 1][1]);
+  float* tail = reinterpret_cast<float*>(blob + 16 * D);
+  if (lane < 4) { tail[2 * lane] = qf.qs0; tail[2 * lane + 1] = qf.qs1; }   // lanes 0-3: columns 2t, 2t+1
+  if (lane == 0) tail[MAX_G] = qf.kscale;
 }
 
 }  // namespace tiles
