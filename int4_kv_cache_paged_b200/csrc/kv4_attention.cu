@@ -407,12 +407,13 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(AttnParams p) {
       } else {
         const int valid[2] = {valid_bits(0), valid_bits(1)};
         const uint32_t tl[2] = {st, st + static_cast<uint32_t>(tile4_bytes(D))};
+        const uint32_t ebs[2] = {eb, eb};
         if (nt == 2) {
-          if (inside) unit_int4<D, 2, false>(tl, qf, ws, lane, valid, eb, eb, cs);
-          else unit_int4<D, 2, true>(tl, qf, ws, lane, valid, eb, eb, cs);
+          if (inside) unit_int4<D, 2, false>(tl, qf, ws, lane, valid, ebs, cs);
+          else unit_int4<D, 2, true>(tl, qf, ws, lane, valid, ebs, cs);
         } else {
-          if (inside) unit_int4<D, 1, false>(tl, qf, ws, lane, valid, eb, eb, cs);
-          else unit_int4<D, 1, true>(tl, qf, ws, lane, valid, eb, eb, cs);
+          if (inside) unit_int4<D, 1, false>(tl, qf, ws, lane, valid, ebs, cs);
+          else unit_int4<D, 1, true>(tl, qf, ws, lane, valid, ebs, cs);
         }
       }
     }

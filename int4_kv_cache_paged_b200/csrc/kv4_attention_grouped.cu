@@ -488,10 +488,10 @@ __device__ __forceinline__ void warp_exit(const AttnParams& p, unsigned long lon
   if (lane == 0) p.state->cta_done = 0;
 }
 
-// PAIR = INT4 tiles per iteration of a consumer warp: 2 (more independent work
-// per warp, 1 CTA per SM) or 1 (fewer registers, 2 CTAs per SM).
+// PAIR = INT4 tiles per iteration of a consumer warp: 2 or 4 (more independent
+// work per warp, 1 CTA per SM) or 1 (fewer registers, 2 CTAs per SM).
 template <int D, int PAIR>
-__global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p, unsigned long long* merge_ctr) {
+__global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(AttnParams p, unsigned long long* merge_ctr) {
   using C = GCfg<D>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int NS = p.ns;
@@ -716,35 +716,40 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
     bool ok = true;
     for (int u = sq.u0; u < u_end && ok;) {
       if (u < g.n4) {
-        // one or two INT4 stages: the tiles of this warp's head
-        const int nt = (PAIR == 2 && u + 1 < u_end && u + 1 < g.n4) ? 2 : 1;
-        const int s0 = s;
-        const uint32_t p0 = par;
-        advance();
-        const int s1 = nt == 2 ? s : s0;
-        const uint32_t p1 = nt == 2 ? par : p0;
-        if (nt == 2) advance();
-        ok = mbar_wait(full0 + 8 * s0, p0, abort_flag, status);
-        if (ok && nt == 2) ok = mbar_wait(full0 + 8 * s1, p1, abort_flag, status);
+        // PAIR INT4 stages at once when the segment has that many left, else one:
+        // the tiles of this warp's head
+        const int avail = min(u_end, g.n4) - u;
+        const int nt = avail >= PAIR ? PAIR : 1;
+        uint32_t tl[PAIR], eb[PAIR];
+        int valid[PAIR];
+#pragma unroll
+        for (int k = 0; k < PAIR; ++k) {
+          if (k < nt) {
+            tl[k] = smem_u32(ring + static_cast<size_t>(s) * C::STAGE + w * tile4_bytes(D));
+            eb[k] = empty0 + 8 * s;
+            if (ok) ok = mbar_wait(full0 + 8 * s, par, abort_flag, status);
+            advance();
+          } else {
+            tl[k] = tl[0];
+            eb[k] = eb[0];
+          }
+        }
         if (!ok) break;
-        const uint32_t tl[2] = {smem_u32(ring + static_cast<size_t>(s0) * C::STAGE + w * tile4_bytes(D)),
-                                smem_u32(ring + static_cast<size_t>(s1) * C::STAGE + w * tile4_bytes(D))};
         const int pos0 = (g.t0 + u) * TILE;
         const bool inside = pos0 >= g.lo4 && pos0 + nt * TILE <= g.hi4;
-        const uint32_t eb0 = empty0 + 8 * s0, eb1 = empty0 + 8 * s1;
         if (inside) {
-          const int valid[2] = {3, 3};
-          if (nt == 2) unit_int4<D, PAIR, false>(tl, qf, ws, lane, valid, eb0, eb1, cs);
-          else unit_int4<D, 1, false>(tl, qf, ws, lane, valid, eb0, eb1, cs);
-        } else {
-          int valid[2];
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
+          for (int k = 0; k < PAIR; ++k) valid[k] = 3;
+          if (nt == PAIR) unit_int4<D, PAIR, false>(tl, qf, ws, lane, valid, eb, cs);
+          else unit_int4<D, 1, false>(tl, qf, ws, lane, valid, eb, cs);
+        } else {
+#pragma unroll
+          for (int k = 0; k < PAIR; ++k) {
             const int pg = pos0 + k * TILE + g8;
             valid[k] = (pg >= g.lo4 && pg < g.hi4 ? 1 : 0) | (pg + 8 >= g.lo4 && pg + 8 < g.hi4 ? 2 : 0);
           }
-          if (nt == 2) unit_int4<D, PAIR, true>(tl, qf, ws, lane, valid, eb0, eb1, cs);
-          else unit_int4<D, 1, true>(tl, qf, ws, lane, valid, eb0, eb1, cs);
+          if (nt == PAIR) unit_int4<D, PAIR, true>(tl, qf, ws, lane, valid, eb, cs);
+          else unit_int4<D, 1, true>(tl, qf, ws, lane, valid, eb, cs);
         }
         u += nt;
       } else {
@@ -851,6 +856,12 @@ __global__ void __launch_bounds__(GTHREADS, 3 - PAIR) gattn_kernel(AttnParams p,
 // ---------------------------------------------------------------------------
 // host side
 
+#ifndef KV4_GROUPED_PAIR
+#define KV4_GROUPED_PAIR 4
+#endif
+constexpr int kPair = KV4_GROUPED_PAIR;   // INT4 tiles per consumer iteration of the compiled variant
+static_assert(kPair == 1 || kPair == 2 || kPair == 4, "tiles per iteration");
+
 inline size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Grid of the kernel variant in use (CTAs per SM x SMs).
@@ -873,7 +884,7 @@ GLayout g_layout(const kv4_cache* c, int n_seqs) {
   return l;
 }
 
-// Ring depth for the kernel variant PAIR at its CTAs per SM (2 for PAIR 1, 1 for PAIR 2).
+// Ring depth for the kernel variant PAIR at its CTAs per SM (2 for PAIR 1, else 1).
 template <int D, int PAIR>
 int g_choose_ring(int device) {
   int optin = 0;
@@ -914,9 +925,7 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e;
-  if (c->gattn_pair == 1) e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, 1>, p, c->merge_ctr);
-  else e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, 2>, p, c->merge_ctr);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair>, p, c->merge_ctr);
   if (c->ev_after) cudaEventRecord(c->ev_after, stream);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
@@ -925,15 +934,9 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream) {
 
 bool grouped_path(const kv4_cache* c) { return !c->bf16 && c->cfg.num_kv_heads % GW == 0; }
 
-#ifndef KV4_GROUPED_PAIR
-#define KV4_GROUPED_PAIR 2
-#endif
-
 int grouped_ring(kv4_cache* c) {
-  c->gattn_pair = KV4_GROUPED_PAIR;
-  if (c->cfg.head_dim == 128)
-    return c->gattn_pair == 1 ? g_choose_ring<128, 1>(c->device) : g_choose_ring<128, 2>(c->device);
-  return c->gattn_pair == 1 ? g_choose_ring<64, 1>(c->device) : g_choose_ring<64, 2>(c->device);
+  c->gattn_pair = kPair;
+  return c->cfg.head_dim == 128 ? g_choose_ring<128, kPair>(c->device) : g_choose_ring<64, kPair>(c->device);
 }
 
 size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs) { return g_layout(c, n_seqs).total; }

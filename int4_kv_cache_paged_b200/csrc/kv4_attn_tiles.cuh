@@ -130,14 +130,14 @@ __device__ __forceinline__ void pv_int4(uint32_t st, WarpState<D>& ws, int lane,
   }
 }
 
-// One unit of NT (1 or 2) INT4 tiles at shared addresses tile[0], tile[1]:
+// One unit of NT INT4 tiles at shared addresses tile[0 .. NT-1]:
 // scores, one online-softmax update for the NT*16 tokens, P.V.  valid[u] bit 0 /
 // bit 1: token g / g+8 of tile u is inside the item's range (used when MASKED).
-// The stage(s) are handed back (empty barriers eb0, and eb1 when it differs)
-// after the last shared-memory load.
+// The stages are handed back (empty barriers eb[0 .. NT-1], each distinct one
+// once) after the last shared-memory load.
 template <int D, int NT, bool MASKED>
-__device__ __forceinline__ void unit_int4(const uint32_t (&tile)[2], const QFrag<D>& qf, WarpState<D>& ws, int lane,
-                                          const int (&valid)[2], uint32_t eb0, uint32_t eb1, const ColSplit& cs) {
+__device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& qf, WarpState<D>& ws, int lane,
+                                          const int* valid, const uint32_t* eb, const ColSplit& cs) {
   float x[NT][4];
   uint4 sz[NT];
   // Q.K^T of the NT tiles on the integer tensor cores: each tile's K codes are
@@ -240,8 +240,9 @@ __device__ __forceinline__ void unit_int4(const uint32_t (&tile)[2], const QFrag
       }
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(eb0);
-        if (eb1 != eb0) mbar_arrive(eb1);
+#pragma unroll
+        for (int k = 0; k < NT; ++k)
+          if (k == 0 || eb[k] != eb[k - 1]) mbar_arrive(eb[k]);
       }
 #pragma unroll
       for (int m = 0; m < D / 16; ++m) {
