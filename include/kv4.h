@@ -175,15 +175,18 @@ int kv4_attention_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_
  *   dev_workspace  >= kv4_attention_workspace_bytes(cache, n_seqs, max L, ...)
  * A sequence of length 0 gives an all-zero output row.  n_seqs <= max_seqs
  * (KV4_ERR_INVALID_ARG otherwise).  Calls on one cache must be ordered on one
- * stream: they share the cache's merge counters.
- * Steps, with num_kv_heads a multiple of 8: one persistent kernel.  Every CTA
+ * stream (they share the cache's state block), and a workspace must not be
+ * shared by calls that can run at the same time.
+ * Steps, with num_kv_heads a multiple of 8: a query kernel (rotation, integer
+ * tensor-core operands), then one persistent attention kernel: every CTA
  * derives the same stream-K split of all (sequence, 8-KV-head group) page
- * stages from the sequence lengths, rotates its query heads into tensor-core
- * operands, streams its stages through shared memory by bulk copies, turns
- * INT4/INT8 codes into operands in registers (online softmax), and stores
- * the rotated-back output; a group split over several CTAs is merged by the
- * last of them (log-sum-exp merge over the workspace partials).  With other
- * head counts: a planning kernel, a per-head split-K kernel and a merge kernel.
+ * stages from the sequence lengths, streams its stages through shared memory
+ * by bulk copies, turns INT4/INT8 codes into operands in registers (online
+ * softmax) and stores the rotated-back output of the groups it covers whole;
+ * groups split over several CTAs are finished by a merge kernel (log-sum-exp
+ * merge of the workspace partials, inverse rotation).  The three kernels are
+ * chained as programmatic dependents.  With other head counts: a planning
+ * kernel, a per-head split-K kernel and a merge kernel.
  */
 int kv4_decode_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs,
                          const void* q, void* out, float softmax_scale, int32_t mode,
@@ -232,7 +235,7 @@ int kv4_get_status(kv4_cache* cache, kv4_stream_t stream, int32_t* device_status
 
 /* Timing hook: record the CUDA events `ev_before` and `ev_after` (cudaEvent_t,
  * created by the caller on the cache's device) on the call's stream right
- * before and right after the split-K attention kernel of every later
+ * before the first and right after the last attention kernel of every later
  * kv4_decode_attention call on this cache.  NULL, NULL turns it off.  The
  * events stay owned by the caller. */
 int kv4_set_attention_events(kv4_cache* cache, void* ev_before, void* ev_after);

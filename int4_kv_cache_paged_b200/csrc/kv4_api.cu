@@ -35,7 +35,7 @@ int check_config(const kv4_config* c, bool bf16) {
 }
 
 struct Sizes {
-  size_t seq_lens, counters, pool, prot, layer_stride, pool_offset, total;
+  size_t seq_lens, pool, prot, layer_stride, pool_offset, total;
 };
 
 Sizes sizes_of(const kv4_config* c, bool bf16) {
@@ -43,15 +43,13 @@ Sizes sizes_of(const kv4_config* c, bool bf16) {
   const size_t Hkv = c->num_kv_heads, D = c->head_dim;
   const size_t tiles_per_page = c->page_size / kv4::TILE;
   s.seq_lens = align_up(sizeof(int32_t) * static_cast<size_t>(c->num_layers) * c->max_seqs);
-  // merge counters of the page-major attention kernel, one per (batch entry, KV head)
-  s.counters = bf16 ? 0 : align_up(sizeof(unsigned long long) * static_cast<size_t>(c->max_seqs) * Hkv);
   const size_t tile = bf16 ? kv4::tile16_bytes(static_cast<int>(D)) : kv4::tile4_bytes(static_cast<int>(D));
   s.pool = align_up(static_cast<size_t>(c->num_pages) * Hkv * tiles_per_page * tile);
   s.prot = bf16 ? 0
                 : align_up(static_cast<size_t>(c->max_seqs) * Hkv * kv4::n_prot_tiles(c->sink_tokens, c->recent_window) *
                            kv4::tile8_bytes(static_cast<int>(D)));
   s.layer_stride = s.pool + s.prot;
-  s.pool_offset = kv4::STATE_BYTES + s.seq_lens + s.counters;
+  s.pool_offset = kv4::STATE_BYTES + s.seq_lens;
   s.total = s.pool_offset + s.layer_stride * c->num_layers;
   return s;
 }
@@ -87,7 +85,6 @@ int create(const kv4_config* cfg, bool bf16, void* dev_buf, size_t bytes, int32_
   c->base = static_cast<uint8_t*>(dev_buf);
   c->state = reinterpret_cast<State*>(c->base);
   c->seq_lens = reinterpret_cast<int32_t*>(c->base + kv4::STATE_BYTES);
-  c->merge_ctr = s.counters ? reinterpret_cast<unsigned long long*>(c->base + kv4::STATE_BYTES + s.seq_lens) : nullptr;
   c->block_table = block_table;
   c->layer_stride = s.layer_stride;
   c->pool_offset = s.pool_offset;

@@ -29,10 +29,10 @@
 // waits for it only before its first operand read).  A group that one CTA
 // covers whole is normalised, rotated back and stored straight from registers;
 // a group split over several CTAs leaves one partial (m, l, o) per segment in
-// the workspace.  After its last segment each warp announces its partials (a
-// counter per batch entry and KV head); the warp that completes a count merges
-// them, stores the output and sets the counter back to zero.  A launch in
-// which a wait gave up zeroes all counters at its end.
+// the workspace, and a merge kernel launched as this kernel's programmatic
+// dependent (its blocks become resident while this grid still runs) combines
+// them, one warp per query head.  Every CTA records where the groups that
+// start in its range sit in the split, for that merge.
 #include "kv4_attn_tiles.cuh"
 
 namespace kv4 {
@@ -64,6 +64,17 @@ struct Group {
 };
 static_assert(sizeof(Group) == 48, "group size");
 
+// Where a head group sits in the split, written once per group by the CTA
+// whose range holds its start (and the totals by CTA 0), read by the merge kernel.
+struct GPlanRec {
+  int start;          // first cost unit of the group
+  int stages;         // its stages (0: an empty sequence)
+};
+struct GPlanHdr {
+  int T, N;           // total cost units, active CTAs
+  int pad[2];
+};
+
 struct SegQ {         // one queued segment
   Group g;
   int u0, n;          // local stages [u0, u0+n)
@@ -73,7 +84,7 @@ struct SegQ {         // one queued segment
 // Per-CTA bookkeeping in shared memory.
 struct GMisc {
   int abort;          // a wait gave up
-  int exited;         // warps of this CTA that are done
+  int pad1;
   int pad0;
   Group first;        // the group holding the CTA's first stage (start filled in)
   int n_empty;        // empty groups this CTA writes zeros for
@@ -255,170 +266,6 @@ __device__ __forceinline__ void store_head(const AttnParams& p, int b, int hkv, 
   }
 }
 
-// The partials of one KV head of a split group: segment k lives on CTA cf + k,
-// in that CTA's slot 0 (its first segment) or slot 1 (its last segment).
-struct PartRef {
-  const float* base;
-  int cf, first_is_last, w, pstride;
-  __device__ __forceinline__ const float* operator()(int k) const {
-    const int sl = (k == 0 && first_is_last) ? 1 : 0;
-    return base + static_cast<size_t>(((cf + k) * 2 + sl) * GW + w) * pstride;
-  }
-};
-
-// Merge of the nseg partials of one KV head (G query heads) and store, lane
-// major: lane l holds dimensions VPL*l .. VPL*l+VPL-1 of every head.  The
-// maxima and the denominators take one pass with a segment per lane; the
-// numerators then stream the partials with U segments' loads in flight, the
-// weight of each segment broadcast from the lane that computed it.
-template <int D, int GG>
-__device__ __noinline__ void merge_store(const AttnParams& p, const PartRef& parts, int nseg, int b, int hkv,
-                                         int lane, bool dry) {
-  constexpr int VPL = D / 32;
-  constexpr int HS = head_stride(D);
-  constexpr int U = GG >= 16 ? 1 : 16 / GG;
-  float M[GG], Lh[GG], acc[GG][VPL];
-#pragma unroll
-  for (int h = 0; h < GG; ++h) {
-    M[h] = NEG_INF;
-    Lh[h] = 0.f;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) acc[h][i] = 0.f;
-  }
-  auto load_o = [&](const float* r, int h, float (&v)[VPL]) {
-    if constexpr (VPL == 4) {
-      const float4 x = __ldcg(reinterpret_cast<const float4*>(r + h * HS) + lane);
-      v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-    } else {
-      const float2 x = __ldcg(reinterpret_cast<const float2*>(r + h * HS) + lane);
-      v[0] = x.x; v[1] = x.y;
-    }
-  };
-  if (nseg <= U) {
-    // one batch of loads: every partial at once
-    float mv[U][GG], lv[U][GG], v[U][GG][VPL];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const float* r = parts(min(u, nseg - 1));
-#pragma unroll
-      for (int h = 0; h < GG; ++h) {
-        mv[u][h] = __ldcg(r + h * HS + D);
-        lv[u][h] = __ldcg(r + h * HS + D + 1);
-        load_o(r, h, v[u][h]);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int h = 0; h < GG; ++h) M[h] = fmaxf(M[h], mv[u][h]);
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int h = 0; h < GG; ++h) {
-        const float f = u < nseg ? ex2(mv[u][h] - M[h]) : 0.f;
-        Lh[h] = fmaf(f, lv[u][h], Lh[h]);
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) acc[h][i] = fmaf(f, v[u][h][i], acc[h][i]);
-      }
-  } else {
-    // maxima with one segment per lane (the first 32 segments' m, l stay in registers)
-    float m0[GG], l0[GG];
-#pragma unroll
-    for (int h = 0; h < GG; ++h) { m0[h] = NEG_INF; l0[h] = 0.f; }
-    if (lane < nseg) {
-      const float* r = parts(lane);
-#pragma unroll
-      for (int h = 0; h < GG; ++h) { m0[h] = __ldcg(r + h * HS + D); l0[h] = __ldcg(r + h * HS + D + 1); M[h] = m0[h]; }
-    }
-    for (int k = lane + 32; k < nseg; k += 32) {
-      const float* r = parts(k);
-#pragma unroll
-      for (int h = 0; h < GG; ++h) M[h] = fmaxf(M[h], __ldcg(r + h * HS + D));
-    }
-#pragma unroll
-    for (int h = 0; h < GG; ++h)
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) M[h] = fmaxf(M[h], __shfl_xor_sync(0xffffffffu, M[h], o));
-    for (int k0 = 0; k0 < nseg; k0 += 32) {
-      float fr[GG];
-      const int k = k0 + lane;
-      if (k0 > 0 && k < nseg) {
-        const float* r = parts(k);
-#pragma unroll
-        for (int h = 0; h < GG; ++h) { m0[h] = __ldcg(r + h * HS + D); l0[h] = __ldcg(r + h * HS + D + 1); }
-      }
-#pragma unroll
-      for (int h = 0; h < GG; ++h) {
-        fr[h] = k < nseg ? ex2(m0[h] - M[h]) : 0.f;
-        Lh[h] = fmaf(fr[h], k < nseg ? l0[h] : 0.f, Lh[h]);
-      }
-      const int cnt = min(32, nseg - k0);
-      for (int kk = 0; kk < cnt; kk += U) {
-        float v[U][GG][VPL];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const float* r = parts(k0 + min(kk + u, cnt - 1));
-#pragma unroll
-          for (int h = 0; h < GG; ++h) load_o(r, h, v[u][h]);
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-#pragma unroll
-          for (int h = 0; h < GG; ++h) {
-            float f = __shfl_sync(0xffffffffu, fr[h], (kk + u) & 31);
-            if (kk + u >= cnt) f = 0.f;
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) acc[h][i] = fmaf(f, v[u][h][i], acc[h][i]);
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < GG; ++h)
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) Lh[h] += __shfl_xor_sync(0xffffffffu, Lh[h], o);
-  }
-  const float rc = p.rot_c;
-  const int Bh = p.Bh;
-#pragma unroll
-  for (int h = 0; h < GG; ++h) {
-    float o[VPL];
-    const float inv = Lh[h] > 0.f ? 1.f / Lh[h] : 0.f;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) o[i] = acc[h][i] * inv;
-    fwht_row<VPL>(o, Bh, lane);   // o = H_blk o_rot (the normalised block Hadamard is its own inverse)
-    const long long off = (static_cast<long long>(b) * p.Hq + hkv * GG + h) * D + VPL * lane;
-    if (dry) continue;
-    if (p.mode & KV4_MODE_OUT_F32) {
-      float* out = static_cast<float*>(p.out) + off;
-      if constexpr (VPL == 4) *reinterpret_cast<float4*>(out) = make_float4(o[0] * rc, o[1] * rc, o[2] * rc, o[3] * rc);
-      else *reinterpret_cast<float2*>(out) = make_float2(o[0] * rc, o[1] * rc);
-    } else {
-      uint16_t* out = static_cast<uint16_t*>(p.out) + off;
-      if constexpr (VPL == 4)
-        *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf162(o[0] * rc, o[1] * rc), pack_bf162(o[2] * rc, o[3] * rc));
-      else
-        *reinterpret_cast<uint32_t*>(out) = pack_bf162(o[0] * rc, o[1] * rc);
-    }
-  }
-}
-
-template <int D>
-__device__ __forceinline__ void merge_store_g(const AttnParams& p, const PartRef& parts, int nseg, int b, int hkv,
-                                              int lane, bool dry = false) {
-  switch (p.G) {
-    case 1: merge_store<D, 1>(p, parts, nseg, b, hkv, lane, dry); break;
-    case 2: merge_store<D, 2>(p, parts, nseg, b, hkv, lane, dry); break;
-    case 3: merge_store<D, 3>(p, parts, nseg, b, hkv, lane, dry); break;
-    case 4: merge_store<D, 4>(p, parts, nseg, b, hkv, lane, dry); break;
-    case 5: merge_store<D, 5>(p, parts, nseg, b, hkv, lane, dry); break;
-    case 6: merge_store<D, 6>(p, parts, nseg, b, hkv, lane, dry); break;
-    case 7: merge_store<D, 7>(p, parts, nseg, b, hkv, lane, dry); break;
-    default: merge_store<D, 8>(p, parts, nseg, b, hkv, lane, dry); break;
-  }
-}
-
-
 // ---------------------------------------------------------------------------
 // query operands: one warp per (batch entry, KV head) rotates its G query
 // heads and stores the integer tensor-core B fragments of both query planes,
@@ -463,35 +310,10 @@ __device__ __forceinline__ const uint8_t* stage_source(const AttnParams& p, cons
                       tile8_bytes(D);
 }
 
-// Every warp of the CTA calls this once on its way out.  The last warp of the
-// CTA counts the CTA done; the last CTA of the launch re-arms the launch
-// counter and, if any CTA gave up a wait (its merges may be incomplete),
-// zeroes every merge counter.
-__device__ __forceinline__ void warp_exit(const AttnParams& p, unsigned long long* merge_ctr, GMisc* misc,
-                                          int lane) {
-  __syncwarp();
-  int last = 0;
-  if (lane == 0 && atomicAdd(&misc->exited, 1) == GW) {
-    if (misc->abort) atomicExch(&p.state->ctr_dirty, 1);
-    __threadfence();
-    last = atomicAdd(&p.state->cta_done, 1) == static_cast<int>(gridDim.x) - 1;
-  }
-  last = __shfl_sync(0xffffffffu, last, 0);
-  if (!last) return;
-  __threadfence();
-  if (*reinterpret_cast<volatile int*>(&p.state->ctr_dirty)) {
-    const int n = p.max_seqs * p.Hkv;
-    for (int i = lane; i < n; i += 32) merge_ctr[i] = 0ull;
-    __syncwarp();
-    if (lane == 0) p.state->ctr_dirty = 0;
-  }
-  if (lane == 0) p.state->cta_done = 0;
-}
-
 // PAIR = INT4 tiles per iteration of a consumer warp: 2 or 4 (more independent
 // work per warp, 1 CTA per SM) or 1 (fewer registers, 2 CTAs per SM).
 template <int D, int PAIR>
-__global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(AttnParams p, unsigned long long* merge_ctr) {
+__global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(AttnParams p, GPlanRec* plan) {
   using C = GCfg<D>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int NS = p.ns;
@@ -507,11 +329,12 @@ __global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(Attn
   const int c = blockIdx.x;
   const int HGN = p.Hkv / GW, n_groups = p.n_seqs * HGN;
 
+  // the merge kernel may be scheduled now: it waits for this grid before reading its results
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, GW); }
     for (int s = 0; s < GQD; ++s) { mbar_init(iqf0 + 8 * s, 1); mbar_init(iqe0 + 8 * s, GW); }
     misc->abort = 0;
-    misc->exited = 0;
     misc->n_empty = 0;
     for (int s = 0; s < MAX_NS; ++s) misc->last_fill[s] = -1;
     fence_barrier_init();
@@ -545,9 +368,11 @@ __global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(Attn
         misc->first = gd;
         misc->first.start = st;
       }
+      if (st >= j0 && st < j1) plan[i] = GPlanRec{st, group_stages(gd)};
     } else {
       const int owner = zero_all ? 0 : cta_of(min(st, T - 1), T, N);
       if (owner == c) {
+        plan[i] = GPlanRec{st, 0};
         const int k = atomicAdd(&misc->n_empty, 1);
         if (k < 32) misc->empty[k] = i;
         else zero_group(p, i, 0, 1);
@@ -568,13 +393,17 @@ __global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(Attn
       base += tot;
     }
   }
+  if (c == 0 && tid == 0) {
+    GPlanHdr* hdr = reinterpret_cast<GPlanHdr*>(plan + n_groups);
+    hdr->T = T;
+    hdr->N = static_cast<int>(N);
+  }
   __syncthreads();
   {
     const int ne = min(misc->n_empty, 32);
     for (int e = 0; e < ne; ++e) zero_group(p, misc->empty[e], tid, GTHREADS);
   }
   if (zero_all || c >= N || j0 >= j1) {
-    warp_exit(p, merge_ctr, misc, lane);
     return;
   }
 
@@ -657,7 +486,6 @@ __global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(Attn
                  globaltimer_ns() - t0 < 1000000000ull) {}
         }
     }
-    warp_exit(p, merge_ctr, misc, lane);
     return;
   }
 
@@ -674,18 +502,13 @@ __global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(Attn
   const int h0 = 2 * t, h1 = 2 * t + 1;
   int s = 0;          // stage of the next CTA-local stage index
   uint32_t par = 0;   // its fill parity
-  // partials whose arrival is deferred to the end: the CTA's first segment and its last
-  struct Deferred {
-    int b, hkv, nseg, k, gstart;
-  };
-  Deferred dfr0{0, 0, 0, 0, 0}, dfr1{0, 0, 0, 0, 0};
-  bool all_ok = true;
+
   auto advance = [&]() {
     if (++s == NS) { s = 0; par ^= 1u; }
   };
   for (int q = 0;; ++q) {
     const int slot = q % GQD;
-    if (!mbar_wait(iqf0 + 8 * slot, (q / GQD) & 1, abort_flag, status)) { all_ok = false; break; }
+    if (!mbar_wait(iqf0 + 8 * slot, (q / GQD) & 1, abort_flag, status)) break;
     const SegQ sq = segq[slot];
     __syncwarp();
     if (lane == 0) mbar_arrive(iqe0 + 8 * slot);
@@ -774,7 +597,7 @@ __global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(Attn
         u += 1;
       }
     }
-    if (!ok) { all_ok = false; break; }
+    if (!ok) break;
 
     // ---- the segment's result for this warp's head
     if (cs.colsplit) {
@@ -803,54 +626,107 @@ __global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(Attn
       store_head<D>(p, g.b, hkv, lane, ws.o, ws.l0, ws.l1);
       continue;
     }
-    // several CTAs share the group: partial to the workspace (slot 0 = this
-    // CTA's first segment, slot 1 = its last); the last of them to arrive merges
-    {
-      const int slotp = (c * 2 + (q == 0 ? 0 : 1)) * GW + w;
-      float* part = p.partials + static_cast<size_t>(slotp) * pstride;
-      if (h0 < G) {
-        float* r = part + h0 * HS;
+    // several CTAs share the group: its partial to the workspace (slot 0 = this
+    // CTA's first segment, slot 1 = its last), merged by the merge kernel
+    const int slotp = (c * 2 + (q == 0 ? 0 : 1)) * GW + w;
+    float* part = p.partials + static_cast<size_t>(slotp) * pstride;
+    if (h0 < G) {
+      float* r = part + h0 * HS;
 #pragma unroll
-        for (int m = 0; m < D / 16; ++m) { r[16 * m + g8] = ws.o[m][0]; r[16 * m + g8 + 8] = ws.o[m][2]; }
-        if (g8 == 0) { r[D] = ws.m0; r[D + 1] = ws.l0; }
-      }
-      if (h1 < G) {
-        float* r = part + h1 * HS;
-#pragma unroll
-        for (int m = 0; m < D / 16; ++m) { r[16 * m + g8] = ws.o[m][1]; r[16 * m + g8 + 8] = ws.o[m][3]; }
-        if (g8 == 0) { r[D] = ws.m1; r[D + 1] = ws.l1; }
-      }
+      for (int m = 0; m < D / 16; ++m) { r[16 * m + g8] = ws.o[m][0]; r[16 * m + g8 + 8] = ws.o[m][2]; }
+      if (g8 == 0) { r[D] = ws.m0; r[D + 1] = ws.l0; }
     }
-    // arrive later: the fence and the counter round trips would stall the next segment
-    Deferred& dr = q == 0 ? dfr0 : dfr1;
-    dr.b = g.b; dr.hkv = hkv; dr.nseg = sq.nseg; dr.k = sq.k; dr.gstart = g.start;
-  }
-  if (all_ok && (dfr0.nseg > 0 || dfr1.nseg > 0)) {
-    __threadfence();
-    __syncwarp();
+    if (h1 < G) {
+      float* r = part + h1 * HS;
 #pragma unroll
-    for (int d = 0; d < 2; ++d) {
-      const Deferred& dr = d == 0 ? dfr0 : dfr1;
-      if (dr.nseg == 0) continue;
-      unsigned long long* ctr = merge_ctr + static_cast<size_t>(dr.b) * p.Hkv + dr.hkv;
-      int arrived = 0;
-      if (lane == 0) arrived = static_cast<int>(atomicAdd(ctr, 1ull)) + 1;
-      arrived = __shfl_sync(0xffffffffu, arrived, 0);
-      if (arrived != dr.nseg) continue;
-      if (lane == 0) *ctr = 0ull;   // every other segment has arrived: re-arm for the next call
-      __threadfence();
-      const int cf = c - dr.k;
-      PartRef pr;
-      pr.base = p.partials;
-      pr.cf = cf;
-      // the group's segment on CTA cf is that CTA's last one when the CTA starts inside an earlier group
-      pr.first_is_last = static_cast<int>(cf * static_cast<long long>(T) / N) < dr.gstart;
-      pr.w = w;
-      pr.pstride = pstride;
-      merge_store_g<D>(p, pr, dr.nseg, dr.b, dr.hkv, lane);
+      for (int m = 0; m < D / 16; ++m) { r[16 * m + g8] = ws.o[m][1]; r[16 * m + g8 + 8] = ws.o[m][3]; }
+      if (g8 == 0) { r[D] = ws.m1; r[D + 1] = ws.l1; }
     }
   }
-  warp_exit(p, merge_ctr, misc, lane);
+}
+
+// ---------------------------------------------------------------------------
+// merge of the split groups: one warp per (batch entry, query head).  Launched
+// as the programmatic dependent of the attention kernel, so its blocks are
+// resident before the attention grid ends; it waits for that grid first.
+
+constexpr int MWARPS = 8;
+
+template <int D>
+__global__ void __launch_bounds__(32 * MWARPS) gmerge_kernel(AttnParams p, const GPlanRec* plan) {
+  constexpr int VPL = D / 32;
+  constexpr int HS = head_stride(D);
+  constexpr int U = 8;   // segments in flight
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * MWARPS + (threadIdx.x >> 5);
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // the partials and the plan are written
+  if (gw >= p.n_seqs * p.Hq) return;
+  const int G = p.G, HGN = p.Hkv / GW;
+  const int b = gw / p.Hq, hq = gw - b * p.Hq, hkv = hq / G, gq = hq - hkv * G;
+  const int hg = hkv / GW, w = hkv - hg * GW;
+  const GPlanHdr* hdr = reinterpret_cast<const GPlanHdr*>(plan + p.n_seqs * HGN);
+  const long long T = __ldcg(&hdr->T), N = __ldcg(&hdr->N);
+  const GPlanRec rec = {__ldcg(&plan[b * HGN + hg].start), __ldcg(&plan[b * HGN + hg].stages)};
+  if (rec.stages == 0 || N <= 0) return;   // empty sequence: zero rows written by the attention kernel
+  const int a = rec.start + GROUP_COST, e = a + rec.stages;
+  const int cf = cta_of(a, T, N);
+  const int nseg = cta_of(e - 1, T, N) - cf + 1;
+  if (nseg == 1) return;                   // stored by the attention kernel
+  // segment k sits on CTA cf + k, in its slot 0 (its first segment) or slot 1 (its last)
+  const bool first_is_last = cf * T / N < rec.start;
+  const int pstride = partial_stride(G, D);
+  auto row = [&](int k) -> const float* {
+    const int sl = (k == 0 && first_is_last) ? 1 : 0;
+    return p.partials + static_cast<size_t>(((cf + k) * 2 + sl) * GW + w) * pstride + gq * HS;
+  };
+  float M = NEG_INF;
+  for (int k = lane; k < nseg; k += 32) M = fmaxf(M, __ldcg(row(k) + D));
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float acc[VPL], L = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+  for (int k0 = 0; k0 < nseg; k0 += U) {
+    float v[U][VPL], mv[U], lv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float* r = row(min(k0 + u, nseg - 1));
+      mv[u] = __ldcg(r + D);
+      lv[u] = __ldcg(r + D + 1);
+      if constexpr (VPL == 4) {
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(r) + lane);
+        v[u][0] = x.x; v[u][1] = x.y; v[u][2] = x.z; v[u][3] = x.w;
+      } else {
+        const float2 x = __ldcg(reinterpret_cast<const float2*>(r) + lane);
+        v[u][0] = x.x; v[u][1] = x.y;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float f = k0 + u < nseg ? ex2(mv[u] - M) : 0.f;
+      L = fmaf(f, lv[u], L);
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) acc[i] = fmaf(f, v[u][i], acc[i]);
+    }
+  }
+  float o[VPL];
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) o[i] = acc[i] * inv;
+  fwht_row<VPL>(o, p.Bh, lane);   // o = H_blk o_rot (the normalised block Hadamard is its own inverse)
+  const float rc = p.rot_c;
+  const long long off = (static_cast<long long>(b) * p.Hq + hq) * D + VPL * lane;
+  if (p.mode & KV4_MODE_OUT_F32) {
+    float* out = static_cast<float*>(p.out) + off;
+    if constexpr (VPL == 4) *reinterpret_cast<float4*>(out) = make_float4(o[0] * rc, o[1] * rc, o[2] * rc, o[3] * rc);
+    else *reinterpret_cast<float2*>(out) = make_float2(o[0] * rc, o[1] * rc);
+  } else {
+    uint16_t* out = static_cast<uint16_t*>(p.out) + off;
+    if constexpr (VPL == 4)
+      *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf162(o[0] * rc, o[1] * rc), pack_bf162(o[2] * rc, o[3] * rc));
+    else
+      *reinterpret_cast<uint32_t*>(out) = pack_bf162(o[0] * rc, o[1] * rc);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -871,7 +747,7 @@ inline int g_grid(const kv4_cache* c) { return c->num_sms * (c->gattn_pair == 1 
 // partial slots per CTA and KV head of a group (the CTA's first and last
 // segment; segments in between cover whole groups and need none).
 struct GLayout {
-  size_t qblob, partials, total;
+  size_t qblob, partials, plan, total;
 };
 
 GLayout g_layout(const kv4_cache* c, int n_seqs) {
@@ -880,7 +756,9 @@ GLayout g_layout(const kv4_cache* c, int n_seqs) {
   GLayout l{};
   l.qblob = 0;
   l.partials = al256(static_cast<size_t>(n_seqs) * cfg.num_kv_heads * qblob_bytes(cfg.head_dim));
-  l.total = l.partials + al256(static_cast<size_t>(g_grid(c)) * 2 * GW * partial_stride(G, cfg.head_dim) * sizeof(float));
+  l.plan = l.partials + al256(static_cast<size_t>(g_grid(c)) * 2 * GW * partial_stride(G, cfg.head_dim) * sizeof(float));
+  const size_t n_groups = static_cast<size_t>(n_seqs) * (cfg.num_kv_heads / GW);
+  l.total = l.plan + al256(n_groups * sizeof(GPlanRec) + sizeof(GPlanHdr));
   return l;
 }
 
@@ -909,6 +787,7 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream) {
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   p.qblob = wsb + l.qblob;
   p.partials = reinterpret_cast<float*>(wsb + l.partials);
+  GPlanRec* plan = reinterpret_cast<GPlanRec*>(wsb + l.plan);
   p.grid = g_grid(c);
   p.cap_parts = p.grid * 2 * GW;
   p.ns = c->gattn_ring;
@@ -925,7 +804,14 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair>, p, c->merge_ctr);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair>, p, plan);
+  if (e == cudaSuccess) {
+    cudaLaunchConfig_t mcfg = cfg;
+    mcfg.gridDim = dim3((p.n_seqs * p.Hq + MWARPS - 1) / MWARPS);
+    mcfg.blockDim = dim3(32 * MWARPS);
+    mcfg.dynamicSmemBytes = 0;
+    e = cudaLaunchKernelEx(&mcfg, gmerge_kernel<D>, p, static_cast<const GPlanRec*>(plan));
+  }
   if (c->ev_after) cudaEventRecord(c->ev_after, stream);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
@@ -943,7 +829,7 @@ size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs) { return g_layout
 
 int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (ws_bytes < g_layout(c, p.n_seqs).total) return KV4_ERR_WORKSPACE;
-  if (c->gattn_ring <= 0 || c->gattn_ring > MAX_NS || !c->merge_ctr) return KV4_ERR_UNSUPPORTED;
+  if (c->gattn_ring <= 0 || c->gattn_ring > MAX_NS) return KV4_ERR_UNSUPPORTED;
   if (p.n_seqs > c->cfg.max_seqs) return KV4_ERR_INVALID_ARG;
   return p.D == 128 ? g_launch<128>(c, p, ws, stream) : g_launch<64>(c, p, ws, stream);
 }

@@ -49,9 +49,7 @@ struct State {
   int n_items[3];      // work items of the current attention call: full chunks, tails, protected
   int n_parts;         // partial slots allocated by the current attention call
   int work;            // next work item to claim (persistent attention kernel)
-  int ctr_dirty;       // a page-major launch gave up: its merge counters need zeroing
-  int cta_done;        // CTAs of the current page-major launch that finished
-  int pad[55];
+  int pad[57];
 };
 static_assert(sizeof(State) == STATE_BYTES, "state block size");
 
@@ -410,7 +408,6 @@ struct kv4_cache {
   int attn_ring;             // ring depth chosen for the per-head attention kernel
   int gattn_ring;            // ring depth of the page-major kernel (0: not used by this cache)
   int gattn_pair;            // INT4 tiles per consumer iteration of the page-major kernel (1 or 2)
-  unsigned long long* merge_ctr;   // [max_seqs][Hkv] arrival counters of the page-major kernel
   cudaEvent_t ev_before;     // optional timing events around the split-K kernel
   cudaEvent_t ev_after;
 };

@@ -47,11 +47,10 @@ def test_host_side_validation_without_a_device():
     good = dict(num_layers=1, max_seqs=2, num_q_heads=8, num_kv_heads=2, head_dim=128, page_size=16, num_pages=10,
                 max_pages_per_seq=5, hadamard_block=128, sink_tokens=4, recent_window=16)
     n = kv4.kv4_cache_required_bytes(kv4.make_config(**good))
-    # state 256 + seq_lens (256) + merge counters 2*2*8 (256) + pool 10*2*1*2176 + INT8 store 2*2*2*4224,
-    # each rounded to 256
+    # state 256 + seq_lens (256) + pool 10*2*1*2176 + INT8 store 2*2*2*4224, each rounded to 256
     pool = ((10 * 2 * 2176 + 255) // 256) * 256
     prot = ((2 * 2 * 2 * 4224 + 255) // 256) * 256
-    assert n == 256 + 256 + 256 + pool + prot
+    assert n == 256 + 256 + pool + prot
     for bad, code in ((dict(head_dim=96), kv4.KV4_ERR_UNSUPPORTED), (dict(num_q_heads=7), kv4.KV4_ERR_INVALID_ARG),
                       (dict(num_q_heads=32, num_kv_heads=2), kv4.KV4_ERR_UNSUPPORTED),
                       (dict(page_size=24), kv4.KV4_ERR_UNSUPPORTED), (dict(hadamard_block=3), kv4.KV4_ERR_INVALID_ARG),
