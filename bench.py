@@ -4,7 +4,8 @@
 One step = the whole hot path for one batch: fused rotate+quantize+append of one
 new token per sequence, then decode attention (query rotation; one persistent
 stream-K kernel over the INT4 pages and the INT8 sink/recent store that plans
-its own split, merges split groups and rotates the output back).  The metric is the algorithmic KV bytes the attention reads
+its own split and stores the groups it covers whole; a merge kernel for the
+groups split over several CTAs).  The metric is the algorithmic KV bytes the attention reads
 per step divided by the step time (GB/s), with decode tokens/s and the fraction
 of the measured HBM bandwidth beside it.
 
@@ -391,13 +392,14 @@ def run_gpu(args):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(achieved / hbm, 4), "traffic": traffic,
                          "kernel": "gattn_kernel: persistent stream-K attention over the INT4 pages and the "
-                                   "INT8 store with the merge of split groups (the events also cover the "
-                                   "query-operand kernel it overlaps)",
+                                   "INT8 store (the events span the whole attention call: the query-operand "
+                                   "kernel before it and the merge kernel after it, both overlapped as "
+                                   "programmatic dependents)",
                          "peak_source": peak_kind, "bytes_per_launch": int(bytes_timed / K)},
             "e2e": ({"value": round(e2e_bytes_all / t_e2e_all / 1e9, 2), "unit": "GB/s",
                      "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                      "tokens_per_s": round(B * world * K / t_e2e_all, 1)} if K_e2e else None),
-            "gpu_launches": 3 * K,   # per step: append_kernel, gq_kernel, gattn_kernel
+            "gpu_launches": 4 * K,   # per step: append_kernel, gq_kernel, gattn_kernel, gmerge_kernel
             "clocks": clk,
             "device_status": status,
             "setup_s": round(setup_s, 1),
