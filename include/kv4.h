@@ -151,6 +151,7 @@ int kv4_seq_reset(kv4_cache* cache, int32_t seq_id, kv4_stream_t stream);
  * p % P; positions p < S and p >= L_new - W are also INT8-encoded into the
  * sequence's protected store (sink slot p, or ring slot S + (p - S) mod W).
  * The sequence length of this layer advances by the number of new rows.
+ * At most 3413 sequences per call (KV4_ERR_UNSUPPORTED above).
  */
 int kv4_rotate_quantize_append(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids,
                                const int32_t* dev_cu_new, int32_t n_seqs, int32_t total_new,

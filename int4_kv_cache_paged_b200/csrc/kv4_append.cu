@@ -135,8 +135,9 @@ __device__ __forceinline__ int find_seq(const int* cu, int n_seqs, int n) {
   return lo;
 }
 
-// Last block of an append launch: advance the sequence lengths and re-arm the counter.
-__device__ void finish_append(const AppendParams& p) {
+// Last block of an append launch: advance the sequence lengths (from the old
+// lengths every block read at its start) and re-arm the counter.
+__device__ void finish_append(const AppendParams& p, const int* s_cu, const int* s_seq, const int* s_len) {
   __shared__ int s_last;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -148,10 +149,10 @@ __device__ void finish_append(const AppendParams& p) {
   __threadfence();
   const int cap = p.max_pages_per_seq * p.P;
   for (int i = threadIdx.x; i < p.n_seqs; i += blockDim.x) {
-    const int seq = p.seq_ids[i];
+    const int seq = s_seq[i];
     if (seq < 0 || seq >= p.max_seqs) continue;
-    const int n = p.cu_new[i + 1] - p.cu_new[i];
-    const int L = p.seq_lens[seq];
+    const int n = s_cu[i + 1] - s_cu[i];
+    const int L = s_len[i];
     if (n > 0 && L + n <= cap) p.seq_lens[seq] = L + n;
   }
   __syncthreads();
@@ -161,10 +162,22 @@ __device__ void finish_append(const AppendParams& p) {
 template <int D, bool BF16>
 __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams p) {
   constexpr int VPL = D / 32;
-  extern __shared__ int s_cu[];
+  // cu_new [n+1], then the sequence ids [n], then their lengths before this append [n]
+  extern __shared__ int s_meta[];
+  int* s_cu = s_meta;
+  int* s_seq = s_meta + p.n_seqs + 1;
+  int* s_len = s_seq + p.n_seqs;
   __shared__ __align__(16) uint8_t s_codes[APPEND_WARPS][2][D];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i <= p.n_seqs; i += blockDim.x) s_cu[i] = p.cu_new[i];
+  for (int i = threadIdx.x; i <= p.n_seqs; i += blockDim.x) {
+    s_cu[i] = p.cu_new[i];
+    if (i < p.n_seqs) s_seq[i] = p.seq_ids[i];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < p.n_seqs; i += blockDim.x) {
+    const int seq = s_seq[i];
+    s_len[i] = (seq >= 0 && seq < p.max_seqs) ? p.seq_lens[seq] : 0;
+  }
   __syncthreads();
 
   const long long job = static_cast<long long>(blockIdx.x) * APPEND_WARPS + warp;
@@ -186,7 +199,7 @@ __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams 
       }
     }
     const int i = find_seq(s_cu, p.n_seqs, n);
-    const int seq = p.seq_ids[i];
+    const int seq = s_seq[i];
     const int cap = p.max_pages_per_seq * p.P;
     bool ok = true;
     if (seq < 0 || seq >= p.max_seqs) {
@@ -195,7 +208,7 @@ __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams 
     }
     int pos = 0, L_new = 0;
     if (ok) {
-      const int L_old = p.seq_lens[seq];
+      const int L_old = s_len[i];
       L_new = L_old + (s_cu[i + 1] - s_cu[i]);
       pos = L_old + (n - s_cu[i]);
       if (L_new > cap) {
@@ -276,7 +289,7 @@ __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams 
       }
     }
   }
-  finish_append(p);
+  finish_append(p, s_cu, s_seq, s_len);
 }
 
 // ---------------------------------------------------------------------------
@@ -388,8 +401,8 @@ int launch_append(kv4_cache* c, int layer, const int32_t* seq_ids, const int32_t
   const long long jobs = static_cast<long long>(total_new) * p.Hkv * 2;
   const long long blocks = (jobs + APPEND_WARPS - 1) / APPEND_WARPS;
   if (blocks > 0x7fffffffLL) return KV4_ERR_UNSUPPORTED;
-  const size_t smem = sizeof(int) * (n_seqs + 1);
-  if (smem > 48 * 1024) return KV4_ERR_UNSUPPORTED;
+  const size_t smem = sizeof(int) * (3 * static_cast<size_t>(n_seqs) + 1);
+  if (smem > 40 * 1024) return KV4_ERR_UNSUPPORTED;
   dim3 grid(static_cast<unsigned>(blocks)), block(32 * APPEND_WARPS);
   if (p.D == 128) {
     if (c->bf16) append_kernel<128, true><<<grid, block, smem, stream>>>(p);
