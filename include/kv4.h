@@ -178,9 +178,9 @@ int kv4_attention_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_
  * (KV4_ERR_INVALID_ARG otherwise).  Calls on one cache must be ordered on one
  * stream (they share the cache's state block), and a workspace must not be
  * shared by calls that can run at the same time.
- * Steps, with num_kv_heads a multiple of 8: a query kernel (rotation, integer
+ * Steps, with num_kv_heads a multiple of 4: a query kernel (rotation, integer
  * tensor-core operands), then one persistent attention kernel: every CTA
- * derives the same stream-K split of all (sequence, 8-KV-head group) page
+ * derives the same stream-K split of all (sequence, 4-KV-head group) page
  * stages from the sequence lengths, streams its stages through shared memory
  * by bulk copies, turns INT4/INT8 codes into operands in registers (online
  * softmax) and stores the rotated-back output of the groups it covers whole;
@@ -207,10 +207,10 @@ int kv4_decode_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq
  *
  * Arguments, results and errors are those of kv4_decode_attention, plus:
  *   KV4_ERR_SCRATCH when kv4_attention_workspace_bytes(cache, n_seqs, 0) is
- *   above KV4_NOALLOC_SCRATCH_BYTES (with 8 or more KV heads that is
+ *   above KV4_NOALLOC_SCRATCH_BYTES (with KV heads a multiple of 4 that is
  *   n_seqs * Hkv * (16*D + 64) bytes of query operands plus
- *   2 * SMs * 8 * G * (D + 4) * 4 bytes of partials, e.g. about 6.1 MB for 64
- *   sequences, 32/8 heads, D = 128, and 13.7 MB for 512 sequences);
+ *   2 * 3 * SMs * 4 * G * (D + 4) * 4 bytes of partials, e.g. about 8.6 MB for
+ *   64 sequences, 32/8 heads, D = 128 on 148 SMs, and 16.2 MB for 512);
  *   nothing is launched then.
  * The scratch is one per device and shared by every cache and stream of the
  * process on that device: calls that can run at the same time (two streams,

@@ -1,5 +1,5 @@
 // Page-major, stream-K decode attention over the paged INT4/INT8 cache, used
-// when the number of KV heads is a multiple of 8.
+// when the number of KV heads is a multiple of the group width (4).
 //
 // Method: "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
 // Serving", Abstract (fused attention over the paged, rotated token-wise INT4
@@ -8,10 +8,12 @@
 //
 // One launch does the attention proper (a small query kernel runs alongside).
 //
-// Work decomposition.  A head group is 8 consecutive KV heads of one sequence.
-// Its work is a list of stages: one stage per 16-token INT4 tile position (the
-// tiles of the 8 heads are contiguous in the head-innermost pool, one 17 KB
-// bulk copy), then two stages per INT8 protected tile (heads 0-3, heads 4-7).
+// Work decomposition.  A head group is GW (4) consecutive KV heads of one
+// sequence.  Its work is a list of stages: one stage per 16-token INT4 tile
+// position (the tiles of the group's heads are contiguous in the head-innermost
+// pool: one 8.7 KB bulk copy at D = 128), then two stages per INT8 protected
+// tile (each half of the heads).  Three CTAs share an SM: four consumer warps
+// per scheduler hide the latency of each warp's dependent tile math.
 // The stage lists of all head groups are concatenated, each group charged a
 // few extra units for the cost of starting it (T units in all), and CTA c of
 // the persistent grid takes units [c*T/N, (c+1)*T/N): every CTA gets the same
@@ -41,18 +43,25 @@ namespace {
 
 using namespace tiles;
 
-constexpr int GW = 8;                   // consumer warps = KV heads per group
+#ifndef KV4_GROUP_HEADS
+#define KV4_GROUP_HEADS 4
+#endif
+constexpr int GW = KV4_GROUP_HEADS;      // consumer warps = KV heads per group (4 or 8)
 constexpr int GTHREADS = 32 * (GW + 1);  // + producer warp
+// CTAs per SM: one with 8 heads; three with 4 heads (4 warps per scheduler,
+// which caps registers at 128 per thread)
+constexpr int CTAS_PER_SM = GW == 4 ? 3 : 1;
+static_assert(GW == 4 || GW == 8, "group width");
 constexpr int GQD = 2;                  // segment queue depth
 
 template <int D>
 struct GCfg {
-  static constexpr int STAGE4 = GW * tile4_bytes(D);        // one tile position, 8 heads
-  static constexpr int STAGE8 = (GW / 2) * tile8_bytes(D);  // one protected tile, 4 heads
+  static constexpr int STAGE4 = GW * tile4_bytes(D);        // one tile position of the group's heads
+  static constexpr int STAGE8 = (GW / 2) * tile8_bytes(D);  // half a protected tile position
   static constexpr int STAGE = STAGE4 > STAGE8 ? STAGE4 : STAGE8;
 };
 
-// One head group of the call: batch entry b, KV heads 8*hg .. 8*hg+7.
+// One head group of the call: batch entry b, KV heads GW*hg .. GW*hg+GW-1.
 struct Group {
   int b, seq, hg, L;  // index into seq_ids, sequence id, head group, sequence length
   int n4;             // INT4 stages (tiles t0 .. t0+n4-1)
@@ -313,7 +322,12 @@ __device__ __forceinline__ const uint8_t* stage_source(const AttnParams& p, cons
 // PAIR = INT4 tiles per iteration of a consumer warp: 2 or 4 (more independent
 // work per warp, 1 CTA per SM) or 1 (fewer registers, 2 CTAs per SM).
 template <int D, int PAIR>
-__global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(AttnParams p, GPlanRec* plan) {
+#if KV4_GROUP_HEADS == 4
+#define KV4_GATTN_BOUNDS __maxnreg__(128)
+#else
+#define KV4_GATTN_BOUNDS __launch_bounds__(GTHREADS, 1)
+#endif
+__global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
   using C = GCfg<D>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int NS = p.ns;
@@ -576,7 +590,7 @@ __global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(Attn
         }
         u += nt;
       } else {
-        // one INT8 stage: half (v & 1) of protected tile (v >> 1) holds heads 4*(v&1) .. +3
+        // one INT8 stage: half (v & 1) of protected tile (v >> 1) holds heads (GW/2)*(v&1) .. +GW/2-1
         const int v = u - g.n4;
         const int s0 = s;
         const uint32_t p0 = par;
@@ -584,8 +598,8 @@ __global__ void __launch_bounds__(GTHREADS, PAIR == 1 ? 2 : 1) gattn_kernel(Attn
         ok = mbar_wait(full0 + 8 * s0, p0, abort_flag, status);
         if (!ok) break;
         const uint32_t eb = empty0 + 8 * s0;
-        if ((v & 1) == (w >> 2)) {
-          const uint32_t st = smem_u32(ring + static_cast<size_t>(s0) * C::STAGE + (w & 3) * tile8_bytes(D));
+        if ((v & 1) == w / (GW / 2)) {
+          const uint32_t st = smem_u32(ring + static_cast<size_t>(s0) * C::STAGE + (w % (GW / 2)) * tile8_bytes(D));
           const int slot0 = (v >> 1) * TILE;
           const bool vg = slot0 + g8 < g.nprot, vg8 = slot0 + g8 + 8 < g.nprot;
           if (slot0 + TILE <= g.nprot) tile_int8<D, false>(st, qf, ws, lane, true, true, eb, cs);
@@ -733,7 +747,7 @@ __global__ void __launch_bounds__(32 * MWARPS) gmerge_kernel(AttnParams p, const
 // host side
 
 #ifndef KV4_GROUPED_PAIR
-#define KV4_GROUPED_PAIR 4
+#define KV4_GROUPED_PAIR (KV4_GROUP_HEADS == 4 ? 2 : 4)
 #endif
 constexpr int kPair = KV4_GROUPED_PAIR;   // INT4 tiles per consumer iteration of the compiled variant
 static_assert(kPair == 1 || kPair == 2 || kPair == 4, "tiles per iteration");
@@ -741,7 +755,7 @@ static_assert(kPair == 1 || kPair == 2 || kPair == 4, "tiles per iteration");
 inline size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Grid of the kernel variant in use (CTAs per SM x SMs).
-inline int g_grid(const kv4_cache* c) { return c->num_sms * (c->gattn_pair == 1 ? 2 : 1); }
+inline int g_grid(const kv4_cache* c) { return c->num_sms * CTAS_PER_SM; }
 
 // Workspace: the query operands of every (batch entry, KV head), then two
 // partial slots per CTA and KV head of a group (the CTA's first and last
@@ -769,7 +783,7 @@ int g_choose_ring(int device) {
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess) return -1;
   if (cudaFuncSetAttribute(gattn_kernel<D, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess)
     return -1;
-  const int want = PAIR == 1 ? 2 : 1;
+  const int want = CTAS_PER_SM;
   for (int ns = MAX_NS; ns >= 2; --ns) {
     const size_t smem = gattn_smem_bytes<D>(ns);
     if (smem > static_cast<size_t>(optin)) continue;

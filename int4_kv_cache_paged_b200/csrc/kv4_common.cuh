@@ -424,7 +424,7 @@ int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs
                      float softmax_scale, int mode, void* ws, size_t ws_bytes, cudaStream_t stream);
 size_t attention_workspace_bytes(const kv4_cache* c, int n_seqs, int max_ctx);
 int attention_blocks_per_sm(kv4_cache* c);
-// page-major path (INT4 cache, KV heads a multiple of 8)
+// page-major path (INT4 cache, KV heads a multiple of 4)
 bool grouped_path(const kv4_cache* c);
 int grouped_ring(kv4_cache* c);
 size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs);

@@ -1,4 +1,4 @@
-"""GPU parity of the page-major attention path (KV heads a multiple of 8) in the
+"""GPU parity of the page-major attention path (KV heads a multiple of 4) in the
 situations its single-launch plan has to get right: more head groups than one
 planning chunk, runs of empty sequences, one sequence spread over every CTA,
 every query-head ratio, and repeated calls (the merge counters of one call must
