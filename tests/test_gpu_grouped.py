@@ -51,7 +51,7 @@ def _populate(pair, rng, seqs, lens, Hkv, D, chunk=64):
 
 
 def test_many_groups_and_runs_of_empty_sequences(kv4):
-    """300 head groups (two planning chunks of the 288-thread CTA), 40 consecutive
+    """600 head groups (four planning chunks of the 160-thread CTA), 40 consecutive
     empty sequences owned by one CTA, many groups split between CTAs."""
     rng = np.random.default_rng(21)
     n, D, Hkv, Hq, mpps = 300, 64, 8, 16, 8
