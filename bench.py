@@ -413,7 +413,8 @@ def run_gpu(args):
 
 
 def compare_legs(torch, kv4, w, wl, K, device, flush):
-    """Attention-only time of the INT4 path, the INT4-only mode and the BF16-KV kernel on identical inputs."""
+    """Attention-only time of the INT4 path, the INT4-only mode, the multi-token query path and the BF16-KV
+    kernel on identical inputs."""
     B, Hkv, D, S, Wn = wl.B, w["Hkv"], w["D"], w["S"], w["W"]
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     qs = [workloads.queries(w, 0, 1000 + i, device=device) for i in range(K)]
@@ -441,6 +442,20 @@ def compare_legs(torch, kv4, w, wl, K, device, flush):
                               "kv_gbs": round(kv_bytes(L_now, Hkv, D, S, Wn) / t_int4 / 1e9, 1)},
            "int4_only": {"attention_ms": round(t_only * 1e3, 4),
                          "kv_gbs": round(kv_bytes(L_now, Hkv, D, S, Wn, int4_only=True) / t_only / 1e9, 1)}}
+    # multi-token query (speculative verification): the most query tokens whose
+    # heads fit one 8-column operand, causal over the same cache
+    T = 8 // (w["Hq"] // Hkv)
+    if T >= 2:
+        gen = torch.Generator(device=device).manual_seed(4242)
+        qx = [torch.randn((B, T, w["Hq"], D), generator=gen, device=device).to(torch.bfloat16) for _ in range(3)]
+        outx = torch.empty((B, T, w["Hq"], D), dtype=torch.bfloat16, device=device)
+        wsx = wl.cache.extend_workspace(B, T)
+        ix = iter(range(1 << 30))
+        t_ext = time_attn(lambda q: wl.cache.extend_attention(0, wl.seq_ids, qx[next(ix) % 3], out=outx,
+                                                                workspace=wsx))
+        res["extend"] = {"q_len": T, "attention_ms": round(t_ext * 1e3, 4),
+                         "kv_gbs": round(kv_bytes(L_now, Hkv, D, S, Wn) / t_ext / 1e9, 1),
+                         "query_tokens_per_s": round(B * T / t_ext, 1)}
     need = bf16_bytes(L_now, Hkv, D)
     free = torch.cuda.mem_get_info()[0]
     if need * 1.3 < free:

@@ -194,6 +194,32 @@ int kv4_decode_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq
                          void* dev_workspace, size_t ws_bytes, kv4_stream_t stream);
 
 /*
+ * Multi-token query (speculative verification, extend): attention of the
+ * last q_len cached positions of every sequence, each over the positions up
+ * to and including its own.  Query token i (0 = oldest) of a sequence of
+ * length L sits at position L - q_len + i and sees positions 0 .. L - q_len + i
+ * of the same effective view as kv4_decode_attention (INT8 for the S sinks and
+ * the last W positions of L, INT4 elsewhere; KV4_MODE_INT4_ONLY reads INT4 for
+ * all).  Append the q_len tokens first.  With q_len = 1 this is
+ * kv4_decode_attention.  ("SAW-INT4 ...", Abstract: fused attention over the
+ * paged quantized cache; the causal mask over the new tokens is the textbook
+ * one.)
+ *   q_len          1 <= q_len, q_len * (Hq/Hkv) <= 8: the query tokens and
+ *                  heads of one KV head share one 8-column tensor-core operand
+ *   q, out         bf16 [n_seqs][q_len][Hq][D] (out fp32 with KV4_MODE_OUT_F32)
+ *   dev_workspace  >= kv4_extend_workspace_bytes(cache, n_seqs, q_len, ...)
+ * A query token with no visible position (L < q_len - i) gets an all-zero row.
+ * Errors: KV4_ERR_UNSUPPORTED when num_kv_heads is not a multiple of 4 or
+ * q_len * Hq/Hkv > 8; the others as kv4_decode_attention.  Same kernels as
+ * kv4_decode_attention with KV heads a multiple of 4, with the operand columns
+ * standing for (query token, query head) pairs.
+ */
+int kv4_extend_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_t q_len, size_t* bytes);
+int kv4_extend_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs, int32_t q_len,
+                         const void* q, void* out, float softmax_scale, int32_t mode,
+                         void* dev_workspace, size_t ws_bytes, kv4_stream_t stream);
+
+/*
  * kv4_decode_attention_noalloc: kv4_decode_attention without a workspace
  * argument.  Its scratch (query operands and split-K partials) lives in a
  * static device array of this library, KV4_NOALLOC_SCRATCH_BYTES (16 MiB) per

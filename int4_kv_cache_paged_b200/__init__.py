@@ -54,7 +54,7 @@ KV4_VIEW_INT4 = 1
 EXPORTS = [
     "kv4_cache_required_bytes", "kv4_cache_create", "kv4_cache_destroy", "kv4_cache_layout", "kv4_seq_reset",
     "kv4_rotate_quantize_append", "kv4_attention_workspace_bytes", "kv4_decode_attention",
-    "kv4_decode_attention_noalloc",
+    "kv4_decode_attention_noalloc", "kv4_extend_workspace_bytes", "kv4_extend_attention",
     "kv4_dequantize_debug", "kv4_get_status", "kv4_set_attention_events", "kv4_status_string", "kv4_version",
     "kv4bf16_cache_required_bytes", "kv4bf16_cache_create", "kv4bf16_cache_destroy", "kv4bf16_cache_layout",
     "kv4bf16_append", "kv4bf16_attention_workspace_bytes", "kv4bf16_decode_attention", "kv4bf16_get_status",
@@ -83,6 +83,8 @@ _sigs = {
     "kv4_attention_workspace_bytes": (_I, [_P, _I, _I, ctypes.POINTER(_SZ)]),
     "kv4_decode_attention": (_I, [_P, _I, _P, _I, _P, _P, ctypes.c_float, _I, _P, _SZ, _P]),
     "kv4_decode_attention_noalloc": (_I, [_P, _I, _P, _I, _P, _P, ctypes.c_float, _I, _P]),
+    "kv4_extend_workspace_bytes": (_I, [_P, _I, _I, ctypes.POINTER(_SZ)]),
+    "kv4_extend_attention": (_I, [_P, _I, _P, _I, _I, _P, _P, ctypes.c_float, _I, _P, _SZ, _P]),
     "kv4_dequantize_debug": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "kv4_get_status": (_I, [_P, _P, ctypes.POINTER(_I)]),
     "kv4_set_attention_events": (_I, [_P, _P, _P]),
@@ -186,6 +188,20 @@ def kv4_decode_attention_noalloc(handle, layer, seq_ids, n_seqs, q, out, softmax
     _check(_lib.kv4_decode_attention_noalloc(handle, layer, _ptr(seq_ids), n_seqs, _ptr(q), _ptr(out),
                                              float(softmax_scale), mode, _stream(stream)),
            "kv4_decode_attention_noalloc")
+
+
+def kv4_extend_workspace_bytes(handle, n_seqs, q_len):
+    n = _SZ()
+    _check(_lib.kv4_extend_workspace_bytes(handle, n_seqs, q_len, ctypes.byref(n)), "kv4_extend_workspace_bytes")
+    return n.value
+
+
+def kv4_extend_attention(handle, layer, seq_ids, n_seqs, q_len, q, out, softmax_scale, mode, workspace,
+                         stream=None):
+    _check(_lib.kv4_extend_attention(handle, layer, _ptr(seq_ids), n_seqs, q_len, _ptr(q), _ptr(out),
+                                     float(softmax_scale), mode, _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)),
+           "kv4_extend_attention")
 
 
 def kv4_dequantize_debug(handle, layer, seq_id, start, count, view, k_out, v_out, stream=None):

@@ -4,7 +4,7 @@ import torch
 
 from . import (make_config, kv4_cache_required_bytes, kv4_cache_create, kv4_cache_destroy, kv4_cache_layout,
                kv4_seq_reset, kv4_rotate_quantize_append, kv4_attention_workspace_bytes, kv4_decode_attention,
-               kv4_decode_attention_noalloc,
+               kv4_decode_attention_noalloc, kv4_extend_workspace_bytes, kv4_extend_attention,
                kv4_dequantize_debug, kv4_get_status, kv4bf16_cache_required_bytes, kv4bf16_cache_create,
                kv4bf16_cache_destroy, kv4bf16_cache_layout, kv4bf16_append, kv4bf16_attention_workspace_bytes,
                kv4bf16_decode_attention, kv4bf16_get_status, KV4_VIEW_EFFECTIVE, KV4_MODE_OUT_F32)
@@ -99,6 +99,25 @@ class KV4Cache(_Base):
         if workspace is None:
             workspace = self.workspace(n)
         kv4_decode_attention(self.handle, layer, seq_ids, n, q, out, scale, mode, workspace, stream)
+        return out
+
+    def extend_workspace(self, n_seqs, q_len):
+        nbytes = kv4_extend_workspace_bytes(self.handle, n_seqs, q_len)
+        if self._ws is None or self._ws.numel() < nbytes:
+            self._ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def extend_attention(self, layer, seq_ids, q, out=None, scale=0.0, mode=0, workspace=None, stream=None):
+        """Attention of the last q.shape[1] positions of every sequence, each causal over the cache.
+
+        q: bf16 [n_seqs, q_len, Hq, D]; returns out of the same shape (fp32 with KV4_MODE_OUT_F32)."""
+        n, q_len = int(seq_ids.numel()), int(q.shape[1])
+        if out is None:
+            dt = torch.float32 if (mode & KV4_MODE_OUT_F32) else torch.bfloat16
+            out = torch.empty(q.shape, dtype=dt, device=self.device)
+        if workspace is None:
+            workspace = self.extend_workspace(n, q_len)
+        kv4_extend_attention(self.handle, layer, seq_ids, n, q_len, q, out, scale, mode, workspace, stream)
         return out
 
     def attention_noalloc(self, layer, seq_ids, q, out, scale=0.0, mode=0, stream=None):

@@ -145,6 +145,23 @@ int attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_t n_seq
   return kv4::launch_attention(c, layer, seq_ids, n_seqs, q, out, softmax_scale, mode, ws, ws_bytes, stream);
 }
 
+int extend_attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_t n_seqs, int32_t q_len,
+                     const void* q, void* out, float softmax_scale, int32_t mode, void* ws, size_t ws_bytes,
+                     cudaStream_t stream) {
+  if (!c || check_layer(c, layer)) return KV4_ERR_INVALID_ARG;
+  if (n_seqs < 0 || n_seqs > c->cfg.max_seqs || q_len < 1) return KV4_ERR_INVALID_ARG;
+  if (!kv4::grouped_path(c)) return KV4_ERR_UNSUPPORTED;
+  if (static_cast<long long>(q_len) * (c->cfg.num_q_heads / c->cfg.num_kv_heads) > kv4::MAX_G) return KV4_ERR_UNSUPPORTED;
+  if (n_seqs == 0) return KV4_OK;
+  if (!seq_ids || !q || !out || !ws) return KV4_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || reinterpret_cast<uintptr_t>(ws) % kAlign) return KV4_ERR_INVALID_ARG;
+  if (mode & ~(KV4_MODE_INT4_ONLY | KV4_MODE_OUT_F32)) return KV4_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return KV4_ERR_INVALID_ARG;
+  if (!select_device(c)) return KV4_ERR_CUDA;
+  return kv4::launch_extend_attention(c, layer, seq_ids, n_seqs, q_len, q, out, softmax_scale, mode, ws, ws_bytes,
+                                      stream);
+}
+
 int get_status(kv4_cache* c, cudaStream_t stream, int32_t* device_status) {
   if (!c || !device_status) return KV4_ERR_INVALID_ARG;
   if (!select_device(c)) return KV4_ERR_CUDA;
@@ -216,6 +233,22 @@ int kv4_decode_attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, in
   if (!c || c->bf16) return KV4_ERR_INVALID_ARG;
   return attention(c, layer, seq_ids, n_seqs, q, out, softmax_scale, mode, ws, ws_bytes,
                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+int kv4_extend_workspace_bytes(const kv4_cache* c, int32_t n_seqs, int32_t q_len, size_t* bytes) {
+  if (!c || c->bf16 || !bytes || n_seqs < 0 || q_len < 1) return KV4_ERR_INVALID_ARG;
+  if (!kv4::grouped_path(c)) return KV4_ERR_UNSUPPORTED;
+  if (static_cast<long long>(q_len) * (c->cfg.num_q_heads / c->cfg.num_kv_heads) > kv4::MAX_G) return KV4_ERR_UNSUPPORTED;
+  *bytes = kv4::grouped_workspace_bytes(c, n_seqs, q_len);
+  return KV4_OK;
+}
+
+int kv4_extend_attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_t n_seqs, int32_t q_len,
+                         const void* q, void* out, float softmax_scale, int32_t mode, void* ws, size_t ws_bytes,
+                         kv4_stream_t stream) {
+  if (!c || c->bf16) return KV4_ERR_INVALID_ARG;
+  return extend_attention(c, layer, seq_ids, n_seqs, q_len, q, out, softmax_scale, mode, ws, ws_bytes,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 int kv4_dequantize_debug(kv4_cache* c, int32_t layer, int32_t seq_id, int32_t start, int32_t count, int32_t view,

@@ -385,9 +385,10 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(AttnParams p) {
       const int nt = min(UT, cur.t_end - tile0);
       const int pos0 = tile0 * TILE;
       const bool inside = pos0 >= cur.lo && pos0 + nt * TILE <= cur.hi;
+      // bits 0-1: token g visible to both columns; bits 2-3: token g+8 (one query token per sequence here)
       auto valid_bits = [&](int k) {
         const int pg = pos0 + k * TILE + g;
-        return (pg >= cur.lo && pg < cur.hi ? 1 : 0) | (pg + 8 >= cur.lo && pg + 8 < cur.hi ? 2 : 0);
+        return (pg >= cur.lo && pg < cur.hi ? 3 : 0) | (pg + 8 >= cur.lo && pg + 8 < cur.hi ? 12 : 0);
       };
       const uint32_t eb = empty0 + 8 * s;
       if constexpr (BF16) {
@@ -398,12 +399,12 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(AttnParams p) {
           auto ok_pos = [&](int r) { return pos0 + r >= cur.lo && pos0 + r < cur.hi; };
           const uint32_t m01 = (ok_pos(2 * t) ? 0x0000FFFFu : 0u) | (ok_pos(2 * t + 1) ? 0xFFFF0000u : 0u);
           const uint32_t m89 = (ok_pos(2 * t + 8) ? 0x0000FFFFu : 0u) | (ok_pos(2 * t + 9) ? 0xFFFF0000u : 0u);
-          tile_bf16<D, true>(st, qf, ws, lane, vb & 1, vb & 2, eb, m01, m89);
+          tile_bf16<D, true>(st, qf, ws, lane, vb & 1, vb & 4, eb, m01, m89);
         }
       } else if (cur.kind == 1) {
         const int vb = valid_bits(0);
-        if (inside) tile_int8<D, false>(st, qf, ws, lane, true, true, eb, cs);
-        else tile_int8<D, true>(st, qf, ws, lane, vb & 1, vb & 2, eb, cs);
+        if (inside) tile_int8<D, false>(st, qf, ws, lane, 15, eb, cs);
+        else tile_int8<D, true>(st, qf, ws, lane, vb, eb, cs);
       } else {
         const int valid[2] = {valid_bits(0), valid_bits(1)};
         const uint32_t tl[2] = {st, st + static_cast<uint32_t>(tile4_bytes(D))};
@@ -667,6 +668,8 @@ void fill_common(const kv4_cache* c, int layer, const int32_t* seq_ids, int n_se
   p.Hq = cfg.num_q_heads;
   p.Hkv = cfg.num_kv_heads;
   p.G = cfg.num_q_heads / cfg.num_kv_heads;
+  p.Gh = p.G;
+  p.qlen = 1;
   p.D = cfg.head_dim;
   p.P = cfg.page_size;
   p.S = cfg.sink_tokens;
@@ -685,7 +688,7 @@ void fill_common(const kv4_cache* c, int layer, const int32_t* seq_ids, int n_se
 }
 
 size_t attention_workspace_bytes(const kv4_cache* c, int n_seqs, int max_ctx) {
-  if (grouped_path(c)) return grouped_workspace_bytes(c, n_seqs);
+  if (grouped_path(c)) return grouped_workspace_bytes(c, n_seqs, 1);
   const kv4_config& cfg = c->cfg;
   const long long cap_ctx = static_cast<long long>(cfg.max_pages_per_seq) * cfg.page_size;
   const long long ctx = (max_ctx <= 0 || max_ctx > cap_ctx) ? cap_ctx : max_ctx;
@@ -693,6 +696,21 @@ size_t attention_workspace_bytes(const kv4_cache* c, int n_seqs, int max_ctx) {
   const int ct = chunk_tiles_for(c, n_seqs);
   const long long cap0 = static_cast<long long>(n_seqs) * cfg.num_kv_heads * ((tiles + ct - 1) / ct);
   return ws_layout(c, n_seqs, static_cast<int>(cap0)).total;
+}
+
+// Attention of the last qlen positions of every sequence (the page-major path
+// with qlen * Hq/Hkv operand columns per KV head; token i of a sequence of
+// length L sees the positions 0 .. L - qlen + i).
+int launch_extend_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, int qlen, const void* q,
+                            void* out, float softmax_scale, int mode, void* ws, size_t ws_bytes,
+                            cudaStream_t stream) {
+  if (!grouped_path(c)) return KV4_ERR_UNSUPPORTED;
+  AttnParams p{};
+  fill_common(c, layer, seq_ids, n_seqs, q, out, softmax_scale, mode, p);
+  p.qlen = qlen;
+  p.G = qlen * p.Gh;
+  if (p.G > MAX_G) return KV4_ERR_UNSUPPORTED;
+  return launch_grouped(c, p, ws, ws_bytes, stream);
 }
 
 int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, const void* q, void* out,
@@ -743,6 +761,8 @@ int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs
   p.Hq = cfg.num_q_heads;
   p.Hkv = cfg.num_kv_heads;
   p.G = G;
+  p.Gh = G;
+  p.qlen = 1;
   p.D = D;
   p.P = cfg.page_size;
   p.S = cfg.sink_tokens;

@@ -186,14 +186,12 @@ __device__ Group describe(const AttnParams& p, int i, int HGN, bool flag_bad) {
 __device__ void zero_group(const AttnParams& p, int i, int e0, int step) {
   const int HGN = p.Hkv / GW;
   const int b = i / HGN, hg = i - b * HGN;
-  const long long base = (static_cast<long long>(b) * p.Hq + hg * GW * p.G) * p.D;
   const int n = GW * p.G * p.D;
-  if (p.mode & KV4_MODE_OUT_F32) {
-    float* out = static_cast<float*>(p.out) + base;
-    for (int e = e0; e < n; e += step) out[e] = 0.f;
-  } else {
-    uint16_t* out = static_cast<uint16_t*>(p.out) + base;
-    for (int e = e0; e < n; e += step) out[e] = 0;
+  for (int e = e0; e < n; e += step) {
+    const int r = e / p.D, d = e - r * p.D;   // r = KV head within the group * G + operand column
+    const long long off = q_row(p, b, hg * GW + r / p.G, r % p.G) * p.D + d;
+    if (p.mode & KV4_MODE_OUT_F32) static_cast<float*>(p.out)[off] = 0.f;
+    else static_cast<uint16_t*>(p.out)[off] = 0;
   }
 }
 
@@ -201,7 +199,7 @@ __device__ void zero_group(const AttnParams& p, int i, int e0, int step) {
 // holds o for heads 2t, 2t+1 (valid when < G) at dimensions 16m+g8 (o[m][0],
 // o[m][1]) and 16m+g8+8 (o[m][2], o[m][3]).  out = c_B * H_blk (o / l): the
 // normalised block Hadamard is its own inverse.
-template <int D>
+template <int D, bool MULTI>
 __device__ __forceinline__ void store_head(const AttnParams& p, int b, int hkv, int lane, float (&o)[D / 16][4],
                                            float l0, float l1) {
   constexpr int NM = D / 16;
@@ -256,7 +254,7 @@ __device__ __forceinline__ void store_head(const AttnParams& p, int b, int hkv, 
   for (int hp = 0; hp < 2; ++hp) {
     const int head = 2 * t + hp;
     if (head >= G) continue;
-    const long long row = (static_cast<long long>(b) * p.Hq + hkv * G + head) * D;
+    const long long row = (MULTI ? q_row(p, b, hkv, head) : static_cast<long long>(b) * p.Hq + hkv * G + head) * D;
     if (p.mode & KV4_MODE_OUT_F32) {
       float* out = static_cast<float*>(p.out) + row;
 #pragma unroll
@@ -320,8 +318,10 @@ __device__ __forceinline__ const uint8_t* stage_source(const AttnParams& p, cons
 }
 
 // PAIR = INT4 tiles per iteration of a consumer warp: 2 or 4 (more independent
-// work per warp, 1 CTA per SM) or 1 (fewer registers, 2 CTAs per SM).
-template <int D, int PAIR>
+// work per warp, 1 CTA per SM) or 1 (fewer registers, 2 CTAs per SM).  MULTI:
+// several query tokens per sequence (causal visibility per operand column);
+// the one-token variant carries none of that code.
+template <int D, int PAIR, bool MULTI>
 #if KV4_GROUP_HEADS == 4
 #define KV4_GATTN_BOUNDS __maxnreg__(128)
 #else
@@ -514,6 +514,10 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
   cs.part0 = cs.colsplit ? (2 * t) / G : 0;
   cs.part1 = cs.colsplit ? (2 * t + 1) / G : 0;
   const int h0 = 2 * t, h1 = 2 * t + 1;
+  // query token of the thread's columns (the last qlen positions are the
+  // query tokens; token i sees the positions up to L - qlen + i)
+  const int qt0 = MULTI ? (cs.colsplit ? h0 % G : h0) / p.Gh : 0;
+  const int qt1 = MULTI ? (cs.colsplit ? h1 % G : h1) / p.Gh : 0;
   int s = 0;          // stage of the next CTA-local stage index
   uint32_t par = 0;   // its fill parity
 
@@ -573,20 +577,26 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
         }
         if (!ok) break;
         const int pos0 = (g.t0 + u) * TILE;
-        const bool inside = pos0 >= g.lo4 && pos0 + nt * TILE <= g.hi4;
+        const int vis = g.L - (MULTI ? p.qlen : 1);   // the last position every query token sees
+        const bool inside = pos0 >= g.lo4 && pos0 + nt * TILE <= (MULTI ? min(g.hi4, vis + 1) : g.hi4);
         if (inside) {
 #pragma unroll
-          for (int k = 0; k < PAIR; ++k) valid[k] = 3;
+          for (int k = 0; k < PAIR; ++k) valid[k] = 15;
           if (nt == PAIR) unit_int4<D, PAIR, false>(tl, qf, ws, lane, valid, eb, cs);
           else unit_int4<D, 1, false>(tl, qf, ws, lane, valid, eb, cs);
         } else {
 #pragma unroll
           for (int k = 0; k < PAIR; ++k) {
             const int pg = pos0 + k * TILE + g8;
-            valid[k] = (pg >= g.lo4 && pg < g.hi4 ? 1 : 0) | (pg + 8 >= g.lo4 && pg + 8 < g.hi4 ? 2 : 0);
+            const bool r0 = pg >= g.lo4 && pg < g.hi4, r8 = pg + 8 >= g.lo4 && pg + 8 < g.hi4;
+            if constexpr (MULTI)
+              valid[k] = (r0 && pg <= vis + qt0 ? 1 : 0) | (r0 && pg <= vis + qt1 ? 2 : 0) |
+                         (r8 && pg + 8 <= vis + qt0 ? 4 : 0) | (r8 && pg + 8 <= vis + qt1 ? 8 : 0);
+            else
+              valid[k] = (r0 ? 3 : 0) | (r8 ? 12 : 0);
           }
-          if (nt == PAIR) unit_int4<D, PAIR, true>(tl, qf, ws, lane, valid, eb, cs);
-          else unit_int4<D, 1, true>(tl, qf, ws, lane, valid, eb, cs);
+          if (nt == PAIR) unit_int4<D, PAIR, true, MULTI>(tl, qf, ws, lane, valid, eb, cs);
+          else unit_int4<D, 1, true, MULTI>(tl, qf, ws, lane, valid, eb, cs);
         }
         u += nt;
       } else {
@@ -601,9 +611,25 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
         if ((v & 1) == w / (GW / 2)) {
           const uint32_t st = smem_u32(ring + static_cast<size_t>(s0) * C::STAGE + (w % (GW / 2)) * tile8_bytes(D));
           const int slot0 = (v >> 1) * TILE;
-          const bool vg = slot0 + g8 < g.nprot, vg8 = slot0 + g8 + 8 < g.nprot;
-          if (slot0 + TILE <= g.nprot) tile_int8<D, false>(st, qf, ws, lane, true, true, eb, cs);
-          else tile_int8<D, true>(st, qf, ws, lane, vg, vg8, eb, cs);
+          if (slot0 + TILE <= g.nprot && !MULTI) {
+            tile_int8<D, false>(st, qf, ws, lane, 15, eb, cs);
+          } else if (!MULTI) {
+            tile_int8<D, true>(st, qf, ws, lane, (slot0 + g8 < g.nprot ? 3 : 0) | (slot0 + g8 + 8 < g.nprot ? 12 : 0),
+                               eb, cs);
+          } else {
+            // position of protected slot sl: a sink below S, else the ring position
+            // in [max(S, L - W), L) congruent to sl - S modulo W
+            const int rlo = max(p.S, g.L - p.W), vis = g.L - p.qlen;
+            auto pos_of = [&](int sl) {
+              return sl < p.S ? sl : rlo + (((sl - p.S) - (rlo - p.S)) % p.W + p.W) % p.W;
+            };
+            const int sa = slot0 + g8, sb = sa + 8;
+            const bool ra = sa < g.nprot, rb = sb < g.nprot;
+            const int pa = pos_of(sa), pb = pos_of(sb);
+            const int vm = (ra && pa <= vis + qt0 ? 1 : 0) | (ra && pa <= vis + qt1 ? 2 : 0) |
+                           (rb && pb <= vis + qt0 ? 4 : 0) | (rb && pb <= vis + qt1 ? 8 : 0);
+            tile_int8<D, true, true>(st, qf, ws, lane, vm, eb, cs);
+          }
         } else {
           __syncwarp();
           if (lane == 0) mbar_arrive(eb);
@@ -637,7 +663,7 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
     for (int m = 0; m < D / 16; ++m) { ws.o[m][0] += ws.z0; ws.o[m][2] += ws.z0; ws.o[m][1] += ws.z1; ws.o[m][3] += ws.z1; }
     const int hkv = g.hg * GW + w;
     if (sq.nseg == 1) {
-      store_head<D>(p, g.b, hkv, lane, ws.o, ws.l0, ws.l1);
+      store_head<D, MULTI>(p, g.b, hkv, lane, ws.o, ws.l0, ws.l1);
       continue;
     }
     // several CTAs share the group: its partial to the workspace (slot 0 = this
@@ -674,9 +700,9 @@ __global__ void __launch_bounds__(32 * MWARPS) gmerge_kernel(AttnParams p, const
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * MWARPS + (threadIdx.x >> 5);
   asm volatile("griddepcontrol.wait;" ::: "memory");   // the partials and the plan are written
-  if (gw >= p.n_seqs * p.Hq) return;
-  const int G = p.G, HGN = p.Hkv / GW;
-  const int b = gw / p.Hq, hq = gw - b * p.Hq, hkv = hq / G, gq = hq - hkv * G;
+  const int G = p.G, HGN = p.Hkv / GW, per_b = p.Hkv * G;   // G: operand columns (query tokens x heads)
+  if (gw >= p.n_seqs * per_b) return;
+  const int b = gw / per_b, r = gw - b * per_b, hkv = r / G, gq = r - hkv * G;
   const int hg = hkv / GW, w = hkv - hg * GW;
   const GPlanHdr* hdr = reinterpret_cast<const GPlanHdr*>(plan + p.n_seqs * HGN);
   const long long T = __ldcg(&hdr->T), N = __ldcg(&hdr->N);
@@ -717,7 +743,8 @@ __global__ void __launch_bounds__(32 * MWARPS) gmerge_kernel(AttnParams p, const
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const float f = k0 + u < nseg ? ex2(mv[u] - M) : 0.f;
+      // a segment (or a column) with no visible position has m = -inf
+      const float f = (k0 + u < nseg && mv[u] != NEG_INF) ? ex2(mv[u] - M) : 0.f;
       L = fmaf(f, lv[u], L);
 #pragma unroll
       for (int i = 0; i < VPL; ++i) acc[i] = fmaf(f, v[u][i], acc[i]);
@@ -729,7 +756,7 @@ __global__ void __launch_bounds__(32 * MWARPS) gmerge_kernel(AttnParams p, const
   for (int i = 0; i < VPL; ++i) o[i] = acc[i] * inv;
   fwht_row<VPL>(o, p.Bh, lane);   // o = H_blk o_rot (the normalised block Hadamard is its own inverse)
   const float rc = p.rot_c;
-  const long long off = (static_cast<long long>(b) * p.Hq + hq) * D + VPL * lane;
+  const long long off = q_row(p, b, hkv, gq) * D + VPL * lane;
   if (p.mode & KV4_MODE_OUT_F32) {
     float* out = static_cast<float*>(p.out) + off;
     if constexpr (VPL == 4) *reinterpret_cast<float4*>(out) = make_float4(o[0] * rc, o[1] * rc, o[2] * rc, o[3] * rc);
@@ -764,9 +791,9 @@ struct GLayout {
   size_t qblob, partials, plan, total;
 };
 
-GLayout g_layout(const kv4_cache* c, int n_seqs) {
+GLayout g_layout(const kv4_cache* c, int n_seqs, int qlen) {
   const kv4_config& cfg = c->cfg;
-  const int G = cfg.num_q_heads / cfg.num_kv_heads;
+  const int G = qlen * (cfg.num_q_heads / cfg.num_kv_heads);   // operand columns per KV head
   GLayout l{};
   l.qblob = 0;
   l.partials = al256(static_cast<size_t>(n_seqs) * cfg.num_kv_heads * qblob_bytes(cfg.head_dim));
@@ -781,23 +808,30 @@ template <int D, int PAIR>
 int g_choose_ring(int device) {
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess) return -1;
-  if (cudaFuncSetAttribute(gattn_kernel<D, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess)
+  if (cudaFuncSetAttribute(gattn_kernel<D, PAIR, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(gattn_kernel<D, PAIR, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) !=
+          cudaSuccess)
     return -1;
   const int want = CTAS_PER_SM;
   for (int ns = MAX_NS; ns >= 2; --ns) {
     const size_t smem = gattn_smem_bytes<D>(ns);
     if (smem > static_cast<size_t>(optin)) continue;
     int blocks = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, gattn_kernel<D, PAIR>, GTHREADS, smem) != cudaSuccess)
+    int blocks_multi = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, gattn_kernel<D, PAIR, false>, GTHREADS, smem) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_multi, gattn_kernel<D, PAIR, true>, GTHREADS, smem) !=
+            cudaSuccess)
       return -1;
-    if (blocks >= want) return ns;
+    if (blocks >= want && blocks_multi >= want) return ns;
   }
   return -1;
 }
 
 template <int D>
 int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream) {
-  const GLayout l = g_layout(c, p.n_seqs);
+  const GLayout l = g_layout(c, p.n_seqs, p.qlen);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   p.qblob = wsb + l.qblob;
   p.partials = reinterpret_cast<float*>(wsb + l.partials);
@@ -818,10 +852,11 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair>, p, plan);
+  cudaError_t e = p.qlen > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true>, p, plan)
+                              : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false>, p, plan);
   if (e == cudaSuccess) {
     cudaLaunchConfig_t mcfg = cfg;
-    mcfg.gridDim = dim3((p.n_seqs * p.Hq + MWARPS - 1) / MWARPS);
+    mcfg.gridDim = dim3((p.n_seqs * p.Hkv * p.G + MWARPS - 1) / MWARPS);
     mcfg.blockDim = dim3(32 * MWARPS);
     mcfg.dynamicSmemBytes = 0;
     e = cudaLaunchKernelEx(&mcfg, gmerge_kernel<D>, p, static_cast<const GPlanRec*>(plan));
@@ -839,10 +874,11 @@ int grouped_ring(kv4_cache* c) {
   return c->cfg.head_dim == 128 ? g_choose_ring<128, kPair>(c->device) : g_choose_ring<64, kPair>(c->device);
 }
 
-size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs) { return g_layout(c, n_seqs).total; }
+size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs, int qlen) { return g_layout(c, n_seqs, qlen).total; }
 
 int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  if (ws_bytes < g_layout(c, p.n_seqs).total) return KV4_ERR_WORKSPACE;
+  if (p.qlen < 1 || p.G != p.qlen * p.Gh || p.G > MAX_G) return KV4_ERR_UNSUPPORTED;
+  if (ws_bytes < g_layout(c, p.n_seqs, p.qlen).total) return KV4_ERR_WORKSPACE;
   if (c->gattn_ring <= 0 || c->gattn_ring > MAX_NS) return KV4_ERR_UNSUPPORTED;
   if (p.n_seqs > c->cfg.max_seqs) return KV4_ERR_INVALID_ARG;
   return p.D == 128 ? g_launch<128>(c, p, ws, stream) : g_launch<64>(c, p, ws, stream);

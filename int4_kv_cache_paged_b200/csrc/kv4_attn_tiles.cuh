@@ -61,7 +61,7 @@ __device__ __forceinline__ void qk_block(int (&hi)[4], int (&lo)[4], uint32_t a0
   imma_u8u8(lo, a0, a1, a2, a3, qf.b[D / 32 + kk][0], qf.b[D / 32 + kk][1]);
 }
 
-template <int D>
+template <int D, bool GUARD = false>
 __device__ __forceinline__ void online_softmax_pv(WarpState<D>& ws, float x0, float x1, float x2, float x3,
                                                   float& p0, float& p1, float& p2, float& p3) {
   float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
@@ -72,7 +72,9 @@ __device__ __forceinline__ void online_softmax_pv(WarpState<D>& ws, float x0, fl
   }
   const float n0 = fmaxf(ws.m0, mx0), n1 = fmaxf(ws.m1, mx1);
   if (__any_sync(0xffffffffu, n0 > ws.m0 || n1 > ws.m1)) {
-    const float a0 = ex2(ws.m0 - n0), a1 = ex2(ws.m1 - n1);
+    // GUARD: a column with no visible position so far keeps m = -inf and a zero state
+    const float a0 = (GUARD && n0 == NEG_INF) ? 1.f : ex2(ws.m0 - n0);
+    const float a1 = (GUARD && n1 == NEG_INF) ? 1.f : ex2(ws.m1 - n1);
     ws.l0 *= a0; ws.l1 *= a1; ws.z0 *= a0; ws.z1 *= a1;
 #pragma unroll
     for (int m = 0; m < D / 16; ++m) {
@@ -80,7 +82,8 @@ __device__ __forceinline__ void online_softmax_pv(WarpState<D>& ws, float x0, fl
     }
     ws.m0 = n0; ws.m1 = n1;
   }
-  p0 = ex2(x0 - ws.m0); p1 = ex2(x1 - ws.m1); p2 = ex2(x2 - ws.m0); p3 = ex2(x3 - ws.m1);
+  const float u0 = (GUARD && ws.m0 == NEG_INF) ? 0.f : ws.m0, u1 = (GUARD && ws.m1 == NEG_INF) ? 0.f : ws.m1;
+  p0 = ex2(x0 - u0); p1 = ex2(x1 - u1); p2 = ex2(x2 - u0); p3 = ex2(x3 - u1);
 }
 
 
@@ -131,11 +134,15 @@ __device__ __forceinline__ void pv_int4(uint32_t st, WarpState<D>& ws, int lane,
 }
 
 // One unit of NT INT4 tiles at shared addresses tile[0 .. NT-1]:
-// scores, one online-softmax update for the NT*16 tokens, P.V.  valid[u] bit 0 /
-// bit 1: token g / g+8 of tile u is inside the item's range (used when MASKED).
+// scores, one online-softmax update for the NT*16 tokens, P.V.  valid[u] bits
+// 0-3 (used when MASKED): token g of tile u is visible to the thread's column
+// 2t / 2t+1, token g+8 to column 2t / 2t+1 (inside the range being read, and
+// not after the column's query position).  Without CAUSAL the columns agree
+// (bits 0 and 2 decide) and every column sees a token of the unit; with it a
+// column may see none, and its state stays at m = -inf, l = 0.
 // The stages are handed back (empty barriers eb[0 .. NT-1], each distinct one
 // once) after the last shared-memory load.
-template <int D, int NT, bool MASKED>
+template <int D, int NT, bool MASKED, bool CAUSAL = false>
 __device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& qf, WarpState<D>& ws, int lane,
                                           const int* valid, const uint32_t* eb, const ColSplit& cs) {
   float x[NT][4];
@@ -182,9 +189,14 @@ __device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& 
     x[u][1] = fmaf(acc2[1], sKg, zKg * qf.qs1);
     x[u][2] = fmaf(acc2[2], sKg8, zKg8 * qf.qs0);
     x[u][3] = fmaf(acc2[3], sKg8, zKg8 * qf.qs1);
-    if constexpr (MASKED) {
+    if constexpr (MASKED && CAUSAL) {
+      if (!(valid[u] & 1)) x[u][0] = NEG_INF;
+      if (!(valid[u] & 2)) x[u][1] = NEG_INF;
+      if (!(valid[u] & 4)) x[u][2] = NEG_INF;
+      if (!(valid[u] & 8)) x[u][3] = NEG_INF;
+    } else if constexpr (MASKED) {
       if (!(valid[u] & 1)) { x[u][0] = NEG_INF; x[u][1] = NEG_INF; }
-      if (!(valid[u] & 2)) { x[u][2] = NEG_INF; x[u][3] = NEG_INF; }
+      if (!(valid[u] & 4)) { x[u][2] = NEG_INF; x[u][3] = NEG_INF; }
     }
   }
   // online softmax over the unit.  The running max only moves when some score
@@ -202,7 +214,9 @@ __device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& 
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
     }
     const float n0 = fmaxf(ws.m0, mx0), n1 = fmaxf(ws.m1, mx1);
-    const float a0 = ex2(ws.m0 - n0), a1 = ex2(ws.m1 - n1);
+    // causal: a column with no visible position so far keeps m = -inf and a zero state
+    const float a0 = (CAUSAL && n0 == NEG_INF) ? 1.f : ex2(ws.m0 - n0);
+    const float a1 = (CAUSAL && n1 == NEG_INF) ? 1.f : ex2(ws.m1 - n1);
     ws.l0 *= a0; ws.l1 *= a1; ws.z0 *= a0; ws.z1 *= a1;
 #pragma unroll
     for (int m = 0; m < D / 16; ++m) {
@@ -210,17 +224,24 @@ __device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& 
     }
     ws.m0 = n0; ws.m1 = n1;
   }
+  const float mu0 = (CAUSAL && ws.m0 == NEG_INF) ? 0.f : ws.m0;
+  const float mu1 = (CAUSAL && ws.m1 == NEG_INF) ? 0.f : ws.m1;
 #pragma unroll
   for (int u = 0; u < NT; ++u) {
-    const float p0 = ex2(x[u][0] - ws.m0), p1 = ex2(x[u][1] - ws.m1);
-    const float p2 = ex2(x[u][2] - ws.m0), p3 = ex2(x[u][3] - ws.m1);
+    const float p0 = ex2(x[u][0] - mu0), p1 = ex2(x[u][1] - mu1);
+    const float p2 = ex2(x[u][2] - mu0), p3 = ex2(x[u][3] - mu1);
     const float sVg = half_lo(sz[u].z), sVg8 = half_lo(sz[u].w);
     const float zVg = fmaf(8.f, sVg, half_hi(sz[u].z)), zVg8 = fmaf(8.f, sVg8, half_hi(sz[u].w));   // centred codes
     float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
     float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
-    if constexpr (MASKED) {   // unwritten slots may hold non-finite scales
+    if constexpr (MASKED && CAUSAL) {   // unwritten slots may hold non-finite scales
+      if (!(valid[u] & 1)) { P0 = 0.f; zg0 = 0.f; }
+      if (!(valid[u] & 2)) { P1 = 0.f; zg1 = 0.f; }
+      if (!(valid[u] & 4)) { P2 = 0.f; zg80 = 0.f; }
+      if (!(valid[u] & 8)) { P3 = 0.f; zg81 = 0.f; }
+    } else if constexpr (MASKED) {
       if (!(valid[u] & 1)) { P0 = 0.f; P1 = 0.f; zg0 = 0.f; zg1 = 0.f; }
-      if (!(valid[u] & 2)) { P2 = 0.f; P3 = 0.f; zg80 = 0.f; zg81 = 0.f; }
+      if (!(valid[u] & 4)) { P2 = 0.f; P3 = 0.f; zg80 = 0.f; zg81 = 0.f; }
     }
     ws.l0 += p0 + p2; ws.l1 += p1 + p3;
     ws.z0 += zg0 + zg80; ws.z1 += zg1 + zg81;
@@ -258,9 +279,9 @@ __device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& 
 }
 
 // One INT8 tile (protected store).
-template <int D, bool MASKED>
-__device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, bool vg,
-                                          bool vg8, uint32_t empty_bar, const ColSplit& cs) {
+template <int D, bool MASKED, bool CAUSAL = false>
+__device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, int vm,
+                                          uint32_t empty_bar, const ColSplit& cs) {
   constexpr int NK = D / 16;
   uint32_t kw[2][NK], vw[2 * NK];
   // K: per row (g, g+8) D/4 bytes at (D/4)*lane; word 2kk + hf holds dims 32kk + 16hf + 4t .. +3
@@ -292,19 +313,29 @@ __device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpS
   float x1 = fmaf(acc[1], sKg, zKg * qf.qs1);
   float x2 = fmaf(acc[2], sKg8, zKg8 * qf.qs0);
   float x3 = fmaf(acc[3], sKg8, zKg8 * qf.qs1);
-  if constexpr (MASKED) {
-    if (!vg) { x0 = NEG_INF; x1 = NEG_INF; }
-    if (!vg8) { x2 = NEG_INF; x3 = NEG_INF; }
+  if constexpr (MASKED && CAUSAL) {   // vm: the visibility bits of unit_int4's valid[]
+    if (!(vm & 1)) x0 = NEG_INF;
+    if (!(vm & 2)) x1 = NEG_INF;
+    if (!(vm & 4)) x2 = NEG_INF;
+    if (!(vm & 8)) x3 = NEG_INF;
+  } else if constexpr (MASKED) {
+    if (!(vm & 1)) { x0 = NEG_INF; x1 = NEG_INF; }
+    if (!(vm & 4)) { x2 = NEG_INF; x3 = NEG_INF; }
   }
   float p0, p1, p2, p3;
-  online_softmax_pv<D>(ws, x0, x1, x2, x3, p0, p1, p2, p3);
+  online_softmax_pv<D, CAUSAL>(ws, x0, x1, x2, x3, p0, p1, p2, p3);
   const float sVg = half_lo(sz.z), sVg8 = half_lo(sz.w);
   const float zVg = fmaf(128.f, sVg, half_hi(sz.z)), zVg8 = fmaf(128.f, sVg8, half_hi(sz.w));   // centred codes
   float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
   float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
-  if constexpr (MASKED) {
-    if (!vg) { P0 = 0.f; P1 = 0.f; zg0 = 0.f; zg1 = 0.f; }
-    if (!vg8) { P2 = 0.f; P3 = 0.f; zg80 = 0.f; zg81 = 0.f; }
+  if constexpr (MASKED && CAUSAL) {
+    if (!(vm & 1)) { P0 = 0.f; zg0 = 0.f; }
+    if (!(vm & 2)) { P1 = 0.f; zg1 = 0.f; }
+    if (!(vm & 4)) { P2 = 0.f; zg80 = 0.f; }
+    if (!(vm & 8)) { P3 = 0.f; zg81 = 0.f; }
+  } else if constexpr (MASKED) {
+    if (!(vm & 1)) { P0 = 0.f; P1 = 0.f; zg0 = 0.f; zg1 = 0.f; }
+    if (!(vm & 4)) { P2 = 0.f; P3 = 0.f; zg80 = 0.f; zg81 = 0.f; }
   }
   ws.l0 += p0 + p2; ws.l1 += p1 + p3;
   ws.z0 += zg0 + zg80; ws.z1 += zg1 + zg81;
@@ -383,7 +414,7 @@ __device__ __forceinline__ void build_qblob(const AttnParams& p, int b, int h, i
   float amax = 0.f;
   const float rot_c = p.rot_c;
   for (int g = 0; g < G; ++g) {
-    const uint16_t* src = p.q + (static_cast<long long>(b) * p.Hq + h * G + g) * D;
+    const uint16_t* src = p.q + q_row(p, b, h, g) * D;
     float x[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) x[i] = __bfloat162float(__ushort_as_bfloat16(src[VPL * lane + i]));
@@ -469,7 +500,7 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
   const bool colsplit = (G == 1 || G == 2 || G == 4);
   const int gsrc = colsplit ? g8 % G : g8;
   const bool active = gsrc < G;
-  const uint16_t* src = p.q + (static_cast<long long>(b) * p.Hq + h * G + (active ? gsrc : 0)) * D + 4 * t;
+  const uint16_t* src = p.q + q_row(p, b, h, active ? gsrc : 0) * D + 4 * t;
   float x[NKK][2][4];
 #pragma unroll
   for (int kk = 0; kk < NKK; ++kk)

@@ -83,7 +83,7 @@ struct AttnParams {
   const int32_t* block_table;
   const int32_t* seq_lens;    // this layer's row [max_seqs]
   const int32_t* seq_ids;
-  const uint16_t* q;          // bf16 [n_seqs][Hq][D]
+  const uint16_t* q;          // bf16 [n_seqs][qlen][Hq][D]
   void* out;
   State* state;
   Item* items[3];             // item regions
@@ -92,7 +92,8 @@ struct AttnParams {
   uint8_t* qblob;             // [n_seqs * Hkv][qblob_bytes]
   float* partials;            // [cap_parts][G][D + 4]: o[D], m, l, pad
   int cap_parts;
-  int n_seqs, Hq, Hkv, G, D, P, S, W, Bh;
+  int n_seqs, Hq, Hkv, G, D, P, S, W, Bh;   // G: operand columns per KV head (qlen * Gh)
+  int qlen, Gh;               // query tokens per sequence (the last qlen positions), query heads per KV head
   int max_seqs, num_pages, max_pages_per_seq;
   int chunk_tiles;
   int mode;
@@ -102,6 +103,14 @@ struct AttnParams {
   int ns;                     // shared-memory ring depth of the attention kernel
   int grid;                   // CTAs of the page-major attention kernel
 };
+
+// Row of q (and of the output) that operand column c of KV head h of batch
+// entry b stands for: query token c / Gh of the entry (the tokens are the
+// last qlen positions, oldest first), query head h * Gh + c % Gh.
+__device__ __forceinline__ long long q_row(const AttnParams& p, int b, int h, int c) {
+  const int i = c / p.Gh, g = c - i * p.Gh;
+  return (static_cast<long long>(b) * p.qlen + i) * p.Hq + h * p.Gh + g;
+}
 
 // ---------------------------------------------------------------------------
 // Self-checks (debug builds, -DKV4_DEBUG_CHECKS): every shared-memory access,
@@ -423,11 +432,13 @@ int launch_dequantize_debug(kv4_cache* c, int layer, int seq_id, int start, int 
 int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, const void* q, void* out,
                      float softmax_scale, int mode, void* ws, size_t ws_bytes, cudaStream_t stream);
 size_t attention_workspace_bytes(const kv4_cache* c, int n_seqs, int max_ctx);
+int launch_extend_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, int qlen, const void* q,
+                            void* out, float softmax_scale, int mode, void* ws, size_t ws_bytes, cudaStream_t stream);
 int attention_blocks_per_sm(kv4_cache* c);
 // page-major path (INT4 cache, KV heads a multiple of 4)
 bool grouped_path(const kv4_cache* c);
 int grouped_ring(kv4_cache* c);
-size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs);
+size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs, int qlen);
 int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 }  // namespace kv4

@@ -26,7 +26,8 @@ Modules:
 * ``layout``    -- byte placement of codes and scales inside a 16-token tile.
 * ``cache``     -- the paged cache: block table, INT4 pages, INT8 sink/ring
                   store, append and the effective (dequantized) view.
-* ``attention`` -- fp64 GQA decode attention over the effective view.
+* ``attention`` -- fp64 GQA decode attention over the effective view, and the
+                  causal attention of several query tokens per sequence.
 
 Parity unpinned: none of the functions here lacks a pin; the end-to-end
 accuracy effect of INT4 versus BF16 (a model-level claim of both pages) is out
@@ -38,4 +39,4 @@ from .hadamard import sylvester_hadamard, block_diag_hadamard, fwht_fp32, rotati
 from .quant import (quantize_groups, dequantize_groups, fp16_round_down, fp16_round_up,  # noqa: F401
                     bf16_round, clamp_fp16_range)
 from .cache import OracleKV4Cache, OracleBF16Cache, prot_slot, n_prot_tiles  # noqa: F401
-from .attention import attention_fp64, decode_attention, decode_attention_bf16  # noqa: F401
+from .attention import attention_fp64, decode_attention, decode_attention_bf16, extend_attention  # noqa: F401

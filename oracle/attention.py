@@ -87,6 +87,38 @@ def decode_attention(cache, layer, seq_ids, q, scale=None, protected=True):
     return {"out_f64": out, "out_bf16": _bf16_of_f64(out), "q_rot": q_rot}
 
 
+def extend_attention(cache, layer, seq_ids, q, scale=None, protected=True):
+    """Attention of several query tokens per sequence: the last T positions.
+
+    q: [n, T, Hq, D] bf16 values, token i (0 = oldest) of a sequence of length
+    L standing at position L - T + i.  Textbook causal attention: token i sees
+    positions 0 .. L - T + i.  Every token reads the same effective view, the
+    one of length L (sinks and the last W positions of L from INT8; that the
+    protected set follows the cache length, not the query position, is this
+    library's reading: the cache holds one view at a time).  A token with no
+    visible position (L - T + i < 0) gets an all-zero row.
+
+    Returns dict out_f64 / out_bf16 [n, T, Hq, D] and q_rot [n, T, Hq, D].
+    """
+    q = np.asarray(q, np.float32)
+    D = cache.D
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(D)
+    H = block_diag_hadamard(D, cache.Bh)
+    n, T = q.shape[0], q.shape[1]
+    out = np.zeros(q.shape, np.float64)
+    q_rot = rotate_query(q, cache.Bh)
+    for b, seq in enumerate(seq_ids):
+        kh, vh = cache.view(layer, int(seq), protected=protected)
+        L = kh.shape[0]
+        for i in range(T):
+            vis = L - T + i + 1           # positions 0 .. L - T + i
+            if vis <= 0:
+                continue
+            out[b, i] = attention_fp64(q_rot[b, i], kh[:vis], vh[:vis], scale) @ H.T
+    return {"out_f64": out, "out_bf16": _bf16_of_f64(out), "q_rot": q_rot}
+
+
 def decode_attention_bf16(cache, layer, seq_ids, q, scale=None):
     """Plain decode attention over an OracleBF16Cache (no rotation, no quantization)."""
     q = np.asarray(q, np.float32)

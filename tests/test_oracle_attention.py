@@ -4,8 +4,8 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import (attention_fp64, decode_attention, decode_attention_bf16, OracleKV4Cache, OracleBF16Cache,
-                    block_diag_hadamard, bf16_round)
+from oracle import (attention_fp64, decode_attention, decode_attention_bf16, extend_attention, OracleKV4Cache,
+                    OracleBF16Cache, block_diag_hadamard, bf16_round)
 
 
 def _sdpa(q, k, v, scale):
@@ -163,3 +163,95 @@ def test_empty_sequence_gives_zero_row():
     q = bf16_round(rng.standard_normal((2, 4, 64)).astype(np.float32))
     out = decode_attention(cache, 0, [0, 1], q)["out_f64"]
     assert np.all(out[0] == 0) and np.all(np.abs(out[1]) > 0)
+
+
+# ---- several query tokens per sequence (causal over the last T positions)
+
+def _sdpa_causal(q, k, v, scale):
+    """torch SDPA with an explicit boolean mask: query token i of T sees keys 0 .. L - T + i."""
+    T, Hq, D = q.shape
+    L, Hkv, _ = k.shape
+    G = Hq // Hkv
+    qt = torch.from_numpy(np.asarray(q, np.float64)).permute(1, 0, 2)          # [Hq, T, D]
+    kt = torch.from_numpy(np.asarray(k, np.float64)).permute(1, 0, 2).repeat_interleave(G, 0)
+    vt = torch.from_numpy(np.asarray(v, np.float64)).permute(1, 0, 2).repeat_interleave(G, 0)
+    mask = torch.arange(L)[None, :] <= (L - T + torch.arange(T))[:, None]     # [T, L]
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale).permute(
+        1, 0, 2).numpy()
+
+
+def test_extend_quantization_free_reduction_to_causal_sdpa():
+    # exact encodings (as in the decode reduction above): the multi-token result
+    # is torch's causally masked attention on the inputs, for the protected view
+    # (INT8 sinks and window, INT4 in between) and for the INT4-only view
+    cfg = _cfg(Bh=1, W=16, Hkv=2, Hq=4)
+    rng = np.random.default_rng(10)
+    L, T = 70, 3
+    codes = rng.integers(0, 16, (L, 2, 64))
+    codes[:, :, 0], codes[:, :, 1] = 0, 15
+    k = (codes * (17 / 64) - 2.0).astype(np.float32)
+    v = (np.roll(codes, 5, axis=2) * (17 / 128) + 1.0).astype(np.float32)
+    q = bf16_round(rng.standard_normal((1, T, 4, 64)).astype(np.float32))
+    cache = OracleKV4Cache(cfg, _table())
+    cache.append(0, [1], [0, L], k, v)
+    want = _sdpa_causal(q[0], k, v, 0.125)
+    for protected in (True, False):
+        got = extend_attention(cache, 0, [1], q, protected=protected)["out_f64"][0]
+        np.testing.assert_allclose(got, want, atol=1e-12)
+
+
+def test_extend_brute_force_loops():
+    # tiny, exact encodings, every score and weight written out by hand
+    cfg = _cfg(Bh=1, S=0, W=4, Hkv=1, Hq=2)
+    rng = np.random.default_rng(11)
+    L, T, D = 6, 3, 64
+    codes = rng.integers(0, 16, (L, 1, D))
+    codes[:, :, 0], codes[:, :, 1] = 0, 15
+    k = (codes * (17 / 64)).astype(np.float32)
+    v = (codes[:, :, ::-1] * (17 / 64) - 1.0).astype(np.float32)
+    q = bf16_round(rng.standard_normal((1, T, 2, D)).astype(np.float32))
+    cache = OracleKV4Cache(cfg, _table())
+    cache.append(0, [0], [0, L], k, v)
+    got = extend_attention(cache, 0, [0], q, scale=0.2)["out_f64"][0]
+    for i in range(T):
+        last = L - T + i
+        for j in range(2):
+            s = [0.2 * sum(float(q[0, i, j, d]) * float(k[p, 0, d]) for d in range(D)) for p in range(last + 1)]
+            m = max(s)
+            e = [np.exp(x - m) for x in s]
+            o = [sum(e[p] * float(v[p, 0, d]) for p in range(last + 1)) / sum(e) for d in range(D)]
+            np.testing.assert_allclose(got[i, j], o, rtol=1e-12, atol=1e-13)
+
+
+def test_extend_later_positions_do_not_reach_earlier_tokens():
+    # changing the newest position changes only the last query token's row
+    cfg = _cfg(D=128, Bh=128, W=32, Hkv=1, Hq=4)
+    rng = np.random.default_rng(12)
+    L, T = 90, 4
+    k = bf16_round(rng.standard_normal((L, 1, 128)).astype(np.float32))
+    v = bf16_round(rng.standard_normal((L, 1, 128)).astype(np.float32))
+    q = bf16_round(rng.standard_normal((1, T, 4, 128)).astype(np.float32))
+    outs = []
+    for bump in (0.0, 3.0):
+        v2 = v.copy()
+        v2[L - 1] += bump
+        cache = OracleKV4Cache(cfg, _table())
+        cache.append(0, [0], [0, L], k, v2)
+        outs.append(extend_attention(cache, 0, [0], q)["out_f64"][0])
+    assert np.array_equal(outs[0][:T - 1], outs[1][:T - 1])
+    assert np.all(np.abs(outs[0][T - 1] - outs[1][T - 1]).max(axis=-1) > 1e-3)
+
+
+def test_extend_one_token_is_decode_and_short_sequences_give_zero_rows():
+    cfg = _cfg(D=64, Bh=64, W=8)
+    rng = np.random.default_rng(13)
+    k = bf16_round(rng.standard_normal((40, 1, 64)).astype(np.float32))
+    cache = OracleKV4Cache(cfg, _table())
+    cache.append(0, [0, 1], [0, 38, 40], k, k * 0.5)                 # lengths 38 and 2
+    q1 = bf16_round(rng.standard_normal((2, 4, 64)).astype(np.float32))
+    np.testing.assert_array_equal(extend_attention(cache, 0, [0, 1], q1[:, None])["out_f64"][:, 0],
+                                  decode_attention(cache, 0, [0, 1], q1)["out_f64"])
+    q5 = bf16_round(rng.standard_normal((2, 5, 4, 64)).astype(np.float32))
+    out = extend_attention(cache, 0, [0, 1], q5)["out_f64"]
+    assert np.all(out[1, :3] == 0) and np.all(np.abs(out[1, 3:]).max(axis=-1) > 0)   # L = 2 < T = 5
+    assert np.all(np.abs(out[0]).max(axis=-1) > 0)

@@ -104,3 +104,42 @@ def test_wrong_ring_slot_fails_the_direct_construction_pin(monkeypatch):
     monkeypatch.undo()
     # reading the mutated store through the correct slot rule gives wrong values
     assert not np.array_equal(bad.view(0, 0)[0], good.view(0, 0)[0])
+
+
+def _extend_with_visibility(shift):
+    """The oracle's multi-token attention with the visible range moved by `shift` positions (a mistake)."""
+    def run(cache, layer, seq_ids, q, scale=None, protected=True):
+        q = np.asarray(q, np.float32)
+        scale = scale if scale else 1.0 / np.sqrt(cache.D)
+        H = oracle.block_diag_hadamard(cache.D, cache.Bh)
+        T = q.shape[1]
+        out = np.zeros(q.shape, np.float64)
+        q_rot = attn_mod.rotate_query(q, cache.Bh)
+        for b, seq in enumerate(seq_ids):
+            kh, vh = cache.view(layer, int(seq), protected=protected)
+            L = kh.shape[0]
+            for i in range(T):
+                vis = min(L, L - T + i + 1 + shift)
+                if vis > 0:
+                    out[b, i] = attn_mod.attention_fp64(q_rot[b, i], kh[:vis], vh[:vis], scale) @ H.T
+        return out
+    return run
+
+
+@pytest.mark.parametrize("shift", [-1, 1])
+def test_causal_off_by_one_fails_the_masked_sdpa_pin(shift):
+    from test_oracle_attention import _sdpa_causal
+    cfg = dict(num_layers=1, max_seqs=1, num_q_heads=4, num_kv_heads=2, head_dim=64, page_size=16,
+               num_pages=8, max_pages_per_seq=8, hadamard_block=1, sink_tokens=4, recent_window=16)
+    rng = np.random.default_rng(3)
+    L, T = 50, 3
+    codes = rng.integers(0, 16, (L, 2, 64))
+    codes[:, :, 0], codes[:, :, 1] = 0, 15
+    k = (codes * (17 / 64) - 2.0).astype(np.float32)
+    v = (np.roll(codes, 5, axis=2) * (17 / 128) + 1.0).astype(np.float32)
+    q = oracle.bf16_round(rng.standard_normal((1, T, 4, 64)).astype(np.float32))
+    c = cache_mod.OracleKV4Cache(cfg, np.arange(8, dtype=np.int32)[None])
+    c.append(0, [0], [0, L], k, v)
+    want = _sdpa_causal(q[0], k, v, 0.125)
+    np.testing.assert_allclose(_extend_with_visibility(0)(c, 0, [0], q)[0], want, atol=1e-12)
+    assert not np.allclose(_extend_with_visibility(shift)(c, 0, [0], q)[0], want, atol=1e-6)
