@@ -74,11 +74,20 @@ enum {
   KV4_DEV_WORKSPACE = 32      /* the attention plan did not fit the workspace              */
 };
 
-/* kv4_decode_attention mode bits. */
+/* kv4_decode_attention / kv4_extend_attention mode bits.
+ * KV4_MODE_Q_ROTATED and KV4_MODE_OUT_ROTATED let a caller fold the block
+ * Hadamard H (normalised, symmetric, its own inverse) into its projections:
+ * with W_q' = H W_q the query arrives rotated (q' = H q, bf16), and with
+ * o_proj' = o_proj H the attention output can stay in the rotated basis.  The
+ * kernels then skip that rotation (the query is used as given, no extra
+ * rounding).  The rotated cache is unchanged.  The BF16 baseline cache ignores
+ * both bits (it has no rotation). */
 enum {
   KV4_MODE_PROTECTED = 0,     /* INT8 for protected positions, INT4 elsewhere (the method) */
   KV4_MODE_INT4_ONLY = 1,     /* read the INT4 pages for every position (ablation)         */
-  KV4_MODE_OUT_F32 = 2        /* write fp32 output instead of bf16 (checking mode)          */
+  KV4_MODE_OUT_F32 = 2,       /* write fp32 output instead of bf16 (checking mode)          */
+  KV4_MODE_Q_ROTATED = 4,     /* q is already H q: do not rotate it                         */
+  KV4_MODE_OUT_ROTATED = 8    /* write the output in the rotated basis (H o): no inverse    */
 };
 
 /* kv4_dequantize_debug views. */

@@ -47,6 +47,8 @@ KV4_DEV_WORKSPACE = 32
 KV4_MODE_PROTECTED = 0
 KV4_MODE_INT4_ONLY = 1
 KV4_MODE_OUT_F32 = 2
+KV4_MODE_Q_ROTATED = 4
+KV4_MODE_OUT_ROTATED = 8
 
 KV4_VIEW_EFFECTIVE = 0
 KV4_VIEW_INT4 = 1

@@ -139,7 +139,8 @@ int attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_t n_seq
   if (n_seqs == 0) return KV4_OK;
   if (!seq_ids || !q || !out || !ws) return KV4_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || reinterpret_cast<uintptr_t>(ws) % kAlign) return KV4_ERR_INVALID_ARG;
-  if (mode & ~(KV4_MODE_INT4_ONLY | KV4_MODE_OUT_F32)) return KV4_ERR_INVALID_ARG;
+  if (mode & ~(KV4_MODE_INT4_ONLY | KV4_MODE_OUT_F32 | KV4_MODE_Q_ROTATED | KV4_MODE_OUT_ROTATED))
+    return KV4_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale)) return KV4_ERR_INVALID_ARG;
   if (!select_device(c)) return KV4_ERR_CUDA;
   return kv4::launch_attention(c, layer, seq_ids, n_seqs, q, out, softmax_scale, mode, ws, ws_bytes, stream);
@@ -155,7 +156,8 @@ int extend_attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_
   if (n_seqs == 0) return KV4_OK;
   if (!seq_ids || !q || !out || !ws) return KV4_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || reinterpret_cast<uintptr_t>(ws) % kAlign) return KV4_ERR_INVALID_ARG;
-  if (mode & ~(KV4_MODE_INT4_ONLY | KV4_MODE_OUT_F32)) return KV4_ERR_INVALID_ARG;
+  if (mode & ~(KV4_MODE_INT4_ONLY | KV4_MODE_OUT_F32 | KV4_MODE_Q_ROTATED | KV4_MODE_OUT_ROTATED))
+    return KV4_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale)) return KV4_ERR_INVALID_ARG;
   if (!select_device(c)) return KV4_ERR_CUDA;
   return kv4::launch_extend_attention(c, layer, seq_ids, n_seqs, q_len, q, out, softmax_scale, mode, ws, ws_bytes,

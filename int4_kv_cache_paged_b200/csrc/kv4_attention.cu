@@ -528,9 +528,9 @@ __global__ void __launch_bounds__(256) merge_kernel(AttnParams p) {
 #pragma unroll
     for (int i = 0; i < VPL; ++i) o[i] *= inv;
     if constexpr (!BF16) {
-      fwht_row<VPL>(o, p.Bh, lane);   // o = H_blk o_rot (the normalised Hadamard matrix is its own inverse)
+      fwht_row<VPL>(o, p.Bh_o, lane);   // o = H_blk o_rot (the normalised Hadamard matrix is its own inverse)
 #pragma unroll
-      for (int i = 0; i < VPL; ++i) o[i] *= p.rot_c;
+      for (int i = 0; i < VPL; ++i) o[i] *= p.rc_o;
     }
   }
   const size_t off = (static_cast<size_t>(b) * p.Hq + hq) * D + VPL * lane;
@@ -651,6 +651,16 @@ int attention_blocks_per_sm(kv4_cache* c) {
   return blocks;
 }
 
+// Rotations the kernels apply to q and to the output: the cache's block
+// Hadamard, unless the mode says the caller folded it into its projections.
+void set_rotations(AttnParams& p, int mode) {
+  const bool qr = (mode & KV4_MODE_Q_ROTATED) != 0, orot = (mode & KV4_MODE_OUT_ROTATED) != 0;
+  p.Bh_q = qr ? 1 : p.Bh;
+  p.rc_q = qr ? 1.f : p.rot_c;
+  p.Bh_o = orot ? 1 : p.Bh;
+  p.rc_o = orot ? 1.f : p.rot_c;
+}
+
 // Fields of AttnParams shared by both attention paths.
 void fill_common(const kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, const void* q, void* out,
                  float softmax_scale, int mode, AttnParams& p) {
@@ -676,6 +686,7 @@ void fill_common(const kv4_cache* c, int layer, const int32_t* seq_ids, int n_se
   p.W = cfg.recent_window;
   p.Bh = c->bf16 ? 1 : cfg.hadamard_block;
   p.rot_c = static_cast<float>(1.0 / sqrt(static_cast<double>(p.Bh)));
+  set_rotations(p, mode);
   p.max_seqs = cfg.max_seqs;
   p.num_pages = cfg.num_pages;
   p.max_pages_per_seq = cfg.max_pages_per_seq;
@@ -769,6 +780,7 @@ int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs
   p.W = cfg.recent_window;
   p.Bh = c->bf16 ? 1 : cfg.hadamard_block;
   p.rot_c = static_cast<float>(1.0 / sqrt(static_cast<double>(p.Bh)));
+  set_rotations(p, mode);
   p.max_seqs = cfg.max_seqs;
   p.num_pages = cfg.num_pages;
   p.max_pages_per_seq = cfg.max_pages_per_seq;

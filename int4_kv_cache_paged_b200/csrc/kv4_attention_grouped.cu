@@ -207,7 +207,7 @@ __device__ __forceinline__ void store_head(const AttnParams& p, int b, int hkv, 
   const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
 #pragma unroll
   for (int m = 0; m < NM; ++m) { o[m][0] *= inv0; o[m][2] *= inv0; o[m][1] *= inv1; o[m][3] *= inv1; }
-  const int Bh = p.Bh;
+  const int Bh = p.Bh_o;
   // stages 1, 2, 4: dimension bits 0-2 are the lane bits 2-4
 #pragma unroll
   for (int hh = 1; hh <= 4; hh <<= 1) {
@@ -248,7 +248,7 @@ __device__ __forceinline__ void store_head(const AttnParams& p, int b, int hkv, 
           }
     }
   }
-  const float rc = p.rot_c;
+  const float rc = p.rc_o;
   const int G = p.G;
 #pragma unroll
   for (int hp = 0; hp < 2; ++hp) {
@@ -754,8 +754,8 @@ __global__ void __launch_bounds__(32 * MWARPS) gmerge_kernel(AttnParams p, const
   const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) o[i] = acc[i] * inv;
-  fwht_row<VPL>(o, p.Bh, lane);   // o = H_blk o_rot (the normalised block Hadamard is its own inverse)
-  const float rc = p.rot_c;
+  fwht_row<VPL>(o, p.Bh_o, lane);   // o = H_blk o_rot (the normalised block Hadamard is its own inverse)
+  const float rc = p.rc_o;
   const long long off = q_row(p, b, hkv, gq) * D + VPL * lane;
   if (p.mode & KV4_MODE_OUT_F32) {
     float* out = static_cast<float*>(p.out) + off;

@@ -513,7 +513,7 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
       x[kk][hf][2] = __uint_as_float(w.y << 16);
       x[kk][hf][3] = __uint_as_float(w.y & 0xFFFF0000u);
     }
-  const int Bh = p.Bh;
+  const int Bh = p.Bh_q;
   // stages 1 and 2: dimension bits 0-1 (j)
 #pragma unroll
   for (int jb = 1; jb <= 2; jb <<= 1) {
@@ -575,7 +575,7 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
             }
     }
   }
-  const float rot_c = p.rot_c;
+  const float rot_c = p.rc_q;
   float amax = 0.f, qs = 0.f;
 #pragma unroll
   for (int kk = 0; kk < NKK; ++kk)

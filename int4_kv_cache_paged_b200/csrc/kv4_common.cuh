@@ -99,6 +99,8 @@ struct AttnParams {
   int mode;
   float scale_log2;           // softmax_scale * log2(e)
   float rot_c;                // fp32(1/sqrt(Bh))
+  int Bh_q, Bh_o;             // block of the rotation applied to q / to the output (1: none, the
+  float rc_q, rc_o;           // caller folded it into the projections), and its fp32(1/sqrt(block))
   size_t pool_bytes, prot_bytes, qblob_total;   // extents, for the self-checks of debug builds
   int ns;                     // shared-memory ring depth of the attention kernel
   int grid;                   // CTAs of the page-major attention kernel

@@ -18,6 +18,10 @@ Readings of this library:
 * GQA grouping is contiguous: query head j uses KV head j // (Hq / Hkv).
 * A sequence with no cached position gives an all-zero output row (the
   library's convention; softmax over an empty set is undefined).
+* Folded rotations (a library option for callers that fold H into W_q and
+  o_proj): with q_rotated the given bf16 query is q_rot itself; with
+  out_rotated the output is o_rot, not H o_rot.  The attention between them
+  is unchanged.
 * The bf16 output is rounded fp64 -> fp32 -> bf16 (two round-to-nearest-even
   steps); the tests allow one bf16 ulp between two bf16 outputs for this
   reason.
@@ -62,10 +66,22 @@ def rotate_query(q, Bh):
     return bf16_round(fwht_fp32(q, Bh))
 
 
-def decode_attention(cache, layer, seq_ids, q, scale=None, protected=True):
+def _query_and_output_rotation(cache, q, q_rotated, out_rotated):
+    """q_rot and the matrix that takes o_rot to the output basis.
+
+    q_rotated: the caller passes H q itself (H folded into its query
+    projection), used as given.  out_rotated: the output stays in the rotated
+    basis (H folded into the output projection), so the map is the identity."""
+    q_rot = np.asarray(q, np.float32) if q_rotated else rotate_query(q, cache.Bh)
+    back = np.eye(cache.D) if out_rotated else block_diag_hadamard(cache.D, cache.Bh).T
+    return q_rot, back
+
+
+def decode_attention(cache, layer, seq_ids, q, scale=None, protected=True, q_rotated=False, out_rotated=False):
     """Decode attention of one query token per sequence over an OracleKV4Cache.
 
-    q: [n, Hq, D] bf16 values.  Returns dict with
+    q: [n, Hq, D] bf16 values (already H q when q_rotated; the output stays
+    in the rotated basis when out_rotated).  Returns dict with
       out_f64  [n, Hq, D]  fp64 output in the original (unrotated) basis,
       out_bf16 [n, Hq, D]  the same rounded to bf16 (held in fp32),
       q_rot    [n, Hq, D]  the rotated bf16 queries.
@@ -74,20 +90,19 @@ def decode_attention(cache, layer, seq_ids, q, scale=None, protected=True):
     D = cache.D
     if scale is None or scale <= 0:
         scale = 1.0 / np.sqrt(D)
-    H = block_diag_hadamard(D, cache.Bh)
     n = len(seq_ids)
     out = np.zeros((n,) + q.shape[1:], np.float64)
-    q_rot = rotate_query(q, cache.Bh)
+    q_rot, back = _query_and_output_rotation(cache, q, q_rotated, out_rotated)
     for i, seq in enumerate(seq_ids):
         kh, vh = cache.view(layer, int(seq), protected=protected)
         if kh.shape[0] == 0:
             continue                      # an empty sequence has an all-zero output row
         o_rot = attention_fp64(q_rot[i], kh, vh, scale)
-        out[i] = o_rot @ H.T
+        out[i] = o_rot @ back
     return {"out_f64": out, "out_bf16": _bf16_of_f64(out), "q_rot": q_rot}
 
 
-def extend_attention(cache, layer, seq_ids, q, scale=None, protected=True):
+def extend_attention(cache, layer, seq_ids, q, scale=None, protected=True, q_rotated=False, out_rotated=False):
     """Attention of several query tokens per sequence: the last T positions.
 
     q: [n, T, Hq, D] bf16 values, token i (0 = oldest) of a sequence of length
@@ -96,7 +111,8 @@ def extend_attention(cache, layer, seq_ids, q, scale=None, protected=True):
     one of length L (sinks and the last W positions of L from INT8; that the
     protected set follows the cache length, not the query position, is this
     library's reading: the cache holds one view at a time).  A token with no
-    visible position (L - T + i < 0) gets an all-zero row.
+    visible position (L - T + i < 0) gets an all-zero row.  q_rotated and
+    out_rotated as in decode_attention.
 
     Returns dict out_f64 / out_bf16 [n, T, Hq, D] and q_rot [n, T, Hq, D].
     """
@@ -104,10 +120,9 @@ def extend_attention(cache, layer, seq_ids, q, scale=None, protected=True):
     D = cache.D
     if scale is None or scale <= 0:
         scale = 1.0 / np.sqrt(D)
-    H = block_diag_hadamard(D, cache.Bh)
     n, T = q.shape[0], q.shape[1]
     out = np.zeros(q.shape, np.float64)
-    q_rot = rotate_query(q, cache.Bh)
+    q_rot, back = _query_and_output_rotation(cache, q, q_rotated, out_rotated)
     for b, seq in enumerate(seq_ids):
         kh, vh = cache.view(layer, int(seq), protected=protected)
         L = kh.shape[0]
@@ -115,7 +130,7 @@ def extend_attention(cache, layer, seq_ids, q, scale=None, protected=True):
             vis = L - T + i + 1           # positions 0 .. L - T + i
             if vis <= 0:
                 continue
-            out[b, i] = attention_fp64(q_rot[b, i], kh[:vis], vh[:vis], scale) @ H.T
+            out[b, i] = attention_fp64(q_rot[b, i], kh[:vis], vh[:vis], scale) @ back
     return {"out_f64": out, "out_bf16": _bf16_of_f64(out), "q_rot": q_rot}
 
 

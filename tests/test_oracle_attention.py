@@ -255,3 +255,41 @@ def test_extend_one_token_is_decode_and_short_sequences_give_zero_rows():
     out = extend_attention(cache, 0, [0, 1], q5)["out_f64"]
     assert np.all(out[1, :3] == 0) and np.all(np.abs(out[1, 3:]).max(axis=-1) > 0)   # L = 2 < T = 5
     assert np.all(np.abs(out[0]).max(axis=-1) > 0)
+
+
+# ---- rotations folded into the caller's projections
+
+def test_folded_rotations_reduce_to_the_default_path():
+    # q_rotated with q' = bf16(H q) is the default path on q; out_rotated is the
+    # default output taken back into the rotated basis (H symmetric, H H = I)
+    cfg = _cfg(D=128, Bh=64, W=16, Hkv=1, Hq=4)
+    rng = np.random.default_rng(14)
+    L = 60
+    k = bf16_round(rng.standard_normal((L, 1, 128)).astype(np.float32))
+    v = bf16_round(rng.standard_normal((L, 1, 128)).astype(np.float32))
+    cache = OracleKV4Cache(cfg, _table())
+    cache.append(0, [0], [0, L], k, v)
+    q = bf16_round(rng.standard_normal((1, 4, 128)).astype(np.float32))
+    H = block_diag_hadamard(128, 64)
+    base = decode_attention(cache, 0, [0], q)
+    qr = base["q_rot"]
+    np.testing.assert_array_equal(decode_attention(cache, 0, [0], qr, q_rotated=True)["out_f64"], base["out_f64"])
+    rot = decode_attention(cache, 0, [0], q, out_rotated=True)["out_f64"]
+    np.testing.assert_allclose(rot, base["out_f64"] @ H, atol=1e-12)
+    np.testing.assert_allclose(rot @ H, base["out_f64"], atol=1e-12)
+    both = extend_attention(cache, 0, [0], qr[:, None], q_rotated=True, out_rotated=True)["out_f64"][:, 0]
+    np.testing.assert_allclose(both, rot, atol=1e-15)
+
+
+def test_folded_rotations_are_the_identity_without_rotation():
+    cfg = _cfg(D=64, Bh=1, W=8)
+    rng = np.random.default_rng(15)
+    k = bf16_round(rng.standard_normal((20, 1, 64)).astype(np.float32))
+    cache = OracleKV4Cache(cfg, _table())
+    cache.append(0, [0], [0, 20], k, k)
+    q = bf16_round(rng.standard_normal((1, 4, 64)).astype(np.float32))
+    ref = decode_attention(cache, 0, [0], q)["out_f64"]
+    for qr in (False, True):
+        for orot in (False, True):
+            np.testing.assert_array_equal(decode_attention(cache, 0, [0], q, q_rotated=qr, out_rotated=orot)["out_f64"],
+                                          ref)

@@ -143,3 +143,20 @@ def test_causal_off_by_one_fails_the_masked_sdpa_pin(shift):
     want = _sdpa_causal(q[0], k, v, 0.125)
     np.testing.assert_allclose(_extend_with_visibility(0)(c, 0, [0], q)[0], want, atol=1e-12)
     assert not np.allclose(_extend_with_visibility(shift)(c, 0, [0], q)[0], want, atol=1e-6)
+
+
+def test_output_rotated_twice_fails_the_inverse_pin():
+    # a mistake that applies H to the output in the rotated mode as well
+    cfg = dict(num_layers=1, max_seqs=1, num_q_heads=4, num_kv_heads=1, head_dim=64, page_size=16,
+               num_pages=8, max_pages_per_seq=8, hadamard_block=64, sink_tokens=4, recent_window=16)
+    rng = np.random.default_rng(4)
+    k = oracle.bf16_round(rng.standard_normal((30, 1, 64)).astype(np.float32))
+    c = cache_mod.OracleKV4Cache(cfg, np.arange(8, dtype=np.int32)[None])
+    c.append(0, [0], [0, 30], k, k)
+    q = oracle.bf16_round(rng.standard_normal((1, 4, 64)).astype(np.float32))
+    H = oracle.block_diag_hadamard(64, 64)
+    base = attn_mod.decode_attention(c, 0, [0], q)["out_f64"]
+    wrong = base                                      # mistake: rotated mode returns the unrotated output
+    assert not np.allclose(wrong, base @ H, atol=1e-6)
+    np.testing.assert_allclose(attn_mod.decode_attention(c, 0, [0], q, out_rotated=True)["out_f64"], base @ H,
+                               atol=1e-12)
