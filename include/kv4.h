@@ -71,7 +71,15 @@ enum {
   KV4_DEV_RANGE = 4,          /* a rotated value was non-finite or beyond +-65504: clamped  */
   KV4_DEV_TIMEOUT = 8,        /* a bounded wait inside a kernel gave up (~1 s)              */
   KV4_DEV_BAD_SEQ = 16,       /* a sequence id outside [0, max_seqs): entry skipped        */
-  KV4_DEV_WORKSPACE = 32      /* the attention plan did not fit the workspace              */
+  KV4_DEV_WORKSPACE = 32,     /* the attention plan did not fit the workspace              */
+  KV4_DEV_ROPE_POS = 64       /* a position at or past the RoPE table: key not written,
+                                 query rotated with the table's last row                    */
+};
+
+/* RoPE pair layouts (kv4_set_rope). */
+enum {
+  KV4_ROPE_NEOX = 0,          /* pairs (i, i + R/2): "rotate half"                          */
+  KV4_ROPE_GPTJ = 1           /* pairs (2i, 2i + 1): interleaved                            */
 };
 
 /* kv4_decode_attention / kv4_extend_attention mode bits.
@@ -87,7 +95,8 @@ enum {
   KV4_MODE_INT4_ONLY = 1,     /* read the INT4 pages for every position (ablation)         */
   KV4_MODE_OUT_F32 = 2,       /* write fp32 output instead of bf16 (checking mode)          */
   KV4_MODE_Q_ROTATED = 4,     /* q is already H q: do not rotate it                         */
-  KV4_MODE_OUT_ROTATED = 8    /* write the output in the rotated basis (H o): no inverse    */
+  KV4_MODE_OUT_ROTATED = 8,   /* write the output in the rotated basis (H o): no inverse    */
+  KV4_MODE_ROPE_Q = 16        /* apply the cache's RoPE table to q at its position first    */
 };
 
 /* kv4_dequantize_debug views. */
@@ -162,6 +171,33 @@ int kv4_seq_reset(kv4_cache* cache, int32_t seq_id, kv4_stream_t stream);
  * The sequence length of this layer advances by the number of new rows.
  * At most 3413 sequences per call (KV4_ERR_UNSUPPORTED above).
  */
+/*
+ * RoPE fused into the append and the query kernel (the step before the
+ * rotation: keys are rotated by position after RoPE, cf. the key transform
+ * applied after RoPE on the method's pages).  kv4_set_rope registers a table
+ * that stays owned by the caller and must outlive its use:
+ *   dev_cos_sin  fp32 [max_pos][R]: row p holds cos(theta_{p,i}) for
+ *                i = 0 .. R/2-1, then sin(theta_{p,i}) (any angles the model
+ *                uses, e.g. theta_{p,i} = p * base^(-2i/R))
+ *   rotary_dim   R: a power of two, 32 <= R <= D; dimensions >= R pass through
+ *   style        KV4_ROPE_NEOX or KV4_ROPE_GPTJ
+ * dev_cos_sin = NULL removes the table.  Pair (a, b) with angle i becomes
+ * (a*c - b*s, b*c + a*s), each product and sum rounded to fp32 (no fused
+ * multiply-add), on the fp32 value of the bf16 input; the result goes to the
+ * Hadamard rotation in fp32 (no bf16 rounding in between).
+ * kv4_rope_rotate_quantize_append is kv4_rotate_quantize_append with RoPE
+ * applied to each new key at its position in the sequence (values are not
+ * rotated); a key at position >= max_pos is not written and sets
+ * KV4_DEV_ROPE_POS.  KV4_MODE_ROPE_Q applies RoPE to each query at its
+ * position (decode: L - 1; kv4_extend_attention: L - q_len + i); it cannot
+ * be combined with KV4_MODE_Q_ROTATED.  Without a table both return
+ * KV4_ERR_INVALID_ARG.
+ */
+int kv4_set_rope(kv4_cache* cache, const float* dev_cos_sin, int32_t max_pos, int32_t rotary_dim, int32_t style);
+int kv4_rope_rotate_quantize_append(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids,
+                                    const int32_t* dev_cu_new, int32_t n_seqs, int32_t total_new,
+                                    const void* k_new, const void* v_new, kv4_stream_t stream);
+
 int kv4_rotate_quantize_append(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids,
                                const int32_t* dev_cu_new, int32_t n_seqs, int32_t total_new,
                                const void* k_new, const void* v_new, kv4_stream_t stream);

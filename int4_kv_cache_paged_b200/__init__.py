@@ -43,12 +43,16 @@ KV4_DEV_RANGE = 4
 KV4_DEV_TIMEOUT = 8
 KV4_DEV_BAD_SEQ = 16
 KV4_DEV_WORKSPACE = 32
+KV4_DEV_ROPE_POS = 64
 
 KV4_MODE_PROTECTED = 0
 KV4_MODE_INT4_ONLY = 1
 KV4_MODE_OUT_F32 = 2
 KV4_MODE_Q_ROTATED = 4
 KV4_MODE_OUT_ROTATED = 8
+KV4_MODE_ROPE_Q = 16
+KV4_ROPE_NEOX = 0
+KV4_ROPE_GPTJ = 1
 
 KV4_VIEW_EFFECTIVE = 0
 KV4_VIEW_INT4 = 1
@@ -57,6 +61,7 @@ EXPORTS = [
     "kv4_cache_required_bytes", "kv4_cache_create", "kv4_cache_destroy", "kv4_cache_layout", "kv4_seq_reset",
     "kv4_rotate_quantize_append", "kv4_attention_workspace_bytes", "kv4_decode_attention",
     "kv4_decode_attention_noalloc", "kv4_extend_workspace_bytes", "kv4_extend_attention",
+    "kv4_set_rope", "kv4_rope_rotate_quantize_append",
     "kv4_dequantize_debug", "kv4_get_status", "kv4_set_attention_events", "kv4_status_string", "kv4_version",
     "kv4bf16_cache_required_bytes", "kv4bf16_cache_create", "kv4bf16_cache_destroy", "kv4bf16_cache_layout",
     "kv4bf16_append", "kv4bf16_attention_workspace_bytes", "kv4bf16_decode_attention", "kv4bf16_get_status",
@@ -86,6 +91,8 @@ _sigs = {
     "kv4_decode_attention": (_I, [_P, _I, _P, _I, _P, _P, ctypes.c_float, _I, _P, _SZ, _P]),
     "kv4_decode_attention_noalloc": (_I, [_P, _I, _P, _I, _P, _P, ctypes.c_float, _I, _P]),
     "kv4_extend_workspace_bytes": (_I, [_P, _I, _I, ctypes.POINTER(_SZ)]),
+    "kv4_set_rope": (_I, [_P, _P, _I, _I, _I]),
+    "kv4_rope_rotate_quantize_append": (_I, [_P, _I, _P, _P, _I, _I, _P, _P, _P]),
     "kv4_extend_attention": (_I, [_P, _I, _P, _I, _I, _P, _P, ctypes.c_float, _I, _P, _SZ, _P]),
     "kv4_dequantize_debug": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "kv4_get_status": (_I, [_P, _P, ctypes.POINTER(_I)]),
@@ -190,6 +197,17 @@ def kv4_decode_attention_noalloc(handle, layer, seq_ids, n_seqs, q, out, softmax
     _check(_lib.kv4_decode_attention_noalloc(handle, layer, _ptr(seq_ids), n_seqs, _ptr(q), _ptr(out),
                                              float(softmax_scale), mode, _stream(stream)),
            "kv4_decode_attention_noalloc")
+
+
+def kv4_set_rope(handle, cos_sin, max_pos, rotary_dim, style):
+    _check(_lib.kv4_set_rope(handle, _ptr(cos_sin) if cos_sin is not None else None, max_pos, rotary_dim, style),
+           "kv4_set_rope")
+
+
+def kv4_rope_rotate_quantize_append(handle, layer, seq_ids, cu_new, n_seqs, total_new, k_new, v_new, stream=None):
+    _check(_lib.kv4_rope_rotate_quantize_append(handle, layer, _ptr(seq_ids), _ptr(cu_new), n_seqs, total_new,
+                                                _ptr(k_new), _ptr(v_new), _stream(stream)),
+           "kv4_rope_rotate_quantize_append")
 
 
 def kv4_extend_workspace_bytes(handle, n_seqs, q_len):

@@ -5,6 +5,7 @@ import torch
 from . import (make_config, kv4_cache_required_bytes, kv4_cache_create, kv4_cache_destroy, kv4_cache_layout,
                kv4_seq_reset, kv4_rotate_quantize_append, kv4_attention_workspace_bytes, kv4_decode_attention,
                kv4_decode_attention_noalloc, kv4_extend_workspace_bytes, kv4_extend_attention,
+               kv4_set_rope, kv4_rope_rotate_quantize_append,
                kv4_dequantize_debug, kv4_get_status, kv4bf16_cache_required_bytes, kv4bf16_cache_create,
                kv4bf16_cache_destroy, kv4bf16_cache_layout, kv4bf16_append, kv4bf16_attention_workspace_bytes,
                kv4bf16_decode_attention, kv4bf16_get_status, KV4_VIEW_EFFECTIVE, KV4_MODE_OUT_F32)
@@ -85,11 +86,23 @@ class KV4Cache(_Base):
         n = shape[0] * shape[1] * shape[2] * shape[3]
         return self._view(ptr, n, shape)
 
-    def append(self, layer, seq_ids, cu_new, k_new, v_new, total_new=None, stream=None):
+    def append(self, layer, seq_ids, cu_new, k_new, v_new, total_new=None, stream=None, rope=False):
+        """rope=True: each new key first gets RoPE at its position from the table of set_rope()."""
         if total_new is None:
             total_new = int(k_new.shape[0])
-        kv4_rotate_quantize_append(self.handle, layer, seq_ids, cu_new, int(seq_ids.numel()), total_new,
-                                   k_new, v_new, stream)
+        fn = kv4_rope_rotate_quantize_append if rope else kv4_rotate_quantize_append
+        fn(self.handle, layer, seq_ids, cu_new, int(seq_ids.numel()), total_new, k_new, v_new, stream)
+
+    def set_rope(self, cos_sin, rotary_dim, style):
+        """Register a RoPE table: fp32 [max_pos, R] on the cache's device (cos of the R/2 angles, then
+        their sin); None removes it.  The cache keeps a reference to the tensor."""
+        if cos_sin is None:
+            kv4_set_rope(self.handle, None, 0, 0, 0)
+            self._rope = None
+            return
+        cos_sin = cos_sin.to(device=self.device, dtype=torch.float32).contiguous()
+        kv4_set_rope(self.handle, cos_sin, int(cos_sin.shape[0]), rotary_dim, style)
+        self._rope = cos_sin
 
     def attention(self, layer, seq_ids, q, out=None, scale=0.0, mode=0, workspace=None, stream=None):
         n = int(seq_ids.numel())

@@ -121,15 +121,24 @@ int check_layer(const kv4_cache* c, int32_t layer) {
 
 bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
 
+// Attention mode bits this cache accepts: RoPE of q needs a registered table
+// and contradicts an already rotated query.
+bool mode_ok(const kv4_cache* c, int32_t mode) {
+  if (mode & ~(KV4_MODE_INT4_ONLY | KV4_MODE_OUT_F32 | KV4_MODE_Q_ROTATED | KV4_MODE_OUT_ROTATED | KV4_MODE_ROPE_Q))
+    return false;
+  if ((mode & KV4_MODE_ROPE_Q) && (c->rope.cs == nullptr || (mode & KV4_MODE_Q_ROTATED))) return false;
+  return true;
+}
+
 int append(kv4_cache* c, int32_t layer, const int32_t* seq_ids, const int32_t* cu_new, int32_t n_seqs,
-           int32_t total_new, const void* k_new, const void* v_new, cudaStream_t stream) {
+           int32_t total_new, const void* k_new, const void* v_new, cudaStream_t stream, bool rope = false) {
   if (!c || check_layer(c, layer)) return KV4_ERR_INVALID_ARG;
   if (n_seqs < 0 || total_new < 0) return KV4_ERR_INVALID_ARG;
   if (n_seqs == 0 || total_new == 0) return KV4_OK;
   if (!seq_ids || !cu_new || !k_new || !v_new) return KV4_ERR_INVALID_ARG;
   if (!aligned16(k_new) || !aligned16(v_new)) return KV4_ERR_INVALID_ARG;
   if (!select_device(c)) return KV4_ERR_CUDA;
-  return kv4::launch_append(c, layer, seq_ids, cu_new, n_seqs, total_new, k_new, v_new, stream);
+  return kv4::launch_append(c, layer, seq_ids, cu_new, n_seqs, total_new, k_new, v_new, rope, stream);
 }
 
 int attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_t n_seqs, const void* q, void* out,
@@ -139,8 +148,7 @@ int attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_t n_seq
   if (n_seqs == 0) return KV4_OK;
   if (!seq_ids || !q || !out || !ws) return KV4_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || reinterpret_cast<uintptr_t>(ws) % kAlign) return KV4_ERR_INVALID_ARG;
-  if (mode & ~(KV4_MODE_INT4_ONLY | KV4_MODE_OUT_F32 | KV4_MODE_Q_ROTATED | KV4_MODE_OUT_ROTATED))
-    return KV4_ERR_INVALID_ARG;
+  if (!mode_ok(c, mode)) return KV4_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale)) return KV4_ERR_INVALID_ARG;
   if (!select_device(c)) return KV4_ERR_CUDA;
   return kv4::launch_attention(c, layer, seq_ids, n_seqs, q, out, softmax_scale, mode, ws, ws_bytes, stream);
@@ -156,8 +164,7 @@ int extend_attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_
   if (n_seqs == 0) return KV4_OK;
   if (!seq_ids || !q || !out || !ws) return KV4_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || reinterpret_cast<uintptr_t>(ws) % kAlign) return KV4_ERR_INVALID_ARG;
-  if (mode & ~(KV4_MODE_INT4_ONLY | KV4_MODE_OUT_F32 | KV4_MODE_Q_ROTATED | KV4_MODE_OUT_ROTATED))
-    return KV4_ERR_INVALID_ARG;
+  if (!mode_ok(c, mode)) return KV4_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale)) return KV4_ERR_INVALID_ARG;
   if (!select_device(c)) return KV4_ERR_CUDA;
   return kv4::launch_extend_attention(c, layer, seq_ids, n_seqs, q_len, q, out, softmax_scale, mode, ws, ws_bytes,
@@ -221,6 +228,28 @@ int kv4_rotate_quantize_append(kv4_cache* c, int32_t layer, const int32_t* seq_i
                                kv4_stream_t stream) {
   if (!c || c->bf16) return KV4_ERR_INVALID_ARG;
   return append(c, layer, seq_ids, cu_new, n_seqs, total_new, k_new, v_new, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int kv4_set_rope(kv4_cache* c, const float* cos_sin, int32_t max_pos, int32_t rotary_dim, int32_t style) {
+  if (!c || c->bf16) return KV4_ERR_INVALID_ARG;
+  if (cos_sin == nullptr) {
+    c->rope = kv4::RopeParams{nullptr, 0, 0, 0};
+    return KV4_OK;
+  }
+  const int R = rotary_dim;
+  if (max_pos < 1 || R < 32 || R > c->cfg.head_dim || (R & (R - 1)) != 0) return KV4_ERR_INVALID_ARG;
+  if (style != KV4_ROPE_NEOX && style != KV4_ROPE_GPTJ) return KV4_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(cos_sin) % alignof(float)) return KV4_ERR_INVALID_ARG;
+  c->rope = kv4::RopeParams{cos_sin, max_pos, R, style};
+  return KV4_OK;
+}
+
+int kv4_rope_rotate_quantize_append(kv4_cache* c, int32_t layer, const int32_t* seq_ids, const int32_t* cu_new,
+                                    int32_t n_seqs, int32_t total_new, const void* k_new, const void* v_new,
+                                    kv4_stream_t stream) {
+  if (!c || c->bf16 || c->rope.cs == nullptr) return KV4_ERR_INVALID_ARG;
+  return append(c, layer, seq_ids, cu_new, n_seqs, total_new, k_new, v_new, reinterpret_cast<cudaStream_t>(stream),
+                true);
 }
 
 int kv4_attention_workspace_bytes(const kv4_cache* c, int32_t n_seqs, int32_t max_ctx, size_t* bytes) {

@@ -37,7 +37,44 @@ struct AppendParams {
   int n_seqs, total_new, Hkv, D, P, S, W, Bh;
   int max_seqs, num_pages, max_pages_per_seq;
   float rot_c;               // fp32(1/sqrt(Bh))
+  RopeParams rope;           // RoPE of the keys at their positions (cs == nullptr: none)
 };
+
+// RoPE of one row held VPL consecutive dims per lane (dims VPL*lane ..), at
+// table row `pos`: pair (a, b) -> (a*c - b*s, b*c + a*s), every product and
+// sum rounded to fp32.  Neox pairs (d, d + R/2) sit R/(2*VPL) lanes apart (R
+// a power of two), gptj pairs (d, d + 1) in one lane.  All lanes call it.
+template <int VPL>
+__device__ __forceinline__ void rope_row(float (&x)[VPL], const RopeParams& r, int pos, int lane) {
+  const float* cs = r.cs + static_cast<long long>(pos) * r.R;
+  const int half = r.R >> 1, d0 = VPL * lane;
+  if (r.style == KV4_ROPE_GPTJ) {
+    if (d0 < r.R) {
+#pragma unroll
+      for (int k = 0; k < VPL; k += 2) {
+        const int i = (d0 + k) >> 1;
+        const float c = __ldg(cs + i), s = __ldg(cs + half + i);
+        const float a = x[k], b = x[k + 1];
+        x[k] = __fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s));
+        x[k + 1] = __fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s));
+      }
+    }
+  } else {
+    float y[VPL];
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) y[k] = __shfl_xor_sync(0xffffffffu, x[k], half / VPL);
+    if (d0 < r.R) {
+      const bool first = d0 < half;   // holds a; the partner lane holds b
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) {
+        const int i = first ? d0 + k : d0 + k - half;
+        const float c = __ldg(cs + i), s = __ldg(cs + half + i);
+        x[k] = first ? __fsub_rn(__fmul_rn(x[k], c), __fmul_rn(y[k], s))
+                     : __fadd_rn(__fmul_rn(x[k], c), __fmul_rn(y[k], s));
+      }
+    }
+  }
+}
 
 template <int VPL>
 __device__ __forceinline__ void fwht_warp(float (&x)[VPL], int Bh, float c, int lane) {
@@ -216,6 +253,10 @@ __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams 
         ok = false;
       }
     }
+    if (ok && tensor == 0 && p.rope.cs != nullptr && pos >= p.rope.max_pos) {
+      if (lane == 0) atomicOr(&p.state->status, KV4_DEV_ROPE_POS);
+      ok = false;
+    }
     int page = -1;
     if (ok) {
       page = p.block_table[static_cast<long long>(seq) * p.max_pages_per_seq + pos / p.P];
@@ -259,6 +300,7 @@ __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams 
           bad |= !(fabsf(v) <= 3.0e38f);
           x[k] = v;
         }
+        if (tensor == 0 && p.rope.cs != nullptr) rope_row<VPL>(x, p.rope, pos, lane);   // the key at its position
         fwht_warp<VPL>(x, p.Bh, p.rot_c, lane);
 #pragma unroll
         for (int k = 0; k < VPL; ++k) {
@@ -373,9 +415,10 @@ __global__ void seq_reset_kernel(int32_t* seq_lens, int num_layers, int max_seqs
 }  // namespace
 
 int launch_append(kv4_cache* c, int layer, const int32_t* seq_ids, const int32_t* cu_new, int n_seqs, int total_new,
-                  const void* k_new, const void* v_new, cudaStream_t stream) {
+                  const void* k_new, const void* v_new, bool rope, cudaStream_t stream) {
   const kv4_config& cfg = c->cfg;
   AppendParams p{};
+  if (rope) p.rope = c->rope;
   uint8_t* lbase = c->base + c->pool_offset + static_cast<size_t>(layer) * c->layer_stride;
   p.pool = lbase;
   p.prot = c->bf16 ? nullptr : lbase + c->pool_bytes;

@@ -687,6 +687,7 @@ void fill_common(const kv4_cache* c, int layer, const int32_t* seq_ids, int n_se
   p.Bh = c->bf16 ? 1 : cfg.hadamard_block;
   p.rot_c = static_cast<float>(1.0 / sqrt(static_cast<double>(p.Bh)));
   set_rotations(p, mode);
+  if (mode & KV4_MODE_ROPE_Q) p.rope = c->rope;
   p.max_seqs = cfg.max_seqs;
   p.num_pages = cfg.num_pages;
   p.max_pages_per_seq = cfg.max_pages_per_seq;
@@ -781,6 +782,7 @@ int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs
   p.Bh = c->bf16 ? 1 : cfg.hadamard_block;
   p.rot_c = static_cast<float>(1.0 / sqrt(static_cast<double>(p.Bh)));
   set_rotations(p, mode);
+  if (mode & KV4_MODE_ROPE_Q) p.rope = c->rope;
   p.max_seqs = cfg.max_seqs;
   p.num_pages = cfg.num_pages;
   p.max_pages_per_seq = cfg.max_pages_per_seq;

@@ -493,6 +493,53 @@ __device__ __forceinline__ void build_qblob(const AttnParams& p, int b, int h, i
 // vector whichever lane holds it.  Then q_rot * 2^e (max |q_rot| * 2^e in
 // [2^14, 2^15)) is rounded to a 16-bit integer and split into the planes
 // hi = floor(q / 256) (signed byte) and lo = q mod 256 (unsigned byte).
+// RoPE of a query held in the fragment layout (x[kk][hf][j] = dim 32kk + 16hf
+// + 4t + j), at table row `pos`, with the arithmetic of the keys' RoPE: neox
+// pairs (d, d + R/2) are 16-dim blocks SH = R/32 apart, gptj pairs (d, d + 1)
+// are neighbours in j; both always sit in the same lane.
+__device__ __forceinline__ void rope_turn(float& a, float& b, float c, float s) {
+  const float a0 = a, b0 = b;
+  a = __fsub_rn(__fmul_rn(a0, c), __fmul_rn(b0, s));
+  b = __fadd_rn(__fmul_rn(b0, c), __fmul_rn(a0, s));
+}
+
+template <int NKK, int SH>
+__device__ __forceinline__ void rope_qfrag_neox(float (&x)[NKK][2][4], const float* cs, int t) {
+  constexpr int HALF = 16 * SH;
+#pragma unroll
+  for (int b1 = 0; b1 < SH; ++b1)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = 16 * b1 + 4 * t + j;
+      rope_turn(x[b1 >> 1][b1 & 1][j], x[(b1 + SH) >> 1][(b1 + SH) & 1][j], __ldg(cs + i), __ldg(cs + HALF + i));
+    }
+}
+
+template <int NKK>
+__device__ __forceinline__ void rope_qfrag(float (&x)[NKK][2][4], const RopeParams& r, int pos, int t) {
+  const float* cs = r.cs + static_cast<long long>(pos) * r.R;
+  if (r.style == KV4_ROPE_GPTJ) {
+    const int half = r.R >> 1;
+#pragma unroll
+    for (int kk = 0; kk < NKK; ++kk)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int d = 32 * kk + 16 * hf + 4 * t;
+        if (d < r.R) {
+          const int i = d >> 1;
+          rope_turn(x[kk][hf][0], x[kk][hf][1], __ldg(cs + i), __ldg(cs + half + i));
+          rope_turn(x[kk][hf][2], x[kk][hf][3], __ldg(cs + i + 1), __ldg(cs + half + i + 1));
+        }
+      }
+  } else if (r.R == 32) {
+    rope_qfrag_neox<NKK, 1>(x, cs, t);
+  } else if (r.R == 64) {
+    rope_qfrag_neox<NKK, 2>(x, cs, t);
+  } else if constexpr (NKK >= 4) {
+    rope_qfrag_neox<NKK, 4>(x, cs, t);   // R = 128
+  }
+}
+
 template <int D>
 __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, int lane, QFrag<D>& qf) {
   constexpr int NKK = D / 32;
@@ -513,6 +560,17 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
       x[kk][hf][2] = __uint_as_float(w.y << 16);
       x[kk][hf][3] = __uint_as_float(w.y & 0xFFFF0000u);
     }
+  if (p.rope.cs != nullptr && active) {
+    // the column's query token sits at position L - qlen + i of its sequence
+    const int seq = p.seq_ids[b];
+    const int L = (seq >= 0 && seq < p.max_seqs) ? p.seq_lens[seq] : 0;
+    int pos = max(L - p.qlen + gsrc / p.Gh, 0);
+    if (pos >= p.rope.max_pos) {
+      atomicOr(&p.state->status, KV4_DEV_ROPE_POS);
+      pos = p.rope.max_pos - 1;
+    }
+    rope_qfrag<NKK>(x, p.rope, pos, t);
+  }
   const int Bh = p.Bh_q;
   // stages 1 and 2: dimension bits 0-1 (j)
 #pragma unroll

@@ -77,6 +77,13 @@ struct SeqHead {
 };
 
 // Parameters shared by the attention kernels.
+// A caller's RoPE table: fp32 [max_pos][R], cos of the R/2 angles then their
+// sin; style KV4_ROPE_NEOX or KV4_ROPE_GPTJ.
+struct RopeParams {
+  const float* cs;
+  int max_pos, R, style;
+};
+
 struct AttnParams {
   const uint8_t* pool;        // INT4 (or BF16) page pool of the layer
   const uint8_t* prot;        // INT8 store of the layer (INT4 mode)
@@ -99,6 +106,7 @@ struct AttnParams {
   int mode;
   float scale_log2;           // softmax_scale * log2(e)
   float rot_c;                // fp32(1/sqrt(Bh))
+  RopeParams rope;            // RoPE of q at its position (cs == nullptr: none)
   int Bh_q, Bh_o;             // block of the rotation applied to q / to the output (1: none, the
   float rc_q, rc_o;           // caller folded it into the projections), and its fp32(1/sqrt(block))
   size_t pool_bytes, prot_bytes, qblob_total;   // extents, for the self-checks of debug builds
@@ -419,6 +427,7 @@ struct kv4_cache {
   int attn_ring;             // ring depth chosen for the per-head attention kernel
   int gattn_ring;            // ring depth of the page-major kernel (0: not used by this cache)
   int gattn_pair;            // INT4 tiles per consumer iteration of the page-major kernel (1 or 2)
+  kv4::RopeParams rope;      // registered RoPE table (cs == nullptr: none)
   cudaEvent_t ev_before;     // optional timing events around the split-K kernel
   cudaEvent_t ev_after;
 };
@@ -427,7 +436,7 @@ namespace kv4 {
 
 // Launchers (defined in the .cu files).
 int launch_append(kv4_cache* c, int layer, const int32_t* seq_ids, const int32_t* cu_new, int n_seqs, int total_new,
-                  const void* k_new, const void* v_new, cudaStream_t stream);
+                  const void* k_new, const void* v_new, bool rope, cudaStream_t stream);
 int launch_seq_reset(kv4_cache* c, int seq_id, cudaStream_t stream);
 int launch_dequantize_debug(kv4_cache* c, int layer, int seq_id, int start, int count, int view, float* k_out,
                             float* v_out, cudaStream_t stream);

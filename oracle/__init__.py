@@ -34,9 +34,10 @@ accuracy effect of INT4 versus BF16 (a model-level claim of both pages) is out
 of scope because it needs trained weights and datasets.
 """
 
-from . import hadamard, quant, layout, cache, attention  # noqa: F401
+from . import hadamard, quant, layout, cache, attention, rope  # noqa: F401
 from .hadamard import sylvester_hadamard, block_diag_hadamard, fwht_fp32, rotation_constant_fp32  # noqa: F401
 from .quant import (quantize_groups, dequantize_groups, fp16_round_down, fp16_round_up,  # noqa: F401
                     bf16_round, clamp_fp16_range)
 from .cache import OracleKV4Cache, OracleBF16Cache, prot_slot, n_prot_tiles  # noqa: F401
 from .attention import attention_fp64, decode_attention, decode_attention_bf16, extend_attention  # noqa: F401
+from .rope import rope_fp32, NEOX as ROPE_NEOX, GPTJ as ROPE_GPTJ  # noqa: F401

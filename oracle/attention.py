@@ -31,6 +31,7 @@ import numpy as np
 
 from .hadamard import fwht_fp32, block_diag_hadamard
 from .quant import bf16_round
+from .rope import rope_fp32
 
 
 def attention_fp64(q, k, v, scale):
@@ -66,22 +67,28 @@ def rotate_query(q, Bh):
     return bf16_round(fwht_fp32(q, Bh))
 
 
-def _query_and_output_rotation(cache, q, q_rotated, out_rotated):
+def _query_and_output_rotation(cache, q, q_rotated, out_rotated, rope=None, qpos=None):
     """q_rot and the matrix that takes o_rot to the output basis.
 
     q_rotated: the caller passes H q itself (H folded into its query
     projection), used as given.  out_rotated: the output stays in the rotated
-    basis (H folded into the output projection), so the map is the identity."""
+    basis (H folded into the output projection), so the map is the identity.
+    rope = (cos_sin, R, style): q first gets RoPE at positions qpos (fp32,
+    no bf16 rounding before the rotation)."""
+    if rope is not None:
+        q = rope_fp32(np.asarray(q, np.float32), qpos, *rope)
     q_rot = np.asarray(q, np.float32) if q_rotated else rotate_query(q, cache.Bh)
     back = np.eye(cache.D) if out_rotated else block_diag_hadamard(cache.D, cache.Bh).T
     return q_rot, back
 
 
-def decode_attention(cache, layer, seq_ids, q, scale=None, protected=True, q_rotated=False, out_rotated=False):
+def decode_attention(cache, layer, seq_ids, q, scale=None, protected=True, q_rotated=False, out_rotated=False,
+                     rope=None):
     """Decode attention of one query token per sequence over an OracleKV4Cache.
 
     q: [n, Hq, D] bf16 values (already H q when q_rotated; the output stays
-    in the rotated basis when out_rotated).  Returns dict with
+    in the rotated basis when out_rotated; rope: RoPE of q at position L - 1
+    first, L the sequence's length).  Returns dict with
       out_f64  [n, Hq, D]  fp64 output in the original (unrotated) basis,
       out_bf16 [n, Hq, D]  the same rounded to bf16 (held in fp32),
       q_rot    [n, Hq, D]  the rotated bf16 queries.
@@ -92,7 +99,9 @@ def decode_attention(cache, layer, seq_ids, q, scale=None, protected=True, q_rot
         scale = 1.0 / np.sqrt(D)
     n = len(seq_ids)
     out = np.zeros((n,) + q.shape[1:], np.float64)
-    q_rot, back = _query_and_output_rotation(cache, q, q_rotated, out_rotated)
+    lens = np.array([int(cache.seq_lens[layer, int(s)]) for s in seq_ids], np.int64)
+    qpos = np.maximum(lens - 1, 0)[:, None]
+    q_rot, back = _query_and_output_rotation(cache, q, q_rotated, out_rotated, rope, qpos)
     for i, seq in enumerate(seq_ids):
         kh, vh = cache.view(layer, int(seq), protected=protected)
         if kh.shape[0] == 0:
@@ -102,7 +111,8 @@ def decode_attention(cache, layer, seq_ids, q, scale=None, protected=True, q_rot
     return {"out_f64": out, "out_bf16": _bf16_of_f64(out), "q_rot": q_rot}
 
 
-def extend_attention(cache, layer, seq_ids, q, scale=None, protected=True, q_rotated=False, out_rotated=False):
+def extend_attention(cache, layer, seq_ids, q, scale=None, protected=True, q_rotated=False, out_rotated=False,
+                     rope=None):
     """Attention of several query tokens per sequence: the last T positions.
 
     q: [n, T, Hq, D] bf16 values, token i (0 = oldest) of a sequence of length
@@ -111,8 +121,8 @@ def extend_attention(cache, layer, seq_ids, q, scale=None, protected=True, q_rot
     one of length L (sinks and the last W positions of L from INT8; that the
     protected set follows the cache length, not the query position, is this
     library's reading: the cache holds one view at a time).  A token with no
-    visible position (L - T + i < 0) gets an all-zero row.  q_rotated and
-    out_rotated as in decode_attention.
+    visible position (L - T + i < 0) gets an all-zero row.  q_rotated,
+    out_rotated as in decode_attention; rope: RoPE of token i at L - T + i.
 
     Returns dict out_f64 / out_bf16 [n, T, Hq, D] and q_rot [n, T, Hq, D].
     """
@@ -122,7 +132,9 @@ def extend_attention(cache, layer, seq_ids, q, scale=None, protected=True, q_rot
         scale = 1.0 / np.sqrt(D)
     n, T = q.shape[0], q.shape[1]
     out = np.zeros(q.shape, np.float64)
-    q_rot, back = _query_and_output_rotation(cache, q, q_rotated, out_rotated)
+    lens = np.array([int(cache.seq_lens[layer, int(s)]) for s in seq_ids], np.int64)
+    qpos = np.maximum(lens[:, None] - T + np.arange(T)[None, :], 0)[:, :, None]
+    q_rot, back = _query_and_output_rotation(cache, q, q_rotated, out_rotated, rope, qpos)
     for b, seq in enumerate(seq_ids):
         kh, vh = cache.view(layer, int(seq), protected=protected)
         L = kh.shape[0]

@@ -23,7 +23,8 @@ Readings of this library (the pages give none of these details):
   pages for every position.
 * K and V are quantized separately, each with its own (s, z), each after the
   same block-diagonal Hadamard rotation.
-* Keys arrive post-RoPE; RoPE is not part of this cache.
+* Keys arrive post-RoPE, or get RoPE at their positions on the way in when a
+  table is given (append(..., rope=...), see rope.py).
 * Device byte order (head-innermost, so that the tiles of all KV heads at one
   page position are contiguous):
     INT4 pool of a layer   uint8 [num_pages][P/16][Hkv][16*D + 128]
@@ -35,6 +36,7 @@ Readings of this library (the pages give none of these details):
 import numpy as np
 
 from .hadamard import fwht_fp32
+from .rope import rope_fp32
 from .quant import quantize_groups, dequantize_groups
 from .layout import TILE, tables, int4_tile_bytes, int8_tile_bytes, bf16_tile_bytes, scale_offset
 
@@ -206,10 +208,11 @@ class OracleKV4Cache:
         xr = fwht_fp32(x, self.Bh)
         return xr, quantize_groups(xr, 4), quantize_groups(xr, 8)
 
-    def append(self, layer, seq_ids, cu_new, k_new, v_new):
+    def append(self, layer, seq_ids, cu_new, k_new, v_new, rope=None):
         """Append new tokens: seq_ids[i] receives rows cu_new[i]:cu_new[i+1] of k_new / v_new.
 
         k_new, v_new: [total_new, Hkv, D] bf16 values (as fp32 or bf16-exact floats).
+        rope: None, or (cos_sin, R, style): each new key first gets RoPE at its position.
         """
         k_new = np.asarray(k_new, np.float32)
         v_new = np.asarray(v_new, np.float32)
@@ -223,9 +226,12 @@ class OracleKV4Cache:
             L_new = L_old + n
             if L_new > cap:
                 raise ValueError("sequence %d would exceed its capacity of %d tokens" % (seq, cap))
-            _, k4, k8 = self.rotate_quantize(k_new[a:b])
-            _, v4, v8 = self.rotate_quantize(v_new[a:b])
             pos = L_old + np.arange(n)
+            kx = k_new[a:b]
+            if rope is not None:
+                kx = rope_fp32(kx, pos[:, None], *rope)
+            _, k4, k8 = self.rotate_quantize(kx)
+            _, v4, v8 = self.rotate_quantize(v_new[a:b])
             self._write_int4(layer, seq, pos, k4, v4)           # every position: INT4 page copy
             prot = (pos < self.S) | (pos >= L_new - self.W)      # sinks, and the last W of this append
             if np.any(prot):

@@ -126,3 +126,13 @@ def cache_config(w, num_pages, max_pages_per_seq, max_seqs=None, layers=None):
                 num_q_heads=w["Hq"], num_kv_heads=w["Hkv"], head_dim=w["D"],
                 page_size=w["P"], num_pages=num_pages, max_pages_per_seq=max_pages_per_seq,
                 hadamard_block=w["Bh"], sink_tokens=w["S"], recent_window=w["W"])
+
+
+def rope_cos_sin(max_pos, rotary_dim, base=1.0e6):
+    """The model's RoPE angle table (an input of the fused append / query kernels):
+    fp32 [max_pos][R], row p = cos(p * base^(-2i/R)) for i < R/2, then the sines.
+    Angles in fp64, each entry rounded once to fp32 (Qwen3 uses base 1e6)."""
+    half = rotary_dim // 2
+    inv = base ** (-2.0 * np.arange(half, dtype=np.float64) / rotary_dim)
+    ang = np.arange(max_pos, dtype=np.float64)[:, None] * inv[None, :]
+    return np.concatenate([np.cos(ang), np.sin(ang)], axis=1).astype(np.float32)
