@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--workload", default="qwen3_8b_layer")
     ap.add_argument("--impl", default="kv4", choices=["kv4", "reference"])
     ap.add_argument("--no-compare", action="store_true", help="skip the BF16-KV and INT4-only legs")
+    ap.add_argument("--rope", action="store_true",
+                    help="fuse RoPE (neox, rotary dim = head dim, base 1e6) into the append and query kernels")
     ap.add_argument("--cpu-seqs", type=int, default=4, help="sequences in the CPU oracle sample")
     ap.add_argument("--kernel-only", action="store_true",
                     help="time the device steps only (no e2e leg, comparison legs or CPU baseline): for profilers")
@@ -189,7 +191,7 @@ class ClockSampler:
 class Workload:
     """One replica: INT4 cache populated to L_b - 1 tokens, per-step new tokens and queries on the device."""
 
-    def __init__(self, w, device, extra_tokens, torch):
+    def __init__(self, w, device, extra_tokens, torch, rope=False):
         import int4_kv_cache_paged_b200 as kv4
         self.w = w
         self.device = device
@@ -203,7 +205,11 @@ class Workload:
         self.cu_one = torch.arange(self.B + 1, dtype=torch.int32, device=device)
         self.steps_k = []  # per step: k [B, Hkv, D] bf16
         self.steps_v = []
-        self.populate(torch, self.cache.append, extra_tokens)
+        self.rope = rope
+        if rope:   # the model's angle table (an input), registered once
+            max_pos = int(np.max(self.L)) + extra_tokens + 1
+            self.cache.set_rope(torch.from_numpy(workloads.rope_cos_sin(max_pos, w["D"])), w["D"], kv4.KV4_ROPE_NEOX)
+        self.populate(torch, lambda *a, **k: self.cache.append(*a, rope=rope, **k), extra_tokens)
 
     def populate(self, torch, append_fn, extra_tokens, layer=0, keep_steps=True):
         w, dev = self.w, self.device
@@ -272,7 +278,8 @@ def run_gpu(args):
         raise SystemExit("the benchmark times single-layer workloads; use the stack test for %s" % args.workload)
     extra = W_ + 2 * K + 1
     t0 = time.time()
-    wl = Workload(w, device, extra, torch)
+    wl = Workload(w, device, extra, torch, rope=args.rope)
+    amode = kv4.KV4_MODE_ROPE_Q if args.rope else 0
     setup_s = time.time() - t0
     B, Hkv, D, S, Wn = wl.B, w["Hkv"], w["D"], w["S"], w["W"]
     ws = wl.cache.workspace(B)
@@ -302,9 +309,9 @@ def run_gpu(args):
             flush.fill_(i & 0xFF)                  # evict the KV of the previous step from L2 (not timed)
             kv4.kv4_set_attention_events(wl.cache.handle, *e_kern[i])
             e_step[i][0].record(stream)
-            wl.cache.append(0, wl.seq_ids, wl.cu_one, wl.steps_k[i], wl.steps_v[i], total_new=B)
+            wl.cache.append(0, wl.seq_ids, wl.cu_one, wl.steps_k[i], wl.steps_v[i], total_new=B, rope=args.rope)
             e_attn[i][0].record(stream)
-            wl.cache.attention(0, wl.seq_ids, qs[i], out=out, workspace=ws)
+            wl.cache.attention(0, wl.seq_ids, qs[i], out=out, workspace=ws, mode=amode)
             e_attn[i][1].record(stream)
             e_step[i][1].record(stream)
             step_bytes.append(kv_bytes(wl.L + i, Hkv, D, S, Wn))
@@ -339,8 +346,8 @@ def run_gpu(args):
         dk.copy_(hk[j], non_blocking=True)
         dv.copy_(hv[j], non_blocking=True)
         dq.copy_(hq[j], non_blocking=True)
-        wl.cache.append(0, wl.seq_ids, wl.cu_one, dk, dv, total_new=B)
-        wl.cache.attention(0, wl.seq_ids, dq, out=out, workspace=ws)
+        wl.cache.append(0, wl.seq_ids, wl.cu_one, dk, dv, total_new=B, rope=args.rope)
+        wl.cache.attention(0, wl.seq_ids, dq, out=out, workspace=ws, mode=amode)
         hout.copy_(out, non_blocking=True)
         e_e2e[j][1].record(stream)
         e2e_bytes += kv_bytes(wl.L + n + j, Hkv, D, S, Wn)
@@ -351,7 +358,7 @@ def run_gpu(args):
 
     # ---- comparison legs on identical inputs (rank-local, untimed by the contract)
     compare = None
-    if not args.no_compare and not args.kernel_only and world == 1:
+    if not args.no_compare and not args.kernel_only and not args.rope and world == 1:
         compare = compare_legs(torch, kv4, w, wl, K, device, flush)
 
     (t_step_all, t_e2e_all), (bytes_all, e2e_bytes_all) = reduce_over_ranks(
@@ -384,7 +391,9 @@ def run_gpu(args):
                        "kv_bytes_per_step_mb": round(bytes_timed / K / 1e6, 1),
                        "l2": "flushed before every step by a 256 MB write outside the timed events; "
                              "per-step KV also exceeds the 126 MB L2",
-                       "parallelism": "replica per GPU" if world > 1 else "single GPU"},
+                       "parallelism": "replica per GPU" if world > 1 else "single GPU",
+                       "rope": ("neox, rotary dim %d, base 1e6, fused into the append and query kernels" % D
+                                if args.rope else "none (keys arrive post-RoPE)")},
             "tokens_per_s": round(B * world * K / t_step_all, 1),
             "hbm_frac_of_%s" % peak_kind: round(value / hbm, 4),
             "attention_kv_gbs": round(bytes_timed / t_attn / 1e9, 2),
@@ -479,22 +488,23 @@ def compare_legs(torch, kv4, w, wl, K, device, flush):
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def run_oracle_sample(w, n_seqs, steps, warm=1):
+def run_oracle_sample(w, n_seqs, steps, warm=1, rope=False):
     """The oracle on `n_seqs` sequences of the workload: populate (untimed), then `steps` decode steps."""
     import torch
     from threadpoolctl import threadpool_limits
-    from oracle import OracleKV4Cache, decode_attention
+    from oracle import OracleKV4Cache, decode_attention, ROPE_NEOX
 
     L = workloads.context_lengths(w)[:n_seqs]
     table, num_pages, mpps = workloads.block_table(dict(w, batch=n_seqs), L, extra_tokens=steps + warm + 1)
     cfg = workloads.cache_config(w, num_pages, mpps, max_seqs=n_seqs)
     orc = OracleKV4Cache(cfg, table)
+    rp = (workloads.rope_cos_sin(int(np.max(L)) + steps + warm + 1, w["D"]), w["D"], ROPE_NEOX) if rope else None
     toks = []
     with threadpool_limits(1):
         for s in range(n_seqs):
             k, v = workloads.kv_sequence(w, 0, s, int(L[s]) + steps + warm, device="cpu")
             k, v = k.float().numpy(), v.float().numpy()
-            orc.append(0, [s], [0, int(L[s]) - 1], k[:L[s] - 1], v[:L[s] - 1])
+            orc.append(0, [s], [0, int(L[s]) - 1], k[:L[s] - 1], v[:L[s] - 1], rope=rp)
             toks.append((k, v))
         times, nbytes = [], []
         for i in range(steps + warm):
@@ -502,8 +512,8 @@ def run_oracle_sample(w, n_seqs, steps, warm=1):
             vn = np.stack([toks[s][1][L[s] - 1 + i] for s in range(n_seqs)])
             q = workloads.queries(w, 0, i, n=n_seqs, device="cpu").float().numpy()
             t0 = time.perf_counter()
-            orc.append(0, list(range(n_seqs)), np.arange(n_seqs + 1), kn, vn)
-            decode_attention(orc, 0, list(range(n_seqs)), q)
+            orc.append(0, list(range(n_seqs)), np.arange(n_seqs + 1), kn, vn, rope=rp)
+            decode_attention(orc, 0, list(range(n_seqs)), q, rope=rp)
             dt = time.perf_counter() - t0
             if i >= warm:
                 times.append(dt)
@@ -511,8 +521,8 @@ def run_oracle_sample(w, n_seqs, steps, warm=1):
     return sum(nbytes) / sum(times) / 1e9, times, int(np.mean(L))
 
 
-def cpu_baseline(w, n_seqs):
-    gbs, times, mean_l = run_oracle_sample(w, n_seqs, steps=2)
+def cpu_baseline(w, n_seqs, rope=False):
+    gbs, times, mean_l = run_oracle_sample(w, n_seqs, steps=2, rope=rope)
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": "%d of %d sequences (mean context %d), 2 decode steps (append + attention), numpy, "
                       "BLAS limited to 1 thread; %.1f s per step" % (n_seqs, w["batch"], mean_l, np.mean(times))}
@@ -524,7 +534,7 @@ def run_reference(args):
         return None
     w = workloads.workload(args.workload)
     n_seqs = max(1, min(args.cpu_seqs, 2))
-    gbs, times, mean_l = run_oracle_sample(w, n_seqs, steps=args.steps, warm=args.warmup)
+    gbs, times, mean_l = run_oracle_sample(w, n_seqs, steps=args.steps, warm=args.warmup, rope=args.rope)
     t = sum(times)
     base = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": "%d of %d sequences (mean context %d) per step, numpy, BLAS limited to 1 thread"
@@ -532,7 +542,8 @@ def run_reference(args):
     return {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 attention, f32 codes",
-            "data": "synthetic", "config": {"workload": args.workload, "batch_sample": n_seqs},
+            "data": "synthetic", "config": {"workload": args.workload, "batch_sample": n_seqs,
+                                            "rope": "neox, fused" if args.rope else "none"},
             "cpu_baseline": base, "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                                           "d2h_bytes_per_step": 0}}
 
@@ -547,7 +558,7 @@ def main():
     res = run_gpu(args)
     if res is not None:
         if res["n_gpus"] == 1 and not args.kernel_only:
-            res["cpu_baseline"] = cpu_baseline(workloads.workload(args.workload), args.cpu_seqs)
+            res["cpu_baseline"] = cpu_baseline(workloads.workload(args.workload), args.cpu_seqs, rope=args.rope)
         print(json.dumps(res))
 
 
