@@ -1,11 +1,13 @@
 #!/usr/bin/env python
 """Decode-step benchmark of the paged INT4/INT8-protected KV cache on B200.
 
-One step = the whole hot path for one batch: fused rotate+quantize+append of one
-new token per sequence, then decode attention (query rotation; one persistent
+One step = the whole hot path for one batch, through one library call
+(kv4_decode_step): fused rotate+quantize+append of one new token per sequence
+and the query operands in one kernel, then decode attention (one persistent
 stream-K kernel over the INT4 pages and the INT8 sink/recent store that plans
 its own split and stores the groups it covers whole; a merge kernel for the
-groups split over several CTAs).  The metric is the algorithmic KV bytes the attention reads
+groups split over several CTAs).  --two-calls times the same step as
+kv4_rotate_quantize_append + kv4_decode_attention.  The metric is the algorithmic KV bytes the attention reads
 per step divided by the step time (GB/s), with decode tokens/s and the fraction
 of the measured HBM bandwidth beside it.
 
@@ -47,6 +49,8 @@ def parse():
     ap.add_argument("--workload", default="qwen3_8b_layer")
     ap.add_argument("--impl", default="kv4", choices=["kv4", "reference"])
     ap.add_argument("--no-compare", action="store_true", help="skip the BF16-KV and INT4-only legs")
+    ap.add_argument("--two-calls", action="store_true",
+                    help="run each step as kv4_rotate_quantize_append + kv4_decode_attention instead of kv4_decode_step")
     ap.add_argument("--rope", action="store_true",
                     help="fuse RoPE (neox, rotary dim = head dim, base 1e6) into the append and query kernels")
     ap.add_argument("--cpu-seqs", type=int, default=4, help="sequences in the CPU oracle sample")
@@ -276,7 +280,7 @@ def run_gpu(args):
         w = workloads.workload(args.workload, seed=w["seed"] + 7919 * rank)   # independent sequences per rank
     if w["layers"] > 1:
         raise SystemExit("the benchmark times single-layer workloads; use the stack test for %s" % args.workload)
-    extra = W_ + 2 * K + 1
+    extra = W_ + 3 * K + 1
     t0 = time.time()
     wl = Workload(w, device, extra, torch, rope=args.rope)
     amode = kv4.KV4_MODE_ROPE_Q if args.rope else 0
@@ -309,10 +313,14 @@ def run_gpu(args):
             flush.fill_(i & 0xFF)                  # evict the KV of the previous step from L2 (not timed)
             kv4.kv4_set_attention_events(wl.cache.handle, *e_kern[i])
             e_step[i][0].record(stream)
-            wl.cache.append(0, wl.seq_ids, wl.cu_one, wl.steps_k[i], wl.steps_v[i], total_new=B, rope=args.rope)
-            e_attn[i][0].record(stream)
-            wl.cache.attention(0, wl.seq_ids, qs[i], out=out, workspace=ws, mode=amode)
-            e_attn[i][1].record(stream)
+            if args.two_calls:
+                wl.cache.append(0, wl.seq_ids, wl.cu_one, wl.steps_k[i], wl.steps_v[i], total_new=B, rope=args.rope)
+                e_attn[i][0].record(stream)
+                wl.cache.attention(0, wl.seq_ids, qs[i], out=out, workspace=ws, mode=amode)
+                e_attn[i][1].record(stream)
+            else:   # one call: append + query operands, then the attention and merge kernels
+                wl.cache.decode_step(0, wl.seq_ids, wl.steps_k[i], wl.steps_v[i], qs[i], out=out, workspace=ws,
+                                     mode=amode)
             e_step[i][1].record(stream)
             step_bytes.append(kv_bytes(wl.L + i, Hkv, D, S, Wn))
         barrier()
@@ -322,8 +330,9 @@ def run_gpu(args):
 
     timed = range(W_, n)
     t_step = sum(e_step[i][0].elapsed_time(e_step[i][1]) for i in timed) / 1e3
-    t_attn = sum(e_attn[i][0].elapsed_time(e_attn[i][1]) for i in timed) / 1e3
     t_kern = sum(e_kern[i][0].elapsed_time(e_kern[i][1]) for i in timed) / 1e3
+    # two calls: the attention call's own events; one call: the attention and merge kernels
+    t_attn = sum(e_attn[i][0].elapsed_time(e_attn[i][1]) for i in timed) / 1e3 if args.two_calls else t_kern
     bytes_timed = sum(step_bytes[i] for i in timed)
     lens_after = wl.L + n - 1                       # length at the last timed attention call
 
@@ -346,8 +355,11 @@ def run_gpu(args):
         dk.copy_(hk[j], non_blocking=True)
         dv.copy_(hv[j], non_blocking=True)
         dq.copy_(hq[j], non_blocking=True)
-        wl.cache.append(0, wl.seq_ids, wl.cu_one, dk, dv, total_new=B, rope=args.rope)
-        wl.cache.attention(0, wl.seq_ids, dq, out=out, workspace=ws, mode=amode)
+        if args.two_calls:
+            wl.cache.append(0, wl.seq_ids, wl.cu_one, dk, dv, total_new=B, rope=args.rope)
+            wl.cache.attention(0, wl.seq_ids, dq, out=out, workspace=ws, mode=amode)
+        else:
+            wl.cache.decode_step(0, wl.seq_ids, dk, dv, dq, out=out, workspace=ws, mode=amode)
         hout.copy_(out, non_blocking=True)
         e_e2e[j][1].record(stream)
         e2e_bytes += kv_bytes(wl.L + n + j, Hkv, D, S, Wn)
@@ -359,7 +371,7 @@ def run_gpu(args):
     # ---- comparison legs on identical inputs (rank-local, untimed by the contract)
     compare = None
     if not args.no_compare and not args.kernel_only and not args.rope and world == 1:
-        compare = compare_legs(torch, kv4, w, wl, K, device, flush)
+        compare = compare_legs(torch, kv4, w, wl, K, device, flush, n + K_e2e)
 
     (t_step_all, t_e2e_all), (bytes_all, e2e_bytes_all) = reduce_over_ranks(
         [t_step, t_e2e], [float(bytes_timed), float(e2e_bytes)], device, world)
@@ -397,18 +409,21 @@ def run_gpu(args):
             "tokens_per_s": round(B * world * K / t_step_all, 1),
             "hbm_frac_of_%s" % peak_kind: round(value / hbm, 4),
             "attention_kv_gbs": round(bytes_timed / t_attn / 1e9, 2),
-            "append_us_per_step": round((t_step - t_attn) / K * 1e6, 2),
+            "api": "two calls: kv4_rotate_quantize_append + kv4_decode_attention" if args.two_calls else
+                   "one call: kv4_decode_step",
+            ("append_us_per_step" if args.two_calls else "append_and_query_us_per_step"):
+                round((t_step - t_attn) / K * 1e6, 2),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(achieved / hbm, 4), "traffic": traffic,
                          "kernel": "gattn_kernel: persistent stream-K attention over the INT4 pages and the "
-                                   "INT8 store (the events span the whole attention call: the query-operand "
-                                   "kernel before it and the merge kernel after it, both overlapped as "
-                                   "programmatic dependents)",
+                                   "INT8 store (the events span it and the merge kernel, its programmatic "
+                                   "dependent; with --two-calls also the query-operand kernel before it)",
                          "peak_source": peak_kind, "bytes_per_launch": int(bytes_timed / K)},
             "e2e": ({"value": round(e2e_bytes_all / t_e2e_all / 1e9, 2), "unit": "GB/s",
                      "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                      "tokens_per_s": round(B * world * K / t_e2e_all, 1)} if K_e2e else None),
-            "gpu_launches": 4 * K,   # per step: append_kernel, gq_kernel, gattn_kernel, gmerge_kernel
+            # per step: gstep_kernel, gattn_kernel, gmerge_kernel (two calls: append_kernel, gq_kernel, gattn, gmerge)
+            "gpu_launches": (4 if args.two_calls else 3) * K,
             "clocks": clk,
             "device_status": status,
             "setup_s": round(setup_s, 1),
@@ -421,14 +436,13 @@ def run_gpu(args):
     return result
 
 
-def compare_legs(torch, kv4, w, wl, K, device, flush):
+def compare_legs(torch, kv4, w, wl, K, device, flush, first_token):
     """Attention-only time of the INT4 path, the INT4-only mode, the multi-token query path and the BF16-KV
     kernel on identical inputs."""
     B, Hkv, D, S, Wn = wl.B, w["Hkv"], w["D"], w["S"], w["W"]
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     qs = [workloads.queries(w, 0, 1000 + i, device=device) for i in range(K)]
     out = torch.empty((B, w["Hq"], D), dtype=torch.bfloat16, device=device)
-    L_now = wl.L + int(wl.cache.seq_lens()[0, 0].item()) - int(wl.L[0])
 
     def time_attn(fn):
         es = [(ev(), ev()) for _ in range(K)]
@@ -444,10 +458,23 @@ def compare_legs(torch, kv4, w, wl, K, device, flush):
         return sum(a.elapsed_time(b) for a, b in es) / 1e3 / K
 
     ws = wl.cache.workspace(B)
+    # the same decode step as two calls (append, then attention) on the next K tokens
+    es = [(ev(), ev()) for _ in range(K)]
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        es[i][0].record()
+        wl.cache.append(0, wl.seq_ids, wl.cu_one, wl.steps_k[first_token + i], wl.steps_v[first_token + i],
+                        total_new=B)
+        wl.cache.attention(0, wl.seq_ids, qs[i], out=out, workspace=ws)
+        es[i][1].record()
+    torch.cuda.synchronize()
+    t_two = sum(a.elapsed_time(b) for a, b in es) / 1e3 / K
+    L_now = wl.L + int(wl.cache.seq_lens()[0, 0].item()) - int(wl.L[0])
     t_int4 = time_attn(lambda q: wl.cache.attention(0, wl.seq_ids, q, out=out, workspace=ws))
     t_only = time_attn(lambda q: wl.cache.attention(0, wl.seq_ids, q, out=out, workspace=ws,
                                                     mode=kv4.KV4_MODE_INT4_ONLY))
-    res = {"int4_protected": {"attention_ms": round(t_int4 * 1e3, 4),
+    res = {"step_as_two_calls": {"ms_per_step": round(t_two * 1e3, 4)},
+           "int4_protected": {"attention_ms": round(t_int4 * 1e3, 4),
                               "kv_gbs": round(kv_bytes(L_now, Hkv, D, S, Wn) / t_int4 / 1e9, 1)},
            "int4_only": {"attention_ms": round(t_only * 1e3, 4),
                          "kv_gbs": round(kv_bytes(L_now, Hkv, D, S, Wn, int4_only=True) / t_only / 1e9, 1)}}

@@ -260,6 +260,26 @@ int kv4_decode_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq
  * standing for (query token, query head) pairs.
  */
 int kv4_extend_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_t q_len, size_t* bytes);
+
+/*
+ * One decode step in one call: append one new token to every listed sequence
+ * (as kv4_rotate_quantize_append with cu_new = 0, 1, ..., n_seqs), then
+ * decode attention of q over the caches including that token (as
+ * kv4_decode_attention).  Codes, lengths and outputs are those of the two
+ * calls in a row.  With KV4_MODE_ROPE_Q the registered RoPE table is applied
+ * to the new keys (as kv4_rope_rotate_quantize_append) and to the queries.
+ *   k_new, v_new   bf16 [n_seqs][Hkv][D], the new token of entry i
+ *   q, out, mode, softmax_scale, dev_workspace   as kv4_decode_attention
+ *                  (the workspace of kv4_attention_workspace_bytes)
+ * The sequence ids must be distinct.  Needs num_kv_heads a multiple of 4 and
+ * at most 16 (KV4_ERR_UNSUPPORTED otherwise; use the two calls then).
+ * Kernels: one block per sequence appends its token (two warps per KV head,
+ * one for K and one for V) and builds the query operands, then the attention
+ * and merge kernels of kv4_decode_attention: three launches instead of four.
+ */
+int kv4_decode_step(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs,
+                    const void* k_new, const void* v_new, const void* q, void* out, float softmax_scale,
+                    int32_t mode, void* dev_workspace, size_t ws_bytes, kv4_stream_t stream);
 int kv4_extend_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs, int32_t q_len,
                          const void* q, void* out, float softmax_scale, int32_t mode,
                          void* dev_workspace, size_t ws_bytes, kv4_stream_t stream);

@@ -61,7 +61,7 @@ EXPORTS = [
     "kv4_cache_required_bytes", "kv4_cache_create", "kv4_cache_destroy", "kv4_cache_layout", "kv4_seq_reset",
     "kv4_rotate_quantize_append", "kv4_attention_workspace_bytes", "kv4_decode_attention",
     "kv4_decode_attention_noalloc", "kv4_extend_workspace_bytes", "kv4_extend_attention",
-    "kv4_set_rope", "kv4_rope_rotate_quantize_append",
+    "kv4_set_rope", "kv4_rope_rotate_quantize_append", "kv4_decode_step",
     "kv4_dequantize_debug", "kv4_get_status", "kv4_set_attention_events", "kv4_status_string", "kv4_version",
     "kv4bf16_cache_required_bytes", "kv4bf16_cache_create", "kv4bf16_cache_destroy", "kv4bf16_cache_layout",
     "kv4bf16_append", "kv4bf16_attention_workspace_bytes", "kv4bf16_decode_attention", "kv4bf16_get_status",
@@ -92,6 +92,7 @@ _sigs = {
     "kv4_decode_attention_noalloc": (_I, [_P, _I, _P, _I, _P, _P, ctypes.c_float, _I, _P]),
     "kv4_extend_workspace_bytes": (_I, [_P, _I, _I, ctypes.POINTER(_SZ)]),
     "kv4_set_rope": (_I, [_P, _P, _I, _I, _I]),
+    "kv4_decode_step": (_I, [_P, _I, _P, _I, _P, _P, _P, _P, ctypes.c_float, _I, _P, _SZ, _P]),
     "kv4_rope_rotate_quantize_append": (_I, [_P, _I, _P, _P, _I, _I, _P, _P, _P]),
     "kv4_extend_attention": (_I, [_P, _I, _P, _I, _I, _P, _P, ctypes.c_float, _I, _P, _SZ, _P]),
     "kv4_dequantize_debug": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
@@ -208,6 +209,14 @@ def kv4_rope_rotate_quantize_append(handle, layer, seq_ids, cu_new, n_seqs, tota
     _check(_lib.kv4_rope_rotate_quantize_append(handle, layer, _ptr(seq_ids), _ptr(cu_new), n_seqs, total_new,
                                                 _ptr(k_new), _ptr(v_new), _stream(stream)),
            "kv4_rope_rotate_quantize_append")
+
+
+def kv4_decode_step(handle, layer, seq_ids, n_seqs, k_new, v_new, q, out, softmax_scale, mode, workspace,
+                    stream=None):
+    _check(_lib.kv4_decode_step(handle, layer, _ptr(seq_ids), n_seqs, _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(out),
+                                float(softmax_scale), mode, _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream)),
+           "kv4_decode_step")
 
 
 def kv4_extend_workspace_bytes(handle, n_seqs, q_len):

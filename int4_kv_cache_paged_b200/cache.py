@@ -5,7 +5,7 @@ import torch
 from . import (make_config, kv4_cache_required_bytes, kv4_cache_create, kv4_cache_destroy, kv4_cache_layout,
                kv4_seq_reset, kv4_rotate_quantize_append, kv4_attention_workspace_bytes, kv4_decode_attention,
                kv4_decode_attention_noalloc, kv4_extend_workspace_bytes, kv4_extend_attention,
-               kv4_set_rope, kv4_rope_rotate_quantize_append,
+               kv4_set_rope, kv4_rope_rotate_quantize_append, kv4_decode_step,
                kv4_dequantize_debug, kv4_get_status, kv4bf16_cache_required_bytes, kv4bf16_cache_create,
                kv4bf16_cache_destroy, kv4bf16_cache_layout, kv4bf16_append, kv4bf16_attention_workspace_bytes,
                kv4bf16_decode_attention, kv4bf16_get_status, KV4_VIEW_EFFECTIVE, KV4_MODE_OUT_F32)
@@ -112,6 +112,17 @@ class KV4Cache(_Base):
         if workspace is None:
             workspace = self.workspace(n)
         kv4_decode_attention(self.handle, layer, seq_ids, n, q, out, scale, mode, workspace, stream)
+        return out
+
+    def decode_step(self, layer, seq_ids, k_new, v_new, q, out=None, scale=0.0, mode=0, workspace=None, stream=None):
+        """Append one token per sequence (k_new, v_new [n, Hkv, D] bf16) and attend q [n, Hq, D] in one call."""
+        n = int(seq_ids.numel())
+        if out is None:
+            dt = torch.float32 if (mode & KV4_MODE_OUT_F32) else torch.bfloat16
+            out = torch.empty(q.shape, dtype=dt, device=self.device)
+        if workspace is None:
+            workspace = self.workspace(n)
+        kv4_decode_step(self.handle, layer, seq_ids, n, k_new, v_new, q, out, scale, mode, workspace, stream)
         return out
 
     def extend_workspace(self, n_seqs, q_len):

@@ -266,6 +266,23 @@ int kv4_decode_attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, in
                    reinterpret_cast<cudaStream_t>(stream));
 }
 
+int kv4_decode_step(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_t n_seqs, const void* k_new,
+                    const void* v_new, const void* q, void* out, float softmax_scale, int32_t mode, void* ws,
+                    size_t ws_bytes, kv4_stream_t stream) {
+  if (!c || c->bf16 || check_layer(c, layer)) return KV4_ERR_INVALID_ARG;
+  if (n_seqs < 0 || n_seqs > c->cfg.max_seqs) return KV4_ERR_INVALID_ARG;
+  if (n_seqs == 0) return KV4_OK;
+  if (!seq_ids || !k_new || !v_new || !q || !out || !ws) return KV4_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(q) || !aligned16(out) ||
+      reinterpret_cast<uintptr_t>(ws) % kAlign)
+    return KV4_ERR_INVALID_ARG;
+  if (!mode_ok(c, mode)) return KV4_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return KV4_ERR_INVALID_ARG;
+  if (!select_device(c)) return KV4_ERR_CUDA;
+  return kv4::launch_decode_step(c, layer, seq_ids, n_seqs, k_new, v_new, q, out, softmax_scale, mode, ws, ws_bytes,
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
 int kv4_extend_workspace_bytes(const kv4_cache* c, int32_t n_seqs, int32_t q_len, size_t* bytes) {
   if (!c || c->bf16 || !bytes || n_seqs < 0 || q_len < 1) return KV4_ERR_INVALID_ARG;
   if (!kv4::grouped_path(c)) return KV4_ERR_UNSUPPORTED;

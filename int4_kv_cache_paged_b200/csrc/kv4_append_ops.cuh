@@ -1,0 +1,228 @@
+// Device pieces of the fused rotate + quantize + append, shared by the append
+// kernel and the fused decode step.  See kv4_append.cu for the arithmetic.
+#pragma once
+#include "kv4_common.cuh"
+
+namespace kv4 {
+
+namespace {
+
+struct AppendParams {
+  uint8_t* pool;             // INT4 or BF16 pool of the layer
+  uint8_t* prot;             // INT8 store of the layer (INT4 cache only)
+  const int32_t* block_table;
+  int32_t* seq_lens;         // this layer's row
+  const int32_t* seq_ids;
+  const int32_t* cu_new;
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  State* state;
+  int n_seqs, total_new, Hkv, D, P, S, W, Bh;
+  int max_seqs, num_pages, max_pages_per_seq;
+  float rot_c;               // fp32(1/sqrt(Bh))
+  RopeParams rope;           // RoPE of the keys at their positions (cs == nullptr: none)
+};
+
+// RoPE of one row held VPL consecutive dims per lane (dims VPL*lane ..), at
+// table row `pos`: pair (a, b) -> (a*c - b*s, b*c + a*s), every product and
+// sum rounded to fp32.  Neox pairs (d, d + R/2) sit R/(2*VPL) lanes apart (R
+// a power of two), gptj pairs (d, d + 1) in one lane.  All lanes call it.
+template <int VPL>
+__device__ __forceinline__ void rope_row(float (&x)[VPL], const RopeParams& r, int pos, int lane) {
+  const float* cs = r.cs + static_cast<long long>(pos) * r.R;
+  const int half = r.R >> 1, d0 = VPL * lane;
+  if (r.style == KV4_ROPE_GPTJ) {
+    if (d0 < r.R) {
+#pragma unroll
+      for (int k = 0; k < VPL; k += 2) {
+        const int i = (d0 + k) >> 1;
+        const float c = __ldg(cs + i), s = __ldg(cs + half + i);
+        const float a = x[k], b = x[k + 1];
+        x[k] = __fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s));
+        x[k + 1] = __fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s));
+      }
+    }
+  } else {
+    float y[VPL];
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) y[k] = __shfl_xor_sync(0xffffffffu, x[k], half / VPL);
+    if (d0 < r.R) {
+      const bool first = d0 < half;   // holds a; the partner lane holds b
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) {
+        const int i = first ? d0 + k : d0 + k - half;
+        const float c = __ldg(cs + i), s = __ldg(cs + half + i);
+        x[k] = first ? __fsub_rn(__fmul_rn(x[k], c), __fmul_rn(y[k], s))
+                     : __fadd_rn(__fmul_rn(x[k], c), __fmul_rn(y[k], s));
+      }
+    }
+  }
+}
+
+template <int VPL>
+__device__ __forceinline__ void fwht_warp(float (&x)[VPL], int Bh, float c, int lane) {
+  fwht_row<VPL>(x, Bh, lane);
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) x[i] = __fmul_rn(x[i], c);
+}
+
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Quantize the warp's group with Q = 2^bits - 1; codes go to smem, (s, z) are returned packed as half2 bits.
+template <int VPL>
+__device__ __forceinline__ uint32_t quantize_group(const float (&x)[VPL], float mn, float mx, float Q,
+                                                   uint8_t* codes, int lane) {
+  const __half z16 = __float2half_rd(mn);
+  const float z = __half2float(z16);
+  const float r = __fsub_rn(mx, z);
+  const __half s16 = (r == 0.f) ? __float2half(1.f) : __float2half_ru(__fdiv_rn(r, Q));
+  const float s = __half2float(s16);
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    float c = rintf(__fdiv_rn(__fsub_rn(x[i], z), s));
+    c = fminf(fmaxf(c, 0.f), Q);
+    codes[VPL * lane + i] = static_cast<uint8_t>(c);
+  }
+  return static_cast<uint32_t>(__half_as_ushort(s16)) | (static_cast<uint32_t>(__half_as_ushort(z16)) << 16);
+}
+
+// Write one token's INT4 codes (K: tensor 0, V: tensor 1) and scales into its tile.
+__device__ __forceinline__ void store_int4(uint8_t* tile, int r, int tensor, const uint8_t* codes, uint32_t sz,
+                                           int D, int lane) {
+  if (tensor == 0) {
+    // word (t, kk): byte j holds dim 32kk + 4t + j (low nibble) and 32kk + 16 + 4t + j (high nibble)
+    const int nkk = D / 32;
+    if (lane < D / 8) {
+      const int t = lane / nkk, kk = lane % nkk;
+      uint32_t w = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        w |= static_cast<uint32_t>(codes[32 * kk + 4 * t + j]) << (8 * j);
+        w |= static_cast<uint32_t>(codes[32 * kk + 16 + 4 * t + j]) << (8 * j + 4);
+      }
+      *reinterpret_cast<uint32_t*>(tile + r * (D / 2) + t * (D / 8) + 4 * kk) = w;
+    }
+  } else {
+    const int t = (r & 7) >> 1, e = r & 1, th = r >> 3;
+    for (int q = lane; q < D / 2; q += 32) {
+      const int m = q >> 3, g = q & 7;
+      const uint8_t b = static_cast<uint8_t>(codes[16 * m + g] | (codes[16 * m + g + 8] << 4));
+      tile[8 * D + 512 * (m >> 2) + 16 * (4 * g + t) + 4 * (m & 3) + th + 2 * e] = b;
+    }
+  }
+  if (lane == 0) *reinterpret_cast<uint32_t*>(tile + 16 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3))) = sz;
+}
+
+// Write one token's INT8 codes and scales into its protected tile.
+__device__ __forceinline__ void store_int8(uint8_t* tile, int r, int tensor, const uint8_t* codes, uint32_t sz,
+                                           int D, int lane) {
+  if (tensor == 0) {
+    // word L = (D/16) t + 2 kk + hf of the token: dims 32kk + 16hf + 4t + 0..3, one per byte
+    if (lane < D / 4) {
+      const int t = lane / (D / 16), wi = lane % (D / 16), kk = wi >> 1, hf = wi & 1;
+      const int d = 32 * kk + 16 * hf + 4 * t;
+      const uint32_t w = static_cast<uint32_t>(codes[d]) | (static_cast<uint32_t>(codes[d + 1]) << 8) |
+                         (static_cast<uint32_t>(codes[d + 2]) << 16) | (static_cast<uint32_t>(codes[d + 3]) << 24);
+      *reinterpret_cast<uint32_t*>(tile + r * D + 4 * lane) = w;
+    }
+  } else {
+    const int t = (r & 7) >> 1, e = r & 1, th = r >> 3;
+    for (int q = lane; q < D / 2; q += 32) {
+      const int m = q >> 3, gg = q & 7;
+      const int w = 2 * m + th;
+      const uint16_t v = static_cast<uint16_t>(codes[16 * m + gg] | (codes[16 * m + gg + 8] << 8));
+      *reinterpret_cast<uint16_t*>(tile + 16 * D + 16 * (32 * (w >> 2) + 4 * gg + t) + 4 * (w & 3) + 2 * e) = v;
+    }
+  }
+  if (lane == 0) *reinterpret_cast<uint32_t*>(tile + 32 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3))) = sz;
+}
+
+// Launch parameters of an append into `layer` of cache c.
+inline AppendParams append_params(const kv4_cache* c, int layer, const int32_t* seq_ids, const int32_t* cu_new,
+                                  int n_seqs, int total_new, const void* k_new, const void* v_new, bool rope) {
+  const kv4_config& cfg = c->cfg;
+  AppendParams p{};
+  if (rope) p.rope = c->rope;
+  uint8_t* lbase = c->base + c->pool_offset + static_cast<size_t>(layer) * c->layer_stride;
+  p.pool = lbase;
+  p.prot = c->bf16 ? nullptr : lbase + c->pool_bytes;
+  p.block_table = c->block_table;
+  p.seq_lens = c->seq_lens + static_cast<size_t>(layer) * cfg.max_seqs;
+  p.seq_ids = seq_ids;
+  p.cu_new = cu_new;
+  p.k_new = static_cast<const uint16_t*>(k_new);
+  p.v_new = static_cast<const uint16_t*>(v_new);
+  p.state = c->state;
+  p.n_seqs = n_seqs;
+  p.total_new = total_new;
+  p.Hkv = cfg.num_kv_heads;
+  p.D = cfg.head_dim;
+  p.P = cfg.page_size;
+  p.S = cfg.sink_tokens;
+  p.W = cfg.recent_window;
+  p.Bh = c->bf16 ? 1 : cfg.hadamard_block;
+  p.max_seqs = cfg.max_seqs;
+  p.num_pages = cfg.num_pages;
+  p.max_pages_per_seq = cfg.max_pages_per_seq;
+  p.rot_c = static_cast<float>(1.0 / sqrt(static_cast<double>(p.Bh)));
+  return p;
+}
+
+// Encode one (token, KV head, K or V) row held as bf16 bits raw[] (dims
+// VPL*lane ..): RoPE of a key when a table is set, rotation, clamp, INT4 codes
+// into its page tile and, for a protected position, INT8 codes into the
+// sequence's protected store.  tile_idx: the row's INT4 tile; r: its slot
+// there.  c4 / c8: the warp's code staging in shared memory.  All lanes call it.
+template <int D>
+__device__ __forceinline__ void encode_row(const AppendParams& p, const uint16_t (&raw)[D / 32], int tensor, int h,
+                                           int seq, int pos, int L_new, long long tile_idx, int r, uint8_t* c4,
+                                           uint8_t* c8, int lane) {
+  constexpr int VPL = D / 32;
+  float x[VPL];
+  bool bad = false;
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) {
+    const float v = __bfloat162float(__ushort_as_bfloat16(raw[k]));
+    bad |= !(fabsf(v) <= 3.0e38f);
+    x[k] = v;
+  }
+  if (tensor == 0 && p.rope.cs != nullptr) rope_row<VPL>(x, p.rope, pos, lane);   // the key at its position
+  fwht_warp<VPL>(x, p.Bh, p.rot_c, lane);
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) {
+    const float c = fminf(fmaxf(x[k], -65504.f), 65504.f);
+    bad |= (c != x[k]);
+    x[k] = c;
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&p.state->status, KV4_DEV_RANGE);
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int k = 1; k < VPL; ++k) { mn = fminf(mn, x[k]); mx = fmaxf(mx, x[k]); }
+  mn = warp_min(mn);
+  mx = warp_max(mx);
+  const uint32_t sz4 = quantize_group<VPL>(x, mn, mx, 15.f, c4, lane);
+  const bool protect = pos < p.S || pos >= L_new - p.W;
+  uint32_t sz8 = 0;
+  if (protect) sz8 = quantize_group<VPL>(x, mn, mx, 255.f, c8, lane);
+  __syncwarp();
+  store_int4(p.pool + tile_idx * tile4_bytes(D), r, tensor, c4, sz4, D, lane);
+  if (protect) {
+    const int slot = pos < p.S ? pos : p.S + (pos - p.S) % p.W;
+    const int npt = n_prot_tiles(p.S, p.W);
+    uint8_t* t8 = p.prot + ((static_cast<long long>(seq) * npt + slot / TILE) * p.Hkv + h) * tile8_bytes(D);
+    store_int8(t8, slot & (TILE - 1), tensor, c8, sz8, D, lane);
+  }
+}
+
+}  // namespace
+
+}  // namespace kv4

@@ -36,6 +36,7 @@
 // them, one warp per query head.  Every CTA records where the groups that
 // start in its range sit in the split, for that merge.
 #include "kv4_attn_tiles.cuh"
+#include "kv4_append_ops.cuh"
 
 namespace kv4 {
 
@@ -291,6 +292,72 @@ __global__ void __launch_bounds__(32 * QWARPS) gq_kernel(AttnParams p) {
   QFrag<D> qf;
   load_qfrag<D>(p, gw / p.Hkv, gw % p.Hkv, lane, qf);
   store_qblob<D>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D), qf, lane);
+}
+
+// ---------------------------------------------------------------------------
+// fused decode step, first kernel: one block per batch entry, two warps per
+// KV head.  Warp (tensor, h) appends the entry's new token of head h, K for
+// tensor 0 and V for tensor 1 (rotate, quantize, INT4 page and INT8 ring);
+// the V warp also builds the query operands of head h as gq_kernel does (RoPE
+// of q, when asked, at the new length).  Each warp loads its new row before
+// the sequence's state arrives.  The block advances the sequence length at
+// the end; the attention kernel follows in stream order, so it sees the new
+// token and the new length.
+
+template <int D>
+__global__ void __launch_bounds__(32 * 32) gstep_kernel(AttnParams p, AppendParams ap) {
+  constexpr int VPL = D / 32;
+  __shared__ __align__(16) uint8_t s_codes[32][2][D];
+  __shared__ int s_seq, s_L, s_ok, s_page;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tensor = warp >= p.Hkv ? 1 : 0, h = warp - tensor * p.Hkv;
+  const int b = blockIdx.x;
+  // this warp's new row: k_new / v_new [n_seqs][Hkv][D], entry b
+  uint16_t raw[VPL];
+  {
+    const uint16_t* src = (tensor ? ap.v_new : ap.k_new) + (static_cast<long long>(b) * p.Hkv + h) * D + VPL * lane;
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) raw[k] = src[k];
+  }
+  if (threadIdx.x == 0) {
+    const int seq = p.seq_ids[b];
+    int ok = seq >= 0 && seq < p.max_seqs;
+    if (!ok) atomicOr(&p.state->status, KV4_DEV_BAD_SEQ);
+    const int L = ok ? p.seq_lens[seq] : 0;
+    if (ok && L + 1 > p.max_pages_per_seq * p.P) {
+      atomicOr(&p.state->status, KV4_DEV_OVERFLOW);
+      ok = 0;
+    }
+    int page = -1;
+    if (ok) {
+      page = p.block_table[static_cast<long long>(seq) * p.max_pages_per_seq + L / p.P];
+      if (page < 0 || page >= p.num_pages) {
+        atomicOr(&p.state->status, KV4_DEV_BAD_PAGE);
+        page = -1;
+      }
+    }
+    s_seq = seq;
+    s_L = L;
+    s_ok = ok;
+    s_page = page;
+  }
+  __syncthreads();
+  const int seq = s_seq, L = s_L, page = s_page;
+  if (tensor == 1) {   // the query operands of head h (independent of the append)
+    QFrag<D> qf;
+    load_qfrag<D>(p, b, h, lane, qf, s_ok ? L + 1 : L);
+    store_qblob<D>(p.qblob + (static_cast<size_t>(b) * p.Hkv + h) * qblob_bytes(D), qf, lane);
+  }
+  if (s_ok && page >= 0) {
+    const long long tile_idx = (static_cast<long long>(page) * (p.P / TILE) + (L % p.P) / TILE) * p.Hkv + h;
+    const bool rope_past = tensor == 0 && ap.rope.cs != nullptr && L >= ap.rope.max_pos;
+    if (rope_past && lane == 0) atomicOr(&p.state->status, KV4_DEV_ROPE_POS);
+    if (!rope_past)
+      encode_row<D>(ap, raw, tensor, h, seq, L, L + 1, tile_idx, L & (TILE - 1), s_codes[warp][0], s_codes[warp][1],
+                    lane);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && s_ok) ap.seq_lens[seq] = L + 1;
 }
 
 // ---------------------------------------------------------------------------
@@ -830,7 +897,7 @@ int g_choose_ring(int device) {
 }
 
 template <int D>
-int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream) {
+int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const AppendParams* step = nullptr) {
   const GLayout l = g_layout(c, p.n_seqs, p.qlen);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   p.qblob = wsb + l.qblob;
@@ -839,9 +906,16 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream) {
   p.grid = g_grid(c);
   p.cap_parts = p.grid * 2 * GW;
   p.ns = c->gattn_ring;
-  if (c->ev_before) cudaEventRecord(c->ev_before, stream);
-  const int pairs = p.n_seqs * p.Hkv;
-  gq_kernel<D><<<(pairs + QWARPS - 1) / QWARPS, 32 * QWARPS, 0, stream>>>(p);
+  if (step) {
+    // fused decode step: the append and the query operands first; the attention
+    // kernel then starts in plain stream order (it plans from the new lengths)
+    gstep_kernel<D><<<p.n_seqs, 64 * p.Hkv, 0, stream>>>(p, *step);
+    if (c->ev_before) cudaEventRecord(c->ev_before, stream);
+  } else {
+    if (c->ev_before) cudaEventRecord(c->ev_before, stream);
+    const int pairs = p.n_seqs * p.Hkv;
+    gq_kernel<D><<<(pairs + QWARPS - 1) / QWARPS, 32 * QWARPS, 0, stream>>>(p);
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.grid);
   cfg.blockDim = dim3(GTHREADS);
@@ -851,7 +925,7 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = step ? 0 : 1;
   cudaError_t e = p.qlen > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true>, p, plan)
                               : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false>, p, plan);
   if (e == cudaSuccess) {
@@ -859,6 +933,7 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream) {
     mcfg.gridDim = dim3((p.n_seqs * p.Hkv * p.G + MWARPS - 1) / MWARPS);
     mcfg.blockDim = dim3(32 * MWARPS);
     mcfg.dynamicSmemBytes = 0;
+    mcfg.numAttrs = 1;   // programmatic dependent of the attention kernel
     e = cudaLaunchKernelEx(&mcfg, gmerge_kernel<D>, p, static_cast<const GPlanRec*>(plan));
   }
   if (c->ev_after) cudaEventRecord(c->ev_after, stream);
@@ -875,6 +950,20 @@ int grouped_ring(kv4_cache* c) {
 }
 
 size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs, int qlen) { return g_layout(c, n_seqs, qlen).total; }
+
+int launch_decode_step(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, const void* k_new,
+                       const void* v_new, const void* q, void* out, float softmax_scale, int mode, void* ws,
+                       size_t ws_bytes, cudaStream_t stream) {
+  if (!grouped_path(c) || c->cfg.num_kv_heads > 16) return KV4_ERR_UNSUPPORTED;   // two warps per KV head
+  if (c->gattn_ring <= 0 || c->gattn_ring > MAX_NS) return KV4_ERR_UNSUPPORTED;
+  if (n_seqs > c->cfg.max_seqs) return KV4_ERR_INVALID_ARG;
+  if (ws_bytes < g_layout(c, n_seqs, 1).total) return KV4_ERR_WORKSPACE;
+  AttnParams p{};
+  fill_common(c, layer, seq_ids, n_seqs, q, out, softmax_scale, mode, p);
+  const AppendParams ap = append_params(c, layer, seq_ids, nullptr, n_seqs, n_seqs, k_new, v_new,
+                                        (mode & KV4_MODE_ROPE_Q) != 0);
+  return p.D == 128 ? g_launch<128>(c, p, ws, stream, &ap) : g_launch<64>(c, p, ws, stream, &ap);
+}
 
 int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (p.qlen < 1 || p.G != p.qlen * p.Gh || p.G > MAX_G) return KV4_ERR_UNSUPPORTED;

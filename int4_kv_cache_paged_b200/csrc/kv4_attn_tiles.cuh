@@ -395,7 +395,8 @@ __device__ __forceinline__ void tile_bf16(uint32_t st, const QFrag<D>& qf, WarpS
 // tail holds sigma*log2(e)*sum(q) per column and the key scale factor.
 // sq: shared scratch of G*D floats for this warp.
 template <int D>
-__device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, int lane, QFrag<D>& qf);
+__device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, int lane, QFrag<D>& qf,
+                                           int L_known = -1);
 template <int D>
 __device__ __forceinline__ void store_qblob(uint8_t* blob, const QFrag<D>& qf, int lane);
 
@@ -540,8 +541,10 @@ __device__ __forceinline__ void rope_qfrag(float (&x)[NKK][2][4], const RopePara
   }
 }
 
+// L_known >= 0: the sequence's length, when the caller already has it (the
+// RoPE position of query token i is L - qlen + i); else it is read.
 template <int D>
-__device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, int lane, QFrag<D>& qf) {
+__device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, int lane, QFrag<D>& qf, int L_known) {
   constexpr int NKK = D / 32;
   const int G = p.G, g8 = lane >> 2, t = lane & 3;
   const bool colsplit = (G == 1 || G == 2 || G == 4);
@@ -562,8 +565,11 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
     }
   if (p.rope.cs != nullptr && active) {
     // the column's query token sits at position L - qlen + i of its sequence
-    const int seq = p.seq_ids[b];
-    const int L = (seq >= 0 && seq < p.max_seqs) ? p.seq_lens[seq] : 0;
+    int L = L_known;
+    if (L < 0) {
+      const int seq = p.seq_ids[b];
+      L = (seq >= 0 && seq < p.max_seqs) ? p.seq_lens[seq] : 0;
+    }
     int pos = max(L - p.qlen + gsrc / p.Gh, 0);
     if (pos >= p.rope.max_pos) {
       atomicOr(&p.state->status, KV4_DEV_ROPE_POS);

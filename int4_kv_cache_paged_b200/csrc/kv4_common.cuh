@@ -446,6 +446,11 @@ size_t attention_workspace_bytes(const kv4_cache* c, int n_seqs, int max_ctx);
 int launch_extend_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, int qlen, const void* q,
                             void* out, float softmax_scale, int mode, void* ws, size_t ws_bytes, cudaStream_t stream);
 int attention_blocks_per_sm(kv4_cache* c);
+void fill_common(const kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, const void* q, void* out,
+                 float softmax_scale, int mode, AttnParams& p);
+int launch_decode_step(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, const void* k_new,
+                       const void* v_new, const void* q, void* out, float softmax_scale, int mode, void* ws,
+                       size_t ws_bytes, cudaStream_t stream);
 // page-major path (INT4 cache, KV heads a multiple of 4)
 bool grouped_path(const kv4_cache* c);
 int grouped_ring(kv4_cache* c);
