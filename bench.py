@@ -130,6 +130,7 @@ class ClockSampler:
         self.samples = []
         self.windows = []
         self.error = None
+        self.nvml = None   # (pynvml, handle, max SM clock, reasons getter) once the thread has them
 
     def _handle(self, pynvml):
         """NVML handle of the torch device, matched by its PCI address (torch reports the parts as integers)."""
@@ -156,11 +157,11 @@ class ClockSampler:
             get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
                 pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
             smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.nvml = (pynvml, h, smax, get_reasons)
             while not self.stop.is_set():
-                t = time.perf_counter()
-                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
-                self.samples.append((t, sm, smax, int(get_reasons(h))))
+                self.sample_now()
                 time.sleep(0.002)
+            self.nvml = None
             pynvml.nvmlShutdown()
         except Exception as e:   # no NVML: reported as unavailable
             self.error = "%s: %s" % (type(e).__name__, e)
@@ -177,6 +178,19 @@ class ClockSampler:
         self.stop.set()
         self.thread.join(timeout=5)
 
+    def sample_now(self, n=1, gap=0.0):
+        """Take n samples from the calling thread (the timed loop calls it while its steps run on the GPU, so
+        that a short timed region has samples even when the sampling thread does not get to run)."""
+        for i in range(n):
+            nv = self.nvml
+            if nv is None:
+                return
+            pynvml, h, smax, get_reasons = nv
+            t = time.perf_counter()
+            self.samples.append((t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), smax, int(get_reasons(h))))
+            if gap:
+                time.sleep(gap)
+
     def window(self, t0, t1):
         self.windows.append((t0, t1))
 
@@ -187,7 +201,8 @@ class ClockSampler:
                     "note": self.error or "no sample inside the timed region"}
         reasons = sorted({name for x in inside for name, bit in self.REASONS if x[3] & bit})
         return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": max(x[2] for x in inside),
-                "reasons": reasons, "samples": len(inside), "source": "NVML, 2 ms period"}
+                "reasons": reasons, "samples": len(inside),
+                "source": "NVML: every 2 ms from a thread, plus samples taken while the timed steps run"}
 
 
 # --------------------------------------------------------------------------- GPU workload
@@ -280,7 +295,7 @@ def run_gpu(args):
         w = workloads.workload(args.workload, seed=w["seed"] + 7919 * rank)   # independent sequences per rank
     if w["layers"] > 1:
         raise SystemExit("the benchmark times single-layer workloads; use the stack test for %s" % args.workload)
-    extra = W_ + 3 * K + 1
+    extra = W_ + 5 * K + 1   # warm-up + timed steps, the kernel-event pass, e2e, two comparison legs
     t0 = time.time()
     wl = Workload(w, device, extra, torch, rope=args.rope)
     amode = kv4.KV4_MODE_ROPE_Q if args.rope else 0
@@ -295,9 +310,16 @@ def run_gpu(args):
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     n = W_ + K
     e_step = [(ev(), ev()) for _ in range(n)]
-    e_attn = [(ev(), ev()) for _ in range(n)]
-    e_kern = [(ev(), ev()) for _ in range(n)]
-    step_bytes = []
+    e_kern = [(ev(), ev()) for _ in range(K)]
+    step_bytes, kern_bytes = [], []
+
+    def one_step(i, q):
+        """The decode step on token i of every sequence: one library call (or the two calls)."""
+        if args.two_calls:
+            wl.cache.append(0, wl.seq_ids, wl.cu_one, wl.steps_k[i], wl.steps_v[i], total_new=B, rope=args.rope)
+            wl.cache.attention(0, wl.seq_ids, q, out=out, workspace=ws, mode=amode)
+        else:   # append + query operands, then the attention and merge kernels
+            wl.cache.decode_step(0, wl.seq_ids, wl.steps_k[i], wl.steps_v[i], q, out=out, workspace=ws, mode=amode)
 
     def barrier():
         if world > 1:
@@ -311,18 +333,24 @@ def run_gpu(args):
                 barrier()
                 t_window = time.perf_counter()
             flush.fill_(i & 0xFF)                  # evict the KV of the previous step from L2 (not timed)
-            kv4.kv4_set_attention_events(wl.cache.handle, *e_kern[i])
             e_step[i][0].record(stream)
-            if args.two_calls:
-                wl.cache.append(0, wl.seq_ids, wl.cu_one, wl.steps_k[i], wl.steps_v[i], total_new=B, rope=args.rope)
-                e_attn[i][0].record(stream)
-                wl.cache.attention(0, wl.seq_ids, qs[i], out=out, workspace=ws, mode=amode)
-                e_attn[i][1].record(stream)
-            else:   # one call: append + query operands, then the attention and merge kernels
-                wl.cache.decode_step(0, wl.seq_ids, wl.steps_k[i], wl.steps_v[i], qs[i], out=out, workspace=ws,
-                                     mode=amode)
+            one_step(i, qs[i])
             e_step[i][1].record(stream)
             step_bytes.append(kv_bytes(wl.L + i, Hkv, D, S, Wn))
+        clocks.sample_now(4, 0.0003)                # while the queued steps run
+        barrier()
+        clocks.window(t_window, time.perf_counter())
+        # the same steps again on the next K tokens, now with the library's events around the attention
+        # kernel and its merge kernel (with --two-calls also the query-operand kernel): they give the
+        # roofline's kernel time.  They are kept out of the loop above because each event marker between
+        # two launches adds about 2 us to the step.
+        t_window = time.perf_counter()
+        for j in range(K):
+            flush.fill_(j & 0xFF)
+            kv4.kv4_set_attention_events(wl.cache.handle, *e_kern[j])
+            one_step(n + j, qs[W_ + j])
+            kern_bytes.append(kv_bytes(wl.L + n + j, Hkv, D, S, Wn))
+        clocks.sample_now(4, 0.0003)
         barrier()
         clocks.window(t_window, time.perf_counter())
     kv4.kv4_set_attention_events(wl.cache.handle, None, None)
@@ -330,11 +358,11 @@ def run_gpu(args):
 
     timed = range(W_, n)
     t_step = sum(e_step[i][0].elapsed_time(e_step[i][1]) for i in timed) / 1e3
-    t_kern = sum(e_kern[i][0].elapsed_time(e_kern[i][1]) for i in timed) / 1e3
-    # two calls: the attention call's own events; one call: the attention and merge kernels
-    t_attn = sum(e_attn[i][0].elapsed_time(e_attn[i][1]) for i in timed) / 1e3 if args.two_calls else t_kern
+    t_kern = sum(a.elapsed_time(b) for a, b in e_kern) / 1e3
+    t_attn = t_kern
     bytes_timed = sum(step_bytes[i] for i in timed)
-    lens_after = wl.L + n - 1                       # length at the last timed attention call
+    bytes_kern = sum(kern_bytes)
+    n += K                                          # tokens used so far
 
     # ---- e2e through the public API with host buffers (pinned), copies inside the timed region
     if args.kernel_only:
@@ -380,7 +408,7 @@ def run_gpu(args):
     if rank == 0:
         peaks, peak_kind = measured_peaks()
         hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
-        achieved = bytes_timed / t_kern / 1e9
+        achieved = bytes_kern / t_kern / 1e9
         value = bytes_all / t_step_all / 1e9
         traffic = profiled_traffic(args.workload)
         clk = clocks.summary()
@@ -408,7 +436,7 @@ def run_gpu(args):
                                 if args.rope else "none (keys arrive post-RoPE)")},
             "tokens_per_s": round(B * world * K / t_step_all, 1),
             "hbm_frac_of_%s" % peak_kind: round(value / hbm, 4),
-            "attention_kv_gbs": round(bytes_timed / t_attn / 1e9, 2),
+            "attention_kv_gbs": round(bytes_kern / t_attn / 1e9, 2),
             "api": "two calls: kv4_rotate_quantize_append + kv4_decode_attention" if args.two_calls else
                    "one call: kv4_decode_step",
             ("append_us_per_step" if args.two_calls else "append_and_query_us_per_step"):
@@ -418,7 +446,9 @@ def run_gpu(args):
                          "kernel": "gattn_kernel: persistent stream-K attention over the INT4 pages and the "
                                    "INT8 store (the events span it and the merge kernel, its programmatic "
                                    "dependent; with --two-calls also the query-operand kernel before it)",
-                         "peak_source": peak_kind, "bytes_per_launch": int(bytes_timed / K)},
+                         "peak_source": peak_kind, "bytes_per_launch": int(bytes_kern / K),
+                         "timing": "CUDA events recorded by the library around the kernels, over K steps that "
+                                   "follow the timed loop on the same workload"},
             "e2e": ({"value": round(e2e_bytes_all / t_e2e_all / 1e9, 2), "unit": "GB/s",
                      "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                      "tokens_per_s": round(B * world * K / t_e2e_all, 1)} if K_e2e else None),
@@ -458,22 +488,30 @@ def compare_legs(torch, kv4, w, wl, K, device, flush, first_token):
         return sum(a.elapsed_time(b) for a, b in es) / 1e3 / K
 
     ws = wl.cache.workspace(B)
-    # the same decode step as two calls (append, then attention) on the next K tokens
-    es = [(ev(), ev()) for _ in range(K)]
-    for i in range(K):
-        flush.fill_(i & 0xFF)
-        es[i][0].record()
-        wl.cache.append(0, wl.seq_ids, wl.cu_one, wl.steps_k[first_token + i], wl.steps_v[first_token + i],
-                        total_new=B)
-        wl.cache.attention(0, wl.seq_ids, qs[i], out=out, workspace=ws)
-        es[i][1].record()
-    torch.cuda.synchronize()
-    t_two = sum(a.elapsed_time(b) for a, b in es) / 1e3 / K
+    # the decode step as two calls (append, then attention), then as one call, on the next 2K tokens
+    def time_steps(fn, t0):
+        es = [(ev(), ev()) for _ in range(K)]
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            es[i][0].record()
+            fn(t0 + i, qs[i])
+            es[i][1].record()
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in es) / 1e3 / K
+
+    def two_calls(i, q):
+        wl.cache.append(0, wl.seq_ids, wl.cu_one, wl.steps_k[i], wl.steps_v[i], total_new=B)
+        wl.cache.attention(0, wl.seq_ids, q, out=out, workspace=ws)
+
+    t_two = time_steps(two_calls, first_token)
+    t_one = time_steps(lambda i, q: wl.cache.decode_step(0, wl.seq_ids, wl.steps_k[i], wl.steps_v[i], q, out=out,
+                                                          workspace=ws), first_token + K)
     L_now = wl.L + int(wl.cache.seq_lens()[0, 0].item()) - int(wl.L[0])
     t_int4 = time_attn(lambda q: wl.cache.attention(0, wl.seq_ids, q, out=out, workspace=ws))
     t_only = time_attn(lambda q: wl.cache.attention(0, wl.seq_ids, q, out=out, workspace=ws,
                                                     mode=kv4.KV4_MODE_INT4_ONLY))
     res = {"step_as_two_calls": {"ms_per_step": round(t_two * 1e3, 4)},
+           "step_as_one_call": {"ms_per_step": round(t_one * 1e3, 4)},
            "int4_protected": {"attention_ms": round(t_int4 * 1e3, 4),
                               "kv_gbs": round(kv_bytes(L_now, Hkv, D, S, Wn) / t_int4 / 1e9, 1)},
            "int4_only": {"attention_ms": round(t_only * 1e3, 4),

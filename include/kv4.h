@@ -249,15 +249,17 @@ int kv4_decode_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq
  * kv4_decode_attention.  ("SAW-INT4 ...", Abstract: fused attention over the
  * paged quantized cache; the causal mask over the new tokens is the textbook
  * one.)
- *   q_len          1 <= q_len, q_len * (Hq/Hkv) <= 8: the query tokens and
- *                  heads of one KV head share one 8-column tensor-core operand
+ *   q_len          >= 1.  The query tokens and heads of one KV head share one
+ *                  8-column tensor-core operand, so one pass over the cache
+ *                  serves 8 / (Hq/Hkv) tokens; more tokens run as several
+ *                  passes in stream order (q_len * Hq/Hkv <= 8: one pass)
  *   q, out         bf16 [n_seqs][q_len][Hq][D] (out fp32 with KV4_MODE_OUT_F32)
  *   dev_workspace  >= kv4_extend_workspace_bytes(cache, n_seqs, q_len, ...)
  * A query token with no visible position (L < q_len - i) gets an all-zero row.
- * Errors: KV4_ERR_UNSUPPORTED when num_kv_heads is not a multiple of 4 or
- * q_len * Hq/Hkv > 8; the others as kv4_decode_attention.  Same kernels as
- * kv4_decode_attention with KV heads a multiple of 4, with the operand columns
- * standing for (query token, query head) pairs.
+ * Errors: KV4_ERR_UNSUPPORTED when num_kv_heads is not a multiple of 4; the
+ * others as kv4_decode_attention.  Same kernels as kv4_decode_attention with
+ * KV heads a multiple of 4, with the operand columns standing for (query
+ * token, query head) pairs.
  */
 int kv4_extend_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_t q_len, size_t* bytes);
 

@@ -160,7 +160,6 @@ int extend_attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_
   if (!c || check_layer(c, layer)) return KV4_ERR_INVALID_ARG;
   if (n_seqs < 0 || n_seqs > c->cfg.max_seqs || q_len < 1) return KV4_ERR_INVALID_ARG;
   if (!kv4::grouped_path(c)) return KV4_ERR_UNSUPPORTED;
-  if (static_cast<long long>(q_len) * (c->cfg.num_q_heads / c->cfg.num_kv_heads) > kv4::MAX_G) return KV4_ERR_UNSUPPORTED;
   if (n_seqs == 0) return KV4_OK;
   if (!seq_ids || !q || !out || !ws) return KV4_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || reinterpret_cast<uintptr_t>(ws) % kAlign) return KV4_ERR_INVALID_ARG;
@@ -286,8 +285,7 @@ int kv4_decode_step(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_t
 int kv4_extend_workspace_bytes(const kv4_cache* c, int32_t n_seqs, int32_t q_len, size_t* bytes) {
   if (!c || c->bf16 || !bytes || n_seqs < 0 || q_len < 1) return KV4_ERR_INVALID_ARG;
   if (!kv4::grouped_path(c)) return KV4_ERR_UNSUPPORTED;
-  if (static_cast<long long>(q_len) * (c->cfg.num_q_heads / c->cfg.num_kv_heads) > kv4::MAX_G) return KV4_ERR_UNSUPPORTED;
-  *bytes = kv4::grouped_workspace_bytes(c, n_seqs, q_len);
+  *bytes = kv4::grouped_workspace_bytes(c, n_seqs, kv4::extend_chunk(c, q_len));
   return KV4_OK;
 }
 

@@ -680,6 +680,8 @@ void fill_common(const kv4_cache* c, int layer, const int32_t* seq_ids, int n_se
   p.G = cfg.num_q_heads / cfg.num_kv_heads;
   p.Gh = p.G;
   p.qlen = 1;
+  p.q0 = 0;
+  p.qtot = 1;
   p.D = cfg.head_dim;
   p.P = cfg.page_size;
   p.S = cfg.sink_tokens;
@@ -710,19 +712,34 @@ size_t attention_workspace_bytes(const kv4_cache* c, int n_seqs, int max_ctx) {
   return ws_layout(c, n_seqs, static_cast<int>(cap0)).total;
 }
 
+// Query tokens of one pass of the multi-token path: as many as fit the
+// 8 operand columns of a KV head.
+int extend_chunk(const kv4_cache* c, int qlen) {
+  const int per = MAX_G / (c->cfg.num_q_heads / c->cfg.num_kv_heads);
+  return qlen < per ? qlen : per;
+}
+
 // Attention of the last qlen positions of every sequence (the page-major path
-// with qlen * Hq/Hkv operand columns per KV head; token i of a sequence of
-// length L sees the positions 0 .. L - qlen + i).
+// with (tokens of a pass) * Hq/Hkv operand columns per KV head; token i of a
+// sequence of length L sees the positions 0 .. L - qlen + i).  More tokens
+// than one operand holds run as several passes over the cache, in stream
+// order, sharing the workspace.
 int launch_extend_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, int qlen, const void* q,
                             void* out, float softmax_scale, int mode, void* ws, size_t ws_bytes,
                             cudaStream_t stream) {
   if (!grouped_path(c)) return KV4_ERR_UNSUPPORTED;
   AttnParams p{};
   fill_common(c, layer, seq_ids, n_seqs, q, out, softmax_scale, mode, p);
-  p.qlen = qlen;
-  p.G = qlen * p.Gh;
-  if (p.G > MAX_G) return KV4_ERR_UNSUPPORTED;
-  return launch_grouped(c, p, ws, ws_bytes, stream);
+  const int chunk = extend_chunk(c, qlen);
+  p.qtot = qlen;
+  for (int q0 = 0; q0 < qlen; q0 += chunk) {
+    p.q0 = q0;
+    p.qlen = qlen - q0 < chunk ? qlen - q0 : chunk;
+    p.G = p.qlen * p.Gh;
+    const int rc = launch_grouped(c, p, ws, ws_bytes, stream);
+    if (rc != KV4_OK) return rc;
+  }
+  return KV4_OK;
 }
 
 int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs, const void* q, void* out,
@@ -775,6 +792,8 @@ int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs
   p.G = G;
   p.Gh = G;
   p.qlen = 1;
+  p.q0 = 0;
+  p.qtot = 1;
   p.D = D;
   p.P = cfg.page_size;
   p.S = cfg.sink_tokens;

@@ -644,7 +644,7 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
         }
         if (!ok) break;
         const int pos0 = (g.t0 + u) * TILE;
-        const int vis = g.L - (MULTI ? p.qlen : 1);   // the last position every query token sees
+        const int vis = MULTI ? g.L - p.qtot + p.q0 : g.L - 1;   // the last position every column sees
         const bool inside = pos0 >= g.lo4 && pos0 + nt * TILE <= (MULTI ? min(g.hi4, vis + 1) : g.hi4);
         if (inside) {
 #pragma unroll
@@ -686,7 +686,7 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
           } else {
             // position of protected slot sl: a sink below S, else the ring position
             // in [max(S, L - W), L) congruent to sl - S modulo W
-            const int rlo = max(p.S, g.L - p.W), vis = g.L - p.qlen;
+            const int rlo = max(p.S, g.L - p.W), vis = g.L - p.qtot + p.q0;
             auto pos_of = [&](int sl) {
               return sl < p.S ? sl : rlo + (((sl - p.S) - (rlo - p.S)) % p.W + p.W) % p.W;
             };
@@ -926,7 +926,8 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = step ? 0 : 1;
-  cudaError_t e = p.qlen > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true>, p, plan)
+  // several query tokens per sequence (even a pass of one of them): the causal variant
+  cudaError_t e = p.qtot > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true>, p, plan)
                               : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false>, p, plan);
   if (e == cudaSuccess) {
     cudaLaunchConfig_t mcfg = cfg;
@@ -966,7 +967,8 @@ int launch_decode_step(kv4_cache* c, int layer, const int32_t* seq_ids, int n_se
 }
 
 int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  if (p.qlen < 1 || p.G != p.qlen * p.Gh || p.G > MAX_G) return KV4_ERR_UNSUPPORTED;
+  if (p.qlen < 1 || p.G != p.qlen * p.Gh || p.G > MAX_G || p.q0 < 0 || p.q0 + p.qlen > p.qtot)
+    return KV4_ERR_UNSUPPORTED;
   if (ws_bytes < g_layout(c, p.n_seqs, p.qlen).total) return KV4_ERR_WORKSPACE;
   if (c->gattn_ring <= 0 || c->gattn_ring > MAX_NS) return KV4_ERR_UNSUPPORTED;
   if (p.n_seqs > c->cfg.max_seqs) return KV4_ERR_INVALID_ARG;

@@ -542,7 +542,7 @@ __device__ __forceinline__ void rope_qfrag(float (&x)[NKK][2][4], const RopePara
 }
 
 // L_known >= 0: the sequence's length, when the caller already has it (the
-// RoPE position of query token i is L - qlen + i); else it is read.
+// RoPE position of query token i is L - qtot + i); else it is read.
 template <int D>
 __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, int lane, QFrag<D>& qf, int L_known) {
   constexpr int NKK = D / 32;
@@ -570,7 +570,7 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
       const int seq = p.seq_ids[b];
       L = (seq >= 0 && seq < p.max_seqs) ? p.seq_lens[seq] : 0;
     }
-    int pos = max(L - p.qlen + gsrc / p.Gh, 0);
+    int pos = max(L - p.qtot + p.q0 + gsrc / p.Gh, 0);
     if (pos >= p.rope.max_pos) {
       atomicOr(&p.state->status, KV4_DEV_ROPE_POS);
       pos = p.rope.max_pos - 1;

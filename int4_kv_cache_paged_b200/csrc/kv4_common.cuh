@@ -100,7 +100,9 @@ struct AttnParams {
   float* partials;            // [cap_parts][G][D + 4]: o[D], m, l, pad
   int cap_parts;
   int n_seqs, Hq, Hkv, G, D, P, S, W, Bh;   // G: operand columns per KV head (qlen * Gh)
-  int qlen, Gh;               // query tokens per sequence (the last qlen positions), query heads per KV head
+  int qlen, Gh;               // query tokens of this launch, query heads per KV head
+  int q0, qtot;               // first query token of this launch, query tokens per sequence (the last qtot
+                              // positions; a call with more tokens than one operand holds runs in chunks)
   int max_seqs, num_pages, max_pages_per_seq;
   int chunk_tiles;
   int mode;
@@ -115,11 +117,11 @@ struct AttnParams {
 };
 
 // Row of q (and of the output) that operand column c of KV head h of batch
-// entry b stands for: query token c / Gh of the entry (the tokens are the
-// last qlen positions, oldest first), query head h * Gh + c % Gh.
+// entry b stands for: query token q0 + c / Gh of the entry (the tokens are the
+// last qtot positions, oldest first), query head h * Gh + c % Gh.
 __device__ __forceinline__ long long q_row(const AttnParams& p, int b, int h, int c) {
   const int i = c / p.Gh, g = c - i * p.Gh;
-  return (static_cast<long long>(b) * p.qlen + i) * p.Hq + h * p.Gh + g;
+  return (static_cast<long long>(b) * p.qtot + p.q0 + i) * p.Hq + h * p.Gh + g;
 }
 
 // ---------------------------------------------------------------------------
@@ -455,6 +457,7 @@ int launch_decode_step(kv4_cache* c, int layer, const int32_t* seq_ids, int n_se
 bool grouped_path(const kv4_cache* c);
 int grouped_ring(kv4_cache* c);
 size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs, int qlen);
+int extend_chunk(const kv4_cache* c, int qlen);
 int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 }  // namespace kv4

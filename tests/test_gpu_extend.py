@@ -2,7 +2,7 @@
 positions of every sequence attend causally over the cache, each query token
 over the positions up to its own.  Compared with the oracle's extend_attention
 on the same seeded inputs: every (query token, head) ratio that fits one
-8-column operand, lengths below T, empty sequences, a recent window shorter
+8-column operand, more query rows than that (several passes), lengths below T, empty sequences, a recent window shorter
 than T (the causal tail then reaches INT4 pages), the INT4-only view, one long
 sequence split over every CTA, and T = 1 against decode attention."""
 
@@ -111,12 +111,25 @@ def test_extend_one_token_is_decode(kv4):
     assert torch.equal(ext[:, 0], dec)
 
 
+@pytest.mark.parametrize("Hq,Hkv,T", [(32, 8, 3), (32, 8, 4), (64, 8, 2), (16, 8, 7)])
+def test_extend_in_several_passes(kv4, Hq, Hkv, T):
+    """More query rows than one 8-column operand: passes of 8 / G tokens, each with its causal offset."""
+    rng = np.random.default_rng(1000 * Hq + T)
+    D, n = 128, 5
+    mpps = 700 // 16 + 2
+    cfg = cfg_dict(D=D, Hq=Hq, Hkv=Hkv, P=16, Bh=128, S=4, W=64, num_pages=n * mpps, mpps=mpps, max_seqs=n)
+    pair = Pair(cfg, random_table(n, mpps, n * mpps, rng))
+    lens = [700, 2, 0, T, 90]
+    _populate(pair, rng, list(range(n)), lens, Hkv, D)
+    seqs = [4, 0, 2, 1, 3]
+    q = bf16_values((n, T, Hq, D), rng)
+    out, _ = _check(kv4, pair, seqs, q)
+    _check(kv4, pair, seqs, q, mode=kv4.KV4_MODE_INT4_ONLY)
+    assert torch.all(out[seqs.index(2)] == 0)
+
+
 def test_extend_rejects_unsupported_shapes(kv4):
     rng = np.random.default_rng(79)
-    cfg = cfg_dict(D=64, Hq=32, Hkv=8, P=16, Bh=64, S=4, W=32, num_pages=8, mpps=4, max_seqs=2)
-    pair = Pair(cfg, random_table(2, 4, 8, rng))
-    with pytest.raises(kv4.KV4Error):                              # 3 tokens x 4 heads > 8 columns
-        _extend(pair, [0, 1], bf16_values((2, 3, 32, 64), rng))
     cfg2 = cfg_dict(D=64, Hq=4, Hkv=2, P=16, Bh=64, S=4, W=32, num_pages=8, mpps=4, max_seqs=2)
     pair2 = Pair(cfg2, random_table(2, 4, 8, rng))
     with pytest.raises(kv4.KV4Error):                              # KV heads not a multiple of 4
