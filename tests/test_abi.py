@@ -64,3 +64,26 @@ def test_host_side_validation_without_a_device():
     assert kv4._lib.kv4_cache_destroy(None) == kv4.KV4_ERR_INVALID_ARG
     assert kv4._lib.kv4_status_string(kv4.KV4_ERR_WORKSPACE) == b"workspace too small"
     assert kv4.version().endswith("sm_100a")
+
+
+def test_newer_entry_points_reject_bad_arguments_without_a_device():
+    """The multi-token, RoPE and fused-step entry points check their arguments on the host first."""
+    import int4_kv_cache_paged_b200 as kv4
+    lib = kv4._lib
+    size = ctypes.c_size_t()
+    assert lib.kv4_extend_workspace_bytes(None, 4, 2, ctypes.byref(size)) == kv4.KV4_ERR_INVALID_ARG
+    assert lib.kv4_extend_attention(None, 0, None, 1, 2, None, None, 0.0, 0, None, 0, None) == kv4.KV4_ERR_INVALID_ARG
+    assert lib.kv4_set_rope(None, None, 16, 64, 0) == kv4.KV4_ERR_INVALID_ARG
+    assert lib.kv4_rope_rotate_quantize_append(None, 0, None, None, 1, 1, None, None, None) == kv4.KV4_ERR_INVALID_ARG
+    assert lib.kv4_decode_step(None, 0, None, 1, None, None, None, None, 0.0, 0, None, 0, None) == \
+        kv4.KV4_ERR_INVALID_ARG
+
+
+def test_mode_bits_of_the_binding_match_the_header():
+    import int4_kv_cache_paged_b200 as kv4
+    text = open(HEADER).read()
+    for name in ("KV4_MODE_INT4_ONLY", "KV4_MODE_OUT_F32", "KV4_MODE_Q_ROTATED", "KV4_MODE_OUT_ROTATED",
+                 "KV4_MODE_ROPE_Q", "KV4_ROPE_NEOX", "KV4_ROPE_GPTJ", "KV4_DEV_ROPE_POS"):
+        m = re.search(r"\b%s\s*=\s*(\d+)" % name, text)
+        assert m is not None, name
+        assert getattr(kv4, name) == int(m.group(1)), name
