@@ -55,7 +55,7 @@ typedef struct CUstream_st* kv4_stream_t;
 enum {
   KV4_OK = 0,
   KV4_ERR_INVALID_ARG = -1,   /* a null pointer, a negative count, a misaligned pointer   */
-  KV4_ERR_UNSUPPORTED = -2,   /* a shape this build does not support (see kv4_config)     */
+  KV4_ERR_UNSUPPORTED = -2,   /* a shape the library does not support (see kv4_config)    */
   KV4_ERR_CAPACITY = -3,      /* a buffer smaller than kv4_cache_required_bytes()          */
   KV4_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed                      */
   KV4_ERR_DEVICE_FAULT = -5,  /* kv4_get_status() found device status bits set             */
