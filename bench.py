@@ -158,6 +158,7 @@ class ClockSampler:
                 pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
             smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
             self.nvml = (pynvml, h, smax, get_reasons)
+            self.ready.set()
             while not self.stop.is_set():
                 self.sample_now()
                 time.sleep(0.002)
@@ -165,13 +166,15 @@ class ClockSampler:
             pynvml.nvmlShutdown()
         except Exception as e:   # no NVML: reported as unavailable
             self.error = "%s: %s" % (type(e).__name__, e)
+        self.ready.set()
 
     def __enter__(self):
         import threading
         self.stop = threading.Event()
+        self.ready = threading.Event()
         self.thread = threading.Thread(target=self._run, daemon=True)
         self.thread.start()
-        time.sleep(0.05)
+        self.ready.wait(10.0)   # NVML is up (or known to be missing) before the timed region starts
         return self
 
     def __exit__(self, *a):

@@ -304,10 +304,12 @@ __global__ void __launch_bounds__(32 * QWARPS) gq_kernel(AttnParams p) {
 // the end; the attention kernel follows in stream order, so it sees the new
 // token and the new length.
 
-template <int D>
-__global__ void __launch_bounds__(32 * 32) gstep_kernel(AttnParams p, AppendParams ap) {
+// MAXW: the most warps a block of this instantiation has (2 * Hkv <= MAXW);
+// 16 for up to 8 KV heads (128 registers a thread), 32 for up to 16.
+template <int D, int MAXW>
+__global__ void __launch_bounds__(32 * MAXW) gstep_kernel(AttnParams p, AppendParams ap) {
   constexpr int VPL = D / 32;
-  __shared__ __align__(16) uint8_t s_codes[32][2][D];
+  __shared__ __align__(16) uint8_t s_codes[MAXW][2][D];
   __shared__ int s_seq, s_L, s_ok, s_page;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int tensor = warp >= p.Hkv ? 1 : 0, h = warp - tensor * p.Hkv;
@@ -909,7 +911,8 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   if (step) {
     // fused decode step: the append and the query operands first; the attention
     // kernel then starts in plain stream order (it plans from the new lengths)
-    gstep_kernel<D><<<p.n_seqs, 64 * p.Hkv, 0, stream>>>(p, *step);
+    if (p.Hkv <= 8) gstep_kernel<D, 16><<<p.n_seqs, 64 * p.Hkv, 0, stream>>>(p, *step);
+    else gstep_kernel<D, 32><<<p.n_seqs, 64 * p.Hkv, 0, stream>>>(p, *step);
     if (c->ev_before) cudaEventRecord(c->ev_before, stream);
   } else {
     if (c->ev_before) cudaEventRecord(c->ev_before, stream);
