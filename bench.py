@@ -1,23 +1,31 @@
 #!/usr/bin/env python
 """Decode-step benchmark of the paged INT4/INT8-protected KV cache on B200.
 
-One step = the whole hot path for one batch, through one library call
-(kv4_decode_step): fused rotate+quantize+append of one new token per sequence
-and the query operands in one kernel, then decode attention (one persistent
-stream-K kernel over the INT4 pages and the INT8 sink/recent store that plans
-its own split and stores the groups it covers whole; a merge kernel for the
-groups split over several CTAs).  --two-calls times the same step as
-kv4_rotate_quantize_append + kv4_decode_attention.  The metric is the algorithmic KV bytes the attention reads
-per step divided by the step time (GB/s), with decode tokens/s and the fraction
-of the measured HBM bandwidth beside it.
+The headline workload is the 36-layer decode stack of a Qwen3-8B-shaped model
+(36 independent layer caches, 256 sequences of 4096-16384 tokens, 32/8 heads,
+head dim 128).  One step is the whole hot path for one decode token of every
+sequence through all 36 layers: per layer one library call, kv4_decode_step
+(fused rotate+quantize+append of the new token and the query operands in one
+kernel, then the persistent stream-K attention kernel over the INT4 pages and
+the INT8 sink/recent store, and a merge kernel for the head groups split over
+several CTAs).  --two-calls times each layer as kv4_rotate_quantize_append +
+kv4_decode_attention.  The metric is the algorithmic KV bytes the attention
+reads per step divided by the step time (GB/s), with decode tokens/s and the
+fraction of the measured HBM bandwidth beside it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl kv4|reference]
+
+Beside the headline line it reports, on the same seeded inputs: the INT4-only
+(no protection) mode and the BF16-KV kernel (on as many layer caches as fit),
+and a `workloads` object with the single-layer workloads (64-sequence layer,
+512-sequence async-RL batch, 8 x 131072 long context), each with its own step
+throughput, roofline fraction and speedup over the BF16-KV kernel.
 
 Under torchrun each rank runs its own replica of the workload (independent
 sequences, weak scaling, no collective on the data path); the step time is the
 device time (CUDA events) summed over the K steps, maximum over ranks.
-`--impl reference` times the CPU oracle (tests-only restatement of the method)
-on a bounded sample of the same workload.
+`--impl reference` times the CPU oracle (the tests-only restatement of the
+method) on a bounded sample of the same workload, one sequence per host core.
 """
 
 import argparse
@@ -25,7 +33,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -39,24 +46,34 @@ import workloads  # noqa: E402
 METRIC = "decode-attention KV GB/s and tokens/s (INT4+INT8-protect), % of B200 HBM peak"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
+SUBLINES = ("qwen3_8b_layer", "async_rl", "long_context")
+BF16_MAX_LAYERS = 12          # distinct BF16 layer caches of the comparison leg on the stack (at most)
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=32)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="qwen3_8b_layer")
+    ap.add_argument("--workload", default="stack36")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="use only the first N layer caches of the workload (profiling a smaller case)")
     ap.add_argument("--impl", default="kv4", choices=["kv4", "reference"])
-    ap.add_argument("--no-compare", action="store_true", help="skip the BF16-KV and INT4-only legs")
+    ap.add_argument("--no-compare", action="store_true", help="skip the BF16-KV, INT4-only and multi-token legs")
+    ap.add_argument("--no-sublines", action="store_true", help="skip the single-layer workloads object")
+    ap.add_argument("--sub-steps", type=int, default=10, help="timed steps of each single-layer sub-line")
     ap.add_argument("--two-calls", action="store_true",
-                    help="run each step as kv4_rotate_quantize_append + kv4_decode_attention instead of kv4_decode_step")
+                    help="run each layer as kv4_rotate_quantize_append + kv4_decode_attention instead of "
+                         "kv4_decode_step")
     ap.add_argument("--rope", action="store_true",
                     help="fuse RoPE (neox, rotary dim = head dim, base 1e6) into the append and query kernels")
-    ap.add_argument("--cpu-seqs", type=int, default=4, help="sequences in the CPU oracle sample")
+    ap.add_argument("--cpu-procs", type=int, default=0,
+                    help="processes of the CPU oracle sample (0: one per host core)")
+    ap.add_argument("--cpu-steps", type=int, default=2, help="timed decode steps of the CPU oracle sample")
     ap.add_argument("--kernel-only", action="store_true",
-                    help="time the device steps only (no e2e leg, comparison legs or CPU baseline): for profilers")
-    return ap.parse_args()
+                    help="time the device steps only (no e2e leg, comparison legs, sub-lines or CPU baseline): "
+                         "for profilers")
+    return ap.parse_args(argv)
 
 
 # --------------------------------------------------------------------------- helpers
@@ -81,7 +98,7 @@ def measured_peaks():
         return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
 
 
-KERNEL_SOURCES = ("kv4_attention_grouped.cu", "kv4_attn_tiles.cuh", "kv4_common.cuh")
+KERNEL_SOURCES = ("kv4_attention_grouped.cu", "kv4_attn_tiles.cuh", "kv4_common.cuh", "kv4_append_ops.cuh")
 
 
 def kernel_source_hash():
@@ -210,55 +227,71 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- GPU workload
 
-class Workload:
-    """One replica: INT4 cache populated to L_b - 1 tokens, per-step new tokens and queries on the device."""
+class Replica:
+    """One replica of a workload on one GPU: a cache of `layers` layer caches, each populated to L_b - 1
+    tokens of every sequence, the new K/V of `extra` decode steps per layer and the queries of `n_q` steps
+    per layer (all on the device)."""
 
-    def __init__(self, w, device, extra_tokens, torch, rope=False):
+    def __init__(self, w, layers, device, extra, n_q, torch, rope=False):
         import int4_kv_cache_paged_b200 as kv4
         self.w = w
+        self.layers = layers
         self.device = device
         self.L = workloads.context_lengths(w)
         self.B = len(self.L)
-        table, num_pages, mpps = workloads.block_table(w, self.L, extra_tokens=extra_tokens)
+        table, num_pages, mpps = workloads.block_table(w, self.L, extra_tokens=extra)
         self.table = table
-        self.cfg = workloads.cache_config(w, num_pages, mpps)
+        self.cfg = workloads.cache_config(w, num_pages, mpps, layers=layers)
         self.cache = kv4.KV4Cache(self.cfg, torch.from_numpy(table), device)
         self.seq_ids = torch.arange(self.B, dtype=torch.int32, device=device)
         self.cu_one = torch.arange(self.B + 1, dtype=torch.int32, device=device)
-        self.steps_k = []  # per step: k [B, Hkv, D] bf16
-        self.steps_v = []
         self.rope = rope
         if rope:   # the model's angle table (an input), registered once
-            max_pos = int(np.max(self.L)) + extra_tokens + 1
+            max_pos = int(np.max(self.L)) + extra + 1
             self.cache.set_rope(torch.from_numpy(workloads.rope_cos_sin(max_pos, w["D"])), w["D"], kv4.KV4_ROPE_NEOX)
-        self.populate(torch, lambda *a, **k: self.cache.append(*a, rope=rope, **k), extra_tokens)
-
-    def populate(self, torch, append_fn, extra_tokens, layer=0, keep_steps=True):
-        w, dev = self.w, self.device
-        batch_k, batch_v, counts, ids = [], [], [], []
-        step_k = [[None] * self.B for _ in range(extra_tokens)]
-        step_v = [[None] * self.B for _ in range(extra_tokens)]
-        budget = 0
-        for s in range(self.B):
-            L = int(self.L[s])
-            k, v = workloads.kv_sequence(w, layer, s, L - 1 + extra_tokens, device=dev)
-            batch_k.append(k[:L - 1])
-            batch_v.append(v[:L - 1])
-            counts.append(L - 1)
-            ids.append(s)
-            for j in range(extra_tokens):
-                step_k[j][s] = k[L - 1 + j]
-                step_v[j][s] = v[L - 1 + j]
-            budget += L
-            if budget > 2_000_000 or s == self.B - 1:
-                cu = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int32, device=dev)
-                append_fn(layer, torch.tensor(ids, dtype=torch.int32, device=dev), cu,
-                          torch.cat(batch_k).contiguous(), torch.cat(batch_v).contiguous(), total_new=int(sum(counts)))
-                batch_k, batch_v, counts, ids, budget = [], [], [], [], 0
-        if keep_steps:
-            self.steps_k = [torch.stack(x).contiguous() for x in step_k]
-            self.steps_v = [torch.stack(x).contiguous() for x in step_v]
+        self.steps_k, self.steps_v = [], []   # per layer: [extra, B, Hkv, D] bf16
+        for layer in range(layers):
+            k, v = populate(torch, w, self.L, lambda *a, **kw: self.cache.append(*a, rope=rope, **kw), layer,
+                            extra, device)
+            self.steps_k.append(k)
+            self.steps_v.append(v)
+        # queries per (layer, step), drawn once (outside every timed region)
+        self.qs = [torch.stack([workloads.queries(w, layer, i, device=device) for i in range(n_q)])
+                   for layer in range(layers)]
         torch.cuda.synchronize()
+
+    def bytes_at(self, tokens_appended, int4_only=False):
+        """Algorithmic KV bytes of one attention call of one layer after `tokens_appended` decode appends."""
+        w = self.w
+        return kv_bytes(self.L - 1 + tokens_appended, w["Hkv"], w["D"], w["S"], w["W"], int4_only)
+
+
+def populate(torch, w, L, append_fn, layer, extra, device, upto=0, budget_tokens=1_000_000):
+    """Append the seeded tokens 0 .. L_b - 2 + upto of every sequence to `layer` (batched calls); return the
+    tokens L_b - 1 + upto .. L_b - 2 + extra of every sequence as [extra - upto, B, Hkv, D] K and V tensors.
+    Each sequence is drawn with length L_b - 1 + extra whatever `upto` is, so the same (L, extra) gives the
+    same token values (the generator draws V after all of K)."""
+    B = len(L)
+    batch_k, batch_v, counts, ids = [], [], [], []
+    step_k = torch.empty((extra - upto, B, w["Hkv"], w["D"]), dtype=torch.bfloat16, device=device)
+    step_v = torch.empty_like(step_k)
+    budget = 0
+    for s in range(B):
+        n = int(L[s]) - 1 + upto
+        k, v = workloads.kv_sequence(w, layer, s, int(L[s]) - 1 + extra, device=device)
+        batch_k.append(k[:n])
+        batch_v.append(v[:n])
+        counts.append(n)
+        ids.append(s)
+        step_k[:, s] = k[n:]
+        step_v[:, s] = v[n:]
+        budget += n
+        if budget > budget_tokens or s == B - 1:
+            cu = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int32, device=device)
+            append_fn(layer, torch.tensor(ids, dtype=torch.int32, device=device), cu,
+                      torch.cat(batch_k).contiguous(), torch.cat(batch_v).contiguous(), total_new=int(sum(counts)))
+            batch_k, batch_v, counts, ids, budget = [], [], [], [], 0
+    return step_k, step_v
 
 
 def reduce_over_ranks(times, counts, device, world):
@@ -278,6 +311,318 @@ def reduce_over_ranks(times, counts, device, world):
     return t.tolist(), c.tolist()
 
 
+def measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=1, compare=True):
+    """Build a replica of workload `w` (its first `layers` layer caches) and time it.
+
+    Returns the per-rank raw figures (step time, bytes, kernel time, e2e) and the rank-local comparison
+    legs.  The collective steps (barriers) are the same on every rank."""
+    import torch.distributed as dist
+    B, Hkv, D, S, Wn, Hq = w["batch"], w["Hkv"], w["D"], w["S"], w["W"], w["Hq"]
+    two, rope = args.two_calls, args.rope
+    amode = kv4.KV4_MODE_ROPE_Q if rope else 0
+    K_e2e = 0 if args.kernel_only else K
+    do_cmp = compare and not args.kernel_only and not rope and world == 1
+    n_cmp = 2 * K if do_cmp else 0              # the step as two calls and as one call
+    extra = W_ + 2 * K + K_e2e + n_cmp + 1       # timed loop, kernel-event pass, e2e, comparison steps
+    t0 = time.time()
+    rep = Replica(w, layers, device, extra, W_ + K, torch, rope=rope)
+    rep.extra = extra
+    setup_s = time.time() - t0
+    cache = rep.cache
+    ws = cache.workspace(B)
+    out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def layer_step(layer, i, qi, o=out):
+        """Decode step of layer `layer` on the i-th new token of every sequence (one call, or the two)."""
+        if two:
+            cache.append(layer, rep.seq_ids, rep.cu_one, rep.steps_k[layer][i], rep.steps_v[layer][i], total_new=B,
+                         rope=rope)
+            cache.attention(layer, rep.seq_ids, rep.qs[layer][qi], out=o, workspace=ws, mode=amode)
+        else:
+            cache.decode_step(layer, rep.seq_ids, rep.steps_k[layer][i], rep.steps_v[layer][i], rep.qs[layer][qi],
+                              out=o, workspace=ws, mode=amode)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- the timed loop: W_ warm-up steps, then K steps, each through every layer
+    n = W_ + K
+    e_step = [(ev(), ev()) for _ in range(n)]
+    barrier()
+    for i in range(n):
+        if i == W_:
+            barrier()
+            t_window = time.perf_counter()
+        flush.fill_(i & 0xFF)                   # evict the previous step's KV from L2 (outside the events)
+        e_step[i][0].record(stream)
+        for layer in range(layers):
+            layer_step(layer, i, i)
+        e_step[i][1].record(stream)
+    clocks.sample_now(4, 0.0003)                # while the queued steps run
+    barrier()
+    clocks.window(t_window, time.perf_counter())
+    t_step = sum(e_step[i][0].elapsed_time(e_step[i][1]) for i in range(W_, n)) / 1e3
+    bytes_timed = sum(rep.bytes_at(i + 1) * layers for i in range(W_, n))
+
+    # ---- the same steps on the next K tokens with the library's events around every layer's attention and
+    # merge kernels (the roofline's kernel time); kept out of the loop above because an event marker between
+    # two launches adds about 2 us to a layer
+    e_kern = [[(ev(), ev()) for _ in range(layers)] for _ in range(K)]
+    t_window = time.perf_counter()
+    for j in range(K):
+        flush.fill_(j & 0xFF)
+        for layer in range(layers):
+            kv4.kv4_set_attention_events(cache.handle, *e_kern[j][layer])
+            layer_step(layer, n + j, W_ + j)
+    clocks.sample_now(4, 0.0003)
+    barrier()
+    clocks.window(t_window, time.perf_counter())
+    kv4.kv4_set_attention_events(cache.handle, None, None)
+    t_kern = sum(a.elapsed_time(b) for row in e_kern for a, b in row) / 1e3
+    bytes_kern = sum(rep.bytes_at(n + j + 1) * layers for j in range(K))
+    used = n + K                                 # new tokens used so far
+
+    # ---- e2e through the public API with host buffers: each step copies every layer's new K, V and q from
+    # pinned host memory (one transfer per layer, on a copy stream, ahead of the layer that reads it) and every
+    # layer's output back to pinned host memory (on a second copy stream, behind the layer that writes it)
+    e2e = None
+    if K_e2e:
+        kv_el, q_el = B * Hkv * D, B * Hq * D
+        per = 2 * kv_el + q_el
+        hin = torch.empty((K_e2e, layers, per), dtype=torch.bfloat16).pin_memory()
+        for j in range(K_e2e):
+            for layer in range(layers):
+                hin[j, layer, :kv_el].copy_(rep.steps_k[layer][used + j].reshape(-1))
+                hin[j, layer, kv_el:2 * kv_el].copy_(rep.steps_v[layer][used + j].reshape(-1))
+                hin[j, layer, 2 * kv_el:].copy_(rep.qs[layer][j % (W_ + K)].reshape(-1))
+        hout = torch.empty((K_e2e, layers, B, Hq, D), dtype=torch.bfloat16).pin_memory()
+        din = torch.empty((layers, per), dtype=torch.bfloat16, device=device)
+        dout = torch.empty((layers, B, Hq, D), dtype=torch.bfloat16, device=device)
+        h2d, d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        ready = [torch.cuda.Event() for _ in range(layers)]
+        consumed = [torch.cuda.Event() for _ in range(layers)]
+        written = [torch.cuda.Event() for _ in range(layers)]
+        drained = [torch.cuda.Event() for _ in range(layers)]
+        e0, e1 = ev(), ev()
+        barrier()
+        e0.record(stream)
+        h2d.wait_event(e0)
+        d2h.wait_event(e0)
+        for j in range(K_e2e):
+            for layer in range(layers):
+                with torch.cuda.stream(h2d):
+                    if j:
+                        h2d.wait_event(consumed[layer])      # the previous step's layer has read din[layer]
+                    din[layer].copy_(hin[j, layer], non_blocking=True)
+                    ready[layer].record(h2d)
+            for layer in range(layers):
+                stream.wait_event(ready[layer])
+                if j:
+                    stream.wait_event(drained[layer])        # the previous output of this layer is on the host
+                dk = din[layer, :kv_el].view(B, Hkv, D)
+                dv = din[layer, kv_el:2 * kv_el].view(B, Hkv, D)
+                dq = din[layer, 2 * kv_el:].view(B, Hq, D)
+                if two:
+                    cache.append(layer, rep.seq_ids, rep.cu_one, dk, dv, total_new=B, rope=rope)
+                    cache.attention(layer, rep.seq_ids, dq, out=dout[layer], workspace=ws, mode=amode)
+                else:
+                    cache.decode_step(layer, rep.seq_ids, dk, dv, dq, out=dout[layer], workspace=ws, mode=amode)
+                consumed[layer].record(stream)
+                written[layer].record(stream)
+                with torch.cuda.stream(d2h):
+                    d2h.wait_event(written[layer])
+                    hout[j, layer].copy_(dout[layer], non_blocking=True)
+                    drained[layer].record(d2h)
+        for layer in range(layers):
+            stream.wait_event(drained[layer])
+        e1.record(stream)
+        barrier()
+        t_e2e = e0.elapsed_time(e1) / 1e3
+        e2e_bytes = sum(rep.bytes_at(used + j + 1) * layers for j in range(K_e2e))
+        e2e = {"t": t_e2e, "bytes": e2e_bytes, "steps": K_e2e, "h2d_bytes_per_step": int(layers * per * 2),
+               "d2h_bytes_per_step": int(layers * B * Hq * D * 2)}
+        used += K_e2e
+        del hin, hout, din, dout
+
+    res = {"rep": rep, "setup_s": setup_s, "t_step": t_step, "bytes_timed": bytes_timed, "t_kern": t_kern,
+           "bytes_kern": bytes_kern, "e2e": e2e, "status": cache.status(), "used": used, "ws": ws, "out": out,
+           "flush": flush}
+    if do_cmp:
+        res["compare"] = compare_int4_legs(torch, kv4, res, K)
+    return res
+
+
+def time_passes(torch, fn, K, layers, flush, q_of):
+    """Attention-only passes over `layers` layers: 3 warm-up passes, then K passes with one event pair per
+    layer call.  Returns the mean time of one call of each layer (s)."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    for i in range(3):
+        for layer in range(layers):
+            fn(layer, q_of(layer, i))
+    torch.cuda.synchronize()
+    es = [[(ev(), ev()) for _ in range(layers)] for _ in range(K)]
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        for layer in range(layers):
+            es[i][layer][0].record()
+            fn(layer, q_of(layer, i))
+            es[i][layer][1].record()
+    torch.cuda.synchronize()
+    return [sum(es[i][layer][0].elapsed_time(es[i][layer][1]) for i in range(K)) / 1e3 / K for layer in range(layers)]
+
+
+def compare_int4_legs(torch, kv4, res, K):
+    """On the INT4 cache of `res`: the step as two calls against one call, attention alone in the protected and
+    the INT4-only modes, and multi-token queries (attention-only figures are per layer call, summed over the
+    layers)."""
+    rep, ws, out, flush = res["rep"], res["ws"], res["out"], res["flush"]
+    w, cache, layers, B = rep.w, rep.cache, rep.layers, rep.B
+    Hkv, D = w["Hkv"], w["D"]
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    nq = rep.qs[0].shape[0]
+
+    def time_steps(fn, t0):
+        es = [(ev(), ev()) for _ in range(K)]
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            es[i][0].record()
+            for layer in range(layers):
+                fn(layer, t0 + i, i % nq)
+            es[i][1].record()
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in es) / 1e3 / K
+
+    def two_calls(layer, i, qi):
+        cache.append(layer, rep.seq_ids, rep.cu_one, rep.steps_k[layer][i], rep.steps_v[layer][i], total_new=B)
+        cache.attention(layer, rep.seq_ids, rep.qs[layer][qi], out=out, workspace=ws)
+
+    def one_call(layer, i, qi):
+        cache.decode_step(layer, rep.seq_ids, rep.steps_k[layer][i], rep.steps_v[layer][i], rep.qs[layer][qi],
+                          out=out, workspace=ws)
+
+    used = res["used"]
+    t_two = time_steps(two_calls, used)
+    t_one = time_steps(one_call, used + K)
+    used += 2 * K
+    res["used"] = used
+    q_of = lambda layer, i: rep.qs[layer][i % nq]  # noqa: E731
+    per_int4 = time_passes(torch, lambda l, q: cache.attention(l, rep.seq_ids, q, out=out, workspace=ws), K, layers,
+                           flush, q_of)
+    per_only = time_passes(torch, lambda l, q: cache.attention(l, rep.seq_ids, q, out=out, workspace=ws,
+                                                              mode=kv4.KV4_MODE_INT4_ONLY), K, layers, flush, q_of)
+    b_prot, b_only = rep.bytes_at(used), rep.bytes_at(used, int4_only=True)
+    t_int4, t_only = sum(per_int4), sum(per_only)
+    cmp = {"step_as_two_calls": {"ms_per_step": round(t_two * 1e3, 4)},
+           "step_as_one_call": {"ms_per_step": round(t_one * 1e3, 4)},
+           "int4_protected": {"attention_ms": round(t_int4 * 1e3, 4), "layers": layers,
+                              "kv_gbs": round(b_prot * layers / t_int4 / 1e9, 1)},
+           "int4_only": {"attention_ms": round(t_only * 1e3, 4), "layers": layers,
+                         "kv_gbs": round(b_only * layers / t_only / 1e9, 1)}}
+    # multi-token query (speculative verification): the most query tokens whose heads fit one 8-column operand
+    T = 8 // (w["Hq"] // Hkv)
+    if T >= 2:
+        gen = torch.Generator(device=rep.device).manual_seed(4242)
+        qx = [torch.randn((B, T, w["Hq"], D), generator=gen, device=rep.device).to(torch.bfloat16) for _ in range(3)]
+        outx = torch.empty((B, T, w["Hq"], D), dtype=torch.bfloat16, device=rep.device)
+        wsx = cache.extend_workspace(B, T)
+        per_ext = time_passes(torch, lambda l, q: cache.extend_attention(l, rep.seq_ids, q, out=outx, workspace=wsx),
+                              K, layers, flush, lambda layer, i: qx[i % 3])
+        t_ext = sum(per_ext)
+        cmp["extend"] = {"q_len": T, "attention_ms": round(t_ext * 1e3, 4),
+                         "kv_gbs": round(b_prot * layers / t_ext / 1e9, 1),
+                         "query_tokens_per_s": round(B * T * layers / t_ext, 1)}
+        del outx, wsx
+    res["per_layer_int4_s"] = per_int4
+    return cmp
+
+
+def bf16_leg(torch, kv4, w, L, extra, used, layers_avail, per_layer_int4, K, device, flush):
+    """The BF16-KV kernel on the same seeded tokens as the INT4 cache (positions 0 .. L_b - 2 + used of every
+    sequence, drawn as the INT4 replica drew them), on as many of the first layers as fit in the free device
+    memory (at most BF16_MAX_LAYERS); compared with the INT4 attention time of the same layers."""
+    L_now = L - 1 + used
+    need_layer = bf16_bytes(L_now, w["Hkv"], w["D"]) * 1.06
+    free = torch.cuda.mem_get_info(device)[0]
+    n = int(min(layers_avail, BF16_MAX_LAYERS, (free * 0.9 - 4e9) // need_layer))
+    if n < 1:
+        return {"skipped": "a BF16 layer cache of %.1f GB does not fit (%.1f GB free)" % (need_layer / 1e9, free / 1e9)}
+    B = len(L_now)
+    table, num_pages, mpps = workloads.block_table(w, L_now + 1, extra_tokens=0)
+    cfg = workloads.cache_config(w, num_pages, mpps, layers=n)
+    cache16 = kv4.BF16Cache(cfg, torch.from_numpy(table), device)
+    for layer in range(n):   # identical tokens: the same per-(layer, sequence) streams up to the current length
+        populate(torch, w, L, cache16.append, layer, extra, device, upto=used)
+    ids = torch.arange(B, dtype=torch.int32, device=device)
+    ws16 = cache16.workspace(B)
+    out = torch.empty((B, w["Hq"], w["D"]), dtype=torch.bfloat16, device=device)
+    qs = [workloads.queries(w, 0, 5000 + i, device=device) for i in range(3)]
+    per = time_passes(torch, lambda l, q: cache16.attention(l, ids, q, out=out, workspace=ws16), K, n, flush,
+                      lambda layer, i: qs[i % 3])
+    t16, t4 = sum(per), sum(per_layer_int4[:n])
+    b16 = bf16_bytes(L_now, w["Hkv"], w["D"]) * n
+    res = {"attention_ms": round(t16 * 1e3, 4), "layers": n, "kv_gbs": round(b16 / t16 / 1e9, 1),
+           "int4_protected_attention_ms_same_layers": round(t4 * 1e3, 4),
+           "speedup_int4_protected_vs_bf16": round(t16 / t4, 3)}
+    if n < layers_avail:
+        res["note"] = ("%d of %d layer caches: the BF16 caches of all layers (%.0f GB) do not fit in HBM; the "
+                       "INT4 time is that of the same %d layers" % (n, layers_avail, need_layer * layers_avail / 1e9, n, n))
+    cache16.close()
+    del cache16, ws16, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def roofline_obj(achieved, hbm, peak_kind, traffic, bytes_per_launch, layers):
+    return {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "traffic": traffic,
+            "kernel": "gattn_kernel: persistent stream-K attention over the INT4 pages and the INT8 store (the "
+                      "events span it and the merge kernel, its programmatic dependent; with --two-calls also the "
+                      "query-operand kernel before it)",
+            "peak_source": peak_kind, "bytes_per_launch": int(bytes_per_launch),
+            "launches_per_step": layers,
+            "timing": "CUDA events recorded by the library around the kernels of every layer, over K steps that "
+                      "follow the timed loop on the same workload"}
+
+
+def sub_line(torch, kv4, name, args, device, clocks, hbm, peak_kind):
+    """A single-layer workload: its step throughput, roofline fraction, INT4-only and BF16 comparisons."""
+    w = workloads.workload(name)
+    K = max(3, min(args.sub_steps, args.steps))
+    r = measure(torch, kv4, w, 1, args, K, 3, device, clocks)
+    rep = r["rep"]
+    value = r["bytes_timed"] / r["t_step"] / 1e9
+    achieved = r["bytes_kern"] / r["t_kern"] / 1e9
+    line = {"value": round(value, 2), "unit": "GB/s", "ms_per_step": round(r["t_step"] / K * 1e3, 4),
+            "tokens_per_s": round(rep.B * K / r["t_step"], 1), "steps": K,
+            "config": {"batch": rep.B, "context": "%s" % (w["ctx"][0],), "page": w["P"], "recent_window": w["W"],
+                       "kv_bytes_per_step_mb": round(r["bytes_timed"] / K / 1e6, 1)},
+            "roofline": roofline_obj(achieved, hbm, peak_kind, profiled_traffic(name), r["bytes_kern"] / K, 1),
+            "device_status": r["status"]}
+    if r["e2e"]:
+        e = r["e2e"]
+        line["e2e"] = {"value": round(e["bytes"] / e["t"] / 1e9, 2), "unit": "GB/s",
+                       "h2d_bytes_per_step": e["h2d_bytes_per_step"], "d2h_bytes_per_step": e["d2h_bytes_per_step"]}
+    cmp = r.get("compare")
+    if cmp:
+        line["compare"] = cmp
+        L0, extra, used = rep.L, rep.extra, r["used"]
+        per = r["per_layer_int4_s"]
+        flush = r["flush"]
+        rep.cache.close()
+        del r, rep
+        torch.cuda.empty_cache()
+        b16 = bf16_leg(torch, kv4, w, L0, extra, used, 1, per, K, device, flush)
+        line["compare"]["bf16_kv"] = b16
+        if "speedup_int4_protected_vs_bf16" in b16:
+            line["speedup_int4_protected_vs_bf16"] = b16["speedup_int4_protected_vs_bf16"]
+    return line
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -290,317 +635,187 @@ def run_gpu(args):
     device = torch.device("cuda", local)
     if world > 1:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=device)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=900), device_id=device)
 
     W_, K = args.warmup, args.steps
     w = workloads.workload(args.workload)
     if rank > 0:
         w = workloads.workload(args.workload, seed=w["seed"] + 7919 * rank)   # independent sequences per rank
-    if w["layers"] > 1:
-        raise SystemExit("the benchmark times single-layer workloads; use the stack test for %s" % args.workload)
-    extra = W_ + 5 * K + 1   # warm-up + timed steps, the kernel-event pass, e2e, two comparison legs
-    t0 = time.time()
-    wl = Workload(w, device, extra, torch, rope=args.rope)
-    amode = kv4.KV4_MODE_ROPE_Q if args.rope else 0
-    setup_s = time.time() - t0
-    B, Hkv, D, S, Wn = wl.B, w["Hkv"], w["D"], w["S"], w["W"]
-    ws = wl.cache.workspace(B)
-    out = torch.empty((B, w["Hq"], D), dtype=torch.bfloat16, device=device)
-    qs = [workloads.queries(w, 0, i, device=device) for i in range(W_ + K)]
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-    stream = torch.cuda.current_stream()
+    layers = w["layers"] if args.layers <= 0 else min(args.layers, w["layers"])
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
 
-    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    n = W_ + K
-    e_step = [(ev(), ev()) for _ in range(n)]
-    e_kern = [(ev(), ev()) for _ in range(K)]
-    step_bytes, kern_bytes = [], []
-
-    def one_step(i, q):
-        """The decode step on token i of every sequence: one library call (or the two calls)."""
-        if args.two_calls:
-            wl.cache.append(0, wl.seq_ids, wl.cu_one, wl.steps_k[i], wl.steps_v[i], total_new=B, rope=args.rope)
-            wl.cache.attention(0, wl.seq_ids, q, out=out, workspace=ws, mode=amode)
-        else:   # append + query operands, then the attention and merge kernels
-            wl.cache.decode_step(0, wl.seq_ids, wl.steps_k[i], wl.steps_v[i], q, out=out, workspace=ws, mode=amode)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    barrier()
     with ClockSampler(device) as clocks:
-        for i in range(n):
-            if i == W_:
-                barrier()
-                t_window = time.perf_counter()
-            flush.fill_(i & 0xFF)                  # evict the KV of the previous step from L2 (not timed)
-            e_step[i][0].record(stream)
-            one_step(i, qs[i])
-            e_step[i][1].record(stream)
-            step_bytes.append(kv_bytes(wl.L + i, Hkv, D, S, Wn))
-        clocks.sample_now(4, 0.0003)                # while the queued steps run
-        barrier()
-        clocks.window(t_window, time.perf_counter())
-        # the same steps again on the next K tokens, now with the library's events around the attention
-        # kernel and its merge kernel (with --two-calls also the query-operand kernel): they give the
-        # roofline's kernel time.  They are kept out of the loop above because each event marker between
-        # two launches adds about 2 us to the step.
-        t_window = time.perf_counter()
-        for j in range(K):
-            flush.fill_(j & 0xFF)
-            kv4.kv4_set_attention_events(wl.cache.handle, *e_kern[j])
-            one_step(n + j, qs[W_ + j])
-            kern_bytes.append(kv_bytes(wl.L + n + j, Hkv, D, S, Wn))
-        clocks.sample_now(4, 0.0003)
-        barrier()
-        clocks.window(t_window, time.perf_counter())
-    kv4.kv4_set_attention_events(wl.cache.handle, None, None)
-    status = wl.cache.status()
-
-    timed = range(W_, n)
-    t_step = sum(e_step[i][0].elapsed_time(e_step[i][1]) for i in timed) / 1e3
-    t_kern = sum(a.elapsed_time(b) for a, b in e_kern) / 1e3
-    t_attn = t_kern
-    bytes_timed = sum(step_bytes[i] for i in timed)
-    bytes_kern = sum(kern_bytes)
-    n += K                                          # tokens used so far
-
-    # ---- e2e through the public API with host buffers (pinned), copies inside the timed region
-    if args.kernel_only:
-        K_e2e = 0
-    else:
-        K_e2e = K
-    # each step's inputs (new K, new V, q) packed in one pinned host buffer: one host->device copy per step
-    kv_elems, q_elems = wl.steps_k[0].numel(), qs[0].numel()
-    hin = []
-    for j in range(K_e2e):
-        h = torch.empty(2 * kv_elems + q_elems, dtype=torch.bfloat16).pin_memory()
-        h[:kv_elems].copy_(wl.steps_k[n + j].reshape(-1).cpu())
-        h[kv_elems:2 * kv_elems].copy_(wl.steps_v[n + j].reshape(-1).cpu())
-        h[2 * kv_elems:].copy_(workloads.queries(w, 0, n + j, device="cpu").reshape(-1))
-        hin.append(h)
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    din = torch.empty(2 * kv_elems + q_elems, dtype=torch.bfloat16, device=device)
-    dk = din[:kv_elems].view(wl.steps_k[0].shape)
-    dv = din[kv_elems:2 * kv_elems].view(wl.steps_v[0].shape)
-    dq = din[2 * kv_elems:].view(qs[0].shape)
-    e_e2e = [(ev(), ev()) for _ in range(K_e2e)]
-    e2e_bytes = 0
-    barrier()
-    for j in range(K_e2e):
-        flush.fill_(j & 0xFF)
-        e_e2e[j][0].record(stream)
-        din.copy_(hin[j], non_blocking=True)
-        if args.two_calls:
-            wl.cache.append(0, wl.seq_ids, wl.cu_one, dk, dv, total_new=B, rope=args.rope)
-            wl.cache.attention(0, wl.seq_ids, dq, out=out, workspace=ws, mode=amode)
-        else:
-            wl.cache.decode_step(0, wl.seq_ids, dk, dv, dq, out=out, workspace=ws, mode=amode)
-        hout.copy_(out, non_blocking=True)
-        e_e2e[j][1].record(stream)
-        e2e_bytes += kv_bytes(wl.L + n + j, Hkv, D, S, Wn)
-    barrier()
-    t_e2e = sum(a.elapsed_time(b) for a, b in e_e2e) / 1e3 if K_e2e else float("nan")
-    h2d = dk.numel() * 2 + dv.numel() * 2 + dq.numel() * 2
-    d2h = hout.numel() * 2
-
-    # ---- comparison legs on identical inputs (rank-local, untimed by the contract)
-    compare = None
-    if not args.no_compare and not args.kernel_only and not args.rope and world == 1:
-        compare = compare_legs(torch, kv4, w, wl, K, device, flush, n + K_e2e)
-
-    (t_step_all, t_e2e_all), (bytes_all, e2e_bytes_all) = reduce_over_ranks(
-        [t_step, t_e2e], [float(bytes_timed), float(e2e_bytes)], device, world)
-
-    result = None
-    if rank == 0:
-        peaks, peak_kind = measured_peaks()
-        hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
-        achieved = bytes_kern / t_kern / 1e9
-        value = bytes_all / t_step_all / 1e9
-        traffic = profiled_traffic(args.workload)
+        r = measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=world, compare=True)
+        rep = r["rep"]
+        e2e = r["e2e"]
+        t_e2e = e2e["t"] if e2e else float("nan")
+        e2e_bytes = e2e["bytes"] if e2e else 0.0
+        (t_step_all, t_e2e_all), (bytes_all, e2e_bytes_all) = reduce_over_ranks(
+            [r["t_step"], t_e2e], [float(r["bytes_timed"]), float(e2e_bytes)], device, world)
         clk = clocks.summary()
-        result = {
-            "metric": METRIC,
-            "value": round(value, 2),
-            "unit": "GB/s",
-            "n_gpus": world,
-            "steps": K,
-            "warmup": W_,
-            "ms_per_step": round(t_step_all / K * 1e3, 4),
-            "higher_is_better": True,
-            "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "int4/int8 codes, fp16 scales, bf16 q/out, fp16 tensor-core operands, fp32 accumulate",
-            "data": "synthetic (seeded N(0,1) K/V with outlier K channels and a large-norm sink, bf16)",
-            "config": {"workload": args.workload, "batch": B, "q_heads": w["Hq"], "kv_heads": Hkv, "head_dim": D,
-                       "page": w["P"], "hadamard_block": w["Bh"], "sinks": S, "recent_window": Wn,
-                       "context": "%s, mean %.0f at the first timed step" % (w["ctx"][0], float(np.mean(wl.L + W_))),
-                       "kv_bytes_per_step_mb": round(bytes_timed / K / 1e6, 1),
-                       "l2": "flushed before every step by a 256 MB write outside the timed events; "
-                             "per-step KV also exceeds the 126 MB L2",
-                       "parallelism": "replica per GPU" if world > 1 else "single GPU",
-                       "rope": ("neox, rotary dim %d, base 1e6, fused into the append and query kernels" % D
-                                if args.rope else "none (keys arrive post-RoPE)")},
-            "tokens_per_s": round(B * world * K / t_step_all, 1),
-            "hbm_frac_of_%s" % peak_kind: round(value / hbm, 4),
-            "attention_kv_gbs": round(bytes_kern / t_attn / 1e9, 2),
-            "api": "two calls: kv4_rotate_quantize_append + kv4_decode_attention" if args.two_calls else
-                   "one call: kv4_decode_step",
-            ("append_us_per_step" if args.two_calls else "append_and_query_us_per_step"):
-                round((t_step - t_attn) / K * 1e6, 2),
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
-                         "frac": round(achieved / hbm, 4), "traffic": traffic,
-                         "kernel": "gattn_kernel: persistent stream-K attention over the INT4 pages and the "
-                                   "INT8 store (the events span it and the merge kernel, its programmatic "
-                                   "dependent; with --two-calls also the query-operand kernel before it)",
-                         "peak_source": peak_kind, "bytes_per_launch": int(bytes_kern / K),
-                         "timing": "CUDA events recorded by the library around the kernels, over K steps that "
-                                   "follow the timed loop on the same workload"},
-            "e2e": ({"value": round(e2e_bytes_all / t_e2e_all / 1e9, 2), "unit": "GB/s",
-                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                     "tokens_per_s": round(B * world * K / t_e2e_all, 1)} if K_e2e else None),
-            # per step: gstep_kernel, gattn_kernel, gmerge_kernel (two calls: append_kernel, gq_kernel, gattn, gmerge)
-            "gpu_launches": (4 if args.two_calls else 3) * K,
-            "clocks": clk,
-            "device_status": status,
-            "setup_s": round(setup_s, 1),
-        }
-        if compare:
-            result["compare"] = compare
+        result = None
+        if rank == 0:
+            B = rep.B
+            achieved = r["bytes_kern"] / r["t_kern"] / 1e9
+            value = bytes_all / t_step_all / 1e9
+            launches = (4 if args.two_calls else 3) * layers
+            result = {
+                "metric": METRIC,
+                "value": round(value, 2),
+                "unit": "GB/s",
+                "n_gpus": world,
+                "steps": K,
+                "warmup": W_,
+                "ms_per_step": round(t_step_all / K * 1e3, 4),
+                "higher_is_better": True,
+                "scaling": "weak",
+                "vs_baseline": None,
+                "dtype": "int4/int8 codes, fp16 scales, bf16 q/out, int8 and fp16 tensor-core operands, "
+                         "fp32 accumulate",
+                "data": "synthetic (seeded N(0,1) K/V with outlier K channels and a large-norm sink, bf16)",
+                "config": {"workload": args.workload, "layers": layers, "batch": B, "q_heads": w["Hq"],
+                           "kv_heads": w["Hkv"], "head_dim": w["D"], "page": w["P"], "hadamard_block": w["Bh"],
+                           "sinks": w["S"], "recent_window": w["W"],
+                           "context": "%s, mean %.0f at the first timed step" % (w["ctx"][0], float(np.mean(rep.L + W_))),
+                           "step": "%d layers x one %s call (append one token per sequence, then attention)"
+                                   % (layers, "two-call" if args.two_calls else "kv4_decode_step"),
+                           "kv_bytes_per_step_mb": round(r["bytes_timed"] / K / 1e6, 1),
+                           "l2": "flushed before every step by a 256 MB write outside the timed events; each "
+                                 "layer's KV also exceeds the 126 MB L2",
+                           "parallelism": "replica per GPU" if world > 1 else "single GPU",
+                           "rope": ("neox, rotary dim %d, base 1e6, fused into the append and query kernels" % w["D"]
+                                    if args.rope else "none (keys arrive post-RoPE)")},
+                "tokens_per_s": round(B * world * K / t_step_all, 1),
+                "hbm_frac_of_%s" % peak_kind: round(value / hbm, 4),
+                "attention_kv_gbs": round(achieved, 2),
+                "api": ("two calls per layer: kv4_rotate_quantize_append + kv4_decode_attention" if args.two_calls
+                        else "one call per layer: kv4_decode_step"),
+                # step time outside the attention and merge kernels, all layers (append + query operands)
+                ("append_us_per_step" if args.two_calls else "append_and_query_us_per_step"):
+                    round(max(r["t_step"] - r["t_kern"], 0.0) / K * 1e6, 2),
+                "roofline": roofline_obj(achieved, hbm, peak_kind, profiled_traffic(args.workload),
+                                         r["bytes_kern"] / (K * layers), layers),
+                "e2e": ({"value": round(e2e_bytes_all / t_e2e_all / 1e9, 2), "unit": "GB/s",
+                         "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                         "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
+                         "tokens_per_s": round(B * world * e2e["steps"] / t_e2e_all, 1),
+                         "ms_per_step": round(t_e2e_all / e2e["steps"] * 1e3, 4),
+                         "how": "per layer: new K, V and q copied from pinned host memory on a copy stream ahead "
+                                "of the layer, the layer's output copied to pinned host memory on a second copy "
+                                "stream behind it; one CUDA-event pair around all steps"} if e2e else None),
+                # per layer: gstep_kernel, gattn_kernel, gmerge_kernel (two calls: append, gq, gattn, gmerge)
+                "gpu_launches": launches * K,
+                "clocks": clk,
+                "device_status": r["status"],
+                "setup_s": round(r["setup_s"], 1),
+            }
+            if "compare" in r:
+                result["compare"] = r["compare"]
+        cmp_ok = "compare" in r
+        L0, extra, used = rep.L, rep.extra, r["used"]
+        per = r.get("per_layer_int4_s")
+        flush = r["flush"]
+        rep.cache.close()
+        del r, rep
+        torch.cuda.empty_cache()
+        if rank == 0 and cmp_ok:
+            result["compare"]["bf16_kv"] = bf16_leg(torch, kv4, w, L0, extra, used, layers, per, K, device, flush)
+        if (rank == 0 and world == 1 and not args.kernel_only and not args.no_sublines and not args.rope
+                and args.workload not in SUBLINES):
+            subs = {}
+            for name in SUBLINES:
+                subs[name] = sub_line(torch, kv4, name, args, device, clocks, hbm, peak_kind)
+                torch.cuda.empty_cache()
+            result["workloads"] = subs
+        del flush
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return result
 
 
-def compare_legs(torch, kv4, w, wl, K, device, flush, first_token):
-    """Attention-only time of the INT4 path, the INT4-only mode, the multi-token query path and the BF16-KV
-    kernel on identical inputs."""
-    B, Hkv, D, S, Wn = wl.B, w["Hkv"], w["D"], w["S"], w["W"]
-    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    qs = [workloads.queries(w, 0, 1000 + i, device=device) for i in range(K)]
-    out = torch.empty((B, w["Hq"], D), dtype=torch.bfloat16, device=device)
-
-    def time_attn(fn):
-        es = [(ev(), ev()) for _ in range(K)]
-        for i in range(3):
-            fn(qs[i])
-        torch.cuda.synchronize()
-        for i in range(K):
-            flush.fill_(i & 0xFF)
-            es[i][0].record()
-            fn(qs[i])
-            es[i][1].record()
-        torch.cuda.synchronize()
-        return sum(a.elapsed_time(b) for a, b in es) / 1e3 / K
-
-    ws = wl.cache.workspace(B)
-    # the decode step as two calls (append, then attention), then as one call, on the next 2K tokens
-    def time_steps(fn, t0):
-        es = [(ev(), ev()) for _ in range(K)]
-        for i in range(K):
-            flush.fill_(i & 0xFF)
-            es[i][0].record()
-            fn(t0 + i, qs[i])
-            es[i][1].record()
-        torch.cuda.synchronize()
-        return sum(a.elapsed_time(b) for a, b in es) / 1e3 / K
-
-    def two_calls(i, q):
-        wl.cache.append(0, wl.seq_ids, wl.cu_one, wl.steps_k[i], wl.steps_v[i], total_new=B)
-        wl.cache.attention(0, wl.seq_ids, q, out=out, workspace=ws)
-
-    t_two = time_steps(two_calls, first_token)
-    t_one = time_steps(lambda i, q: wl.cache.decode_step(0, wl.seq_ids, wl.steps_k[i], wl.steps_v[i], q, out=out,
-                                                          workspace=ws), first_token + K)
-    L_now = wl.L + int(wl.cache.seq_lens()[0, 0].item()) - int(wl.L[0])
-    t_int4 = time_attn(lambda q: wl.cache.attention(0, wl.seq_ids, q, out=out, workspace=ws))
-    t_only = time_attn(lambda q: wl.cache.attention(0, wl.seq_ids, q, out=out, workspace=ws,
-                                                    mode=kv4.KV4_MODE_INT4_ONLY))
-    res = {"step_as_two_calls": {"ms_per_step": round(t_two * 1e3, 4)},
-           "step_as_one_call": {"ms_per_step": round(t_one * 1e3, 4)},
-           "int4_protected": {"attention_ms": round(t_int4 * 1e3, 4),
-                              "kv_gbs": round(kv_bytes(L_now, Hkv, D, S, Wn) / t_int4 / 1e9, 1)},
-           "int4_only": {"attention_ms": round(t_only * 1e3, 4),
-                         "kv_gbs": round(kv_bytes(L_now, Hkv, D, S, Wn, int4_only=True) / t_only / 1e9, 1)}}
-    # multi-token query (speculative verification): the most query tokens whose
-    # heads fit one 8-column operand, causal over the same cache
-    T = 8 // (w["Hq"] // Hkv)
-    if T >= 2:
-        gen = torch.Generator(device=device).manual_seed(4242)
-        qx = [torch.randn((B, T, w["Hq"], D), generator=gen, device=device).to(torch.bfloat16) for _ in range(3)]
-        outx = torch.empty((B, T, w["Hq"], D), dtype=torch.bfloat16, device=device)
-        wsx = wl.cache.extend_workspace(B, T)
-        ix = iter(range(1 << 30))
-        t_ext = time_attn(lambda q: wl.cache.extend_attention(0, wl.seq_ids, qx[next(ix) % 3], out=outx,
-                                                                workspace=wsx))
-        res["extend"] = {"q_len": T, "attention_ms": round(t_ext * 1e3, 4),
-                         "kv_gbs": round(kv_bytes(L_now, Hkv, D, S, Wn) / t_ext / 1e9, 1),
-                         "query_tokens_per_s": round(B * T / t_ext, 1)}
-    need = bf16_bytes(L_now, Hkv, D)
-    free = torch.cuda.mem_get_info()[0]
-    if need * 1.3 < free:
-        cache16 = kv4.BF16Cache(wl.cfg, torch.from_numpy(wl.table), device)
-        lens = L_now
-        extra_w = dict(w)
-        # identical K/V values: regenerate the same per-sequence tokens up to the current length
-        tmp = Workload.__new__(Workload)
-        tmp.w, tmp.device, tmp.B = w, device, B
-        tmp.L = lens + 1
-        tmp.populate(torch, cache16.append, 0, keep_steps=False)
-        ws16 = cache16.workspace(B)
-        t_bf16 = time_attn(lambda q: cache16.attention(0, wl.seq_ids, q, out=out, workspace=ws16))
-        res["bf16_kv"] = {"attention_ms": round(t_bf16 * 1e3, 4), "kv_gbs": round(need / t_bf16 / 1e9, 1),
-                          "speedup_int4_protected_vs_bf16": round(t_bf16 / t_int4, 3)}
-        del cache16, extra_w
-    else:
-        res["bf16_kv"] = {"skipped": "BF16 cache of %.1f GB does not fit" % (need / 1e9)}
-    return res
-
-
 # --------------------------------------------------------------------------- CPU oracle
 
-def run_oracle_sample(w, n_seqs, steps, warm=1, rope=False):
-    """The oracle on `n_seqs` sequences of the workload: populate (untimed), then `steps` decode steps."""
-    import torch
-    from threadpoolctl import threadpool_limits
-    from oracle import OracleKV4Cache, decode_attention, ROPE_NEOX
+def _oracle_proc(w, seq, steps, warm, rope, barrier, results):
+    """One process of the CPU sample: the oracle on sequence `seq` of layer 0 of `w`: populate (untimed), wait
+    for every process, then `warm` + `steps` decode steps (append one token, attend), timed with the
+    system-wide monotonic clock.  Numpy only, one BLAS thread."""
+    try:
+        from threadpoolctl import threadpool_limits
+        from oracle import OracleKV4Cache, decode_attention, ROPE_NEOX
+        with threadpool_limits(1):
+            L = int(workloads.context_lengths(w)[seq])
+            n_steps = steps + warm
+            one = dict(w, batch=1)
+            table, num_pages, mpps = workloads.block_table(one, [L], extra_tokens=n_steps + 1)
+            cfg = workloads.cache_config(w, num_pages, mpps, max_seqs=1, layers=1)
+            orc = OracleKV4Cache(cfg, table)
+            rp = (workloads.rope_cos_sin(L + n_steps + 1, w["D"]), w["D"], ROPE_NEOX) if rope else None
+            k, v = workloads.kv_sequence_np(w, 0, seq, L - 1 + n_steps)
+            orc.append(0, [0], [0, L - 1], k[:L - 1], v[:L - 1], rope=rp)
+            barrier.wait(timeout=600)
+            times, nbytes = [], 0
+            for i in range(n_steps):
+                q = workloads.queries_np(w, 0, i, n=1)
+                t0 = time.perf_counter()
+                orc.append(0, [0], [0, 1], k[L - 1 + i:L + i], v[L - 1 + i:L + i], rope=rp)
+                decode_attention(orc, 0, [0], q, rope=rp)
+                t1 = time.perf_counter()
+                if i >= warm:
+                    times.append((t0, t1))
+                    nbytes += kv_bytes([L + i], w["Hkv"], w["D"], w["S"], w["W"])
+            results.put((seq, times, nbytes, L))
+    except Exception as e:   # reported by the parent
+        results.put((seq, None, repr(e), 0))
 
-    L = workloads.context_lengths(w)[:n_seqs]
-    table, num_pages, mpps = workloads.block_table(dict(w, batch=n_seqs), L, extra_tokens=steps + warm + 1)
-    cfg = workloads.cache_config(w, num_pages, mpps, max_seqs=n_seqs)
-    orc = OracleKV4Cache(cfg, table)
-    rp = (workloads.rope_cos_sin(int(np.max(L)) + steps + warm + 1, w["D"]), w["D"], ROPE_NEOX) if rope else None
-    toks = []
-    with threadpool_limits(1):
-        for s in range(n_seqs):
-            k, v = workloads.kv_sequence(w, 0, s, int(L[s]) + steps + warm, device="cpu")
-            k, v = k.float().numpy(), v.float().numpy()
-            orc.append(0, [s], [0, int(L[s]) - 1], k[:L[s] - 1], v[:L[s] - 1], rope=rp)
-            toks.append((k, v))
-        times, nbytes = [], []
-        for i in range(steps + warm):
-            kn = np.stack([toks[s][0][L[s] - 1 + i] for s in range(n_seqs)])
-            vn = np.stack([toks[s][1][L[s] - 1 + i] for s in range(n_seqs)])
-            q = workloads.queries(w, 0, i, n=n_seqs, device="cpu").float().numpy()
-            t0 = time.perf_counter()
-            orc.append(0, list(range(n_seqs)), np.arange(n_seqs + 1), kn, vn, rope=rp)
-            decode_attention(orc, 0, list(range(n_seqs)), q, rope=rp)
-            dt = time.perf_counter() - t0
-            if i >= warm:
-                times.append(dt)
-                nbytes.append(kv_bytes(L + i, w["Hkv"], w["D"], w["S"], w["W"]))
-    return sum(nbytes) / sum(times) / 1e9, times, int(np.mean(L))
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
 
 
-def cpu_baseline(w, n_seqs, rope=False):
-    gbs, times, mean_l = run_oracle_sample(w, n_seqs, steps=2, rope=rope)
-    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": "%d of %d sequences (mean context %d), 2 decode steps (append + attention), numpy, "
-                      "BLAS limited to 1 thread; %.1f s per step" % (n_seqs, w["batch"], mean_l, np.mean(times))}
+def oracle_sample(w, procs, steps, warm, rope=False):
+    """The oracle on `procs` sequences of the workload's layer 0 at once, one process per sequence (spawned:
+    no fork of a process that holds a CUDA context).  Returns (GB/s over the timed window, per-step wall times,
+    mean context, processes)."""
+    import multiprocessing as mp
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"
+    ctx = mp.get_context("spawn")
+    B = w["batch"]
+    seqs = [int(s) for s in np.linspace(0, B - 1, procs).round().astype(int)] if procs <= B else \
+        [s % B for s in range(procs)]
+    barrier = ctx.Barrier(len(seqs))
+    results = ctx.Queue()
+    ps = [ctx.Process(target=_oracle_proc, args=(w, s, steps, warm, rope, barrier, results)) for s in seqs]
+    for p in ps:
+        p.start()
+    got = [results.get(timeout=1800) for _ in ps]
+    for p in ps:
+        p.join(timeout=60)
+    bad = [g for g in got if g[1] is None]
+    if bad:
+        raise RuntimeError("oracle process failed: %s" % (bad[0][2],))
+    t0 = min(t[0] for g in got for t in g[1])
+    t1 = max(t[1] for g in got for t in g[1])
+    nbytes = sum(g[2] for g in got)
+    # wall time of step i: from the first start to the last end of step i over the processes
+    per_step = [max(g[1][i][1] for g in got) - min(g[1][i][0] for g in got) for i in range(steps)]
+    return nbytes / (t1 - t0) / 1e9, per_step, float(np.mean([g[3] for g in got])), len(seqs)
+
+
+def cpu_baseline(w, args):
+    procs = args.cpu_procs or host_cores()
+    gbs, per_step, mean_l, n = oracle_sample(w, procs, args.cpu_steps, 1, rope=args.rope)
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": n, "kind": "oracle",
+            "host_cores": host_cores(),
+            "sample": "%d sequences of layer 0 (mean context %.0f), one per process, %d decode steps each (append "
+                      "+ attention) after one warm-up step, numpy with one BLAS thread per process; K/V and q drawn "
+                      "with numpy's generator from the workload's recipe; %.2f s per step over all processes"
+                      % (n, mean_l, args.cpu_steps, float(np.mean(per_step)))}
 
 
 def run_reference(args):
@@ -608,16 +823,16 @@ def run_reference(args):
     if rank != 0:
         return None
     w = workloads.workload(args.workload)
-    n_seqs = max(1, min(args.cpu_seqs, 2))
-    gbs, times, mean_l = run_oracle_sample(w, n_seqs, steps=args.steps, warm=args.warmup, rope=args.rope)
-    t = sum(times)
-    base = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": "%d of %d sequences (mean context %d) per step, numpy, BLAS limited to 1 thread"
-                      % (n_seqs, w["batch"], mean_l)}
+    procs = args.cpu_procs or host_cores()
+    gbs, per_step, mean_l, n = oracle_sample(w, procs, args.steps, args.warmup, rope=args.rope)
+    t = sum(per_step)
+    base = {"value": round(gbs, 4), "unit": "GB/s", "cores": n, "kind": "oracle", "host_cores": host_cores(),
+            "sample": "%d sequences of layer 0 (mean context %.0f) per step, one per process, numpy with one BLAS "
+                      "thread per process" % (n, mean_l)}
     return {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 attention, f32 codes",
-            "data": "synthetic", "config": {"workload": args.workload, "batch_sample": n_seqs,
+            "data": "synthetic", "config": {"workload": args.workload, "batch_sample": n,
                                             "rope": "neox, fused" if args.rope else "none"},
             "cpu_baseline": base, "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                                           "d2h_bytes_per_step": 0}}
@@ -633,7 +848,7 @@ def main():
     res = run_gpu(args)
     if res is not None:
         if res["n_gpus"] == 1 and not args.kernel_only:
-            res["cpu_baseline"] = cpu_baseline(workloads.workload(args.workload), args.cpu_seqs, rope=args.rope)
+            res["cpu_baseline"] = cpu_baseline(workloads.workload(args.workload), args)
         print(json.dumps(res))
 
 

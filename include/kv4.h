@@ -29,10 +29,13 @@
  *   queued on the stream has finished.  The library never allocates device
  *   memory.  A cache lives on the device that holds its buffer; every call on
  *   it runs there, whatever device the calling thread has selected, and the
- *   stream must belong to that device.
+ *   stream must belong to that device.  A call makes that device current only
+ *   for its own duration: the calling thread's current device is the same
+ *   before and after it.
  * - Calls on one cache handle must be ordered on one stream; a handle is not
  *   thread-safe.  Caches on different handles are independent.
- * - Keys are passed after RoPE; RoPE is not part of this library.
+ * - Keys arrive after RoPE, unless the RoPE entry points below (kv4_set_rope,
+ *   kv4_rope_rotate_quantize_append, KV4_MODE_ROPE_Q) apply it on the way in.
  * - GQA grouping is contiguous: query head j reads KV head j / (Hq / Hkv).
  * - bf16 arrays are IEEE bfloat16 bit patterns (uint16); the layout of the
  *   cache buffer is defined by this library (16-token tiles whose byte order
@@ -72,8 +75,10 @@ enum {
   KV4_DEV_TIMEOUT = 8,        /* a bounded wait inside a kernel gave up (~1 s)              */
   KV4_DEV_BAD_SEQ = 16,       /* a sequence id outside [0, max_seqs): entry skipped        */
   KV4_DEV_WORKSPACE = 32,     /* the attention plan did not fit the workspace              */
-  KV4_DEV_ROPE_POS = 64       /* a position at or past the RoPE table: key not written,
+  KV4_DEV_ROPE_POS = 64,      /* a position at or past the RoPE table: key not written,
                                  query rotated with the table's last row                    */
+  KV4_DEV_BAD_CU = 128        /* append row offsets not 0 = cu[0] <= ... <= cu[n] =
+                                 total_new: nothing appended, no length changed              */
 };
 
 /* RoPE pair layouts (kv4_set_rope). */
@@ -163,7 +168,8 @@ int kv4_seq_reset(kv4_cache* cache, int32_t seq_id, kv4_stream_t stream);
  *   dev_seq_ids  int32 [n_seqs], distinct sequence ids
  *   dev_cu_new   int32 [n_seqs+1], cu_new[0] = 0, non-decreasing; sequence
  *                seq_ids[i] receives rows cu_new[i] .. cu_new[i+1]-1
- *   total_new    = cu_new[n_seqs] (host copy, sizes the launch)
+ *   total_new    = cu_new[n_seqs] (host copy, sizes the launch); offsets that
+ *                break either rule set KV4_DEV_BAD_CU and append nothing
  *   k_new, v_new bf16 [total_new][Hkv][D], post-RoPE keys and values
  * Every new position p is INT4-encoded into page block_table[s][p / P], slot
  * p % P; positions p < S and p >= L_new - W are also INT8-encoded into the
@@ -223,16 +229,15 @@ int kv4_attention_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_
  * (KV4_ERR_INVALID_ARG otherwise).  Calls on one cache must be ordered on one
  * stream (they share the cache's state block), and a workspace must not be
  * shared by calls that can run at the same time.
- * Steps, with num_kv_heads a multiple of 4: a query kernel (rotation, integer
- * tensor-core operands), then one persistent attention kernel: every CTA
- * derives the same stream-K split of all (sequence, 4-KV-head group) page
- * stages from the sequence lengths, streams its stages through shared memory
- * by bulk copies, turns INT4/INT8 codes into operands in registers (online
- * softmax) and stores the rotated-back output of the groups it covers whole;
- * groups split over several CTAs are finished by a merge kernel (log-sum-exp
- * merge of the workspace partials, inverse rotation).  The three kernels are
- * chained as programmatic dependents.  With other head counts: a planning
- * kernel, a per-head split-K kernel and a merge kernel.
+ * Steps: a query kernel (rotation, integer tensor-core operands), then one
+ * persistent attention kernel: every CTA derives the same stream-K split of
+ * all (sequence, KV-head group) page stages from the sequence lengths (groups
+ * of 4 KV heads; of 2 or 1 when num_kv_heads is not a multiple of 4), streams
+ * its stages through shared memory by bulk copies, turns INT4/INT8 codes into
+ * operands in registers (online softmax) and stores the rotated-back output
+ * of the groups it covers whole; groups split over several CTAs are finished
+ * by a merge kernel (log-sum-exp merge of the workspace partials, inverse
+ * rotation).  The three kernels are chained as programmatic dependents.
  */
 int kv4_decode_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs,
                          const void* q, void* out, float softmax_scale, int32_t mode,
@@ -256,10 +261,8 @@ int kv4_decode_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq
  *   q, out         bf16 [n_seqs][q_len][Hq][D] (out fp32 with KV4_MODE_OUT_F32)
  *   dev_workspace  >= kv4_extend_workspace_bytes(cache, n_seqs, q_len, ...)
  * A query token with no visible position (L < q_len - i) gets an all-zero row.
- * Errors: KV4_ERR_UNSUPPORTED when num_kv_heads is not a multiple of 4; the
- * others as kv4_decode_attention.  Same kernels as kv4_decode_attention with
- * KV heads a multiple of 4, with the operand columns standing for (query
- * token, query head) pairs.
+ * Errors as kv4_decode_attention.  Same kernels as kv4_decode_attention,
+ * with the operand columns standing for (query token, query head) pairs.
  */
 int kv4_extend_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_t q_len, size_t* bytes);
 
@@ -273,8 +276,8 @@ int kv4_extend_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_t q
  *   k_new, v_new   bf16 [n_seqs][Hkv][D], the new token of entry i
  *   q, out, mode, softmax_scale, dev_workspace   as kv4_decode_attention
  *                  (the workspace of kv4_attention_workspace_bytes)
- * The sequence ids must be distinct.  Needs num_kv_heads a multiple of 4 and
- * at most 16 (KV4_ERR_UNSUPPORTED otherwise; use the two calls then).
+ * The sequence ids must be distinct.  Needs num_kv_heads <= 16
+ * (KV4_ERR_UNSUPPORTED otherwise; use the two calls then).
  * Kernels: one block per sequence appends its token (two warps per KV head,
  * one for K and one for V) and builds the query operands, then the attention
  * and merge kernels of kv4_decode_attention: three launches instead of four.
@@ -300,9 +303,9 @@ int kv4_extend_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq
  *
  * Arguments, results and errors are those of kv4_decode_attention, plus:
  *   KV4_ERR_SCRATCH when kv4_attention_workspace_bytes(cache, n_seqs, 0) is
- *   above KV4_NOALLOC_SCRATCH_BYTES (with KV heads a multiple of 4 that is
- *   n_seqs * Hkv * (16*D + 64) bytes of query operands plus
- *   2 * 3 * SMs * 4 * G * (D + 4) * 4 bytes of partials, e.g. about 8.6 MB for
+ *   above KV4_NOALLOC_SCRATCH_BYTES (that is n_seqs * Hkv * (16*D + 64)
+ *   bytes of query operands plus 2 * 3 * SMs * w * G * (D + 4) * 4 bytes of
+ *   partials, w = 4, 2 or 1 KV heads per group, e.g. about 8.6 MB for
  *   64 sequences, 32/8 heads, D = 128 on 148 SMs, and 16.2 MB for 512);
  *   nothing is launched then.
  * The scratch is one per device and shared by every cache and stream of the
@@ -310,7 +313,9 @@ int kv4_extend_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq
  * two host threads) race on it and give wrong results, so order them (one
  * stream, or events).  Nothing in it has to start at zero.  The first call
  * on a device looks the array up (cudaGetSymbolAddress, with the cache's
- * device current) and should come before any stream capture.
+ * device current) and should come before any stream capture.  The address
+ * is kept for the life of the process: do not use this call on a device
+ * after cudaDeviceReset() (or any other teardown of its primary context).
  */
 #define KV4_NOALLOC_SCRATCH_BYTES (16u << 20)
 int kv4_decode_attention_noalloc(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs,

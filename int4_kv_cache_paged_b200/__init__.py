@@ -44,6 +44,7 @@ KV4_DEV_TIMEOUT = 8
 KV4_DEV_BAD_SEQ = 16
 KV4_DEV_WORKSPACE = 32
 KV4_DEV_ROPE_POS = 64
+KV4_DEV_BAD_CU = 128
 
 KV4_MODE_PROTECTED = 0
 KV4_MODE_INT4_ONLY = 1

@@ -34,8 +34,11 @@ def build(verbose_ptxas=False, force=False):
     """Compile every source to an object in _build/ and link libkv4.so next to this file."""
     os.makedirs(OBJDIR, exist_ok=True)
     objs = []
-    headers = [os.path.join(HERE, "csrc", h) for h in ("kv4_common.cuh", "kv4_attn_tiles.cuh")] + \
-        [os.path.join(ROOT, "include", "kv4.h")]
+    # every header a source can include: an edit to any of them rebuilds every object
+    headers = [os.path.join(HERE, "csrc", h) for h in sorted(os.listdir(os.path.join(HERE, "csrc")))
+               if h.endswith((".cuh", ".h"))] + \
+        [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.join(ROOT, "include")))
+         if h.endswith(".h")]
     newest_header = max(os.path.getmtime(h) for h in headers)
     for src in SOURCES:
         path = os.path.join(HERE, "csrc", src)

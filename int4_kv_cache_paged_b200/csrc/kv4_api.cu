@@ -77,8 +77,8 @@ int create(const kv4_config* cfg, bool bf16, void* dev_buf, size_t bytes, int32_
     return KV4_ERR_INVALID_ARG;
   }
   c->device = attr.device;
-  if (cudaSetDevice(c->device) != cudaSuccess ||
-      cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
+  const kv4::DeviceScope dev(c->device);
+  if (!dev.ok() || cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
     delete c;
     return KV4_ERR_CUDA;
   }
@@ -90,10 +90,13 @@ int create(const kv4_config* cfg, bool bf16, void* dev_buf, size_t bytes, int32_
   c->pool_offset = s.pool_offset;
   c->pool_bytes = s.pool;
   c->prot_bytes = s.prot;
-  c->attn_blocks_per_sm = kv4::attention_blocks_per_sm(c);
-  if (c->attn_blocks_per_sm <= 0) {
-    delete c;
-    return KV4_ERR_CUDA;
+  c->attn_blocks_per_sm = 0;
+  if (bf16) {   // the BF16 baseline: per-head split-K kernel
+    c->attn_blocks_per_sm = kv4::attention_blocks_per_sm(c);
+    if (c->attn_blocks_per_sm <= 0) {
+      delete c;
+      return KV4_ERR_CUDA;
+    }
   }
   c->gattn_ring = 0;
   if (kv4::grouped_path(c)) {
@@ -111,9 +114,6 @@ int create(const kv4_config* cfg, bool bf16, void* dev_buf, size_t bytes, int32_
   return KV4_OK;
 }
 
-// Every call runs on the cache's device (the library's runtime keeps its own
-// current device, independent of the caller's framework).
-bool select_device(const kv4_cache* c) { return cudaSetDevice(c->device) == cudaSuccess; }
 
 int check_layer(const kv4_cache* c, int32_t layer) {
   return (layer < 0 || layer >= c->cfg.num_layers) ? KV4_ERR_INVALID_ARG : KV4_OK;
@@ -137,7 +137,8 @@ int append(kv4_cache* c, int32_t layer, const int32_t* seq_ids, const int32_t* c
   if (n_seqs == 0 || total_new == 0) return KV4_OK;
   if (!seq_ids || !cu_new || !k_new || !v_new) return KV4_ERR_INVALID_ARG;
   if (!aligned16(k_new) || !aligned16(v_new)) return KV4_ERR_INVALID_ARG;
-  if (!select_device(c)) return KV4_ERR_CUDA;
+  const kv4::DeviceScope dev(c->device);   // the cache's device, restored on return
+  if (!dev.ok()) return KV4_ERR_CUDA;
   return kv4::launch_append(c, layer, seq_ids, cu_new, n_seqs, total_new, k_new, v_new, rope, stream);
 }
 
@@ -150,7 +151,8 @@ int attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_t n_seq
   if (!aligned16(q) || !aligned16(out) || reinterpret_cast<uintptr_t>(ws) % kAlign) return KV4_ERR_INVALID_ARG;
   if (!mode_ok(c, mode)) return KV4_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale)) return KV4_ERR_INVALID_ARG;
-  if (!select_device(c)) return KV4_ERR_CUDA;
+  const kv4::DeviceScope dev(c->device);   // the cache's device, restored on return
+  if (!dev.ok()) return KV4_ERR_CUDA;
   return kv4::launch_attention(c, layer, seq_ids, n_seqs, q, out, softmax_scale, mode, ws, ws_bytes, stream);
 }
 
@@ -165,14 +167,16 @@ int extend_attention(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_
   if (!aligned16(q) || !aligned16(out) || reinterpret_cast<uintptr_t>(ws) % kAlign) return KV4_ERR_INVALID_ARG;
   if (!mode_ok(c, mode)) return KV4_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale)) return KV4_ERR_INVALID_ARG;
-  if (!select_device(c)) return KV4_ERR_CUDA;
+  const kv4::DeviceScope dev(c->device);   // the cache's device, restored on return
+  if (!dev.ok()) return KV4_ERR_CUDA;
   return kv4::launch_extend_attention(c, layer, seq_ids, n_seqs, q_len, q, out, softmax_scale, mode, ws, ws_bytes,
                                       stream);
 }
 
 int get_status(kv4_cache* c, cudaStream_t stream, int32_t* device_status) {
   if (!c || !device_status) return KV4_ERR_INVALID_ARG;
-  if (!select_device(c)) return KV4_ERR_CUDA;
+  const kv4::DeviceScope dev(c->device);   // the cache's device, restored on return
+  if (!dev.ok()) return KV4_ERR_CUDA;
   int32_t v = 0;
   if (cudaMemcpyAsync(&v, &c->state->status, sizeof(v), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return KV4_ERR_CUDA;
@@ -218,7 +222,8 @@ int kv4_cache_layout(const kv4_cache* c, int32_t layer, void** dev_pages, void**
 
 int kv4_seq_reset(kv4_cache* c, int32_t seq_id, kv4_stream_t stream) {
   if (!c || seq_id < 0 || seq_id >= c->cfg.max_seqs) return KV4_ERR_INVALID_ARG;
-  if (!select_device(c)) return KV4_ERR_CUDA;
+  const kv4::DeviceScope dev(c->device);   // the cache's device, restored on return
+  if (!dev.ok()) return KV4_ERR_CUDA;
   return kv4::launch_seq_reset(c, seq_id, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -277,7 +282,8 @@ int kv4_decode_step(kv4_cache* c, int32_t layer, const int32_t* seq_ids, int32_t
     return KV4_ERR_INVALID_ARG;
   if (!mode_ok(c, mode)) return KV4_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale)) return KV4_ERR_INVALID_ARG;
-  if (!select_device(c)) return KV4_ERR_CUDA;
+  const kv4::DeviceScope dev(c->device);   // the cache's device, restored on return
+  if (!dev.ok()) return KV4_ERR_CUDA;
   return kv4::launch_decode_step(c, layer, seq_ids, n_seqs, k_new, v_new, q, out, softmax_scale, mode, ws, ws_bytes,
                                  reinterpret_cast<cudaStream_t>(stream));
 }
@@ -306,7 +312,8 @@ int kv4_dequantize_debug(kv4_cache* c, int32_t layer, int32_t seq_id, int32_t st
     return KV4_ERR_INVALID_ARG;
   if (count == 0) return KV4_OK;
   if (!k_out || !v_out) return KV4_ERR_INVALID_ARG;
-  if (!select_device(c)) return KV4_ERR_CUDA;
+  const kv4::DeviceScope dev(c->device);   // the cache's device, restored on return
+  if (!dev.ok()) return KV4_ERR_CUDA;
   return kv4::launch_dequantize_debug(c, layer, seq_id, start, count, view, k_out, v_out,
                                       reinterpret_cast<cudaStream_t>(stream));
 }

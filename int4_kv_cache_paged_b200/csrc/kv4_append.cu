@@ -34,8 +34,10 @@ __device__ __forceinline__ int find_seq(const int* cu, int n_seqs, int n) {
 }
 
 // Last block of an append launch: advance the sequence lengths (from the old
-// lengths every block read at its start) and re-arm the counter.
-__device__ void finish_append(const AppendParams& p, const int* s_cu, const int* s_seq, const int* s_len) {
+// lengths every block read at its start; not when the row offsets were
+// invalid) and re-arm the counter.
+__device__ void finish_append(const AppendParams& p, const int* s_cu, const int* s_seq, const int* s_len,
+                              bool bad_cu) {
   __shared__ int s_last;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -46,7 +48,7 @@ __device__ void finish_append(const AppendParams& p, const int* s_cu, const int*
   if (!s_last) return;
   __threadfence();
   const int cap = p.max_pages_per_seq * p.P;
-  for (int i = threadIdx.x; i < p.n_seqs; i += blockDim.x) {
+  for (int i = threadIdx.x; i < (bad_cu ? 0 : p.n_seqs); i += blockDim.x) {
     const int seq = s_seq[i];
     if (seq < 0 || seq >= p.max_seqs) continue;
     const int n = s_cu[i + 1] - s_cu[i];
@@ -72,15 +74,21 @@ __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams 
     if (i < p.n_seqs) s_seq[i] = p.seq_ids[i];
   }
   __syncthreads();
+  // the row offsets must run 0 = cu[0] <= cu[1] <= ... <= cu[n] = total_new: otherwise a
+  // row could land past its sequence's new length, so nothing is written
+  int bad = 0;
   for (int i = threadIdx.x; i < p.n_seqs; i += blockDim.x) {
     const int seq = s_seq[i];
     s_len[i] = (seq >= 0 && seq < p.max_seqs) ? p.seq_lens[seq] : 0;
+    bad |= s_cu[i] > s_cu[i + 1];
   }
-  __syncthreads();
+  if (threadIdx.x == 0) bad |= s_cu[0] != 0 || s_cu[p.n_seqs] != p.total_new;
+  const bool bad_cu = __syncthreads_or(bad) != 0;
+  if (bad_cu && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(&p.state->status, KV4_DEV_BAD_CU);
 
   const long long job = static_cast<long long>(blockIdx.x) * APPEND_WARPS + warp;
   const long long n_jobs = static_cast<long long>(p.total_new) * p.Hkv * 2;
-  if (job < n_jobs) {
+  if (job < n_jobs && !bad_cu) {
     const int tensor = static_cast<int>(job & 1);
     const int h = static_cast<int>((job >> 1) % p.Hkv);
     const int n = static_cast<int>((job >> 1) / p.Hkv);
@@ -157,7 +165,7 @@ __global__ void __launch_bounds__(32 * APPEND_WARPS) append_kernel(AppendParams 
       }
     }
   }
-  finish_append(p, s_cu, s_seq, s_len);
+  finish_append(p, s_cu, s_seq, s_len, bad_cu);
 }
 
 // ---------------------------------------------------------------------------

@@ -1,4 +1,6 @@
-// Split-K decode attention over the paged INT4/INT8 cache (and the BF16 baseline).
+// Per-head split-K decode attention of the BF16 baseline cache.  (The INT4/INT8
+// cache uses the page-major kernel of kv4_attention_grouped.cu for every head
+// count; the INT4 branches of the templates below are not instantiated.)
 //
 // Method: "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
 // Serving", Abstract -- fused attention over a paged, token-wise INT4 cache whose
@@ -640,12 +642,11 @@ extern "C" int kv4_debug_read(unsigned long long* out4) {
 #endif
 
 int attention_blocks_per_sm(kv4_cache* c) {
+  if (!c->bf16) return -1;   // INT4 caches use the page-major kernel (kv4_attention_grouped.cu)
   const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
-  int blocks = 0, ns;
-  if (c->cfg.head_dim == 128)
-    ns = c->bf16 ? choose_ring<128, true>(c->device, G, &blocks) : choose_ring<128, false>(c->device, G, &blocks);
-  else
-    ns = c->bf16 ? choose_ring<64, true>(c->device, G, &blocks) : choose_ring<64, false>(c->device, G, &blocks);
+  int blocks = 0;
+  const int ns = c->cfg.head_dim == 128 ? choose_ring<128, true>(c->device, G, &blocks)
+                                        : choose_ring<64, true>(c->device, G, &blocks);
   if (ns <= 0) return -1;
   c->attn_ring = ns;
   return blocks;
@@ -810,8 +811,8 @@ int launch_attention(kv4_cache* c, int layer, const int32_t* seq_ids, int n_seqs
   p.mode = mode;
   const double scale = softmax_scale > 0.f ? static_cast<double>(softmax_scale) : 1.0 / sqrt(static_cast<double>(D));
   p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
-  if (D == 128) return c->bf16 ? launch_attention_t<128, true>(c, p, stream) : launch_attention_t<128, false>(c, p, stream);
-  return c->bf16 ? launch_attention_t<64, true>(c, p, stream) : launch_attention_t<64, false>(c, p, stream);
+  if (!c->bf16) return KV4_ERR_UNSUPPORTED;   // INT4 caches took the page-major path above
+  return D == 128 ? launch_attention_t<128, true>(c, p, stream) : launch_attention_t<64, true>(c, p, stream);
 }
 
 }  // namespace kv4

@@ -1,5 +1,6 @@
-// Page-major, stream-K decode attention over the paged INT4/INT8 cache, used
-// when the number of KV heads is a multiple of the group width (4).
+// Page-major, stream-K decode attention over the paged INT4/INT8 cache (every
+// KV-head count: groups of 4 KV heads, or of 2 or 1 when the count is not a
+// multiple of 4).
 //
 // Method: "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
 // Serving", Abstract (fused attention over the paged, rotated token-wise INT4
@@ -8,12 +9,14 @@
 //
 // One launch does the attention proper (a small query kernel runs alongside).
 //
-// Work decomposition.  A head group is GW (4) consecutive KV heads of one
-// sequence.  Its work is a list of stages: one stage per 16-token INT4 tile
-// position (the tiles of the group's heads are contiguous in the head-innermost
-// pool: one 8.7 KB bulk copy at D = 128), then two stages per INT8 protected
-// tile (each half of the heads).  Three CTAs share an SM: four consumer warps
-// per scheduler hide the latency of each warp's dependent tile math.
+// Work decomposition.  A head group is GWR consecutive KV heads of one
+// sequence (4 when the KV-head count is a multiple of 4, else 2 or 1).  Its
+// work is a list of stages: one stage per 16-token INT4 tile position (the
+// tiles of the group's heads are contiguous in the head-innermost pool: one
+// 8.7 KB bulk copy for 4 heads at D = 128), then one or two stages per INT8
+// protected tile (two halves of the heads when the group has 2 or 4).  Three
+// CTAs share an SM: with 4-head groups, four consumer warps per scheduler hide
+// the latency of each warp's dependent tile math.
 // The stage lists of all head groups are concatenated, each group charged a
 // few extra units for the cost of starting it (T units in all), and CTA c of
 // the persistent grid takes units [c*T/N, (c+1)*T/N): every CTA gets the same
@@ -44,30 +47,38 @@ namespace {
 
 using namespace tiles;
 
-#ifndef KV4_GROUP_HEADS
-#define KV4_GROUP_HEADS 4
-#endif
-constexpr int GW = KV4_GROUP_HEADS;      // consumer warps = KV heads per group (4 or 8)
-constexpr int GTHREADS = 32 * (GW + 1);  // + producer warp
-// CTAs per SM: one with 8 heads; three with 4 heads (4 warps per scheduler,
-// which caps registers at 128 per thread)
-constexpr int CTAS_PER_SM = GW == 4 ? 3 : 1;
-static_assert(GW == 4 || GW == 8, "group width");
+// CTAs per SM: three (with 4-head groups, 4 warps per scheduler, which caps
+// registers at 128 per thread)
+constexpr int CTAS_PER_SM = 3;
 constexpr int GQD = 2;                  // segment queue depth
 
-template <int D>
+// Shape of a kernel instantiation with groups of GWR KV heads (one consumer
+// warp per head, plus the producer warp).  A protected tile position of the
+// group's heads is H8 heads per stage, S8 stages.
+template <int GWR>
+struct GShape {
+  static_assert(GWR == 1 || GWR == 2 || GWR == 4, "group width");
+  static constexpr int THREADS = 32 * (GWR + 1);
+  static constexpr int H8 = GWR >= 2 ? GWR / 2 : 1;
+  static constexpr int S8 = GWR / H8;
+};
+
+template <int D, int GWR>
 struct GCfg {
-  static constexpr int STAGE4 = GW * tile4_bytes(D);        // one tile position of the group's heads
-  static constexpr int STAGE8 = (GW / 2) * tile8_bytes(D);  // half a protected tile position
+  static constexpr int STAGE4 = GWR * tile4_bytes(D);                  // one tile position of the group's heads
+  static constexpr int STAGE8 = GShape<GWR>::H8 * tile8_bytes(D);      // part of a protected tile position
   static constexpr int STAGE = STAGE4 > STAGE8 ? STAGE4 : STAGE8;
 };
 
-// One head group of the call: batch entry b, KV heads GW*hg .. GW*hg+GW-1.
+// KV heads per group for a cache: 4, else 2, else 1.
+inline int group_width(int Hkv) { return Hkv % 4 == 0 ? 4 : (Hkv % 2 == 0 ? 2 : 1); }
+
+// One head group of the call: batch entry b, KV heads GWR*hg .. GWR*hg+GWR-1.
 struct Group {
   int b, seq, hg, L;  // index into seq_ids, sequence id, head group, sequence length
   int n4;             // INT4 stages (tiles t0 .. t0+n4-1)
   int t0, lo4, hi4;   // first INT4 tile, valid INT4 positions [lo4, hi4)
-  int n8;             // INT8 tiles (2 stages each), valid slots [0, nprot)
+  int n8;             // INT8 tiles (S8 stages each), valid slots [0, nprot)
   int nprot;
   int start;          // first global stage index
   int pad;
@@ -114,10 +125,12 @@ constexpr int MIN_STAGES = 16;
 // fewer stages.
 constexpr int GROUP_COST = 4;
 
-__host__ __device__ inline int group_stages(const Group& g) { return g.n4 + 2 * g.n8; }
+template <int GWR>
+__host__ __device__ inline int group_stages(const Group& g) { return g.n4 + GShape<GWR>::S8 * g.n8; }
 // Length of a group in the units of the split: its stages plus the start cost (0 when empty).
+template <int GWR>
 __host__ __device__ inline int group_cost(const Group& g) {
-  const int n = group_stages(g);
+  const int n = group_stages<GWR>(g);
   return n > 0 ? n + GROUP_COST : 0;
 }
 
@@ -126,9 +139,9 @@ __device__ __forceinline__ int cta_of(long long j, long long T, long long N) {
   return static_cast<int>(((j + 1) * N - 1) / T);
 }
 
-template <int D>
+template <int D, int GWR>
 __host__ __device__ inline size_t gattn_smem_bytes(int ns) {
-  using C = GCfg<D>;
+  using C = GCfg<D, GWR>;
   return static_cast<size_t>(ns) * C::STAGE + GQD * sizeof(SegQ) + (2 * ns + 2 * GQD) * sizeof(uint64_t) +
          sizeof(GMisc);
 }
@@ -184,13 +197,14 @@ __device__ Group describe(const AttnParams& p, int i, int HGN, bool flag_bad) {
 }
 
 // Zeros for the output rows of head group i (a sequence of length 0), elements e0, e0+step, ...
+template <int GWR>
 __device__ void zero_group(const AttnParams& p, int i, int e0, int step) {
-  const int HGN = p.Hkv / GW;
+  const int HGN = p.Hkv / GWR;
   const int b = i / HGN, hg = i - b * HGN;
-  const int n = GW * p.G * p.D;
+  const int n = GWR * p.G * p.D;
   for (int e = e0; e < n; e += step) {
     const int r = e / p.D, d = e - r * p.D;   // r = KV head within the group * G + operand column
-    const long long off = q_row(p, b, hg * GW + r / p.G, r % p.G) * p.D + d;
+    const long long off = q_row(p, b, hg * GWR + r / p.G, r % p.G) * p.D + d;
     if (p.mode & KV4_MODE_OUT_F32) static_cast<float*>(p.out)[off] = 0.f;
     else static_cast<uint16_t*>(p.out)[off] = 0;
   }
@@ -365,9 +379,10 @@ __global__ void __launch_bounds__(32 * MAXW) gstep_kernel(AttnParams p, AppendPa
 // ---------------------------------------------------------------------------
 // the attention kernel
 
-template <int D>
+template <int D, int GWR>
 __device__ __forceinline__ const uint8_t* stage_source(const AttnParams& p, const Group& g, int u, uint32_t& bytes) {
-  using C = GCfg<D>;
+  using C = GCfg<D, GWR>;
+  using SH = GShape<GWR>;
   if (u < g.n4) {
     const int pos = (g.t0 + u) * TILE;
     int page = p.block_table[static_cast<long long>(g.seq) * p.max_pages_per_seq + pos / p.P];
@@ -376,28 +391,25 @@ __device__ __forceinline__ const uint8_t* stage_source(const AttnParams& p, cons
       page = 0;
     }
     bytes = C::STAGE4;
-    return p.pool + ((static_cast<long long>(page) * (p.P / TILE) + (pos % p.P) / TILE) * p.Hkv + g.hg * GW) *
+    return p.pool + ((static_cast<long long>(page) * (p.P / TILE) + (pos % p.P) / TILE) * p.Hkv + g.hg * GWR) *
                         tile4_bytes(D);
   }
+  // part (v % S8) of protected tile v / S8: heads H8 * (v % S8) .. of the group
   const int v = u - g.n4;
   bytes = C::STAGE8;
-  return p.prot + ((static_cast<long long>(g.seq) * n_prot_tiles(p.S, p.W) + (v >> 1)) * p.Hkv + g.hg * GW +
-                   (v & 1) * (GW / 2)) *
+  return p.prot + ((static_cast<long long>(g.seq) * n_prot_tiles(p.S, p.W) + v / SH::S8) * p.Hkv + g.hg * GWR +
+                   (v % SH::S8) * SH::H8) *
                       tile8_bytes(D);
 }
 
-// PAIR = INT4 tiles per iteration of a consumer warp: 2 or 4 (more independent
-// work per warp, 1 CTA per SM) or 1 (fewer registers, 2 CTAs per SM).  MULTI:
+// PAIR = INT4 tiles per iteration of a consumer warp (1, 2 or 4).  MULTI:
 // several query tokens per sequence (causal visibility per operand column);
-// the one-token variant carries none of that code.
-template <int D, int PAIR, bool MULTI>
-#if KV4_GROUP_HEADS == 4
-#define KV4_GATTN_BOUNDS __maxnreg__(128)
-#else
-#define KV4_GATTN_BOUNDS __launch_bounds__(GTHREADS, 1)
-#endif
-__global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
-  using C = GCfg<D>;
+// the one-token variant carries none of that code.  GWR: KV heads per group.
+template <int D, int PAIR, bool MULTI, int GWR>
+__global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
+  using C = GCfg<D, GWR>;
+  using SH = GShape<GWR>;
+  constexpr int GTHREADS = SH::THREADS;
   extern __shared__ __align__(128) uint8_t smem[];
   const int NS = p.ns;
   uint8_t* ring = smem;
@@ -410,13 +422,13 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int* status = &p.state->status;
   const int c = blockIdx.x;
-  const int HGN = p.Hkv / GW, n_groups = p.n_seqs * HGN;
+  const int HGN = p.Hkv / GWR, n_groups = p.n_seqs * HGN;
 
   // the merge kernel may be scheduled now: it waits for this grid before reading its results
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
-    for (int s = 0; s < NS; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, GW); }
-    for (int s = 0; s < GQD; ++s) { mbar_init(iqf0 + 8 * s, 1); mbar_init(iqe0 + 8 * s, GW); }
+    for (int s = 0; s < NS; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, GWR); }
+    for (int s = 0; s < GQD; ++s) { mbar_init(iqf0 + 8 * s, 1); mbar_init(iqe0 + 8 * s, GWR); }
     misc->abort = 0;
     misc->n_empty = 0;
     for (int s = 0; s < MAX_NS; ++s) misc->last_fill[s] = -1;
@@ -434,7 +446,7 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
     Group gd{};
     if (i < n_groups) gd = describe(p, i, HGN, c == 0);
     int tot;
-    const int ex = block_exclusive_scan(group_cost(gd), misc->red, &tot);
+    const int ex = block_exclusive_scan(group_cost<GWR>(gd), misc->red, &tot);
     if (c0 == 0) { my_g = gd; my_start = ex; }
     T += tot;
   }
@@ -445,20 +457,20 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
   const int j1 = zero_all ? 0 : static_cast<int>((c + 1) * static_cast<long long>(T) / N);
   auto visit = [&](int i, const Group& gd, int st) {
     if (i >= n_groups) return;
-    const int n = group_cost(gd);
+    const int n = group_cost<GWR>(gd);
     if (n > 0) {
       if (st <= j0 && j0 < st + n) {
         misc->first = gd;
         misc->first.start = st;
       }
-      if (st >= j0 && st < j1) plan[i] = GPlanRec{st, group_stages(gd)};
+      if (st >= j0 && st < j1) plan[i] = GPlanRec{st, group_stages<GWR>(gd)};
     } else {
       const int owner = zero_all ? 0 : cta_of(min(st, T - 1), T, N);
       if (owner == c) {
         plan[i] = GPlanRec{st, 0};
         const int k = atomicAdd(&misc->n_empty, 1);
         if (k < 32) misc->empty[k] = i;
-        else zero_group(p, i, 0, 1);
+        else zero_group<GWR>(p, i, 0, 1);
       }
     }
   };
@@ -471,7 +483,7 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
       Group gd{};
       if (i < n_groups) gd = describe(p, i, HGN, false);
       int tot;
-      const int ex = block_exclusive_scan(group_cost(gd), misc->red, &tot);
+      const int ex = block_exclusive_scan(group_cost<GWR>(gd), misc->red, &tot);
       visit(i, gd, base + ex);
       base += tot;
     }
@@ -484,13 +496,13 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
   __syncthreads();
   {
     const int ne = min(misc->n_empty, 32);
-    for (int e = 0; e < ne; ++e) zero_group(p, misc->empty[e], tid, GTHREADS);
+    for (int e = 0; e < ne; ++e) zero_group<GWR>(p, misc->empty[e], tid, GTHREADS);
   }
   if (zero_all || c >= N || j0 >= j1) {
     return;
   }
 
-  if (warp == GW) {
+  if (warp == GWR) {
     // ------------------------------------------------------------ producer
     const int nbatch = NS < 32 ? NS : 32;
     Group g = misc->first;
@@ -500,7 +512,7 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
     int q = 0;
     bool ok = true;
     while (j < j1 && ok) {
-      const int gst = group_stages(g);
+      const int gst = group_stages<GWR>(g);
       const int a = g.start + GROUP_COST, e = a + gst;   // the group's stages in cost units
       if (a >= j1) break;                                // only its start cost falls in this range
       const int u = max(j, a) - a;
@@ -529,7 +541,7 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
         bool lane_ok = true;
         if (lane < nbatch && base + lane < n) {
           uint32_t bytes;
-          const uint8_t* src = stage_source<D>(p, g, u + base + lane, bytes);
+          const uint8_t* src = stage_source<D, GWR>(p, g, u + base + lane, bytes);
           const uint32_t jl = jj + base + lane;
           const int s = jl % NS;
           lane_ok = mbar_wait(empty0 + 8 * s, ((jl / NS) & 1) ^ 1, abort_flag, status);
@@ -548,7 +560,7 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
       j = e;
       ++q;
       if (j < j1 && ok) {
-        while (group_stages(nxt) == 0) nxt = describe(p, ++gn, HGN, false);   // empty sequences own no stage
+        while (group_stages<GWR>(nxt) == 0) nxt = describe(p, ++gn, HGN, false);   // empty sequences own no stage
         nxt.start = e;
         gi = gn;
         g = nxt;
@@ -604,7 +616,7 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
     if (q == 0) asm volatile("griddepcontrol.wait;" ::: "memory");   // the query operands are written
     QFrag<D> qf;
     {
-      const uint8_t* blob = p.qblob + static_cast<size_t>(g.b * p.Hkv + g.hg * GW + w) * qblob_bytes(D);
+      const uint8_t* blob = p.qblob + static_cast<size_t>(g.b * p.Hkv + g.hg * GWR + w) * qblob_bytes(D);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         const uint4 v = __ldcg(reinterpret_cast<const uint4*>(blob) + 32 * cc + lane);
@@ -669,7 +681,7 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
         }
         u += nt;
       } else {
-        // one INT8 stage: half (v & 1) of protected tile (v >> 1) holds heads (GW/2)*(v&1) .. +GW/2-1
+        // one INT8 stage: part (v % S8) of protected tile v / S8 holds heads H8*(v % S8) .. +H8-1
         const int v = u - g.n4;
         const int s0 = s;
         const uint32_t p0 = par;
@@ -677,9 +689,9 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
         ok = mbar_wait(full0 + 8 * s0, p0, abort_flag, status);
         if (!ok) break;
         const uint32_t eb = empty0 + 8 * s0;
-        if ((v & 1) == w / (GW / 2)) {
-          const uint32_t st = smem_u32(ring + static_cast<size_t>(s0) * C::STAGE + (w % (GW / 2)) * tile8_bytes(D));
-          const int slot0 = (v >> 1) * TILE;
+        if (v % SH::S8 == w / SH::H8) {
+          const uint32_t st = smem_u32(ring + static_cast<size_t>(s0) * C::STAGE + (w % SH::H8) * tile8_bytes(D));
+          const int slot0 = (v / SH::S8) * TILE;
           if (slot0 + TILE <= g.nprot && !MULTI) {
             tile_int8<D, false>(st, qf, ws, lane, 15, eb, cs);
           } else if (!MULTI) {
@@ -730,14 +742,14 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
     }
 #pragma unroll
     for (int m = 0; m < D / 16; ++m) { ws.o[m][0] += ws.z0; ws.o[m][2] += ws.z0; ws.o[m][1] += ws.z1; ws.o[m][3] += ws.z1; }
-    const int hkv = g.hg * GW + w;
+    const int hkv = g.hg * GWR + w;
     if (sq.nseg == 1) {
       store_head<D, MULTI>(p, g.b, hkv, lane, ws.o, ws.l0, ws.l1);
       continue;
     }
     // several CTAs share the group: its partial to the workspace (slot 0 = this
     // CTA's first segment, slot 1 = its last), merged by the merge kernel
-    const int slotp = (c * 2 + (q == 0 ? 0 : 1)) * GW + w;
+    const int slotp = (c * 2 + (q == 0 ? 0 : 1)) * GWR + w;
     float* part = p.partials + static_cast<size_t>(slotp) * pstride;
     if (h0 < G) {
       float* r = part + h0 * HS;
@@ -761,7 +773,7 @@ __global__ void KV4_GATTN_BOUNDS gattn_kernel(AttnParams p, GPlanRec* plan) {
 
 constexpr int MWARPS = 8;
 
-template <int D>
+template <int D, int GWR>
 __global__ void __launch_bounds__(32 * MWARPS) gmerge_kernel(AttnParams p, const GPlanRec* plan) {
   constexpr int VPL = D / 32;
   constexpr int HS = head_stride(D);
@@ -769,10 +781,10 @@ __global__ void __launch_bounds__(32 * MWARPS) gmerge_kernel(AttnParams p, const
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * MWARPS + (threadIdx.x >> 5);
   asm volatile("griddepcontrol.wait;" ::: "memory");   // the partials and the plan are written
-  const int G = p.G, HGN = p.Hkv / GW, per_b = p.Hkv * G;   // G: operand columns (query tokens x heads)
+  const int G = p.G, HGN = p.Hkv / GWR, per_b = p.Hkv * G;   // G: operand columns (query tokens x heads)
   if (gw >= p.n_seqs * per_b) return;
   const int b = gw / per_b, r = gw - b * per_b, hkv = r / G, gq = r - hkv * G;
-  const int hg = hkv / GW, w = hkv - hg * GW;
+  const int hg = hkv / GWR, w = hkv - hg * GWR;
   const GPlanHdr* hdr = reinterpret_cast<const GPlanHdr*>(plan + p.n_seqs * HGN);
   const long long T = __ldcg(&hdr->T), N = __ldcg(&hdr->N);
   const GPlanRec rec = {__ldcg(&plan[b * HGN + hg].start), __ldcg(&plan[b * HGN + hg].stages)};
@@ -786,7 +798,7 @@ __global__ void __launch_bounds__(32 * MWARPS) gmerge_kernel(AttnParams p, const
   const int pstride = partial_stride(G, D);
   auto row = [&](int k) -> const float* {
     const int sl = (k == 0 && first_is_last) ? 1 : 0;
-    return p.partials + static_cast<size_t>(((cf + k) * 2 + sl) * GW + w) * pstride + gq * HS;
+    return p.partials + static_cast<size_t>(((cf + k) * 2 + sl) * GWR + w) * pstride + gq * HS;
   };
   float M = NEG_INF;
   for (int k = lane; k < nseg; k += 32) M = fmaxf(M, __ldcg(row(k) + D));
@@ -843,7 +855,7 @@ __global__ void __launch_bounds__(32 * MWARPS) gmerge_kernel(AttnParams p, const
 // host side
 
 #ifndef KV4_GROUPED_PAIR
-#define KV4_GROUPED_PAIR (KV4_GROUP_HEADS == 4 ? 2 : 4)
+#define KV4_GROUPED_PAIR 2
 #endif
 constexpr int kPair = KV4_GROUPED_PAIR;   // INT4 tiles per consumer iteration of the compiled variant
 static_assert(kPair == 1 || kPair == 2 || kPair == 4, "tiles per iteration");
@@ -863,50 +875,52 @@ struct GLayout {
 GLayout g_layout(const kv4_cache* c, int n_seqs, int qlen) {
   const kv4_config& cfg = c->cfg;
   const int G = qlen * (cfg.num_q_heads / cfg.num_kv_heads);   // operand columns per KV head
+  const int gw = group_width(cfg.num_kv_heads);
   GLayout l{};
   l.qblob = 0;
   l.partials = al256(static_cast<size_t>(n_seqs) * cfg.num_kv_heads * qblob_bytes(cfg.head_dim));
-  l.plan = l.partials + al256(static_cast<size_t>(g_grid(c)) * 2 * GW * partial_stride(G, cfg.head_dim) * sizeof(float));
-  const size_t n_groups = static_cast<size_t>(n_seqs) * (cfg.num_kv_heads / GW);
+  l.plan = l.partials + al256(static_cast<size_t>(g_grid(c)) * 2 * gw * partial_stride(G, cfg.head_dim) * sizeof(float));
+  const size_t n_groups = static_cast<size_t>(n_seqs) * (cfg.num_kv_heads / gw);
   l.total = l.plan + al256(n_groups * sizeof(GPlanRec) + sizeof(GPlanHdr));
   return l;
 }
 
-// Ring depth for the kernel variant PAIR at its CTAs per SM (2 for PAIR 1, else 1).
-template <int D, int PAIR>
+// Deepest ring (at most MAX_NS stages) that keeps CTAS_PER_SM CTAs of both
+// variants (one and several query tokens) resident per SM.
+template <int D, int PAIR, int GWR>
 int g_choose_ring(int device) {
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess) return -1;
-  if (cudaFuncSetAttribute(gattn_kernel<D, PAIR, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) !=
+  if (cudaFuncSetAttribute(gattn_kernel<D, PAIR, false, GWR>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) !=
           cudaSuccess ||
-      cudaFuncSetAttribute(gattn_kernel<D, PAIR, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) !=
+      cudaFuncSetAttribute(gattn_kernel<D, PAIR, true, GWR>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) !=
           cudaSuccess)
     return -1;
   const int want = CTAS_PER_SM;
   for (int ns = MAX_NS; ns >= 2; --ns) {
-    const size_t smem = gattn_smem_bytes<D>(ns);
+    const size_t smem = gattn_smem_bytes<D, GWR>(ns);
     if (smem > static_cast<size_t>(optin)) continue;
     int blocks = 0;
     int blocks_multi = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, gattn_kernel<D, PAIR, false>, GTHREADS, smem) !=
-            cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_multi, gattn_kernel<D, PAIR, true>, GTHREADS, smem) !=
-            cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, gattn_kernel<D, PAIR, false, GWR>,
+                                                      GShape<GWR>::THREADS, smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_multi, gattn_kernel<D, PAIR, true, GWR>,
+                                                      GShape<GWR>::THREADS, smem) != cudaSuccess)
       return -1;
     if (blocks >= want && blocks_multi >= want) return ns;
   }
   return -1;
 }
 
-template <int D>
-int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const AppendParams* step = nullptr) {
+template <int D, int GWR>
+int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const AppendParams* step) {
   const GLayout l = g_layout(c, p.n_seqs, p.qlen);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   p.qblob = wsb + l.qblob;
   p.partials = reinterpret_cast<float*>(wsb + l.partials);
   GPlanRec* plan = reinterpret_cast<GPlanRec*>(wsb + l.plan);
   p.grid = g_grid(c);
-  p.cap_parts = p.grid * 2 * GW;
+  p.cap_parts = p.grid * 2 * GWR;
   p.ns = c->gattn_ring;
   if (step) {
     // fused decode step: the append and the query operands first; the attention
@@ -921,8 +935,8 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.grid);
-  cfg.blockDim = dim3(GTHREADS);
-  cfg.dynamicSmemBytes = gattn_smem_bytes<D>(p.ns);
+  cfg.blockDim = dim3(GShape<GWR>::THREADS);
+  cfg.dynamicSmemBytes = gattn_smem_bytes<D, GWR>(p.ns);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -930,27 +944,46 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   cfg.attrs = attr;
   cfg.numAttrs = step ? 0 : 1;
   // several query tokens per sequence (even a pass of one of them): the causal variant
-  cudaError_t e = p.qtot > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true>, p, plan)
-                              : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false>, p, plan);
+  cudaError_t e = p.qtot > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true, GWR>, p, plan)
+                              : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false, GWR>, p, plan);
   if (e == cudaSuccess) {
     cudaLaunchConfig_t mcfg = cfg;
     mcfg.gridDim = dim3((p.n_seqs * p.Hkv * p.G + MWARPS - 1) / MWARPS);
     mcfg.blockDim = dim3(32 * MWARPS);
     mcfg.dynamicSmemBytes = 0;
     mcfg.numAttrs = 1;   // programmatic dependent of the attention kernel
-    e = cudaLaunchKernelEx(&mcfg, gmerge_kernel<D>, p, static_cast<const GPlanRec*>(plan));
+    e = cudaLaunchKernelEx(&mcfg, gmerge_kernel<D, GWR>, p, static_cast<const GPlanRec*>(plan));
   }
   if (c->ev_after) cudaEventRecord(c->ev_after, stream);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
 
+template <int D>
+int g_launch_gw(kv4_cache* c, const AttnParams& p, void* ws, cudaStream_t stream, const AppendParams* step = nullptr) {
+  switch (group_width(p.Hkv)) {
+    case 4: return g_launch<D, 4>(c, p, ws, stream, step);
+    case 2: return g_launch<D, 2>(c, p, ws, stream, step);
+    default: return g_launch<D, 1>(c, p, ws, stream, step);
+  }
+}
+
+template <int D>
+int g_choose_ring_gw(int device, int Hkv) {
+  switch (group_width(Hkv)) {
+    case 4: return g_choose_ring<D, kPair, 4>(device);
+    case 2: return g_choose_ring<D, kPair, 2>(device);
+    default: return g_choose_ring<D, kPair, 1>(device);
+  }
+}
+
 }  // namespace
 
-bool grouped_path(const kv4_cache* c) { return !c->bf16 && c->cfg.num_kv_heads % GW == 0; }
+bool grouped_path(const kv4_cache* c) { return !c->bf16; }
 
 int grouped_ring(kv4_cache* c) {
   c->gattn_pair = kPair;
-  return c->cfg.head_dim == 128 ? g_choose_ring<128, kPair>(c->device) : g_choose_ring<64, kPair>(c->device);
+  return c->cfg.head_dim == 128 ? g_choose_ring_gw<128>(c->device, c->cfg.num_kv_heads)
+                                : g_choose_ring_gw<64>(c->device, c->cfg.num_kv_heads);
 }
 
 size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs, int qlen) { return g_layout(c, n_seqs, qlen).total; }
@@ -966,7 +999,7 @@ int launch_decode_step(kv4_cache* c, int layer, const int32_t* seq_ids, int n_se
   fill_common(c, layer, seq_ids, n_seqs, q, out, softmax_scale, mode, p);
   const AppendParams ap = append_params(c, layer, seq_ids, nullptr, n_seqs, n_seqs, k_new, v_new,
                                         (mode & KV4_MODE_ROPE_Q) != 0);
-  return p.D == 128 ? g_launch<128>(c, p, ws, stream, &ap) : g_launch<64>(c, p, ws, stream, &ap);
+  return p.D == 128 ? g_launch_gw<128>(c, p, ws, stream, &ap) : g_launch_gw<64>(c, p, ws, stream, &ap);
 }
 
 int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -975,7 +1008,7 @@ int launch_grouped(kv4_cache* c, const AttnParams& p, void* ws, size_t ws_bytes,
   if (ws_bytes < g_layout(c, p.n_seqs, p.qlen).total) return KV4_ERR_WORKSPACE;
   if (c->gattn_ring <= 0 || c->gattn_ring > MAX_NS) return KV4_ERR_UNSUPPORTED;
   if (p.n_seqs > c->cfg.max_seqs) return KV4_ERR_INVALID_ARG;
-  return p.D == 128 ? g_launch<128>(c, p, ws, stream) : g_launch<64>(c, p, ws, stream);
+  return p.D == 128 ? g_launch_gw<128>(c, p, ws, stream) : g_launch_gw<64>(c, p, ws, stream);
 }
 
 }  // namespace kv4

@@ -1,7 +1,7 @@
 // Tile routines of the split-K decode attention kernels: turn the codes of one
 // 16-token tile in shared memory into 16x8x16 tensor-core operands, run the
-// scores, the online softmax and P.V.  Shared by the per-head and the
-// page-major kernels.
+// scores, the online softmax and P.V.  Used by the page-major INT4/INT8
+// kernel and (the BF16 tile) by the per-head BF16 baseline kernel.
 //
 // Method: "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
 // Serving", Abstract (fused attention over the rotated token-wise INT4 cache);

@@ -436,6 +436,31 @@ struct kv4_cache {
 
 namespace kv4 {
 
+// Makes the cache's device current for the lifetime of the object and gives
+// the calling thread its previous current device back afterwards, so a call
+// into the library leaves the caller's device selection as it found it.
+class DeviceScope {
+ public:
+  explicit DeviceScope(int device) {
+    if (cudaGetDevice(&prev_) != cudaSuccess) {
+      cudaGetLastError();
+      prev_ = -1;
+    }
+    ok_ = prev_ == device || cudaSetDevice(device) == cudaSuccess;
+  }
+  ~DeviceScope() {
+    int cur = -1;
+    if (prev_ >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev_) cudaSetDevice(prev_);
+  }
+  DeviceScope(const DeviceScope&) = delete;
+  DeviceScope& operator=(const DeviceScope&) = delete;
+  bool ok() const { return ok_; }
+
+ private:
+  int prev_ = -1;
+  bool ok_ = false;
+};
+
 // Launchers (defined in the .cu files).
 int launch_append(kv4_cache* c, int layer, const int32_t* seq_ids, const int32_t* cu_new, int n_seqs, int total_new,
                   const void* k_new, const void* v_new, bool rope, cudaStream_t stream);

@@ -49,7 +49,8 @@ extern "C" int kv4_decode_attention_noalloc(kv4_cache* c, int32_t layer, const i
   int rc = kv4_attention_workspace_bytes(c, n_seqs, 0, &need);
   if (rc != KV4_OK) return rc;
   if (need > kScratchBytes) return KV4_ERR_SCRATCH;
-  if (cudaSetDevice(c->device) != cudaSuccess) return KV4_ERR_CUDA;
+  const kv4::DeviceScope dev(c->device);   // the cache's device, restored on return
+  if (!dev.ok()) return KV4_ERR_CUDA;
   void* scratch = nullptr;
   rc = scratch_of(c->device, &scratch);
   if (rc != KV4_OK) return rc;

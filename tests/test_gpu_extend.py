@@ -128,9 +128,24 @@ def test_extend_in_several_passes(kv4, Hq, Hkv, T):
     assert torch.all(out[seqs.index(2)] == 0)
 
 
-def test_extend_rejects_unsupported_shapes(kv4):
+@pytest.mark.parametrize("Hq,Hkv,T", [(4, 1, 2), (8, 2, 2), (6, 2, 3), (3, 3, 2)])
+def test_extend_head_groups_of_one_and_two(kv4, Hq, Hkv, T):
+    """KV-head counts that are not a multiple of 4 run in groups of 2 or 1 KV heads."""
+    rng = np.random.default_rng(500 + 10 * Hkv + T)
+    D, n = 64, 4
+    mpps = 700 // 16 + 2
+    cfg = cfg_dict(D=D, Hq=Hq, Hkv=Hkv, P=16, Bh=64, S=4, W=32, num_pages=n * mpps, mpps=mpps, max_seqs=n)
+    pair = Pair(cfg, random_table(n, mpps, n * mpps, rng))
+    _populate(pair, rng, list(range(n)), [700, 1, 0, 45], Hkv, D, chunk=128)
+    q = bf16_values((n, T, Hq, D), rng)
+    out, _ = _check(kv4, pair, [3, 0, 2, 1], q)
+    _check(kv4, pair, [3, 0, 2, 1], q, mode=kv4.KV4_MODE_INT4_ONLY)
+    assert torch.all(out[2] == 0)
+
+
+def test_extend_rejects_bad_arguments(kv4):
     rng = np.random.default_rng(79)
     cfg2 = cfg_dict(D=64, Hq=4, Hkv=2, P=16, Bh=64, S=4, W=32, num_pages=8, mpps=4, max_seqs=2)
     pair2 = Pair(cfg2, random_table(2, 4, 8, rng))
-    with pytest.raises(kv4.KV4Error):                              # KV heads not a multiple of 4
-        _extend(pair2, [0, 1], bf16_values((2, 2, 4, 64), rng))
+    with pytest.raises(kv4.KV4Error):                              # q_len < 1
+        _extend(pair2, [0, 1], bf16_values((2, 0, 4, 64), rng))

@@ -1,8 +1,8 @@
 """GPU parity of the folded-rotation modes: KV4_MODE_Q_ROTATED (the query
 arrives as H q and is used as given) and KV4_MODE_OUT_ROTATED (the output
 stays in the rotated basis), alone and together, on the page-major path
-(decode and multi-token) and on the per-head path, against the oracle with
-the same options."""
+(decode and multi-token) with groups of 4, 2 and 1 KV heads, against the
+oracle with the same options."""
 
 import numpy as np
 import pytest

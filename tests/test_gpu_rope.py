@@ -1,9 +1,9 @@
 """GPU parity of the fused RoPE path: kv4_rope_rotate_quantize_append (RoPE of
 each key at its position, then rotation and quantization) against the oracle
 byte for byte, and attention with KV4_MODE_ROPE_Q (RoPE of each query at its
-position) against the oracle, for both pair layouts, partial rotary dims, the
-page-major and the per-head paths, decode and multi-token queries; a key
-past the table is flagged and not written."""
+position) against the oracle, for both pair layouts, partial rotary dims,
+groups of 4, 2 and 1 KV heads, decode and multi-token queries; a key past
+the table is flagged and not written."""
 
 import numpy as np
 import pytest

@@ -49,7 +49,9 @@ def _twins(Hq, Hkv, D, Bh, lens, seed, rope=None):
 
 
 @pytest.mark.parametrize("Hq,Hkv,D,Bh,rope", [(32, 8, 128, 128, None), (16, 4, 64, 64, None),
-                                              (32, 8, 128, 128, (128, 0)), (8, 8, 64, 32, (32, 1))])
+                                              (32, 8, 128, 128, (128, 0)), (8, 8, 64, 32, (32, 1)),
+                                              (4, 1, 64, 64, None), (8, 2, 128, 128, None), (6, 6, 64, 64, None),
+                                              (4, 2, 64, 64, (64, 0))])
 def test_step_equals_append_then_attention(kv4, Hq, Hkv, D, Bh, rope):
     lens = [300, 0, 15, 31, 47, 1]
     a, b, rng, cs = _twins(Hq, Hkv, D, Bh, lens, Hq + D + (0 if rope is None else rope[1] + 1), rope)
@@ -82,7 +84,7 @@ def test_step_equals_append_then_attention(kv4, Hq, Hkv, D, Bh, rope):
         assert compare_int8_store(pair, 0, list(range(n))) == []
 
 
-def test_step_flags_an_unmapped_page_and_rejects_other_head_counts(kv4):
+def test_step_flags_an_unmapped_page_and_rejects_too_many_kv_heads(kv4):
     rng = np.random.default_rng(90)
     cfg = cfg_dict(D=64, Hq=8, Hkv=4, P=16, Bh=64, S=4, W=16, num_pages=4, mpps=4, max_seqs=2)
     table = np.full((2, 4), -1, np.int32)
@@ -94,7 +96,11 @@ def test_step_flags_an_unmapped_page_and_rejects_other_head_counts(kv4):
     pair.gpu.decode_step(0, ids, k, v, q)
     torch.cuda.synchronize()
     assert pair.gpu.status() & kv4.KV4_DEV_BAD_PAGE          # sequence 1 has no page
-    cfg2 = cfg_dict(D=64, Hq=4, Hkv=2, P=16, Bh=64, S=4, W=16, num_pages=8, mpps=4, max_seqs=2)
+    # the step kernel runs two warps per KV head in one block: at most 16 KV heads
+    cfg2 = cfg_dict(D=64, Hq=32, Hkv=32, P=16, Bh=64, S=4, W=16, num_pages=8, mpps=4, max_seqs=2)
     pair2 = Pair(cfg2, random_table(2, 4, 8, rng))
-    with pytest.raises(kv4.KV4Error):
-        pair2.gpu.decode_step(0, ids, k[:, :2].contiguous(), v[:, :2].contiguous(), q[:, :4].contiguous())
+    k2, v2, q2 = (bf16_values((2, 32, 64), rng).cuda(), bf16_values((2, 32, 64), rng).cuda(),
+                  bf16_values((2, 32, 64), rng).cuda())
+    with pytest.raises(kv4.KV4Error) as e:
+        pair2.gpu.decode_step(0, ids, k2, v2, q2)
+    assert e.value.code == kv4.KV4_ERR_UNSUPPORTED

@@ -21,6 +21,9 @@ Workloads (one decode layer each unless stated):
 * stack36         -- 36 independent layer caches, batch 256, contexts uniform in
                      [4096, 16384], page 16, S=4, W=128, 4 steps.
 
+kv_sequence_np / queries_np draw the same recipe with numpy's generator (other
+values, same distributions) for CPU processes that do not load torch.
+
 rope_cos_sin(max_pos, R, base) gives the RoPE angle table that the fused
 RoPE append and query kernels take as an input (the model's angles).
 
@@ -32,4 +35,4 @@ sides of a comparison (values are copied, never regenerated, across devices).
 """
 
 from .synth import (WORKLOADS, workload, context_lengths, block_table, kv_sequence,  # noqa: F401
-                    queries, cache_config, make_seed, rope_cos_sin)
+                    queries, cache_config, make_seed, rope_cos_sin, kv_sequence_np, queries_np)

@@ -1,9 +1,12 @@
-"""Seeded synthetic inputs (no arithmetic of the method lives here)."""
+"""Seeded synthetic inputs (no arithmetic of the method lives here).
+
+torch is imported only by the generators that return tensors, so CPU worker
+processes that use the numpy generators (kv_sequence_np, queries_np) do not
+load it."""
 
 import math
 
 import numpy as np
-import torch
 
 WORKLOADS = {
     "tiny": dict(index=0, layers=1, batch=2, Hq=4, Hkv=1, D=64, P=16, Bh=64, S=4, W=32,
@@ -94,6 +97,7 @@ def kv_sequence(w, layer, seq, length, device="cpu"):
     position 0 multiplied by sink_factor, and optionally a random-walk mean
     along the positions; both are then rounded to bf16.
     """
+    import torch
     Hkv, D = w["Hkv"], w["D"]
     g = torch.Generator(device=device)
     g.manual_seed(make_seed(w["seed"], 4, layer, seq))
@@ -113,10 +117,44 @@ def kv_sequence(w, layer, seq, length, device="cpu"):
 
 def queries(w, layer, step, n=None, device="cpu"):
     """bf16 queries [batch, Hq, D] ~ N(0, 1) for one decode step."""
+    import torch
     B = w["batch"] if n is None else n
     g = torch.Generator(device=device)
     g.manual_seed(make_seed(w["seed"], 5, layer, step))
     return torch.randn((B, w["Hq"], w["D"]), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
+def _bf16_bits_np(x):
+    """fp32 -> bf16 round-to-nearest-even, returned as fp32 values (numpy; finite inputs)."""
+    u = np.ascontiguousarray(x, np.float32).view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return r.view(np.float32)
+
+
+def kv_sequence_np(w, layer, seq, length):
+    """The recipe of kv_sequence drawn with numpy's generator (PCG64, same seed): fp32 arrays of bf16 values
+    [length, Hkv, D].  Same shapes and distributions, different values from the torch generators; for CPU
+    processes that time the oracle on a sample of a workload."""
+    Hkv, D = w["Hkv"], w["D"]
+    rng = np.random.default_rng(make_seed(w["seed"], 4, layer, seq))
+    k = rng.standard_normal((length, Hkv, D), dtype=np.float32)
+    v = rng.standard_normal((length, Hkv, D), dtype=np.float32)
+    if w["n_outlier"] > 0:
+        for h, ch in enumerate(_outlier_channels(w, layer)):
+            k[:, h, ch] *= np.float32(w["outlier_factor"])
+    if length > 0 and w["sink_factor"] != 1.0:
+        k[0] *= np.float32(w["sink_factor"])
+    if w["drift_sigma"] > 0:
+        steps = rng.standard_normal((length, Hkv, D), dtype=np.float32)
+        k += np.cumsum(steps * np.float32(w["drift_sigma"]), axis=0, dtype=np.float32)
+    return _bf16_bits_np(k), _bf16_bits_np(v)
+
+
+def queries_np(w, layer, step, n=None):
+    """The recipe of queries drawn with numpy's generator: fp32 array of bf16 values [n, Hq, D]."""
+    B = w["batch"] if n is None else n
+    rng = np.random.default_rng(make_seed(w["seed"], 5, layer, step))
+    return _bf16_bits_np(rng.standard_normal((B, w["Hq"], w["D"]), dtype=np.float32))
 
 
 def cache_config(w, num_pages, max_pages_per_seq, max_seqs=None, layers=None):
