@@ -570,7 +570,7 @@ def bf16_leg(torch, kv4, w, L, extra, used, layers_avail, per_layer_int4, K, dev
            "speedup_int4_protected_vs_bf16": round(t16 / t4, 3)}
     if n < layers_avail:
         res["note"] = ("%d of %d layer caches: the BF16 caches of all layers (%.0f GB) do not fit in HBM; the "
-                       "INT4 time is that of the same %d layers" % (n, layers_avail, need_layer * layers_avail / 1e9, n, n))
+                       "INT4 time is that of the same %d layers" % (n, layers_avail, need_layer * layers_avail / 1e9, n))
     cache16.close()
     del cache16, ws16, out
     torch.cuda.empty_cache()
