@@ -339,6 +339,18 @@ int kv4_get_status(kv4_cache* cache, kv4_stream_t stream, int32_t* device_status
  * events stay owned by the caller. */
 int kv4_set_attention_events(kv4_cache* cache, void* ev_before, void* ev_after);
 
+/* Testing hook for the bounded waits inside the attention kernel: in the
+ * next kv4_decode_attention, kv4_decode_step or kv4_extend_attention call on
+ * this cache (its first pass), the first CTA of the attention kernel does not
+ * fill its stage number `stage` (counted from 0 in that CTA's share of the
+ * work; no effect if the share is shorter).  That CTA's waits then give up
+ * after about a second: the kernel lets its copies in flight land, sets
+ * KV4_DEV_TIMEOUT and returns, the call's output is not valid, and later
+ * calls on the cache are unaffected.  The hook applies to one call and then
+ * clears itself; stage < 0 clears it.  Not for production use: it exists so
+ * that tests can exercise the timeout path without a device fault. */
+int kv4_test_stall_next_attention(kv4_cache* cache, int32_t stage);
+
 /* Static text for a return code. */
 const char* kv4_status_string(int status);
 

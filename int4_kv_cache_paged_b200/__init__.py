@@ -63,7 +63,8 @@ EXPORTS = [
     "kv4_rotate_quantize_append", "kv4_attention_workspace_bytes", "kv4_decode_attention",
     "kv4_decode_attention_noalloc", "kv4_extend_workspace_bytes", "kv4_extend_attention",
     "kv4_set_rope", "kv4_rope_rotate_quantize_append", "kv4_decode_step",
-    "kv4_dequantize_debug", "kv4_get_status", "kv4_set_attention_events", "kv4_status_string", "kv4_version",
+    "kv4_dequantize_debug", "kv4_get_status", "kv4_set_attention_events", "kv4_test_stall_next_attention",
+    "kv4_status_string", "kv4_version",
     "kv4bf16_cache_required_bytes", "kv4bf16_cache_create", "kv4bf16_cache_destroy", "kv4bf16_cache_layout",
     "kv4bf16_append", "kv4bf16_attention_workspace_bytes", "kv4bf16_decode_attention", "kv4bf16_get_status",
     "kv4bf16_set_attention_events",
@@ -99,6 +100,7 @@ _sigs = {
     "kv4_dequantize_debug": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "kv4_get_status": (_I, [_P, _P, ctypes.POINTER(_I)]),
     "kv4_set_attention_events": (_I, [_P, _P, _P]),
+    "kv4_test_stall_next_attention": (_I, [_P, _I]),
     "kv4bf16_set_attention_events": (_I, [_P, _P, _P]),
     "kv4_status_string": (ctypes.c_char_p, [_I]),
     "kv4_version": (ctypes.c_char_p, []),
@@ -260,6 +262,11 @@ def kv4_set_attention_events(handle, ev_before, ev_after):
     """ev_before / ev_after: torch.cuda.Event(enable_timing=True) or None."""
     _check(_lib.kv4_set_attention_events(handle, _event_handle(ev_before), _event_handle(ev_after)),
            "kv4_set_attention_events")
+
+
+def kv4_test_stall_next_attention(handle, stage):
+    """Testing hook: the next attention call's first CTA leaves `stage` unfilled (its bounded wait runs out)."""
+    _check(_lib.kv4_test_stall_next_attention(handle, int(stage)), "kv4_test_stall_next_attention")
 
 
 def kv4bf16_set_attention_events(handle, ev_before, ev_after):

@@ -5,7 +5,7 @@ import torch
 from . import (make_config, kv4_cache_required_bytes, kv4_cache_create, kv4_cache_destroy, kv4_cache_layout,
                kv4_seq_reset, kv4_rotate_quantize_append, kv4_attention_workspace_bytes, kv4_decode_attention,
                kv4_decode_attention_noalloc, kv4_extend_workspace_bytes, kv4_extend_attention,
-               kv4_set_rope, kv4_rope_rotate_quantize_append, kv4_decode_step,
+               kv4_set_rope, kv4_rope_rotate_quantize_append, kv4_decode_step, kv4_test_stall_next_attention,
                kv4_dequantize_debug, kv4_get_status, kv4bf16_cache_required_bytes, kv4bf16_cache_create,
                kv4bf16_cache_destroy, kv4bf16_cache_layout, kv4bf16_append, kv4bf16_attention_workspace_bytes,
                kv4bf16_decode_attention, kv4bf16_get_status, KV4_VIEW_EFFECTIVE, KV4_MODE_OUT_F32)
@@ -148,6 +148,11 @@ class KV4Cache(_Base):
         """Attention with the library's static scratch (no workspace); `out` must be given."""
         kv4_decode_attention_noalloc(self.handle, layer, seq_ids, int(seq_ids.numel()), q, out, scale, mode, stream)
         return out
+
+    def stall_next_attention(self, stage):
+        """Testing hook: the next attention call's first CTA leaves its stage `stage` unfilled, so its bounded
+        wait runs out (KV4_DEV_TIMEOUT); see kv4_test_stall_next_attention in kv4.h."""
+        kv4_test_stall_next_attention(self.handle, stage)
 
     def dequantize(self, layer, seq, start, count, view=KV4_VIEW_EFFECTIVE, stream=None):
         c = self.cfg

@@ -69,6 +69,7 @@ int create(const kv4_config* cfg, bool bf16, void* dev_buf, size_t bytes, int32_
   if (!c) return KV4_ERR_INVALID_ARG;
   c->cfg = *cfg;
   c->bf16 = bf16;
+  c->test_stall = -1;
   // the cache lives on the device that owns its buffer
   cudaPointerAttributes attr{};
   if (cudaPointerGetAttributes(&attr, dev_buf) != cudaSuccess || attr.type != cudaMemoryTypeDevice) {
@@ -321,6 +322,12 @@ int kv4_dequantize_debug(kv4_cache* c, int32_t layer, int32_t seq_id, int32_t st
 int kv4_get_status(kv4_cache* c, kv4_stream_t stream, int32_t* device_status) {
   if (!c || c->bf16) return KV4_ERR_INVALID_ARG;
   return get_status(c, reinterpret_cast<cudaStream_t>(stream), device_status);
+}
+
+int kv4_test_stall_next_attention(kv4_cache* c, int32_t stage) {
+  if (!c || c->bf16) return KV4_ERR_INVALID_ARG;
+  c->test_stall = stage < 0 ? -1 : stage;
+  return KV4_OK;
 }
 
 int kv4_set_attention_events(kv4_cache* c, void* ev_before, void* ev_after) {

@@ -546,9 +546,13 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
           const int s = jl % NS;
           lane_ok = mbar_wait(empty0 + 8 * s, ((jl / NS) & 1) ^ 1, abort_flag, status);
           if (lane_ok) {
-            mbar_arrive_expect_tx(full0 + 8 * s, bytes);
-            bulk_g2s(smem_u32(ring + static_cast<size_t>(s) * C::STAGE), src, bytes, full0 + 8 * s);
-            misc->last_fill[s] = static_cast<int>(jl);
+            // test hook (kv4_test_stall_next_attention): the first CTA leaves one stage unfilled, so its
+            // consumers' bounded wait runs out
+            if (c != 0 || static_cast<int>(jl) != p.stall_stage) {
+              mbar_arrive_expect_tx(full0 + 8 * s, bytes);
+              bulk_g2s(smem_u32(ring + static_cast<size_t>(s) * C::STAGE), src, bytes, full0 + 8 * s);
+              misc->last_fill[s] = static_cast<int>(jl);
+            }
           } else {
             *abort_flag = 1;
           }
@@ -572,8 +576,9 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
       if (lane == 0 && ok) { segq[slot].n = -1; mbar_arrive(iqf0 + 8 * slot); }
       ok = __shfl_sync(0xffffffffu, ok, 0);
     }
-    if (!ok && lane == 0) {
-      // let the copies in flight land before the CTA's shared memory goes away
+    if (lane == 0) {
+      // let every copy this warp issued land before it exits: consumers that gave up a wait may have left
+      // the CTA already, and its shared memory must not go away under a copy in flight
       for (int st = 0; st < NS; ++st)
         if (misc->last_fill[st] >= 0) {
           const uint64_t t0 = globaltimer_ns();
@@ -922,6 +927,8 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   p.grid = g_grid(c);
   p.cap_parts = p.grid * 2 * GWR;
   p.ns = c->gattn_ring;
+  p.stall_stage = c->test_stall;   // test hook, for this launch only
+  c->test_stall = -1;
   if (step) {
     // fused decode step: the append and the query operands first; the attention
     // kernel then starts in plain stream order (it plans from the new lengths)

@@ -114,6 +114,7 @@ struct AttnParams {
   size_t pool_bytes, prot_bytes, qblob_total;   // extents, for the self-checks of debug builds
   int ns;                     // shared-memory ring depth of the attention kernel
   int grid;                   // CTAs of the page-major attention kernel
+  int stall_stage;            // test hook: stage the first CTA leaves unfilled (-1: none)
 };
 
 // Row of q (and of the output) that operand column c of KV head h of batch
@@ -432,6 +433,7 @@ struct kv4_cache {
   kv4::RopeParams rope;      // registered RoPE table (cs == nullptr: none)
   cudaEvent_t ev_before;     // optional timing events around the split-K kernel
   cudaEvent_t ev_after;
+  int test_stall;            // kv4_test_stall_next_attention: stage to leave unfilled in the next call (-1: none)
 };
 
 namespace kv4 {
