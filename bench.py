@@ -389,7 +389,8 @@ def measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=1, compare
 
     # ---- e2e through the public API with host buffers: each step copies every layer's new K, V and q from
     # pinned host memory (one transfer per layer, on a copy stream, ahead of the layer that reads it) and every
-    # layer's output back to pinned host memory (on a second copy stream, behind the layer that writes it)
+    # layer's output back to pinned host memory (on a second copy stream, behind the layer that writes it).
+    # The device staging buffers are doubled (step parity), so the copies of step j+1 overlap step j.
     e2e = None
     if K_e2e:
         kv_el, q_el = B * Hkv * D, B * Hq * D
@@ -401,45 +402,47 @@ def measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=1, compare
                 hin[j, layer, kv_el:2 * kv_el].copy_(rep.steps_v[layer][used + j].reshape(-1))
                 hin[j, layer, 2 * kv_el:].copy_(rep.qs[layer][j % (W_ + K)].reshape(-1))
         hout = torch.empty((K_e2e, layers, B, Hq, D), dtype=torch.bfloat16).pin_memory()
-        din = torch.empty((layers, per), dtype=torch.bfloat16, device=device)
-        dout = torch.empty((layers, B, Hq, D), dtype=torch.bfloat16, device=device)
+        din = torch.empty((2, layers, per), dtype=torch.bfloat16, device=device)
+        dout = torch.empty((2, layers, B, Hq, D), dtype=torch.bfloat16, device=device)
         h2d, d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
-        ready = [torch.cuda.Event() for _ in range(layers)]
-        consumed = [torch.cuda.Event() for _ in range(layers)]
-        written = [torch.cuda.Event() for _ in range(layers)]
-        drained = [torch.cuda.Event() for _ in range(layers)]
+        ready = [[torch.cuda.Event() for _ in range(layers)] for _ in range(2)]
+        consumed = [[torch.cuda.Event() for _ in range(layers)] for _ in range(2)]
+        written = [[torch.cuda.Event() for _ in range(layers)] for _ in range(2)]
+        drained = [[torch.cuda.Event() for _ in range(layers)] for _ in range(2)]
         e0, e1 = ev(), ev()
         barrier()
         e0.record(stream)
         h2d.wait_event(e0)
         d2h.wait_event(e0)
         for j in range(K_e2e):
+            b = j & 1                                        # staging slot of this step
             for layer in range(layers):
                 with torch.cuda.stream(h2d):
-                    if j:
-                        h2d.wait_event(consumed[layer])      # the previous step's layer has read din[layer]
-                    din[layer].copy_(hin[j, layer], non_blocking=True)
-                    ready[layer].record(h2d)
+                    if j >= 2:
+                        h2d.wait_event(consumed[b][layer])   # step j-2 has read this slot of the layer
+                    din[b, layer].copy_(hin[j, layer], non_blocking=True)
+                    ready[b][layer].record(h2d)
             for layer in range(layers):
-                stream.wait_event(ready[layer])
-                if j:
-                    stream.wait_event(drained[layer])        # the previous output of this layer is on the host
-                dk = din[layer, :kv_el].view(B, Hkv, D)
-                dv = din[layer, kv_el:2 * kv_el].view(B, Hkv, D)
-                dq = din[layer, 2 * kv_el:].view(B, Hq, D)
+                stream.wait_event(ready[b][layer])
+                if j >= 2:
+                    stream.wait_event(drained[b][layer])     # step j-2's output of the layer is on the host
+                dk = din[b, layer, :kv_el].view(B, Hkv, D)
+                dv = din[b, layer, kv_el:2 * kv_el].view(B, Hkv, D)
+                dq = din[b, layer, 2 * kv_el:].view(B, Hq, D)
                 if two:
                     cache.append(layer, rep.seq_ids, rep.cu_one, dk, dv, total_new=B, rope=rope)
-                    cache.attention(layer, rep.seq_ids, dq, out=dout[layer], workspace=ws, mode=amode)
+                    cache.attention(layer, rep.seq_ids, dq, out=dout[b, layer], workspace=ws, mode=amode)
                 else:
-                    cache.decode_step(layer, rep.seq_ids, dk, dv, dq, out=dout[layer], workspace=ws, mode=amode)
-                consumed[layer].record(stream)
-                written[layer].record(stream)
+                    cache.decode_step(layer, rep.seq_ids, dk, dv, dq, out=dout[b, layer], workspace=ws, mode=amode)
+                consumed[b][layer].record(stream)
+                written[b][layer].record(stream)
                 with torch.cuda.stream(d2h):
-                    d2h.wait_event(written[layer])
-                    hout[j, layer].copy_(dout[layer], non_blocking=True)
-                    drained[layer].record(d2h)
-        for layer in range(layers):
-            stream.wait_event(drained[layer])
+                    d2h.wait_event(written[b][layer])
+                    hout[j, layer].copy_(dout[b, layer], non_blocking=True)
+                    drained[b][layer].record(d2h)
+        for b in range(min(2, K_e2e)):
+            for layer in range(layers):
+                stream.wait_event(drained[b][layer])
         e1.record(stream)
         barrier()
         t_e2e = e0.elapsed_time(e1) / 1e3
@@ -703,7 +706,8 @@ def run_gpu(args):
                          "ms_per_step": round(t_e2e_all / e2e["steps"] * 1e3, 4),
                          "how": "per layer: new K, V and q copied from pinned host memory on a copy stream ahead "
                                 "of the layer, the layer's output copied to pinned host memory on a second copy "
-                                "stream behind it; one CUDA-event pair around all steps"} if e2e else None),
+                                "stream behind it, device staging doubled so the copies of a step overlap the "
+                                "previous step; one CUDA-event pair around all steps"} if e2e else None),
                 # per layer: gstep_kernel, gattn_kernel, gmerge_kernel (two calls: append, gq, gattn, gmerge)
                 "gpu_launches": launches * K,
                 "clocks": clk,
