@@ -40,6 +40,10 @@
 // start in its range sit in the split, for that merge.
 #include "kv4_attn_tiles.cuh"
 #include "kv4_append_ops.cuh"
+#include "kv4_tc.cuh"
+
+#include <stdlib.h>
+#include <string.h>
 
 namespace kv4 {
 
@@ -305,7 +309,13 @@ __global__ void __launch_bounds__(32 * QWARPS) gq_kernel(AttnParams p) {
   if (gw >= p.n_seqs * p.Hkv) return;
   QFrag<D> qf;
   load_qfrag<D>(p, gw / p.Hkv, gw % p.Hkv, lane, qf);
-  store_qblob<D>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D), qf, lane);
+  uint8_t* blob = p.qblob + static_cast<size_t>(gw) * qblob_bytes(D);
+  if constexpr (D == 128) {
+    if (p.qfmt) store_qblob_tc<D>(blob, qf, lane);
+    else store_qblob<D>(blob, qf, lane);
+  } else {
+    store_qblob<D>(blob, qf, lane);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -362,7 +372,13 @@ __global__ void __launch_bounds__(32 * MAXW) gstep_kernel(AttnParams p, AppendPa
   if (tensor == 1) {   // the query operands of head h (independent of the append)
     QFrag<D> qf;
     load_qfrag<D>(p, b, h, lane, qf, s_ok ? L + 1 : L);
-    store_qblob<D>(p.qblob + (static_cast<size_t>(b) * p.Hkv + h) * qblob_bytes(D), qf, lane);
+    uint8_t* blob = p.qblob + (static_cast<size_t>(b) * p.Hkv + h) * qblob_bytes(D);
+    if constexpr (D == 128) {
+      if (p.qfmt) store_qblob_tc<D>(blob, qf, lane);
+      else store_qblob<D>(blob, qf, lane);
+    } else {
+      store_qblob<D>(blob, qf, lane);
+    }
   }
   if (s_ok && page >= 0) {
     const long long tile_idx = (static_cast<long long>(page) * (p.P / TILE) + (L % p.P) / TILE) * p.Hkv + h;
@@ -402,46 +418,25 @@ __device__ __forceinline__ const uint8_t* stage_source(const AttnParams& p, cons
                       tile8_bytes(D);
 }
 
-// PAIR = INT4 tiles per iteration of a consumer warp (1, 2 or 4).  MULTI:
-// several query tokens per sequence (causal visibility per operand column);
-// the one-token variant carries none of that code.  GWR: KV heads per group.
-template <int D, int PAIR, bool MULTI, int GWR>
-__global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
-  using C = GCfg<D, GWR>;
-  using SH = GShape<GWR>;
-  constexpr int GTHREADS = SH::THREADS;
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int NS = p.ns;
-  uint8_t* ring = smem;
-  SegQ* segq = reinterpret_cast<SegQ*>(ring + static_cast<size_t>(NS) * C::STAGE);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(segq + GQD);
-  GMisc* misc = reinterpret_cast<GMisc*>(bars + 2 * NS + 2 * GQD);
-  volatile int* abort_flag = &misc->abort;
-  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * NS;
-  const uint32_t iqf0 = full0 + 16 * NS, iqe0 = iqf0 + 8 * GQD;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int* status = &p.state->status;
-  const int c = blockIdx.x;
+// The CTA's share of the stream-K split.  Every CTA derives the same plan
+// from the sequence lengths: the costs of all head groups (a block scan) give
+// T, and CTA c takes units [c*T/N, (c+1)*T/N).  Group i spans
+// [S_i, S_i + GROUP_COST + n_i) in cost units; its stage u sits at
+// S_i + GROUP_COST + u.  The CTA whose range holds a group's start records the
+// group in `plan` (for the merge kernel), CTA 0 the totals; empty sequences get
+// zero rows.  misc->first = the group holding the CTA's first unit.  Called by
+// every thread of the block; returns whether the CTA has stages to stream.
+template <int GWR>
+__device__ bool plan_share(const AttnParams& p, GPlanRec* plan, GMisc* misc, int c, int tid, int nthreads,
+                           long long& T_out, long long& N_out, int& j0_out, int& j1_out) {
   const int HGN = p.Hkv / GWR, n_groups = p.n_seqs * HGN;
-
-  // the merge kernel may be scheduled now: it waits for this grid before reading its results
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (tid == 0) {
-    for (int s = 0; s < NS; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, GWR); }
-    for (int s = 0; s < GQD; ++s) { mbar_init(iqf0 + 8 * s, 1); mbar_init(iqe0 + 8 * s, GWR); }
-    misc->abort = 0;
-    misc->n_empty = 0;
-    for (int s = 0; s < MAX_NS; ++s) misc->last_fill[s] = -1;
-    fence_barrier_init();
-  }
-
   // ---- plan (every CTA the same): costs of all head groups -> T, then the
   // stream-K range [j0, j1) of this CTA and the group holding j0.  Group i
   // spans [S_i, S_i + GROUP_COST + n_i) in cost units; its stage u sits at
   // S_i + GROUP_COST + u.
   Group my_g{};
   int my_start = 0, T = 0;
-  for (int c0 = 0; c0 < n_groups; c0 += GTHREADS) {
+  for (int c0 = 0; c0 < n_groups; c0 += nthreads) {
     const int i = c0 + tid;
     Group gd{};
     if (i < n_groups) gd = describe(p, i, HGN, c == 0);
@@ -474,11 +469,11 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
       }
     }
   };
-  if (n_groups <= GTHREADS) {
+  if (n_groups <= nthreads) {
     visit(tid, my_g, my_start);
   } else {
     int base = 0;
-    for (int c0 = 0; c0 < n_groups; c0 += GTHREADS) {
+    for (int c0 = 0; c0 < n_groups; c0 += nthreads) {
       const int i = c0 + tid;
       Group gd{};
       if (i < n_groups) gd = describe(p, i, HGN, false);
@@ -496,96 +491,150 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
   __syncthreads();
   {
     const int ne = min(misc->n_empty, 32);
-    for (int e = 0; e < ne; ++e) zero_group<GWR>(p, misc->empty[e], tid, GTHREADS);
+    for (int e = 0; e < ne; ++e) zero_group<GWR>(p, misc->empty[e], tid, nthreads);
   }
-  if (zero_all || c >= N || j0 >= j1) {
-    return;
+  T_out = T;
+  N_out = N;
+  j0_out = j0;
+  j1_out = j1;
+  return !(zero_all || c >= N || j0 >= j1);
+}
+
+// The producer warp of a CTA: walks the CTA's range [j0, j1) of the split,
+// queues one segment descriptor per head group it touches, and issues the
+// group's stages as 1-D bulk copies into the shared-memory ring (each lane one
+// stage of a batch, mbarrier completion).  Consumers release a stage once per
+// group of consumers (the empty barriers count GWR arrivals).  Every wait is
+// bounded; before the warp exits, every copy it issued has landed.
+template <int D, int GWR>
+__device__ void produce(const AttnParams& p, GMisc* misc, SegQ* segq, uint8_t* ring, int NS, uint32_t full0,
+                        uint32_t empty0, uint32_t iqf0, uint32_t iqe0, int c, int j0, int j1, long long T, long long N,
+                        int lane, volatile int* abort_flag, int* status) {
+  using C = GCfg<D, GWR>;
+  const int HGN = p.Hkv / GWR;
+  // ------------------------------------------------------------ producer
+  const int nbatch = NS < 32 ? NS : 32;
+  Group g = misc->first;
+  int gi = g.b * HGN + g.hg;
+  int j = j0;        // position in cost units
+  uint32_t jj = 0;   // CTA-local stage counter
+  int q = 0;
+  bool ok = true;
+  while (j < j1 && ok) {
+    const int gst = group_stages<GWR>(g);
+    const int a = g.start + GROUP_COST, e = a + gst;   // the group's stages in cost units
+    if (a >= j1) break;                                // only its start cost falls in this range
+    const int u = max(j, a) - a;
+    const int n = min(e, j1) - max(j, a);
+    const int slot = q % GQD;
+    if (lane == 0) ok = mbar_wait(iqe0 + 8 * slot, ((q / GQD) & 1) ^ 1, abort_flag, status);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) break;
+    if (lane == 0) {
+      SegQ sq;
+      sq.g = g;
+      sq.u0 = u;
+      sq.n = n;
+      const int cf = cta_of(a, T, N);
+      sq.k = c - cf;
+      sq.nseg = cta_of(e - 1, T, N) - cf + 1;
+      segq[slot] = sq;
+      mbar_arrive(iqf0 + 8 * slot);
+    }
+    // the next group's descriptor (its loads overlap the copies below)
+    int gn = gi + 1;
+    Group nxt{};
+    if (e < j1) nxt = describe(p, gn, HGN, false);
+    // stages u .. u+n-1: one lane per stage, batches of at most NS stages
+    for (int base = 0; base < n; base += nbatch) {
+      bool lane_ok = true;
+      if (lane < nbatch && base + lane < n) {
+        uint32_t bytes;
+        const uint8_t* src = stage_source<D, GWR>(p, g, u + base + lane, bytes);
+        const uint32_t jl = jj + base + lane;
+        const int s = jl % NS;
+        lane_ok = mbar_wait(empty0 + 8 * s, ((jl / NS) & 1) ^ 1, abort_flag, status);
+        if (lane_ok) {
+          // test hook (kv4_test_stall_next_attention): the first CTA leaves one stage unfilled, so its
+          // consumers' bounded wait runs out
+          if (c != 0 || static_cast<int>(jl) != p.stall_stage) {
+            mbar_arrive_expect_tx(full0 + 8 * s, bytes);
+            bulk_g2s(smem_u32(ring + static_cast<size_t>(s) * C::STAGE), src, bytes, full0 + 8 * s);
+            misc->last_fill[s] = static_cast<int>(jl);
+          }
+        } else {
+          *abort_flag = 1;
+        }
+      }
+      ok = __all_sync(0xffffffffu, lane_ok);
+      if (!ok) break;
+    }
+    jj += n;
+    j = e;
+    ++q;
+    if (j < j1 && ok) {
+      while (group_stages<GWR>(nxt) == 0) nxt = describe(p, ++gn, HGN, false);   // empty sequences own no stage
+      nxt.start = e;
+      gi = gn;
+      g = nxt;
+    }
+  }
+  if (ok) {
+    const int slot = q % GQD;
+    if (lane == 0) ok = mbar_wait(iqe0 + 8 * slot, ((q / GQD) & 1) ^ 1, abort_flag, status);
+    if (lane == 0 && ok) { segq[slot].n = -1; mbar_arrive(iqf0 + 8 * slot); }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+  }
+  if (lane == 0) {
+    // let every copy this warp issued land before it exits: consumers that gave up a wait may have left
+    // the CTA already, and its shared memory must not go away under a copy in flight
+    for (int st = 0; st < NS; ++st)
+      if (misc->last_fill[st] >= 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(full0 + 8 * st, (misc->last_fill[st] / NS) & 1) &&
+               globaltimer_ns() - t0 < 1000000000ull) {}
+      }
+  }
+}
+
+// PAIR = INT4 tiles per iteration of a consumer warp (1, 2 or 4).  MULTI:
+// several query tokens per sequence (causal visibility per operand column);
+// the one-token variant carries none of that code.  GWR: KV heads per group.
+template <int D, int PAIR, bool MULTI, int GWR>
+__global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
+  using C = GCfg<D, GWR>;
+  using SH = GShape<GWR>;
+  constexpr int GTHREADS = SH::THREADS;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int NS = p.ns;
+  uint8_t* ring = smem;
+  SegQ* segq = reinterpret_cast<SegQ*>(ring + static_cast<size_t>(NS) * C::STAGE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(segq + GQD);
+  GMisc* misc = reinterpret_cast<GMisc*>(bars + 2 * NS + 2 * GQD);
+  volatile int* abort_flag = &misc->abort;
+  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * NS;
+  const uint32_t iqf0 = full0 + 16 * NS, iqe0 = iqf0 + 8 * GQD;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int* status = &p.state->status;
+  const int c = blockIdx.x;
+
+  // the merge kernel may be scheduled now: it waits for this grid before reading its results
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, GWR); }
+    for (int s = 0; s < GQD; ++s) { mbar_init(iqf0 + 8 * s, 1); mbar_init(iqe0 + 8 * s, GWR); }
+    misc->abort = 0;
+    misc->n_empty = 0;
+    for (int s = 0; s < MAX_NS; ++s) misc->last_fill[s] = -1;
+    fence_barrier_init();
   }
 
+  long long T = 0, N = 0;
+  int j0 = 0, j1 = 0;
+  if (!plan_share<GWR>(p, plan, misc, c, tid, GTHREADS, T, N, j0, j1)) return;
+
   if (warp == GWR) {
-    // ------------------------------------------------------------ producer
-    const int nbatch = NS < 32 ? NS : 32;
-    Group g = misc->first;
-    int gi = g.b * HGN + g.hg;
-    int j = j0;        // position in cost units
-    uint32_t jj = 0;   // CTA-local stage counter
-    int q = 0;
-    bool ok = true;
-    while (j < j1 && ok) {
-      const int gst = group_stages<GWR>(g);
-      const int a = g.start + GROUP_COST, e = a + gst;   // the group's stages in cost units
-      if (a >= j1) break;                                // only its start cost falls in this range
-      const int u = max(j, a) - a;
-      const int n = min(e, j1) - max(j, a);
-      const int slot = q % GQD;
-      if (lane == 0) ok = mbar_wait(iqe0 + 8 * slot, ((q / GQD) & 1) ^ 1, abort_flag, status);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      if (lane == 0) {
-        SegQ sq;
-        sq.g = g;
-        sq.u0 = u;
-        sq.n = n;
-        const int cf = cta_of(a, T, N);
-        sq.k = c - cf;
-        sq.nseg = cta_of(e - 1, T, N) - cf + 1;
-        segq[slot] = sq;
-        mbar_arrive(iqf0 + 8 * slot);
-      }
-      // the next group's descriptor (its loads overlap the copies below)
-      int gn = gi + 1;
-      Group nxt{};
-      if (e < j1) nxt = describe(p, gn, HGN, false);
-      // stages u .. u+n-1: one lane per stage, batches of at most NS stages
-      for (int base = 0; base < n; base += nbatch) {
-        bool lane_ok = true;
-        if (lane < nbatch && base + lane < n) {
-          uint32_t bytes;
-          const uint8_t* src = stage_source<D, GWR>(p, g, u + base + lane, bytes);
-          const uint32_t jl = jj + base + lane;
-          const int s = jl % NS;
-          lane_ok = mbar_wait(empty0 + 8 * s, ((jl / NS) & 1) ^ 1, abort_flag, status);
-          if (lane_ok) {
-            // test hook (kv4_test_stall_next_attention): the first CTA leaves one stage unfilled, so its
-            // consumers' bounded wait runs out
-            if (c != 0 || static_cast<int>(jl) != p.stall_stage) {
-              mbar_arrive_expect_tx(full0 + 8 * s, bytes);
-              bulk_g2s(smem_u32(ring + static_cast<size_t>(s) * C::STAGE), src, bytes, full0 + 8 * s);
-              misc->last_fill[s] = static_cast<int>(jl);
-            }
-          } else {
-            *abort_flag = 1;
-          }
-        }
-        ok = __all_sync(0xffffffffu, lane_ok);
-        if (!ok) break;
-      }
-      jj += n;
-      j = e;
-      ++q;
-      if (j < j1 && ok) {
-        while (group_stages<GWR>(nxt) == 0) nxt = describe(p, ++gn, HGN, false);   // empty sequences own no stage
-        nxt.start = e;
-        gi = gn;
-        g = nxt;
-      }
-    }
-    if (ok) {
-      const int slot = q % GQD;
-      if (lane == 0) ok = mbar_wait(iqe0 + 8 * slot, ((q / GQD) & 1) ^ 1, abort_flag, status);
-      if (lane == 0 && ok) { segq[slot].n = -1; mbar_arrive(iqf0 + 8 * slot); }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-    }
-    if (lane == 0) {
-      // let every copy this warp issued land before it exits: consumers that gave up a wait may have left
-      // the CTA already, and its shared memory must not go away under a copy in flight
-      for (int st = 0; st < NS; ++st)
-        if (misc->last_fill[st] >= 0) {
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(full0 + 8 * st, (misc->last_fill[st] / NS) & 1) &&
-                 globaltimer_ns() - t0 < 1000000000ull) {}
-        }
-    }
+    produce<D, GWR>(p, misc, segq, ring, NS, full0, empty0, iqf0, iqe0, c, j0, j1, T, N, lane, abort_flag, status);
     return;
   }
 
@@ -857,6 +906,518 @@ __global__ void __launch_bounds__(32 * MWARPS) gmerge_kernel(AttnParams p, const
 }
 
 // ---------------------------------------------------------------------------
+// The attention kernel on the fifth-generation tensor cores (tcgen05, operands
+// and accumulators in tensor memory), for 4-KV-head groups at D = 128 and one
+// query token.  Same split, producer warp, stage ring and merge kernel as
+// gattn_kernel; one CTA per SM with four consumer warpgroups, warpgroup h
+// handling KV head h of every stage, 128 tokens (8 tiles) per block:
+//   K phase   thread i = token i of the block: its 128 K codes as bytes
+//             (INT4 nibbles unpacked; INT8 rows as stored) to TMEM lane i;
+//   scores    16 multiplies M=128 tokens x N=8 x K=32 (kind::i8, A = codes in
+//             TMEM, B = the two 8-bit planes of the rotated query in shared
+//             memory) -> int32 scores in TMEM, one token per thread;
+//   softmax   per token and query head, no column duplicates; the running max
+//             is kept per warpgroup and moved only when a score passes it by
+//             more than TAU (a vote), so most blocks need no reduction;
+//   weights   w = p * s_V as 32-bit fixed point (F = 2^(32-TAU) / s_ref, s_ref
+//             an upper bound of the V scales seen), stored as 4 bytes per
+//             head: the four byte planes of 4 heads are the N = 16 columns;
+//   V phase   thread i = dim i: its 16 codes of every tile as bytes to TMEM;
+//   P.V       4 multiplies M=128 dims x N=16 x K=32 tokens (kind::i8) into an
+//             exact int32 accumulator in TMEM, folded into fp32 per-dim sums
+//             only when the max or s_ref moves and at the end of a segment.
+// The zero points enter through sum_p p z (exact fp32 per token) and the scale
+// of K through the per-token factor of the integer score, as in the folded
+// form of the other kernels.
+
+constexpr int TC_WG = 4;                           // consumer warpgroups = KV heads of a group
+constexpr int TC_THREADS = 32 * (4 * TC_WG + 1);   // + producer warp
+constexpr int TC_BLOCK = 8;                        // 16-token tiles per block (128 tokens = TMEM lanes)
+constexpr uint32_t TC_COLS = 512;                  // TMEM columns of the CTA, 128 per warpgroup
+constexpr uint32_t TC_AK = 0;                      // QK A operand: 128 tokens x 128 code bytes (32 columns)
+constexpr uint32_t TC_S = 32;                      // scores: hi query plane 32..39, lo plane 40..47
+constexpr uint32_t TC_AV = 48;                     // P.V A operands, two buffers of 32 columns
+constexpr uint32_t TC_O = 112;                     // P.V accumulator: 4 heads x 4 byte planes
+constexpr int TC_QB = 2048;                        // query planes: hi 1 KB, lo 1 KB (K-major, N = 8)
+constexpr int TC_PB = 2048;                        // one weight buffer: 128 tokens x 16 bytes (MN-major)
+constexpr int TC_SCR = 2048;                       // reduction / rotation scratch
+constexpr int TC_WGSMEM = TC_QB + 2 * TC_PB + TC_SCR;
+constexpr float TC_TAU = 2.f;                      // allowed excess of a score over the running max (log2)
+constexpr int TC_FLUSH_BLOCKS = 512;               // fold the int32 accumulator at least every 65536 tokens
+constexpr uint32_t TC_IDESC_QK_HI = tc::idesc_i8(8, true, false);
+constexpr uint32_t TC_IDESC_QK_LO = tc::idesc_i8(8, false, false);
+constexpr uint32_t TC_IDESC_PV = tc::idesc_i8(16, false, true);
+
+template <int D>
+__host__ __device__ inline size_t tattn_smem_bytes(int ns) {
+  using C = GCfg<D, 4>;
+  size_t off = static_cast<size_t>(ns) * C::STAGE + GQD * sizeof(SegQ) + (2 * ns + 2 * GQD) * sizeof(uint64_t) +
+               sizeof(GMisc);
+  off = (off + 127) & ~static_cast<size_t>(127);
+  return off + TC_WG * TC_WGSMEM + 3 * TC_WG * sizeof(uint64_t) + 64;
+}
+
+__device__ __forceinline__ void wg_sync(int h) { asm volatile("bar.sync %0, 128;" ::"r"(1 + h) : "memory"); }
+// Warpgroup barrier that also ANDs a predicate over its 128 threads: every exit decision after a bounded
+// wait is taken here, the same for the whole warpgroup, so no thread leaves while others wait at a barrier.
+__device__ __forceinline__ bool wg_and(int h, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbarrier.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(1 + h)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 6, 512;" ::: "memory"); }
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+__device__ __forceinline__ uint32_t f2u_sat(float x) {
+  uint32_t r;
+  asm("cvt.rni.sat.u32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float fold_planes(const uint32_t* o) {   // 4 byte planes (lowest first) of one head
+  return fmaf(static_cast<float>(static_cast<int>(o[3])), 16777216.f,
+              fmaf(static_cast<float>(static_cast<int>(o[2])), 65536.f,
+                   fmaf(static_cast<float>(static_cast<int>(o[1])), 256.f, static_cast<float>(static_cast<int>(o[0])))));
+}
+// Row of the weight buffer (= A column order) of token r of a tile: the V codes of a tile come out of
+// the stored words in the token order 0, 8, 1, 9, 2, 10, ... (word t gives tokens 2t, 8+2t, 2t+1, 9+2t).
+__device__ __forceinline__ int tc_row_of(int r) { return 4 * ((r & 7) >> 1) + 2 * (r & 1) + (r >> 3); }
+
+template <int D>
+__global__ void __launch_bounds__(TC_THREADS, 1) tattn_kernel(AttnParams p, GPlanRec* plan) {
+  static_assert(D == 128, "the tensor-memory kernel covers D = 128");
+  using C = GCfg<D, 4>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int NS = p.ns;
+  uint8_t* ring = smem;
+  SegQ* segq = reinterpret_cast<SegQ*>(ring + static_cast<size_t>(NS) * C::STAGE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(segq + GQD);
+  GMisc* misc = reinterpret_cast<GMisc*>(bars + 2 * NS + 2 * GQD);
+  size_t off = static_cast<size_t>(reinterpret_cast<uint8_t*>(misc + 1) - smem);
+  off = (off + 127) & ~static_cast<size_t>(127);
+  uint8_t* wgbase = smem + off;
+  uint64_t* tbars = reinterpret_cast<uint64_t*>(wgbase + TC_WG * TC_WGSMEM);   // per warpgroup: scores, P.V x2
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tbars + 3 * TC_WG);
+  int* flags = reinterpret_cast<int*>(tmem_slot + 2);                          // per warpgroup: 2 words
+  volatile int* abort_flag = &misc->abort;
+  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * NS;
+  const uint32_t iqf0 = full0 + 16 * NS, iqe0 = iqf0 + 8 * GQD;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int* status = &p.state->status;
+  const int c = blockIdx.x;
+
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, TC_WG); }
+    for (int s = 0; s < GQD; ++s) { mbar_init(iqf0 + 8 * s, 1); mbar_init(iqe0 + 8 * s, TC_WG); }
+    for (int i = 0; i < 3 * TC_WG; ++i) mbar_init(smem_u32(tbars + i), 1);
+    for (int i = 0; i < 2 * TC_WG; ++i) flags[i] = 0;
+    misc->abort = 0;
+    misc->n_empty = 0;
+    for (int s = 0; s < MAX_NS; ++s) misc->last_fill[s] = -1;
+    fence_barrier_init();
+  }
+
+  long long T = 0, N = 0;
+  int j0 = 0, j1 = 0;
+  if (!plan_share<4>(p, plan, misc, c, tid, TC_THREADS, T, N, j0, j1)) return;
+
+  if (warp == 4 * TC_WG) {
+    produce<D, 4>(p, misc, segq, ring, NS, full0, empty0, iqf0, iqe0, c, j0, j1, T, N, lane, abort_flag, status);
+    return;
+  }
+
+  // ---------------------------------------------------------------- consumers
+  const int h = warp >> 2, wt = tid & 127;
+  if (warp == 0) {
+    tc::alloc(smem_u32(tmem_slot), TC_COLS);
+    tc::relinquish();
+  }
+  tc::fence_before();
+  consumers_sync();
+  tc::fence_after();
+  const uint32_t tcol = *tmem_slot + 128u * static_cast<uint32_t>(h);                 // lane 0 (multiplies)
+  const uint32_t tlane = tcol + (static_cast<uint32_t>(32 * (warp & 3)) << 16);     // this warp's lanes
+  uint8_t* wgs = wgbase + h * TC_WGSMEM;
+  const uint32_t qB = smem_u32(wgs), PB = qB + TC_QB;
+  float* scratch = reinterpret_cast<float*>(wgs + TC_QB + 2 * TC_PB);
+  const uint32_t sbar = smem_u32(tbars + 3 * h), pvbar0 = sbar + 8;
+  int* myflags = flags + 2 * h;
+  constexpr int HS = head_stride(D);
+  const int pstride = partial_stride(p.G, D);
+  const float NEGINF = -INFINITY;
+
+  uint32_t s = 0, par = 0;   // ring position of the next stage and its fill parity
+  uint32_t nb = 0;           // blocks issued by this warpgroup (phases of its tensor-core barriers)
+  uint32_t n_qk = 0, n_pv = 0;   // tensor-core commits issued on the score and P.V barriers
+  bool ok = true;
+  for (int q = 0; ok; ++q) {
+    const int slot = q % GQD;
+    ok = mbar_wait(iqf0 + 8 * slot, (q / GQD) & 1, abort_flag, status);
+    const SegQ sq = segq[slot];
+    ok = wg_and(h, ok);
+    if (!ok) break;
+    if (wt == 0) mbar_arrive(iqe0 + 8 * slot);
+    if (sq.n < 0) break;
+    const Group g = sq.g;
+    if (q == 0) asm volatile("griddepcontrol.wait;" ::: "memory");   // the query operands are written
+    const int hkv = g.hg * 4 + h;
+    const uint8_t* blob = p.qblob + static_cast<size_t>(g.b * p.Hkv + hkv) * qblob_bytes(D);
+    {
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(blob) + wt);   // 128 threads x 16 B = both planes
+      sts128(qB + 16 * wt, v.x, v.y, v.z, v.w);
+    }
+    const float* tail = reinterpret_cast<const float*>(blob + 16 * D);
+    float qs[4];
+#pragma unroll
+    for (int hh = 0; hh < 4; ++hh) qs[hh] = __ldcg(tail + hh);
+    const float kscale = __ldcg(tail + MAX_G);
+    fence_proxy_async_smem();   // the planes are read by the tensor cores
+
+    float m[4], l[4], zs[4], oacc[4];
+#pragma unroll
+    for (int hh = 0; hh < 4; ++hh) { m[hh] = NEGINF; l[hh] = 0.f; zs[hh] = 0.f; oacc[hh] = 0.f; }
+    float sref = 0.f, F = 0.f;
+    bool ostarted = false;
+    int since_fold = 0;
+
+    int u = sq.u0;
+    const int u_end = sq.u0 + sq.n;
+    while (u < u_end) {
+      // ---- the next block: up to 8 tiles of this head, and the stages they span
+      uint32_t ts[TC_BLOCK];
+      int tp[TC_BLOCK];
+      uint32_t tk = 0;   // bit i: tile i is INT8
+      int nt = 0, nst = 0;
+      const uint32_t s_first = s;
+      while (u < u_end && nt < TC_BLOCK) {
+        const bool int8 = u >= g.n4;
+        const int v = u - g.n4;
+        if (!int8 || (v & 1) == (h >> 1)) {
+          ts[nt] = s;
+          tp[nt] = int8 ? (v >> 1) * TILE : (g.t0 + u) * TILE;
+          if (int8) tk |= 1u << nt;
+          ++nt;
+        }
+        if (ok && !mbar_wait(full0 + 8 * s, par, abort_flag, status)) ok = false;
+        if (++s == static_cast<uint32_t>(NS)) { s = 0; par ^= 1u; }
+        ++nst;
+        ++u;
+      }
+      if (nt == 0) {   // only the other half of a protected tile: hand the stages back
+        ok = wg_and(h, ok);
+        if (!ok) break;
+        if (wt == 0)
+          for (int k = 0, ss = static_cast<int>(s_first); k < nst; ++k, ss = (ss + 1 == NS) ? 0 : ss + 1)
+            mbar_arrive(empty0 + 8 * ss);
+        continue;
+      }
+      const uint32_t buf = nb & 1u;
+
+      // ---- K phase: thread wt = token wt of the block
+      const int it = wt >> 4, r = wt & 15;
+      float sK = 0.f, zK = 0.f, sV = 0.f, zV = 0.f;
+      bool valid = false;
+      {
+        uint32_t kw[32];
+        if (it < nt) {
+          const bool i8 = (tk >> it) & 1u;
+          const uint32_t ta = smem_u32(ring + static_cast<size_t>(ts[it]) * C::STAGE) +
+                              (i8 ? (h & 1) * tile8_bytes(D) : h * tile4_bytes(D));
+          if (!i8) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 w = lds128(ta + r * (D / 2) + 16 * i);
+              kw[8 * i + 0] = w.x & 0x0F0F0F0Fu; kw[8 * i + 1] = (w.x >> 4) & 0x0F0F0F0Fu;
+              kw[8 * i + 2] = w.y & 0x0F0F0F0Fu; kw[8 * i + 3] = (w.y >> 4) & 0x0F0F0F0Fu;
+              kw[8 * i + 4] = w.z & 0x0F0F0F0Fu; kw[8 * i + 5] = (w.z >> 4) & 0x0F0F0F0Fu;
+              kw[8 * i + 6] = w.w & 0x0F0F0F0Fu; kw[8 * i + 7] = (w.w >> 4) & 0x0F0F0F0Fu;
+            }
+            const uint32_t so = ta + 16 * D + 16 * (r & 7) + 4 * (r >> 3);
+            const uint32_t szk = lds32(so), szv = lds32(so + 8);
+            sK = half_lo(szk); zK = half_hi(szk); sV = half_lo(szv); zV = half_hi(szv);
+            const int pos = tp[it] + r;
+            valid = pos >= g.lo4 && pos < g.hi4;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint4 w = lds128(ta + r * D + 16 * i);
+              kw[4 * i + 0] = w.x; kw[4 * i + 1] = w.y; kw[4 * i + 2] = w.z; kw[4 * i + 3] = w.w;
+            }
+            const uint32_t so = ta + 32 * D + 16 * (r & 7) + 4 * (r >> 3);
+            const uint32_t szk = lds32(so), szv = lds32(so + 8);
+            sK = half_lo(szk); zK = half_hi(szk); sV = half_lo(szv); zV = half_hi(szv);
+            valid = tp[it] + r < g.nprot;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) kw[i] = 0u;
+        }
+        tc::st32x32(tlane + TC_AK, kw);
+      }
+      tc::wait_st();
+      tc::fence_before();
+      ok = wg_and(h, ok);                           // the K codes of the block are in TMEM
+      tc::fence_after();
+      if (!ok) break;
+      if (wt == 0) {
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+          tc::mma_i8(tcol + TC_S, tcol + TC_AK + 8 * j, tc::sdesc(qB + 256 * j, 128, 256), TC_IDESC_QK_HI, j > 0);
+          tc::mma_i8(tcol + TC_S + 8, tcol + TC_AK + 8 * j, tc::sdesc(qB + 1024 + 256 * j, 128, 256), TC_IDESC_QK_LO,
+                     j > 0);
+        }
+        tc::commit(sbar);
+      }
+      // ---- V phase: thread wt = dim wt; the buffer's previous multiplies (block nb - 2) must be done
+      if (ok && nb >= 2 && !mbar_wait(pvbar0 + 8 * buf, ((nb - 2) >> 1) & 1u, abort_flag, status)) ok = false;
+      {
+        uint32_t vw[32];
+        const int d = wt, mb = d >> 4, dh = (d >> 3) & 1, gg = d & 7;
+#pragma unroll
+        for (int i = 0; i < TC_BLOCK; ++i) {
+          if (i < nt) {
+            const bool i8 = (tk >> i) & 1u;
+            const uint32_t ta = smem_u32(ring + static_cast<size_t>(ts[i]) * C::STAGE) +
+                                (i8 ? (h & 1) * tile8_bytes(D) : h * tile4_bytes(D));
+            if (!i8) {
+              const uint32_t va = ta + 8 * D + 512 * (mb >> 2) + 64 * gg + 4 * (mb & 3);
+#pragma unroll
+              for (int t = 0; t < 4; ++t) vw[4 * i + t] = (lds32(va + 16 * t) >> (4 * dh)) & 0x0F0F0F0Fu;
+            } else {
+              // words of th = 0 and th = 1 of the pair (w = 2 mb, 2 mb + 1) sit 4 bytes apart
+              const uint32_t va = ta + 16 * D + 16 * (32 * (mb >> 1) + 4 * gg) + 4 * (2 * (mb & 1));
+              const uint32_t sel = dh ? 0x7351u : 0x6240u;
+#pragma unroll
+              for (int t = 0; t < 4; ++t) vw[4 * i + t] = __byte_perm(lds32(va + 16 * t), lds32(va + 16 * t + 4), sel);
+            }
+          } else {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) vw[4 * i + t] = 0u;
+          }
+        }
+        tc::st32x32(tlane + TC_AV + 32 * buf, vw);
+      }
+      tc::wait_st();   // the V codes are in TMEM (read by the P.V multiplies after the next barrier)
+      ++n_qk;
+      ok = ok && mbar_wait(sbar, nb & 1u, abort_flag, status);
+      tc::fence_after();
+      uint32_t sr[16];
+      if (ok) {
+        tc::ld32x16(tlane + TC_S, sr);
+        tc::wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sr[i] = 0u;
+      }
+
+      // ---- softmax of token wt (4 query heads), weights with the current max and scale
+      const float sKs = sK * kscale;
+      float x[4], pr[4];
+      bool need = since_fold >= TC_FLUSH_BLOCKS;
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh) {
+        x[hh] = valid ? fmaf(static_cast<float>(static_cast<int>(sr[hh]) * 256 + static_cast<int>(sr[8 + hh])), sKs,
+                             zK * qs[hh])
+                      : NEGINF;
+        need |= x[hh] > m[hh] + TC_TAU;
+      }
+      need |= valid && sV > sref;
+      if (__any_sync(0xffffffffu, need) && lane == 0) atomicOr(myflags + (nb & 1u), 1);
+      if (wt == 0) myflags[(nb + 1) & 1u] = 0;   // the next block's flag (last read before this block began)
+      const int row = 16 * it + tc_row_of(r);
+      const uint32_t prow = PB + TC_PB * buf + 16 * row;
+      {
+        const float sVF = sV * F;
+        uint32_t W[4];
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) {
+          pr[hh] = valid ? ex2(x[hh] - m[hh]) : 0.f;
+          W[hh] = valid ? f2u_sat(pr[hh] * sVF) : 0u;
+        }
+        sts128(prow, W[0], W[1], W[2], W[3]);
+      }
+      fence_proxy_async_smem();
+      tc::fence_before();
+      ok = wg_and(h, ok);                           // weights stored, V codes in TMEM, the stages read
+      tc::fence_after();
+      if (!ok) break;
+      if (wt == 0)
+        for (int k = 0, ss = static_cast<int>(s_first); k < nst; ++k, ss = (ss + 1 == NS) ? 0 : ss + 1)
+          mbar_arrive(empty0 + 8 * ss);
+      if (*reinterpret_cast<volatile int*>(myflags + (nb & 1u))) {
+        // ---- rare path (the whole warpgroup): block maxima, new max and fixed-point scale, fold the
+        // accumulator into the fp32 sums in the old scale, then redo this block's weights
+        float bm[5] = {x[0], x[1], x[2], x[3], valid ? sV : 0.f};
+#pragma unroll
+        for (int i = 0; i < 5; ++i)
+#pragma unroll
+          for (int o = 16; o; o >>= 1) bm[i] = fmaxf(bm[i], __shfl_xor_sync(0xffffffffu, bm[i], o));
+        if (lane == 0)
+#pragma unroll
+          for (int i = 0; i < 5; ++i) scratch[8 * (warp & 3) + i] = bm[i];
+        wg_sync(h);
+#pragma unroll
+        for (int i = 0; i < 5; ++i)
+          bm[i] = fmaxf(fmaxf(scratch[i], scratch[8 + i]), fmaxf(scratch[16 + i], scratch[24 + i]));
+        wg_sync(h);
+        float alpha[4];
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) {
+          const float mn = fmaxf(m[hh], bm[hh]);
+          alpha[hh] = (m[hh] == NEGINF) ? 0.f : ex2(m[hh] - mn);
+          m[hh] = mn;
+        }
+        if (ostarted) {
+          const uint32_t pb = (nb - 1) & 1u;
+          ok = wg_and(h, mbar_wait(pvbar0 + 8 * pb, ((nb - 1) >> 1) & 1u, abort_flag, status));
+          if (!ok) break;
+          tc::fence_after();
+          uint32_t o16[16];
+          tc::ld32x16(tlane + TC_O, o16);
+          tc::wait_ld();
+          const float invF = F > 0.f ? 1.f / F : 0.f;
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh) oacc[hh] = fmaf(fold_planes(o16 + 4 * hh), invF, oacc[hh]);
+          ostarted = false;
+        }
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) { oacc[hh] *= alpha[hh]; l[hh] *= alpha[hh]; zs[hh] *= alpha[hh]; }
+        if (2.f * bm[4] > sref) {
+          sref = 2.f * bm[4];
+          F = 1073741824.f / sref;   // 2^(32 - TAU) / s_ref
+        }
+        since_fold = 0;
+        const float sVF = sV * F;
+        uint32_t W[4];
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) {
+          pr[hh] = (valid && m[hh] != NEGINF) ? ex2(x[hh] - m[hh]) : 0.f;
+          W[hh] = valid ? f2u_sat(pr[hh] * sVF) : 0u;
+        }
+        sts128(prow, W[0], W[1], W[2], W[3]);
+        fence_proxy_async_smem();
+        tc::fence_before();
+        wg_sync(h);
+        tc::fence_after();
+      }
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh) { l[hh] += pr[hh]; zs[hh] = fmaf(pr[hh], zV, zs[hh]); }
+      // ---- P.V: 4 multiplies of 32 tokens into the int32 accumulator
+      if (wt == 0) {
+#pragma unroll
+        for (int j = 0; j < TC_BLOCK / 2; ++j)
+          tc::mma_i8(tcol + TC_O, tcol + TC_AV + 32 * buf + 8 * j, tc::sdesc(PB + TC_PB * buf + 512 * j, 128, 512),
+                     TC_IDESC_PV, (ostarted || j > 0) ? 1u : 0u);
+        tc::commit(pvbar0 + 8 * buf);
+      }
+      ++n_pv;
+      ostarted = true;
+      ++since_fold;
+      ++nb;
+    }
+    if (!ok) break;
+
+    // ---- the segment's result: fold the accumulator, sum l and z over the warpgroup's tokens
+    if (ostarted) {
+      const uint32_t pb = (nb - 1) & 1u;
+      ok = wg_and(h, mbar_wait(pvbar0 + 8 * pb, ((nb - 1) >> 1) & 1u, abort_flag, status));
+      if (!ok) break;
+      tc::fence_after();
+      uint32_t o16[16];
+      tc::ld32x16(tlane + TC_O, o16);
+      tc::wait_ld();
+      const float invF = F > 0.f ? 1.f / F : 0.f;
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh) oacc[hh] = fmaf(fold_planes(o16 + 4 * hh), invF, oacc[hh]);
+    }
+    float red[8] = {l[0], l[1], l[2], l[3], zs[0], zs[1], zs[2], zs[3]};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int o = 16; o; o >>= 1) red[i] += __shfl_xor_sync(0xffffffffu, red[i], o);
+    if (lane == 0)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) scratch[8 * (warp & 3) + i] = red[i];
+    wg_sync(h);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[i] = (scratch[i] + scratch[8 + i]) + (scratch[16 + i] + scratch[24 + i]);
+    wg_sync(h);
+    float o[4];
+#pragma unroll
+    for (int hh = 0; hh < 4; ++hh) o[hh] = oacc[hh] + red[4 + hh];   // unnormalised o_rot of dim wt
+    if (sq.nseg == 1) {
+      const int d = wt;
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh) o[hh] *= red[hh] > 0.f ? 1.f / red[hh] : 0.f;
+      // o = H_blk o_rot: ascending butterfly stages over the dims (one dim per thread)
+      const int Bh = p.Bh_o;
+#pragma unroll
+      for (int st = 1; st < 32; st <<= 1)
+        if (st < Bh)
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh) {
+            const float other = __shfl_xor_sync(0xffffffffu, o[hh], st);
+            o[hh] = (d & st) ? other - o[hh] : o[hh] + other;
+          }
+      for (int st = 32; st < D && st < Bh; st <<= 1) {
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) scratch[4 * d + hh] = o[hh];
+        wg_sync(h);
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) {
+          const float other = scratch[4 * (d ^ st) + hh];
+          o[hh] = (d & st) ? other - o[hh] : o[hh] + other;
+        }
+        wg_sync(h);
+      }
+      const float rc = p.rc_o;
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh) {
+        const long long off = (static_cast<long long>(g.b) * p.Hq + hkv * 4 + hh) * D + d;
+        if (p.mode & KV4_MODE_OUT_F32) static_cast<float*>(p.out)[off] = o[hh] * rc;
+        else static_cast<uint16_t*>(p.out)[off] = __bfloat16_as_ushort(__float2bfloat16_rn(o[hh] * rc));
+      }
+    } else {
+      // a group split over several CTAs: this segment's partial (m, l, unnormalised o) for the merge kernel
+      float* part = p.partials + static_cast<size_t>((c * 2 + (q == 0 ? 0 : 1)) * 4 + h) * pstride;
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh) part[hh * HS + wt] = o[hh];
+      if (wt == 0)
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) { part[hh * HS + D] = m[hh]; part[hh * HS + D + 1] = red[hh]; }
+    }
+  }
+  // no multiply may be in flight when the tensor memory is freed: after an abort, wait (bounded) for the
+  // last commits this warpgroup issued (the P.V ones of block n_pv - 1, the score ones of block n_qk - 1)
+  if (!ok) {
+    if (n_pv > 0) {
+      const uint32_t b = n_pv - 1;
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(pvbar0 + 8 * (b & 1u), (b >> 1) & 1u) && globaltimer_ns() - t0 < 1000000000ull) {}
+    }
+    if (n_qk > 0) {
+      const uint64_t t1 = globaltimer_ns();
+      while (!mbar_try_wait(sbar, (n_qk - 1) & 1u) && globaltimer_ns() - t1 < 1000000000ull) {}
+    }
+  }
+  tc::fence_before();
+  consumers_sync();
+  tc::fence_after();
+  if (warp == 0) tc::dealloc(*tmem_slot, TC_COLS);
+}
+
+// ---------------------------------------------------------------------------
 // host side
 
 #ifndef KV4_GROUPED_PAIR
@@ -924,9 +1485,12 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   p.qblob = wsb + l.qblob;
   p.partials = reinterpret_cast<float*>(wsb + l.partials);
   GPlanRec* plan = reinterpret_cast<GPlanRec*>(wsb + l.plan);
-  p.grid = g_grid(c);
+  // one query token, 4-head groups, D = 128: the tensor-memory kernel, one CTA per SM
+  const bool tcpath = D == 128 && GWR == 4 && c->use_tc && p.qtot == 1;
+  p.qfmt = tcpath ? 1 : 0;
+  p.grid = tcpath ? c->num_sms : g_grid(c);
   p.cap_parts = p.grid * 2 * GWR;
-  p.ns = c->gattn_ring;
+  p.ns = tcpath ? c->tattn_ring : c->gattn_ring;
   p.stall_stage = c->test_stall;   // test hook, for this launch only
   c->test_stall = -1;
   if (step) {
@@ -942,8 +1506,8 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.grid);
-  cfg.blockDim = dim3(GShape<GWR>::THREADS);
-  cfg.dynamicSmemBytes = gattn_smem_bytes<D, GWR>(p.ns);
+  cfg.blockDim = dim3(tcpath ? TC_THREADS : GShape<GWR>::THREADS);
+  cfg.dynamicSmemBytes = tcpath ? tattn_smem_bytes<D>(p.ns) : gattn_smem_bytes<D, GWR>(p.ns);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -951,8 +1515,15 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   cfg.attrs = attr;
   cfg.numAttrs = step ? 0 : 1;
   // several query tokens per sequence (even a pass of one of them): the causal variant
-  cudaError_t e = p.qtot > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true, GWR>, p, plan)
-                              : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false, GWR>, p, plan);
+  cudaError_t e;
+  if constexpr (D == 128 && GWR == 4) {
+    if (tcpath) e = cudaLaunchKernelEx(&cfg, tattn_kernel<D>, p, plan);
+    else if (p.qtot > 1) e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true, GWR>, p, plan);
+    else e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false, GWR>, p, plan);
+  } else {
+    e = p.qtot > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true, GWR>, p, plan)
+                   : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false, GWR>, p, plan);
+  }
   if (e == cudaSuccess) {
     cudaLaunchConfig_t mcfg = cfg;
     mcfg.gridDim = dim3((p.n_seqs * p.Hkv * p.G + MWARPS - 1) / MWARPS);
@@ -983,12 +1554,43 @@ int g_choose_ring_gw(int device, int Hkv) {
   }
 }
 
+// Ring depth of the tensor-memory kernel (one CTA per SM), or -1 when it cannot run.
+int tattn_choose_ring(int device) {
+  int optin = 0;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess) return -1;
+  if (cudaFuncSetAttribute(tattn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess)
+    return -1;
+  for (int ns = MAX_NS; ns >= 2 * TC_BLOCK; --ns) {
+    const size_t smem = tattn_smem_bytes<128>(ns);
+    if (smem > static_cast<size_t>(optin)) continue;
+    int blocks = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, tattn_kernel<128>, TC_THREADS, smem) != cudaSuccess)
+      return -1;
+    if (blocks >= 1) return ns;
+  }
+  return -1;
+}
+
 }  // namespace
 
 bool grouped_path(const kv4_cache* c) { return !c->bf16; }
 
 int grouped_ring(kv4_cache* c) {
   c->gattn_pair = kPair;
+  c->use_tc = false;
+  c->tattn_ring = 0;
+  if (c->cfg.head_dim == 128 && group_width(c->cfg.num_kv_heads) == 4) {
+    const char* env = getenv("KV4_ATTENTION_KERNEL");   // "mma": keep the mma.sync kernel (comparisons)
+    if (!(env && strcmp(env, "mma") == 0)) {
+      const int ns = tattn_choose_ring(c->device);
+      if (ns > 0) {
+        c->use_tc = true;
+        c->tattn_ring = ns;
+      } else {
+        cudaGetLastError();
+      }
+    }
+  }
   return c->cfg.head_dim == 128 ? g_choose_ring_gw<128>(c->device, c->cfg.num_kv_heads)
                                 : g_choose_ring_gw<64>(c->device, c->cfg.num_kv_heads);
 }

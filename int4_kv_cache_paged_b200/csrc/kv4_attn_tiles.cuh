@@ -696,5 +696,31 @@ __device__ __forceinline__ void store_qblob(uint8_t* blob, const QFrag<D>& qf, i
   if (lane == 0) tail[MAX_G] = qf.kscale;
 }
 
+// The same query operand in the layout of the tensor-memory kernel: the two
+// 8-bit planes as B matrices of its score multiplies (K-major, no swizzle;
+// N = 8 columns, K = the 128 code bytes of a TMEM row), hi plane in the first
+// 1 KB, lo plane in the second; the tail as in store_qblob.  Code byte p of a
+// row (p = (D/4) t + 8 kk + 4 hf + j) holds dim 32 kk + 16 hf + 4 t + j; byte
+// (column n, p) of a plane sits at 128 (p / 16) + 16 n + p % 16.
+template <int D>
+__device__ __forceinline__ void store_qblob_tc(uint8_t* blob, const QFrag<D>& qf, int lane) {
+  static_assert(D == 128, "the tensor-memory kernel covers D = 128");
+  constexpr int NKK = D / 32;
+  const int n = lane >> 2, t = lane & 3;
+  uint32_t* w = reinterpret_cast<uint32_t*>(blob);
+#pragma unroll
+  for (int kk = 0; kk < NKK; ++kk)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int pos = (D / 4) * t + 8 * kk + 4 * hf;
+      const int a = (128 * (pos >> 4) + 16 * n + (pos & 15)) >> 2;
+      w[a] = qf.b[kk][hf];
+      w[256 + a] = qf.b[NKK + kk][hf];
+    }
+  float* tail = reinterpret_cast<float*>(blob + 16 * D);
+  if (lane < 4) { tail[2 * lane] = qf.qs0; tail[2 * lane + 1] = qf.qs1; }
+  if (lane == 0) tail[MAX_G] = qf.kscale;
+}
+
 }  // namespace tiles
 }  // namespace kv4

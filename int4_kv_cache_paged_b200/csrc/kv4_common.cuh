@@ -115,6 +115,7 @@ struct AttnParams {
   int ns;                     // shared-memory ring depth of the attention kernel
   int grid;                   // CTAs of the page-major attention kernel
   int stall_stage;            // test hook: stage the first CTA leaves unfilled (-1: none)
+  int qfmt;                   // query operand layout the query kernels write: 0 fragments, 1 tensor-memory kernel
 };
 
 // Row of q (and of the output) that operand column c of KV head h of batch
@@ -434,6 +435,8 @@ struct kv4_cache {
   cudaEvent_t ev_before;     // optional timing events around the split-K kernel
   cudaEvent_t ev_after;
   int test_stall;            // kv4_test_stall_next_attention: stage to leave unfilled in the next call (-1: none)
+  bool use_tc;               // one-token attention with 4-head groups at D = 128 runs the tensor-memory kernel
+  int tattn_ring;            // its ring depth
 };
 
 namespace kv4 {
