@@ -25,9 +25,15 @@ Readings of this library (the pages give none of these details):
   same block-diagonal Hadamard rotation.
 * Keys arrive post-RoPE, or get RoPE at their positions on the way in when a
   table is given (append(..., rope=...), see rope.py).
+* Page format (config key "page_format"): 0 = INT4 (the method), 1 = NVFP4,
+  the alternative format of the "KV Cache Quantization" topic page, item 3
+  (see nvfp4.py).  The format changes only what the pages hold; the rotation,
+  the INT8 store of the protected positions and the effective view are the
+  same.  Below, "INT4 page" means the page copy in either format.
 * Device byte order (head-innermost, so that the tiles of all KV heads at one
   page position are contiguous):
     INT4 pool of a layer   uint8 [num_pages][P/16][Hkv][16*D + 128]
+    NVFP4 pool of a layer  uint8 [num_pages][P/16][Hkv][18*D]
     INT8 store of a layer  uint8 [max_seqs][ceil((S+W)/16)][Hkv][32*D + 128]
     BF16 pool of a layer   bf16  [num_pages][P/16][Hkv][32*D]
   The arrays below use the same order per page / per sequence.
@@ -38,7 +44,8 @@ import numpy as np
 from .hadamard import fwht_fp32
 from .rope import rope_fp32
 from .quant import quantize_groups, dequantize_groups
-from .layout import TILE, tables, int4_tile_bytes, int8_tile_bytes, bf16_tile_bytes, scale_offset
+from .nvfp4 import quantize_nvfp4, dequantize_nvfp4
+from .layout import TILE, tables, int4_tile_bytes, int8_tile_bytes, bf16_tile_bytes, fp4_tile_bytes, scale_offset
 
 CONFIG_FIELDS = ("num_layers", "max_seqs", "num_q_heads", "num_kv_heads", "head_dim",
                  "page_size", "num_pages", "max_pages_per_seq", "hadamard_block",
@@ -81,18 +88,23 @@ class OracleKV4Cache:
         self.S = c["sink_tokens"]
         self.W = c["recent_window"]
         self.Bh = c["hadamard_block"]
+        self.fmt = int(c.get("page_format", 0))
+        if self.fmt not in (0, 1):
+            raise ValueError("page_format must be 0 (INT4) or 1 (NVFP4)")
         self.block_table = np.asarray(block_table, dtype=np.int64)
         self.seq_lens = np.zeros((c["num_layers"], c["max_seqs"]), np.int64)
         self.pages = {}
         self.prot = {}
         self.t4 = tables("int4", self.D)
         self.t8 = tables("int8", self.D)
+        self.tf = tables("nvfp4", self.D)
+        self.page_tile_bytes = fp4_tile_bytes(self.D) if self.fmt == 1 else int4_tile_bytes(self.D)
 
     # -- storage helpers -------------------------------------------------
     def _page_tiles(self, layer, page):
         key = (layer, page)
         if key not in self.pages:
-            self.pages[key] = np.zeros((self.P // TILE, self.Hkv, int4_tile_bytes(self.D)), np.uint8)
+            self.pages[key] = np.zeros((self.P // TILE, self.Hkv, self.page_tile_bytes), np.uint8)
         return self.pages[key]
 
     def _prot_tiles(self, layer, seq):
@@ -154,6 +166,54 @@ class OracleKV4Cache:
                 off = 16 * D + np.array([scale_offset(int(x), tensor) for x in rs])
                 self._scatter(tiles, ts, off[:, None] + np.arange(4), self._sz_bytes(s16[sel], z16[sel]))
 
+    def _write_fp4(self, layer, seq, pos, enc_k, enc_v):
+        """NVFP4 codes and block scales of positions `pos` (enc_*: codes [m, Hkv, D], scales [m, Hkv, D/16]).
+
+        A V byte holds one dim of two tokens: only this token's nibble of it changes."""
+        D, tf = self.D, self.tf
+        page = self._pages_of(seq, pos)
+        r = pos % TILE
+        ti = (pos % self.P) // TILE
+        for pg in np.unique(page):
+            sel = page == pg
+            tiles = self._page_tiles(layer, int(pg))
+            rs, ts = r[sel], ti[sel]
+            kc, ks = enc_k[0][sel], enc_k[1][sel]
+            lo_c = np.take_along_axis(kc, tf.k_lo[rs][:, None, :], axis=2)
+            hi_c = np.take_along_axis(kc, tf.k_hi[rs][:, None, :], axis=2)
+            self._scatter(tiles, ts, tf.k_byte[rs], lo_c | (hi_c << 4))
+            self._scatter(tiles, ts, tf.ks_byte[rs], ks)
+            self._scatter(tiles, ts, tf.vs_byte[rs], enc_v[1][sel])
+            vc = enc_v[0][sel]                                            # [m, Hkv, D]
+            for j in range(len(rs)):
+                byte = 8 * D + tf.v_byte[rs[j]]                           # [D]
+                shift = 4 * tf.v_nib[rs[j]]
+                for h in range(self.Hkv):
+                    old = tiles[ts[j], h, byte].astype(np.int64)
+                    new = (old & ~(15 << shift)) | (vc[j, h].astype(np.int64) << shift)
+                    tiles[ts[j], h, byte] = new.astype(np.uint8)
+
+    def _read_fp4(self, layer, seq, pos):
+        """Dequantized K^, V^ [m, Hkv, D] of positions `pos` from NVFP4 pages."""
+        D, tf = self.D, self.tf
+        page = self._pages_of(seq, pos)
+        r = pos % TILE
+        ti = (pos % self.P) // TILE
+        out = [np.zeros((len(pos), self.Hkv, D), np.float32) for _ in range(2)]
+        for pg in np.unique(page):
+            sel = np.nonzero(page == pg)[0]
+            tiles = self._page_tiles(layer, int(pg))
+            rs, ts = r[sel], ti[sel]
+            b = self._gather(tiles, ts, tf.k_byte[rs])                       # [m, Hkv, D/2]
+            kc = np.zeros((len(sel), self.Hkv, D), np.uint8)
+            np.put_along_axis(kc, tf.k_lo[rs][:, None, :], b & 15, axis=2)
+            np.put_along_axis(kc, tf.k_hi[rs][:, None, :], b >> 4, axis=2)
+            out[0][sel] = dequantize_nvfp4(kc, self._gather(tiles, ts, tf.ks_byte[rs]))
+            vb = self._gather(tiles, ts, 8 * D + tf.v_byte[rs])               # [m, Hkv, D]
+            vc = ((vb >> (4 * tf.v_nib[rs])[:, None, :]) & 15).astype(np.uint8)
+            out[1][sel] = dequantize_nvfp4(vc, self._gather(tiles, ts, tf.vs_byte[rs]))
+        return out
+
     def _write_int8(self, layer, seq, slots, enc_k, enc_v):
         D, t8 = self.D, self.t8
         tiles = self._prot_tiles(layer, seq)
@@ -204,9 +264,11 @@ class OracleKV4Cache:
 
     # -- the method --------------------------------------------------------
     def rotate_quantize(self, x):
-        """x: [n, Hkv, D] values (bf16 held in fp32).  Returns the rotation and both encodings."""
+        """x: [n, Hkv, D] values (bf16 held in fp32).  Returns the rotation, the page encoding (INT4
+        (codes, s16, z16) or NVFP4 (codes, scales)) and the INT8 encoding."""
         xr = fwht_fp32(x, self.Bh)
-        return xr, quantize_groups(xr, 4), quantize_groups(xr, 8)
+        page = quantize_nvfp4(xr) if self.fmt == 1 else quantize_groups(xr, 4)
+        return xr, page, quantize_groups(xr, 8)
 
     def append(self, layer, seq_ids, cu_new, k_new, v_new, rope=None):
         """Append new tokens: seq_ids[i] receives rows cu_new[i]:cu_new[i+1] of k_new / v_new.
@@ -232,7 +294,10 @@ class OracleKV4Cache:
                 kx = rope_fp32(kx, pos[:, None], *rope)
             _, k4, k8 = self.rotate_quantize(kx)
             _, v4, v8 = self.rotate_quantize(v_new[a:b])
-            self._write_int4(layer, seq, pos, k4, v4)           # every position: INT4 page copy
+            if self.fmt == 1:                                    # every position: the page copy
+                self._write_fp4(layer, seq, pos, k4, v4)
+            else:
+                self._write_int4(layer, seq, pos, k4, v4)
             prot = (pos < self.S) | (pos >= L_new - self.W)      # sinks, and the last W of this append
             if np.any(prot):
                 j = np.nonzero(prot)[0]
@@ -262,6 +327,8 @@ class OracleKV4Cache:
             if src:
                 slots = np.array([prot_slot(int(p), self.S, self.W) for p in pos[sel]])
                 kv = self._read_int8(layer, seq, slots)
+            elif self.fmt == 1:
+                kv = self._read_fp4(layer, seq, pos[sel])
             else:
                 kv = self._read_int4(layer, seq, pos[sel])
             out[0][sel], out[1][sel] = kv

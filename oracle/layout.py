@@ -10,6 +10,7 @@ Unit of storage: a tile of 16 consecutive token slots of one KV head.
 
 INT4 tile (16*D + 128 bytes):   [K codes 8*D][V codes 8*D][scales 128]
 INT8 tile (32*D + 128 bytes):   [K codes 16*D][V codes 16*D][scales 128]
+NVFP4 tile (18*D bytes):        [K codes 8*D][V codes 8*D][K scales D][V scales D]
 BF16 tile (64*D bytes):         [K 16*D bf16][V 16*D bf16]      (baseline cache)
 
 Inside the code blocks the order of nibbles/bytes follows the operand order
@@ -23,6 +24,12 @@ token can be written without reading its neighbours).
 Scales: a 128-byte block of 32 half2 (s, z) entries.  Entry for token r of
 tensor T (K = 0, V = 1) sits at byte 16*(r % 8) + 4*(2*T + r // 8); the half
 at +0 is the scale s, the half at +2 the zero point z.
+
+The NVFP4 tile (the alternative page format, see nvfp4.py) feeds 16x8x16 fp16
+multiplies for both products.  Its K bytes belong to one token each; each V
+byte holds one dim of two neighbouring tokens (2i, 2i + 1), the pair that one
+fp16x2 operand register of the P.V multiply takes, so a token's V codes are
+written nibble by nibble.  One E4M3 scale byte per (token, 16-dim block).
 """
 
 import numpy as np
@@ -40,6 +47,10 @@ def int8_tile_bytes(D):
 
 def bf16_tile_bytes(D):
     return 64 * D
+
+
+def fp4_tile_bytes(D):
+    return 18 * D
 
 
 def int4_k_nibble(D, r, d):
@@ -119,6 +130,50 @@ def bf16_v_elem(D, r, d):
     return 8 * (32 * m + 4 * g + t) + 2 * reg + e
 
 
+def fp4_k_nibble(D, r, d):
+    """(byte offset inside the NVFP4 K code block, nibble) of token r, dim d.
+
+    With r = 8*rh + g (g < 8) and d = 16*b + 4*t + 2*j + e (b < D/16, t < 4,
+    j < 2, e < 2), the code is nibble e of byte rh + 2*j of the 32-bit word at
+    16*(4*g + t) + 4*(b % 4) + 512*(b // 4): lane 4g + t of a warp reads, per
+    16-dim block b, one word whose four bytes are the E2M1 pairs of its four
+    16x8x16 A-operand registers (tokens g, g + 8; dims 4t, 4t+1 and 4t+2, 4t+3).
+    """
+    rh, g = divmod(r, 8)
+    b, rem = divmod(d, 16)
+    t, rem = divmod(rem, 4)
+    j, e = divmod(rem, 2)
+    return 16 * (4 * g + t) + 4 * (b % 4) + 512 * (b // 4) + rh + 2 * j, e
+
+
+def fp4_v_nibble(D, r, d):
+    """(byte offset inside the NVFP4 V code block, nibble) of token r, dim d.
+
+    With d = 16*m + 8*dh + g and r = 8*th + 2*t + e, the code is nibble e of
+    byte dh + 2*th of the word at 16*(4*g + t) + 4*(m % 4) + 512*(m // 4): the
+    word of lane 4g + t and dim block m holds the four A-operand pairs (dims g,
+    g + 8; tokens 2t, 2t+1 and 2t+8, 2t+9) of the transposed P.V multiply.
+    """
+    m, rr = divmod(d, 16)
+    dh, g = divmod(rr, 8)
+    th, tt = divmod(r, 8)
+    t, e = divmod(tt, 2)
+    return 16 * (4 * g + t) + 4 * (m % 4) + 512 * (m // 4) + dh + 2 * th, e
+
+
+def fp4_k_scale_byte(D, r, b):
+    """Byte offset inside the tile of the E4M3 scale of token r, K block b: 16*D + (D/8)*g + 2*b + rh."""
+    rh, g = divmod(r, 8)
+    return 16 * D + (D // 8) * g + 2 * b + rh
+
+
+def fp4_v_scale_byte(D, r, m):
+    """Byte offset inside the tile of the E4M3 scale of token r, V block m: 17*D + (D/4)*t + 4*m + 2*th + e."""
+    th, tt = divmod(r, 8)
+    t, e = divmod(tt, 2)
+    return 17 * D + (D // 4) * t + 4 * m + 2 * th + e
+
+
 def scale_offset(r, tensor):
     """Byte offset of the half2 (s, z) of token r inside the 128-byte scale block; tensor 0 = K, 1 = V."""
     return 16 * (r % 8) + 4 * (2 * tensor + r // 8)
@@ -171,11 +226,37 @@ class BF16Tables:
         self.v_elem = np.array([[bf16_v_elem(D, r, d) for d in range(D)] for r in range(TILE)], np.int64)
 
 
+class Fp4Tables:
+    """For token slot r: the K bytes it owns (D/2) with their low / high dims; per dim its V byte and
+    nibble (D); its scale bytes per 16-dim block (D/16) for K and V."""
+
+    def __init__(self, D):
+        self.D = D
+        self.k_byte = np.zeros((TILE, D // 2), np.int64)
+        self.k_lo = np.zeros((TILE, D // 2), np.int64)
+        self.k_hi = np.zeros((TILE, D // 2), np.int64)
+        for r in range(TILE):
+            owned = {}
+            for d in range(D):
+                byte, half = fp4_k_nibble(D, r, d)
+                owned.setdefault(byte, [None, None])[half] = d
+            if len(owned) != D // 2 or any(None in v for v in owned.values()):
+                raise AssertionError("NVFP4 K layout: token %d does not own whole bytes" % r)
+            for n, byte in enumerate(sorted(owned)):
+                self.k_byte[r, n] = byte
+                self.k_lo[r, n], self.k_hi[r, n] = owned[byte]
+        vb = [[fp4_v_nibble(D, r, d) for d in range(D)] for r in range(TILE)]
+        self.v_byte = np.array([[x[0] for x in row] for row in vb], np.int64)
+        self.v_nib = np.array([[x[1] for x in row] for row in vb], np.int64)
+        self.ks_byte = np.array([[fp4_k_scale_byte(D, r, b) for b in range(D // 16)] for r in range(TILE)], np.int64)
+        self.vs_byte = np.array([[fp4_v_scale_byte(D, r, m) for m in range(D // 16)] for r in range(TILE)], np.int64)
+
+
 _cache = {}
 
 
 def tables(kind, D):
     key = (kind, D)
     if key not in _cache:
-        _cache[key] = {"int4": Int4Tables, "int8": Int8Tables, "bf16": BF16Tables}[kind](D)
+        _cache[key] = {"int4": Int4Tables, "int8": Int8Tables, "bf16": BF16Tables, "nvfp4": Fp4Tables}[kind](D)
     return _cache[key]
