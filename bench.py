@@ -323,7 +323,8 @@ def measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=1, compare
     K_e2e = 0 if args.kernel_only else K
     do_cmp = compare and not args.kernel_only and not rope and world == 1
     n_cmp = 2 * K if do_cmp else 0              # the step as two calls and as one call
-    extra = W_ + 2 * K + K_e2e + n_cmp + 1       # timed loop, kernel-event pass, e2e, comparison steps
+    n_diag = min(K_e2e, 5)                       # the e2e breakdown
+    extra = W_ + 2 * K + K_e2e + n_diag + n_cmp + 1   # timed loop, kernel-event pass, e2e, comparison steps
     t0 = time.time()
     rep = Replica(w, layers, device, extra, W_ + K, torch, rope=rope)
     rep.extra = extra
@@ -450,6 +451,34 @@ def measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=1, compare
         e2e = {"t": t_e2e, "bytes": e2e_bytes, "steps": K_e2e, "h2d_bytes_per_step": int(layers * per * 2),
                "d2h_bytes_per_step": int(layers * B * Hq * D * 2)}
         used += K_e2e
+        # diagnostic (outside the e2e figure): the same three pieces of a step one after another on one
+        # stream, each between its own events -- the copy in, the library calls, the copy out
+        nd = min(K_e2e, 5)
+        ev3 = [[ev() for _ in range(4)] for _ in range(nd)]
+        barrier()
+        for j in range(nd):
+            flush.fill_(j & 0xFF)
+            ev3[j][0].record(stream)
+            for layer in range(layers):
+                din[0, layer].copy_(hin[j, layer], non_blocking=True)
+            ev3[j][1].record(stream)
+            for layer in range(layers):
+                dk = din[0, layer, :kv_el].view(B, Hkv, D)
+                dv = din[0, layer, kv_el:2 * kv_el].view(B, Hkv, D)
+                dq = din[0, layer, 2 * kv_el:].view(B, Hq, D)
+                cache.decode_step(layer, rep.seq_ids, dk, dv, dq, out=dout[0, layer], workspace=ws, mode=amode)
+            ev3[j][2].record(stream)
+            for layer in range(layers):
+                hout[j, layer].copy_(dout[0, layer], non_blocking=True)
+            ev3[j][3].record(stream)
+        barrier()
+        if nd:
+            parts = [sum(ev3[j][i].elapsed_time(ev3[j][i + 1]) for j in range(nd)) / nd * 1e3 for i in range(3)]
+            e2e["breakdown_us"] = {"h2d": round(parts[0], 2), "step": round(parts[1], 2), "d2h": round(parts[2], 2),
+                                   "serial_sum": round(sum(parts), 2),
+                                   "how": "%d steps with the three pieces serialised on one stream, each between "
+                                          "its own CUDA events (not the e2e figure, which overlaps them)" % nd}
+        used += nd
         del hin, hout, din, dout
 
     res = {"rep": rep, "setup_s": setup_s, "t_step": t_step, "bytes_timed": bytes_timed, "t_kern": t_kern,
@@ -609,7 +638,8 @@ def sub_line(torch, kv4, name, args, device, clocks, hbm, peak_kind):
     if r["e2e"]:
         e = r["e2e"]
         line["e2e"] = {"value": round(e["bytes"] / e["t"] / 1e9, 2), "unit": "GB/s",
-                       "h2d_bytes_per_step": e["h2d_bytes_per_step"], "d2h_bytes_per_step": e["d2h_bytes_per_step"]}
+                       "h2d_bytes_per_step": e["h2d_bytes_per_step"], "d2h_bytes_per_step": e["d2h_bytes_per_step"],
+                       "ms_per_step": round(e["t"] / e["steps"] * 1e3, 4), "breakdown_us": e.get("breakdown_us")}
     cmp = r.get("compare")
     if cmp:
         line["compare"] = cmp
@@ -704,6 +734,7 @@ def run_gpu(args):
                          "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
                          "tokens_per_s": round(B * world * e2e["steps"] / t_e2e_all, 1),
                          "ms_per_step": round(t_e2e_all / e2e["steps"] * 1e3, 4),
+                         "breakdown_us": e2e.get("breakdown_us"),
                          "how": "per layer: new K, V and q copied from pinned host memory on a copy stream ahead "
                                 "of the layer, the layer's output copied to pinned host memory on a second copy "
                                 "stream behind it, device staging doubled so the copies of a step overlap the "

@@ -1159,6 +1159,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tattn_kernel(AttnParams p, GPla
             sK = half_lo(szk); zK = half_hi(szk); sV = half_lo(szv); zV = half_hi(szv);
             valid = tp[it] + r < g.nprot;
           }
+          if (!valid) { sK = 0.f; zK = 0.f; sV = 0.f; zV = 0.f; }   // unwritten slots may hold non-finite scales
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) kw[i] = 0u;
@@ -1181,6 +1182,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tattn_kernel(AttnParams p, GPla
       }
       // ---- V phase: thread wt = dim wt; the buffer's previous multiplies (block nb - 2) must be done
       if (ok && nb >= 2 && !mbar_wait(pvbar0 + 8 * buf, ((nb - 2) >> 1) & 1u, abort_flag, status)) ok = false;
+      tc::fence_after();   // the tensor-memory stores below follow those multiplies
       {
         uint32_t vw[32];
         const int d = wt, mb = d >> 4, dh = (d >> 3) & 1, gg = d & 7;
@@ -1580,8 +1582,9 @@ int grouped_ring(kv4_cache* c) {
   c->use_tc = false;
   c->tattn_ring = 0;
   if (c->cfg.head_dim == 128 && group_width(c->cfg.num_kv_heads) == 4) {
-    const char* env = getenv("KV4_ATTENTION_KERNEL");   // "mma": keep the mma.sync kernel (comparisons)
-    if (!(env && strcmp(env, "mma") == 0)) {
+    // "tc": the tensor-memory kernel, an opt-in alternative (slower than the mma.sync kernel on B200)
+    const char* env = getenv("KV4_ATTENTION_KERNEL");
+    if (env && strcmp(env, "tc") == 0) {
       const int ns = tattn_choose_ring(c->device);
       if (ns > 0) {
         c->use_tc = true;

@@ -1,7 +1,7 @@
 """The two one-token attention kernels of 4-KV-head groups at D = 128 -- the
-tensor-memory kernel (tcgen05 multiplies, the default) and the mma.sync kernel
-(KV4_ATTENTION_KERNEL=mma when the cache is created) -- against the oracle on
-the same caches.  The inputs make the tensor-memory kernel move its running
+mma.sync kernel (the default) and the tensor-memory kernel (tcgen05
+multiplies, KV4_ATTENTION_KERNEL=tc when the cache is created) -- against the
+oracle on the same caches.  The inputs make the tensor-memory kernel move its running
 max late (a large-norm key at the last positions and at the sink, which it
 reads last) and its fixed-point scale (V magnitudes growing along the
 sequence), so its accumulator is folded several times within one segment."""
@@ -28,8 +28,8 @@ def kv4():
 def _pair(cfg, table, kernel):
     old = os.environ.get("KV4_ATTENTION_KERNEL")
     try:
-        if kernel == "mma":
-            os.environ["KV4_ATTENTION_KERNEL"] = "mma"
+        if kernel == "tc":
+            os.environ["KV4_ATTENTION_KERNEL"] = "tc"
         else:
             os.environ.pop("KV4_ATTENTION_KERNEL", None)
         return Pair(cfg, table)
@@ -56,11 +56,13 @@ def test_both_kernels_match_the_oracle(kv4, lens):
             ramp = torch.linspace(0.3, 4.0, L)[:, None, None]   # V magnitudes grow along the sequence
             v[off:off + L] *= ramp
             k[off] *= 9.0                                       # large-norm sink at position 0
-            k[off + max(L - 3, 0):off + L] *= 3.0               # and large keys among the last positions
+            k[off + max(L - 3, 1):off + L] *= 3.0               # and large keys among the last positions
         off += L
     k, v = k.to(torch.bfloat16), v.to(torch.bfloat16)
     pairs = {name: _pair(cfg, table, name) for name in ("tc", "mma")}
     for pr in pairs.values():
+        pr.gpu.pages(0).fill_(0xFF)          # unwritten slots hold NaN scales and codes
+        pr.gpu.protected(0).fill_(0xFF)
         pr.append(0, list(range(n)), list(lens), k, v)
     seqs = list(range(n))[::-1]
     q = bf16_values((n, Hq, D), rng)
