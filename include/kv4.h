@@ -16,6 +16,13 @@
  * same Hadamard transform, attends over the mixed INT4/INT8 cache and rotates
  * the output back.
  *
+ * Alternative page format: with page_format = KV4_FORMAT_NVFP4 the pages hold
+ * NVFP4 instead of INT4 ("KV Cache Quantization" topic page, item 3: the
+ * NVFP4 paged KV cache of SGLang, about 56 % of the FP8 bytes per token):
+ * E2M1 codes in blocks of 16 dims sharing one E4M3 scale (per-tensor scale
+ * 1), after the same rotation; the INT8 store of the protected positions and
+ * every entry point are the same.
+ *
  * Conventions
  * -----------
  * - Every function returns KV4_OK (0) or a negative KV4_ERR_* code; nothing
@@ -97,17 +104,24 @@ enum {
  * both bits (it has no rotation). */
 enum {
   KV4_MODE_PROTECTED = 0,     /* INT8 for protected positions, INT4 elsewhere (the method) */
-  KV4_MODE_INT4_ONLY = 1,     /* read the INT4 pages for every position (ablation)         */
+  KV4_MODE_INT4_ONLY = 1,     /* read the pages (INT4 or NVFP4) for every position         */
   KV4_MODE_OUT_F32 = 2,       /* write fp32 output instead of bf16 (checking mode)          */
   KV4_MODE_Q_ROTATED = 4,     /* q is already H q: do not rotate it                         */
   KV4_MODE_OUT_ROTATED = 8,   /* write the output in the rotated basis (H o): no inverse    */
   KV4_MODE_ROPE_Q = 16        /* apply the cache's RoPE table to q at its position first    */
 };
 
+/* Page formats (kv4_config.page_format). */
+enum {
+  KV4_FORMAT_INT4 = 0,        /* token-wise asymmetric INT4, fp16 scale and zero point      */
+  KV4_FORMAT_NVFP4 = 1        /* E2M1 codes, one E4M3 scale per 16 dims (values beyond
+                                 +-2688 saturate)                                          */
+};
+
 /* kv4_dequantize_debug views. */
 enum {
   KV4_VIEW_EFFECTIVE = 0,     /* what attention reads in KV4_MODE_PROTECTED                 */
-  KV4_VIEW_INT4 = 1           /* the INT4 page copy of every position                       */
+  KV4_VIEW_INT4 = 1           /* the page copy (INT4 or NVFP4) of every position            */
 };
 
 /*
@@ -123,12 +137,15 @@ enum {
  *   hadamard_block      Bh, a power of two dividing D (1 = no rotation)
  *   sink_tokens         S >= 0
  *   recent_window       W >= 1, S + W <= 4096
+ *   page_format         KV4_FORMAT_INT4 (0) or KV4_FORMAT_NVFP4 (1); the BF16
+ *                       baseline cache needs 0
  */
 typedef struct {
   int32_t num_layers, max_seqs, num_q_heads, num_kv_heads, head_dim;
   int32_t page_size, num_pages, max_pages_per_seq;
   int32_t hadamard_block;
   int32_t sink_tokens, recent_window;
+  int32_t page_format;
 } kv4_config;
 
 typedef struct kv4_cache kv4_cache;   /* opaque host handle owned by the library */
@@ -150,7 +167,8 @@ int kv4_cache_create(const kv4_config* cfg, void* dev_buf, size_t bytes, int32_t
 int kv4_cache_destroy(kv4_cache* cache);
 
 /* Device addresses inside the cache buffer for layer `layer` (any pointer may
- * be NULL): the INT4 page pool, uint8 [num_pages][P/16][Hkv][16*D+128]; the
+ * be NULL): the page pool, uint8 [num_pages][P/16][Hkv][16*D+128] (INT4) or
+ * [num_pages][P/16][Hkv][18*D] (NVFP4); the
  * INT8 store, uint8 [max_seqs][ceil((S+W)/16)][Hkv][32*D+128]; and the
  * sequence lengths int32 [num_layers][max_seqs] (all layers).  KV heads are
  * innermost, so the 16-token tiles of all heads at one page position are
@@ -324,7 +342,8 @@ int kv4_decode_attention_noalloc(kv4_cache* cache, int32_t layer, const int32_t*
 
 /* Dequantized keys/values of positions [start, start+count) of one sequence,
  * fp32 [count][Hkv][D], in the rotated basis: x^ = fma(code, s, z) from the
- * INT4 page or the INT8 store as `view` selects.  For inspection and tests. */
+ * INT4 page or the INT8 store as `view` selects (NVFP4 pages: x^ = e2m1(code)
+ * * e4m3(scale)).  For inspection and tests. */
 int kv4_dequantize_debug(kv4_cache* cache, int32_t layer, int32_t seq_id, int32_t start, int32_t count,
                          int32_t view, float* dev_k_out, float* dev_v_out, kv4_stream_t stream);
 

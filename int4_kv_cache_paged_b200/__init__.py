@@ -58,6 +58,9 @@ KV4_ROPE_GPTJ = 1
 KV4_VIEW_EFFECTIVE = 0
 KV4_VIEW_INT4 = 1
 
+KV4_FORMAT_INT4 = 0
+KV4_FORMAT_NVFP4 = 1
+
 EXPORTS = [
     "kv4_cache_required_bytes", "kv4_cache_create", "kv4_cache_destroy", "kv4_cache_layout", "kv4_seq_reset",
     "kv4_rotate_quantize_append", "kv4_attention_workspace_bytes", "kv4_decode_attention",
@@ -74,7 +77,7 @@ EXPORTS = [
 class kv4_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "num_layers", "max_seqs", "num_q_heads", "num_kv_heads", "head_dim", "page_size", "num_pages",
-        "max_pages_per_seq", "hadamard_block", "sink_tokens", "recent_window")]
+        "max_pages_per_seq", "hadamard_block", "sink_tokens", "recent_window", "page_format")]
 
 
 _P = ctypes.c_void_p

@@ -25,6 +25,10 @@ def _tile16(D):
     return 64 * D
 
 
+def _tilef(D):
+    return 18 * D
+
+
 class _Base:
     def _view(self, ptr, nbytes, shape):
         off = ptr - self.buf.data_ptr()
@@ -74,7 +78,8 @@ class KV4Cache(_Base):
     def pages(self, layer):
         c = self.cfg
         ptr, _, _ = kv4_cache_layout(self.handle, layer)
-        shape = (c["num_pages"], c["page_size"] // TILE, c["num_kv_heads"], _tile4(c["head_dim"]))
+        tile = _tilef(c["head_dim"]) if c.get("page_format", 0) == 1 else _tile4(c["head_dim"])
+        shape = (c["num_pages"], c["page_size"] // TILE, c["num_kv_heads"], tile)
         n = shape[0] * shape[1] * shape[2] * shape[3]
         return self._view(ptr, n, shape)
 

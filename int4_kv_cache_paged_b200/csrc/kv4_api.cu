@@ -26,6 +26,7 @@ int check_config(const kv4_config* c, bool bf16) {
   if (c->head_dim != 64 && c->head_dim != 128) return KV4_ERR_UNSUPPORTED;
   if (c->page_size < 16 || c->page_size % 16 || c->page_size > 1024) return KV4_ERR_UNSUPPORTED;
   if (static_cast<long long>(c->max_pages_per_seq) * c->page_size > (1LL << 30)) return KV4_ERR_UNSUPPORTED;
+  if (c->page_format != KV4_FORMAT_INT4 && (bf16 || c->page_format != KV4_FORMAT_NVFP4)) return KV4_ERR_INVALID_ARG;
   if (!bf16) {
     if (!is_pow2(c->hadamard_block) || c->head_dim % c->hadamard_block) return KV4_ERR_INVALID_ARG;
     if (c->sink_tokens < 0 || c->recent_window < 1) return KV4_ERR_INVALID_ARG;
@@ -43,7 +44,8 @@ Sizes sizes_of(const kv4_config* c, bool bf16) {
   const size_t Hkv = c->num_kv_heads, D = c->head_dim;
   const size_t tiles_per_page = c->page_size / kv4::TILE;
   s.seq_lens = align_up(sizeof(int32_t) * static_cast<size_t>(c->num_layers) * c->max_seqs);
-  const size_t tile = bf16 ? kv4::tile16_bytes(static_cast<int>(D)) : kv4::tile4_bytes(static_cast<int>(D));
+  const size_t tile = bf16 ? kv4::tile16_bytes(static_cast<int>(D))
+                           : kv4::page_tile_bytes(static_cast<int>(D), c->page_format);
   s.pool = align_up(static_cast<size_t>(c->num_pages) * Hkv * tiles_per_page * tile);
   s.prot = bf16 ? 0
                 : align_up(static_cast<size_t>(c->max_seqs) * Hkv * kv4::n_prot_tiles(c->sink_tokens, c->recent_window) *

@@ -180,6 +180,7 @@ struct DequantParams {
   float* v_out;
   int seq, start, count, view;
   int Hkv, D, P, S, W, max_pages_per_seq, num_pages;
+  int fmt;   // page format
 };
 
 __global__ void dequant_kernel(DequantParams p) {
@@ -220,6 +221,30 @@ __global__ void dequant_kernel(DequantParams p) {
       return;
     }
     const int r = pos & 15;
+    if (p.fmt == KV4_FORMAT_NVFP4) {   // x^ = e2m1(code) * e4m3(scale of the 16-dim block)
+      const uint8_t* tile = p.pool + ((static_cast<long long>(page) * (p.P / 16) + (pos % p.P) / 16) * p.Hkv + h) *
+                                         tilef_bytes(D);
+      const int g = r & 7, rh = r >> 3, th = r >> 3, t = (r & 7) >> 1, e = r & 1;
+      for (int d = lane; d < D; d += 32) {
+        int byte, half, sbyte;
+        if (tensor == 0) {
+          const int b = d >> 4, tt = (d >> 2) & 3, j = (d >> 1) & 1;
+          byte = 16 * (4 * g + tt) + 4 * (b & 3) + 512 * (b >> 2) + rh + 2 * j;
+          half = d & 1;
+          sbyte = 16 * D + (D / 8) * g + 2 * b + rh;
+        } else {
+          const int m = d >> 4, dh = (d >> 3) & 1, gg = d & 7;
+          byte = 8 * D + 16 * (4 * gg + t) + 4 * (m & 3) + 512 * (m >> 2) + dh + 2 * th;
+          half = e;
+          sbyte = 17 * D + (D / 4) * t + 4 * m + 2 * th + e;
+        }
+        const uint32_t code = (tile[byte] >> (4 * half)) & 15u;
+        const uint32_t ee = (code >> 1) & 3u, mm = code & 1u;
+        const float mag = ee == 0u ? 0.5f * static_cast<float>(mm) : ldexpf(1.f + 0.5f * static_cast<float>(mm), ee - 1);
+        out[d] = (code & 8u ? -mag : mag) * e4m3_value(tile[sbyte]);
+      }
+      return;
+    }
     const uint8_t* tile = p.pool + ((static_cast<long long>(page) * (p.P / 16) + (pos % p.P) / 16) * p.Hkv + h) *
                                        tile4_bytes(D);
     const uint32_t sz = *reinterpret_cast<const uint32_t*>(tile + 16 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3)));
@@ -290,6 +315,7 @@ int launch_dequantize_debug(kv4_cache* c, int layer, int seq_id, int start, int 
   p.W = cfg.recent_window;
   p.max_pages_per_seq = cfg.max_pages_per_seq;
   p.num_pages = cfg.num_pages;
+  p.fmt = cfg.page_format;
   const long long threads = static_cast<long long>(count) * p.Hkv * 2 * 32;
   const long long blocks = (threads + 255) / 256;
   dequant_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);

@@ -19,6 +19,7 @@ struct AppendParams {
   State* state;
   int n_seqs, total_new, Hkv, D, P, S, W, Bh;
   int max_seqs, num_pages, max_pages_per_seq;
+  int fmt;                   // page format: KV4_FORMAT_INT4 or KV4_FORMAT_NVFP4
   float rot_c;               // fp32(1/sqrt(Bh))
   RopeParams rope;           // RoPE of the keys at their positions (cs == nullptr: none)
 };
@@ -122,6 +123,89 @@ __device__ __forceinline__ void store_int4(uint8_t* tile, int r, int tensor, con
   if (lane == 0) *reinterpret_cast<uint32_t*>(tile + 16 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3))) = sz;
 }
 
+// ---------------------------------------------------------------------------
+// NVFP4 pages ("KV Cache Quantization" topic page, item 3: NVFP4 storage of the
+// paged KV cache; blocks of 16 dims, E2M1 codes, one E4M3 scale, per-tensor
+// scale 1).  Per block: amax = max |x| (exact), s = fp32(amax / 6), s8 = s
+// rounded to the nearest E4M3 value (ties to even, saturating at 448); code =
+// the nearest E2M1 magnitude of fp32(x / s8) (ties to the even mantissa,
+// saturating at 6), sign bit only for a nonzero magnitude; s8 = 0 gives codes 0.
+
+// E4M3 code of s >= 0 (round to nearest even, saturated at 448).
+__device__ __forceinline__ uint32_t e4m3_rn(float s) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(r) : "f"(s));
+  return r & 0xFFu;
+}
+// Value of an E4M3 code (exact in fp32).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(code & 0xFFu)));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu)));
+}
+// E2M1 code of q: seven comparisons on |q| (ties at 0.25, 1.25, 2.5, 5 stay down, at 0.75, 1.75, 3.5
+// go up: the even mantissa), saturating at 6; the sign bit only for a nonzero magnitude.
+__device__ __forceinline__ uint32_t e2m1_code(float q) {
+  const float a = fabsf(q);
+  const uint32_t mag = static_cast<uint32_t>(a > 0.25f) + static_cast<uint32_t>(a >= 0.75f) +
+                       static_cast<uint32_t>(a > 1.25f) + static_cast<uint32_t>(a >= 1.75f) +
+                       static_cast<uint32_t>(a > 2.5f) + static_cast<uint32_t>(a >= 3.5f) +
+                       static_cast<uint32_t>(a > 5.f);
+  return mag | ((q < 0.f && mag != 0u) ? 8u : 0u);
+}
+
+// Quantize the warp's row (VPL dims per lane) in blocks of 16 dims: codes (one byte per dim) to smem,
+// the E4M3 scale code of the lane's block returned.
+template <int VPL>
+__device__ __forceinline__ uint32_t quantize_fp4(const float (&x)[VPL], uint8_t* codes, int lane) {
+  constexpr int LPB = 16 / VPL;   // lanes per block
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) a = fmaxf(a, fabsf(x[i]));
+#pragma unroll
+  for (int o = 1; o < LPB; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  const uint32_t s8 = e4m3_rn(__fdiv_rn(a, 6.f));
+  const float s = e4m3_value(s8);
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) codes[VPL * lane + i] = static_cast<uint8_t>(s > 0.f ? e2m1_code(__fdiv_rn(x[i], s)) : 0u);
+  return s8;
+}
+
+// Write one token's NVFP4 codes and scales into its page tile (layout: see the tile description of the
+// attention kernel).  K bytes belong to the token; a V byte holds one dim of tokens 2i and 2i+1, so the
+// token's V nibbles go in with atomic and/or on their 32-bit words (the other token may be written by
+// another warp of the same launch).  s8: the E4M3 code of the lane's block (VPL dims per lane).
+template <int VPL>
+__device__ __forceinline__ void store_fp4(uint8_t* tile, int r, int tensor, const uint8_t* codes, uint32_t s8,
+                                          int D, int lane) {
+  constexpr int LPB = 16 / VPL;
+  const int nb = D / 16;
+  const uint32_t sb = __shfl_sync(0xffffffffu, s8, (lane % nb) * LPB);   // lane b < nb: the scale of block b
+  if (tensor == 0) {
+    const int g = r & 7, rh = r >> 3;
+    for (int q = lane; q < D / 2; q += 32) {   // q = 8 b + 2 t + j: dims 16 b + 4 t + 2 j, +1
+      const int j = q & 1, t = (q >> 1) & 3, b = q >> 3;
+      const int d = 16 * b + 4 * t + 2 * j;
+      tile[16 * (4 * g + t) + 4 * (b & 3) + 512 * (b >> 2) + rh + 2 * j] =
+          static_cast<uint8_t>(codes[d] | (codes[d + 1] << 4));
+    }
+    if (lane < nb) tile[16 * D + (D / 8) * g + 2 * lane + rh] = static_cast<uint8_t>(sb);
+  } else {
+    const int th = r >> 3, t = (r & 7) >> 1, e = r & 1;
+    for (int q = lane; q < D / 2; q += 32) {   // q = 8 m + gg: dims 16 m + gg (byte 2 th) and + 8 (byte 2 th + 1)
+      const int m = q >> 3, gg = q & 7;
+      uint32_t* w = reinterpret_cast<uint32_t*>(tile + 8 * D + 16 * (4 * gg + t) + 4 * (m & 3) + 512 * (m >> 2));
+      const int sh = 16 * th + 4 * e;
+      const uint32_t mask = (0xFu << sh) | (0xFu << (sh + 8));
+      const uint32_t val = (static_cast<uint32_t>(codes[16 * m + gg]) << sh) |
+                           (static_cast<uint32_t>(codes[16 * m + gg + 8]) << (sh + 8));
+      atomicAnd(w, ~mask);
+      atomicOr(w, val);
+    }
+    if (lane < nb) tile[17 * D + (D / 4) * t + 4 * lane + 2 * th + e] = static_cast<uint8_t>(sb);
+  }
+}
+
 // Write one token's INT8 codes and scales into its protected tile.
 __device__ __forceinline__ void store_int8(uint8_t* tile, int r, int tensor, const uint8_t* codes, uint32_t sz,
                                            int D, int lane) {
@@ -174,6 +258,7 @@ inline AppendParams append_params(const kv4_cache* c, int layer, const int32_t* 
   p.num_pages = cfg.num_pages;
   p.max_pages_per_seq = cfg.max_pages_per_seq;
   p.rot_c = static_cast<float>(1.0 / sqrt(static_cast<double>(p.Bh)));
+  p.fmt = c->bf16 ? KV4_FORMAT_INT4 : cfg.page_format;
   return p;
 }
 
@@ -209,12 +294,14 @@ __device__ __forceinline__ void encode_row(const AppendParams& p, const uint16_t
   for (int k = 1; k < VPL; ++k) { mn = fminf(mn, x[k]); mx = fmaxf(mx, x[k]); }
   mn = warp_min(mn);
   mx = warp_max(mx);
-  const uint32_t sz4 = quantize_group<VPL>(x, mn, mx, 15.f, c4, lane);
+  const bool fp4 = p.fmt == KV4_FORMAT_NVFP4;
+  const uint32_t sz4 = fp4 ? quantize_fp4<VPL>(x, c4, lane) : quantize_group<VPL>(x, mn, mx, 15.f, c4, lane);
   const bool protect = pos < p.S || pos >= L_new - p.W;
   uint32_t sz8 = 0;
   if (protect) sz8 = quantize_group<VPL>(x, mn, mx, 255.f, c8, lane);
   __syncwarp();
-  store_int4(p.pool + tile_idx * tile4_bytes(D), r, tensor, c4, sz4, D, lane);
+  if (fp4) store_fp4<VPL>(p.pool + tile_idx * tilef_bytes(D), r, tensor, c4, sz4, D, lane);
+  else store_int4(p.pool + tile_idx * tile4_bytes(D), r, tensor, c4, sz4, D, lane);
   if (protect) {
     const int slot = pos < p.S ? pos : p.S + (pos - p.S) % p.W;
     const int npt = n_prot_tiles(p.S, p.W);

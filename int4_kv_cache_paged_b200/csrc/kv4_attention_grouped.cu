@@ -67,9 +67,10 @@ struct GShape {
   static constexpr int S8 = GWR / H8;
 };
 
-template <int D, int GWR>
+// F: page format (0 INT4, 1 NVFP4)
+template <int D, int GWR, int F = 0>
 struct GCfg {
-  static constexpr int STAGE4 = GWR * tile4_bytes(D);                  // one tile position of the group's heads
+  static constexpr int STAGE4 = GWR * page_tile_bytes(D, F);          // one tile position of the group's heads
   static constexpr int STAGE8 = GShape<GWR>::H8 * tile8_bytes(D);      // part of a protected tile position
   static constexpr int STAGE = STAGE4 > STAGE8 ? STAGE4 : STAGE8;
 };
@@ -143,9 +144,9 @@ __device__ __forceinline__ int cta_of(long long j, long long T, long long N) {
   return static_cast<int>(((j + 1) * N - 1) / T);
 }
 
-template <int D, int GWR>
+template <int D, int GWR, int F = 0>
 __host__ __device__ inline size_t gattn_smem_bytes(int ns) {
-  using C = GCfg<D, GWR>;
+  using C = GCfg<D, GWR, F>;
   return static_cast<size_t>(ns) * C::STAGE + GQD * sizeof(SegQ) + (2 * ns + 2 * GQD) * sizeof(uint64_t) +
          sizeof(GMisc);
 }
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(32 * QWARPS) gq_kernel(AttnParams p) {
   load_qfrag<D>(p, gw / p.Hkv, gw % p.Hkv, lane, qf);
   uint8_t* blob = p.qblob + static_cast<size_t>(gw) * qblob_bytes(D);
   if constexpr (D == 128) {
-    if (p.qfmt) store_qblob_tc<D>(blob, qf, lane);
+    if (p.qfmt == 1) store_qblob_tc<D>(blob, qf, lane);
     else store_qblob<D>(blob, qf, lane);
   } else {
     store_qblob<D>(blob, qf, lane);
@@ -374,7 +375,7 @@ __global__ void __launch_bounds__(32 * MAXW) gstep_kernel(AttnParams p, AppendPa
     load_qfrag<D>(p, b, h, lane, qf, s_ok ? L + 1 : L);
     uint8_t* blob = p.qblob + (static_cast<size_t>(b) * p.Hkv + h) * qblob_bytes(D);
     if constexpr (D == 128) {
-      if (p.qfmt) store_qblob_tc<D>(blob, qf, lane);
+      if (p.qfmt == 1) store_qblob_tc<D>(blob, qf, lane);
       else store_qblob<D>(blob, qf, lane);
     } else {
       store_qblob<D>(blob, qf, lane);
@@ -395,9 +396,9 @@ __global__ void __launch_bounds__(32 * MAXW) gstep_kernel(AttnParams p, AppendPa
 // ---------------------------------------------------------------------------
 // the attention kernel
 
-template <int D, int GWR>
+template <int D, int GWR, int F>
 __device__ __forceinline__ const uint8_t* stage_source(const AttnParams& p, const Group& g, int u, uint32_t& bytes) {
-  using C = GCfg<D, GWR>;
+  using C = GCfg<D, GWR, F>;
   using SH = GShape<GWR>;
   if (u < g.n4) {
     const int pos = (g.t0 + u) * TILE;
@@ -408,7 +409,7 @@ __device__ __forceinline__ const uint8_t* stage_source(const AttnParams& p, cons
     }
     bytes = C::STAGE4;
     return p.pool + ((static_cast<long long>(page) * (p.P / TILE) + (pos % p.P) / TILE) * p.Hkv + g.hg * GWR) *
-                        tile4_bytes(D);
+                        page_tile_bytes(D, F);
   }
   // part (v % S8) of protected tile v / S8: heads H8 * (v % S8) .. of the group
   const int v = u - g.n4;
@@ -506,11 +507,11 @@ __device__ bool plan_share(const AttnParams& p, GPlanRec* plan, GMisc* misc, int
 // stage of a batch, mbarrier completion).  Consumers release a stage once per
 // group of consumers (the empty barriers count GWR arrivals).  Every wait is
 // bounded; before the warp exits, every copy it issued has landed.
-template <int D, int GWR>
+template <int D, int GWR, int F = 0>
 __device__ void produce(const AttnParams& p, GMisc* misc, SegQ* segq, uint8_t* ring, int NS, uint32_t full0,
                         uint32_t empty0, uint32_t iqf0, uint32_t iqe0, int c, int j0, int j1, long long T, long long N,
                         int lane, volatile int* abort_flag, int* status) {
-  using C = GCfg<D, GWR>;
+  using C = GCfg<D, GWR, F>;
   const int HGN = p.Hkv / GWR;
   // ------------------------------------------------------------ producer
   const int nbatch = NS < 32 ? NS : 32;
@@ -550,7 +551,7 @@ __device__ void produce(const AttnParams& p, GMisc* misc, SegQ* segq, uint8_t* r
       bool lane_ok = true;
       if (lane < nbatch && base + lane < n) {
         uint32_t bytes;
-        const uint8_t* src = stage_source<D, GWR>(p, g, u + base + lane, bytes);
+        const uint8_t* src = stage_source<D, GWR, F>(p, g, u + base + lane, bytes);
         const uint32_t jl = jj + base + lane;
         const int s = jl % NS;
         lane_ok = mbar_wait(empty0 + 8 * s, ((jl / NS) & 1) ^ 1, abort_flag, status);
@@ -600,9 +601,10 @@ __device__ void produce(const AttnParams& p, GMisc* misc, SegQ* segq, uint8_t* r
 // PAIR = INT4 tiles per iteration of a consumer warp (1, 2 or 4).  MULTI:
 // several query tokens per sequence (causal visibility per operand column);
 // the one-token variant carries none of that code.  GWR: KV heads per group.
-template <int D, int PAIR, bool MULTI, int GWR>
+// F: page format (0 INT4, 1 NVFP4; the INT8 store is the same).
+template <int D, int PAIR, bool MULTI, int GWR, int F = 0>
 __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
-  using C = GCfg<D, GWR>;
+  using C = GCfg<D, GWR, F>;
   using SH = GShape<GWR>;
   constexpr int GTHREADS = SH::THREADS;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -634,7 +636,8 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
   if (!plan_share<GWR>(p, plan, misc, c, tid, GTHREADS, T, N, j0, j1)) return;
 
   if (warp == GWR) {
-    produce<D, GWR>(p, misc, segq, ring, NS, full0, empty0, iqf0, iqe0, c, j0, j1, T, N, lane, abort_flag, status);
+    produce<D, GWR, F>(p, misc, segq, ring, NS, full0, empty0, iqf0, iqe0, c, j0, j1, T, N, lane, abort_flag,
+                       status);
     return;
   }
 
@@ -701,7 +704,7 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
 #pragma unroll
         for (int k = 0; k < PAIR; ++k) {
           if (k < nt) {
-            tl[k] = smem_u32(ring + static_cast<size_t>(s) * C::STAGE + w * tile4_bytes(D));
+            tl[k] = smem_u32(ring + static_cast<size_t>(s) * C::STAGE + w * page_tile_bytes(D, F));
             eb[k] = empty0 + 8 * s;
             if (ok) ok = mbar_wait(full0 + 8 * s, par, abort_flag, status);
             advance();
@@ -717,8 +720,13 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
         if (inside) {
 #pragma unroll
           for (int k = 0; k < PAIR; ++k) valid[k] = 15;
-          if (nt == PAIR) unit_int4<D, PAIR, false>(tl, qf, ws, lane, valid, eb, cs);
-          else unit_int4<D, 1, false>(tl, qf, ws, lane, valid, eb, cs);
+          if constexpr (F == 1) {
+            if (nt == PAIR) unit_fp4<D, PAIR, false>(tl, qf, ws, lane, valid, valid, eb, cs);
+            else unit_fp4<D, 1, false>(tl, qf, ws, lane, valid, valid, eb, cs);
+          } else {
+            if (nt == PAIR) unit_int4<D, PAIR, false>(tl, qf, ws, lane, valid, eb, cs);
+            else unit_int4<D, 1, false>(tl, qf, ws, lane, valid, eb, cs);
+          }
         } else {
 #pragma unroll
           for (int k = 0; k < PAIR; ++k) {
@@ -730,8 +738,16 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
             else
               valid[k] = (r0 ? 3 : 0) | (r8 ? 12 : 0);
           }
-          if (nt == PAIR) unit_int4<D, PAIR, true, MULTI>(tl, qf, ws, lane, valid, eb, cs);
-          else unit_int4<D, 1, true, MULTI>(tl, qf, ws, lane, valid, eb, cs);
+          if constexpr (F == 1) {
+            int nwr[PAIR];   // written slots of each tile (the sequence's positions below L)
+#pragma unroll
+            for (int k = 0; k < PAIR; ++k) nwr[k] = min(max(g.L - (pos0 + k * TILE), 0), TILE);
+            if (nt == PAIR) unit_fp4<D, PAIR, true, MULTI>(tl, qf, ws, lane, valid, nwr, eb, cs);
+            else unit_fp4<D, 1, true, MULTI>(tl, qf, ws, lane, valid, nwr, eb, cs);
+          } else {
+            if (nt == PAIR) unit_int4<D, PAIR, true, MULTI>(tl, qf, ws, lane, valid, eb, cs);
+            else unit_int4<D, 1, true, MULTI>(tl, qf, ws, lane, valid, eb, cs);
+          }
         }
         u += nt;
       } else {
@@ -747,10 +763,11 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
           const uint32_t st = smem_u32(ring + static_cast<size_t>(s0) * C::STAGE + (w % SH::H8) * tile8_bytes(D));
           const int slot0 = (v / SH::S8) * TILE;
           if (slot0 + TILE <= g.nprot && !MULTI) {
-            tile_int8<D, false>(st, qf, ws, lane, 15, eb, cs);
+            tile_int8<D, false, false, F == 1>(st, qf, ws, lane, 15, eb, cs);
           } else if (!MULTI) {
-            tile_int8<D, true>(st, qf, ws, lane, (slot0 + g8 < g.nprot ? 3 : 0) | (slot0 + g8 + 8 < g.nprot ? 12 : 0),
-                               eb, cs);
+            tile_int8<D, true, false, F == 1>(st, qf, ws, lane,
+                                              (slot0 + g8 < g.nprot ? 3 : 0) | (slot0 + g8 + 8 < g.nprot ? 12 : 0),
+                                              eb, cs);
           } else {
             // position of protected slot sl: a sink below S, else the ring position
             // in [max(S, L - W), L) congruent to sl - S modulo W
@@ -763,7 +780,7 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
             const int pa = pos_of(sa), pb = pos_of(sb);
             const int vm = (ra && pa <= vis + qt0 ? 1 : 0) | (ra && pa <= vis + qt1 ? 2 : 0) |
                            (rb && pb <= vis + qt0 ? 4 : 0) | (rb && pb <= vis + qt1 ? 8 : 0);
-            tile_int8<D, true, true>(st, qf, ws, lane, vm, eb, cs);
+            tile_int8<D, true, true, F == 1>(st, qf, ws, lane, vm, eb, cs);
           }
         } else {
           __syncwarp();
@@ -1454,25 +1471,25 @@ GLayout g_layout(const kv4_cache* c, int n_seqs, int qlen) {
 }
 
 // Deepest ring (at most MAX_NS stages) that keeps CTAS_PER_SM CTAs of both
-// variants (one and several query tokens) resident per SM.
-template <int D, int PAIR, int GWR>
+// variants (one and several query tokens) of page format F resident per SM.
+template <int D, int PAIR, int GWR, int F>
 int g_choose_ring(int device) {
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess) return -1;
-  if (cudaFuncSetAttribute(gattn_kernel<D, PAIR, false, GWR>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(gattn_kernel<D, PAIR, true, GWR>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) !=
-          cudaSuccess)
+  if (cudaFuncSetAttribute(gattn_kernel<D, PAIR, false, GWR, F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           optin) != cudaSuccess ||
+      cudaFuncSetAttribute(gattn_kernel<D, PAIR, true, GWR, F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           optin) != cudaSuccess)
     return -1;
   const int want = CTAS_PER_SM;
   for (int ns = MAX_NS; ns >= 2; --ns) {
-    const size_t smem = gattn_smem_bytes<D, GWR>(ns);
+    const size_t smem = gattn_smem_bytes<D, GWR, F>(ns);
     if (smem > static_cast<size_t>(optin)) continue;
     int blocks = 0;
     int blocks_multi = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, gattn_kernel<D, PAIR, false, GWR>,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, gattn_kernel<D, PAIR, false, GWR, F>,
                                                       GShape<GWR>::THREADS, smem) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_multi, gattn_kernel<D, PAIR, true, GWR>,
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_multi, gattn_kernel<D, PAIR, true, GWR, F>,
                                                       GShape<GWR>::THREADS, smem) != cudaSuccess)
       return -1;
     if (blocks >= want && blocks_multi >= want) return ns;
@@ -1487,9 +1504,10 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   p.qblob = wsb + l.qblob;
   p.partials = reinterpret_cast<float*>(wsb + l.partials);
   GPlanRec* plan = reinterpret_cast<GPlanRec*>(wsb + l.plan);
-  // one query token, 4-head groups, D = 128: the tensor-memory kernel, one CTA per SM
-  const bool tcpath = D == 128 && GWR == 4 && c->use_tc && p.qtot == 1;
-  p.qfmt = tcpath ? 1 : 0;
+  // one query token, 4-head groups, D = 128, INT4 pages: the tensor-memory kernel when selected, one CTA per SM
+  const bool fp4 = c->cfg.page_format == KV4_FORMAT_NVFP4;
+  const bool tcpath = D == 128 && GWR == 4 && c->use_tc && p.qtot == 1 && !fp4;
+  p.qfmt = tcpath ? 1 : (fp4 ? 2 : 0);
   p.grid = tcpath ? c->num_sms : g_grid(c);
   p.cap_parts = p.grid * 2 * GWR;
   p.ns = tcpath ? c->tattn_ring : c->gattn_ring;
@@ -1509,7 +1527,8 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.grid);
   cfg.blockDim = dim3(tcpath ? TC_THREADS : GShape<GWR>::THREADS);
-  cfg.dynamicSmemBytes = tcpath ? tattn_smem_bytes<D>(p.ns) : gattn_smem_bytes<D, GWR>(p.ns);
+  cfg.dynamicSmemBytes = tcpath ? tattn_smem_bytes<D>(p.ns)
+                                : (fp4 ? gattn_smem_bytes<D, GWR, 1>(p.ns) : gattn_smem_bytes<D, GWR>(p.ns));
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1518,7 +1537,10 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   cfg.numAttrs = step ? 0 : 1;
   // several query tokens per sequence (even a pass of one of them): the causal variant
   cudaError_t e;
-  if constexpr (D == 128 && GWR == 4) {
+  if (fp4) {
+    e = p.qtot > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true, GWR, 1>, p, plan)
+                   : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false, GWR, 1>, p, plan);
+  } else if constexpr (D == 128 && GWR == 4) {
     if (tcpath) e = cudaLaunchKernelEx(&cfg, tattn_kernel<D>, p, plan);
     else if (p.qtot > 1) e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true, GWR>, p, plan);
     else e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false, GWR>, p, plan);
@@ -1547,12 +1569,12 @@ int g_launch_gw(kv4_cache* c, const AttnParams& p, void* ws, cudaStream_t stream
   }
 }
 
-template <int D>
+template <int D, int F>
 int g_choose_ring_gw(int device, int Hkv) {
   switch (group_width(Hkv)) {
-    case 4: return g_choose_ring<D, kPair, 4>(device);
-    case 2: return g_choose_ring<D, kPair, 2>(device);
-    default: return g_choose_ring<D, kPair, 1>(device);
+    case 4: return g_choose_ring<D, kPair, 4, F>(device);
+    case 2: return g_choose_ring<D, kPair, 2, F>(device);
+    default: return g_choose_ring<D, kPair, 1, F>(device);
   }
 }
 
@@ -1581,7 +1603,7 @@ int grouped_ring(kv4_cache* c) {
   c->gattn_pair = kPair;
   c->use_tc = false;
   c->tattn_ring = 0;
-  if (c->cfg.head_dim == 128 && group_width(c->cfg.num_kv_heads) == 4) {
+  if (c->cfg.head_dim == 128 && group_width(c->cfg.num_kv_heads) == 4 && c->cfg.page_format == KV4_FORMAT_INT4) {
     // "tc": the tensor-memory kernel, an opt-in alternative (slower than the mma.sync kernel on B200)
     const char* env = getenv("KV4_ATTENTION_KERNEL");
     if (env && strcmp(env, "tc") == 0) {
@@ -1594,8 +1616,10 @@ int grouped_ring(kv4_cache* c) {
       }
     }
   }
-  return c->cfg.head_dim == 128 ? g_choose_ring_gw<128>(c->device, c->cfg.num_kv_heads)
-                                : g_choose_ring_gw<64>(c->device, c->cfg.num_kv_heads);
+  const int Hkv = c->cfg.num_kv_heads;
+  if (c->cfg.page_format == KV4_FORMAT_NVFP4)
+    return c->cfg.head_dim == 128 ? g_choose_ring_gw<128, 1>(c->device, Hkv) : g_choose_ring_gw<64, 1>(c->device, Hkv);
+  return c->cfg.head_dim == 128 ? g_choose_ring_gw<128, 0>(c->device, Hkv) : g_choose_ring_gw<64, 0>(c->device, Hkv);
 }
 
 size_t grouped_workspace_bytes(const kv4_cache* c, int n_seqs, int qlen) { return g_layout(c, n_seqs, qlen).total; }

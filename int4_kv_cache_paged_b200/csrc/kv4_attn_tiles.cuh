@@ -278,8 +278,188 @@ __device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& 
   }
 }
 
+// ---------------------------------------------------------------------------
+// NVFP4 pages ("KV Cache Quantization" topic page, item 3: NVFP4 storage of
+// the paged KV cache).  A tile holds E2M1 codes and one E4M3 scale per token
+// and 16 dims.  Both products run on 16x8x16 fp16 multiplies: the hardware
+// conversion turns each code byte into an fp16 pair, and the block scale
+// multiplies it exactly (e2m1 * e4m3 has at most 5 significant bits and stays
+// in the normal fp16 range), so the operands are the dequantized values
+// themselves.  The query is the fp16 fragment form (q * 2^e, exact for bf16
+// values): block b of the K operand holds dims 16b + 4t, 4t+1 (k 2t, 2t+1) and
+// 4t+2, 4t+3 (k 2t+8, 2t+9), and the query fragments use the same order.
+
+// The four E2M1 pairs of a word (byte i: its low nibble -> low half) as fp16x2.
+__device__ __forceinline__ void e2m1x8_to_half2(uint32_t w, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                                uint32_t& r3) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+      : "r"(w));
+}
+// Two E4M3 bytes (bits 0-7 -> low half, 8-15 -> high half) as fp16x2.
+__device__ __forceinline__ uint32_t e4m3x2_to_half2(uint32_t w) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(static_cast<uint16_t>(w & 0xFFFFu)));
+  return r;
+}
+__device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
+  const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+// (lo, lo) and (hi, hi) of a half2.
+__device__ __forceinline__ uint32_t half2_lolo(uint32_t x) { return __byte_perm(x, 0u, 0x1010); }
+__device__ __forceinline__ uint32_t half2_hihi(uint32_t x) { return __byte_perm(x, 0u, 0x3232); }
+
+// One unit of NT NVFP4 tiles at shared addresses tile[0 .. NT-1]: as unit_int4
+// (valid[] the same visibility bits), without zero points.  nwr[u]: slots of
+// tile u that hold written tokens (the rest may hold non-finite scales, which
+// must not reach the P.V operands); used when MASKED.
+template <int D, int NT, bool MASKED, bool CAUSAL = false>
+__device__ __forceinline__ void unit_fp4(const uint32_t* tile, const QFrag<D>& qf, WarpState<D>& ws, int lane,
+                                         const int* valid, const int* nwr, const uint32_t* eb, const ColSplit& cs) {
+  constexpr int NB = D / 16;
+  const int g8 = lane >> 2, t = lane & 3;
+  float x[NT][4];
+  uint32_t kw[NT][NB];
+  uint32_t ks[NT][NB / 2];   // K scale pairs (token g, token g+8) of blocks 2i (bits 0-15) and 2i+1
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    if constexpr (D == 128) {
+      const uint4 a = lds128(tile[u] + lane * 16), b = lds128(tile[u] + 512 + lane * 16);
+      kw[u][0] = a.x; kw[u][1] = a.y; kw[u][2] = a.z; kw[u][3] = a.w;
+      kw[u][4] = b.x; kw[u][5] = b.y; kw[u][6] = b.z; kw[u][7] = b.w;
+      const uint4 sc = lds128(tile[u] + 16 * D + 16 * g8);
+      ks[u][0] = sc.x; ks[u][1] = sc.y; ks[u][2] = sc.z; ks[u][3] = sc.w;
+    } else {
+      const uint4 a = lds128(tile[u] + lane * 16);
+      kw[u][0] = a.x; kw[u][1] = a.y; kw[u][2] = a.z; kw[u][3] = a.w;
+      const uint2 sc = lds64(tile[u] + 16 * D + 8 * g8);
+      ks[u][0] = sc.x; ks[u][1] = sc.y;
+    }
+  }
+  float acc[NT][4];
+#pragma unroll
+  for (int u = 0; u < NT; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[u][i] = 0.f;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      uint32_t a0, a1, a2, a3;   // (token g | g+8) x (dims 4t, 4t+1 | 4t+2, 4t+3) of block b
+      e2m1x8_to_half2(kw[u][b], a0, a1, a2, a3);
+      const uint32_t s2 = e4m3x2_to_half2(ks[u][b >> 1] >> (16 * (b & 1)));
+      const uint32_t sg = half2_lolo(s2), sg8 = half2_hihi(s2);
+      mma_f16(acc[u], hmul2_u(a0, sg), hmul2_u(a1, sg8), hmul2_u(a2, sg), hmul2_u(a3, sg8), qf.b[b][0],
+              qf.b[b][1]);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[u][i] = acc[u][i] * qf.kscale;
+    if constexpr (MASKED && CAUSAL) {
+      if (!(valid[u] & 1)) x[u][0] = NEG_INF;
+      if (!(valid[u] & 2)) x[u][1] = NEG_INF;
+      if (!(valid[u] & 4)) x[u][2] = NEG_INF;
+      if (!(valid[u] & 8)) x[u][3] = NEG_INF;
+    } else if constexpr (MASKED) {
+      if (!(valid[u] & 1)) { x[u][0] = NEG_INF; x[u][1] = NEG_INF; }
+      if (!(valid[u] & 4)) { x[u][2] = NEG_INF; x[u][3] = NEG_INF; }
+    }
+  }
+  // online softmax over the unit (as unit_int4)
+  float mx0 = fmaxf(x[0][0], x[0][2]), mx1 = fmaxf(x[0][1], x[0][3]);
+#pragma unroll
+  for (int u = 1; u < NT; ++u) {
+    mx0 = fmaxf(mx0, fmaxf(x[u][0], x[u][2]));
+    mx1 = fmaxf(mx1, fmaxf(x[u][1], x[u][3]));
+  }
+  if (__any_sync(0xffffffffu, mx0 > ws.m0 || mx1 > ws.m1)) {
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float n0 = fmaxf(ws.m0, mx0), n1 = fmaxf(ws.m1, mx1);
+    const float a0 = (CAUSAL && n0 == NEG_INF) ? 1.f : ex2(ws.m0 - n0);
+    const float a1 = (CAUSAL && n1 == NEG_INF) ? 1.f : ex2(ws.m1 - n1);
+    ws.l0 *= a0; ws.l1 *= a1;
+#pragma unroll
+    for (int m = 0; m < D / 16; ++m) {
+      ws.o[m][0] *= a0; ws.o[m][1] *= a1; ws.o[m][2] *= a0; ws.o[m][3] *= a1;
+    }
+    ws.m0 = n0; ws.m1 = n1;
+  }
+  const float mu0 = (CAUSAL && ws.m0 == NEG_INF) ? 0.f : ws.m0;
+  const float mu1 = (CAUSAL && ws.m1 == NEG_INF) ? 0.f : ws.m1;
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    float P0 = ex2(x[u][0] - mu0), P1 = ex2(x[u][1] - mu1);
+    float P2 = ex2(x[u][2] - mu0), P3 = ex2(x[u][3] - mu1);
+    if constexpr (MASKED && CAUSAL) {
+      if (!(valid[u] & 1)) P0 = 0.f;
+      if (!(valid[u] & 2)) P1 = 0.f;
+      if (!(valid[u] & 4)) P2 = 0.f;
+      if (!(valid[u] & 8)) P3 = 0.f;
+    } else if constexpr (MASKED) {
+      if (!(valid[u] & 1)) { P0 = 0.f; P1 = 0.f; }
+      if (!(valid[u] & 4)) { P2 = 0.f; P3 = 0.f; }
+    }
+    ws.l0 += P0 + P2; ws.l1 += P1 + P3;
+    uint32_t B0, B1, C0, C1;
+    pv_operands(P0, P1, P2, P3, cs.part0, cs.part1, cs.colsplit, B0, B1, C0, C1);
+    // V: the word of lane 4g + t and dim block m holds (dims g, g + 8) x (tokens 2t, 2t+1 | 2t+8, 2t+9);
+    // the scales of those tokens in block m are the 4 bytes at 17D + (D/4) t + 4m
+    const uint32_t tv = tile[u];
+    uint32_t vw[NB], vs[NB];
+    if constexpr (D == 128) {
+      const uint4 v0 = lds128(tv + 8 * D + lane * 16), v1 = lds128(tv + 8 * D + 512 + lane * 16);
+      vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+      vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
+      const uint4 s0 = lds128(tv + 17 * D + (D / 4) * t), s1 = lds128(tv + 17 * D + (D / 4) * t + 16);
+      vs[0] = s0.x; vs[1] = s0.y; vs[2] = s0.z; vs[3] = s0.w;
+      vs[4] = s1.x; vs[5] = s1.y; vs[6] = s1.z; vs[7] = s1.w;
+    } else {
+      const uint4 v0 = lds128(tv + 8 * D + lane * 16);
+      vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+      const uint4 s0 = lds128(tv + 17 * D + (D / 4) * t);
+      vs[0] = s0.x; vs[1] = s0.y; vs[2] = s0.z; vs[3] = s0.w;
+    }
+    if (u == NT - 1) {   // the last loads of the unit are done: hand the stage(s) back
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int k = 0; k < NT; ++k)
+          if (k == 0 || eb[k] != eb[k - 1]) mbar_arrive(eb[k]);
+      }
+    }
+    if constexpr (MASKED) {
+      // unwritten slots (>= nwr[u]) may hold non-finite scales: zero them (their weights are zero)
+      const int n = nwr[u];
+      const uint32_t keep = (2 * t < n ? 0x000000FFu : 0u) | (2 * t + 1 < n ? 0x0000FF00u : 0u) |
+                            (2 * t + 8 < n ? 0x00FF0000u : 0u) | (2 * t + 9 < n ? 0xFF000000u : 0u);
+#pragma unroll
+      for (int m = 0; m < NB; ++m) vs[m] &= keep;
+    }
+#pragma unroll
+    for (int m = 0; m < NB; ++m) {
+      uint32_t a0, a1, a2, a3;   // (dim g | g+8) x (tokens 2t, 2t+1 | 2t+8, 2t+9)
+      e2m1x8_to_half2(vw[m], a0, a1, a2, a3);
+      const uint32_t s01 = e4m3x2_to_half2(vs[m]), s89 = e4m3x2_to_half2(vs[m] >> 16);
+      a0 = hmul2_u(a0, s01); a1 = hmul2_u(a1, s01); a2 = hmul2_u(a2, s89); a3 = hmul2_u(a3, s89);
+      mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
+      if (!cs.colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
+    }
+  }
+}
+
 // One INT8 tile (protected store).
-template <int D, bool MASKED, bool CAUSAL = false>
+// HQ: the query operand holds fp16 B fragments (the cache's pages are NVFP4, see unit_fp4); the K
+// codes then enter 16x8x16 fp16 multiplies as c - 128 (exact), the zero point as z + 128 s.
+template <int D, bool MASKED, bool CAUSAL = false, bool HQ = false>
 __device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, int vm,
                                           uint32_t empty_bar, const ColSplit& cs) {
   constexpr int NK = D / 16;
@@ -300,15 +480,26 @@ __device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpS
   const uint4 sz = lds128(st + 32 * D + (lane >> 2) * 16);
   __syncwarp();
   if (lane == 0) mbar_arrive(empty_bar);
-  int ahi[4] = {0, 0, 0, 0}, alo[4] = {0, 0, 0, 0};
-#pragma unroll
-  for (int kk = 0; kk < D / 32; ++kk)
-    qk_block<D>(ahi, alo, kw[0][2 * kk], kw[1][2 * kk], kw[0][2 * kk + 1], kw[1][2 * kk + 1], qf, kk);
   float acc[4];
+  if constexpr (HQ) {
+    // word k of a row holds dims 16k + 4t .. 16k + 4t + 3: the fp16 fragments' dim order
 #pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i] = static_cast<float>(ahi[i] * 256 + alo[i]);
-  const float sKg = half_lo(sz.x) * qf.kscale, zKg = half_hi(sz.x);
-  const float sKg8 = half_lo(sz.y) * qf.kscale, zKg8 = half_hi(sz.y);
+    for (int i = 0; i < 4; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int k = 0; k < NK; ++k)
+      mma_f16(acc, bytes01_c(kw[0][k]), bytes01_c(kw[1][k]), bytes23_c(kw[0][k]), bytes23_c(kw[1][k]), qf.b[k][0],
+              qf.b[k][1]);
+  } else {
+    int ahi[4] = {0, 0, 0, 0}, alo[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int kk = 0; kk < D / 32; ++kk)
+      qk_block<D>(ahi, alo, kw[0][2 * kk], kw[1][2 * kk], kw[0][2 * kk + 1], kw[1][2 * kk + 1], qf, kk);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = static_cast<float>(ahi[i] * 256 + alo[i]);
+  }
+  const float sKg = half_lo(sz.x) * qf.kscale, sKg8 = half_lo(sz.y) * qf.kscale;
+  const float zKg = HQ ? fmaf(128.f, half_lo(sz.x), half_hi(sz.x)) : half_hi(sz.x);
+  const float zKg8 = HQ ? fmaf(128.f, half_lo(sz.y), half_hi(sz.y)) : half_hi(sz.y);
   float x0 = fmaf(acc[0], sKg, zKg * qf.qs0);
   float x1 = fmaf(acc[1], sKg, zKg * qf.qs1);
   float x2 = fmaf(acc[2], sKg8, zKg8 * qf.qs0);
@@ -662,20 +853,32 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
     frexpf(amax, &ex);
     e = 15 - ex;
   }
+  if (p.qfmt == 2) {
+    // fp16 B fragments of 16x8x16 multiplies (NVFP4 pages): block 2kk + hf holds dims 4t, 4t+1
+    // (register 0) and 4t+2, 4t+3 (register 1) of column g, times 2^e (exact for bf16 values)
 #pragma unroll
-  for (int kk = 0; kk < NKK; ++kk)
+    for (int kk = 0; kk < NKK; ++kk)
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      uint32_t whi = 0u, wlo = 0u;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int qi = __float2int_rn(ldexpf(x[kk][hf][j], e));   // |qi| < 2^15
-        whi |= (static_cast<uint32_t>(qi >> 8) & 0xFFu) << (8 * j);
-        wlo |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * j);
+      for (int hf = 0; hf < 2; ++hf) {
+        qf.b[2 * kk + hf][0] = pack_half2(ldexpf(x[kk][hf][0], e), ldexpf(x[kk][hf][1], e));
+        qf.b[2 * kk + hf][1] = pack_half2(ldexpf(x[kk][hf][2], e), ldexpf(x[kk][hf][3], e));
       }
-      qf.b[kk][hf] = whi;
-      qf.b[NKK + kk][hf] = wlo;
-    }
+  } else {
+#pragma unroll
+    for (int kk = 0; kk < NKK; ++kk)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t whi = 0u, wlo = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int qi = __float2int_rn(ldexpf(x[kk][hf][j], e));   // |qi| < 2^15
+          whi |= (static_cast<uint32_t>(qi >> 8) & 0xFFu) << (8 * j);
+          wlo |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * j);
+        }
+        qf.b[kk][hf] = whi;
+        qf.b[NKK + kk][hf] = wlo;
+      }
+  }
   // sum(q) of the heads of this lane's columns 2t and 2t+1 (held by lanes 8t and 8t+4)
   qf.qs0 = __shfl_sync(0xffffffffu, qs, 8 * t) * p.scale_log2;
   qf.qs1 = __shfl_sync(0xffffffffu, qs, 8 * t + 4) * p.scale_log2;

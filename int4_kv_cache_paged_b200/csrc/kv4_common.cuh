@@ -39,6 +39,9 @@ constexpr int STATE_BYTES = 256;
 __host__ __device__ constexpr int tile4_bytes(int D) { return 16 * D + 128; }
 __host__ __device__ constexpr int tile8_bytes(int D) { return 32 * D + 128; }
 __host__ __device__ constexpr int tile16_bytes(int D) { return 64 * D; }
+// NVFP4 page tile: K codes 8*D, V codes 8*D, K scales D, V scales D (one E4M3 byte per token and 16 dims)
+__host__ __device__ constexpr int tilef_bytes(int D) { return 18 * D; }
+__host__ __device__ constexpr int page_tile_bytes(int D, int fmt) { return fmt == 1 ? tilef_bytes(D) : tile4_bytes(D); }
 __host__ __device__ constexpr int qblob_bytes(int D) { return 16 * D + 64; }
 __host__ __device__ inline int n_prot_tiles(int S, int W) { return (S + W + TILE - 1) / TILE; }
 
@@ -115,7 +118,8 @@ struct AttnParams {
   int ns;                     // shared-memory ring depth of the attention kernel
   int grid;                   // CTAs of the page-major attention kernel
   int stall_stage;            // test hook: stage the first CTA leaves unfilled (-1: none)
-  int qfmt;                   // query operand layout the query kernels write: 0 fragments, 1 tensor-memory kernel
+  int qfmt;                   // query operand layout the query kernels write: 0 integer fragments, 1 tensor-memory
+                              // kernel, 2 fp16 fragments (NVFP4 pages)
 };
 
 // Row of q (and of the output) that operand column c of KV head h of batch
@@ -367,6 +371,18 @@ __device__ __forceinline__ uint32_t nib_hi_c(uint32_t w) {  // nibbles at bits 4
 
 __device__ __forceinline__ uint32_t byte_lo_c(uint32_t w) {  // bytes 0 and 2, minus 128
   uint32_t x = lop3_and_or(w, 0x00FF00FFu, 0x64006400u);
+  __half2 h = __hsub2(*reinterpret_cast<__half2*>(&x), __half2(__half(1152.f), __half(1152.f)));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Bytes 0, 1 (or 2, 3) of w as an fp16 pair, minus 128 (exact).
+__device__ __forceinline__ uint32_t bytes01_c(uint32_t w) {
+  uint32_t x = __byte_perm(w, 0x64646464u, 0x4140);
+  __half2 h = __hsub2(*reinterpret_cast<__half2*>(&x), __half2(__half(1152.f), __half(1152.f)));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t bytes23_c(uint32_t w) {
+  uint32_t x = __byte_perm(w, 0x64646464u, 0x4342);
   __half2 h = __hsub2(*reinterpret_cast<__half2*>(&x), __half2(__half(1152.f), __half(1152.f)));
   return *reinterpret_cast<uint32_t*>(&h);
 }

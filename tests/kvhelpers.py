@@ -19,9 +19,10 @@ BF16_REL_L2 = 5e-3
 BF16_MAX_ABS = 4 * 2.0 ** -8
 
 
-def cfg_dict(D=128, Hq=32, Hkv=8, P=16, Bh=128, S=4, W=128, num_pages=64, mpps=16, max_seqs=4, layers=1):
+def cfg_dict(D=128, Hq=32, Hkv=8, P=16, Bh=128, S=4, W=128, num_pages=64, mpps=16, max_seqs=4, layers=1, fmt=0):
     return dict(num_layers=layers, max_seqs=max_seqs, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D, page_size=P,
-                num_pages=num_pages, max_pages_per_seq=mpps, hadamard_block=Bh, sink_tokens=S, recent_window=W)
+                num_pages=num_pages, max_pages_per_seq=mpps, hadamard_block=Bh, sink_tokens=S, recent_window=W,
+                page_format=fmt)
 
 
 def random_table(max_seqs, mpps, num_pages, rng):
@@ -99,6 +100,32 @@ def compare_int4_pages(pair, layer, seqs):
             o = pair.orc.pages[(layer, page)][ti][:, idx]
             if not np.array_equal(g, o):
                 bad.append((seq, p, int(np.sum(g != o))))
+    return bad
+
+
+def compare_fp4_pages(pair, layer, seqs):
+    """Bit-exact comparison of every NVFP4 code and scale owned by a written position of `seqs` (its K
+    bytes and scale bytes, and its nibble of each shared V byte)."""
+    c = pair.cfg
+    D, P = c["head_dim"], c["page_size"]
+    tf = tables("nvfp4", D)
+    pages = pair.gpu.pages(layer).cpu().numpy()
+    bad = []
+    for seq in seqs:
+        L = int(pair.orc.seq_lens[layer, seq])
+        for p in range(L):
+            page = int(pair.table[seq, p // P])
+            ti, r = (p % P) // TILE, p % TILE
+            idx = np.concatenate([tf.k_byte[r], tf.ks_byte[r], tf.vs_byte[r]])
+            g = pages[page, ti][:, idx]
+            o = pair.orc.pages[(layer, page)][ti][:, idx]
+            vb = 8 * D + tf.v_byte[r]
+            sh = 4 * tf.v_nib[r]
+            gv = (pages[page, ti][:, vb] >> sh) & 15
+            ov = (pair.orc.pages[(layer, page)][ti][:, vb] >> sh) & 15
+            n = int(np.sum(g != o)) + int(np.sum(gv != ov))
+            if n:
+                bad.append((seq, p, n))
     return bad
 
 

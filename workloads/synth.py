@@ -157,13 +157,13 @@ def queries_np(w, layer, step, n=None):
     return _bf16_bits_np(rng.standard_normal((B, w["Hq"], w["D"]), dtype=np.float32))
 
 
-def cache_config(w, num_pages, max_pages_per_seq, max_seqs=None, layers=None):
+def cache_config(w, num_pages, max_pages_per_seq, max_seqs=None, layers=None, page_format=0):
     """The cache configuration (field names of the C-ABI struct) for a workload."""
     return dict(num_layers=w["layers"] if layers is None else layers,
                 max_seqs=w["batch"] if max_seqs is None else max_seqs,
                 num_q_heads=w["Hq"], num_kv_heads=w["Hkv"], head_dim=w["D"],
                 page_size=w["P"], num_pages=num_pages, max_pages_per_seq=max_pages_per_seq,
-                hadamard_block=w["Bh"], sink_tokens=w["S"], recent_window=w["W"])
+                hadamard_block=w["Bh"], sink_tokens=w["S"], recent_window=w["W"], page_format=page_format)
 
 
 def rope_cos_sin(max_pos, rotary_dim, base=1.0e6):
