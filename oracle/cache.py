@@ -27,13 +27,16 @@ Readings of this library (the pages give none of these details):
   table is given (append(..., rope=...), see rope.py).
 * Page format (config key "page_format"): 0 = INT4 (the method), 1 = NVFP4,
   the alternative format of the "KV Cache Quantization" topic page, item 3
-  (see nvfp4.py).  The format changes only what the pages hold; the rotation,
-  the INT8 store of the protected positions and the effective view are the
-  same.  Below, "INT4 page" means the page copy in either format.
+  (see nvfp4.py), 2 = INT2, the folded-scale 2-bit variant of the same page's
+  item 2 (the token-wise quantizer of quant.py with Q = 3).  The format
+  changes only what the pages hold; the rotation, the INT8 store of the
+  protected positions and the effective view are the same.  Below, "INT4
+  page" means the page copy in any format.
 * Device byte order (head-innermost, so that the tiles of all KV heads at one
   page position are contiguous):
     INT4 pool of a layer   uint8 [num_pages][P/16][Hkv][16*D + 128]
     NVFP4 pool of a layer  uint8 [num_pages][P/16][Hkv][18*D]
+    INT2 pool of a layer   uint8 [num_pages][P/16][Hkv][8*D + 128]
     INT8 store of a layer  uint8 [max_seqs][ceil((S+W)/16)][Hkv][32*D + 128]
     BF16 pool of a layer   bf16  [num_pages][P/16][Hkv][32*D]
   The arrays below use the same order per page / per sequence.
@@ -45,7 +48,8 @@ from .hadamard import fwht_fp32
 from .rope import rope_fp32
 from .quant import quantize_groups, dequantize_groups
 from .nvfp4 import quantize_nvfp4, dequantize_nvfp4
-from .layout import TILE, tables, int4_tile_bytes, int8_tile_bytes, bf16_tile_bytes, fp4_tile_bytes, scale_offset
+from .layout import (TILE, tables, int4_tile_bytes, int8_tile_bytes, bf16_tile_bytes, fp4_tile_bytes,
+                     int2_tile_bytes, scale_offset)
 
 CONFIG_FIELDS = ("num_layers", "max_seqs", "num_q_heads", "num_kv_heads", "head_dim",
                  "page_size", "num_pages", "max_pages_per_seq", "hadamard_block",
@@ -89,8 +93,8 @@ class OracleKV4Cache:
         self.W = c["recent_window"]
         self.Bh = c["hadamard_block"]
         self.fmt = int(c.get("page_format", 0))
-        if self.fmt not in (0, 1):
-            raise ValueError("page_format must be 0 (INT4) or 1 (NVFP4)")
+        if self.fmt not in (0, 1, 2):
+            raise ValueError("page_format must be 0 (INT4), 1 (NVFP4) or 2 (INT2)")
         self.block_table = np.asarray(block_table, dtype=np.int64)
         self.seq_lens = np.zeros((c["num_layers"], c["max_seqs"]), np.int64)
         self.pages = {}
@@ -98,7 +102,8 @@ class OracleKV4Cache:
         self.t4 = tables("int4", self.D)
         self.t8 = tables("int8", self.D)
         self.tf = tables("nvfp4", self.D)
-        self.page_tile_bytes = fp4_tile_bytes(self.D) if self.fmt == 1 else int4_tile_bytes(self.D)
+        self.t2 = tables("int2", self.D)
+        self.page_tile_bytes = {0: int4_tile_bytes, 1: fp4_tile_bytes, 2: int2_tile_bytes}[self.fmt](self.D)
 
     # -- storage helpers -------------------------------------------------
     def _page_tiles(self, layer, page):
@@ -214,6 +219,50 @@ class OracleKV4Cache:
             out[1][sel] = dequantize_nvfp4(vc, self._gather(tiles, ts, tf.vs_byte[rs]))
         return out
 
+    def _write_int2(self, layer, seq, pos, enc_k, enc_v):
+        """INT2 codes (four a byte, token-owned bytes) and the half2 (s, z) of positions `pos`."""
+        D, t2 = self.D, self.t2
+        page = self._pages_of(seq, pos)
+        r = pos % TILE
+        ti = (pos % self.P) // TILE
+        for pg in np.unique(page):
+            sel = page == pg
+            tiles = self._page_tiles(layer, int(pg))
+            rs, ts = r[sel], ti[sel]
+            for tensor, (codes, s16, z16) in enumerate((enc_k, enc_v)):
+                byte = (t2.k_byte if tensor == 0 else 4 * D + t2.v_byte)[rs]              # [m, D/4]
+                dims = (t2.k_dims if tensor == 0 else t2.v_dims)[rs]                      # [m, D/4, 4]
+                c = codes[sel].astype(np.uint32)                                          # [m, Hkv, D]
+                packed = np.zeros(c.shape[:2] + (D // 4,), np.uint32)
+                for k in range(4):
+                    packed |= np.take_along_axis(c, dims[:, None, :, k], axis=2) << (2 * k)
+                self._scatter(tiles, ts, byte, packed.astype(np.uint8))
+                off = 8 * D + np.array([scale_offset(int(x), tensor) for x in rs])
+                self._scatter(tiles, ts, off[:, None] + np.arange(4), self._sz_bytes(s16[sel], z16[sel]))
+
+    def _read_int2(self, layer, seq, pos):
+        """Dequantized K^, V^ [m, Hkv, D] of positions `pos` from INT2 pages."""
+        D, t2 = self.D, self.t2
+        page = self._pages_of(seq, pos)
+        r = pos % TILE
+        ti = (pos % self.P) // TILE
+        out = [np.zeros((len(pos), self.Hkv, D), np.float32) for _ in range(2)]
+        for pg in np.unique(page):
+            sel = np.nonzero(page == pg)[0]
+            tiles = self._page_tiles(layer, int(pg))
+            rs, ts = r[sel], ti[sel]
+            for tensor in (0, 1):
+                byte = (t2.k_byte if tensor == 0 else 4 * D + t2.v_byte)[rs]
+                dims = (t2.k_dims if tensor == 0 else t2.v_dims)[rs]
+                b = self._gather(tiles, ts, byte)                                         # [m, Hkv, D/4]
+                codes = np.zeros((len(sel), self.Hkv, D), np.uint8)
+                for k in range(4):
+                    np.put_along_axis(codes, dims[:, None, :, k], (b >> (2 * k)) & 3, axis=2)
+                off = 8 * D + np.array([scale_offset(int(x), tensor) for x in rs])
+                s16, z16 = self._sz_values(self._gather(tiles, ts, off[:, None] + np.arange(4)))
+                out[tensor][sel] = dequantize_groups(codes, s16, z16)
+        return out
+
     def _write_int8(self, layer, seq, slots, enc_k, enc_v):
         D, t8 = self.D, self.t8
         tiles = self._prot_tiles(layer, seq)
@@ -264,10 +313,10 @@ class OracleKV4Cache:
 
     # -- the method --------------------------------------------------------
     def rotate_quantize(self, x):
-        """x: [n, Hkv, D] values (bf16 held in fp32).  Returns the rotation, the page encoding (INT4
-        (codes, s16, z16) or NVFP4 (codes, scales)) and the INT8 encoding."""
+        """x: [n, Hkv, D] values (bf16 held in fp32).  Returns the rotation, the page encoding (INT4 or
+        INT2 (codes, s16, z16), NVFP4 (codes, scales)) and the INT8 encoding."""
         xr = fwht_fp32(x, self.Bh)
-        page = quantize_nvfp4(xr) if self.fmt == 1 else quantize_groups(xr, 4)
+        page = quantize_nvfp4(xr) if self.fmt == 1 else quantize_groups(xr, 2 if self.fmt == 2 else 4)
         return xr, page, quantize_groups(xr, 8)
 
     def append(self, layer, seq_ids, cu_new, k_new, v_new, rope=None):
@@ -296,6 +345,8 @@ class OracleKV4Cache:
             _, v4, v8 = self.rotate_quantize(v_new[a:b])
             if self.fmt == 1:                                    # every position: the page copy
                 self._write_fp4(layer, seq, pos, k4, v4)
+            elif self.fmt == 2:
+                self._write_int2(layer, seq, pos, k4, v4)
             else:
                 self._write_int4(layer, seq, pos, k4, v4)
             prot = (pos < self.S) | (pos >= L_new - self.W)      # sinks, and the last W of this append
@@ -329,6 +380,8 @@ class OracleKV4Cache:
                 kv = self._read_int8(layer, seq, slots)
             elif self.fmt == 1:
                 kv = self._read_fp4(layer, seq, pos[sel])
+            elif self.fmt == 2:
+                kv = self._read_int2(layer, seq, pos[sel])
             else:
                 kv = self._read_int4(layer, seq, pos[sel])
             out[0][sel], out[1][sel] = kv

@@ -11,6 +11,7 @@ Unit of storage: a tile of 16 consecutive token slots of one KV head.
 INT4 tile (16*D + 128 bytes):   [K codes 8*D][V codes 8*D][scales 128]
 INT8 tile (32*D + 128 bytes):   [K codes 16*D][V codes 16*D][scales 128]
 NVFP4 tile (18*D bytes):        [K codes 8*D][V codes 8*D][K scales D][V scales D]
+INT2 tile (8*D + 128 bytes):    [K codes 4*D][V codes 4*D][scales 128]
 BF16 tile (64*D bytes):         [K 16*D bf16][V 16*D bf16]      (baseline cache)
 
 Inside the code blocks the order of nibbles/bytes follows the operand order
@@ -51,6 +52,10 @@ def bf16_tile_bytes(D):
 
 def fp4_tile_bytes(D):
     return 18 * D
+
+
+def int2_tile_bytes(D):
+    return 8 * D + 128
 
 
 def int4_k_nibble(D, r, d):
@@ -128,6 +133,39 @@ def bf16_v_elem(D, r, d):
     t, e = divmod(tt, 2)
     reg = dh + 2 * th
     return 8 * (32 * m + 4 * g + t) + 2 * reg + e
+
+
+def int2_k_crumb(D, r, d):
+    """(byte offset inside the INT2 K code block, crumb 0..3 = bits 2c, 2c+1) of token r, dim d.
+
+    Token r owns the D/4 bytes [r*D/4, (r+1)*D/4).  With d = 64*kq + 16*c + 4*t + j
+    (kq < D/64, c < 4, t < 4, j < 4), the code is crumb c of byte j of the 32-bit
+    word at r*D/4 + t*D/16 + 4*kq: shifting the word right by 2c and masking it
+    with 0x03030303 gives the four dims 4t..4t+3 of 16-dim block 4kq + c as bytes
+    (the INT4 layout's integer-multiply operand order, two bits a code).
+    """
+    kq, rem = divmod(d, 64)
+    c, rem = divmod(rem, 16)
+    t, j = divmod(rem, 4)
+    return r * (D // 4) + t * (D // 16) + 4 * kq + j, c
+
+
+def int2_v_crumb(D, r, d):
+    """(byte offset inside the INT2 V code block, crumb) of token r, dim d.
+
+    With d = 16*m + 8*dh + g (m = 2*mp + mb) and r = 8*th + 2*t + e, the code is
+    crumb i % 4 of byte i // 4 of the word at (D/8)*(4*g + t) + 4*mp, where
+    i = dh + 2*mb + 4*th + 8*e: a byte holds four dims of one token, and the
+    codes of tokens 2t and 2t+1 (e = 0, 1) sit 16 bits apart, the two halves of
+    one fp16x2 operand register.
+    """
+    m, rr = divmod(d, 16)
+    mp, mb = divmod(m, 2)
+    dh, g = divmod(rr, 8)
+    th, tt = divmod(r, 8)
+    t, e = divmod(tt, 2)
+    i = dh + 2 * mb + 4 * th + 8 * e
+    return (D // 8) * (4 * g + t) + 4 * mp + i // 4, i % 4
 
 
 def fp4_k_nibble(D, r, d):
@@ -226,6 +264,28 @@ class BF16Tables:
         self.v_elem = np.array([[bf16_v_elem(D, r, d) for d in range(D)] for r in range(TILE)], np.int64)
 
 
+class Int2Tables:
+    """For token slot r: the K and V bytes it owns (D/4 each) and, per byte, the dims of its four crumbs."""
+
+    def __init__(self, D):
+        self.D = D
+        for which, fn in (("k", int2_k_crumb), ("v", int2_v_crumb)):
+            byte = np.zeros((TILE, D // 4), np.int64)
+            dims = np.zeros((TILE, D // 4, 4), np.int64)
+            for r in range(TILE):
+                owned = {}
+                for d in range(D):
+                    b, c = fn(D, r, d)
+                    owned.setdefault(b, [None] * 4)[c] = d
+                if len(owned) != D // 4 or any(None in v for v in owned.values()):
+                    raise AssertionError("INT2 %s layout: token %d does not own whole bytes" % (which, r))
+                for n, b in enumerate(sorted(owned)):
+                    byte[r, n] = b
+                    dims[r, n] = owned[b]
+            setattr(self, which + "_byte", byte)
+            setattr(self, which + "_dims", dims)
+
+
 class Fp4Tables:
     """For token slot r: the K bytes it owns (D/2) with their low / high dims; per dim its V byte and
     nibble (D); its scale bytes per 16-dim block (D/16) for K and V."""
@@ -258,5 +318,6 @@ _cache = {}
 def tables(kind, D):
     key = (kind, D)
     if key not in _cache:
-        _cache[key] = {"int4": Int4Tables, "int8": Int8Tables, "bf16": BF16Tables, "nvfp4": Fp4Tables}[kind](D)
+        _cache[key] = {"int4": Int4Tables, "int8": Int8Tables, "bf16": BF16Tables, "nvfp4": Fp4Tables,
+                       "int2": Int2Tables}[kind](D)
     return _cache[key]

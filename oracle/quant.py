@@ -9,7 +9,9 @@ Sources:
 
 One quantization group is the D rotated values of one (token, KV head, K or V).
 Each group gets its own scale s and zero point z, stored as fp16; the codes
-are unsigned b-bit integers (b = 4 or 8, Q = 2^b - 1).
+are unsigned b-bit integers (b = 4 or 8, Q = 2^b - 1; b = 2 for the INT2 page
+format, the folded-scale INT2 variant of the "KV Cache Quantization" topic
+page, item 2, with the same token-wise groups and rounding rule).
 
 Rounding rule (a reading of this library; the pages fix none of it):
 
@@ -64,8 +66,8 @@ def quantize_groups(x, bits):
 
     Returns (codes uint8 [..., D], s16 float16 [...], z16 float16 [...]).
     """
-    if bits not in (4, 8):
-        raise ValueError("bits must be 4 or 8")
+    if bits not in (2, 4, 8):
+        raise ValueError("bits must be 2, 4 or 8")
     Q = np.float32(2 ** bits - 1)
     x = clamp_fp16_range(x)
     mn = x.min(axis=-1)

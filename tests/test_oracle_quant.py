@@ -55,7 +55,7 @@ def _golden():
 def test_worked_example():
     g = _golden()
     x = g["x"].astype(np.float32)[None]
-    for bits in (4, 8):
+    for bits in (2, 4, 8):
         c, s, z = quantize_groups(x, bits)
         p = "int%d." % bits
         np.testing.assert_array_equal(c[0], g[p + "codes"].astype(np.uint8))
@@ -75,7 +75,7 @@ def _groups(seed, n=400, D=128):
     return x.astype(np.float32)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [2, 4, 8])
 def test_codes_in_range_and_error_bound(bits):
     Q = 2 ** bits - 1
     x = _groups(1)
@@ -89,7 +89,7 @@ def test_codes_in_range_and_error_bound(bits):
     assert np.all(err <= s64 / 2 + slack)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [2, 4, 8])
 def test_scale_zero_definition(bits):
     Q = 2 ** bits - 1
     x = _groups(2)
@@ -109,7 +109,7 @@ def test_scale_zero_definition(bits):
     np.testing.assert_array_equal(sd, want)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [2, 4, 8])
 def test_exact_round_trip_on_representable_groups(bits):
     Q = 2 ** bits - 1
     rng = np.random.default_rng(3)
@@ -127,7 +127,7 @@ def test_exact_round_trip_on_representable_groups(bits):
         np.testing.assert_array_equal(dequantize_groups(c, s16, z16), x)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [2, 4, 8])
 def test_brute_force_nearest_code(bits):
     Q = 2 ** bits - 1
     rng = np.random.default_rng(4)
