@@ -78,12 +78,12 @@ def parse(argv=None):
 
 # --------------------------------------------------------------------------- helpers
 
-def kv_bytes(lengths, Hkv, D, S, W, int4_only=False, nvfp4=False):
-    """Algorithmic KV bytes one attention call reads: INT4 136 B (NVFP4 pages 144 B) and INT8 264 B per token and
-    KV head at D=128."""
+def kv_bytes(lengths, Hkv, D, S, W, int4_only=False, fmt=0):
+    """Algorithmic KV bytes one attention call reads: INT4 136 B (NVFP4 pages 144 B, INT2 pages 72 B) and INT8
+    264 B per token and KV head at D=128."""
     L = np.asarray(lengths, np.int64)
     prot = np.zeros_like(L) if int4_only else np.minimum(L, S + W)
-    page = 2 * (D // 2 + D // 16) if nvfp4 else 2 * (D // 2 + 4)
+    page = {0: 2 * (D // 2 + 4), 1: 2 * (D // 2 + D // 16), 2: 2 * (D // 4 + 4)}[fmt]
     return int(np.sum(Hkv * ((L - prot) * page + prot * 2 * (D + 4))))
 
 
@@ -611,19 +611,20 @@ def bf16_leg(torch, kv4, w, L, extra, used, layers_avail, per_layer_int4, K, dev
     return res
 
 
-def nvfp4_leg(torch, kv4, w, L, extra, used, layers_avail, per_layer_int4, K, device, flush):
-    """The NVFP4 page format (the alternative format of the "KV Cache Quantization" topic page, item 3) on the
-    same seeded tokens as the INT4 cache, at the same lengths, on as many of the first layers as fit (at most
-    BF16_MAX_LAYERS): decode attention in the protected mode, against the INT4 attention time of those layers."""
+def format_leg(torch, kv4, fmt, w, L, extra, used, layers_avail, per_layer_int4, K, device, flush):
+    """An alternative page format (NVFP4: the "KV Cache Quantization" topic page, item 3; INT2: its item 2) on
+    the same seeded tokens as the INT4 cache, at the same lengths, on as many of the first layers as fit (at
+    most BF16_MAX_LAYERS): decode attention in the protected mode, against the INT4 attention time of those
+    layers."""
     L_now = L - 1 + used
-    need_layer = kv_bytes(L_now, w["Hkv"], w["D"], w["S"], w["W"], nvfp4=True) * 1.08
+    need_layer = kv_bytes(L_now, w["Hkv"], w["D"], w["S"], w["W"], fmt=fmt) * 1.08
     free = torch.cuda.mem_get_info(device)[0]
     n = int(min(layers_avail, BF16_MAX_LAYERS, (free * 0.9 - 4e9) // need_layer))
     if n < 1:
-        return {"skipped": "an NVFP4 layer cache of %.1f GB does not fit (%.1f GB free)" % (need_layer / 1e9, free / 1e9)}
+        return {"skipped": "a layer cache of %.1f GB does not fit (%.1f GB free)" % (need_layer / 1e9, free / 1e9)}
     B = len(L_now)
     table, num_pages, mpps = workloads.block_table(w, L_now + 1, extra_tokens=0)
-    cfg = workloads.cache_config(w, num_pages, mpps, layers=n, page_format=kv4.KV4_FORMAT_NVFP4)
+    cfg = workloads.cache_config(w, num_pages, mpps, layers=n, page_format=fmt)
     cache = kv4.KV4Cache(cfg, torch.from_numpy(table), device)
     for layer in range(n):
         populate(torch, w, L, cache.append, layer, extra, device, upto=used)
@@ -635,7 +636,7 @@ def nvfp4_leg(torch, kv4, w, L, extra, used, layers_avail, per_layer_int4, K, de
                       lambda layer, i: qs[i % 3])
     status = cache.status()
     tf, t4 = sum(per), sum(per_layer_int4[:n])
-    bf = kv_bytes(L_now, w["Hkv"], w["D"], w["S"], w["W"], nvfp4=True) * n
+    bf = kv_bytes(L_now, w["Hkv"], w["D"], w["S"], w["W"], fmt=fmt) * n
     res = {"attention_ms": round(tf * 1e3, 4), "layers": n, "kv_gbs": round(bf / tf / 1e9, 1),
            "kv_bytes_vs_int4": round(bf / (kv_bytes(L_now, w["Hkv"], w["D"], w["S"], w["W"]) * n), 4),
            "int4_protected_attention_ms_same_layers": round(t4 * 1e3, 4), "time_vs_int4": round(tf / t4, 3),
@@ -690,7 +691,8 @@ def sub_line(torch, kv4, name, args, device, clocks, hbm, peak_kind):
         torch.cuda.empty_cache()
         b16 = bf16_leg(torch, kv4, w, L0, extra, used, 1, per, K, device, flush)
         line["compare"]["bf16_kv"] = b16
-        line["compare"]["nvfp4"] = nvfp4_leg(torch, kv4, w, L0, extra, used, 1, per, K, device, flush)
+        for key, fmt in (("nvfp4", kv4.KV4_FORMAT_NVFP4), ("int2", kv4.KV4_FORMAT_INT2)):
+            line["compare"][key] = format_leg(torch, kv4, fmt, w, L0, extra, used, 1, per, K, device, flush)
         if "speedup_int4_protected_vs_bf16" in b16:
             line["speedup_int4_protected_vs_bf16"] = b16["speedup_int4_protected_vs_bf16"]
     return line
@@ -796,7 +798,8 @@ def run_gpu(args):
         torch.cuda.empty_cache()
         if rank == 0 and cmp_ok:
             result["compare"]["bf16_kv"] = bf16_leg(torch, kv4, w, L0, extra, used, layers, per, K, device, flush)
-            result["compare"]["nvfp4"] = nvfp4_leg(torch, kv4, w, L0, extra, used, layers, per, K, device, flush)
+            for key, fmt in (("nvfp4", kv4.KV4_FORMAT_NVFP4), ("int2", kv4.KV4_FORMAT_INT2)):
+                result["compare"][key] = format_leg(torch, kv4, fmt, w, L0, extra, used, layers, per, K, device, flush)
         if (rank == 0 and world == 1 and not args.kernel_only and not args.no_sublines and not args.rope
                 and args.workload not in SUBLINES):
             subs = {}

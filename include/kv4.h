@@ -21,7 +21,10 @@
  * NVFP4 paged KV cache of SGLang, about 56 % of the FP8 bytes per token):
  * E2M1 codes in blocks of 16 dims sharing one E4M3 scale (per-tensor scale
  * 1), after the same rotation; the INT8 store of the protected positions and
- * every entry point are the same.
+ * every entry point are the same.  With KV4_FORMAT_INT2 they hold 2-bit codes
+ * of the same token-wise quantizer ("KV Cache Quantization" topic page, item
+ * 2: INT2 KV with the scale and offset folded into the other operand and the
+ * partial product, as the attention kernel does for INT4).
  *
  * Conventions
  * -----------
@@ -114,8 +117,9 @@ enum {
 /* Page formats (kv4_config.page_format). */
 enum {
   KV4_FORMAT_INT4 = 0,        /* token-wise asymmetric INT4, fp16 scale and zero point      */
-  KV4_FORMAT_NVFP4 = 1        /* E2M1 codes, one E4M3 scale per 16 dims (values beyond
+  KV4_FORMAT_NVFP4 = 1,       /* E2M1 codes, one E4M3 scale per 16 dims (values beyond
                                  +-2688 saturate)                                          */
+  KV4_FORMAT_INT2 = 2         /* token-wise asymmetric INT2, fp16 scale and zero point      */
 };
 
 /* kv4_dequantize_debug views. */
@@ -137,8 +141,8 @@ enum {
  *   hadamard_block      Bh, a power of two dividing D (1 = no rotation)
  *   sink_tokens         S >= 0
  *   recent_window       W >= 1, S + W <= 4096
- *   page_format         KV4_FORMAT_INT4 (0) or KV4_FORMAT_NVFP4 (1); the BF16
- *                       baseline cache needs 0
+ *   page_format         KV4_FORMAT_INT4 (0), KV4_FORMAT_NVFP4 (1) or
+ *                       KV4_FORMAT_INT2 (2); the BF16 baseline cache needs 0
  */
 typedef struct {
   int32_t num_layers, max_seqs, num_q_heads, num_kv_heads, head_dim;
@@ -167,8 +171,9 @@ int kv4_cache_create(const kv4_config* cfg, void* dev_buf, size_t bytes, int32_t
 int kv4_cache_destroy(kv4_cache* cache);
 
 /* Device addresses inside the cache buffer for layer `layer` (any pointer may
- * be NULL): the page pool, uint8 [num_pages][P/16][Hkv][16*D+128] (INT4) or
- * [num_pages][P/16][Hkv][18*D] (NVFP4); the
+ * be NULL): the page pool, uint8 [num_pages][P/16][Hkv][16*D+128] (INT4),
+ * [num_pages][P/16][Hkv][18*D] (NVFP4) or [num_pages][P/16][Hkv][8*D+128]
+ * (INT2); the
  * INT8 store, uint8 [max_seqs][ceil((S+W)/16)][Hkv][32*D+128]; and the
  * sequence lengths int32 [num_layers][max_seqs] (all layers).  KV heads are
  * innermost, so the 16-token tiles of all heads at one page position are

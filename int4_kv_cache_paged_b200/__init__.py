@@ -60,6 +60,7 @@ KV4_VIEW_INT4 = 1
 
 KV4_FORMAT_INT4 = 0
 KV4_FORMAT_NVFP4 = 1
+KV4_FORMAT_INT2 = 2
 
 EXPORTS = [
     "kv4_cache_required_bytes", "kv4_cache_create", "kv4_cache_destroy", "kv4_cache_layout", "kv4_seq_reset",

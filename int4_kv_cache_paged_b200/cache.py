@@ -29,6 +29,10 @@ def _tilef(D):
     return 18 * D
 
 
+def _tile2(D):
+    return 8 * D + 128
+
+
 class _Base:
     def _view(self, ptr, nbytes, shape):
         off = ptr - self.buf.data_ptr()
@@ -78,7 +82,7 @@ class KV4Cache(_Base):
     def pages(self, layer):
         c = self.cfg
         ptr, _, _ = kv4_cache_layout(self.handle, layer)
-        tile = _tilef(c["head_dim"]) if c.get("page_format", 0) == 1 else _tile4(c["head_dim"])
+        tile = {0: _tile4, 1: _tilef, 2: _tile2}[c.get("page_format", 0)](c["head_dim"])
         shape = (c["num_pages"], c["page_size"] // TILE, c["num_kv_heads"], tile)
         n = shape[0] * shape[1] * shape[2] * shape[3]
         return self._view(ptr, n, shape)

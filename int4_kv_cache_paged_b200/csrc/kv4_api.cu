@@ -26,7 +26,9 @@ int check_config(const kv4_config* c, bool bf16) {
   if (c->head_dim != 64 && c->head_dim != 128) return KV4_ERR_UNSUPPORTED;
   if (c->page_size < 16 || c->page_size % 16 || c->page_size > 1024) return KV4_ERR_UNSUPPORTED;
   if (static_cast<long long>(c->max_pages_per_seq) * c->page_size > (1LL << 30)) return KV4_ERR_UNSUPPORTED;
-  if (c->page_format != KV4_FORMAT_INT4 && (bf16 || c->page_format != KV4_FORMAT_NVFP4)) return KV4_ERR_INVALID_ARG;
+  if (c->page_format != KV4_FORMAT_INT4 &&
+      (bf16 || (c->page_format != KV4_FORMAT_NVFP4 && c->page_format != KV4_FORMAT_INT2)))
+    return KV4_ERR_INVALID_ARG;
   if (!bf16) {
     if (!is_pow2(c->hadamard_block) || c->head_dim % c->hadamard_block) return KV4_ERR_INVALID_ARG;
     if (c->sink_tokens < 0 || c->recent_window < 1) return KV4_ERR_INVALID_ARG;

@@ -245,6 +245,28 @@ __global__ void dequant_kernel(DequantParams p) {
       }
       return;
     }
+    if (p.fmt == KV4_FORMAT_INT2) {   // x^ = fma(code, s, z), 2-bit codes
+      const uint8_t* tile = p.pool + ((static_cast<long long>(page) * (p.P / 16) + (pos % p.P) / 16) * p.Hkv + h) *
+                                         tile2_bytes(D);
+      const uint32_t sz = *reinterpret_cast<const uint32_t*>(tile + 8 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3)));
+      const float s = half_lo(sz), z = half_hi(sz);
+      const int th = r >> 3, t = (r & 7) >> 1, e = r & 1;
+      for (int d = lane; d < D; d += 32) {
+        int byte, c;
+        if (tensor == 0) {
+          const int kq = d >> 6, cc = (d >> 4) & 3, tt = (d >> 2) & 3, j = d & 3;
+          byte = r * (D / 4) + tt * (D / 16) + 4 * kq + j;
+          c = cc;
+        } else {
+          const int m = d >> 4, mp = m >> 1, mb = m & 1, dh = (d >> 3) & 1, g = d & 7;
+          byte = 4 * D + (D / 8) * (4 * g + t) + 4 * mp + th + 2 * e;
+          c = dh + 2 * mb;
+        }
+        const int code = (tile[byte] >> (2 * c)) & 3;
+        out[d] = __fmaf_rn(static_cast<float>(code), s, z);
+      }
+      return;
+    }
     const uint8_t* tile = p.pool + ((static_cast<long long>(page) * (p.P / 16) + (pos % p.P) / 16) * p.Hkv + h) *
                                        tile4_bytes(D);
     const uint32_t sz = *reinterpret_cast<const uint32_t*>(tile + 16 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3)));

@@ -206,6 +206,34 @@ __device__ __forceinline__ void store_fp4(uint8_t* tile, int r, int tensor, cons
   }
 }
 
+// Write one token's INT2 codes (four a byte; every byte belongs to the token) and scales into its page
+// tile: K byte r D/4 + t D/16 + 4 kq + j holds dims 64 kq + 16 c + 4 t + j in bits 2c, 2c+1; V byte
+// 4D + (D/8)(4 g + t) + 4 mp + th + 2 e (token 8 th + 2 t + e) holds dims 16 (2 mp + mb) + 8 dh + g in
+// bits 2 (dh + 2 mb); the half2 (s, z) block at 8D as in the INT4 tile.
+__device__ __forceinline__ void store_int2(uint8_t* tile, int r, int tensor, const uint8_t* codes, uint32_t sz,
+                                           int D, int lane) {
+  for (int q = lane; q < D / 4; q += 32) {
+    uint32_t b = 0u;
+    int off;
+    if (tensor == 0) {
+      const int t = q / (D / 16), rem = q % (D / 16), kq = rem >> 2, j = rem & 3;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) b |= static_cast<uint32_t>(codes[64 * kq + 16 * c + 4 * t + j]) << (2 * c);
+      off = r * (D / 4) + q;
+    } else {
+      const int th = r >> 3, t = (r & 7) >> 1, e = r & 1, g = q & 7, mp = q >> 3;
+#pragma unroll
+      for (int mb = 0; mb < 2; ++mb)
+#pragma unroll
+        for (int dh = 0; dh < 2; ++dh)
+          b |= static_cast<uint32_t>(codes[16 * (2 * mp + mb) + 8 * dh + g]) << (2 * (dh + 2 * mb));
+      off = 4 * D + (D / 8) * (4 * g + t) + 4 * mp + th + 2 * e;
+    }
+    tile[off] = static_cast<uint8_t>(b);
+  }
+  if (lane == 0) *reinterpret_cast<uint32_t*>(tile + 8 * D + 16 * (r & 7) + 4 * (2 * tensor + (r >> 3))) = sz;
+}
+
 // Write one token's INT8 codes and scales into its protected tile.
 __device__ __forceinline__ void store_int8(uint8_t* tile, int r, int tensor, const uint8_t* codes, uint32_t sz,
                                            int D, int lane) {
@@ -294,13 +322,15 @@ __device__ __forceinline__ void encode_row(const AppendParams& p, const uint16_t
   for (int k = 1; k < VPL; ++k) { mn = fminf(mn, x[k]); mx = fmaxf(mx, x[k]); }
   mn = warp_min(mn);
   mx = warp_max(mx);
-  const bool fp4 = p.fmt == KV4_FORMAT_NVFP4;
-  const uint32_t sz4 = fp4 ? quantize_fp4<VPL>(x, c4, lane) : quantize_group<VPL>(x, mn, mx, 15.f, c4, lane);
+  const bool fp4 = p.fmt == KV4_FORMAT_NVFP4, int2 = p.fmt == KV4_FORMAT_INT2;
+  const uint32_t sz4 = fp4 ? quantize_fp4<VPL>(x, c4, lane)
+                           : quantize_group<VPL>(x, mn, mx, int2 ? 3.f : 15.f, c4, lane);
   const bool protect = pos < p.S || pos >= L_new - p.W;
   uint32_t sz8 = 0;
   if (protect) sz8 = quantize_group<VPL>(x, mn, mx, 255.f, c8, lane);
   __syncwarp();
   if (fp4) store_fp4<VPL>(p.pool + tile_idx * tilef_bytes(D), r, tensor, c4, sz4, D, lane);
+  else if (int2) store_int2(p.pool + tile_idx * tile2_bytes(D), r, tensor, c4, sz4, D, lane);
   else store_int4(p.pool + tile_idx * tile4_bytes(D), r, tensor, c4, sz4, D, lane);
   if (protect) {
     const int slot = pos < p.S ? pos : p.S + (pos - p.S) % p.W;

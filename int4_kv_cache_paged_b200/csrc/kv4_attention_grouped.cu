@@ -67,7 +67,7 @@ struct GShape {
   static constexpr int S8 = GWR / H8;
 };
 
-// F: page format (0 INT4, 1 NVFP4)
+// F: page format (0 INT4, 1 NVFP4, 2 INT2)
 template <int D, int GWR, int F = 0>
 struct GCfg {
   static constexpr int STAGE4 = GWR * page_tile_bytes(D, F);          // one tile position of the group's heads
@@ -601,7 +601,7 @@ __device__ void produce(const AttnParams& p, GMisc* misc, SegQ* segq, uint8_t* r
 // PAIR = INT4 tiles per iteration of a consumer warp (1, 2 or 4).  MULTI:
 // several query tokens per sequence (causal visibility per operand column);
 // the one-token variant carries none of that code.  GWR: KV heads per group.
-// F: page format (0 INT4, 1 NVFP4; the INT8 store is the same).
+// F: page format (0 INT4, 1 NVFP4, 2 INT2; the INT8 store is the same).
 template <int D, int PAIR, bool MULTI, int GWR, int F = 0>
 __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
   using C = GCfg<D, GWR, F>;
@@ -724,8 +724,9 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
             if (nt == PAIR) unit_fp4<D, PAIR, false>(tl, qf, ws, lane, valid, valid, eb, cs);
             else unit_fp4<D, 1, false>(tl, qf, ws, lane, valid, valid, eb, cs);
           } else {
-            if (nt == PAIR) unit_int4<D, PAIR, false>(tl, qf, ws, lane, valid, eb, cs);
-            else unit_int4<D, 1, false>(tl, qf, ws, lane, valid, eb, cs);
+            constexpr int BITS = F == 2 ? 2 : 4;
+            if (nt == PAIR) unit_int4<D, PAIR, false, false, BITS>(tl, qf, ws, lane, valid, eb, cs);
+            else unit_int4<D, 1, false, false, BITS>(tl, qf, ws, lane, valid, eb, cs);
           }
         } else {
 #pragma unroll
@@ -745,8 +746,9 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
             if (nt == PAIR) unit_fp4<D, PAIR, true, MULTI>(tl, qf, ws, lane, valid, nwr, eb, cs);
             else unit_fp4<D, 1, true, MULTI>(tl, qf, ws, lane, valid, nwr, eb, cs);
           } else {
-            if (nt == PAIR) unit_int4<D, PAIR, true, MULTI>(tl, qf, ws, lane, valid, eb, cs);
-            else unit_int4<D, 1, true, MULTI>(tl, qf, ws, lane, valid, eb, cs);
+            constexpr int BITS = F == 2 ? 2 : 4;
+            if (nt == PAIR) unit_int4<D, PAIR, true, MULTI, BITS>(tl, qf, ws, lane, valid, eb, cs);
+            else unit_int4<D, 1, true, MULTI, BITS>(tl, qf, ws, lane, valid, eb, cs);
           }
         }
         u += nt;
@@ -988,11 +990,6 @@ __device__ __forceinline__ bool wg_and(int h, bool pred) {
   return r != 0;
 }
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 6, 512;" ::: "memory"); }
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
 __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
@@ -1505,8 +1502,8 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   p.partials = reinterpret_cast<float*>(wsb + l.partials);
   GPlanRec* plan = reinterpret_cast<GPlanRec*>(wsb + l.plan);
   // one query token, 4-head groups, D = 128, INT4 pages: the tensor-memory kernel when selected, one CTA per SM
-  const bool fp4 = c->cfg.page_format == KV4_FORMAT_NVFP4;
-  const bool tcpath = D == 128 && GWR == 4 && c->use_tc && p.qtot == 1 && !fp4;
+  const bool fp4 = c->cfg.page_format == KV4_FORMAT_NVFP4, int2 = c->cfg.page_format == KV4_FORMAT_INT2;
+  const bool tcpath = D == 128 && GWR == 4 && c->use_tc && p.qtot == 1 && c->cfg.page_format == KV4_FORMAT_INT4;
   p.qfmt = tcpath ? 1 : (fp4 ? 2 : 0);
   p.grid = tcpath ? c->num_sms : g_grid(c);
   p.cap_parts = p.grid * 2 * GWR;
@@ -1528,7 +1525,8 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   cfg.gridDim = dim3(p.grid);
   cfg.blockDim = dim3(tcpath ? TC_THREADS : GShape<GWR>::THREADS);
   cfg.dynamicSmemBytes = tcpath ? tattn_smem_bytes<D>(p.ns)
-                                : (fp4 ? gattn_smem_bytes<D, GWR, 1>(p.ns) : gattn_smem_bytes<D, GWR>(p.ns));
+                                : (fp4 ? gattn_smem_bytes<D, GWR, 1>(p.ns)
+                                       : (int2 ? gattn_smem_bytes<D, GWR, 2>(p.ns) : gattn_smem_bytes<D, GWR>(p.ns)));
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1540,6 +1538,9 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   if (fp4) {
     e = p.qtot > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true, GWR, 1>, p, plan)
                    : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false, GWR, 1>, p, plan);
+  } else if (int2) {
+    e = p.qtot > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true, GWR, 2>, p, plan)
+                   : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false, GWR, 2>, p, plan);
   } else if constexpr (D == 128 && GWR == 4) {
     if (tcpath) e = cudaLaunchKernelEx(&cfg, tattn_kernel<D>, p, plan);
     else if (p.qtot > 1) e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true, GWR>, p, plan);
@@ -1619,6 +1620,8 @@ int grouped_ring(kv4_cache* c) {
   const int Hkv = c->cfg.num_kv_heads;
   if (c->cfg.page_format == KV4_FORMAT_NVFP4)
     return c->cfg.head_dim == 128 ? g_choose_ring_gw<128, 1>(c->device, Hkv) : g_choose_ring_gw<64, 1>(c->device, Hkv);
+  if (c->cfg.page_format == KV4_FORMAT_INT2)
+    return c->cfg.head_dim == 128 ? g_choose_ring_gw<128, 2>(c->device, Hkv) : g_choose_ring_gw<64, 2>(c->device, Hkv);
   return c->cfg.head_dim == 128 ? g_choose_ring_gw<128, 0>(c->device, Hkv) : g_choose_ring_gw<64, 0>(c->device, Hkv);
 }
 

@@ -111,23 +111,62 @@ __device__ __forceinline__ void pv_operands(float P0, float P1, float P2, float 
   }
 }
 
-// P.V of one INT4 tile: o^T[m] += V^T codes * (hi + lo) weights.
-template <int D>
+// The V code words a lane reads from a page tile: BITS = 4 (INT4 pages), D/16 words at 8D + 16 lane
+// (+512), one per 16-dim block; BITS = 2 (INT2 pages), D/32 words at 4D + (D/8) lane, one per pair of
+// blocks.
+template <int D, int BITS>
+__device__ __forceinline__ void load_v_words(uint32_t st, int lane, uint32_t (&vw)[D / 16]) {
+  if constexpr (BITS == 4) {
+    if constexpr (D == 128) {
+      const uint4 v0 = lds128(st + 8 * D + lane * 16), v1 = lds128(st + 8 * D + 512 + lane * 16);
+      vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+      vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
+    } else {
+      const uint4 v0 = lds128(st + 8 * D + lane * 16);
+      vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+    }
+  } else {
+    if constexpr (D == 128) {
+      const uint4 v0 = lds128(st + 4 * D + lane * 16);
+      vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+    } else {
+      const uint2 v0 = lds64(st + 4 * D + lane * 8);
+      vw[0] = v0.x; vw[1] = v0.y;
+    }
+  }
+}
+
+// Crumbs at bits 0-1 and 16-17 as an fp16 pair, minus 2 (exact).
+__device__ __forceinline__ uint32_t crumb_c(uint32_t w) {
+  uint32_t x = lop3_and_or(w, 0x00030003u, 0x64006400u);
+  __half2 h = __hsub2(*reinterpret_cast<__half2*>(&x), __half2(__half(1026.f), __half(1026.f)));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// The four centred A registers of the P.V multiply of dim block m: (dim g | g+8) x (tokens 2t, 2t+1 |
+// 2t+8, 2t+9), codes minus 8 (INT4) or minus 2 (INT2).
+template <int BITS>
+__device__ __forceinline__ void v_operands(const uint32_t* vw, int m, uint32_t& a0, uint32_t& a1, uint32_t& a2,
+                                           uint32_t& a3) {
+  if constexpr (BITS == 4) {
+    const uint32_t w = vw[m], u = w >> 8;
+    a0 = nib_lo_c(w); a1 = nib_hi_c(w); a2 = nib_lo_c(u); a3 = nib_hi_c(u);
+  } else {
+    const uint32_t w = vw[m >> 1] >> (4 * (m & 1));
+    a0 = crumb_c(w); a1 = crumb_c(w >> 2); a2 = crumb_c(w >> 8); a3 = crumb_c(w >> 10);
+  }
+}
+
+// P.V of one INT4 (or INT2) tile: o^T[m] += V^T codes * (hi + lo) weights.
+template <int D, int BITS = 4>
 __device__ __forceinline__ void pv_int4(uint32_t st, WarpState<D>& ws, int lane, uint32_t B0, uint32_t B1,
                                         uint32_t C0, uint32_t C1, bool colsplit) {
   uint32_t vw[D / 16];
-  if constexpr (D == 128) {
-    const uint4 v0 = lds128(st + 8 * D + lane * 16), v1 = lds128(st + 8 * D + 512 + lane * 16);
-    vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
-    vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
-  } else {
-    const uint4 v0 = lds128(st + 8 * D + lane * 16);
-    vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
-  }
+  load_v_words<D, BITS>(st, lane, vw);
 #pragma unroll
   for (int m = 0; m < D / 16; ++m) {
-    const uint32_t w = vw[m], u = w >> 8;
-    const uint32_t a0 = nib_lo_c(w), a1 = nib_hi_c(w), a2 = nib_lo_c(u), a3 = nib_hi_c(u);
+    uint32_t a0, a1, a2, a3;
+    v_operands<BITS>(vw, m, a0, a1, a2, a3);
     mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
     if (!colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
   }
@@ -141,28 +180,35 @@ __device__ __forceinline__ void pv_int4(uint32_t st, WarpState<D>& ws, int lane,
 // (bits 0 and 2 decide) and every column sees a token of the unit; with it a
 // column may see none, and its state stays at m = -inf, l = 0.
 // The stages are handed back (empty barriers eb[0 .. NT-1], each distinct one
-// once) after the last shared-memory load.
-template <int D, int NT, bool MASKED, bool CAUSAL = false>
+// once) after the last shared-memory load.  BITS = 2: INT2 pages (the same
+// folded form with 2-bit codes: four a byte, the half2 scales at 8D).
+template <int D, int NT, bool MASKED, bool CAUSAL = false, int BITS = 4>
 __device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& qf, WarpState<D>& ws, int lane,
                                           const int* valid, const uint32_t* eb, const ColSplit& cs) {
+  static_assert(BITS == 4 || BITS == 2, "code width");
+  constexpr int SZOFF = BITS == 4 ? 16 * D : 8 * D;          // the half2 (s, z) block of the tile
+  constexpr float VCENTRE = BITS == 4 ? 8.f : 2.f;          // P.V takes the codes minus this
   float x[NT][4];
   uint4 sz[NT];
   // Q.K^T of the NT tiles on the integer tensor cores: each tile's K codes are
   // unpacked to bytes with one mask per plane and multiplied by both query
   // planes (2*NT independent accumulator chains of D/32 multiplies).
   constexpr int NKK = D / 32;
-  uint32_t kw[NT][2][NKK];
+  uint32_t kw[NT][2][NKK];   // INT2: the first NKK / 2 words of each row
 #pragma unroll
   for (int u = 0; u < NT; ++u) {
-    if constexpr (D == 128) {
+    if constexpr (BITS == 4 && D == 128) {
       const uint4 a = lds128(tile[u] + lane * 16), bq = lds128(tile[u] + 512 + lane * 16);
       kw[u][0][0] = a.x; kw[u][0][1] = a.y; kw[u][0][2] = a.z; kw[u][0][3] = a.w;
       kw[u][1][0] = bq.x; kw[u][1][1] = bq.y; kw[u][1][2] = bq.z; kw[u][1][3] = bq.w;
-    } else {
-      const uint2 a = lds64(tile[u] + lane * 8), bq = lds64(tile[u] + 256 + lane * 8);
+    } else if constexpr (BITS == 4 || D == 128) {   // INT4 at D = 64, INT2 at D = 128: 8 bytes per row
+      const uint2 a = lds64(tile[u] + lane * 8), bq = lds64(tile[u] + 256 + lane * 8);   // rows g + 8
       kw[u][0][0] = a.x; kw[u][0][1] = a.y; kw[u][1][0] = bq.x; kw[u][1][1] = bq.y;
+    } else {                                        // INT2 at D = 64: one word per row
+      kw[u][0][0] = lds32(tile[u] + lane * 4);
+      kw[u][1][0] = lds32(tile[u] + 128 + lane * 4);
     }
-    sz[u] = lds128(tile[u] + 16 * D + (lane >> 2) * 16);
+    sz[u] = lds128(tile[u] + SZOFF + (lane >> 2) * 16);
   }
   int ahi[NT][4], alo[NT][4];
 #pragma unroll
@@ -173,9 +219,16 @@ __device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& 
   for (int kk = 0; kk < NKK; ++kk) {
 #pragma unroll
     for (int u = 0; u < NT; ++u) {
-      const uint32_t w0 = kw[u][0][kk], w1 = kw[u][1][kk];
-      qk_block<D>(ahi[u], alo[u], w0 & 0x0F0F0F0Fu, w1 & 0x0F0F0F0Fu, (w0 >> 4) & 0x0F0F0F0Fu,
-                  (w1 >> 4) & 0x0F0F0F0Fu, qf, kk);
+      if constexpr (BITS == 4) {
+        const uint32_t w0 = kw[u][0][kk], w1 = kw[u][1][kk];
+        qk_block<D>(ahi[u], alo[u], w0 & 0x0F0F0F0Fu, w1 & 0x0F0F0F0Fu, (w0 >> 4) & 0x0F0F0F0Fu,
+                    (w1 >> 4) & 0x0F0F0F0Fu, qf, kk);
+      } else {   // crumbs 2(kk % 2) and 2(kk % 2) + 1 of word kk / 2: the two 16-dim halves of block kk
+        const int sh = 4 * (kk & 1);
+        const uint32_t w0 = kw[u][0][kk >> 1] >> sh, w1 = kw[u][1][kk >> 1] >> sh;
+        qk_block<D>(ahi[u], alo[u], w0 & 0x03030303u, w1 & 0x03030303u, (w0 >> 2) & 0x03030303u,
+                    (w1 >> 2) & 0x03030303u, qf, kk);
+      }
     }
   }
 #pragma unroll
@@ -231,7 +284,7 @@ __device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& 
     const float p0 = ex2(x[u][0] - mu0), p1 = ex2(x[u][1] - mu1);
     const float p2 = ex2(x[u][2] - mu0), p3 = ex2(x[u][3] - mu1);
     const float sVg = half_lo(sz[u].z), sVg8 = half_lo(sz[u].w);
-    const float zVg = fmaf(8.f, sVg, half_hi(sz[u].z)), zVg8 = fmaf(8.f, sVg8, half_hi(sz[u].w));   // centred codes
+    const float zVg = fmaf(VCENTRE, sVg, half_hi(sz[u].z)), zVg8 = fmaf(VCENTRE, sVg8, half_hi(sz[u].w));   // centred
     float P0 = p0 * sVg, P1 = p1 * sVg, P2 = p2 * sVg8, P3 = p3 * sVg8;
     float zg0 = p0 * zVg, zg1 = p1 * zVg, zg80 = p2 * zVg8, zg81 = p3 * zVg8;
     if constexpr (MASKED && CAUSAL) {   // unwritten slots may hold non-finite scales
@@ -251,14 +304,7 @@ __device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& 
       // last tile: load its V codes, then hand the stage(s) back before the math
       const uint32_t t = tile[u];
       uint32_t vw[D / 16];
-      if constexpr (D == 128) {
-        const uint4 v0 = lds128(t + 8 * D + lane * 16), v1 = lds128(t + 8 * D + 512 + lane * 16);
-        vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
-        vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
-      } else {
-        const uint4 v0 = lds128(t + 8 * D + lane * 16);
-        vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
-      }
+      load_v_words<D, BITS>(t, lane, vw);
       __syncwarp();
       if (lane == 0) {
 #pragma unroll
@@ -267,13 +313,13 @@ __device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& 
       }
 #pragma unroll
       for (int m = 0; m < D / 16; ++m) {
-        const uint32_t w = vw[m], uu = w >> 8;
-        const uint32_t a0 = nib_lo_c(w), a1 = nib_hi_c(w), a2 = nib_lo_c(uu), a3 = nib_hi_c(uu);
+        uint32_t a0, a1, a2, a3;
+        v_operands<BITS>(vw, m, a0, a1, a2, a3);
         mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
         if (!cs.colsplit) mma_f16(ws.o[m], a0, a1, a2, a3, C0, C1);
       }
     } else {
-      pv_int4<D>(tile[u], ws, lane, B0, B1, C0, C1, cs.colsplit);
+      pv_int4<D, BITS>(tile[u], ws, lane, B0, B1, C0, C1, cs.colsplit);
     }
   }
 }

@@ -41,7 +41,11 @@ __host__ __device__ constexpr int tile8_bytes(int D) { return 32 * D + 128; }
 __host__ __device__ constexpr int tile16_bytes(int D) { return 64 * D; }
 // NVFP4 page tile: K codes 8*D, V codes 8*D, K scales D, V scales D (one E4M3 byte per token and 16 dims)
 __host__ __device__ constexpr int tilef_bytes(int D) { return 18 * D; }
-__host__ __device__ constexpr int page_tile_bytes(int D, int fmt) { return fmt == 1 ? tilef_bytes(D) : tile4_bytes(D); }
+// INT2 page tile: K codes 4*D, V codes 4*D, the half2 (s, z) block of 128 bytes
+__host__ __device__ constexpr int tile2_bytes(int D) { return 8 * D + 128; }
+__host__ __device__ constexpr int page_tile_bytes(int D, int fmt) {
+  return fmt == 1 ? tilef_bytes(D) : (fmt == 2 ? tile2_bytes(D) : tile4_bytes(D));
+}
 __host__ __device__ constexpr int qblob_bytes(int D) { return 16 * D + 64; }
 __host__ __device__ inline int n_prot_tiles(int S, int W) { return (S + W + TILE - 1) / TILE; }
 
@@ -258,6 +262,12 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
   if (!KV4_SMEM_OK(addr, 8, 8, 9)) return make_uint2(0, 0);
   asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  if (!KV4_SMEM_OK(addr, 4, 4, 14)) return 0u;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
 

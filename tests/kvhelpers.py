@@ -129,6 +129,35 @@ def compare_fp4_pages(pair, layer, seqs):
     return bad
 
 
+def compare_int2_pages(pair, layer, seqs):
+    """Bit-exact comparison of every INT2 byte owned by a written position of `seqs` (K and V code bytes,
+    its half2 scale entries)."""
+    c = pair.cfg
+    D, P = c["head_dim"], c["page_size"]
+    t2 = tables("int2", D)
+    pages = pair.gpu.pages(layer).cpu().numpy()
+    ar4 = np.arange(4)
+    bad = []
+    for seq in seqs:
+        L = int(pair.orc.seq_lens[layer, seq])
+        for p in range(L):
+            page = int(pair.table[seq, p // P])
+            ti, r = (p % P) // TILE, p % TILE
+            idx = np.concatenate([t2.k_byte[r], 4 * D + t2.v_byte[r], 8 * D + scale_offset(r, 0) + ar4,
+                                  8 * D + scale_offset(r, 1) + ar4])
+            g = pages[page, ti][:, idx]
+            o = pair.orc.pages[(layer, page)][ti][:, idx]
+            if not np.array_equal(g, o):
+                bad.append((seq, p, int(np.sum(g != o))))
+    return bad
+
+
+def compare_page_copy(pair, layer, seqs):
+    """The page comparison of the cache's page format."""
+    fmt = pair.cfg.get("page_format", 0)
+    return {0: compare_int4_pages, 1: compare_fp4_pages, 2: compare_int2_pages}[fmt](pair, layer, seqs)
+
+
 def compare_int8_store(pair, layer, seqs):
     """Bit-exact comparison of the protected slots [0, min(L, S+W)) of `seqs`."""
     c = pair.cfg

@@ -56,13 +56,16 @@ def test_host_side_validation_without_a_device():
                       (dict(page_size=24), kv4.KV4_ERR_UNSUPPORTED), (dict(hadamard_block=3), kv4.KV4_ERR_INVALID_ARG),
                       (dict(hadamard_block=256), kv4.KV4_ERR_INVALID_ARG), (dict(recent_window=0), kv4.KV4_ERR_INVALID_ARG),
                       (dict(sink_tokens=-1), kv4.KV4_ERR_INVALID_ARG), (dict(num_pages=0), kv4.KV4_ERR_INVALID_ARG),
-                      (dict(page_format=2), kv4.KV4_ERR_INVALID_ARG), (dict(page_format=-1), kv4.KV4_ERR_INVALID_ARG)):
+                      (dict(page_format=3), kv4.KV4_ERR_INVALID_ARG), (dict(page_format=-1), kv4.KV4_ERR_INVALID_ARG)):
         with pytest.raises(kv4.KV4Error) as e:
             kv4.kv4_cache_required_bytes(kv4.make_config(**dict(good, **bad)))
         assert e.value.code == code, bad
     # NVFP4 pages: 18*D bytes per 16-token tile (the INT8 store is the same)
     nf = kv4.kv4_cache_required_bytes(kv4.make_config(**dict(good, page_format=kv4.KV4_FORMAT_NVFP4)))
     assert nf == 256 + 256 + ((10 * 2 * 2304 + 255) // 256) * 256 + prot
+    # INT2 pages: 8*D + 128 bytes per tile
+    n2 = kv4.kv4_cache_required_bytes(kv4.make_config(**dict(good, page_format=kv4.KV4_FORMAT_INT2)))
+    assert n2 == 256 + 256 + ((10 * 2 * 1152 + 255) // 256) * 256 + prot
     # BF16 cache ignores the quantization fields, but has one page format
     kv4.kv4bf16_cache_required_bytes(kv4.make_config(**dict(good, hadamard_block=3, recent_window=0)))
     with pytest.raises(kv4.KV4Error) as e:

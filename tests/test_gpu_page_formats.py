@@ -1,23 +1,29 @@
-"""GPU parity of the NVFP4 page format (kv4_config.page_format = KV4_FORMAT_NVFP4): the
-CUDA path against the oracle on identical seeded inputs.
+"""GPU parity of the alternative page formats (kv4_config.page_format): the CUDA
+path against the oracle on identical seeded inputs.
 
-Source of the format: "KV Cache Quantization" topic page, item 3 (SGLang's NVFP4
-paged KV cache); the block quantizer's readings are the library's (E2M1 codes,
-one E4M3 scale per 16 dims, per-tensor scale 1).  Codes and scales must match
-bit for bit -- including each token's nibble of the V bytes it shares with its
-neighbour, written by different warps or different calls; the INT8 store of
-the protected positions is the INT4 cache's; attention, the multi-token query,
-the fused step and the debug view within the tolerances of the INT4 format."""
+* KV4_FORMAT_NVFP4 -- "KV Cache Quantization" topic page, item 3 (SGLang's NVFP4
+  paged KV cache); the block quantizer's readings are the library's (E2M1
+  codes, one E4M3 scale per 16 dims, per-tensor scale 1).
+* KV4_FORMAT_INT2 -- the same page, item 2 (INT2 KV with folded scale and
+  offset): the method's token-wise quantizer with 2-bit codes.
+
+Codes and scales must match bit for bit -- for NVFP4 including each token's
+nibble of the V bytes it shares with its neighbour, written by different warps
+or different calls; the INT8 store of the protected positions is the INT4
+cache's; attention, the multi-token query, the fused step and the debug view
+within the tolerances of the INT4 format."""
 
 import numpy as np
 import pytest
 import torch
 
-from kvhelpers import (Pair, cfg_dict, random_table, bf16_values, f32, compare_fp4_pages, compare_int8_store,
+from kvhelpers import (Pair, cfg_dict, random_table, bf16_values, f32, compare_page_copy, compare_int8_store,
                        check_bf16_out, check_f32_out, REL_L2, MAX_ABS)
 from oracle import extend_attention
 
 pytestmark = pytest.mark.gpu
+
+FORMATS = [1, 2]   # KV4_FORMAT_NVFP4, KV4_FORMAT_INT2
 
 
 @pytest.fixture(scope="module")
@@ -69,18 +75,18 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("fmt", FORMATS)
 @pytest.mark.parametrize("D,Hq,Hkv,P,Bh,S,W,lens", CASES)
-def test_codes_scales_and_attention(kv4, D, Hq, Hkv, P, Bh, S, W, lens):
+def test_codes_scales_and_attention(kv4, fmt, D, Hq, Hkv, P, Bh, S, W, lens):
     rng = np.random.default_rng(sum(lens) + D + Hkv)
     n = len(lens)
     mpps = max(lens) // P + 2
-    cfg = cfg_dict(D=D, Hq=Hq, Hkv=Hkv, P=P, Bh=Bh, S=S, W=W, num_pages=n * mpps, mpps=mpps, max_seqs=n,
-                   fmt=kv4.KV4_FORMAT_NVFP4)
+    cfg = cfg_dict(D=D, Hq=Hq, Hkv=Hkv, P=P, Bh=Bh, S=S, W=W, num_pages=n * mpps, mpps=mpps, max_seqs=n, fmt=fmt)
     pair = Pair(cfg, random_table(n, mpps, n * mpps, rng))
     seqs = list(range(n))
     _populate(pair, rng, seqs, lens, Hkv, D)
     np.testing.assert_array_equal(pair.gpu.seq_lens()[0, :n].cpu().numpy(), lens)
-    assert compare_fp4_pages(pair, 0, seqs) == []
+    assert compare_page_copy(pair, 0, seqs) == []
     assert compare_int8_store(pair, 0, seqs) == []
     q = bf16_values((n, Hq, D), rng)
     order = seqs[::-1]
@@ -88,12 +94,13 @@ def test_codes_scales_and_attention(kv4, D, Hq, Hkv, P, Bh, S, W, lens):
     _check(kv4, pair, order, q[order], protected=False)
 
 
-def test_debug_view_is_the_oracle_view(kv4):
+@pytest.mark.parametrize("fmt", FORMATS)
+@pytest.mark.parametrize("D", [64, 128])
+def test_debug_view_is_the_oracle_view(kv4, fmt, D):
     rng = np.random.default_rng(11)
-    D, Hkv, n = 128, 4, 2
+    Hkv, n = 4, 2
     lens = [300, 40]
-    cfg = cfg_dict(D=D, Hq=16, Hkv=Hkv, P=32, Bh=128, S=4, W=32, num_pages=24, mpps=12, max_seqs=n,
-                   fmt=kv4.KV4_FORMAT_NVFP4)
+    cfg = cfg_dict(D=D, Hq=16, Hkv=Hkv, P=32, Bh=D, S=4, W=32, num_pages=24, mpps=12, max_seqs=n, fmt=fmt)
     pair = Pair(cfg, random_table(n, 12, 24, rng))
     _populate(pair, rng, [0, 1], lens, Hkv, D)
     for s, L in enumerate(lens):
@@ -104,16 +111,16 @@ def test_debug_view_is_the_oracle_view(kv4):
             np.testing.assert_array_equal(v.cpu().numpy(), vo)
 
 
-def test_decode_steps_fused_and_two_calls(kv4):
-    """kv4_decode_step on NVFP4 pages equals append + attention bit for bit over 12 steps (the tokens of
-    a shared V byte arrive in consecutive steps), and matches the oracle."""
+@pytest.mark.parametrize("fmt", FORMATS)
+def test_decode_steps_fused_and_two_calls(kv4, fmt):
+    """kv4_decode_step on these pages equals append + attention bit for bit over 12 steps (for NVFP4 the
+    tokens of a shared V byte arrive in consecutive steps), and matches the oracle."""
     rng = np.random.default_rng(12)
     D, Hq, Hkv = 128, 32, 8
     lens = [500, 33, 1000, 0]
     n = len(lens)
     mpps = (max(lens) + 20) // 16 + 2
-    cfg = cfg_dict(D=D, Hq=Hq, Hkv=Hkv, P=16, Bh=128, S=4, W=32, num_pages=n * mpps, mpps=mpps, max_seqs=n,
-                   fmt=kv4.KV4_FORMAT_NVFP4)
+    cfg = cfg_dict(D=D, Hq=Hq, Hkv=Hkv, P=16, Bh=128, S=4, W=32, num_pages=n * mpps, mpps=mpps, max_seqs=n, fmt=fmt)
     table = random_table(n, mpps, n * mpps, rng)
     a, b = Pair(cfg, table), Pair(cfg, table)
     k = bf16_values((sum(lens), Hkv, D), rng, 2.0)
@@ -130,7 +137,7 @@ def test_decode_steps_fused_and_two_calls(kv4):
         torch.cuda.synchronize()
         assert torch.equal(out_a, out_b), step
         a.orc.append(0, [2, 0, 3, 1], np.arange(n + 1), f32(kn), f32(vn))
-    assert compare_fp4_pages(a, 0, list(range(n))) == []
+    assert compare_page_copy(a, 0, list(range(n))) == []
     torch.cuda.synchronize()
     assert torch.equal(a.gpu.pages(0), b.gpu.pages(0))
     rel, excess = check_bf16_out(out_b, a.oracle_attention(0, [2, 0, 3, 1], q))
@@ -138,15 +145,15 @@ def test_decode_steps_fused_and_two_calls(kv4):
     assert a.gpu.status() == 0 and b.gpu.status() == 0
 
 
+@pytest.mark.parametrize("fmt", FORMATS)
 @pytest.mark.parametrize("Hq,Hkv,T", [(32, 8, 2), (16, 8, 4), (32, 8, 5)])
-def test_multi_token_queries(kv4, Hq, Hkv, T):
+def test_multi_token_queries(kv4, fmt, Hq, Hkv, T):
     rng = np.random.default_rng(13 + T)
     D = 128
     lens = [700, 3, 0, 140]
     n = len(lens)
     mpps = max(lens) // 16 + 2
-    cfg = cfg_dict(D=D, Hq=Hq, Hkv=Hkv, P=16, Bh=128, S=4, W=64, num_pages=n * mpps, mpps=mpps, max_seqs=n,
-                   fmt=kv4.KV4_FORMAT_NVFP4)
+    cfg = cfg_dict(D=D, Hq=Hq, Hkv=Hkv, P=16, Bh=128, S=4, W=64, num_pages=n * mpps, mpps=mpps, max_seqs=n, fmt=fmt)
     pair = Pair(cfg, random_table(n, mpps, n * mpps, rng))
     _populate(pair, rng, list(range(n)), lens, Hkv, D)
     q = bf16_values((n, T, Hq, D), rng)
@@ -165,13 +172,13 @@ def test_multi_token_queries(kv4, Hq, Hkv, T):
         assert rel32 <= REL_L2 and mx32 <= MAX_ABS, (rel32, mx32)
 
 
-def test_one_long_sequence_over_every_cta(kv4):
+@pytest.mark.parametrize("fmt", FORMATS)
+def test_one_long_sequence_over_every_cta(kv4, fmt):
     rng = np.random.default_rng(14)
     D, Hq, Hkv = 128, 32, 8
     L = 40000
     mpps = L // 16 + 2
-    cfg = cfg_dict(D=D, Hq=Hq, Hkv=Hkv, P=16, Bh=128, S=4, W=128, num_pages=mpps, mpps=mpps, max_seqs=1,
-                   fmt=kv4.KV4_FORMAT_NVFP4)
+    cfg = cfg_dict(D=D, Hq=Hq, Hkv=Hkv, P=16, Bh=128, S=4, W=128, num_pages=mpps, mpps=mpps, max_seqs=1, fmt=fmt)
     pair = Pair(cfg, random_table(1, mpps, mpps, rng))
     _populate(pair, rng, [0], [L], Hkv, D, chunk=4096, fill=False)
     q = bf16_values((1, Hq, D), rng)
