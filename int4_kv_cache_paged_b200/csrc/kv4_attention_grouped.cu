@@ -217,16 +217,21 @@ __device__ void zero_group(const AttnParams& p, int i, int e0, int step) {
 
 // Normalise, rotate back and store the output of one KV head: lane (g8, t)
 // holds o for heads 2t, 2t+1 (valid when < G) at dimensions 16m+g8 (o[m][0],
-// o[m][1]) and 16m+g8+8 (o[m][2], o[m][3]).  out = c_B * H_blk (o / l): the
-// normalised block Hadamard is its own inverse.
-template <int D, bool MULTI>
+// o[m][1]) and 16m+g8+8 (o[m][2], o[m][3]); with paired columns (PC) it holds
+// head t alone, in o[m][0] and o[m][2], and l1 is unused.  out = c_B * H_blk
+// (o / l): the normalised block Hadamard is its own inverse.
+template <int D, bool MULTI, bool PC = false>
 __device__ __forceinline__ void store_head(const AttnParams& p, int b, int hkv, int lane, float (&o)[D / 16][4],
                                            float l0, float l1) {
   constexpr int NM = D / 16;
+  constexpr int IS = PC ? 2 : 1;   // step over the lane's o[m][i] that hold values
   const int g8 = lane >> 2, t = lane & 3;
   const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
 #pragma unroll
-  for (int m = 0; m < NM; ++m) { o[m][0] *= inv0; o[m][2] *= inv0; o[m][1] *= inv1; o[m][3] *= inv1; }
+  for (int m = 0; m < NM; ++m) {
+    o[m][0] *= inv0; o[m][2] *= inv0;
+    if constexpr (!PC) { o[m][1] *= inv1; o[m][3] *= inv1; }
+  }
   const int Bh = p.Bh_o;
   // stages 1, 2, 4: dimension bits 0-2 are the lane bits 2-4
 #pragma unroll
@@ -236,7 +241,7 @@ __device__ __forceinline__ void store_head(const AttnParams& p, int b, int hkv, 
 #pragma unroll
       for (int m = 0; m < NM; ++m)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 4; i += IS) {
           const float other = __shfl_xor_sync(0xffffffffu, o[m][i], 4 * hh);
           o[m][i] = upper ? other - o[m][i] : o[m][i] + other;
         }
@@ -247,7 +252,7 @@ __device__ __forceinline__ void store_head(const AttnParams& p, int b, int hkv, 
 #pragma unroll
     for (int m = 0; m < NM; ++m)
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < 2; i += IS) {
         const float a = o[m][i], c = o[m][i + 2];
         o[m][i] = a + c;
         o[m][i + 2] = a - c;
@@ -261,7 +266,7 @@ __device__ __forceinline__ void store_head(const AttnParams& p, int b, int hkv, 
       for (int m = 0; m < NM; ++m)
         if ((m & mb) == 0)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < 4; i += IS) {
             const float a = o[m][i], c = o[m + mb][i];
             o[m][i] = a + c;
             o[m + mb][i] = a - c;
@@ -271,8 +276,8 @@ __device__ __forceinline__ void store_head(const AttnParams& p, int b, int hkv, 
   const float rc = p.rc_o;
   const int G = p.G;
 #pragma unroll
-  for (int hp = 0; hp < 2; ++hp) {
-    const int head = 2 * t + hp;
+  for (int hp = 0; hp < (PC ? 1 : 2); ++hp) {
+    const int head = PC ? t : 2 * t + hp;
     if (head >= G) continue;
     const long long row = (MULTI ? q_row(p, b, hkv, head) : static_cast<long long>(b) * p.Hq + hkv * G + head) * D;
     if (p.mode & KV4_MODE_OUT_F32) {
@@ -313,9 +318,9 @@ __global__ void __launch_bounds__(32 * QWARPS) gq_kernel(AttnParams p) {
   uint8_t* blob = p.qblob + static_cast<size_t>(gw) * qblob_bytes(D);
   if constexpr (D == 128) {
     if (p.qfmt == 1) store_qblob_tc<D>(blob, qf, lane);
-    else store_qblob<D>(blob, qf, lane);
+    else store_qblob<D>(blob, qf, lane, p.qfmt == 3);
   } else {
-    store_qblob<D>(blob, qf, lane);
+    store_qblob<D>(blob, qf, lane, p.qfmt == 3);
   }
 }
 
@@ -376,9 +381,9 @@ __global__ void __launch_bounds__(32 * MAXW) gstep_kernel(AttnParams p, AppendPa
     uint8_t* blob = p.qblob + (static_cast<size_t>(b) * p.Hkv + h) * qblob_bytes(D);
     if constexpr (D == 128) {
       if (p.qfmt == 1) store_qblob_tc<D>(blob, qf, lane);
-      else store_qblob<D>(blob, qf, lane);
+      else store_qblob<D>(blob, qf, lane, p.qfmt == 3);
     } else {
-      store_qblob<D>(blob, qf, lane);
+      store_qblob<D>(blob, qf, lane, p.qfmt == 3);
     }
   }
   if (s_ok && page >= 0) {
@@ -602,8 +607,11 @@ __device__ void produce(const AttnParams& p, GMisc* misc, SegQ* segq, uint8_t* r
 // several query tokens per sequence (causal visibility per operand column);
 // the one-token variant carries none of that code.  GWR: KV heads per group.
 // F: page format (0 INT4, 1 NVFP4, 2 INT2; the INT8 store is the same).
-template <int D, int PAIR, bool MULTI, int GWR, int F = 0>
+// PCOL: paired columns (one query token, at most 4 query heads per KV head,
+// integer query planes; see unit_int4_pc).
+template <int D, int PAIR, bool MULTI, int GWR, int F = 0, bool PCOL = false>
 __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
+  static_assert(!PCOL || (!MULTI && F != 1), "paired columns: one query token, integer query planes");
   using C = GCfg<D, GWR, F>;
   using SH = GShape<GWR>;
   constexpr int GTHREADS = SH::THREADS;
@@ -675,7 +683,7 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
     {
       const uint8_t* blob = p.qblob + static_cast<size_t>(g.b * p.Hkv + g.hg * GWR + w) * qblob_bytes(D);
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = 0; cc < (PCOL ? D / 64 : D / 32); ++cc) {
         const uint4 v = __ldcg(reinterpret_cast<const uint4*>(blob) + 32 * cc + lane);
         qf.b[2 * cc][0] = v.x; qf.b[2 * cc][1] = v.y; qf.b[2 * cc + 1][0] = v.z; qf.b[2 * cc + 1][1] = v.w;
       }
@@ -723,6 +731,10 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
           if constexpr (F == 1) {
             if (nt == PAIR) unit_fp4<D, PAIR, false>(tl, qf, ws, lane, valid, valid, eb, cs);
             else unit_fp4<D, 1, false>(tl, qf, ws, lane, valid, valid, eb, cs);
+          } else if constexpr (PCOL) {
+            constexpr int BITS = F == 2 ? 2 : 4;
+            if (nt == PAIR) unit_int4_pc<D, PAIR, false, BITS>(tl, qf, ws, lane, valid, eb);
+            else unit_int4_pc<D, 1, false, BITS>(tl, qf, ws, lane, valid, eb);
           } else {
             constexpr int BITS = F == 2 ? 2 : 4;
             if (nt == PAIR) unit_int4<D, PAIR, false, false, BITS>(tl, qf, ws, lane, valid, eb, cs);
@@ -745,6 +757,10 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
             for (int k = 0; k < PAIR; ++k) nwr[k] = min(max(g.L - (pos0 + k * TILE), 0), TILE);
             if (nt == PAIR) unit_fp4<D, PAIR, true, MULTI>(tl, qf, ws, lane, valid, nwr, eb, cs);
             else unit_fp4<D, 1, true, MULTI>(tl, qf, ws, lane, valid, nwr, eb, cs);
+          } else if constexpr (PCOL) {
+            constexpr int BITS = F == 2 ? 2 : 4;
+            if (nt == PAIR) unit_int4_pc<D, PAIR, true, BITS>(tl, qf, ws, lane, valid, eb);
+            else unit_int4_pc<D, 1, true, BITS>(tl, qf, ws, lane, valid, eb);
           } else {
             constexpr int BITS = F == 2 ? 2 : 4;
             if (nt == PAIR) unit_int4<D, PAIR, true, MULTI, BITS>(tl, qf, ws, lane, valid, eb, cs);
@@ -764,7 +780,10 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
         if (v % SH::S8 == w / SH::H8) {
           const uint32_t st = smem_u32(ring + static_cast<size_t>(s0) * C::STAGE + (w % SH::H8) * tile8_bytes(D));
           const int slot0 = (v / SH::S8) * TILE;
-          if (slot0 + TILE <= g.nprot && !MULTI) {
+          if constexpr (PCOL) {
+            if (slot0 + TILE <= g.nprot) tile_int8_pc<D, false>(st, qf, ws, lane, 15, eb);
+            else tile_int8_pc<D, true>(st, qf, ws, lane, (slot0 + g8 < g.nprot ? 3 : 0) | (slot0 + g8 + 8 < g.nprot ? 12 : 0), eb);
+          } else if (slot0 + TILE <= g.nprot && !MULTI) {
             tile_int8<D, false, false, F == 1>(st, qf, ws, lane, 15, eb, cs);
           } else if (!MULTI) {
             tile_int8<D, true, false, F == 1>(st, qf, ws, lane,
@@ -794,6 +813,31 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
     if (!ok) break;
 
     // ---- the segment's result for this warp's head
+    if constexpr (PCOL) {
+      // head t: its two column sums, then l and the zero-point sum over the lane's row groups
+#pragma unroll
+      for (int m = 0; m < D / 16; ++m) { ws.o[m][0] += ws.o[m][1]; ws.o[m][2] += ws.o[m][3]; }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        ws.l0 += __shfl_xor_sync(0xffffffffu, ws.l0, o);
+        ws.z0 += __shfl_xor_sync(0xffffffffu, ws.z0, o);
+      }
+#pragma unroll
+      for (int m = 0; m < D / 16; ++m) { ws.o[m][0] += ws.z0; ws.o[m][2] += ws.z0; }
+      const int hkv = g.hg * GWR + w;
+      if (sq.nseg == 1) {
+        store_head<D, false, true>(p, g.b, hkv, lane, ws.o, ws.l0, 0.f);
+        continue;
+      }
+      const int slotp = (c * 2 + (q == 0 ? 0 : 1)) * GWR + w;
+      if (t < G) {
+        float* r = p.partials + static_cast<size_t>(slotp) * pstride + t * HS;
+#pragma unroll
+        for (int m = 0; m < D / 16; ++m) { r[16 * m + g8] = ws.o[m][0]; r[16 * m + g8 + 8] = ws.o[m][2]; }
+        if (g8 == 0) { r[D] = ws.m0; r[D + 1] = ws.l0; }
+      }
+      continue;
+    }
     if (cs.colsplit) {
       if (G == 1) {
 #pragma unroll
@@ -1441,6 +1485,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tattn_kernel(AttnParams p, GPla
 #endif
 constexpr int kPair = KV4_GROUPED_PAIR;   // INT4 tiles per consumer iteration of the compiled variant
 static_assert(kPair == 1 || kPair == 2 || kPair == 4, "tiles per iteration");
+#ifndef KV4_PC_PAIR
+#define KV4_PC_PAIR 4
+#endif
+// INT4 tiles per iteration of the paired-column variant: it has the registers for four (117 at D = 128),
+// which measured 2-3 % faster than two on batches of 256 and 512 sequences
+constexpr int kPairPC = KV4_PC_PAIR;
+static_assert(kPairPC == 1 || kPairPC == 2 || kPairPC == 4, "tiles per iteration");
 
 inline size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -1469,27 +1520,36 @@ GLayout g_layout(const kv4_cache* c, int n_seqs, int qlen) {
 
 // Deepest ring (at most MAX_NS stages) that keeps CTAS_PER_SM CTAs of both
 // variants (one and several query tokens) of page format F resident per SM.
-template <int D, int PAIR, int GWR, int F>
+template <int D, int PAIR, int PAIRPC, int GWR, int F>
 int g_choose_ring(int device) {
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess) return -1;
+  // the paired-column variant exists for the integer page formats (the NVFP4 one instantiates the plain one twice)
+  constexpr bool PCV = F != 1;
   if (cudaFuncSetAttribute(gattn_kernel<D, PAIR, false, GWR, F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            optin) != cudaSuccess ||
       cudaFuncSetAttribute(gattn_kernel<D, PAIR, true, GWR, F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           optin) != cudaSuccess ||
+      cudaFuncSetAttribute(gattn_kernel<D, PAIRPC, false, GWR, F, PCV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            optin) != cudaSuccess)
     return -1;
   const int want = CTAS_PER_SM;
-  for (int ns = MAX_NS; ns >= 2; --ns) {
+  // a consumer warp holds up to PAIR stages of a unit at once: keep as many more in flight
+  constexpr int NS_MIN = 2 * (PAIR > PAIRPC ? PAIR : PAIRPC);
+  for (int ns = MAX_NS; ns >= NS_MIN; --ns) {
     const size_t smem = gattn_smem_bytes<D, GWR, F>(ns);
     if (smem > static_cast<size_t>(optin)) continue;
     int blocks = 0;
     int blocks_multi = 0;
+    int blocks_pc = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, gattn_kernel<D, PAIR, false, GWR, F>,
                                                       GShape<GWR>::THREADS, smem) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_multi, gattn_kernel<D, PAIR, true, GWR, F>,
+                                                      GShape<GWR>::THREADS, smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_pc, gattn_kernel<D, PAIRPC, false, GWR, F, PCV>,
                                                       GShape<GWR>::THREADS, smem) != cudaSuccess)
       return -1;
-    if (blocks >= want && blocks_multi >= want) return ns;
+    if (blocks >= want && blocks_multi >= want && blocks_pc >= want) return ns;
   }
   return -1;
 }
@@ -1504,7 +1564,9 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   // one query token, 4-head groups, D = 128, INT4 pages: the tensor-memory kernel when selected, one CTA per SM
   const bool fp4 = c->cfg.page_format == KV4_FORMAT_NVFP4, int2 = c->cfg.page_format == KV4_FORMAT_INT2;
   const bool tcpath = D == 128 && GWR == 4 && c->use_tc && p.qtot == 1 && c->cfg.page_format == KV4_FORMAT_INT4;
-  p.qfmt = tcpath ? 1 : (fp4 ? 2 : 0);
+  // one query token and at most 4 query heads per KV head on integer pages: paired columns
+  const bool pcol = !tcpath && !fp4 && p.qtot == 1 && p.G <= 4;
+  p.qfmt = tcpath ? 1 : (fp4 ? 2 : (pcol ? 3 : 0));
   p.grid = tcpath ? c->num_sms : g_grid(c);
   p.cap_parts = p.grid * 2 * GWR;
   p.ns = tcpath ? c->tattn_ring : c->gattn_ring;
@@ -1540,13 +1602,14 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
                    : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false, GWR, 1>, p, plan);
   } else if (int2) {
     e = p.qtot > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true, GWR, 2>, p, plan)
+        : pcol     ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPairPC, false, GWR, 2, true>, p, plan)
                    : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false, GWR, 2>, p, plan);
-  } else if constexpr (D == 128 && GWR == 4) {
-    if (tcpath) e = cudaLaunchKernelEx(&cfg, tattn_kernel<D>, p, plan);
-    else if (p.qtot > 1) e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true, GWR>, p, plan);
-    else e = cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false, GWR>, p, plan);
+  } else if (tcpath) {
+    if constexpr (D == 128 && GWR == 4) e = cudaLaunchKernelEx(&cfg, tattn_kernel<D>, p, plan);
+    else e = cudaErrorInvalidValue;
   } else {
     e = p.qtot > 1 ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, true, GWR>, p, plan)
+        : pcol     ? cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPairPC, false, GWR, 0, true>, p, plan)
                    : cudaLaunchKernelEx(&cfg, gattn_kernel<D, kPair, false, GWR>, p, plan);
   }
   if (e == cudaSuccess) {
@@ -1573,9 +1636,9 @@ int g_launch_gw(kv4_cache* c, const AttnParams& p, void* ws, cudaStream_t stream
 template <int D, int F>
 int g_choose_ring_gw(int device, int Hkv) {
   switch (group_width(Hkv)) {
-    case 4: return g_choose_ring<D, kPair, 4, F>(device);
-    case 2: return g_choose_ring<D, kPair, 2, F>(device);
-    default: return g_choose_ring<D, kPair, 1, F>(device);
+    case 4: return g_choose_ring<D, kPair, kPairPC, 4, F>(device);
+    case 2: return g_choose_ring<D, kPair, kPairPC, 2, F>(device);
+    default: return g_choose_ring<D, kPair, kPairPC, 1, F>(device);
   }
 }
 

@@ -325,6 +325,147 @@ __device__ __forceinline__ void unit_int4(const uint32_t* tile, const QFrag<D>& 
 }
 
 // ---------------------------------------------------------------------------
+// Paired columns: one query token and at most 4 query heads per KV head.
+// Column 2c of the 16x8x32 score multiply holds the high byte of query head c,
+// column 2c+1 its low byte, both signed (q = 256 hi + lo, |q| < 2^14), so one
+// integer multiply per 32 dims gives both planes and lane (g, t) ends up with
+// the two partial sums of head t for tokens g and g+8.  Each lane then owns
+// head t alone through the softmax (m0, l0, z0 of WarpState), with no score
+// handled twice.  The P.V weights pair the same way: column 2t carries
+// fp16(P), column 2t+1 fp16(P - fp16(P)), and one 16x8x16 multiply per 16 dims
+// accumulates both; o[m][0] + o[m][1] (dim 16m+g) and o[m][2] + o[m][3]
+// (dim 16m+g+8) is head t's sum at the end of a segment.
+
+// Online-softmax update of head t with the scores of n tokens (x[i], -inf for
+// a token outside the range; every unit holds at least one visible token).
+template <int D, int N>
+__device__ __forceinline__ void softmax_pc(WarpState<D>& ws, const float (&x)[N], float (&pr)[N]) {
+  float mx = x[0];
+#pragma unroll
+  for (int i = 1; i < N; ++i) mx = fmaxf(mx, x[i]);
+  if (__any_sync(0xffffffffu, mx > ws.m0)) {
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float n0 = fmaxf(ws.m0, mx);
+    const float a0 = ex2(ws.m0 - n0);
+    ws.l0 *= a0; ws.z0 *= a0;
+#pragma unroll
+    for (int m = 0; m < D / 16; ++m) { ws.o[m][0] *= a0; ws.o[m][1] *= a0; ws.o[m][2] *= a0; ws.o[m][3] *= a0; }
+    ws.m0 = n0;
+  }
+#pragma unroll
+  for (int i = 0; i < N; ++i) pr[i] = ex2(x[i] - ws.m0);
+}
+
+// P.V weights of head t for tokens g and g+8 as the B fragments of one 16x8x16 multiply (fp16 P in
+// column 2t, the fp16 remainder in column 2t+1).
+__device__ __forceinline__ void pv_operands_pc(float P0, float P1, uint32_t& B0, uint32_t& B1) {
+  const uint32_t h = pack_half2(P0, P1);
+  const uint32_t l = pack_half2(P0 - half_lo(h), P1 - half_hi(h));
+  B0 = movmatrix_trans(__byte_perm(h, l, 0x5410));   // token g: (hi, lo)
+  B1 = movmatrix_trans(__byte_perm(h, l, 0x7632));   // token g+8
+}
+
+// Scores of head t from the paired integer sums, the zero point folded in.
+__device__ __forceinline__ float score_pc(int hi, int lo, uint32_t szk, float kscale, float qs) {
+  return fmaf(static_cast<float>(hi * 256 + lo), half_lo(szk) * kscale, half_hi(szk) * qs);
+}
+
+// unit_int4 with paired columns (one query token).  valid[u]: bit 0 token g,
+// bit 2 token g+8 of tile u inside the range being read (MASKED).
+template <int D, int NT, bool MASKED, int BITS = 4>
+__device__ __forceinline__ void unit_int4_pc(const uint32_t* tile, const QFrag<D>& qf, WarpState<D>& ws, int lane,
+                                             const int* valid, const uint32_t* eb) {
+  static_assert(BITS == 4 || BITS == 2, "code width");
+  constexpr int SZOFF = BITS == 4 ? 16 * D : 8 * D;
+  constexpr float VCENTRE = BITS == 4 ? 8.f : 2.f;
+  constexpr int NKK = D / 32;
+  uint32_t kw[NT][2][NKK];
+  uint4 sz[NT];
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    if constexpr (BITS == 4 && D == 128) {
+      const uint4 a = lds128(tile[u] + lane * 16), bq = lds128(tile[u] + 512 + lane * 16);
+      kw[u][0][0] = a.x; kw[u][0][1] = a.y; kw[u][0][2] = a.z; kw[u][0][3] = a.w;
+      kw[u][1][0] = bq.x; kw[u][1][1] = bq.y; kw[u][1][2] = bq.z; kw[u][1][3] = bq.w;
+    } else if constexpr (BITS == 4 || D == 128) {
+      const uint2 a = lds64(tile[u] + lane * 8), bq = lds64(tile[u] + 256 + lane * 8);
+      kw[u][0][0] = a.x; kw[u][0][1] = a.y; kw[u][1][0] = bq.x; kw[u][1][1] = bq.y;
+    } else {
+      kw[u][0][0] = lds32(tile[u] + lane * 4);
+      kw[u][1][0] = lds32(tile[u] + 128 + lane * 4);
+    }
+    sz[u] = lds128(tile[u] + SZOFF + (lane >> 2) * 16);
+  }
+  int acc[NT][4];
+#pragma unroll
+  for (int u = 0; u < NT; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[u][i] = 0;
+#pragma unroll
+  for (int kk = 0; kk < NKK; ++kk) {
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      if constexpr (BITS == 4) {
+        const uint32_t w0 = kw[u][0][kk], w1 = kw[u][1][kk];
+        imma_u8s8(acc[u], w0 & 0x0F0F0F0Fu, w1 & 0x0F0F0F0Fu, (w0 >> 4) & 0x0F0F0F0Fu, (w1 >> 4) & 0x0F0F0F0Fu,
+                  qf.b[kk][0], qf.b[kk][1]);
+      } else {
+        const int sh = 4 * (kk & 1);
+        const uint32_t w0 = kw[u][0][kk >> 1] >> sh, w1 = kw[u][1][kk >> 1] >> sh;
+        imma_u8s8(acc[u], w0 & 0x03030303u, w1 & 0x03030303u, (w0 >> 2) & 0x03030303u, (w1 >> 2) & 0x03030303u,
+                  qf.b[kk][0], qf.b[kk][1]);
+      }
+    }
+  }
+  float x[2 * NT];
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    x[2 * u] = score_pc(acc[u][0], acc[u][1], sz[u].x, qf.kscale, qf.qs0);
+    x[2 * u + 1] = score_pc(acc[u][2], acc[u][3], sz[u].y, qf.kscale, qf.qs0);
+    if constexpr (MASKED) {
+      if (!(valid[u] & 1)) x[2 * u] = NEG_INF;
+      if (!(valid[u] & 4)) x[2 * u + 1] = NEG_INF;
+    }
+  }
+  float pr[2 * NT];
+  softmax_pc<D, 2 * NT>(ws, x, pr);
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    const float p0 = pr[2 * u], p1 = pr[2 * u + 1];
+    const float sVg = half_lo(sz[u].z), sVg8 = half_lo(sz[u].w);
+    const float zVg = fmaf(VCENTRE, sVg, half_hi(sz[u].z)), zVg8 = fmaf(VCENTRE, sVg8, half_hi(sz[u].w));   // centred
+    float P0 = p0 * sVg, P1 = p1 * sVg8;
+    float zg = p0 * zVg, zg8 = p1 * zVg8;
+    if constexpr (MASKED) {   // unwritten slots may hold non-finite scales
+      if (!(valid[u] & 1)) { P0 = 0.f; zg = 0.f; }
+      if (!(valid[u] & 4)) { P1 = 0.f; zg8 = 0.f; }
+    }
+    ws.l0 += p0 + p1;
+    ws.z0 += zg + zg8;
+    uint32_t B0, B1;
+    pv_operands_pc(P0, P1, B0, B1);
+    uint32_t vw[D / 16];
+    load_v_words<D, BITS>(tile[u], lane, vw);
+    if (u == NT - 1) {
+      // the last V loads are done: hand the stage(s) back before the math
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int k = 0; k < NT; ++k)
+          if (k == 0 || eb[k] != eb[k - 1]) mbar_arrive(eb[k]);
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < D / 16; ++m) {
+      uint32_t a0, a1, a2, a3;
+      v_operands<BITS>(vw, m, a0, a1, a2, a3);
+      mma_f16(ws.o[m], a0, a1, a2, a3, B0, B1);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // NVFP4 pages ("KV Cache Quantization" topic page, item 3: NVFP4 storage of
 // the paged KV cache).  A tile holds E2M1 codes and one E4M3 scale per token
 // and 16 dims.  Both products run on 16x8x16 fp16 multiplies: the hardware
@@ -587,6 +728,58 @@ __device__ __forceinline__ void tile_int8(uint32_t st, const QFrag<D>& qf, WarpS
   }
 }
 
+// tile_int8 with paired columns (one query token, integer query planes).  vm:
+// bit 0 token g, bit 2 token g+8 inside the protected range (MASKED).
+template <int D, bool MASKED>
+__device__ __forceinline__ void tile_int8_pc(uint32_t st, const QFrag<D>& qf, WarpState<D>& ws, int lane, int vm,
+                                             uint32_t empty_bar) {
+  constexpr int NK = D / 16;
+  uint32_t kw[2][NK], vw[2 * NK];
+#pragma unroll
+  for (int rowhi = 0; rowhi < 2; ++rowhi)
+#pragma unroll
+    for (int kq = 0; kq < D / 64; ++kq) {
+      const uint4 a = lds128(st + rowhi * 8 * D + (D / 4) * lane + 16 * kq);
+      kw[rowhi][4 * kq] = a.x; kw[rowhi][4 * kq + 1] = a.y; kw[rowhi][4 * kq + 2] = a.z; kw[rowhi][4 * kq + 3] = a.w;
+    }
+#pragma unroll
+  for (int q4 = 0; q4 < NK / 2; ++q4) {
+    const uint4 a = lds128(st + 16 * D + 16 * (32 * q4 + lane));
+    vw[4 * q4] = a.x; vw[4 * q4 + 1] = a.y; vw[4 * q4 + 2] = a.z; vw[4 * q4 + 3] = a.w;
+  }
+  const uint4 sz = lds128(st + 32 * D + (lane >> 2) * 16);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty_bar);
+  int acc[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int kk = 0; kk < D / 32; ++kk)
+    imma_u8s8(acc, kw[0][2 * kk], kw[1][2 * kk], kw[0][2 * kk + 1], kw[1][2 * kk + 1], qf.b[kk][0], qf.b[kk][1]);
+  float x[2] = {score_pc(acc[0], acc[1], sz.x, qf.kscale, qf.qs0), score_pc(acc[2], acc[3], sz.y, qf.kscale, qf.qs0)};
+  if constexpr (MASKED) {
+    if (!(vm & 1)) x[0] = NEG_INF;
+    if (!(vm & 4)) x[1] = NEG_INF;
+  }
+  float pr[2];
+  softmax_pc<D, 2>(ws, x, pr);
+  const float sVg = half_lo(sz.z), sVg8 = half_lo(sz.w);
+  const float zVg = fmaf(128.f, sVg, half_hi(sz.z)), zVg8 = fmaf(128.f, sVg8, half_hi(sz.w));   // centred codes
+  float P0 = pr[0] * sVg, P1 = pr[1] * sVg8;
+  float zg = pr[0] * zVg, zg8 = pr[1] * zVg8;
+  if constexpr (MASKED) {
+    if (!(vm & 1)) { P0 = 0.f; zg = 0.f; }
+    if (!(vm & 4)) { P1 = 0.f; zg8 = 0.f; }
+  }
+  ws.l0 += pr[0] + pr[1];
+  ws.z0 += zg + zg8;
+  uint32_t B0, B1;
+  pv_operands_pc(P0, P1, B0, B1);
+#pragma unroll
+  for (int m = 0; m < NK; ++m) {
+    const uint32_t w0 = vw[2 * m], w1 = vw[2 * m + 1];
+    mma_f16(ws.o[m], byte_lo_c(w0), byte_lo_c(w0 >> 8), byte_lo_c(w1), byte_lo_c(w1 >> 8), B0, B1);
+  }
+}
+
 // One BF16 tile (baseline cache).  Holds the stage until the V loads are done.
 // vmask01 / vmask89: per-thread masks of the V operand halves of tokens 2t, 2t+1
 // and 2t+8, 2t+9 (unwritten slots of a page may hold NaN bit patterns, and
@@ -635,7 +828,7 @@ template <int D>
 __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, int lane, QFrag<D>& qf,
                                            int L_known = -1);
 template <int D>
-__device__ __forceinline__ void store_qblob(uint8_t* blob, const QFrag<D>& qf, int lane);
+__device__ __forceinline__ void store_qblob(uint8_t* blob, const QFrag<D>& qf, int lane, bool paired);
 
 template <int D, bool BF16>
 __device__ __forceinline__ void build_qblob(const AttnParams& p, int b, int h, int lane, float* sq) {
@@ -645,7 +838,7 @@ __device__ __forceinline__ void build_qblob(const AttnParams& p, int b, int h, i
   if constexpr (!BF16) {   // INT4/INT8 caches: the integer query planes
     QFrag<D> qf;
     load_qfrag<D>(p, b, h, lane, qf);
-    store_qblob<D>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D), qf, lane);
+    store_qblob<D>(p.qblob + static_cast<size_t>(gw) * qblob_bytes(D), qf, lane, p.qfmt == 3);
     return;
   }
   float qsum[MAX_G];
@@ -785,7 +978,8 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
   constexpr int NKK = D / 32;
   const int G = p.G, g8 = lane >> 2, t = lane & 3;
   const bool colsplit = (G == 1 || G == 2 || G == 4);
-  const int gsrc = colsplit ? g8 % G : g8;
+  const bool pc = p.qfmt == 3;   // paired columns: column g8 is plane g8 % 2 of head g8 / 2
+  const int gsrc = pc ? (g8 >> 1) : (colsplit ? g8 % G : g8);
   const bool active = gsrc < G;
   const uint16_t* src = p.q + q_row(p, b, h, active ? gsrc : 0) * D + 4 * t;
   float x[NKK][2][4];
@@ -898,6 +1092,9 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
     int ex;
     frexpf(amax, &ex);
     e = 15 - ex;
+    // paired columns: 256 hi + lo with both signed bytes reaches 32639; the one scaled bf16 value above
+    // it (32640, an all-ones mantissa at the top of the range) takes one bit less for the whole operand
+    if (pc && ldexpf(amax, e) > 32639.f) e = 14 - ex;
   }
   if (p.qfmt == 2) {
     // fp16 B fragments of 16x8x16 multiplies (NVFP4 pages): block 2kk + hf holds dims 4t, 4t+1
@@ -908,6 +1105,22 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
       for (int hf = 0; hf < 2; ++hf) {
         qf.b[2 * kk + hf][0] = pack_half2(ldexpf(x[kk][hf][0], e), ldexpf(x[kk][hf][1], e));
         qf.b[2 * kk + hf][1] = pack_half2(ldexpf(x[kk][hf][2], e), ldexpf(x[kk][hf][3], e));
+      }
+  } else if (pc) {
+    // |q| <= 32639: hi = round(q / 256) and lo = q - 256 hi are both signed bytes
+#pragma unroll
+    for (int kk = 0; kk < NKK; ++kk)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t w = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int qi = __float2int_rn(ldexpf(x[kk][hf][j], e));
+          const int hi = (qi + 128) >> 8;
+          w |= (static_cast<uint32_t>((g8 & 1) ? qi - 256 * hi : hi) & 0xFFu) << (8 * j);
+        }
+        qf.b[kk][hf] = w;
+        qf.b[NKK + kk][hf] = 0u;
       }
   } else {
 #pragma unroll
@@ -925,7 +1138,8 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
         qf.b[NKK + kk][hf] = wlo;
       }
   }
-  // sum(q) of the heads of this lane's columns 2t and 2t+1 (held by lanes 8t and 8t+4)
+  // sum(q) of the heads of this lane's columns 2t and 2t+1 (held by lanes 8t and 8t+4); with paired
+  // columns lane 8t holds head t, the one this lane owns
   qf.qs0 = __shfl_sync(0xffffffffu, qs, 8 * t) * p.scale_log2;
   qf.qs1 = __shfl_sync(0xffffffffu, qs, 8 * t + 4) * p.scale_log2;
   qf.kscale = ldexpf(p.scale_log2, -e);
@@ -935,11 +1149,13 @@ __device__ __forceinline__ void load_qfrag(const AttnParams& p, int b, int h, in
 // the 16-byte B-fragment words of every lane, then the sums of the 8 columns
 // and kscale.
 template <int D>
-__device__ __forceinline__ void store_qblob(uint8_t* blob, const QFrag<D>& qf, int lane) {
+__device__ __forceinline__ void store_qblob(uint8_t* blob, const QFrag<D>& qf, int lane, bool paired) {
+  // paired columns: both planes share b[0 .. D/32), half the words
 #pragma unroll
   for (int cc = 0; cc < D / 32; ++cc)
-    reinterpret_cast<uint4*>(blob)[cc * 32 + lane] =
-        make_uint4(qf.b[2 * cc][0], qf.b[2 * cc][1], qf.b[2 * cc + 1][0], qf.b[2 * cc + 1][1]);
+    if (cc < D / 64 || !paired)
+      reinterpret_cast<uint4*>(blob)[cc * 32 + lane] =
+          make_uint4(qf.b[2 * cc][0], qf.b[2 * cc][1], qf.b[2 * cc + 1][0], qf.b[2 * cc + 1][1]);
   float* tail = reinterpret_cast<float*>(blob + 16 * D);
   if (lane < 4) { tail[2 * lane] = qf.qs0; tail[2 * lane + 1] = qf.qs1; }   // lanes 0-3: columns 2t, 2t+1
   if (lane == 0) tail[MAX_G] = qf.kscale;

@@ -123,7 +123,8 @@ struct AttnParams {
   int grid;                   // CTAs of the page-major attention kernel
   int stall_stage;            // test hook: stage the first CTA leaves unfilled (-1: none)
   int qfmt;                   // query operand layout the query kernels write: 0 integer fragments, 1 tensor-memory
-                              // kernel, 2 fp16 fragments (NVFP4 pages)
+                              // kernel, 2 fp16 fragments (NVFP4 pages), 3 paired integer columns (one query
+                              // token, at most 4 query heads per KV head)
 };
 
 // Row of q (and of the output) that operand column c of KV head h of batch
