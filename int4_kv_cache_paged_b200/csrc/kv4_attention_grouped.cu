@@ -337,13 +337,15 @@ __global__ void __launch_bounds__(32 * QWARPS) gq_kernel(AttnParams p) {
 // MAXW: the most warps a block of this instantiation has (2 * Hkv <= MAXW);
 // 16 for up to 8 KV heads (128 registers a thread), 32 for up to 16.
 template <int D, int MAXW>
-__global__ void __launch_bounds__(32 * MAXW) gstep_kernel(AttnParams p, AppendParams ap) {
+__global__ void __launch_bounds__(32 * MAXW, 32 / MAXW) gstep_kernel(AttnParams p, AppendParams ap) {
   constexpr int VPL = D / 32;
   __shared__ __align__(16) uint8_t s_codes[MAXW][2][D];
   __shared__ int s_seq, s_L, s_ok, s_page;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int tensor = warp >= p.Hkv ? 1 : 0, h = warp - tensor * p.Hkv;
   const int b = blockIdx.x;
+  // the attention kernel may be scheduled as blocks of this grid retire (it waits for the whole grid)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // this warp's new row: k_new / v_new [n_seqs][Hkv][D], entry b
   uint16_t raw[VPL];
   {
@@ -630,6 +632,8 @@ __global__ void __maxnreg__(128) gattn_kernel(AttnParams p, GPlanRec* plan) {
 
   // the merge kernel may be scheduled now: it waits for this grid before reading its results
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // after the fused step kernel: its lengths, pages and query operands are written once that grid is done
+  if (p.wait_first) asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, GWR); }
     for (int s = 0; s < GQD; ++s) { mbar_init(iqf0 + 8 * s, 1); mbar_init(iqe0 + 8 * s, GWR); }
@@ -1075,6 +1079,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tattn_kernel(AttnParams p, GPla
   const int c = blockIdx.x;
 
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (p.wait_first) asm volatile("griddepcontrol.wait;" ::: "memory");   // after the fused step kernel
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, TC_WG); }
     for (int s = 0; s < GQD; ++s) { mbar_init(iqf0 + 8 * s, 1); mbar_init(iqe0 + 8 * s, TC_WG); }
@@ -1594,7 +1599,11 @@ int g_launch(kv4_cache* c, AttnParams p, void* ws, cudaStream_t stream, const Ap
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = step ? 0 : 1;
+  // programmatic dependent of the query kernel (it waits only before its first query read) or of the
+  // fused step kernel (it waits before its first instruction); an event marker between the two launches
+  // leaves them in plain stream order
+  cfg.numAttrs = (step && c->ev_before) ? 0 : 1;
+  p.wait_first = step ? 1 : 0;
   // several query tokens per sequence (even a pass of one of them): the causal variant
   cudaError_t e;
   if (fp4) {

@@ -125,6 +125,8 @@ struct AttnParams {
   int qfmt;                   // query operand layout the query kernels write: 0 integer fragments, 1 tensor-memory
                               // kernel, 2 fp16 fragments (NVFP4 pages), 3 paired integer columns (one query
                               // token, at most 4 query heads per KV head)
+  int wait_first;             // the attention kernel is the programmatic dependent of the fused step kernel: it
+                              // waits for that grid before its first instruction (the plan reads the new lengths)
 };
 
 // Row of q (and of the output) that operand column c of KV head h of batch
