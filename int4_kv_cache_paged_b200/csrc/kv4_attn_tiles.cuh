@@ -136,10 +136,15 @@ __device__ __forceinline__ void load_v_words(uint32_t st, int lane, uint32_t (&v
   }
 }
 
-// Crumbs at bits 0-1 and 16-17 as an fp16 pair, minus 2 (exact).
+// Crumbs at bits P, P+1 and 16+P, 17+P (P <= 8) as an fp16 pair, minus 2 (exact): under the magic
+// exponent the crumb is the half 1024 + c 2^P, and one fma by 2^-P takes away 1024 2^-P + 2.
+template <int P>
 __device__ __forceinline__ uint32_t crumb_c(uint32_t w) {
-  uint32_t x = lop3_and_or(w, 0x00030003u, 0x64006400u);
-  __half2 h = __hsub2(*reinterpret_cast<__half2*>(&x), __half2(__half(1026.f), __half(1026.f)));
+  static_assert(P >= 0 && P <= 8, "crumb inside the fp16 mantissa");
+  uint32_t x = lop3_and_or(w, 0x00030003u << P, 0x64006400u);
+  const __half sc = __float2half_rn(1.f / static_cast<float>(1 << P));
+  const __half b = __float2half_rn(-(1024.f / static_cast<float>(1 << P) + 2.f));
+  __half2 h = __hfma2(*reinterpret_cast<__half2*>(&x), __half2(sc, sc), __half2(b, b));
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
@@ -152,8 +157,14 @@ __device__ __forceinline__ void v_operands(const uint32_t* vw, int m, uint32_t& 
     const uint32_t w = vw[m], u = w >> 8;
     a0 = nib_lo_c(w); a1 = nib_hi_c(w); a2 = nib_lo_c(u); a3 = nib_hi_c(u);
   } else {
-    const uint32_t w = vw[m >> 1] >> (4 * (m & 1));
-    a0 = crumb_c(w); a1 = crumb_c(w >> 2); a2 = crumb_c(w >> 8); a3 = crumb_c(w >> 10);
+    // block m of the pair sits at bits 4 (m % 2) + {0, 2} (dims g, g+8) of the low byte of each half (tokens
+    // 2t, 2t+1) and 8 further (tokens 2t+8, 2t+9); a crumb above bit 8 of a half takes one shift
+    const uint32_t w = vw[m >> 1], u = w >> 8;
+    if (m & 1) {
+      a0 = crumb_c<4>(w); a1 = crumb_c<6>(w); a2 = crumb_c<4>(u); a3 = crumb_c<6>(u);
+    } else {
+      a0 = crumb_c<0>(w); a1 = crumb_c<2>(w); a2 = crumb_c<8>(w); a3 = crumb_c<2>(u);
+    }
   }
 }
 
