@@ -313,6 +313,26 @@ def reduce_over_ranks(times, counts, device, world):
     return t.tolist(), c.tolist()
 
 
+class Nvtx:
+    """NVTX ranges through torch, or nothing where its build has none."""
+
+    def __init__(self, torch):
+        self.m = getattr(torch.cuda, "nvtx", None)
+        try:
+            self.m.range_push("kv4")
+            self.m.range_pop()
+        except Exception:   # noqa: BLE001 -- any failure: no ranges
+            self.m = None
+
+    def push(self, name):
+        if self.m is not None:
+            self.m.range_push(name)
+
+    def pop(self):
+        if self.m is not None:
+            self.m.range_pop()
+
+
 def measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=1, compare=True):
     """Build a replica of workload `w` (its first `layers` layer caches) and time it.
 
@@ -353,10 +373,13 @@ def measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=1, compare
             dist.barrier()
         torch.cuda.synchronize()
 
+    nvtx = Nvtx(torch)       # phase ranges for profilers (no per-layer markers in the timed loops)
+
     # ---- the timed loop: W_ warm-up steps, then K steps, each through every layer
     n = W_ + K
     e_step = [(ev(), ev()) for _ in range(n)]
     barrier()
+    nvtx.push("kv4 timed steps")
     for i in range(n):
         if i == W_:
             barrier()
@@ -368,6 +391,7 @@ def measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=1, compare
         e_step[i][1].record(stream)
     clocks.sample_now(4, 0.0003)                # while the queued steps run
     barrier()
+    nvtx.pop()
     clocks.window(t_window, time.perf_counter())
     t_step = sum(e_step[i][0].elapsed_time(e_step[i][1]) for i in range(W_, n)) / 1e3
     bytes_timed = sum(rep.bytes_at(i + 1) * layers for i in range(W_, n))
@@ -377,6 +401,7 @@ def measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=1, compare
     # two launches adds about 2 us to a layer
     e_kern = [[(ev(), ev()) for _ in range(layers)] for _ in range(K)]
     e_kstep = [(ev(), ev()) for _ in range(K)]   # the steps of this pass, for the time outside the kernels
+    nvtx.push("kv4 steps with kernel events")
     t_window = time.perf_counter()
     for j in range(K):
         flush.fill_(j & 0xFF)
@@ -387,6 +412,7 @@ def measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=1, compare
         e_kstep[j][1].record(stream)
     clocks.sample_now(4, 0.0003)
     barrier()
+    nvtx.pop()
     clocks.window(t_window, time.perf_counter())
     kv4.kv4_set_attention_events(cache.handle, None, None)
     t_kern = sum(a.elapsed_time(b) for row in e_kern for a, b in row) / 1e3
@@ -418,6 +444,7 @@ def measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=1, compare
         drained = [[torch.cuda.Event() for _ in range(layers)] for _ in range(2)]
         e0, e1 = ev(), ev()
         barrier()
+        nvtx.push("kv4 e2e steps")
         e0.record(stream)
         h2d.wait_event(e0)
         d2h.wait_event(e0)
@@ -452,6 +479,7 @@ def measure(torch, kv4, w, layers, args, K, W_, device, clocks, world=1, compare
                 stream.wait_event(drained[b][layer])
         e1.record(stream)
         barrier()
+        nvtx.pop()
         t_e2e = e0.elapsed_time(e1) / 1e3
         e2e_bytes = sum(rep.bytes_at(used + j + 1) * layers for j in range(K_e2e))
         e2e = {"t": t_e2e, "bytes": e2e_bytes, "steps": K_e2e, "h2d_bytes_per_step": int(layers * per * 2),
@@ -792,6 +820,8 @@ def run_gpu(args):
                 "clocks": clk,
                 "device_status": r["status"],
                 "setup_s": round(r["setup_s"], 1),
+                "gpu": torch.cuda.get_device_name(device),
+                "kernel_source_digest": kernel_source_hash(),
             }
             if "compare" in r:
                 result["compare"] = r["compare"]
