@@ -46,7 +46,7 @@ import workloads  # noqa: E402
 METRIC = "decode-attention KV GB/s and tokens/s (INT4+INT8-protect), % of B200 HBM peak"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
-SUBLINES = ("qwen3_8b_layer", "async_rl", "long_context")
+SUBLINES = ("qwen3_8b_layer", "async_rl", "long_context", "tiny")   # tiny: the parity fixture, a latency
 BF16_MAX_LAYERS = 12          # distinct BF16 layer caches of the comparison leg on the stack (at most)
 
 
