@@ -348,7 +348,10 @@ int kv4_decode_attention_noalloc(kv4_cache* cache, int32_t layer, const int32_t*
 /* Dequantized keys/values of positions [start, start+count) of one sequence,
  * fp32 [count][Hkv][D], in the rotated basis: x^ = fma(code, s, z) from the
  * INT4 page or the INT8 store as `view` selects (NVFP4 pages: x^ = e2m1(code)
- * * e4m3(scale)).  For inspection and tests. */
+ * * e4m3(scale)).  For inspection and tests.  KV4_ERR_INVALID_ARG when the
+ * range passes the sequence's capacity (max_pages_per_seq * page_size),
+ * KV4_ERR_UNSUPPORTED when count * Hkv is too large for one launch; nothing
+ * is launched then. */
 int kv4_dequantize_debug(kv4_cache* cache, int32_t layer, int32_t seq_id, int32_t start, int32_t count,
                          int32_t view, float* dev_k_out, float* dev_v_out, kv4_stream_t stream);
 

@@ -340,6 +340,7 @@ int launch_dequantize_debug(kv4_cache* c, int layer, int seq_id, int start, int 
   p.fmt = cfg.page_format;
   const long long threads = static_cast<long long>(count) * p.Hkv * 2 * 32;
   const long long blocks = (threads + 255) / 256;
+  if (blocks > 0x7fffffffLL) return KV4_ERR_UNSUPPORTED;
   dequant_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
