@@ -30,6 +30,11 @@ def flags(verbose_ptxas=False):
     return f
 
 
+def up_to_date(obj, deps, same_flags):
+    """An object can be reused when it was compiled with the current flags after its last dependency changed."""
+    return same_flags and os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(d) for d in deps)
+
+
 def build(verbose_ptxas=False, force=False):
     """Compile every source to an object in _build/ and link libkv4.so next to this file."""
     os.makedirs(OBJDIR, exist_ok=True)
@@ -39,16 +44,27 @@ def build(verbose_ptxas=False, force=False):
                if h.endswith((".cuh", ".h"))] + \
         [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.join(ROOT, "include")))
          if h.endswith(".h")]
-    newest_header = max(os.path.getmtime(h) for h in headers)
+    # the flags the objects were compiled with (a self-checking build and a normal one share _build/)
+    stamp = os.path.join(OBJDIR, "flags")
+    f = flags()
+    want = " ".join(x for i, x in enumerate(f) if x != "-I" and (i == 0 or f[i - 1] != "-I"))   # paths aside
+    try:
+        with open(stamp) as f:
+            same_flags = f.read() == want
+    except OSError:
+        same_flags = False
+    if not same_flags and os.path.exists(stamp):
+        os.remove(stamp)
     for src in SOURCES:
         path = os.path.join(HERE, "csrc", src)
         obj = os.path.join(OBJDIR, src.replace(".cu", ".o"))
         objs.append(obj)
-        if (not force and os.environ.get("KV4_DEBUG_CHECKS") != "1" and os.path.exists(obj) and os.path.getmtime(obj) >= os.path.getmtime(path)
-                and os.path.getmtime(obj) >= newest_header and not verbose_ptxas):
+        if not force and not verbose_ptxas and up_to_date(obj, [path] + headers, same_flags):
             continue
         cmd = [nvcc()] + flags(verbose_ptxas) + ["-c", path, "-o", obj]
         subprocess.run(cmd, check=True)
+    with open(stamp, "w") as f:
+        f.write(want)
     cmd = [nvcc(), "-shared", "-cudart", "static", "-gencode", "arch=compute_100a,code=sm_100a", "-o", LIB] + objs
     subprocess.run(cmd, check=True)
     return LIB
