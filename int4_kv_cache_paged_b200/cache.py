@@ -8,9 +8,29 @@ from . import (make_config, kv4_cache_required_bytes, kv4_cache_create, kv4_cach
                kv4_set_rope, kv4_rope_rotate_quantize_append, kv4_decode_step, kv4_test_stall_next_attention,
                kv4_dequantize_debug, kv4_get_status, kv4bf16_cache_required_bytes, kv4bf16_cache_create,
                kv4bf16_cache_destroy, kv4bf16_cache_layout, kv4bf16_append, kv4bf16_attention_workspace_bytes,
-               kv4bf16_decode_attention, kv4bf16_get_status, KV4_VIEW_EFFECTIVE, KV4_MODE_OUT_F32)
+               kv4bf16_decode_attention, kv4bf16_get_status, KV4_VIEW_EFFECTIVE, KV4_MODE_OUT_F32, KV4Error,
+               KV4_ERR_INVALID_ARG)
 
 TILE = 16
+_BF16 = (torch.bfloat16,)
+_I32 = (torch.int32,)
+
+
+def need(t, what, dtypes, numel, device):
+    """Refuse, before anything is launched, a tensor the kernels would misread: one that is not on the cache's
+    device, not contiguous, of another dtype (dtypes None: any) or holding fewer elements than the call reads.
+    Raises KV4Error(KV4_ERR_INVALID_ARG)."""
+    if (isinstance(t, torch.Tensor) and t.device == device and t.is_contiguous()
+            and (dtypes is None or t.dtype in dtypes) and t.numel() >= numel):
+        return
+    got = ("%s %s on %s%s" % (tuple(t.shape), t.dtype, t.device, "" if t.is_contiguous() else ", not contiguous")
+           if isinstance(t, torch.Tensor) else type(t).__name__)
+    raise KV4Error(KV4_ERR_INVALID_ARG, "%s must be a contiguous %s tensor of at least %d elements on %s, not %s"
+                   % (what, "/".join(str(d) for d in dtypes) if dtypes else "", numel, device, got))
+
+
+def _out_dtypes(mode):
+    return (torch.float32,) if (mode & KV4_MODE_OUT_F32) else _BF16
 
 
 def _tile4(D):
@@ -42,6 +62,26 @@ class _Base:
         c = self.cfg
         return self._view(self._lens_ptr, 4 * c["num_layers"] * c["max_seqs"], (-1,)).view(torch.int32).view(
             c["num_layers"], c["max_seqs"])
+
+    def _check_rows(self, seq_ids, cu_new, k_new, v_new, total_new):
+        n, dev = int(seq_ids.numel()), self.buf.device
+        rows = total_new * self.cfg["num_kv_heads"] * self.cfg["head_dim"]
+        if n == 0 or total_new == 0:
+            return
+        need(seq_ids, "seq_ids", _I32, n, dev)
+        need(cu_new, "cu_new", _I32, n + 1, dev)
+        need(k_new, "k_new", _BF16, rows, dev)
+        need(v_new, "v_new", _BF16, rows, dev)
+
+    def _check_attention(self, n, q_rows, q, out, mode, workspace, seq_ids):
+        if n == 0:
+            return
+        dev, cols = self.buf.device, self.cfg["num_q_heads"] * self.cfg["head_dim"]
+        need(seq_ids, "seq_ids", _I32, n, dev)
+        need(q, "q", _BF16, q_rows * cols, dev)
+        need(out, "out", _out_dtypes(mode), q_rows * cols, dev)
+        if workspace is not None:
+            need(workspace, "workspace", None, 0, dev)
 
     def workspace(self, n_seqs, max_ctx=0):
         nbytes = self._ws_bytes(self.handle, n_seqs, max_ctx)
@@ -99,6 +139,7 @@ class KV4Cache(_Base):
         """rope=True: each new key first gets RoPE at its position from the table of set_rope()."""
         if total_new is None:
             total_new = int(k_new.shape[0])
+        self._check_rows(seq_ids, cu_new, k_new, v_new, total_new)
         fn = kv4_rope_rotate_quantize_append if rope else kv4_rotate_quantize_append
         fn(self.handle, layer, seq_ids, cu_new, int(seq_ids.numel()), total_new, k_new, v_new, stream)
 
@@ -120,6 +161,7 @@ class KV4Cache(_Base):
             out = torch.empty(q.shape, dtype=dt, device=self.device)
         if workspace is None:
             workspace = self.workspace(n)
+        self._check_attention(n, n, q, out, mode, workspace, seq_ids)
         kv4_decode_attention(self.handle, layer, seq_ids, n, q, out, scale, mode, workspace, stream)
         return out
 
@@ -131,6 +173,11 @@ class KV4Cache(_Base):
             out = torch.empty(q.shape, dtype=dt, device=self.device)
         if workspace is None:
             workspace = self.workspace(n)
+        self._check_attention(n, n, q, out, mode, workspace, seq_ids)
+        if n:
+            rows = n * self.cfg["num_kv_heads"] * self.cfg["head_dim"]
+            need(k_new, "k_new", _BF16, rows, self.buf.device)
+            need(v_new, "v_new", _BF16, rows, self.buf.device)
         kv4_decode_step(self.handle, layer, seq_ids, n, k_new, v_new, q, out, scale, mode, workspace, stream)
         return out
 
@@ -150,11 +197,14 @@ class KV4Cache(_Base):
             out = torch.empty(q.shape, dtype=dt, device=self.device)
         if workspace is None:
             workspace = self.extend_workspace(n, q_len)
+        self._check_attention(n, n * q_len, q, out, mode, workspace, seq_ids)
         kv4_extend_attention(self.handle, layer, seq_ids, n, q_len, q, out, scale, mode, workspace, stream)
         return out
 
     def attention_noalloc(self, layer, seq_ids, q, out, scale=0.0, mode=0, stream=None):
         """Attention with the library's static scratch (no workspace); `out` must be given."""
+        n = int(seq_ids.numel())
+        self._check_attention(n, n, q, out, mode, None, seq_ids)
         kv4_decode_attention_noalloc(self.handle, layer, seq_ids, int(seq_ids.numel()), q, out, scale, mode, stream)
         return out
 
@@ -207,6 +257,7 @@ class BF16Cache(_Base):
     def append(self, layer, seq_ids, cu_new, k_new, v_new, total_new=None, stream=None):
         if total_new is None:
             total_new = int(k_new.shape[0])
+        self._check_rows(seq_ids, cu_new, k_new, v_new, total_new)
         kv4bf16_append(self.handle, layer, seq_ids, cu_new, int(seq_ids.numel()), total_new, k_new, v_new, stream)
 
     def attention(self, layer, seq_ids, q, out=None, scale=0.0, mode=0, workspace=None, stream=None):
@@ -216,6 +267,7 @@ class BF16Cache(_Base):
             out = torch.empty(q.shape, dtype=dt, device=self.device)
         if workspace is None:
             workspace = self.workspace(n)
+        self._check_attention(n, n, q, out, mode & KV4_MODE_OUT_F32, workspace, seq_ids)
         kv4bf16_decode_attention(self.handle, layer, seq_ids, n, q, out, scale, mode, workspace, stream)
         return out
 
