@@ -91,6 +91,26 @@ def bf16_bytes(lengths, Hkv, D):
     return int(np.sum(np.asarray(lengths, np.int64) * Hkv * 2 * D * 2))
 
 
+def side_bytes(lengths, w, layers):
+    """Bytes a decode step moves outside the KV stream (not in `value`), summed over `layers`: the bf16 queries
+    read and outputs written, the new token's bf16 K and V read and its codes written (INT4 pages and the INT8
+    store: the newest position is always protected), and the block-table entries the attention kernel reads
+    (one int32 per page and group of 4, 2 or 1 KV heads).  `lengths` are the cache lengths the step attends."""
+    L = np.asarray(lengths, np.int64)
+    B, Hq, Hkv, D, P = len(L), w["Hq"], w["Hkv"], w["D"], w["P"]
+    gwr = 4 if Hkv % 4 == 0 else (2 if Hkv % 2 == 0 else 1)
+    q = B * Hq * D * 2
+    new_read = B * Hkv * 2 * D * 2
+    new_written = B * Hkv * (2 * (D // 2 + 4) + 2 * (D + 4))
+    table = int(np.sum(-(-L // P))) * (Hkv // gwr) * 4
+    per_layer = {"q_read": q, "out_written": q, "new_kv_read": new_read, "new_kv_written": new_written,
+                 "block_table_read": table}
+    res = {k: v * layers for k, v in per_layer.items()}
+    res["total"] = sum(res.values())
+    res["kv_stream"] = kv_bytes(L, Hkv, D, w["S"], w["W"]) * layers
+    return res
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -705,7 +725,8 @@ def sub_line(torch, kv4, name, args, device, clocks, hbm, peak_kind):
     line = {"value": round(value, 2), "unit": "GB/s", "ms_per_step": round(r["t_step"] / K * 1e3, 4),
             "tokens_per_s": round(rep.B * K / r["t_step"], 1), "steps": K,
             "config": {"batch": rep.B, "context": "%s" % (w["ctx"][0],), "page": w["P"], "recent_window": w["W"],
-                       "kv_bytes_per_step_mb": round(r["bytes_timed"] / K / 1e6, 1)},
+                       "kv_bytes_per_step_mb": round(r["bytes_timed"] / K / 1e6, 1),
+                       "side_bytes_per_step": side_bytes(rep.L + 3, w, 1)},
             "roofline": roofline_obj(achieved, hbm, peak_kind, profiled_traffic(name), r["bytes_kern"] / K, 1),
             "device_status": r["status"]}
     if r["e2e"]:
@@ -789,6 +810,7 @@ def run_gpu(args):
                            "step": "%d layers x one %s call (append one token per sequence, then attention)"
                                    % (layers, "two-call" if args.two_calls else "kv4_decode_step"),
                            "kv_bytes_per_step_mb": round(r["bytes_timed"] / K / 1e6, 1),
+                           "side_bytes_per_step": side_bytes(rep.L + W_, w, layers),
                            "l2": "flushed before every step by a 256 MB write outside the timed events; each "
                                  "layer's KV also exceeds the 126 MB L2",
                            "parallelism": "replica per GPU" if world > 1 else "single GPU",
