@@ -97,3 +97,18 @@ def test_mode_bits_of_the_binding_match_the_header():
         m = re.search(r"\b%s\s*=\s*(\d+)" % name, text)
         assert m is not None, name
         assert getattr(kv4, name) == int(m.group(1)), name
+
+
+def test_every_header_constant_has_the_same_value_in_the_binding():
+    """Status codes, device status bits, modes, views, page formats and RoPE styles: each enum constant of the
+    header exists in the binding with its value, and the binding defines no KV4_ constant the header lacks."""
+    import int4_kv_cache_paged_b200 as kv4
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    header = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(KV4_[A-Z0-9_]+)\s*=\s*(-?\d+)", text)}
+    assert len(header) >= 29          # 8 status codes, 8 device bits, 6 modes, 2 views, 3 formats, 2 RoPE styles
+    for name, value in header.items():
+        assert getattr(kv4, name) == value, name
+    m = re.search(r"#define\s+KV4_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", text)
+    assert m and kv4.KV4_NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+    binding = {n for n in dir(kv4) if re.fullmatch(r"KV4_[A-Z0-9_]+", n)}
+    assert binding - set(header) == {"KV4_NOALLOC_SCRATCH_BYTES"}
