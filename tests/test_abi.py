@@ -112,3 +112,12 @@ def test_every_header_constant_has_the_same_value_in_the_binding():
     assert m and kv4.KV4_NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
     binding = {n for n in dir(kv4) if re.fullmatch(r"KV4_[A-Z0-9_]+", n)}
     assert binding - set(header) == {"KV4_NOALLOC_SCRATCH_BYTES"}
+
+
+def test_every_status_code_has_a_message():
+    import int4_kv_cache_paged_b200 as kv4
+    codes = [getattr(kv4, n) for n in dir(kv4) if n == "KV4_OK" or n.startswith("KV4_ERR_")]
+    assert len(codes) == 8
+    msgs = [kv4._lib.kv4_status_string(c).decode() for c in codes]
+    assert "unknown status" not in msgs and len(set(msgs)) == len(msgs)
+    assert kv4._lib.kv4_status_string(-99).decode() == "unknown status"
