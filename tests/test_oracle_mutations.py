@@ -160,3 +160,69 @@ def test_output_rotated_twice_fails_the_inverse_pin():
     assert not np.allclose(wrong, base @ H, atol=1e-6)
     np.testing.assert_allclose(attn_mod.decode_attention(c, 0, [0], q, out_rotated=True)["out_f64"], base @ H,
                                atol=1e-12)
+
+
+def test_scale_rounded_down_fails_the_definition_pin(monkeypatch):
+    import test_oracle_quant as tq
+    monkeypatch.setattr(quant, "fp16_round_up", quant.fp16_round_down)   # mistake: s may no longer cover the range
+    for bits in (2, 4, 8):
+        with pytest.raises(AssertionError):
+            tq.test_scale_zero_definition(bits)
+
+
+def _quantize_extra_level(x, bits):
+    """The quantizer with 2^bits levels above zero instead of 2^bits - 1 (a mistake)."""
+    Q = np.float32(2 ** bits)
+    x = quant.clamp_fp16_range(x)
+    z16 = quant.fp16_round_down(x.min(-1))
+    z = z16.astype(np.float32)
+    r = (x.max(-1) - z).astype(np.float32)
+    s16 = np.where(r == 0, np.float16(1), quant.fp16_round_up((r / Q).astype(np.float32))).astype(np.float16)
+    s = s16.astype(np.float32)
+    c = np.clip(np.rint(((x - z[..., None]).astype(np.float32) / s[..., None]).astype(np.float32)), 0, Q)
+    return c.astype(np.uint8), s16, z16
+
+
+def test_extra_quantization_level_fails_the_range_pins(monkeypatch):
+    import test_oracle_quant as tq
+    monkeypatch.setattr(tq, "quantize_groups", _quantize_extra_level)
+    for bits in (2, 4, 8):
+        with pytest.raises(AssertionError):
+            tq.test_codes_in_range_and_error_bound(bits)
+
+
+PROTECTION_MISTAKES = {
+    "window one short": lambda p, L, S, W: p < S or p > L - W,
+    "one sink too many": lambda p, L, S, W: p <= S or p >= L - W,
+    "window one long": lambda p, L, S, W: p < S or p >= L - W - 1,
+}
+
+
+@pytest.mark.parametrize("name", sorted(PROTECTION_MISTAKES))
+def test_protection_boundary_mistakes_fail_the_view_pins(monkeypatch, name):
+    import test_oracle_cache as tc
+    bad = PROTECTION_MISTAKES[name]
+    S, W = 4, 32
+    # the rule itself: its protected slots must be the prefix [0, min(L, S + W)) of the store
+    assert any(sorted(cache_mod.prot_slot(p, S, W) for p in range(L) if bad(p, L, S, W)) != list(range(min(L, S + W)))
+               for L in range(1, 200))
+    # the cache's effective view read through it differs from the per-position construction
+    monkeypatch.setattr(cache_mod, "is_protected", bad)
+    with pytest.raises(AssertionError):
+        tc.test_effective_view_equals_direct_construction([1] * 120)
+
+
+def test_rope_turned_backwards_fails_the_complex_pin():
+    import workloads
+    R = 64
+    cs = workloads.rope_cos_sin(5000, R, base=1e4)
+    x = oracle.bf16_round(np.random.default_rng(9).standard_normal((6, 128)).astype(np.float32))
+    pos = np.array([1, 17, 255, 1024, 3333, 4999])
+    c, s = cs[pos, :R // 2], cs[pos, R // 2:]
+    a, b = x[:, 0:R:2], x[:, 1:R:2]
+    wrong = np.empty_like(x[:, :R])
+    wrong[:, 0::2], wrong[:, 1::2] = a * c + b * s, b * c - a * s      # mistake: turned by -theta
+    z = (a.astype(np.float64) + 1j * b) * (c.astype(np.float64) + 1j * s)
+    assert not np.allclose(wrong[:, 0::2], z.real, rtol=0, atol=4e-6 * np.abs(x).max())
+    right = oracle.rope_fp32(x, pos, cs, R, oracle.ROPE_GPTJ)
+    np.testing.assert_allclose(right[:, 0:R:2], z.real, rtol=0, atol=4e-6 * np.abs(x).max())
