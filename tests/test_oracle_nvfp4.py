@@ -237,3 +237,27 @@ def test_tie_rule_mistake_fails_the_worked_example(monkeypatch):
     g = _golden()
     codes, _ = F.quantize_nvfp4(np.array(g["a.x"], np.float32)[None])
     assert not np.array_equal(codes[0], np.array(g["a.codes"], np.uint8))
+
+
+def _e4m3_truncate(s):
+    """E4M3 code of the largest value not above s (a mistake: truncation instead of the nearest value)."""
+    s = np.minimum(np.asarray(s, np.float64), F.E4M3_MAX)
+    return (np.searchsorted(F.E4M3_GRID, s, side="right") - 1).astype(np.uint8)
+
+
+@pytest.mark.parametrize("mistake", ["scale from amax / 4", "scale truncated to E4M3"])
+def test_block_scale_mistakes_fail_the_worked_example(monkeypatch, mistake):
+    """Two plausible slips in the block scale -- dividing amax by 4 (the largest normal E2M1 power of two)
+    instead of by 6, or truncating it to E4M3 instead of rounding to the nearest value -- each break at
+    least one hand-derived block."""
+    if mistake == "scale from amax / 4":
+        monkeypatch.setattr(F, "E2M1_MAX", 4.0)
+    else:
+        monkeypatch.setattr(F, "e4m3_round", _e4m3_truncate)
+    failed = 0
+    for blk in "abcdef":
+        try:
+            test_worked_example(blk)
+        except AssertionError:
+            failed += 1
+    assert failed >= 1
