@@ -200,6 +200,10 @@ int kv4_seq_reset(kv4_cache* cache, int32_t seq_id, kv4_stream_t stream);
  * The sequence length of this layer advances by the number of new rows.
  * At most 3413 sequences per call (KV4_ERR_UNSUPPORTED above).
  */
+int kv4_rotate_quantize_append(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids,
+                               const int32_t* dev_cu_new, int32_t n_seqs, int32_t total_new,
+                               const void* k_new, const void* v_new, kv4_stream_t stream);
+
 /*
  * RoPE fused into the append and the query kernel (the step before the
  * rotation: keys are rotated by position after RoPE, cf. the key transform
@@ -226,10 +230,6 @@ int kv4_set_rope(kv4_cache* cache, const float* dev_cos_sin, int32_t max_pos, in
 int kv4_rope_rotate_quantize_append(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids,
                                     const int32_t* dev_cu_new, int32_t n_seqs, int32_t total_new,
                                     const void* k_new, const void* v_new, kv4_stream_t stream);
-
-int kv4_rotate_quantize_append(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids,
-                               const int32_t* dev_cu_new, int32_t n_seqs, int32_t total_new,
-                               const void* k_new, const void* v_new, kv4_stream_t stream);
 
 /* Workspace bytes for kv4_decode_attention over up to `n_seqs` sequences of at
  * most `max_ctx` tokens each (max_ctx <= 0: the cache capacity
@@ -288,6 +288,9 @@ int kv4_decode_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq
  * with the operand columns standing for (query token, query head) pairs.
  */
 int kv4_extend_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_t q_len, size_t* bytes);
+int kv4_extend_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs, int32_t q_len,
+                         const void* q, void* out, float softmax_scale, int32_t mode,
+                         void* dev_workspace, size_t ws_bytes, kv4_stream_t stream);
 
 /*
  * One decode step in one call: append one new token to every listed sequence
@@ -308,9 +311,6 @@ int kv4_extend_workspace_bytes(const kv4_cache* cache, int32_t n_seqs, int32_t q
 int kv4_decode_step(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs,
                     const void* k_new, const void* v_new, const void* q, void* out, float softmax_scale,
                     int32_t mode, void* dev_workspace, size_t ws_bytes, kv4_stream_t stream);
-int kv4_extend_attention(kv4_cache* cache, int32_t layer, const int32_t* dev_seq_ids, int32_t n_seqs, int32_t q_len,
-                         const void* q, void* out, float softmax_scale, int32_t mode,
-                         void* dev_workspace, size_t ws_bytes, kv4_stream_t stream);
 
 /*
  * kv4_decode_attention_noalloc: kv4_decode_attention without a workspace
@@ -390,6 +390,14 @@ const char* kv4_version(void);
  * quantization, no protected store).  It exists to measure what the INT4
  * format saves; hadamard_block, sink_tokens and recent_window are ignored.
  * Page pool: bf16 [num_pages][P/16][Hkv][16-token tile of 32*D elements].
+ * Each kv4bf16_* call takes the arguments of its kv4_* namesake, with the
+ * same layouts, ownership and error codes: kv4bf16_append stores k_new and
+ * v_new (bf16 [total_new][Hkv][D]) unchanged, with the same row-offset rules
+ * and device status bits (KV4_DEV_BAD_PAGE, _OVERFLOW, _BAD_SEQ, _BAD_CU);
+ * kv4bf16_decode_attention reads bf16 q [n_seqs][Hq][D] and writes out in
+ * the same layout, with a workspace of kv4bf16_attention_workspace_bytes
+ * bytes (max_ctx <= 0: the cache capacity).  kv4bf16_cache_layout has no
+ * protected store to report.
  */
 typedef struct kv4bf16_cache kv4bf16_cache;
 
