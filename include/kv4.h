@@ -173,11 +173,10 @@ int kv4_cache_destroy(kv4_cache* cache);
 /* Device addresses inside the cache buffer for layer `layer` (any pointer may
  * be NULL): the page pool, uint8 [num_pages][P/16][Hkv][16*D+128] (INT4),
  * [num_pages][P/16][Hkv][18*D] (NVFP4) or [num_pages][P/16][Hkv][8*D+128]
- * (INT2); the
- * INT8 store, uint8 [max_seqs][ceil((S+W)/16)][Hkv][32*D+128]; and the
- * sequence lengths int32 [num_layers][max_seqs] (all layers).  KV heads are
- * innermost, so the 16-token tiles of all heads at one page position are
- * contiguous (one bulk copy feeds eight heads). */
+ * (INT2); the INT8 store, uint8 [max_seqs][ceil((S+W)/16)][Hkv][32*D+128];
+ * and the sequence lengths int32 [num_layers][max_seqs] (all layers).  KV
+ * heads are innermost, so the 16-token tiles of all heads at one page
+ * position are contiguous (one bulk copy feeds a group of four heads). */
 int kv4_cache_layout(const kv4_cache* cache, int32_t layer, void** dev_pages, void** dev_protected,
                      int32_t** dev_seq_lens);
 

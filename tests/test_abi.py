@@ -121,3 +121,19 @@ def test_every_status_code_has_a_message():
     msgs = [kv4._lib.kv4_status_string(c).decode() for c in codes]
     assert "unknown status" not in msgs and len(set(msgs)) == len(msgs)
     assert kv4._lib.kv4_status_string(-99).decode() == "unknown status"
+
+
+def test_every_declaration_follows_its_comment():
+    """Each entry point of the header sits right after a comment block that documents it (or in a run of
+    declarations that follows one, for a mirror family), so its arguments and errors are stated beside it."""
+    lines = open(HEADER).read().splitlines()
+    decl = re.compile(r"^(int|const char\*)\s+(kv4\w+)\(")
+    for i, line in enumerate(lines):
+        m = decl.match(line)
+        if not m:
+            continue
+        j = i - 1
+        while j >= 0 and ((lines[j].startswith((" ", "\t")) and not lines[j].lstrip().startswith("*"))
+                          or decl.match(lines[j]) or lines[j].startswith("#define")):   # continuation, sibling
+            j -= 1
+        assert j >= 0 and lines[j].rstrip().endswith("*/"), m.group(2)
