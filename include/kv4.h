@@ -383,6 +383,8 @@ const char* kv4_status_string(int status);
 /* Build identification: "kv4 <version> sm_100a". */
 const char* kv4_version(void);
 
+typedef struct kv4bf16_cache kv4bf16_cache;   /* opaque host handle of the BF16 baseline cache */
+
 /*
  * BF16 baseline cache: the same paging, block table, split-K attention and
  * merge, with bf16 keys/values stored as they arrive (no rotation, no
@@ -398,8 +400,6 @@ const char* kv4_version(void);
  * bytes (max_ctx <= 0: the cache capacity).  kv4bf16_cache_layout has no
  * protected store to report.
  */
-typedef struct kv4bf16_cache kv4bf16_cache;
-
 int kv4bf16_cache_required_bytes(const kv4_config* cfg, size_t* bytes);
 int kv4bf16_cache_create(const kv4_config* cfg, void* dev_buf, size_t bytes, int32_t* dev_block_table,
                          kv4_stream_t stream, kv4bf16_cache** out);
