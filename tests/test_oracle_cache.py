@@ -141,3 +141,24 @@ def test_bf16_cache_round_trip():
     kk, vv = cache.view(0, 1)
     np.testing.assert_array_equal(kk, k)
     np.testing.assert_array_equal(vv, v)
+
+
+def test_largest_page_and_protected_window():
+    """The largest shapes the library accepts: 1024-token pages and S + W = 4096 protected positions. The
+    effective view after ragged appends equals the per-position construction, the protected slots fill the
+    store's prefix, and the window wraps once the sequence passes S + W."""
+    S, W = 96, 4000
+    cfg = _cfg(D=64, Hkv=1, P=1024, S=S, W=W, Bh=64, pages=6, mpps=6, seqs=1, layers=1)
+    cache = OracleKV4Cache(cfg, _table(cfg))
+    k, v = _kv(4300, 1, 64, 7)
+    pos = 0
+    for n in (3000, 1, 1095, 204):                      # crosses S + W = 4096 and four page boundaries
+        cache.append(0, [0], [0, n], k[pos:pos + n], v[pos:pos + n])
+        pos += n
+    assert pos == 4300 and cache.seq_lens[0, 0] == 4300
+    kh, vh = cache.view(0, 0)
+    np.testing.assert_array_equal(kh, _direct_view(k, 64, pos, S, W))
+    np.testing.assert_array_equal(vh, _direct_view(v, 64, pos, S, W))
+    assert n_prot_tiles(S, W) == 256
+    slots = sorted(prot_slot(p, S, W) for p in range(pos) if is_protected(p, pos, S, W))
+    assert slots == list(range(S + W))
